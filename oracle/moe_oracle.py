@@ -1,0 +1,367 @@
+"""Float64 CPU oracle of the top-k routed Mixture-of-Experts FFN forward pass.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline legs of ``bench.py`` may import this module.  The CUDA library never
+imports it, and it imports nothing from the library: the two share no code.
+Inputs come from ``synth`` (seeded draws) as numpy arrays holding the exact
+bf16 / fp32 input values; everything here widens them to float64.
+
+What it computes, and where each step is defined on the pages it follows:
+
+1. Router logits z = x W_r^T (+ bias_e): the router of "Sharding d'experts"
+   (Kvasir wiki), section "Backbone x worker" (``cur @ router``), and
+   ``MoEFFN.forward`` in moe_stream.py (``self.gate`` is a bias-free Linear
+   [E, d]; the per-expert exploration bias is added to the logits before the
+   softmax).
+2. p = softmax(z) over experts; top-k experts in order of decreasing z, lowest
+   expert index first among equal logits (softmax is monotone, so this is the
+   top-k of p); w_j = p[idx_j], optionally renormalised to sum to one
+   (``MoEFFN.forward``: softmax, topk, divide by the sum).  The renormalising
+   denominator carries no epsilon here (reading: the sum is at least k/E > 0).
+3. Load-balance statistic: f_e = counts_e / T, P_e = sum_t p[t,e] / T,
+   aux = E * sum_e f_e P_e (``MoEFFN.forward``, "Load balancing loss", batch
+   local fractions).
+4. Grouping by expert with each (token, slot) identity kept (ExpertMesh
+   README: "Activation grouping that preserves token and top-k slot
+   identity"; flowchart "Group activations by expert owner").  Groups are in
+   expert order; inside a group, rows are in token order.  With a capacity C
+   (MoEEvolve README: capacity-factor dispatch with static shapes), group e
+   occupies rows [e*C, (e+1)*C) and an assignment whose in-group rank is >= C
+   is dropped (reading: ranks counted in token order).
+5. Expert FFN, gated: h = act(x W1^T) * (x W3^T), y = h W2^T, with SwiGLU
+   (act = SiLU) or GeGLU (act = exact-erf GELU, the torch ``nn.GELU`` default
+   used by moe_stream.py) -- MoEEvolve README ("SwiGLU hidden 256"), the
+   Kvasir worker's "3 mat-muls", kieve-moe ("top-k GeGLU MoE").
+6. Weighted top-k reduction back to token order plus an always-on shared
+   expert at weight one: out_t = sum_j w_j y_{e_j}(x_t) + y_shared(x_t)
+   (Kvasir "Backbone x worker": ``combine(p, partials) + shared(cur)``;
+   ExpertMesh flowchart "Weighted top-k reduction"; ``MoEFFN.forward``:
+   ``out[mask] += w * expert_out``).  No residual and no norm.
+7. Group-scaled signed INT4 weights (ExpertMesh README: HIP routed-expert
+   kernel for group-scaled signed INT4 weights; layout [expert, output,
+   packed_input]): one scale per 128 consecutive inputs of an output row,
+   s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7), two nibbles per byte
+   with the even input index in the low nibble; dequantised exactly as q*s.
+   The float decisions (max, division, rounding to bf16, rint) are taken in
+   fp32, the precision the library's quantiser uses.
+
+Parity pins: every function here is checked by ``tests/test_oracle_*.py``
+against closed forms, textbook values (``tests/golden``), brute force on tiny
+inputs, the dense compute-all-experts-then-mask evaluation (kieve-moe "Tests":
+dense <-> parallel equivalence; Kvasir "Mesure": sharded == monolithic), and
+invariants.  Absolute output values of random full-size layers rest on this
+independent float64 evaluation (no page prints a worked example).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+ACT_SWIGLU = 0
+ACT_GEGLU = 1
+GROUP = 128   # inputs per INT4 scale group
+
+
+# ---------------------------------------------------------------- bf16 / fp32 helpers
+
+def bf16_round(a) -> np.ndarray:
+    """Round fp32 values to the nearest bf16 (ties to even), returned as float32."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).reshape(f.shape)
+
+
+def bf16_bits_to_f32(bits) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32)
+
+
+# ---------------------------------------------------------------- step 1-3: router
+
+def router_logits(x, w_router, bias=None) -> np.ndarray:
+    """z[t,e] = sum_i x[t,i] * W_r[e,i] (+ bias[e]), float64."""
+    z = np.asarray(x, np.float64) @ np.asarray(w_router, np.float64).T
+    if bias is not None:
+        z = z + np.asarray(bias, np.float64)[None, :]
+    return z
+
+
+def softmax(z) -> np.ndarray:
+    z = np.asarray(z, np.float64)
+    m = z.max(axis=1, keepdims=True)
+    ez = np.exp(z - m)
+    return ez / ez.sum(axis=1, keepdims=True)
+
+
+def topk_select(z, k: int) -> np.ndarray:
+    """Indices [T,k] of the k largest entries per row, larger first, lower index first on ties.
+
+    A stable sort of -z keeps equal keys in index order; -0.0 and +0.0 compare
+    equal, so the index decides between them.
+    """
+    z = np.asarray(z)
+    order = np.argsort(-z, axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def topk_margin(z, k: int) -> np.ndarray:
+    """Gap between the k-th and (k+1)-th largest logit of each row (inf when k == E)."""
+    z = np.asarray(z, np.float64)
+    if k >= z.shape[1]:
+        return np.full(z.shape[0], np.inf)
+    s = -np.sort(-z, axis=1)
+    return s[:, k - 1] - s[:, k]
+
+
+def gate_weights(p, idx, renorm: bool) -> np.ndarray:
+    w = np.take_along_axis(np.asarray(p, np.float64), np.asarray(idx, np.int64), axis=1)
+    if renorm:
+        w = w / w.sum(axis=1, keepdims=True)
+    return w
+
+
+def expert_counts(idx, E: int) -> np.ndarray:
+    """counts[e] = number of tokens that selected e (before any capacity drop)."""
+    return np.bincount(np.asarray(idx, np.int64).ravel(), minlength=E).astype(np.int64)
+
+
+def load_balance(counts, p, T: int, E: int):
+    """(f, P, aux): f_e = counts_e/T, P_e = mean_t p[t,e], aux = E * sum_e f_e P_e."""
+    f = np.asarray(counts, np.float64) / T
+    P = np.asarray(p, np.float64).sum(axis=0) / T
+    return f, P, E * float(np.sum(f * P))
+
+
+def route(x, w_router, bias, k: int, renorm: bool):
+    """Steps 1-3 on float64 logits.  Returns dict(z, p, idx, w, counts, f, P, aux)."""
+    z = router_logits(x, w_router, bias)
+    return route_from_logits(z, k, renorm)
+
+
+def route_from_logits(z, k: int, renorm: bool):
+    z = np.asarray(z, np.float64)
+    T, E = z.shape
+    p = softmax(z)
+    idx = topk_select(z, k)
+    w = gate_weights(p, idx, renorm)
+    counts = expert_counts(idx, E)
+    f, P, aux = load_balance(counts, p, T, E)
+    return dict(z=z, p=p, idx=idx, w=w, counts=counts, f=f, P=P, aux=aux)
+
+
+# ---------------------------------------------------------------- step 4: grouping
+
+def capacity(T: int, k: int, E: int, factor: float) -> int:
+    """C = ceil(factor * T * k / E); 0 when no capacity limit is set."""
+    if not factor:
+        return 0
+    from fractions import Fraction
+    return int(math.ceil(Fraction(factor).limit_denominator(10**6) * T * k / E))
+
+
+def permute(idx, E: int, cap: int = 0):
+    """Group the (token, slot) assignments by expert.
+
+    Returns dict with
+      counts [E]    tokens that chose e;
+      kept   [E]    rows of group e actually filled (min(counts, C) with a capacity);
+      offsets [E+1] first row of each group (e*C with a capacity, else an exclusive
+                    prefix sum of counts) and the row total R at [E];
+      rank  [T,k]   position of (t,j) among the tokens that chose idx[t,j], in token order;
+      slot_pos [T,k] row of (t,j) in the grouped buffer, -1 if dropped;
+      drop  [T,k]   1 where dropped;
+      row_src [R]   t*k + j of the assignment in each row, -1 for unfilled rows.
+    """
+    idx = np.asarray(idx, np.int64)
+    T, k = idx.shape
+    flat = idx.ravel()                               # token-major order t*k + j
+    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    order = np.argsort(flat, kind="stable")          # grouped by expert, token order inside
+    starts = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rank_sorted = np.arange(flat.size) - np.repeat(starts, counts)
+    rank = np.empty(flat.size, np.int64)
+    rank[order] = rank_sorted
+    if cap > 0:
+        kept = np.minimum(counts, cap)
+        offsets = np.arange(E + 1, dtype=np.int64) * cap
+        keep = rank < cap
+    else:
+        kept = counts.copy()
+        offsets = np.concatenate([[0], np.cumsum(counts)])
+        keep = np.ones(flat.size, bool)
+    slot = np.where(keep, offsets[flat] + rank, -1)
+    R = int(offsets[E])
+    row_src = np.full(R, -1, np.int64)
+    row_src[slot[keep]] = np.nonzero(keep)[0]
+    return dict(counts=counts, kept=kept, offsets=offsets, rank=rank.reshape(T, k),
+                slot_pos=slot.reshape(T, k), drop=(~keep).astype(np.uint8).reshape(T, k),
+                row_src=row_src)
+
+
+def gather_rows(x, row_src, k: int) -> np.ndarray:
+    """x_perm[r] = x[row_src[r] // k]; unfilled rows are zero."""
+    x = np.asarray(x, np.float64)
+    out = np.zeros((row_src.size, x.shape[1]))
+    m = row_src >= 0
+    out[m] = x[row_src[m] // k]
+    return out
+
+
+# ---------------------------------------------------------------- step 5: expert FFN
+
+def silu(z):
+    z = np.asarray(z, np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def gelu_erf(z):
+    z = np.asarray(z, np.float64)
+    return 0.5 * z * (1.0 + _erf(z / math.sqrt(2.0)))
+
+
+def glu_hidden(x, w13, act: int) -> np.ndarray:
+    """h = act(x W1^T) * (x W3^T) with w13 = [W1; W3] stacked as [2H, d]."""
+    w13 = np.asarray(w13, np.float64)
+    H = w13.shape[0] // 2
+    xz = np.asarray(x, np.float64) @ w13.T
+    g, u = xz[:, :H], xz[:, H:]
+    a = silu(g) if act == ACT_SWIGLU else gelu_erf(g)
+    return a * u
+
+
+def expert_ffn(x, w13, w2, act: int) -> np.ndarray:
+    """One expert: y = (act(x W1^T) * (x W3^T)) W2^T, w2 = [d, H]."""
+    return glu_hidden(x, w13, act) @ np.asarray(w2, np.float64).T
+
+
+def grouped_ffn(x_perm, offsets, kept, w13, w2, act: int) -> np.ndarray:
+    """Apply expert e to rows [offsets[e], offsets[e] + kept[e]); other rows stay zero."""
+    x_perm = np.asarray(x_perm, np.float64)
+    y = np.zeros((x_perm.shape[0], np.asarray(w2).shape[1]))
+    for e in range(len(kept)):
+        n = int(kept[e])
+        if n == 0:
+            continue
+        a = int(offsets[e])
+        y[a:a + n] = expert_ffn(x_perm[a:a + n], w13[e], w2[e], act)
+    return y
+
+
+# ---------------------------------------------------------------- step 6: combine
+
+def combine(y_perm, slot_pos, w, y_shared=None) -> np.ndarray:
+    """out[t] = sum_j w[t,j] * y_perm[slot_pos[t,j]] over kept slots, plus y_shared[t]."""
+    slot_pos = np.asarray(slot_pos, np.int64)
+    T, k = slot_pos.shape
+    y_perm = np.asarray(y_perm, np.float64)
+    out = np.zeros((T, y_perm.shape[1]))
+    for j in range(k):
+        m = slot_pos[:, j] >= 0
+        out[m] += np.asarray(w, np.float64)[m, j, None] * y_perm[slot_pos[m, j]]
+    if y_shared is not None:
+        out += np.asarray(y_shared, np.float64)
+    return out
+
+
+# ---------------------------------------------------------------- the whole layer
+
+def moe_forward(x, w_router, bias, w13, w2, *, k: int, act: int = ACT_SWIGLU, renorm: bool = True,
+                cap: int = 0, w13_sh=None, w2_sh=None, routing=None):
+    """Routed layer: route -> group -> expert FFN -> combine (+ shared expert).
+
+    ``routing`` may carry a precomputed ``route()`` result.  Returns a dict with
+    ``out`` and every intermediate.
+    """
+    E = np.asarray(w_router).shape[0] if w_router is not None else len(w13)
+    r = routing if routing is not None else route(x, w_router, bias, k, renorm)
+    g = permute(r["idx"], E, cap)
+    x_perm = gather_rows(x, g["row_src"], k)
+    y_perm = grouped_ffn(x_perm, g["offsets"], g["kept"], w13, w2, act)
+    y_sh = None
+    if w13_sh is not None:
+        y_sh = expert_ffn(x, np.asarray(w13_sh)[0], np.asarray(w2_sh)[0], act)
+    out = combine(y_perm, g["slot_pos"], r["w"], y_sh)
+    res = dict(r)
+    res.update(g)
+    res.update(x_perm=x_perm, y_perm=y_perm, y_shared=y_sh, out=out)
+    return res
+
+
+def dense_moe_forward(x, w13, w2, idx, w, drop=None, *, act: int = ACT_SWIGLU, w13_sh=None, w2_sh=None):
+    """Dense evaluation: every expert on every token, mixed by the masked gate matrix.
+
+    G[t,e] = w[t,j] where idx[t,j] = e and (t,j) is kept, else 0;
+    out = sum_e G[:,e] * FFN_e(x) (+ shared).  Equal to the routed layer by
+    construction of the grouping (kieve-moe "Tests": dense <-> parallel MoE
+    equivalence).
+    """
+    x = np.asarray(x, np.float64)
+    idx = np.asarray(idx, np.int64)
+    T, k = idx.shape
+    E = len(w13)
+    G = np.zeros((T, E))
+    for j in range(k):
+        keep = np.ones(T, bool) if drop is None else (np.asarray(drop)[:, j] == 0)
+        G[np.arange(T)[keep], idx[keep, j]] += np.asarray(w, np.float64)[keep, j]
+    out = np.zeros((T, np.asarray(w2).shape[1]))
+    for e in range(E):
+        if np.any(G[:, e] != 0):
+            out += G[:, e:e + 1] * expert_ffn(x, w13[e], w2[e], act)
+    if w13_sh is not None:
+        out += expert_ffn(x, np.asarray(w13_sh)[0], np.asarray(w2_sh)[0], act)
+    return out
+
+
+# ---------------------------------------------------------------- step 7: INT4 weights
+
+def quantize_int4_g128(w):
+    """Symmetric signed INT4 with one bf16 scale per 128 inputs.
+
+    w [..., N, K] (float32 values, K % 128 == 0) -> (q int8 [..., N, K] in
+    [-8, 7], s float32 [..., N, K/128] holding bf16 values).  Decisions in fp32:
+    s = bf16(max|w_g| / 7), q = clamp(rint(w / s), -8, 7), q = 0 where s == 0.
+    """
+    w = np.asarray(w, np.float32)
+    *lead, N, K = w.shape
+    assert K % GROUP == 0
+    wg = w.reshape(*lead, N, K // GROUP, GROUP)
+    amax = np.abs(wg).max(axis=-1)
+    s = bf16_round(amax / np.float32(7.0))
+    safe = np.where(s == 0, np.float32(1.0), s).astype(np.float32)
+    q = np.rint(wg / safe[..., None])
+    q = np.where(s[..., None] == 0, 0.0, q)
+    q = np.clip(q, -8, 7).astype(np.int8)
+    return q.reshape(*lead, N, K), s.astype(np.float32)
+
+
+def pack_int4(q) -> np.ndarray:
+    """Two signed nibbles per byte: input index 2i in the low nibble, 2i+1 in the high one."""
+    q = np.asarray(q, np.int8)
+    lo = (q[..., 0::2].astype(np.int16) & 0xF)
+    hi = (q[..., 1::2].astype(np.int16) & 0xF)
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed) -> np.ndarray:
+    b = np.asarray(packed, np.uint8).astype(np.int16)
+    lo = b & 0xF
+    hi = (b >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def dequantize_int4_g128(packed, scales) -> np.ndarray:
+    """Exact float64 weights q * s from packed nibbles [..., N, K/2] and scales [..., N, K/128]."""
+    q = unpack_int4(packed).astype(np.float64)
+    *lead, N, K = q.shape
+    s = np.asarray(scales, np.float64)
+    return (q.reshape(*lead, N, K // GROUP, GROUP) * s[..., None]).reshape(*lead, N, K)

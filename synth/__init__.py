@@ -1,0 +1,12 @@
+"""Seeded synthetic workloads for the routed MoE FFN forward pass.
+
+This package holds the five workload shapes and the seeded generators that
+draw their inputs.  It holds none of the layer's arithmetic: no routing, no
+grouping, no expert FFN, no quantisation.  Both the CUDA path (tests, bench)
+and the float64 oracle (tests) receive the tensors it draws.
+"""
+
+from .workloads import WORKLOADS, Workload, get_workload, make_inputs, expert_weights_f32, draw_topk_idx, draw_logits
+
+__all__ = ["WORKLOADS", "Workload", "get_workload", "make_inputs", "expert_weights_f32",
+           "draw_topk_idx", "draw_logits"]
