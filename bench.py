@@ -1,0 +1,338 @@
+"""Benchmark of the routed MoE FFN forward on B200: tokens/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one ``moe_forward`` (router -> grouping -> grouped gate/up GEMM with
+GLU epilogue -> down GEMM -> shared expert -> combine) over one batch of
+seeded synthetic tokens already resident in HBM.  L2 is flushed (a 256 MiB
+write) before every timed step, outside the timed interval.  Under torchrun
+(N > 1) every rank runs an independent replica on its own GPU and its own
+tokens (the layer does not shard here; no collective on the data path); the
+reported time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload (the reference arm).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor-core or HBM roofline"
+DEFAULT_WORKLOAD = "small"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def hbm_roofline_tokens_per_s(bandwidth_bytes_per_s: float, active_bytes_per_token: float) -> float:
+    """Ideal bandwidth-bound decode rate: bandwidth / bytes of active weights per token."""
+    return bandwidth_bytes_per_s / active_bytes_per_token
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload setup
+
+
+def setup(wl, seed, device):
+    import torch
+
+    import sparse_mixture_experts_expert_b200 as moe
+    import synth
+    inp = synth.make_inputs(wl, seed=0, device=device)                # weights: same on every replica
+    if seed:
+        inp["x"] = synth.make_inputs(wl, seed=seed, device=device, with_expert_weights=False)["x"]
+    C = moe.moe_capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+    s = moe.MoeShape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, H=wl.H, H_s=wl.H_s, capacity=C, act=wl.act, wfmt=wl.wfmt,
+                     renorm=wl.renorm)
+    ws = moe.workspace(s, device)
+    out = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=device)
+    return s, inp, ws, out
+
+
+def run_forward(moe, s, inp, ws, out, aux):
+    return moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
+                           w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), out=out, ws=ws, aux=aux)
+
+
+def stage_times(moe, s, inp, ws, wl, flush, reps=10):
+    """Per-stage device time (us) through the component entry points, L2 flushed before each rep."""
+    import torch
+    st = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    acc = {"route": [], "permute": [], "expert_ffn": [], "shared_ffn": [], "combine": []}
+    for _ in range(reps):
+        flush()
+        ev[0].record(st)
+        r = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"], ws=ws)
+        ev[1].record(st)
+        p = moe.moe_permute(s, inp["x"], r["topk_idx"], ws=ws)
+        ev[2].record(st)
+        h, y = moe.moe_expert_ffn(s, p["x_perm"], inp["w13"], inp["w2"], group_start=p["offsets"],
+                                  group_rows=p["kept"])
+        ev[3].record(st)
+        ysh = None
+        if wl.H_s:
+            _, ysh = moe.moe_expert_ffn(s, inp["x"], inp["w13_sh"], inp["w2_sh"], hidden=wl.H_s)
+        ev[4].record(st)
+        moe.moe_combine(s, y, p["slot_pos"], r["topk_w"], ysh)
+        ev[5].record(st)
+        torch.cuda.synchronize()
+        for i, k in enumerate(acc):
+            acc[k].append(ev[i].elapsed_time(ev[i + 1]) * 1e3)
+        kept = int(p["kept"].sum())
+    return {k: statistics.median(v) for k, v in acc.items()}, kept
+
+
+def cpu_oracle_sample(wl, budget_s=12.0, max_tokens=None):
+    """Time the float64 oracle on a bounded token sample of the workload; returns (tokens/s, sample, cores)."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    import synth
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+    except Exception:  # noqa: BLE001
+        threads = cores
+    n = min(wl.T, max_tokens or wl.T)
+    sub = wl.replace(T=n)
+    inp = synth.make_inputs(sub, seed=0, device="cpu")
+    f64 = lambda t: t.to(torch.float64).numpy() if t is not None else None  # noqa: E731
+    args = dict(x=f64(inp["x"]), w_router=f64(inp["w_router"]), bias=f64(inp["bias"]), w13=f64(inp["w13"]),
+                w2=f64(inp["w2"]), w13_sh=f64(inp.get("w13_sh")), w2_sh=f64(inp.get("w2_sh")))
+    cap = O.capacity(n, wl.k, wl.E, wl.capacity_factor)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        O.moe_forward(args["x"], args["w_router"], args["bias"], args["w13"], args["w2"], k=wl.k, act=wl.act,
+                      renorm=bool(wl.renorm), cap=cap, w13_sh=args["w13_sh"], w2_sh=args["w2_sh"])
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, f"{done} tokens ({done // n} x {n}-token batches of the {wl.name} workload) in {el:.1f} s", \
+        min(cores, threads) if threads else cores
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    import synth
+    wl = synth.get_workload(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = []
+        for i in range(args.warmup + args.steps):
+            v, sample, cores = cpu_oracle_sample(wl, budget_s=2.0, max_tokens=min(wl.T, 2048))
+            if i >= args.warmup:
+                steps.append(v)
+        val = statistics.median(steps)
+        line = {"metric": METRIC, "value": val, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.T / val * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "H": wl.H, "H_s": wl.H_s},
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_expert_b200 as moe
+    moe.load()
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    s, inp, ws, out = setup(wl, rank, device)
+    flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def flush():
+        flushbuf.fill_(1)
+
+    st = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        run_forward(moe, s, inp, ws, out, wl.aux)
+    torch.cuda.synchronize()
+    status, site = moe.moe_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} at {site:#x} during warm-up")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = moe.moe_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for a, b in evs:
+            flush()
+            a.record(st)
+            run_forward(moe, s, inp, ws, out, wl.aux)
+            b.record(st)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = moe.moe_launch_count() - launches0
+    step_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    step_ms = max_over_ranks(step_ms, world)
+    value = world * wl.T / (step_ms * 1e-3)
+
+    # end to end through the public API with host buffers: pinned H2D of x, forward, D2H of out
+    x_host = inp["x"].cpu().pin_memory()
+    out_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    inp_e2e = dict(inp)
+    inp_e2e["x"] = x_dev
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in e2e_ev:
+        flush()
+        a.record(st)
+        x_dev.copy_(x_host, non_blocking=True)
+        run_forward(moe, s, inp_e2e, ws, out, wl.aux)
+        out_host.copy_(out, non_blocking=True)
+        b.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
+
+    # stage breakdown and the roofline of the grouped expert GEMMs
+    stages, kept = stage_times(moe, s, inp, ws, wl, flush)
+    peaks = load_peaks()
+    flops = wl.flops_tc(kept)
+    gemm_us = stages["expert_ffn"] + stages["shared_ffn"]
+    achieved_tf = flops / (gemm_us * 1e-6) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": "k_grouped_gemm (gate/up + GLU, down; routed + shared)",
+                "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
+                "peak_source": peaks["source"] + " burst bf16", "traffic": None,
+                "alg_flops_per_step": flops, "gemm_us": gemm_us}
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v, sample, cores = cpu_oracle_sample(wl, budget_s=12.0, max_tokens=min(wl.T, 4096))
+            cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "H": wl.H,
+                           "H_s": wl.H_s, "capacity": s.capacity, "act": "geglu" if wl.act else "swiglu",
+                           "wfmt": "int4_g128" if wl.wfmt else "bf16", "router": "fp32",
+                           "l2": "flushed before every step (256 MiB write), outside the timed interval",
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "roofline": roofline, "stages_us": stages, "cpu_baseline": cpu,
+                "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 2},
+                "gpu_launches": launches, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

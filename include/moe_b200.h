@@ -1,0 +1,238 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) routed Mixture-of-Experts FFN
+ * forward pass.
+ *
+ * The layer (one GPU, forward only):
+ *
+ *   z      = x W_r^T (+ bias)                      router logits, fp32
+ *   p      = softmax(z); (idx, w) = top-k of z     lowest expert index wins ties
+ *   w     /= sum(w)                                if renorm
+ *   group (token, slot) pairs by expert, token order inside a group,
+ *         dropping ranks >= C when a capacity C is set
+ *   h      = act(x W1_e^T) * (x W3_e^T)            act = SiLU (SwiGLU) or erf-GELU (GeGLU)
+ *   y      = h W2_e^T
+ *   out_t  = sum_j w[t,j] y_{idx[t,j]}(x_t) + y_shared(x_t)
+ *
+ * Sources: "Sharding d'experts" (Kvasir wiki), section "Backbone x worker":
+ * the router runs softmax and top-k over ``cur @ router``, the worker does the
+ * three expert matmuls, the backbone adds ``combine(p, partials) +
+ * shared(cur)``.  moe_stream.py (MoE-Stream), ``MoEFFN.forward``: bias-free
+ * Linear gate, additive per-expert logit bias, softmax, topk, renormalised
+ * gates, ``out[mask] += w * expert_out``, batch-local load-balance statistic.
+ * ExpertMesh README: grouping that keeps token and top-k slot identity,
+ * weighted top-k reduction, group-scaled signed INT4 experts in an [expert,
+ * output, packed_input] layout behind a stable C ABI.  MoEEvolve README:
+ * granular SwiGLU experts, one always-active shared expert, capacity-factor
+ * static-shape dispatch.  kieve-moe: top-k GeGLU experts, load-balancing
+ * auxiliary statistic.
+ *
+ * Conventions (every entry point):
+ *  - Pointers named as device pointers must be device memory of the current
+ *    device, 16-byte aligned.  All are borrowed: the caller owns them, the
+ *    library keeps no reference after the call returns.
+ *  - The library allocates no device memory.  Scratch comes from the caller's
+ *    `workspace` (size from moe_workspace_size()).
+ *  - Work is enqueued asynchronously on `stream`; no entry point synchronises
+ *    the host except moe_get_status().
+ *  - Errors found on the host (bad pointers, shapes, sizes) are returned
+ *    before anything is enqueued.  A device-side bounded wait that gives up
+ *    records MOE_DEVICE_TIMEOUT in a per-device status word read by
+ *    moe_get_status(); kernels never trap.
+ *  - Inputs must be finite; routing of NaN logits is undefined.
+ *  - Layouts are row-major.  bf16 tensors are passed as void*.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum moe_status {
+  MOE_OK = 0,
+  MOE_INVALID_ARGUMENT = 1,    /* NULL where a buffer is required, misaligned pointer, k > E ... */
+  MOE_UNSUPPORTED_SHAPE = 2,   /* shape outside the limits below */
+  MOE_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < moe_workspace_size() */
+  MOE_CUDA_ERROR = 4,          /* a CUDA runtime / driver call failed */
+  MOE_DEVICE_TIMEOUT = 5       /* a device-side bounded wait gave up (read via moe_get_status) */
+};
+
+enum moe_act { MOE_ACT_SWIGLU = 0, MOE_ACT_GEGLU = 1 };
+enum moe_wfmt { MOE_WFMT_BF16 = 0, MOE_WFMT_INT4_G128 = 1 };
+
+/*
+ * Layer shape.
+ *   T        tokens (1 .. 2^24)
+ *   d        model width (multiple of 16; multiple of 128 for INT4)
+ *   E        routed experts (1 .. 512)
+ *   k        experts per token (1 .. min(E, 16))
+ *   H        routed expert hidden width (multiple of 16; of 128 for INT4)
+ *   H_s      shared expert hidden width, 0 = no shared expert (same rules as H)
+ *   capacity rows per expert group C, 0 = unbounded (see moe_capacity)
+ *   act      enum moe_act
+ *   wfmt     enum moe_wfmt
+ *   renorm   1: divide the k gates by their sum; 0: gates are the softmax probabilities
+ */
+typedef struct moe_shape {
+  int64_t T;
+  int32_t d, E, k, H, H_s, capacity, act, wfmt, renorm;
+} moe_shape;
+
+/*
+ * Expert weight layouts ([expert, out, in], the ExpertMesh "[expert, output,
+ * packed_input]" order):
+ *   MOE_WFMT_BF16:      w13 [E, 2H, d] bf16, rows [0,H) = W1 (gate), rows [H,2H) = W3 (up);
+ *                       w2  [E, d, H]  bf16.
+ *   MOE_WFMT_INT4_G128: w13 [E, 2H, d/2] uint8, w2 [E, d, H/2] uint8: two's-complement
+ *                       nibbles, input index 2i in the low nibble of byte i;
+ *                       s13 [E, 2H, d/128] bf16, s2 [E, d, H/128] bf16: one scale per
+ *                       128 consecutive inputs of an output row; weight = q * s.
+ * The shared expert uses the same layouts with E = 1 and H = H_s.
+ */
+
+/* Number of grouped rows R: E * capacity with a capacity, else T * k. */
+int64_t moe_grouped_rows(const moe_shape* s);
+
+/*
+ * C = ceil(factor * T * k / E), the per-expert capacity of the MoEEvolve
+ * README's capacity-factor dispatch; factor <= 0 gives 0 (unbounded).
+ * The factor is read as a decimal with at most 6 fractional digits.
+ */
+int moe_capacity(int64_t T, int32_t k, int32_t E, double factor, int32_t* capacity);
+
+/* Scratch bytes moe_forward needs for this shape (an upper bound for every entry point). */
+int moe_workspace_size(const moe_shape* s, size_t* bytes);
+
+/*
+ * Router (Kvasir "Backbone x worker" router line; moe_stream.py MoEFFN.forward).
+ *   x        [T, d] bf16                 in
+ *   w_router [E, d] fp32                 in   (a bias-free Linear(d, E))
+ *   bias     [E] fp32 or NULL            in   added to the logits before softmax/top-k
+ *   logits   [T, E] fp32 or NULL         out  x W_r^T + bias, the values softmax and top-k see
+ *   topk_idx [T, k] int32                out  experts by decreasing logit, lowest index on ties
+ *   topk_w   [T, k] fp32                 out  softmax probability of each pick (renormalised if renorm)
+ *   counts   [E] int32                   out  tokens choosing each expert
+ *   aux_f, aux_p [E] fp32 or NULL        out  counts/T and mean softmax probability
+ *   aux      [1] fp32 or NULL            out  E * sum_e f_e P_e
+ * Deterministic: identical inputs give bit-identical outputs.
+ */
+int moe_route(const moe_shape* s, const void* x, const float* w_router, const float* bias, float* logits,
+              int32_t* topk_idx, float* topk_w, int32_t* counts, float* aux_f, float* aux_p, float* aux,
+              void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * The softmax / top-k / gates / statistics half of moe_route on caller
+ * logits [T, E] fp32 (any bias already added).  Same outputs and rules.
+ */
+int moe_route_from_logits(const moe_shape* s, const float* logits, int32_t* topk_idx, float* topk_w,
+                          int32_t* counts, float* aux_f, float* aux_p, float* aux, void* workspace,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Grouping by expert with (token, slot) identity kept (ExpertMesh README,
+ * "Activation grouping that preserves token and top-k slot identity"; the
+ * MoEEvolve capacity-factor dispatch).
+ *   x         [T, d] bf16        in
+ *   topk_idx  [T, k] int32       in   k distinct experts per token, each in [0, E)
+ *   slot_pos  [T, k] int32       out  row of (t, j) in the grouped buffer, -1 if dropped
+ *   drop_mask [T, k] uint8 / NULL out 1 where (t, j) was dropped by the capacity
+ *   counts    [E] int32 / NULL   out  tokens choosing each expert (before drops)
+ *   kept      [E] int32          out  rows filled in group e
+ *   offsets   [E+1] int32        out  first row of group e (e*C with a capacity, else
+ *                                     prefix sum of counts); offsets[E] = R
+ *   row_src   [R] int32 / NULL   out  t*k + j for filled rows, -1 for unfilled rows
+ *   x_perm    [R, d] bf16        out  x_perm[slot_pos[t,j]] = x[t]; unfilled rows untouched
+ * Rows of a group are in token order; an assignment is dropped when its rank
+ * (tokens before it that chose the same expert) is >= C.  Bit-exact and
+ * deterministic.
+ */
+int moe_permute(const moe_shape* s, const void* x, const int32_t* topk_idx, int32_t* slot_pos,
+                uint8_t* drop_mask, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_src,
+                void* x_perm, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Grouped gated expert FFN (MoEEvolve SwiGLU experts; kieve-moe GeGLU; the
+ * Kvasir worker's three matmuls; ExpertMesh INT4 routed-expert product).
+ * Group g holds rows [group_start[g], group_start[g] + group_rows[g]) of
+ * x_grouped and uses expert g's weights.  group_start / group_rows are device
+ * arrays [n_groups]; both NULL means one group of all R rows.
+ *   hidden        H of these experts (s->H for routed experts, s->H_s for the shared one)
+ *   x_grouped     [R, d] bf16             in
+ *   w13, w2       expert weights, layout per s->wfmt (n_groups experts)
+ *   s13, s2       INT4 scales (NULL for bf16)
+ *   h             [R, hidden] bf16        out (scratch the caller may read)
+ *   y             [R, d] bf16             out  rows outside every group are untouched
+ * Accumulation is fp32; h is rounded to bf16 once, y once.
+ */
+int moe_expert_ffn(const moe_shape* s, int32_t n_groups, int32_t hidden, int64_t R, const void* x_grouped,
+                   const int32_t* group_start, const int32_t* group_rows, const void* w13, const void* s13,
+                   const void* w2, const void* s2, void* h, void* y, moe_stream_t stream);
+
+/*
+ * Weighted top-k reduction back to token order (ExpertMesh flowchart
+ * "Weighted top-k reduction"; moe_stream.py ``out[mask] += w * expert_out``;
+ * Kvasir ``combine(p, partials) + shared(cur)``).
+ *   y_perm   [R, d] bf16       in
+ *   slot_pos [T, k] int32      in   -1 = dropped, contributes nothing
+ *   topk_w   [T, k] fp32       in
+ *   y_shared [T, d] bf16/NULL  in   added at weight one
+ *   out      [T, d] bf16       out  sum in fp32 in slot order, then shared, one rounding
+ */
+int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
+                const void* y_shared, void* out, moe_stream_t stream);
+
+/*
+ * The whole layer: route -> permute -> grouped FFN -> shared expert -> combine,
+ * enqueued on `stream` with no host synchronisation.
+ *   x, w_router, bias          as moe_route
+ *   w13, s13, w2, s2           routed experts (layout per s->wfmt; scales NULL for bf16)
+ *   w13_sh, s13_sh, w2_sh, s2_sh  shared expert (E = 1, H = H_s); NULL when H_s == 0
+ *   out        [T, d] bf16     out
+ *   topk_idx, topk_w, counts, drop_mask, aux_f, aux_p, aux: optional outputs (NULL = not returned)
+ *   workspace  >= moe_workspace_size() bytes of device memory, 256-byte aligned
+ */
+int moe_forward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                const void* s13, const void* w2, const void* s2, const void* w13_sh, const void* s13_sh,
+                const void* w2_sh, const void* s2_sh, void* out, int32_t* topk_idx, float* topk_w,
+                int32_t* counts, uint8_t* drop_mask, float* aux_f, float* aux_p, float* aux, void* workspace,
+                size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Group-scaled signed INT4 quantiser (ExpertMesh README: signed INT4 weights
+ * with group scales).  For each row of w [rows, K] fp32 (K % 128 == 0) and
+ * each group of 128 inputs: s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7)
+ * (q = 0 when s = 0), decisions in fp32.
+ *   q      [rows, K/2] uint8 out   low nibble = even input index
+ *   scales [rows, K/128] bf16 out
+ */
+int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's status word.
+ * *device_status receives MOE_OK or the first device-side error recorded
+ * (MOE_DEVICE_TIMEOUT); *site (may be NULL) where it happened.  Returns
+ * MOE_CUDA_ERROR if the synchronisation itself failed.
+ */
+int moe_get_status(moe_stream_t stream, int32_t* device_status, uint32_t* site);
+
+/* Upper bound, in nanoseconds, of every device-side wait (default 2e9). */
+int moe_set_wait_limit_ns(uint64_t ns);
+
+/* Enqueue a kernel whose bounded wait on an mbarrier nobody arrives on must give
+ * up after the wait limit: exercises the MOE_DEVICE_TIMEOUT path safely. */
+int moe_selftest_wait_timeout(moe_stream_t stream);
+
+/* Kernels this library has launched since load (all entry points, all threads). */
+uint64_t moe_launch_count(void);
+
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,277 @@
+// Grouped expert GEMM on the 5th-generation tensor cores (tcgen05 + TMA).
+//
+// out[rows of group g] = epilogue( A[rows of group g] . B_g^T )
+//   GEMM 1 (gated): A = grouped tokens [R, d], B_g = w13[g] [2H, d]; the tile
+//     loads H/..-wide slices of the gate rows W1 and of the up rows W3 side by
+//     side, so one 128 x 256 fp32 accumulator holds g and u for 128 hidden
+//     columns and the epilogue writes h = act(g) * u in bf16 (SwiGLU: SiLU;
+//     GeGLU: exact-erf GELU).  MoEEvolve README "SwiGLU hidden 256",
+//     kieve-moe "top-k GeGLU", the Kvasir worker's "3 mat-muls".
+//   GEMM 2 (down): A = h [R, H], B_g = w2[g] [d, H], epilogue writes y in bf16.
+// The ExpertMesh README names a grouped GEMM with fused gate/up/down as the
+// optimisation path of its routed-expert kernel; this is that GEMM for sm_100a.
+//
+// Structure: persistent CTAs (one per SM), 8 warps.
+//   warp 0 lane 0  TMA producer: A tile 128 x 64 and B tile N x 64 per stage
+//                  (128-byte swizzle), ring of kStages stages.
+//   warp 1         allocates 2 x BN TMEM columns; lane 0 issues tcgen05.mma
+//                  (M=128, N=BN, K=16, bf16 -> fp32) and commits stages back.
+//   warps 4..7     epilogue: tcgen05.ld of their 32 TMEM lanes, activation,
+//                  bf16 rounding, masked row stores.  Two accumulators in
+//                  TMEM let the epilogue of tile i overlap the MMAs of i+1.
+// Tiles: for each group, ceil(rows/128) row tiles x ceil(N_out/cols) column
+// tiles, enumerated from the device-side group table (no host sync).  Row tiles
+// that run past a group's end read the next group's rows (or TMA zero fill);
+// their outputs are masked.  Every wait is bounded.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2 };
+
+struct GemmParams {
+  const int32_t* group_start;  // [n_groups] or nullptr (one group of R rows)
+  const int32_t* group_rows;   // [n_groups] or nullptr
+  int n_groups;
+  long long R;
+  int K;          // reduction length
+  int N;          // output columns
+  int up_row0;    // GLU: first row of the up half in B (= H)
+  __nv_bfloat16* out;
+  long long ldo;
+  unsigned long long wait_limit_ns;
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // one 128-byte swizzle atom of bf16
+constexpr int kMaxGroupsSmem = 1024;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kTmemCols = 2 * BN;  // two accumulators
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes;
+};
+
+__device__ __forceinline__ float act_silu(float g) { return g / (1.0f + __expf(-g)); }
+__device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + erff(g * 0.7071067811865476f)); }
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(256, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr bool kGLU = MODE != kModePlain;
+  constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
+  constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box
+  constexpr int S = Cfg::kStages;
+  constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_full[S], bar_empty[S], bar_tfull[2], bar_tempty[2], bar_final;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_prefix[kMaxGroupsSmem + 1];
+
+  const int warp = warp_id(), lane = lane_id();
+  const int n_tiles = (p.N + OUTN - 1) / OUTN;
+  const int nk = (p.K + kBK - 1) / kBK;
+  const bool single = p.group_rows == nullptr;
+  const int G = single ? 1 : p.n_groups;
+
+  // group row-tile prefix (warp 2), barriers (warp 0), TMEM (warp 1)
+  if (warp == 2) {
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+      const long long rows = single ? p.R : (long long)p.group_rows[g];
+      local += (int)((rows + kBM - 1) / kBM);
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+      s_prefix[g] = run;
+      const long long rows = single ? p.R : (long long)p.group_rows[g];
+      run += (int)((rows + kBM - 1) / kBM);
+    }
+    if (lane == 31) s_prefix[G] = incl;
+  }
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&bar_full[s], 1); mbar_init(&bar_empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&bar_tfull[a], 1); mbar_init(&bar_tempty[a], 128); }
+    mbar_init(&bar_final, 1);
+    s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem;
+  const int total_m = s_prefix[G];
+  const long long total = (long long)total_m * n_tiles;
+
+  auto locate = [&](long long tile, int& g, long long& row0, int& rows_valid, int& n0) {
+    const int mt = (int)(tile / n_tiles);
+    const int nt = (int)(tile - (long long)mt * n_tiles);
+    int lo = 0, hi = G - 1;  // last g with s_prefix[g] <= mt
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const long long m_local = (long long)(mt - s_prefix[g]) * kBM;
+    const long long start = single ? 0 : (long long)p.group_start[g];
+    const long long rows = single ? p.R : (long long)p.group_rows[g];
+    row0 = start + m_local;
+    rows_valid = (int)min((long long)kBM, rows - m_local);
+    n0 = nt * OUTN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+        int g, rows_valid, n0;
+        long long row0;
+        locate(tile, g, row0, rows_valid, n0);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&bar_empty[stage], phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0101)) break;
+          uint8_t* a_s = smem + (size_t)stage * Cfg::kStageBytes;
+          uint8_t* b_s = a_s + Cfg::kABytes;
+          mbar_arrive_expect_tx(&bar_full[stage], Cfg::kStageBytes);
+          tma_load_2d(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0);
+          if (kGLU) {
+            tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
+            tma_load_3d(b_s + BOXB * 128, &tmB, &bar_full[stage], kb * kBK, p.up_row0 + n0, g);
+          } else {
+            tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
+          }
+          ++issued;
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Make sure no copy is still landing in shared memory when the CTA ends.
+      const int last = (int)(issued < S ? issued : (long long)S);
+      for (int i = 1; i <= last; ++i) {
+        const long long n = issued - i;
+        const int st = (int)(n % S);
+        const uint32_t ph = (uint32_t)((n / S) & 1);
+        volatile int dummy = 0;
+        mbar_wait(&bar_full[st], ph, p.wait_limit_ns, &dummy, 0x0102);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+        if (!mbar_wait(&bar_tempty[acc], acc_phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0103)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&bar_full[stage], phase, p.wait_limit_ns, &s_abort, 0x0104)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + (size_t)stage * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bar_empty[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&bar_tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all issued MMAs complete before TMEM is released
+      tc_commit(&bar_final);
+      volatile int dummy = 0;
+      mbar_wait(&bar_final, 0, p.wait_limit_ns, &dummy, 0x0105);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter
+    const int r = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+      int g, rows_valid, n0;
+      long long row0;
+      locate(tile, g, row0, rows_valid, n0);
+      if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0106)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const bool row_ok = r < rows_valid;
+      __nv_bfloat16* orow = p.out + (row0 + r) * p.ldo;
+#pragma unroll 1
+      for (int c = 0; c < OUTN; c += 16) {
+        uint32_t v[16];
+        uint32_t o[8];
+        if (kGLU) {
+          uint32_t u[16];
+          tmem_ld16(t_row + c, v);
+          tmem_ld16(t_row + OUTN + c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            const float a0 = MODE == kModeSwiGLU ? act_silu(g0) : act_gelu(g0);
+            const float a1 = MODE == kModeSwiGLU ? act_silu(g1) : act_gelu(g1);
+            o[i] = pack_bf16x2(a0 * u0, a1 * u1);
+          }
+        } else {
+          tmem_ld16(t_row + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        if (row_ok && n0 + c < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + n0 + c);
+          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,504 @@
+// C ABI of the routed MoE FFN forward pass: argument checks, workspace layout,
+// TMA descriptors and kernel launches.  One translation unit so the device
+// status word is shared by every kernel.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "permute.cuh"
+#include "quant.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+static std::atomic<unsigned long long> g_launches{0};
+static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+static inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+#define MOE_CUDA_TRY(expr)                       \
+  do {                                           \
+    cudaError_t err_ = (expr);                   \
+    if (err_ != cudaSuccess) return MOE_CUDA_ERROR; \
+  } while (0)
+
+#define MOE_LAUNCH_CHECK()                       \
+  do {                                           \
+    count_launch();                              \
+    if (cudaGetLastError() != cudaSuccess) return MOE_CUDA_ERROR; \
+  } while (0)
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+static inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------ shape checks
+
+static int check_shape(const moe_shape* s) {
+  if (s == nullptr) return MOE_INVALID_ARGUMENT;
+  if (s->T < 1 || s->T > (1ll << 24)) return MOE_UNSUPPORTED_SHAPE;
+  if (s->E < 1 || s->E > kMaxE) return MOE_UNSUPPORTED_SHAPE;
+  if (s->k < 1 || s->k > 16) return MOE_UNSUPPORTED_SHAPE;
+  if (s->k > s->E) return MOE_INVALID_ARGUMENT;
+  if (s->d < 16 || s->d % 16 != 0 || s->d > 65536) return MOE_UNSUPPORTED_SHAPE;
+  if (s->H < 16 || s->H % 16 != 0 || s->H > 65536) return MOE_UNSUPPORTED_SHAPE;
+  if (s->H_s < 0 || s->H_s % 16 != 0 || s->H_s > 65536) return MOE_UNSUPPORTED_SHAPE;
+  if (s->capacity < 0) return MOE_INVALID_ARGUMENT;
+  if (s->act != MOE_ACT_SWIGLU && s->act != MOE_ACT_GEGLU) return MOE_INVALID_ARGUMENT;
+  if (s->wfmt != MOE_WFMT_BF16 && s->wfmt != MOE_WFMT_INT4_G128) return MOE_INVALID_ARGUMENT;
+  if (s->renorm != 0 && s->renorm != 1) return MOE_INVALID_ARGUMENT;
+  if (s->wfmt == MOE_WFMT_INT4_G128 && (s->d % 128 != 0 || s->H % 128 != 0 || s->H_s % 128 != 0))
+    return MOE_UNSUPPORTED_SHAPE;
+  const long long R = s->capacity > 0 ? (long long)s->E * s->capacity : s->T * s->k;
+  if (R >= (1ll << 31) - 256) return MOE_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+static inline long long grouped_rows(const moe_shape* s) {
+  return s->capacity > 0 ? (long long)s->E * s->capacity : s->T * s->k;
+}
+
+static int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Router split-K so that small-T, wide-d routers still fill the GPU.
+static int router_splits(const moe_shape* s, int* k_per_split) {
+  const long long ctas = cdiv(s->T, kLgBM) * cdiv(s->E, kLgBN);
+  int ns = 1;
+  const long long want = 2ll * num_sms();
+  if (ctas < want) ns = (int)std::min<long long>(cdiv(want, ctas), std::max(1, s->d / 256));
+  int kps = (int)cdiv(cdiv(s->d, ns), kLgBK) * kLgBK;
+  ns = (int)cdiv(s->d, kps);
+  *k_per_split = kps;
+  return ns;
+}
+
+// ------------------------------------------------------------------ workspace layout
+
+struct Workspace {
+  size_t part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+};
+
+static Workspace ws_layout(const moe_shape* s) {
+  Workspace L{};
+  int kps = 0;
+  const int ns = router_splits(s, &kps);
+  const long long nchunks = cdiv(s->T, kChunk);
+  const long long R = grouped_rows(s);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  L.part = take((size_t)ns * s->T * s->E * 4);
+  L.cnt = take((size_t)nchunks * s->E * 4);
+  L.psum = take((size_t)nchunks * s->E * 4);
+  L.idx = take((size_t)s->T * s->k * 4);
+  L.w = take((size_t)s->T * s->k * 4);
+  L.counts = take((size_t)s->E * 4);
+  L.fP = take((size_t)2 * s->E * 4 + 16);
+  L.slot = take((size_t)s->T * s->k * 4);
+  L.drop = take((size_t)s->T * s->k);
+  L.kept = take((size_t)s->E * 4);
+  L.offs = take((size_t)(s->E + 1) * 4);
+  L.xperm = take((size_t)R * s->d * 2);
+  L.h = take((size_t)R * s->H * 2);
+  L.yperm = take((size_t)R * s->d * 2);
+  L.hs = take((size_t)s->T * std::max(s->H_s, 16) * 2);
+  L.ys = take((size_t)s->T * s->d * 2);
+  L.shtab = take(64);
+  L.total = o;
+  return L;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [outer..., rows, K] (K innermost), box = 64 x box_rows (x 1).
+static int make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, int box_rows) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return MOE_CUDA_ERROR;
+  cuuint64_t strides[2];
+  strides[0] = dims[0] * 2;
+  if (rank == 3) strides[1] = dims[0] * dims[1] * 2;
+  cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_CUDA_ERROR;
+}
+
+template <int MODE, int BN>
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, long long ub_mtiles,
+                         cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int OUTN = MODE != kModePlain ? BN / 2 : BN;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)Cfg::kSmemBytes));
+  const long long tiles = ub_mtiles * cdiv(p.N, OUTN);
+  const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
+  k_grouped_gemm<MODE, BN><<<grid, 256, Cfg::kSmemBytes, st>>>(ta, tb, p);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+// out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
+static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
+                        int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
+                        cudaStream_t st) {
+  if (R == 0) return MOE_OK;
+  int BN;
+  if (mode == kModePlain) BN = N >= 256 ? 256 : (N >= 128 ? 128 : 64);
+  else BN = N >= 128 ? 256 : (N >= 64 ? 128 : 64);
+  const int box_rows = mode == kModePlain ? BN : BN / 2;
+  CUtensorMap ta, tb;
+  cuuint64_t da[2] = {(cuuint64_t)K, (cuuint64_t)R};
+  cuuint64_t db[3] = {(cuuint64_t)K, (cuuint64_t)b_rows, (cuuint64_t)n_groups};
+  int rc = make_map(&ta, A, 2, da, kBM);
+  if (rc) return rc;
+  rc = make_map(&tb, B, 3, db, box_rows);
+  if (rc) return rc;
+  GemmParams p;
+  p.group_start = gstart;
+  p.group_rows = grows;
+  p.n_groups = n_groups;
+  p.R = R;
+  p.K = K;
+  p.N = N;
+  p.up_row0 = up_row0;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.ldo = N;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
+#define MOE_GEMM_CASE(M_, BN_) \
+  if (mode == M_ && BN == BN_) return launch_gemm_t<M_, BN_>(ta, tb, p, ub, st);
+  MOE_GEMM_CASE(kModePlain, 256) MOE_GEMM_CASE(kModePlain, 128) MOE_GEMM_CASE(kModePlain, 64)
+  MOE_GEMM_CASE(kModeSwiGLU, 256) MOE_GEMM_CASE(kModeSwiGLU, 128) MOE_GEMM_CASE(kModeSwiGLU, 64)
+  MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
+#undef MOE_GEMM_CASE
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
+// ------------------------------------------------------------------ launch helpers
+
+static int launch_topk(const moe_shape* s, const float* part, int nsplit, const float* bias, float* logits,
+                       int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st) {
+  const int nchunks = (int)cdiv(s->T, kChunk);
+  const int epl = (int)cdiv(s->E, 32);
+#define MOE_TOPK_CASE(N_)                                                                                         \
+  if (epl <= N_) {                                                                                                \
+    k_router_topk<N_><<<nchunks, 256, 0, st>>>(part, nsplit, bias, logits, idx, w, cnt, psum, (int)s->T, s->E,   \
+                                               s->k, s->renorm);                                                  \
+    MOE_LAUNCH_CHECK();                                                                                           \
+    return MOE_OK;                                                                                                \
+  }
+  MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(4) MOE_TOPK_CASE(8) MOE_TOPK_CASE(16)
+#undef MOE_TOPK_CASE
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
+static int launch_scan(const moe_shape* s, int32_t* cnt, const float* psum, int32_t* counts, float* f, float* P,
+                       cudaStream_t st) {
+  const int nchunks = (int)cdiv(s->T, kChunk);
+  k_chunk_scan<<<(int)cdiv(s->E, 8), 256, 0, st>>>(cnt, psum, counts, f, P, nchunks, s->E, (int)s->T);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx, const int32_t* cbase,
+                          const int32_t* counts, int32_t* slot, uint8_t* drop, int32_t* row_src, void* x_perm,
+                          int32_t* kept, int32_t* offs, cudaStream_t st) {
+  const int nchunks = (int)cdiv(s->T, kChunk);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(x_perm);
+#define MOE_SCATTER_CASE(N_)                                                                                  \
+  if (s->k <= N_) {                                                                                           \
+    k_scatter<N_><<<nchunks, 128, 0, st>>>(xb, idx, cbase, counts, (int)s->T, s->d, s->E, s->k, s->capacity, \
+                                           slot, drop, row_src, xp, kept, offs);                              \
+    MOE_LAUNCH_CHECK();                                                                                       \
+    return MOE_OK;                                                                                            \
+  }
+  MOE_SCATTER_CASE(2) MOE_SCATTER_CASE(4) MOE_SCATTER_CASE(8) MOE_SCATTER_CASE(16)
+#undef MOE_SCATTER_CASE
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
+static int route_impl(const moe_shape* s, const void* x, const float* w_router, const float* bias,
+                      const float* logits_in, float* logits, int32_t* idx, float* w, int32_t* counts, float* aux_f,
+                      float* aux_p, float* aux, uint8_t* ws, cudaStream_t st) {
+  const Workspace L = ws_layout(s);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  float* psum = reinterpret_cast<float*>(ws + L.psum);
+  float* f = aux_f ? aux_f : reinterpret_cast<float*>(ws + L.fP);
+  float* P = aux_p ? aux_p : reinterpret_cast<float*>(ws + L.fP) + s->E;
+  int rc;
+  int nsplit = 1;
+  if (logits_in == nullptr) {
+    int kps = 0;
+    nsplit = router_splits(s, &kps);
+    dim3 grid((unsigned)cdiv(s->T, kLgBM), (unsigned)cdiv(s->E, kLgBN), (unsigned)nsplit);
+    k_router_logits<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, part, (int)s->T,
+                                          s->d, s->E, kps);
+    MOE_LAUNCH_CHECK();
+    rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum, st);
+  } else {
+    rc = launch_topk(s, logits_in, 1, nullptr, nullptr, idx, w, cnt, psum, st);
+  }
+  if (rc) return rc;
+  const bool want_fp = aux_f || aux_p || aux;
+  rc = launch_scan(s, cnt, want_fp ? psum : nullptr, counts, want_fp ? f : nullptr, want_fp ? P : nullptr, st);
+  if (rc) return rc;
+  if (aux) {
+    k_aux_finalize<<<1, 32, 0, st>>>(f, P, aux, s->E);
+    MOE_LAUNCH_CHECK();
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_INVALID_ARGUMENT: return "invalid argument";
+    case MOE_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_CUDA_ERROR: return "CUDA error";
+    case MOE_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+int moe_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return MOE_INVALID_ARGUMENT;
+  g_wait_limit_ns.store(ns);
+  return MOE_OK;
+}
+
+int64_t moe_grouped_rows(const moe_shape* s) { return s ? grouped_rows(s) : -1; }
+
+int moe_capacity(int64_t T, int32_t k, int32_t E, double factor, int32_t* capacity) {
+  if (!capacity || T < 1 || k < 1 || E < 1 || !std::isfinite(factor)) return MOE_INVALID_ARGUMENT;
+  if (factor <= 0.0) { *capacity = 0; return MOE_OK; }
+  // factor as an exact decimal num / 10^6, then C = ceil(num * T * k / (10^6 * E)) in integers
+  const long long num = llround(factor * 1e6);
+  const __int128 top = (__int128)num * T * k;
+  const __int128 den = (__int128)1000000 * E;
+  const __int128 c = (top + den - 1) / den;
+  if (c > (1ll << 30)) return MOE_UNSUPPORTED_SHAPE;
+  *capacity = (int32_t)c;
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_shape* s, size_t* bytes) {
+  if (!bytes) return MOE_INVALID_ARGUMENT;
+  int rc = check_shape(s);
+  if (rc) return rc;
+  *bytes = ws_layout(s).total;
+  return MOE_OK;
+}
+
+int moe_route(const moe_shape* s, const void* x, const float* w_router, const float* bias, float* logits,
+              int32_t* topk_idx, float* topk_w, int32_t* counts, float* aux_f, float* aux_p, float* aux,
+              void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!x || !w_router || !topk_idx || !topk_w || !counts || !workspace) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(workspace)) return MOE_INVALID_ARGUMENT;
+  if (ws_bytes < ws_layout(s).total) return MOE_WORKSPACE_TOO_SMALL;
+  return route_impl(s, x, w_router, bias, nullptr, logits, topk_idx, topk_w, counts, aux_f, aux_p, aux,
+                    reinterpret_cast<uint8_t*>(workspace), stream);
+}
+
+int moe_route_from_logits(const moe_shape* s, const float* logits, int32_t* topk_idx, float* topk_w,
+                          int32_t* counts, float* aux_f, float* aux_p, float* aux, void* workspace,
+                          size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!logits || !topk_idx || !topk_w || !counts || !workspace) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(workspace)) return MOE_INVALID_ARGUMENT;
+  if (ws_bytes < ws_layout(s).total) return MOE_WORKSPACE_TOO_SMALL;
+  return route_impl(s, nullptr, nullptr, nullptr, logits, nullptr, topk_idx, topk_w, counts, aux_f, aux_p, aux,
+                    reinterpret_cast<uint8_t*>(workspace), stream);
+}
+
+int moe_permute(const moe_shape* s, const void* x, const int32_t* topk_idx, int32_t* slot_pos,
+                uint8_t* drop_mask, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_src,
+                void* x_perm, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!x || !topk_idx || !slot_pos || !kept || !offsets || !x_perm || !workspace) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(workspace)) return MOE_INVALID_ARGUMENT;
+  const Workspace L = ws_layout(s);
+  if (ws_bytes < L.total) return MOE_WORKSPACE_TOO_SMALL;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  int32_t* cts = counts ? counts : reinterpret_cast<int32_t*>(ws + L.counts);
+  const int nchunks = (int)cdiv(s->T, kChunk);
+  k_chunk_hist<<<nchunks, 256, s->E * sizeof(int), stream>>>(topk_idx, cnt, (int)s->T, s->E, s->k);
+  MOE_LAUNCH_CHECK();
+  rc = launch_scan(s, cnt, nullptr, cts, nullptr, nullptr, stream);
+  if (rc) return rc;
+  return launch_scatter(s, x, topk_idx, cnt, cts, slot_pos, drop_mask, row_src, x_perm, kept, offsets, stream);
+}
+
+int moe_expert_ffn(const moe_shape* s, int32_t n_groups, int32_t hidden, int64_t R, const void* x_grouped,
+                   const int32_t* group_start, const int32_t* group_rows, const void* w13, const void* s13,
+                   const void* w2, const void* s2, void* h, void* y, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (n_groups < 1 || n_groups > kMaxGroupsSmem || R < 0 || R >= (1ll << 31) - 256) return MOE_INVALID_ARGUMENT;
+  if (hidden < 16 || hidden % 16 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if ((group_start == nullptr) != (group_rows == nullptr)) return MOE_INVALID_ARGUMENT;
+  if (group_start == nullptr && n_groups != 1) return MOE_INVALID_ARGUMENT;
+  if (!x_grouped || !w13 || !w2 || !h || !y) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x_grouped) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
+    return MOE_INVALID_ARGUMENT;
+  if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
+  const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
+  rc = grouped_gemm(mode, x_grouped, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, group_start, group_rows,
+                    h, stream);
+  if (rc) return rc;
+  return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, group_start, group_rows, y, stream);
+}
+
+int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
+                const void* y_shared, void* out, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!y_perm || !slot_pos || !topk_w || !out) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(y_perm) || !aligned16(out) || (y_shared && !aligned16(y_shared))) return MOE_INVALID_ARGUMENT;
+  k_combine<<<(unsigned)cdiv(s->T, 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(y_perm), slot_pos, topk_w,
+      reinterpret_cast<const __nv_bfloat16*>(y_shared), reinterpret_cast<__nv_bfloat16*>(out), (int)s->T, s->d,
+      s->k);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+int moe_forward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                const void* s13, const void* w2, const void* s2, const void* w13_sh, const void* s13_sh,
+                const void* w2_sh, const void* s2_sh, void* out, int32_t* topk_idx, float* topk_w,
+                int32_t* counts, uint8_t* drop_mask, float* aux_f, float* aux_p, float* aux, void* workspace,
+                size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!x || !w_router || !w13 || !w2 || !out || !workspace) return MOE_INVALID_ARGUMENT;
+  if (s->H_s > 0 && (!w13_sh || !w2_sh)) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return MOE_INVALID_ARGUMENT;
+  if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
+  const Workspace L = ws_layout(s);
+  if (ws_bytes < L.total) return MOE_WORKSPACE_TOO_SMALL;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* idx = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = topk_w ? topk_w : reinterpret_cast<float*>(ws + L.w);
+  int32_t* cts = counts ? counts : reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + L.slot);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
+  int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offs);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  void* xperm = ws + L.xperm;
+  void* hbuf = ws + L.h;
+  void* yperm = ws + L.yperm;
+  const long long R = grouped_rows(s);
+
+  rc = route_impl(s, x, w_router, bias, nullptr, nullptr, idx, w, cts, aux_f, aux_p, aux, ws, stream);
+  if (rc) return rc;
+  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream);
+  if (rc) return rc;
+  const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
+  rc = grouped_gemm(mode, xperm, R, s->d, w13, s->E, 2 * s->H, s->H, s->H, offs, kept, hbuf, stream);
+  if (rc) return rc;
+  rc = grouped_gemm(kModePlain, hbuf, R, s->H, w2, s->E, s->d, 0, s->d, offs, kept, yperm, stream);
+  if (rc) return rc;
+  void* ys = nullptr;
+  if (s->H_s > 0) {
+    void* hs = ws + L.hs;
+    ys = ws + L.ys;
+    rc = grouped_gemm(mode, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, s->H_s, s->H_s, nullptr, nullptr, hs, stream);
+    if (rc) return rc;
+    rc = grouped_gemm(kModePlain, hs, s->T, s->H_s, w2_sh, 1, s->d, 0, s->d, nullptr, nullptr, ys, stream);
+    if (rc) return rc;
+  }
+  return moe_combine(s, yperm, slot, w, ys, out, stream);
+}
+
+int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream) {
+  if (!w || !q || !scales || rows < 0 || K <= 0 || K % 128 != 0) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(w) || (reinterpret_cast<uintptr_t>(q) & 1u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return MOE_INVALID_ARGUMENT;
+  if (rows == 0) return MOE_OK;
+  const long long items = rows * (K / 128);
+  k_quantize_int4<<<(unsigned)cdiv(items, 8), 256, 0, stream>>>(w, rows, K, q,
+                                                                 reinterpret_cast<__nv_bfloat16*>(scales));
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+int moe_get_status(moe_stream_t stream, int32_t* device_status, uint32_t* site) {
+  if (!device_status) return MOE_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_CUDA_ERROR;
+  unsigned int st = 0, where = 0, zero = 0;
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(&st, g_status, sizeof(st)));
+  MOE_CUDA_TRY(cudaMemcpyFromSymbol(&where, g_status_site, sizeof(where)));
+  MOE_CUDA_TRY(cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)));
+  MOE_CUDA_TRY(cudaMemcpyToSymbol(g_status_site, &zero, sizeof(zero)));
+  *device_status = (int32_t)st;
+  if (site) *site = where;
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace moe {
+// One mbarrier that nothing arrives on; the bounded wait must give up.
+__global__ void k_selftest_wait(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, limit_ns, &abort_flag, 0x7F01);
+}
+}  // namespace moe
+
+extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
+  moe::k_selftest_wait<<<1, 32, 0, stream>>>(moe::g_wait_limit_ns.load());
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR;
+}

@@ -1,0 +1,246 @@
+// Grouping by expert with (token, slot) identity kept, and the weighted combine.
+//
+// Grouping: ExpertMesh README ("Activation grouping that preserves token and
+// top-k slot identity"; flowchart "Group activations by expert owner"), with
+// the MoEEvolve README's capacity-factor static-shape dispatch: group e holds
+// rows [e*C, e*C + kept_e), overflow dropped in token order.  The rank of an
+// assignment is the number of earlier tokens that chose the same expert,
+// computed from per-chunk prefix sums and in-warp ballots, never from atomics
+// whose order varies, so the layout is canonical and bit-reproducible.
+//
+// Combine: ExpertMesh flowchart "Weighted top-k reduction", moe_stream.py
+// ``out[mask] += w * expert_out``, Kvasir ``combine(p, partials) + shared(cur)``.
+#pragma once
+
+#include "common.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+constexpr int kMaxE = 512;
+
+// Block-wide exclusive scan of group sizes (blockDim.x == 128, E <= 512):
+// s_off[e] = first row of group e, s_off[E] = total.  With cap > 0 the groups
+// are fixed slabs of cap rows.
+__device__ __forceinline__ void group_offsets(const int32_t* __restrict__ counts, int E, int cap, int* s_off,
+                                              int* s_kept, int* s_tmp) {
+  const int tid = threadIdx.x;
+  const int per = (E + 127) / 128;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int local = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    const int kv = cap > 0 ? min(c, cap) : c;
+    s_kept[e] = kv;
+    local += cap > 0 ? cap : kv;
+  }
+  int incl = local;
+  const int lane = lane_id(), warp = warp_id();
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_tmp[warp] = incl;
+  __syncthreads();
+  int wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += s_tmp[w];
+  int run = wbase + incl - local;
+  for (int e = e0; e < e1; ++e) {
+    s_off[e] = run;
+    run += cap > 0 ? cap : s_kept[e];
+  }
+  if (tid == 127) s_off[E] = wbase + incl;
+  __syncthreads();
+}
+
+// One CTA (128 threads, one token per thread) per chunk of 128 tokens.
+template <int KMAX>
+__global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict__ x,
+                                                 const int32_t* __restrict__ topk_idx,
+                                                 const int32_t* __restrict__ cbase, const int32_t* __restrict__ counts,
+                                                 int T, int d, int E, int k, int cap, int32_t* __restrict__ slot_pos,
+                                                 uint8_t* __restrict__ drop, int32_t* __restrict__ row_src,
+                                                 __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ kept_out,
+                                                 int32_t* __restrict__ offsets_out) {
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_kept[kMaxE];
+  __shared__ int s_base[kMaxE];
+  __shared__ int s_wcnt[4][kMaxE];
+  __shared__ int s_tmp[4];
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  const int chunk = blockIdx.x;
+
+  group_offsets(counts, E, cap, s_off, s_kept, s_tmp);
+  if (chunk == 0) {
+    for (int e = tid; e < E; e += 128) {
+      if (kept_out) kept_out[e] = s_kept[e];
+      if (offsets_out) offsets_out[e] = s_off[e];
+    }
+    if (tid == 0 && offsets_out) offsets_out[E] = s_off[E];
+  }
+  for (int e = tid; e < E; e += 128) {
+    s_base[e] = cbase[(size_t)chunk * E + e];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) s_wcnt[w][e] = 0;
+  }
+  __syncthreads();
+
+  const int t = chunk * kChunk + tid;
+  const bool valid = t < T;
+  int ex[KMAX], rk[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    ex[j] = (valid && j < k) ? topk_idx[(size_t)t * k + j] : -1;
+    rk[j] = 0;
+  }
+  unsigned pending = valid ? ((1u << k) - 1u) : 0u;
+  const unsigned lt = (1u << lane) - 1u;
+  // In-warp ranks: one ballot per distinct expert present in the warp.
+  while (true) {
+    const unsigned active = __ballot_sync(0xffffffffu, pending != 0u);
+    if (active == 0u) break;
+    const int leader = __ffs(active) - 1;
+    int mykey = -1;
+    if (pending) {
+      const int jj = __ffs(pending) - 1;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j == jj) mykey = ex[j];
+    }
+    const int key = __shfl_sync(0xffffffffu, mykey, leader);
+    int myslot = -1;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (((pending >> j) & 1u) && ex[j] == key) myslot = j;
+    const unsigned mask = __ballot_sync(0xffffffffu, myslot >= 0);
+    if (myslot >= 0) {
+      const int r = __popc(mask & lt);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j == myslot) rk[j] = r;
+      pending &= ~(1u << myslot);
+    }
+    if (lane == leader) s_wcnt[warp][key] = __popc(mask);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += 128) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int v = s_wcnt[w][e];
+      s_wcnt[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+
+  int pos[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    pos[j] = -1;
+    if (valid && j < k) {
+      const int e = ex[j];
+      const int rank = s_base[e] + s_wcnt[warp][e] + rk[j];
+      const bool dropped = cap > 0 && rank >= cap;
+      pos[j] = dropped ? -1 : s_off[e] + rank;
+      slot_pos[(size_t)t * k + j] = pos[j];
+      if (drop) drop[(size_t)t * k + j] = dropped ? 1 : 0;
+      if (!dropped && row_src) row_src[pos[j]] = t * k + j;
+    }
+  }
+
+  // Row moves: the warp copies each of its tokens' rows to the token's kept rows, 16 bytes per lane.
+  const int nvec = d >> 3;
+  for (int tok = 0; tok < 32; ++tok) {
+    const int tt = chunk * kChunk + warp * 32 + tok;
+    if (tt >= T) break;
+    int p[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) p[j] = __shfl_sync(0xffffffffu, pos[j], tok);
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tt * d);
+    for (int v = lane; v < nvec; v += 32) {
+      const uint4 val = src[v];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && p[j] >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)p[j] * d)[v] = val;
+    }
+  }
+}
+
+// Write the group table of moe_permute-style outputs without moving rows:
+// used by moe_forward when only the tables are needed.  (kept, offsets)
+__global__ void __launch_bounds__(128) k_group_table(const int32_t* __restrict__ counts, int E, int cap,
+                                                     int32_t* __restrict__ kept_out, int32_t* __restrict__ offsets_out) {
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_kept[kMaxE];
+  __shared__ int s_tmp[4];
+  group_offsets(counts, E, cap, s_off, s_kept, s_tmp);
+  for (int e = threadIdx.x; e < E; e += 128) {
+    kept_out[e] = s_kept[e];
+    offsets_out[e] = s_off[e];
+  }
+  if (threadIdx.x == 0) offsets_out[E] = s_off[E];
+}
+
+// ---------------------------------------------------------------------------
+// Combine: one warp per token, fp32 sum over slots j = 0..k-1 in order, then
+// the shared expert, one bf16 rounding.  Columns processed 1024 at a time.
+__global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ y_perm,
+                                                 const int32_t* __restrict__ slot_pos, const float* __restrict__ w,
+                                                 const __nv_bfloat16* __restrict__ y_shared,
+                                                 __nv_bfloat16* __restrict__ out, int T, int d, int k) {
+  const int t = blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (t >= T) return;
+  const int nvec = d >> 3;
+  for (int v0 = 0; v0 < nvec; v0 += 128) {
+    float acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int p = slot_pos[(size_t)t * k + j];
+      if (p < 0) continue;
+      const float g = w[(size_t)t * k + j];
+      const uint4* src = reinterpret_cast<const uint4*>(y_perm + (size_t)p * d);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int v = v0 + lane + 32 * i;
+        if (v < nvec) {
+          const uint4 u = src[v];
+          acc[i][0] = fmaf(g, bf16lo(u.x), acc[i][0]); acc[i][1] = fmaf(g, bf16hi(u.x), acc[i][1]);
+          acc[i][2] = fmaf(g, bf16lo(u.y), acc[i][2]); acc[i][3] = fmaf(g, bf16hi(u.y), acc[i][3]);
+          acc[i][4] = fmaf(g, bf16lo(u.z), acc[i][4]); acc[i][5] = fmaf(g, bf16hi(u.z), acc[i][5]);
+          acc[i][6] = fmaf(g, bf16lo(u.w), acc[i][6]); acc[i][7] = fmaf(g, bf16hi(u.w), acc[i][7]);
+        }
+      }
+    }
+    if (y_shared != nullptr) {
+      const uint4* src = reinterpret_cast<const uint4*>(y_shared + (size_t)t * d);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int v = v0 + lane + 32 * i;
+        if (v < nvec) {
+          const uint4 u = src[v];
+          acc[i][0] += bf16lo(u.x); acc[i][1] += bf16hi(u.x); acc[i][2] += bf16lo(u.y); acc[i][3] += bf16hi(u.y);
+          acc[i][4] += bf16lo(u.z); acc[i][5] += bf16hi(u.z); acc[i][6] += bf16lo(u.w); acc[i][7] += bf16hi(u.w);
+        }
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * d);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int v = v0 + lane + 32 * i;
+      if (v < nvec) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[i][0], acc[i][1]); o.y = pack_bf16x2(acc[i][2], acc[i][3]);
+        o.z = pack_bf16x2(acc[i][4], acc[i][5]); o.w = pack_bf16x2(acc[i][6], acc[i][7]);
+        dst[v] = o;
+      }
+    }
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,289 @@
+// Router: logits GEMM (fp32 SIMT), then per-token softmax, top-k with
+// lowest-index tie-break, gates, and per-chunk statistics.
+//
+// Follows "Sharding d'experts" (Kvasir wiki), "Backbone x worker":
+// ``ids, p = top_k(softmax(cur @ router), k)`` and moe_stream.py
+// ``MoEFFN.forward`` (bias-free gate Linear, additive exploration bias on the
+// logits, softmax, topk, gates divided by their sum, batch-local load-balance
+// fractions).  Top-k is taken on the logits: softmax is monotone, and the
+// logits carry the tie information that rounded probabilities can lose.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kChunk = 128;  // tokens per router / permute chunk (one CTA)
+
+// ---------------------------------------------------------------------------
+// logits_part[split][T][E] = sum over this split's K range of x[t,i] * W_r[e,i]
+//   x bf16 [T, d], W_r fp32 [E, d].  128 x 64 output tile per CTA, 128 threads,
+//   8 x 8 outputs per thread, K staged through shared memory 32 at a time.
+constexpr int kLgBM = 128, kLgBN = 64, kLgBK = 32;
+
+__global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ W, float* __restrict__ part,
+                                                       int T, int d, int E, int k_per_split) {
+  __shared__ __align__(16) float As[kLgBK][kLgBM + 4];
+  __shared__ __align__(16) float Bs[kLgBK][kLgBN + 4];
+  const int m0 = blockIdx.x * kLgBM, n0 = blockIdx.y * kLgBN;
+  const int kbeg = blockIdx.z * k_per_split;
+  const int kend = min(d, kbeg + k_per_split);
+  const int tid = threadIdx.x;
+  const int tx = tid & 7, ty = tid >> 3;  // 8 x 16 threads: n block tx*8, m block ty*8
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = kbeg; k0 < kend; k0 += kLgBK) {
+    // A: 128 rows x 32 bf16 = 512 chunks of 8 bf16; 4 per thread
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int c = tid + it * 128;
+      const int r = c >> 2, kc = (c & 3) * 8;
+      const int gm = m0 + r, gk = k0 + kc;
+      float v[8];
+      if (gm < T && gk + 8 <= kend) {
+        const uint4 u = *reinterpret_cast<const uint4*>(x + (size_t)gm * d + gk);
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+        v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          v[q] = (gm < T && gk + q < kend) ? __bfloat162float(x[(size_t)gm * d + gk + q]) : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) As[kc + q][r] = v[q];
+    }
+    // B: 64 rows x 32 fp32 = 512 chunks of 4; 4 per thread
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int c = tid + it * 128;
+      const int r = c >> 3, kc = (c & 7) * 4;
+      const int gn = n0 + r, gk = k0 + kc;
+      float4 v;
+      if (gn < E && gk + 4 <= kend) {
+        v = *reinterpret_cast<const float4*>(W + (size_t)gn * d + gk);
+      } else {
+        v.x = (gn < E && gk + 0 < kend) ? W[(size_t)gn * d + gk + 0] : 0.f;
+        v.y = (gn < E && gk + 1 < kend) ? W[(size_t)gn * d + gk + 1] : 0.f;
+        v.z = (gn < E && gk + 2 < kend) ? W[(size_t)gn * d + gk + 2] : 0.f;
+        v.w = (gn < E && gk + 3 < kend) ? W[(size_t)gn * d + gk + 3] : 0.f;
+      }
+      Bs[kc + 0][r] = v.x; Bs[kc + 1][r] = v.y; Bs[kc + 2][r] = v.z; Bs[kc + 3][r] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kLgBK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = part + (size_t)blockIdx.z * T * E;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int gm = m0 + ty * 8 + i;
+    if (gm >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gn = n0 + tx * 8 + j;
+      if (gn < E) out[(size_t)gm * E + gn] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One warp per token.  Lane l holds the logits of experts l, l+32, ...
+//   logits = sum_split part[split] (+ bias); softmax; top-k; gates.
+// Per chunk of kChunk tokens (one CTA, 8 warps x 16 tokens):
+//   cnt[chunk][e]  tokens of the chunk that chose e
+//   psum[chunk][e] sum over the chunk's tokens of p[t,e] (fixed order)
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ part, int nsplit,
+                                                     const float* __restrict__ bias, float* __restrict__ logits_out,
+                                                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                                     int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
+                                                     int E, int k, int renorm) {
+  __shared__ float s_p[8][EPL * 32];
+  __shared__ int s_c[8][EPL * 32];
+  const int lane = lane_id(), warp = warp_id();
+  const int chunk = blockIdx.x;
+  float pacc[EPL];
+  int cacc[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) { pacc[i] = 0.f; cacc[i] = 0; }
+  float b[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    b[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+  }
+
+  for (int tt = 0; tt < kChunk / 8; ++tt) {
+    const int t = chunk * kChunk + warp * (kChunk / 8) + tt;
+    if (t >= T) break;
+    float z[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      float v = -INFINITY;
+      if (e < E) {
+        v = part[(size_t)t * E + e];
+        for (int s = 1; s < nsplit; ++s) v += part[(size_t)s * T * E + (size_t)t * E + e];
+        if (bias != nullptr) v += b[i];
+        if (logits_out != nullptr) logits_out[(size_t)t * E + e] = v;
+      }
+      z[i] = v;
+    }
+    // softmax
+    float m = z[0];
+#pragma unroll
+    for (int i = 1; i < EPL; ++i) m = fmaxf(m, z[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ez[EPL], ssum = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      ez[i] = (lane + 32 * i < E) ? expf(z[i] - m) : 0.f;
+      ssum += ez[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    const float inv = 1.f / ssum;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) pacc[i] += ez[i] * inv;
+
+    // top-k: k rounds of warp argmax on (logit desc, index asc)
+    unsigned taken = 0u;
+    float wsel[16];
+    int isel[16];
+    float wsum = 0.f;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) {
+        const int i = bi >> 5;
+        taken |= 1u << i;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+          if (q == i) cacc[q] += 1;
+      }
+      const float pj = expf(bv - m) * inv;
+      wsel[j] = pj;
+      isel[j] = bi;
+      wsum += pj;
+    }
+    if (lane < k) {
+      float wv = 0.f;
+      int iv = 0;
+      for (int j = 0; j < k; ++j)
+        if (j == lane) { wv = wsel[j]; iv = isel[j]; }
+      topk_idx[(size_t)t * k + lane] = iv;
+      topk_w[(size_t)t * k + lane] = renorm ? wv / wsum : wv;
+    }
+  }
+  // chunk statistics: warps combined in fixed order
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) { s_p[warp][lane + 32 * i] = pacc[i]; s_c[warp][lane + 32 * i] = cacc[i]; }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ps = 0.f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
+    cnt[(size_t)chunk * E + e] = cs;
+    psum[(size_t)chunk * E + e] = ps;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-chunk expert histogram from caller routing (moe_permute without moe_route).
+__global__ void __launch_bounds__(256) k_chunk_hist(const int32_t* __restrict__ topk_idx, int32_t* __restrict__ cnt,
+                                                    int T, int E, int k) {
+  extern __shared__ int s_h[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_h[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kChunk;
+  const int n = min(kChunk, T - t0) * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = topk_idx[(size_t)t0 * k + i];
+    atomicAdd(&s_h[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)blockIdx.x * E + e] = s_h[e];
+}
+
+// ---------------------------------------------------------------------------
+// One warp per expert: cnt[c][e] -> exclusive prefix over chunks (in place),
+// counts[e]; optional f[e] = counts/T, P[e] = sum_c psum[c][e] / T.
+__global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, const float* __restrict__ psum,
+                                                    int32_t* __restrict__ counts, float* __restrict__ f_out,
+                                                    float* __restrict__ p_out, int nchunks, int E, int T) {
+  const int e = blockIdx.x * 8 + warp_id();
+  const int lane = lane_id();
+  if (e >= E) return;
+  const int per = (nchunks + 31) / 32;
+  const int c0 = min(nchunks, lane * per), c1 = min(nchunks, c0 + per);
+  int seg = 0;
+  float ps = 0.f;
+  for (int c = c0; c < c1; ++c) {
+    seg += cnt[(size_t)c * E + e];
+    if (psum != nullptr) ps += psum[(size_t)c * E + e];
+  }
+  int incl = seg;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - seg;
+  for (int c = c0; c < c1; ++c) {
+    const int v = cnt[(size_t)c * E + e];
+    cnt[(size_t)c * E + e] = run;
+    run += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (psum != nullptr) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+  }
+  if (lane == 0) {
+    if (counts != nullptr) counts[e] = total;
+    if (f_out != nullptr) f_out[e] = (float)total / (float)T;
+    if (p_out != nullptr && psum != nullptr) p_out[e] = ps / (float)T;
+  }
+}
+
+// aux = E * sum_e f_e P_e, one warp, fixed order.
+__global__ void k_aux_finalize(const float* __restrict__ f, const float* __restrict__ P, float* __restrict__ aux,
+                               int E) {
+  float s = 0.f;
+  for (int e = lane_id(); e < E; e += 32) s += f[e] * P[e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane_id() == 0) *aux = (float)E * s;
+}
+
+}  // namespace moe

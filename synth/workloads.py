@@ -193,3 +193,23 @@ def draw_logits(T: int, E: int, seed: int = 0, mode: str = "normal", device="cpu
     if mode == "equal":
         return torch.full((T, E), 0.5, device=device, dtype=torch.float32)
     raise ValueError(mode)
+
+
+def draw_groups(n_groups: int, max_rows: int, seed: int = 0, cap: int = 0, device="cpu"):
+    """Random group table for grouped-FFN tests: (start [G] int32, rows [G] int32, R).
+
+    Sizes are drawn in [0, max_rows] with some empty groups and some larger
+    than one 128-row tile.  ``cap > 0`` lays groups out as fixed slabs of
+    ``cap`` rows (sizes clipped to cap), else back to back.
+    """
+    g = _gen(seed, 5, "cpu")
+    rows = torch.randint(0, max_rows + 1, (n_groups,), generator=g)
+    rows[torch.randint(0, n_groups, (max(1, n_groups // 4),), generator=g)] = 0
+    if cap > 0:
+        rows = rows.clamp(max=cap)
+        start = torch.arange(n_groups) * cap
+        R = n_groups * cap
+    else:
+        start = torch.cumsum(rows, 0) - rows
+        R = int(rows.sum())
+    return start.to(torch.int32).to(device), rows.to(torch.int32).to(device), R

@@ -1,0 +1,311 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Routing, grouping and quantised codes must match bit for bit; float outputs
+must meet the layer tolerance (relative Frobenius <= 5e-3, max|delta| <= 3e-2)
+or the per-step tolerances derived in each test.  Inputs are drawn by
+``synth`` with fixed seeds; the oracle never receives a value computed by the
+CUDA path.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from helpers import MARGIN, assert_out_close, np64, npi, rel_frob, shape_of
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _shape(moe, T, E, k, d=16, H=16, H_s=0, cap=0, act=0, renorm=1, wfmt=0):
+    return moe.MoeShape(T=T, d=d, E=E, k=k, H=H, H_s=H_s, capacity=cap, act=act, wfmt=wfmt, renorm=renorm)
+
+
+# ---------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("T,E,k,renorm,mode", [(300, 8, 2, 1, "normal"), (1000, 192, 4, 1, "coarse"),
+                                               (257, 384, 8, 0, "signed_zero"), (64, 33, 5, 1, "equal"),
+                                               (130, 512, 16, 1, "normal"), (5, 3, 3, 0, "coarse"),
+                                               (129, 1, 1, 1, "normal")])
+def test_route_from_logits_bit_exact(lib, T, E, k, renorm, mode):
+    moe = lib
+    z = synth.draw_logits(T, E, seed=T + E, mode=mode)
+    s = _shape(moe, T, E, k, renorm=renorm)
+    r = moe.moe_route_from_logits(s, z.to(DEV), aux=True)
+    torch.cuda.synchronize()
+    z64 = z.double().numpy()
+    ref = O.route_from_logits(z64, k, bool(renorm))
+    assert (npi(r["topk_idx"]) == ref["idx"]).all()
+    assert (npi(r["counts"]) == ref["counts"]).all()
+    # fp32 softmax with expf and an E-term sum: relative error well inside 2e-5
+    np.testing.assert_allclose(np64(r["topk_w"]), ref["w"], rtol=2e-5, atol=1e-30)
+    np.testing.assert_allclose(np64(r["aux_f"]), ref["f"], rtol=1e-7)
+    np.testing.assert_allclose(np64(r["aux_p"]), ref["P"], rtol=2e-5, atol=1e-12)
+    np.testing.assert_allclose(np64(r["aux"])[0], ref["aux"], rtol=2e-5)
+
+
+def _route_case(moe, wl, T, seed):
+    wl = wl.replace(T=T)
+    inp = synth.make_inputs(wl, seed=seed, device="cpu", with_expert_weights=False)
+    s = shape_of(moe, wl)
+    bias = inp["bias"].to(DEV) if inp["bias"] is not None else None
+    r = moe.moe_route(s, inp["x"].to(DEV), inp["w_router"].to(DEV), bias, logits=True, aux=True)
+    torch.cuda.synchronize()
+    x64 = np64(inp["x"])
+    W64 = np64(inp["w_router"])
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref = O.route(x64, W64, b64, wl.k, bool(wl.renorm))
+    return wl, inp, r, ref, x64, W64, b64
+
+
+@pytest.mark.parametrize("name,T", [("tiny", 256), ("small", 4096), ("skewed", 3000), ("geglu", 2000),
+                                    ("decode_int4", 64)])
+def test_route_matches_oracle(lib, name, T):
+    wl, inp, r, ref, x64, W64, b64 = _route_case(lib, synth.get_workload(name), T, seed=1)
+    # logits: fp32 accumulation of d products; rigorous bound gamma_{d+2} * sum|x_i w_i| (+ |bias|)
+    zg = np64(r["logits"])
+    bound = (wl.d + 2) * 2.0 ** -24 * (np.abs(x64) @ np.abs(W64).T + (np.abs(b64) if b64 is not None else 0))
+    assert (np.abs(zg - ref["z"]) <= bound).all()
+    typical = np.abs(zg - ref["z"]).max()
+    assert typical < 2e-5, typical
+    # top-k: bit-exact where the oracle's k-th/(k+1)-th margin is >= 1e-5; inside the band any choice
+    # within the band is valid
+    margin = O.topk_margin(ref["z"], wl.k)
+    amb = margin < MARGIN
+    idx = npi(r["topk_idx"])
+    assert (idx[~amb] == ref["idx"][~amb]).all()
+    for t in np.nonzero(amb)[0]:
+        kth = np.sort(ref["z"][t])[::-1][wl.k - 1]
+        assert len(set(idx[t].tolist())) == wl.k
+        assert (ref["z"][t, idx[t]] >= kth - MARGIN).all()
+    if not amb.any():
+        assert (npi(r["counts"]) == ref["counts"]).all()
+        np.testing.assert_allclose(np64(r["topk_w"]), ref["w"], rtol=5e-5)
+        np.testing.assert_allclose(np64(r["aux_p"]), ref["P"], rtol=5e-5)
+        np.testing.assert_allclose(np64(r["aux"])[0], ref["aux"], rtol=5e-5)
+
+
+# ---------------------------------------------------------------- grouping
+
+
+@pytest.mark.parametrize("T,E,k,cap,skew,d", [(256, 8, 2, 0, 0.0, 64), (256, 8, 2, 32, 0.0, 64),
+                                              (1000, 192, 4, 0, 1.2, 768), (1000, 192, 4, 27, 1.2, 768),
+                                              (70, 384, 8, 0, 0.0, 256), (129, 5, 5, 0, 0.0, 16),
+                                              (4096, 32, 2, 300, 1.2, 128), (1, 4, 2, 1, 0.0, 32),
+                                              (300, 512, 16, 0, 0.5, 48)])
+def test_permute_bit_exact(lib, T, E, k, cap, skew, d):
+    moe = lib
+    idx = synth.draw_topk_idx(T, E, k, seed=T * 7 + E, skew=skew)
+    g = torch.Generator().manual_seed(T)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    s = _shape(moe, T, E, k, d=d, cap=cap)
+    r = moe.moe_permute(s, x.to(DEV), idx.to(DEV))
+    torch.cuda.synchronize()
+    ref = O.permute(npi(idx), E, cap)
+    for key in ("slot_pos", "counts", "kept", "offsets", "row_src"):
+        assert (npi(r[key]) == ref[key]).all(), key
+    assert (npi(r["drop_mask"]) == ref["drop"]).all()
+    rs = ref["row_src"]
+    filled = rs >= 0
+    xp = npi(r["x_perm"].view(torch.int16))
+    xs = npi(x.view(torch.int16))
+    assert (xp[filled] == xs[rs[filled] // k]).all()          # bit-exact row moves
+
+
+# ---------------------------------------------------------------- grouped expert FFN
+
+
+@pytest.mark.parametrize("E,d,H,act,max_rows,cap", [(4, 64, 128, 0, 300, 0), (8, 256, 1024, 0, 200, 0),
+                                                    (6, 768, 256, 1, 400, 300), (3, 128, 64, 0, 130, 0),
+                                                    (2, 64, 32, 1, 100, 0), (1, 96, 48, 0, 200, 0),
+                                                    (5, 256, 4096, 1, 140, 0)])
+def test_expert_ffn_matches_oracle(lib, E, d, H, act, max_rows, cap):
+    moe = lib
+    start, rows, R = synth.draw_groups(E, max_rows, seed=E * d + H, cap=cap)
+    wl = synth.Workload("t", T=1, d=d, E=E, k=1, H=H, act=act)
+    w13 = torch.stack([synth.expert_weights_f32(wl, 3, e)[0] for e in range(E)]).to(torch.bfloat16)
+    w2 = torch.stack([synth.expert_weights_f32(wl, 3, e)[1] for e in range(E)]).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(E + d)
+    xg = torch.randn(R, d, generator=g).to(torch.bfloat16)
+    s = _shape(moe, 1, E, 1, d=d, H=H, act=act)
+    h, y = moe.moe_expert_ffn(s, xg.to(DEV), w13.to(DEV), w2.to(DEV), hidden=H, group_start=start.to(DEV),
+                              group_rows=rows.to(DEV))
+    torch.cuda.synchronize()
+    x64, w13_64, w2_64 = np64(xg), np64(w13), np64(w2)
+    hg, yg = np64(h), np64(y)
+    for e in range(E):
+        a, n = int(start[e]), int(rows[e])
+        if n == 0:
+            continue
+        h_ref = O.glu_hidden(x64[a:a + n], w13_64[e], act)
+        y_ref = h_ref @ w2_64[e].T
+        assert_out_close(hg[a:a + n], h_ref, f"h[e={e}]")
+        assert_out_close(yg[a:a + n], y_ref, f"y[e={e}]")
+
+
+def test_expert_ffn_single_dense_group(lib):
+    moe = lib
+    wl = synth.Workload("t", T=1000, d=256, E=1, k=1, H=512)
+    w13, w2 = synth.expert_weights_f32(wl, 5, 0)
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(1000, 256, generator=g).to(torch.bfloat16)
+    s = _shape(moe, 1000, 1, 1, d=256, H=512)
+    h, y = moe.moe_expert_ffn(s, x.to(DEV), w13.to(torch.bfloat16)[None].to(DEV),
+                              w2.to(torch.bfloat16)[None].to(DEV), hidden=512)
+    torch.cuda.synchronize()
+    ref = O.expert_ffn(np64(x), np64(w13.to(torch.bfloat16)), np64(w2.to(torch.bfloat16)), 0)
+    assert_out_close(np64(y), ref)
+
+
+# ---------------------------------------------------------------- combine
+
+
+@pytest.mark.parametrize("T,E,k,cap,d,shared", [(256, 8, 2, 0, 64, False), (500, 16, 4, 100, 256, True),
+                                                (64, 384, 8, 0, 7168, True), (33, 4, 3, 5, 16, False)])
+def test_combine_matches_oracle(lib, T, E, k, cap, d, shared):
+    moe = lib
+    idx = synth.draw_topk_idx(T, E, k, seed=11, skew=1.0)
+    g = torch.Generator().manual_seed(T + d)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    s = _shape(moe, T, E, k, d=d, cap=cap)
+    p = moe.moe_permute(s, x.to(DEV), idx.to(DEV))
+    ref = O.permute(npi(idx), E, cap)
+    R = s.R
+    y_perm = torch.randn(R, d, generator=g).to(torch.bfloat16)
+    w = torch.rand(T, k, generator=g)
+    ysh = torch.randn(T, d, generator=g).to(torch.bfloat16) if shared else None
+    out = moe.moe_combine(s, y_perm.to(DEV), p["slot_pos"], w.to(DEV), ysh.to(DEV) if shared else None)
+    torch.cuda.synchronize()
+    assert (npi(p["slot_pos"]) == ref["slot_pos"]).all()
+    want = O.combine(np64(y_perm), ref["slot_pos"], np64(w), np64(ysh) if shared else None)
+    # fp32 sum of <= k+1 terms, one bf16 rounding: |delta| <= 2^-8 |out| + k * 2^-23 sum|terms|
+    got = np64(out)
+    bound = 2.0 ** -8 * np.abs(want) + 1e-6 * (np.abs(want) + 1)
+    assert (np.abs(got - want) <= bound).all()
+
+
+# ---------------------------------------------------------------- whole layer
+
+
+def _forward_case(moe, wl, seed=0, device="cpu"):
+    inp = synth.make_inputs(wl, seed=seed, device=device)
+    s = shape_of(moe, wl)
+    d_ = {k_: (v.to(DEV) if v is not None else None) for k_, v in inp.items()}
+    r = moe.moe_forward(s, d_["x"], d_["w_router"], d_["w13"], d_["w2"], bias=d_["bias"],
+                        w13_sh=d_.get("w13_sh"), w2_sh=d_.get("w2_sh"), routing=True, aux=wl.aux)
+    torch.cuda.synchronize()
+    st, site = moe.moe_get_status()
+    assert st == 0, (st, hex(site))
+    return inp, s, r
+
+
+def _check_forward(wl, inp, s, r, sample=None):
+    """Compare a GPU forward with the oracle; returns (n_excluded, rel, maxabs)."""
+    x64 = np64(inp["x"])
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref_r = O.route(x64, np64(inp["w_router"]), b64, wl.k, bool(wl.renorm))
+    idx_g = npi(r["topk_idx"])
+    amb = O.topk_margin(ref_r["z"], wl.k) < MARGIN
+    assert (idx_g[~amb] == ref_r["idx"][~amb]).all()
+    flipped = np.nonzero((idx_g != ref_r["idx"]).any(1))[0]
+    cap = s.capacity
+    perm = O.permute(ref_r["idx"], wl.E, cap)
+    excl = np.zeros(wl.T, bool)
+    excl[flipped] = True
+    if cap and flipped.size:
+        # a flipped token shifts the ranks of later tokens of the experts involved
+        aff = set(idx_g[flipped].ravel().tolist()) | set(ref_r["idx"][flipped].ravel().tolist())
+        later = np.arange(wl.T) > flipped.min()
+        excl |= later & np.isin(ref_r["idx"], list(aff)).any(1)
+        excl |= later & np.isin(idx_g, list(aff)).any(1)
+    assert (npi(r["drop_mask"])[~excl] == perm["drop"][~excl]).all()
+    if not flipped.size:
+        assert (npi(r["counts"]) == ref_r["counts"]).all()
+    toks = np.arange(wl.T) if sample is None else np.asarray(sample)
+    toks = toks[~excl[toks]]
+    w13 = inp["w13"]
+    w2 = inp["w2"]
+    out_ref = np.zeros((toks.size, wl.d))
+    for n, t in enumerate(toks):
+        for j in range(wl.k):
+            if perm["drop"][t, j]:
+                continue
+            e = int(ref_r["idx"][t, j])
+            out_ref[n] += ref_r["w"][t, j] * O.expert_ffn(x64[t:t + 1], np64(w13[e]), np64(w2[e]), wl.act)[0]
+    if wl.H_s:
+        out_ref += O.expert_ffn(x64[toks], np64(inp["w13_sh"][0]), np64(inp["w2_sh"][0]), wl.act)
+    got = np64(r["out"])[toks]
+    rel, mx = assert_out_close(got, out_ref)
+    if wl.aux:
+        np.testing.assert_allclose(np64(r["aux"])[0], ref_r["aux"], rtol=5e-5)
+    return int(excl.sum()), rel, mx
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("small", {}), ("tiny", {"capacity_factor": 0.5}),
+                                       ("tiny", {"H_s": 64, "act": 1, "skew": 1.2}),
+                                       ("tiny", {"renorm": 0, "k": 3}),
+                                       ("granular", {"T": 2048}), ("skewed", {"T": 2048}),
+                                       ("geglu", {"T": 512}),
+                                       ("granular", {"T": 1024, "skew": 1.2, "capacity_factor": 1.25})])
+def test_forward_matches_oracle(lib, name, over):
+    wl = synth.get_workload(name).replace(**over)
+    inp, s, r = _forward_case(lib, wl)
+    n_ex, rel, mx = _check_forward(wl, inp, s, r)
+    assert n_ex <= max(2, wl.T // 500)
+    if over.get("capacity_factor") == 0.5:
+        assert npi(r["drop_mask"]).sum() > 0
+
+
+@pytest.mark.parametrize("name", ["granular", "skewed", "geglu"])
+def test_forward_full_size_sampled(lib, name):
+    """Full workload size, the launch configuration the benchmark times; oracle on sampled tokens."""
+    wl = synth.get_workload(name)
+    inp, s, r = _forward_case(lib, wl, device=DEV)
+    inp = {k_: (v.cpu() if v is not None else None) for k_, v in inp.items()}
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([rng.choice(wl.T, 96, replace=False), [0, wl.T - 1]]))
+    n_ex, rel, mx = _check_forward(wl, inp, s, r, sample=sample)
+    assert n_ex <= wl.T // 500
+
+
+# ---------------------------------------------------------------- INT4 quantiser
+
+
+@pytest.mark.parametrize("rows,K", [(7, 128), (300, 7168), (4096, 256)])
+def test_quantize_int4_bit_exact(lib, rows, K):
+    moe = lib
+    g = torch.Generator().manual_seed(rows + K)
+    w = torch.randn(rows, K, generator=g) / math.sqrt(K)
+    w[0, :128] = 0.0                   # an all-zero group
+    w[1, :6] = torch.tensor([7.0, 0.5, 1.5, 2.5, -0.5, -7.0]) * 0.01
+    q, sc = moe.moe_quantize_int4(w.to(DEV))
+    torch.cuda.synchronize()
+    q_ref, s_ref = O.quantize_int4_g128(w.numpy())
+    assert (npi(q) == O.pack_int4(q_ref)).all()
+    assert (npi(sc.view(torch.int16)) == (s_ref.view(np.uint32) >> 16).astype(np.int16)).all()
+
+
+# ---------------------------------------------------------------- failure detection
+
+
+def test_bounded_wait_reports_timeout(lib):
+    moe = lib
+    L = moe.load()
+    assert moe.moe_get_status()[0] == 0
+    assert L.moe_set_wait_limit_ns(20_000_000) == 0           # 20 ms
+    try:
+        assert L.moe_selftest_wait_timeout(None) == 0
+        st, site = moe.moe_get_status(torch.cuda.default_stream())
+        assert st == 5                                         # MOE_DEVICE_TIMEOUT
+        assert site == 0x7F01
+        assert moe.moe_get_status()[0] == 0                    # read clears it
+    finally:
+        L.moe_set_wait_limit_ns(2_000_000_000)
+    # the context is still usable
+    x = torch.ones(4, device=DEV)
+    assert float(x.sum()) == 4.0
