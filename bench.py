@@ -50,6 +50,14 @@ def hbm_roofline_tokens_per_s(bandwidth_bytes_per_s: float, active_bytes_per_tok
     return bandwidth_bytes_per_s / active_bytes_per_token
 
 
+def int4_step_bytes(wl, touched: int) -> int:
+    """Algorithmic HBM bytes of one INT4 forward: touched experts' packed weights and scales, the shared
+    expert, the router weight, x in and out."""
+    per_expert = (2 * wl.H * wl.d + wl.d * wl.H) // 2 + (2 * wl.H * wl.d + wl.d * wl.H) // 128 * 2
+    shared = ((2 * wl.H_s * wl.d + wl.d * wl.H_s) // 2 + (2 * wl.H_s * wl.d + wl.d * wl.H_s) // 128 * 2) if wl.H_s else 0
+    return touched * per_expert + shared + wl.E * wl.d * 4 + 2 * wl.T * wl.d * 2
+
+
 def max_over_ranks(value: float, world: int) -> float:
     if world <= 1:
         return value
@@ -125,6 +133,8 @@ def setup(wl, seed, device):
     inp = synth.make_inputs(wl, seed=0, device=device)                # weights: same on every replica
     if seed:
         inp["x"] = synth.make_inputs(wl, seed=seed, device=device, with_expert_weights=False)["x"]
+    if wl.wfmt == synth.WFMT_INT4_G128:
+        inp.update(int4_weights(moe, wl, 0, device))
     C = moe.moe_capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
     s = moe.MoeShape(T=wl.T, d=wl.d, E=wl.E, k=wl.k, H=wl.H, H_s=wl.H_s, capacity=C, act=wl.act, wfmt=wl.wfmt,
                      renorm=wl.renorm)
@@ -133,9 +143,34 @@ def setup(wl, seed, device):
     return s, inp, ws, out
 
 
+def int4_weights(moe, wl, seed, device):
+    """Experts drawn in fp32 one at a time (synth) and packed by the library's INT4 quantiser."""
+    import torch
+
+    import synth
+    E, d, H = wl.E, wl.d, wl.H
+    out = dict(w13=torch.empty(E, 2 * H, d // 2, dtype=torch.uint8, device=device),
+               s13=torch.empty(E, 2 * H, d // 128, dtype=torch.bfloat16, device=device),
+               w2=torch.empty(E, d, H // 2, dtype=torch.uint8, device=device),
+               s2=torch.empty(E, d, H // 128, dtype=torch.bfloat16, device=device))
+    for e in range(E):
+        a, b = synth.expert_weights_f32(wl, seed, e, device)
+        moe.moe_quantize_int4(a, q=out["w13"][e], scales=out["s13"][e])
+        moe.moe_quantize_int4(b, q=out["w2"][e], scales=out["s2"][e])
+    if wl.H_s:
+        a, b = synth.expert_weights_f32(wl, seed, E, device)
+        q13, s13 = moe.moe_quantize_int4(a)
+        q2, s2 = moe.moe_quantize_int4(b)
+        out.update(w13_sh=q13[None], s13_sh=s13[None], w2_sh=q2[None], s2_sh=s2[None])
+    torch.cuda.synchronize()
+    return out
+
+
 def run_forward(moe, s, inp, ws, out, aux):
     return moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
-                           w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), out=out, ws=ws, aux=aux)
+                           s13=inp.get("s13"), s2=inp.get("s2"), w13_sh=inp.get("w13_sh"),
+                           s13_sh=inp.get("s13_sh"), w2_sh=inp.get("w2_sh"), s2_sh=inp.get("s2_sh"), out=out,
+                           ws=ws, aux=aux)
 
 
 def stage_times(moe, s, inp, ws, wl, flush, reps=10):
@@ -152,11 +187,12 @@ def stage_times(moe, s, inp, ws, wl, flush, reps=10):
         p = moe.moe_permute(s, inp["x"], r["topk_idx"], ws=ws)
         ev[2].record(st)
         h, y = moe.moe_expert_ffn(s, p["x_perm"], inp["w13"], inp["w2"], group_start=p["offsets"],
-                                  group_rows=p["kept"])
+                                  group_rows=p["kept"], s13=inp.get("s13"), s2=inp.get("s2"))
         ev[3].record(st)
         ysh = None
         if wl.H_s:
-            _, ysh = moe.moe_expert_ffn(s, inp["x"], inp["w13_sh"], inp["w2_sh"], hidden=wl.H_s)
+            _, ysh = moe.moe_expert_ffn(s, inp["x"], inp["w13_sh"], inp["w2_sh"], hidden=wl.H_s,
+                                        s13=inp.get("s13_sh"), s2=inp.get("s2_sh"))
         ev[4].record(st)
         moe.moe_combine(s, y, p["slot_pos"], r["topk_w"], ysh)
         ev[5].record(st)
@@ -164,7 +200,8 @@ def stage_times(moe, s, inp, ws, wl, flush, reps=10):
         for i, k in enumerate(acc):
             acc[k].append(ev[i].elapsed_time(ev[i + 1]) * 1e3)
         kept = int(p["kept"].sum())
-    return {k: statistics.median(v) for k, v in acc.items()}, kept
+        touched = int((p["kept"] > 0).sum())
+    return {k: statistics.median(v) for k, v in acc.items()}, kept, touched
 
 
 def cpu_oracle_sample(wl, budget_s=12.0, max_tokens=None):
@@ -180,6 +217,8 @@ def cpu_oracle_sample(wl, budget_s=12.0, max_tokens=None):
         threads = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
     except Exception:  # noqa: BLE001
         threads = cores
+    if wl.wfmt != 0:
+        return cpu_oracle_sample_int4(wl, budget_s, cores, threads)
     n = min(wl.T, max_tokens or wl.T)
     sub = wl.replace(T=n)
     inp = synth.make_inputs(sub, seed=0, device="cpu")
@@ -197,6 +236,43 @@ def cpu_oracle_sample(wl, budget_s=12.0, max_tokens=None):
             break
     return done / el, f"{done} tokens ({done // n} x {n}-token batches of the {wl.name} workload) in {el:.1f} s", \
         min(cores, threads) if threads else cores
+
+
+def cpu_oracle_sample_int4(wl, budget_s, cores, threads):  # noqa: C901
+    """INT4 workload: the oracle routes the whole batch, then quantises, dequantises and applies each
+    token's experts one token at a time until the time budget is spent."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    import synth
+    inp = synth.make_inputs(wl, seed=0, device="cpu", with_expert_weights=False)
+    x = inp["x"].to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    r = O.route(x, inp["w_router"].to(torch.float64).numpy(), None, wl.k, bool(wl.renorm))
+
+    def expert(e):
+        a, b = synth.expert_weights_f32(wl, 0, e, "cpu")
+        qa, sa = O.quantize_int4_g128(a.numpy())
+        qb, sb = O.quantize_int4_g128(b.numpy())
+        return O.dequantize_int4_g128(O.pack_int4(qa), sa), O.dequantize_int4_g128(O.pack_int4(qb), sb)
+
+    done = 0
+    while True:
+        t = done % wl.T
+        out = np.zeros(wl.d)
+        for j in range(wl.k):
+            w13, w2 = expert(int(r["idx"][t, j]))
+            out += r["w"][t, j] * O.expert_ffn(x[t:t + 1], w13, w2, wl.act)[0]
+        if wl.H_s:
+            w13, w2 = expert(wl.E)
+            out += O.expert_ffn(x[t:t + 1], w13, w2, wl.act)[0]
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, f"{done} tokens of the {wl.name} workload, routed in a full batch, experts dequantised " \
+        f"per token, {el:.1f} s", min(cores, threads) if threads else cores
 
 
 # ------------------------------------------------------------------ main
@@ -300,16 +376,26 @@ def main():
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
 
     # stage breakdown and the roofline of the grouped expert GEMMs
-    stages, kept = stage_times(moe, s, inp, ws, wl, flush)
+    stages, kept, touched = stage_times(moe, s, inp, ws, wl, flush)
     peaks = load_peaks()
     flops = wl.flops_tc(kept)
     gemm_us = stages["expert_ffn"] + stages["shared_ffn"]
-    achieved_tf = flops / (gemm_us * 1e-6) / 1e12
-    peak_tf = peaks["bf16_tflops"]
-    roofline = {"bound": "tensor", "kernel": "k_grouped_gemm (gate/up + GLU, down; routed + shared)",
-                "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                "peak_source": peaks["source"] + " burst bf16", "traffic": None,
-                "alg_flops_per_step": flops, "gemm_us": gemm_us}
+    if wl.wfmt == synth.WFMT_INT4_G128:
+        alg_bytes = int4_step_bytes(wl, touched)
+        achieved = alg_bytes / (step_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roofline = {"bound": "hbm", "kernel": "whole moe_forward (INT4 weight streaming dominates)",
+                    "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "peak_source": peaks["source"] + " HBM copy", "traffic": None,
+                    "alg_bytes_per_step": alg_bytes, "touched_experts": touched,
+                    "int4_gemm_GBps": (alg_bytes - wl.T * wl.d * 4 - wl.E * wl.d * 4) / (gemm_us * 1e-6) / 1e9}
+    else:
+        achieved_tf = flops / (gemm_us * 1e-6) / 1e12
+        peak_tf = peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "kernel": "k_grouped_gemm (gate/up + GLU, down; routed + shared)",
+                    "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
+                    "peak_source": peaks["source"] + " burst bf16", "traffic": None,
+                    "alg_flops_per_step": flops, "gemm_us": gemm_us}
 
     if rank == 0:
         cpu = None

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
+#include "int4_gemm.cuh"
 #include "permute.cuh"
 #include "quant.cuh"
 #include "router.cuh"
@@ -244,6 +245,49 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   return MOE_UNSUPPORTED_SHAPE;
 }
 
+static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const void* wq, const void* wsc,
+                     int n_groups, int b_rows, int up_row0, int N, const int32_t* gstart, const int32_t* grows,
+                     void* out, cudaStream_t st) {
+  if (R == 0) return MOE_OK;
+  Int4Params p;
+  p.wq = reinterpret_cast<const uint8_t*>(wq);
+  p.ws = reinterpret_cast<const __nv_bfloat16*>(wsc);
+  p.act = reinterpret_cast<const __nv_bfloat16*>(A);
+  p.group_start = gstart;
+  p.group_rows = grows;
+  p.n_groups = n_groups;
+  p.R = R;
+  p.K = K;
+  p.N = N;
+  p.b_rows = b_rows;
+  p.up_row0 = up_row0;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.ldo = N;
+  const long long ub_tasks = (long long)(grows ? std::min<long long>(n_groups, R) : 1) * (N / 16);
+  const int grid = (int)std::max<long long>(1, std::min<long long>(2ll * num_sms(), cdiv(ub_tasks, 8)));
+  if (!glu) k_int4_gemm<false, kModePlain><<<grid, 256, 0, st>>>(p);
+  else if (act == MOE_ACT_SWIGLU) k_int4_gemm<true, kModeSwiGLU><<<grid, 256, 0, st>>>(p);
+  else k_int4_gemm<true, kModeGeGLU><<<grid, 256, 0, st>>>(p);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+// Gated expert FFN over groups of rows: h = act(A W1^T) * (A W3^T), y = h W2^T.
+static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const void* A, const int32_t* gstart,
+                           const int32_t* grows, int n_groups, const void* w13, const void* s13, const void* w2,
+                           const void* s2, void* h, void* y, cudaStream_t st) {
+  int rc;
+  if (s->wfmt == MOE_WFMT_INT4_G128) {
+    rc = int4_gemm(true, s->act, A, R, s->d, w13, s13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st);
+    if (rc) return rc;
+    return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
+  }
+  const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
+  rc = grouped_gemm(mode, A, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st);
+  if (rc) return rc;
+  return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
+}
+
 static int route_impl(const moe_shape* s, const void* x, const float* w_router, const float* bias,
                       const float* logits_in, float* logits, int32_t* idx, float* w, int32_t* counts, float* aux_f,
                       float* aux_p, float* aux, uint8_t* ws, cudaStream_t st) {
@@ -381,15 +425,16 @@ int moe_expert_ffn(const moe_shape* s, int32_t n_groups, int32_t hidden, int64_t
   if (hidden < 16 || hidden % 16 != 0) return MOE_UNSUPPORTED_SHAPE;
   if ((group_start == nullptr) != (group_rows == nullptr)) return MOE_INVALID_ARGUMENT;
   if (group_start == nullptr && n_groups != 1) return MOE_INVALID_ARGUMENT;
+  if (R == 0) return MOE_OK;
   if (!x_grouped || !w13 || !w2 || !h || !y) return MOE_INVALID_ARGUMENT;
   if (!aligned16(x_grouped) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
     return MOE_INVALID_ARGUMENT;
-  if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
-  const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
-  rc = grouped_gemm(mode, x_grouped, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, group_start, group_rows,
-                    h, stream);
-  if (rc) return rc;
-  return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, group_start, group_rows, y, stream);
+  if (s->wfmt == MOE_WFMT_INT4_G128) {
+    if (hidden % 128 != 0) return MOE_UNSUPPORTED_SHAPE;
+    if (!s13 || !s2 || !aligned16(s13) || !aligned16(s2)) return MOE_INVALID_ARGUMENT;
+  }
+  return expert_ffn_impl(s, hidden, R, x_grouped, group_start, group_rows, n_groups, w13, s13, w2, s2, h, y,
+                         stream);
 }
 
 int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
@@ -418,7 +463,9 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return MOE_INVALID_ARGUMENT;
-  if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
+  if (s->wfmt == MOE_WFMT_INT4_G128 &&
+      (!s13 || !s2 || !aligned16(s13) || !aligned16(s2) || (s->H_s > 0 && (!s13_sh || !s2_sh))))
+    return MOE_INVALID_ARGUMENT;
   const Workspace L = ws_layout(s);
   if (ws_bytes < L.total) return MOE_WORKSPACE_TOO_SMALL;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
@@ -438,18 +485,13 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   if (rc) return rc;
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream);
   if (rc) return rc;
-  const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
-  rc = grouped_gemm(mode, xperm, R, s->d, w13, s->E, 2 * s->H, s->H, s->H, offs, kept, hbuf, stream);
-  if (rc) return rc;
-  rc = grouped_gemm(kModePlain, hbuf, R, s->H, w2, s->E, s->d, 0, s->d, offs, kept, yperm, stream);
+  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream);
   if (rc) return rc;
   void* ys = nullptr;
   if (s->H_s > 0) {
-    void* hs = ws + L.hs;
     ys = ws + L.ys;
-    rc = grouped_gemm(mode, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, s->H_s, s->H_s, nullptr, nullptr, hs, stream);
-    if (rc) return rc;
-    rc = grouped_gemm(kModePlain, hs, s->T, s->H_s, w2_sh, 1, s->d, 0, s->d, nullptr, nullptr, ys, stream);
+    rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
+                         stream);
     if (rc) return rc;
   }
   return moe_combine(s, yperm, slot, w, ys, out, stream);

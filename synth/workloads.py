@@ -204,7 +204,9 @@ def draw_groups(n_groups: int, max_rows: int, seed: int = 0, cap: int = 0, devic
     """
     g = _gen(seed, 5, "cpu")
     rows = torch.randint(0, max_rows + 1, (n_groups,), generator=g)
-    rows[torch.randint(0, n_groups, (max(1, n_groups // 4),), generator=g)] = 0
+    if n_groups >= 4:
+        rows[torch.randint(0, n_groups, (n_groups // 4,), generator=g)] = 0
+    rows[0] = max(int(rows[0]), 1)
     if cap > 0:
         rows = rows.clamp(max=cap)
         start = torch.arange(n_groups) * cap

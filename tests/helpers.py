@@ -42,3 +42,53 @@ def assert_out_close(got, want, what="out", rel=REL_FROB, atol=MAX_ABS):
     m = float(np.abs(got - want).max()) if got.size else 0.0
     assert r <= rel and m <= atol, f"{what}: rel Frobenius {r:.3e} (<= {rel}), max|d| {m:.3e} (<= {atol})"
     return r, m
+
+
+def assert_bf16_rounded(got, want, scale, what="value"):
+    """Elementwise bound for a bf16-rounded intermediate: |got - want| <= 2^-8 * (|want| + scale).
+
+    ``scale`` carries the propagated error of bf16-rounded inputs (e.g. |h| @ |W2|^T for y = h W2^T);
+    one bf16 rounding is at most 2^-9 relative, the factor 2 covers fp32 accumulation and the
+    approximate exp of the activation.
+    """
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    bound = 2.0 ** -8 * (np.abs(want) + scale) + 1e-6
+    bad = np.abs(got - want) > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements outside the bf16 bound, worst " \
+        f"{float((np.abs(got - want) / bound).max()):.2f}x"
+
+
+def int4_expert_weights(moe, wl, seed=0, device="cuda", experts=None):
+    """Draw every expert's fp32 weights with synth (on ``device``) and pack them with the library's INT4 quantiser.
+
+    Returns dict w13 [E,2H,d/2] u8, s13 [E,2H,d/128] bf16, w2 [E,d,H/2] u8, s2 [E,d,H/128] bf16 and, when
+    H_s > 0, the shared expert's w13_sh, s13_sh, w2_sh, s2_sh with a leading dim of 1.
+    """
+    import synth
+    E, d, H = wl.E, wl.d, wl.H
+    out = dict(w13=torch.empty(E, 2 * H, d // 2, dtype=torch.uint8, device=device),
+               s13=torch.empty(E, 2 * H, d // 128, dtype=torch.bfloat16, device=device),
+               w2=torch.empty(E, d, H // 2, dtype=torch.uint8, device=device),
+               s2=torch.empty(E, d, H // 128, dtype=torch.bfloat16, device=device))
+    for e in range(E):
+        a, b = synth.expert_weights_f32(wl, seed, e, device)
+        moe.moe_quantize_int4(a, q=out["w13"][e], scales=out["s13"][e])
+        moe.moe_quantize_int4(b, q=out["w2"][e], scales=out["s2"][e])
+    if wl.H_s:
+        a, b = synth.expert_weights_f32(wl, seed, E, device)
+        q13, s13 = moe.moe_quantize_int4(a)
+        q2, s2 = moe.moe_quantize_int4(b)
+        out.update(w13_sh=q13[None], s13_sh=s13[None], w2_sh=q2[None], s2_sh=s2[None])
+    return out
+
+
+def oracle_int4_expert(wl, seed, e, device="cuda"):
+    """float64 (w13, w2) of expert e after the oracle's own quantise -> dequantise of the same fp32 draws."""
+    import oracle as O
+    import synth
+    a, b = synth.expert_weights_f32(wl, seed, e, device)
+    qa, sa = O.quantize_int4_g128(a.cpu().numpy())
+    qb, sb = O.quantize_int4_g128(b.cpu().numpy())
+    return (O.dequantize_int4_g128(O.pack_int4(qa), sa), O.dequantize_int4_g128(O.pack_int4(qb), sb))
