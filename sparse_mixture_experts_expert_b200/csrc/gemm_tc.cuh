@@ -29,7 +29,7 @@
 
 namespace moe {
 
-enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2 };
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3 };
 
 struct GemmParams {
   const int32_t* group_start;  // [n_groups] or nullptr (one group of R rows)
@@ -42,6 +42,9 @@ struct GemmParams {
   __nv_bfloat16* out;
   long long ldo;
   unsigned long long wait_limit_ns;
+  int a_kwrap;         // > 0: the A operand repeats every a_kwrap columns of the reduction (split router)
+  float* out_f32;      // kModeF32: fp32 output [R, N]
+  const float* bias;   // kModeF32: optional per-column bias [N]
 };
 
 constexpr int kBM = 128;
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   using Cfg = GemmCfg<BN>;
-  constexpr bool kGLU = MODE != kModePlain;
+  constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
   constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
   constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box
   constexpr int S = Cfg::kStages;
@@ -160,7 +163,8 @@ __global__ void __launch_bounds__(256, 1)
           uint8_t* a_s = smem + (size_t)stage * Cfg::kStageBytes;
           uint8_t* b_s = a_s + Cfg::kABytes;
           mbar_arrive_expect_tx(&bar_full[stage], Cfg::kStageBytes);
-          tma_load_2d(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0);
+          const int ka = p.a_kwrap > 0 ? (kb * kBK) % p.a_kwrap : kb * kBK;
+          tma_load_2d(a_s, &tmA, &bar_full[stage], ka, (int)row0);
           if (kGLU) {
             tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
             tma_load_3d(b_s + BOXB * 128, &tmB, &bar_full[stage], kb * kBK, p.up_row0 + n0, g);
@@ -249,6 +253,21 @@ __global__ void __launch_bounds__(256, 1)
             const float a1 = MODE == kModeSwiGLU ? act_silu(g1) : act_gelu(g1);
             o[i] = pack_bf16x2(a0 * u0, a1 * u1);
           }
+        } else if (MODE == kModeF32) {
+          tmem_ld16(t_row + c, v);
+          tmem_ld_wait();
+          if (row_ok) {
+            float* frow = p.out_f32 + (row0 + r) * p.ldo + n0 + c;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (n0 + c + i < p.N) {
+                float f = __uint_as_float(v[i]);
+                if (p.bias != nullptr) f += p.bias[n0 + c + i];
+                frow[i] = f;
+              }
+            }
+          }
+          continue;
         } else {
           tmem_ld16(t_row + c, v);
           tmem_ld_wait();

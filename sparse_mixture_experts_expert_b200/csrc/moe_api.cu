@@ -84,7 +84,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+  size_t part, wsplit, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
 };
 
 static Workspace ws_layout(const moe_shape* s) {
@@ -96,6 +96,7 @@ static Workspace ws_layout(const moe_shape* s) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   L.part = take((size_t)ns * s->T * s->E * 4);
+  L.wsplit = take((size_t)3 * s->E * s->d * 2);
   L.cnt = take((size_t)nchunks * s->E * 4);
   L.psum = take((size_t)nchunks * s->E * 4);
   L.idx = take((size_t)s->T * s->k * 4);
@@ -154,7 +155,7 @@ template <int MODE, int BN>
 static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, long long ub_mtiles,
                          cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
-  constexpr int OUTN = MODE != kModePlain ? BN / 2 : BN;
+  constexpr int OUTN = (MODE == kModeSwiGLU || MODE == kModeGeGLU) ? BN / 2 : BN;
   MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)Cfg::kSmemBytes));
   const long long tiles = ub_mtiles * cdiv(p.N, OUTN);
@@ -165,16 +166,32 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
+// Column tile: the largest of 256/128/64 unless a narrower one fills the SMs in fewer
+// tile-widths of work (cost = waves x tile width, ties to the wider tile).
+static int pick_bn(bool glu, int N, long long mtiles) {
+  const int sms = num_sms();
+  int best = 0;
+  long long best_cost = 0;
+  for (int bn : {256, 128, 64}) {
+    const int outn = glu ? bn / 2 : bn;
+    if (bn > 64 && outn / 2 >= N) continue;  // mostly padding
+    const long long tiles = mtiles * cdiv(N, outn);
+    const long long cost = cdiv(tiles, sms) * bn;
+    if (best == 0 || cost * 100 < best_cost * 95) { best = bn; best_cost = cost; }
+  }
+  return best == 0 ? 64 : best;
+}
+
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
                         int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
-                        cudaStream_t st) {
+                        cudaStream_t st, int a_kwrap = 0, const float* bias = nullptr) {
   if (R == 0) return MOE_OK;
-  int BN;
-  if (mode == kModePlain) BN = N >= 256 ? 256 : (N >= 128 ? 128 : 64);
-  else BN = N >= 128 ? 256 : (N >= 64 ? 128 : 64);
-  const int box_rows = mode == kModePlain ? BN : BN / 2;
+  const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
+  const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
+  const int BN = pick_bn(glu, N, ub_m);
+  const int box_rows = glu ? BN / 2 : BN;
   CUtensorMap ta, tb;
-  cuuint64_t da[2] = {(cuuint64_t)K, (cuuint64_t)R};
+  cuuint64_t da[2] = {(cuuint64_t)(a_kwrap > 0 ? a_kwrap : K), (cuuint64_t)R};
   cuuint64_t db[3] = {(cuuint64_t)K, (cuuint64_t)b_rows, (cuuint64_t)n_groups};
   int rc = make_map(&ta, A, 2, da, kBM);
   if (rc) return rc;
@@ -191,12 +208,16 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ldo = N;
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.a_kwrap = a_kwrap;
+  p.out_f32 = reinterpret_cast<float*>(out);
+  p.bias = bias;
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
 #define MOE_GEMM_CASE(M_, BN_) \
   if (mode == M_ && BN == BN_) return launch_gemm_t<M_, BN_>(ta, tb, p, ub, st);
   MOE_GEMM_CASE(kModePlain, 256) MOE_GEMM_CASE(kModePlain, 128) MOE_GEMM_CASE(kModePlain, 64)
   MOE_GEMM_CASE(kModeSwiGLU, 256) MOE_GEMM_CASE(kModeSwiGLU, 128) MOE_GEMM_CASE(kModeSwiGLU, 64)
   MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
+  MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 128) MOE_GEMM_CASE(kModeF32, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -288,6 +309,12 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
   return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
 }
 
+// Large routers go to the tensor cores as an exact three-way bf16 split of W_r
+// (fp32 accumulation); small ones stay on the fp32 CUDA-core GEMM.
+static bool use_tc_router(const moe_shape* s) {
+  return s->E % 16 == 0 && s->d % 64 == 0 && (double)s->T * s->E * s->d >= (double)(1ll << 28);
+}
+
 static int route_impl(const moe_shape* s, const void* x, const float* w_router, const float* bias,
                       const float* logits_in, float* logits, int32_t* idx, float* w, int32_t* counts, float* aux_f,
                       float* aux_p, float* aux, uint8_t* ws, cudaStream_t st) {
@@ -299,7 +326,16 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   float* P = aux_p ? aux_p : reinterpret_cast<float*>(ws + L.fP) + s->E;
   int rc;
   int nsplit = 1;
-  if (logits_in == nullptr) {
+  if (logits_in == nullptr && use_tc_router(s)) {
+    __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
+    const long long n = (long long)s->E * s->d;
+    k_router_split<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(w_router, wsplit, s->E, s->d);
+    MOE_LAUNCH_CHECK();
+    rc = grouped_gemm(kModeF32, x, s->T, 3 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
+                      bias);
+    if (rc) return rc;
+    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, st);
+  } else if (logits_in == nullptr) {
     int kps = 0;
     nsplit = router_splits(s, &kps);
     dim3 grid((unsigned)cdiv(s->T, kLgBM), (unsigned)cdiv(s->E, kLgBN), (unsigned)nsplit);

@@ -104,6 +104,28 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 }
 
 // ---------------------------------------------------------------------------
+// Exact three-way bf16 split of the fp32 router weight: W = hi + mid + lo with
+// each part a bf16 value (24 significand bits = 3 x 8), written as one
+// [E, 3d] bf16 operand [hi | mid | lo].  x is bf16, so every product x * part
+// is exact in fp32 and x W^T = [x | x | x] [hi | mid | lo]^T.
+__global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
+                                                      int E, int d) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)E * d) return;
+  const long long e = i / d, k = i - e * d;
+  const float w = W[i];
+  const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+  __nv_bfloat16* row = Ws + e * 3 * d;
+  row[k] = hi;
+  row[d + k] = mid;
+  row[2 * d + k] = lo;
+}
+
+// ---------------------------------------------------------------------------
 // One warp per token.  Lane l holds the logits of experts l, l+32, ...
 //   logits = sum_split part[split] (+ bias); softmax; top-k; gates.
 // Per chunk of kChunk tokens (one CTA, 8 warps x 16 tokens):

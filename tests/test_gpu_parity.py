@@ -250,7 +250,9 @@ def _check_forward(wl, inp, s, r, sample=None):
     rel, mx = assert_out_close(got, out_ref)
     if wl.aux:
         np.testing.assert_allclose(np64(r["aux"])[0], ref_r["aux"], rtol=5e-5)
-    return int(excl.sum()), rel, mx
+    print(f"{wl.name}: T={wl.T} ambiguous={int(amb.sum())} flipped={flipped.size} excluded={int(excl.sum())} "
+          f"compared={toks.size} rel={rel:.2e} max={mx:.2e}")
+    return int(flipped.size), rel, mx
 
 
 @pytest.mark.parametrize("name,over", [("tiny", {}), ("small", {}), ("tiny", {"capacity_factor": 0.5}),
@@ -262,8 +264,8 @@ def _check_forward(wl, inp, s, r, sample=None):
 def test_forward_matches_oracle(lib, name, over):
     wl = synth.get_workload(name).replace(**over)
     inp, s, r = _forward_case(lib, wl)
-    n_ex, rel, mx = _check_forward(wl, inp, s, r)
-    assert n_ex <= max(2, wl.T // 500)
+    n_flip, rel, mx = _check_forward(wl, inp, s, r)
+    assert n_flip <= max(2, wl.T // 5000)
     if over.get("capacity_factor") == 0.5:
         assert npi(r["drop_mask"]).sum() > 0
 
@@ -276,8 +278,8 @@ def test_forward_full_size_sampled(lib, name):
     inp = {k_: (v.cpu() if v is not None else None) for k_, v in inp.items()}
     rng = np.random.default_rng(0)
     sample = np.unique(np.concatenate([rng.choice(wl.T, 96, replace=False), [0, wl.T - 1]]))
-    n_ex, rel, mx = _check_forward(wl, inp, s, r, sample=sample)
-    assert n_ex <= wl.T // 500
+    n_flip, rel, mx = _check_forward(wl, inp, s, r, sample=sample)
+    assert n_flip <= max(2, wl.T // 5000)
 
 
 # ---------------------------------------------------------------- INT4 quantiser
