@@ -174,33 +174,60 @@ def run_forward(moe, s, inp, ws, out, aux):
 
 
 def stage_times(moe, s, inp, ws, wl, flush, reps=10):
-    """Per-stage device time (us) through the component entry points, L2 flushed before each rep."""
+    """Per-stage device time (us): each stage of the pipeline is captured through its component entry point
+    (moe_route, moe_permute, moe_expert_ffn routed / shared, moe_combine) into its own CUDA graph; the
+    graphs are replayed back to back with events between them, L2 flushed before each repetition."""
     import torch
+    names = ["route", "permute", "expert_ffn", "shared_ffn", "combine"]
+    ws2 = torch.empty_like(ws)   # the permute reads the chunk table the route left in its own workspace
+    state = {}
+
+    def st_route():
+        state["r"] = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"], ws=ws)
+
+    def st_permute():
+        state["p"] = moe.moe_permute(s, inp["x"], state["r"]["topk_idx"], ws=ws2)
+
+    def st_ffn():
+        p = state["p"]
+        state["y"] = moe.moe_expert_ffn(s, p["x_perm"], inp["w13"], inp["w2"], group_start=p["offsets"],
+                                        group_rows=p["kept"], s13=inp.get("s13"), s2=inp.get("s2"))[1]
+
+    def st_shared():
+        state["ysh"] = None
+        if wl.H_s:
+            state["ysh"] = moe.moe_expert_ffn(s, inp["x"], inp["w13_sh"], inp["w2_sh"], hidden=wl.H_s,
+                                              s13=inp.get("s13_sh"), s2=inp.get("s2_sh"))[1]
+
+    def st_combine():
+        state["out"] = moe.moe_combine(s, state["y"], state["p"]["slot_pos"], state["r"]["topk_w"], state["ysh"])
+
+    fns = [st_route, st_permute, st_ffn, st_shared, st_combine]
+    for f in fns:                       # eager warm-up (allocations, attributes)
+        f()
+    torch.cuda.synchronize()
+    graphs = []
+    for f in fns:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        graphs.append(g)
+    torch.cuda.synchronize()
     st = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-    acc = {"route": [], "permute": [], "expert_ffn": [], "shared_ffn": [], "combine": []}
+    acc = {k: [] for k in names}
     for _ in range(reps):
         flush()
         ev[0].record(st)
-        r = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"], ws=ws)
-        ev[1].record(st)
-        p = moe.moe_permute(s, inp["x"], r["topk_idx"], ws=ws)
-        ev[2].record(st)
-        h, y = moe.moe_expert_ffn(s, p["x_perm"], inp["w13"], inp["w2"], group_start=p["offsets"],
-                                  group_rows=p["kept"], s13=inp.get("s13"), s2=inp.get("s2"))
-        ev[3].record(st)
-        ysh = None
-        if wl.H_s:
-            _, ysh = moe.moe_expert_ffn(s, inp["x"], inp["w13_sh"], inp["w2_sh"], hidden=wl.H_s,
-                                        s13=inp.get("s13_sh"), s2=inp.get("s2_sh"))
-        ev[4].record(st)
-        moe.moe_combine(s, y, p["slot_pos"], r["topk_w"], ysh)
-        ev[5].record(st)
+        for i, g in enumerate(graphs):
+            g.replay()
+            ev[i + 1].record(st)
         torch.cuda.synchronize()
-        for i, k in enumerate(acc):
+        for i, k in enumerate(names):
             acc[k].append(ev[i].elapsed_time(ev[i + 1]) * 1e3)
-        kept = int(p["kept"].sum())
-        touched = int((p["kept"] > 0).sum())
+    kept = int(state["p"]["kept"].sum())
+    touched = int((state["p"]["kept"] > 0).sum())
+    del graphs
     return {k: statistics.median(v) for k, v in acc.items()}, kept, touched
 
 
@@ -339,8 +366,19 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status} at {site:#x} during warm-up")
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # One forward captured into a CUDA graph (the launch-bound small workloads would otherwise time the
+    # host); the graph replays exactly the kernels moe_forward enqueues.
     launches0 = moe.moe_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_forward(moe, s, inp, ws, out, wl.aux)
+    per_step_launches = moe.moe_launch_count() - launches0
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -348,13 +386,16 @@ def main():
         for a, b in evs:
             flush()
             a.record(st)
-            run_forward(moe, s, inp, ws, out, wl.aux)
+            graph.replay()
             b.record(st)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    launches = moe.moe_launch_count() - launches0
+    launches = per_step_launches * args.steps
     step_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    status, site = moe.moe_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
     step_ms = max_over_ranks(step_ms, world)
     value = world * wl.T / (step_ms * 1e-3)
 
@@ -413,7 +454,9 @@ def main():
                 "roofline": roofline, "stages_us": stages, "cpu_baseline": cpu,
                 "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 2},
-                "gpu_launches": launches, "clocks": clk.summary()}
+                "gpu_launches": launches, "launches_per_step": per_step_launches,
+                "timing": "CUDA graph of one moe_forward replayed per step (value); e2e calls the API eagerly",
+                "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -49,19 +49,24 @@ struct GemmParams {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle atom of bf16
-constexpr int kMaxGroupsSmem = 1024;
+constexpr int kMaxGroupsSmem = 512;
+constexpr int kEpiW = 64;                                   // columns staged per epilogue round
+constexpr int kEpiRow = kEpiW + 8;                          // padded staging row (bf16), conflict-free
+constexpr int kEpiBytes = 4 * 32 * kEpiRow * 2;             // four epilogue warps x 32 rows
 
 template <int BN>
 struct GemmCfg {
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kBudget = 219 * 1024 - 1024 - kEpiBytes;
+  static constexpr int kStages = kBudget / kStageBytes > 8 ? 8 : kBudget / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
-  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes;
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kEpiBytes;
 };
 
-__device__ __forceinline__ float act_silu(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU with the fast exponential and division: h is rounded to bf16 right after.
+__device__ __forceinline__ float act_silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + erff(g * 0.7071067811865476f)); }
 
 template <int MODE, int BN>
@@ -81,6 +86,8 @@ __global__ void __launch_bounds__(256, 1)
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_prefix[kMaxGroupsSmem + 1];
+  __shared__ int s_gstart[kMaxGroupsSmem];
+  __shared__ int s_grows[kMaxGroupsSmem];
 
   const int warp = warp_id(), lane = lane_id();
   const int n_tiles = (p.N + OUTN - 1) / OUTN;
@@ -107,6 +114,8 @@ __global__ void __launch_bounds__(256, 1)
     for (int g = g0; g < g1; ++g) {
       s_prefix[g] = run;
       const long long rows = single ? p.R : (long long)p.group_rows[g];
+      s_grows[g] = (int)rows;
+      s_gstart[g] = single ? 0 : p.group_start[g];
       run += (int)((rows + kBM - 1) / kBM);
     }
     if (lane == 31) s_prefix[G] = incl;
@@ -141,8 +150,8 @@ __global__ void __launch_bounds__(256, 1)
     }
     g = lo;
     const long long m_local = (long long)(mt - s_prefix[g]) * kBM;
-    const long long start = single ? 0 : (long long)p.group_start[g];
-    const long long rows = single ? p.R : (long long)p.group_rows[g];
+    const long long start = s_gstart[g];
+    const long long rows = s_grows[g];
     row0 = start + m_local;
     rows_valid = (int)min((long long)kBM, rows - m_local);
     n0 = nt * OUTN;
@@ -223,8 +232,17 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue
+    // TMEM -> registers -> activation / bf16 -> per-warp staging rows in shared
+    // memory -> coalesced row-segment stores (128 contiguous bytes per row per
+    // 8 lanes).  The accumulator is handed back to the MMA warp as soon as its
+    // last TMEM load has completed.
     const int q = warp & 3;  // TMEM lane quarter
     const int r = q * 32 + lane;
+    constexpr int OUTW = OUTN < kEpiW ? OUTN : kEpiW;
+    constexpr int ROUNDS = OUTN / OUTW;
+    constexpr int LPR = OUTW / 8;   // lanes per staged row in the copy-out
+    constexpr int RPI = 32 / LPR;   // rows per copy-out iteration
+    __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)S * Cfg::kStageBytes) + q * 32 * kEpiRow;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
@@ -234,26 +252,11 @@ __global__ void __launch_bounds__(256, 1)
       if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0106)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const bool row_ok = r < rows_valid;
-      __nv_bfloat16* orow = p.out + (row0 + r) * p.ldo;
+      if (MODE == kModeF32) {
+        const bool row_ok = r < rows_valid;
 #pragma unroll 1
-      for (int c = 0; c < OUTN; c += 16) {
-        uint32_t v[16];
-        uint32_t o[8];
-        if (kGLU) {
-          uint32_t u[16];
-          tmem_ld16(t_row + c, v);
-          tmem_ld16(t_row + OUTN + c, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
-            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-            const float a0 = MODE == kModeSwiGLU ? act_silu(g0) : act_gelu(g0);
-            const float a1 = MODE == kModeSwiGLU ? act_silu(g1) : act_gelu(g1);
-            o[i] = pack_bf16x2(a0 * u0, a1 * u1);
-          }
-        } else if (MODE == kModeF32) {
+        for (int c = 0; c < OUTN; c += 16) {
+          uint32_t v[16];
           tmem_ld16(t_row + c, v);
           tmem_ld_wait();
           if (row_ok) {
@@ -267,21 +270,59 @@ __global__ void __launch_bounds__(256, 1)
               }
             }
           }
-          continue;
-        } else {
-          tmem_ld16(t_row + c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
-        if (row_ok && n0 + c < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + n0 + c);
-          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        tc_fence_before();
+        mbar_arrive(&bar_tempty[acc]);
+      } else {
+#pragma unroll 1
+        for (int rd = 0; rd < ROUNDS; ++rd) {
+#pragma unroll
+          for (int c = 0; c < OUTW; c += 16) {
+            const int cc = rd * OUTW + c;
+            uint32_t v[16];
+            uint32_t o[8];
+            if (kGLU) {
+              uint32_t u[16];
+              tmem_ld16(t_row + cc, v);
+              tmem_ld16(t_row + OUTN + cc, u);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
+                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                const float a0 = MODE == kModeSwiGLU ? act_silu(g0) : act_gelu(g0);
+                const float a1 = MODE == kModeSwiGLU ? act_silu(g1) : act_gelu(g1);
+                o[i] = pack_bf16x2(a0 * u0, a1 * u1);
+              }
+            } else {
+              tmem_ld16(t_row + cc, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            uint4* sp = reinterpret_cast<uint4*>(stg + lane * kEpiRow + c);
+            sp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            sp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          if (rd == ROUNDS - 1) {
+            tc_fence_before();
+            mbar_arrive(&bar_tempty[acc]);
+          }
+          __syncwarp();
+          const int cb = (lane % LPR) * 8;
+          const int col = n0 + rd * OUTW + cb;
+#pragma unroll
+          for (int it = 0; it < 32 / RPI; ++it) {
+            const int rr = it * RPI + lane / LPR;
+            if (q * 32 + rr < rows_valid && col < p.N) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * kEpiRow + cb);
+              *reinterpret_cast<uint4*>(p.out + (row0 + q * 32 + rr) * p.ldo + col) = val;
+            }
+          }
+          __syncwarp();
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bar_tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }

@@ -22,8 +22,9 @@
 //   * the fp32 partial of each 128-group is scaled by its bf16 scale and
 //     added to the fp32 total: w = q * s is applied exactly;
 //   * gated mode writes h = act(x W1^T) * (x W3^T) in bf16, plain mode y.
-// Groups with more than 8 rows take several passes over the same weights
-// (the repeat reads hit L2).
+// Groups with more than 8 rows are split into 8-row chunks, one task each;
+// the chunks of one 16-row block run on neighbouring warps, so the repeat
+// weight reads hit L2.
 #pragma once
 
 #include "common.cuh"
@@ -120,12 +121,17 @@ __global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
   const int lane = lane_id(), warp = warp_id();
   const bool single = p.group_rows == nullptr;
   const int G = single ? 1 : p.n_groups;
-  const int tasks_per_group = p.N / 16;
+  const int oblocks = p.N / 16;
+  // tasks of group g: oblocks x ceil(rows / 8) (16 output rows x 8 activation rows each)
+  auto group_tasks = [&](int g) -> int {
+    const long long rows = single ? p.R : (long long)p.group_rows[g];
+    return (int)(oblocks * ((rows + 7) / 8));
+  };
   if (warp == 0) {
     const int per = (G + 31) / 32;
     const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
     int local = 0;
-    for (int g = g0; g < g1; ++g) local += ((single ? p.R : (long long)p.group_rows[g]) > 0) ? tasks_per_group : 0;
+    for (int g = g0; g < g1; ++g) local += group_tasks(g);
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -135,7 +141,7 @@ __global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
     int run = incl - local;
     for (int g = g0; g < g1; ++g) {
       s_prefix[g] = run;
-      run += ((single ? p.R : (long long)p.group_rows[g]) > 0) ? tasks_per_group : 0;
+      run += group_tasks(g);
     }
     if (lane == 31) s_prefix[G] = incl;
   }
@@ -152,9 +158,12 @@ __global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
       if (s_prefix[mid] <= task) lo = mid; else hi = mid - 1;
     }
     const int g = lo;
-    const int o0 = (task - s_prefix[g]) * 16;
     const long long row0 = single ? 0 : p.group_start[g];
     const int n_rows = (int)(single ? p.R : (long long)p.group_rows[g]);
+    const int nchunks = (n_rows + 7) / 8;
+    const int tg = task - s_prefix[g];
+    const int o0 = (tg / nchunks) * 16;  // chunks of one row block are adjacent tasks: the repeat reads hit L2
+    const int n0 = (tg % nchunks) * 8;
     const long long wbase = (long long)g * p.b_rows;
     // this thread's weight rows: gate (or plain) rows o0+gq, o0+gq+8; up rows up_row0 + same
     const uint8_t* wg0 = p.wq + (wbase + o0 + gq) * wrow_bytes + c * 16;
@@ -166,7 +175,7 @@ __global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
     const __nv_bfloat16* su0 = p.ws + (wbase + p.up_row0 + o0 + gq) * ngroups_k;
     const __nv_bfloat16* su1 = su0 + 8 * ngroups_k;
 
-    for (int n0 = 0; n0 < n_rows; n0 += 8) {
+    {
       const int tok = n0 + gq;            // B column this thread feeds
       const bool tok_ok = tok < n_rows;
       const __nv_bfloat16* xrow = p.act + (row0 + (tok_ok ? tok : 0)) * (long long)p.K + c * 32;

@@ -63,10 +63,23 @@ static inline long long grouped_rows(const moe_shape* s) {
   return s->capacity > 0 ? (long long)s->E * s->capacity : s->T * s->k;
 }
 
+static int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return dev;
+}
+
+// SM count of the current device, queried once per device.
 static int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  static std::atomic<int> cache[64];
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // Router split-K so that small-T, wide-d routers still fill the GPU.
@@ -84,7 +97,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, wsplit, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+  size_t part, wsplit, wmax, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
 };
 
 static Workspace ws_layout(const moe_shape* s) {
@@ -97,6 +110,7 @@ static Workspace ws_layout(const moe_shape* s) {
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   L.part = take((size_t)ns * s->T * s->E * 4);
   L.wsplit = take((size_t)3 * s->E * s->d * 2);
+  L.wmax = take(16);
   L.cnt = take((size_t)nchunks * s->E * 4);
   L.psum = take((size_t)nchunks * s->E * 4);
   L.idx = take((size_t)s->T * s->k * 4);
@@ -156,8 +170,15 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
                          cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
   constexpr int OUTN = (MODE == kModeSwiGLU || MODE == kModeGeGLU) ? BN / 2 : BN;
-  MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)Cfg::kSmemBytes));
+  // the shared-memory opt-in is set once per device for each instantiation
+  static std::atomic<unsigned long long> done_mask{0};
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(done_mask.load(std::memory_order_relaxed) & bit)) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)Cfg::kSmemBytes));
+    done_mask.fetch_or(bit);
+  }
   const long long tiles = ub_mtiles * cdiv(p.N, OUTN);
   const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
   k_grouped_gemm<MODE, BN><<<grid, 256, Cfg::kSmemBytes, st>>>(ta, tb, p);
@@ -225,13 +246,14 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
 // ------------------------------------------------------------------ launch helpers
 
 static int launch_topk(const moe_shape* s, const float* part, int nsplit, const float* bias, float* logits,
-                       int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st) {
+                       int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st,
+                       RefineArgs refine = RefineArgs{nullptr, nullptr, nullptr, nullptr, 0, 0.f}) {
   const int nchunks = (int)cdiv(s->T, kChunk);
   const int epl = (int)cdiv(s->E, 32);
 #define MOE_TOPK_CASE(N_)                                                                                         \
   if (epl <= N_) {                                                                                                \
     k_router_topk<N_><<<nchunks, 256, 0, st>>>(part, nsplit, bias, logits, idx, w, cnt, psum, (int)s->T, s->E,   \
-                                               s->k, s->renorm);                                                  \
+                                               s->k, s->renorm, refine);                                          \
     MOE_LAUNCH_CHECK();                                                                                           \
     return MOE_OK;                                                                                                \
   }
@@ -284,7 +306,7 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
   p.up_row0 = up_row0;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ldo = N;
-  const long long ub_tasks = (long long)(grows ? std::min<long long>(n_groups, R) : 1) * (N / 16);
+  const long long ub_tasks = (long long)(N / 16) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8));
   const int grid = (int)std::max<long long>(1, std::min<long long>(2ll * num_sms(), cdiv(ub_tasks, 8)));
   if (!glu) k_int4_gemm<false, kModePlain><<<grid, 256, 0, st>>>(p);
   else if (act == MOE_ACT_SWIGLU) k_int4_gemm<true, kModeSwiGLU><<<grid, 256, 0, st>>>(p);
@@ -331,10 +353,16 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     const long long n = (long long)s->E * s->d;
     k_router_split<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(w_router, wsplit, s->E, s->d);
     MOE_LAUNCH_CHECK();
+    float* wmax = reinterpret_cast<float*>(ws + L.wmax);
+    k_router_wmax<<<1, 256, 0, st>>>(w_router, wmax, s->E, s->d);
+    MOE_LAUNCH_CHECK();
     rc = grouped_gemm(kModeF32, x, s->T, 3 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
                       bias);
     if (rc) return rc;
-    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, st);
+    // screening bound: fp32 accumulation of 3d products (any rounding direction) plus the bias add
+    RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wmax, s->d,
+                   (float)((3.0 * s->d + 2.0) * std::ldexp(1.0, -23) * (1.0 + std::ldexp(1.0, -7)))};
+    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, st, ref);
   } else if (logits_in == nullptr) {
     int kps = 0;
     nsplit = router_splits(s, &kps);

@@ -125,9 +125,66 @@ __global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ 
   row[2 * d + k] = lo;
 }
 
+// wmax[0] = max_e ||W_r[e]||_2 (one CTA, fixed order).
+__global__ void __launch_bounds__(256) k_router_wmax(const float* __restrict__ W, float* __restrict__ wmax, int E,
+                                                     int d) {
+  __shared__ float s_m[8];
+  float m = 0.f;
+  for (int e = warp_id(); e < E; e += 8) {
+    float ss = 0.f;
+    for (int i = lane_id(); i < d; i += 32) ss = fmaf(W[(size_t)e * d + i], W[(size_t)e * d + i], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    m = fmaxf(m, sqrtf(ss));
+  }
+  if (lane_id() == 0) s_m[warp_id()] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = s_m[0];
+    for (int w = 1; w < 8; ++w) r = fmaxf(r, s_m[w]);
+    *wmax = r;
+  }
+}
+
 // ---------------------------------------------------------------------------
+// Warp argmax over the lanes' (value, index) pairs: larger value first, lower
+// index first among equal values (-0.0 == +0.0, so the index decides).
+__device__ __forceinline__ void warp_argmax(float& bv, int& bi) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+}
+
+// Exact fp32 logit of one expert for one token, computed by the whole warp:
+// lane l accumulates inputs l, l+32, ... with fmaf, then a fixed xor tree.
+__device__ __forceinline__ float warp_dot(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ wr, int d) {
+  float acc = 0.f;
+  for (int i = lane_id(); i < d; i += 32) acc = fmaf(__bfloat162float(xr[i]), wr[i], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+struct RefineArgs {
+  const __nv_bfloat16* x;  // [T, d]; nullptr = logits are final
+  const float* W;          // [E, d] fp32 router weight
+  const float* bias;       // [E] or nullptr
+  const float* wmax;       // max_e ||W_r[e]||_2 (one float)
+  int d;
+  float gamma;             // bound factor of the screening logits: |err| <= gamma * ||x_t|| * ||w_e||
+};
+
 // One warp per token.  Lane l holds the logits of experts l, l+32, ...
 //   logits = sum_split part[split] (+ bias); softmax; top-k; gates.
+// With refine.x set, `part` holds screening logits from the tensor cores whose
+// error is at most gamma * ||x_t|| * ||w_e||.  Every expert that could still be
+// in the top k under that bound (screening logit >= k-th largest - 2 bound) is
+// recomputed as a plain fp32 dot product, so the top-k decision is made on
+// fp32 FMA logits exactly as in the CUDA-core router; the others are
+// certified out of the top k.
 // Per chunk of kChunk tokens (one CTA, 8 warps x 16 tokens):
 //   cnt[chunk][e]  tokens of the chunk that chose e
 //   psum[chunk][e] sum over the chunk's tokens of p[t,e] (fixed order)
@@ -136,7 +193,7 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
                                                      const float* __restrict__ bias, float* __restrict__ logits_out,
                                                      int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                                      int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
-                                                     int E, int k, int renorm) {
+                                                     int E, int k, int renorm, const RefineArgs refine) {
   __shared__ float s_p[8][EPL * 32];
   __shared__ int s_c[8][EPL * 32];
   const int lane = lane_id(), warp = warp_id();
@@ -151,22 +208,76 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
     const int e = lane + 32 * i;
     b[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   }
+  const float wmax = refine.x != nullptr ? *refine.wmax : 0.f;
+  const int t_first = chunk * kChunk + warp * (kChunk / 8);
+  const int t_end = min(T, t_first + kChunk / 8);
 
-  for (int tt = 0; tt < kChunk / 8; ++tt) {
-    const int t = chunk * kChunk + warp * (kChunk / 8) + tt;
-    if (t >= T) break;
-    float z[EPL];
+  auto load_z = [&](int t, float (&z)[EPL]) {
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       float v = -INFINITY;
-      if (e < E) {
+      if (e < E && t < t_end) {
         v = part[(size_t)t * E + e];
         for (int s = 1; s < nsplit; ++s) v += part[(size_t)s * T * E + (size_t)t * E + e];
         if (bias != nullptr) v += b[i];
-        if (logits_out != nullptr) logits_out[(size_t)t * E + e] = v;
       }
       z[i] = v;
+    }
+  };
+
+  float znext[EPL];
+  load_z(t_first, znext);
+  for (int t = t_first; t < t_end; ++t) {
+    float z[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = znext[i];
+    load_z(t + 1, znext);  // prefetch the next token's logits
+
+    if (refine.x != nullptr) {
+      // k-th largest screening logit
+      unsigned tk = 0u;
+      float kth = -INFINITY;
+      for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          if (e < E && !((tk >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
+        }
+        warp_argmax(bv, bi);
+        if ((bi & 31) == lane) tk |= 1u << (bi >> 5);
+        kth = bv;
+      }
+      const __nv_bfloat16* xr = refine.x + (size_t)t * refine.d;
+      float ss = 0.f;
+      for (int i = lane; i < refine.d; i += 32) {
+        const float v = __bfloat162float(xr[i]);
+        ss = fmaf(v, v, ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float bound = refine.gamma * sqrtf(ss) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
+      const float thr = kth - 2.f * bound;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e0 = 32 * i;
+        unsigned cand = __ballot_sync(0xffffffffu, lane + e0 < E && z[i] >= thr);
+        while (cand) {
+          const int l = __ffs(cand) - 1;
+          cand &= cand - 1;
+          const int e = e0 + l;
+          float v = warp_dot(xr, refine.W + (size_t)e * refine.d, refine.d);
+          if (refine.bias != nullptr) v += refine.bias[e];
+          if (lane == l) z[i] = v;
+        }
+      }
+    }
+    if (logits_out != nullptr) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i < E) logits_out[(size_t)t * E + lane + 32 * i] = z[i];
     }
     // softmax
     float m = z[0];
@@ -188,9 +299,8 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
 
     // top-k: k rounds of warp argmax on (logit desc, index asc)
     unsigned taken = 0u;
-    float wsel[16];
-    int isel[16];
-    float wsum = 0.f;
+    float wv = 0.f, wsum = 0.f;
+    int iv = 0;
     for (int j = 0; j < k; ++j) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
@@ -199,12 +309,7 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
         const int e = lane + 32 * i;
         if (e < E && !((taken >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
+      warp_argmax(bv, bi);
       if ((bi & 31) == lane) {
         const int i = bi >> 5;
         taken |= 1u << i;
@@ -213,15 +318,10 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
           if (q == i) cacc[q] += 1;
       }
       const float pj = expf(bv - m) * inv;
-      wsel[j] = pj;
-      isel[j] = bi;
+      if (lane == j) { wv = pj; iv = bi; }
       wsum += pj;
     }
     if (lane < k) {
-      float wv = 0.f;
-      int iv = 0;
-      for (int j = 0; j < k; ++j)
-        if (j == lane) { wv = wsel[j]; iv = isel[j]; }
       topk_idx[(size_t)t * k + lane] = iv;
       topk_w[(size_t)t * k + lane] = renorm ? wv / wsum : wv;
     }

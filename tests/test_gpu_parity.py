@@ -67,12 +67,15 @@ def _route_case(moe, wl, T, seed):
                                     ("decode_int4", 64)])
 def test_route_matches_oracle(lib, name, T):
     wl, inp, r, ref, x64, W64, b64 = _route_case(lib, synth.get_workload(name), T, seed=1)
-    # logits: fp32 accumulation of d products; rigorous bound gamma_{d+2} * sum|x_i w_i| (+ |bias|)
+    # Logits.  Every logit is within the bound of an fp32 accumulation of 3d products in any rounding
+    # direction (the tensor-core screening pass); the logits of the chosen experts are plain fp32 FMA dot
+    # products, within the round-to-nearest bound gamma_{d+2} * sum|x_i w_i| (+ |bias|).
     zg = np64(r["logits"])
-    bound = (wl.d + 2) * 2.0 ** -24 * (np.abs(x64) @ np.abs(W64).T + (np.abs(b64) if b64 is not None else 0))
-    assert (np.abs(zg - ref["z"]) <= bound).all()
-    typical = np.abs(zg - ref["z"]).max()
-    assert typical < 2e-5, typical
+    mag = np.abs(x64) @ np.abs(W64).T + (np.abs(b64) if b64 is not None else 0)
+    assert (np.abs(zg - ref["z"]) <= (3 * wl.d + 2) * 2.0 ** -23 * 1.01 * mag + 1e-7).all()
+    sel = np.take_along_axis(np.abs(zg - ref["z"]) - (wl.d + 2) * 2.0 ** -24 * mag, npi(r["topk_idx"]).astype(np.int64),
+                             axis=1)
+    assert (sel <= 0).all()
     # top-k: bit-exact where the oracle's k-th/(k+1)-th margin is >= 1e-5; inside the band any choice
     # within the band is valid
     margin = O.topk_margin(ref["z"], wl.k)
