@@ -276,10 +276,13 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   const int nchunks = (int)cdiv(s->T, kChunk);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(x_perm);
+  const unsigned mv_blocks = (unsigned)cdiv(s->T * (long long)(s->d / 8), 256);
 #define MOE_SCATTER_CASE(N_)                                                                                  \
   if (s->k <= N_) {                                                                                           \
     k_scatter<N_><<<nchunks, 128, 0, st>>>(xb, idx, cbase, counts, (int)s->T, s->d, s->E, s->k, s->capacity, \
                                            slot, drop, row_src, xp, kept, offs);                              \
+    MOE_LAUNCH_CHECK();                                                                                       \
+    k_move_rows<N_><<<mv_blocks, 256, 0, st>>>(xb, slot, (int)s->T, s->d, s->k, xp);                         \
     MOE_LAUNCH_CHECK();                                                                                       \
     return MOE_OK;                                                                                            \
   }
@@ -331,6 +334,38 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
   return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
 }
 
+// Fused CUDA-core router when W_r^T fits in shared memory: returns its experts-per-lane template, else 0.
+static int fused_router_epl(const moe_shape* s) {
+  const int epl = s->E <= 32 ? 1 : s->E <= 64 ? 2 : s->E <= 128 ? 4 : s->E <= 256 ? 8 : 16;
+  const size_t bytes = (size_t)s->d * (epl * 32 + 1) * 4;
+  return bytes <= 160 * 1024 ? epl : 0;
+}
+
+static int launch_fused_router(const moe_shape* s, int epl, const void* x, const float* w_router, const float* bias,
+                               float* logits, int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st) {
+  const int nchunks = (int)cdiv(s->T, kChunk);
+  const size_t smem = (size_t)s->d * (epl * 32 + 1) * 4;
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+#define MOE_FUSED_CASE(N_)                                                                                        \
+  if (epl == N_) {                                                                                                \
+    static std::atomic<unsigned long long> done{0};                                                               \
+    if (!(done.load() & bit)) {                                                                                   \
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_fused<N_>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                        160 * 1024));                                                             \
+      done.fetch_or(bit);                                                                                         \
+    }                                                                                                             \
+    k_router_fused<N_><<<nchunks, 256, smem, st>>>(xb, w_router, bias, logits, idx, w, cnt, psum, (int)s->T, s->d, \
+                                                   s->E, s->k, s->renorm);                                        \
+    MOE_LAUNCH_CHECK();                                                                                           \
+    return MOE_OK;                                                                                                \
+  }
+  MOE_FUSED_CASE(1) MOE_FUSED_CASE(2) MOE_FUSED_CASE(4) MOE_FUSED_CASE(8) MOE_FUSED_CASE(16)
+#undef MOE_FUSED_CASE
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
 // Large routers go to the tensor cores as an exact three-way bf16 split of W_r
 // (fp32 accumulation); small ones stay on the fp32 CUDA-core GEMM.
 static bool use_tc_router(const moe_shape* s) {
@@ -348,7 +383,10 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   float* P = aux_p ? aux_p : reinterpret_cast<float*>(ws + L.fP) + s->E;
   int rc;
   int nsplit = 1;
-  if (logits_in == nullptr && use_tc_router(s)) {
+  const int epl_fused = fused_router_epl(s);
+  if (logits_in == nullptr && epl_fused > 0) {
+    rc = launch_fused_router(s, epl_fused, x, w_router, bias, logits, idx, w, cnt, psum, st);
+  } else if (logits_in == nullptr && use_tc_router(s)) {
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
     const long long n = (long long)s->E * s->d;
     k_router_split<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(w_router, wsplit, s->E, s->d);
@@ -363,6 +401,11 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wmax, s->d,
                    (float)((3.0 * s->d + 2.0) * std::ldexp(1.0, -23) * (1.0 + std::ldexp(1.0, -7)))};
     rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, st, ref);
+  } else if (logits_in == nullptr && s->T <= 256) {
+    k_router_skinny<32><<<(unsigned)cdiv(s->E, 2), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router,
+                                                                 part, (int)s->T, s->d, s->E);
+    MOE_LAUNCH_CHECK();
+    rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum, st);
   } else if (logits_in == nullptr) {
     int kps = 0;
     nsplit = router_splits(s, &kps);
@@ -507,12 +550,19 @@ int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos,
   if (rc) return rc;
   if (!y_perm || !slot_pos || !topk_w || !out) return MOE_INVALID_ARGUMENT;
   if (!aligned16(y_perm) || !aligned16(out) || (y_shared && !aligned16(y_shared))) return MOE_INVALID_ARGUMENT;
-  k_combine<<<(unsigned)cdiv(s->T, 8), 256, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(y_perm), slot_pos, topk_w,
-      reinterpret_cast<const __nv_bfloat16*>(y_shared), reinterpret_cast<__nv_bfloat16*>(out), (int)s->T, s->d,
-      s->k);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  const __nv_bfloat16* yp = reinterpret_cast<const __nv_bfloat16*>(y_perm);
+  const __nv_bfloat16* ysh = reinterpret_cast<const __nv_bfloat16*>(y_shared);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  const unsigned blocks = (unsigned)cdiv(s->T, 8);
+#define MOE_COMBINE_CASE(N_)                                                                                   \
+  if (s->k <= N_) {                                                                                            \
+    k_combine<N_><<<blocks, 256, 0, stream>>>(yp, slot_pos, topk_w, ysh, o, (int)s->T, s->d, s->k);           \
+    MOE_LAUNCH_CHECK();                                                                                        \
+    return MOE_OK;                                                                                             \
+  }
+  MOE_COMBINE_CASE(2) MOE_COMBINE_CASE(4) MOE_COMBINE_CASE(8) MOE_COMBINE_CASE(16)
+#undef MOE_COMBINE_CASE
+  return MOE_UNSUPPORTED_SHAPE;
 }
 
 int moe_forward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,

@@ -150,22 +150,26 @@ __global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict
     }
   }
 
-  // Row moves: the warp copies each of its tokens' rows to the token's kept rows, 16 bytes per lane.
+}
+
+// Row moves: one thread per (token, 16-byte column slice); it copies the slice
+// of x[t] to every kept row of the token.  Fully parallel and coalesced.
+template <int KMAX>
+__global__ void __launch_bounds__(256) k_move_rows(const __nv_bfloat16* __restrict__ x,
+                                                   const int32_t* __restrict__ slot_pos, int T, int d, int k,
+                                                   __nv_bfloat16* __restrict__ x_perm) {
   const int nvec = d >> 3;
-  for (int tok = 0; tok < 32; ++tok) {
-    const int tt = chunk * kChunk + warp * 32 + tok;
-    if (tt >= T) break;
-    int p[KMAX];
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)T * nvec) return;
+  const long long t = i / nvec;
+  const int v = (int)(i - t * nvec);
+  int p[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) p[j] = __shfl_sync(0xffffffffu, pos[j], tok);
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tt * d);
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 val = src[v];
+  for (int j = 0; j < KMAX; ++j) p[j] = j < k ? slot_pos[t * k + j] : -1;
+  const uint4 val = reinterpret_cast<const uint4*>(x + t * d)[v];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k && p[j] >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)p[j] * d)[v] = val;
-    }
-  }
+  for (int j = 0; j < KMAX; ++j)
+    if (p[j] >= 0) reinterpret_cast<uint4*>(x_perm + (size_t)p[j] * d)[v] = val;
 }
 
 // Write the group table of moe_permute-style outputs without moving rows:
@@ -185,7 +189,9 @@ __global__ void __launch_bounds__(128) k_group_table(const int32_t* __restrict__
 
 // ---------------------------------------------------------------------------
 // Combine: one warp per token, fp32 sum over slots j = 0..k-1 in order, then
-// the shared expert, one bf16 rounding.  Columns processed 1024 at a time.
+// the shared expert, one bf16 rounding.  Each lane owns 16-byte column slices;
+// the k row loads of a slice are issued together.
+template <int KMAX>
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ y_perm,
                                                  const int32_t* __restrict__ slot_pos, const float* __restrict__ w,
                                                  const __nv_bfloat16* __restrict__ y_shared,
@@ -194,52 +200,40 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
   const int lane = lane_id();
   if (t >= T) return;
   const int nvec = d >> 3;
-  for (int v0 = 0; v0 < nvec; v0 += 128) {
-    float acc[4][8];
+  int p[KMAX];
+  float g[KMAX];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int j = 0; j < KMAX; ++j) {
+    p[j] = j < k ? slot_pos[(size_t)t * k + j] : -1;
+    g[j] = j < k ? w[(size_t)t * k + j] : 0.f;
+  }
+  for (int v = lane; v < nvec; v += 32) {
+    uint4 u[KMAX];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[i][q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int p = slot_pos[(size_t)t * k + j];
-      if (p < 0) continue;
-      const float g = w[(size_t)t * k + j];
-      const uint4* src = reinterpret_cast<const uint4*>(y_perm + (size_t)p * d);
+    for (int j = 0; j < KMAX; ++j)
+      u[j] = p[j] >= 0 ? reinterpret_cast<const uint4*>(y_perm + (size_t)p[j] * d)[v] : make_uint4(0, 0, 0, 0);
+    uint4 us = make_uint4(0, 0, 0, 0);
+    if (y_shared != nullptr) us = reinterpret_cast<const uint4*>(y_shared + (size_t)t * d)[v];
+    float acc[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int v = v0 + lane + 32 * i;
-        if (v < nvec) {
-          const uint4 u = src[v];
-          acc[i][0] = fmaf(g, bf16lo(u.x), acc[i][0]); acc[i][1] = fmaf(g, bf16hi(u.x), acc[i][1]);
-          acc[i][2] = fmaf(g, bf16lo(u.y), acc[i][2]); acc[i][3] = fmaf(g, bf16hi(u.y), acc[i][3]);
-          acc[i][4] = fmaf(g, bf16lo(u.z), acc[i][4]); acc[i][5] = fmaf(g, bf16hi(u.z), acc[i][5]);
-          acc[i][6] = fmaf(g, bf16lo(u.w), acc[i][6]); acc[i][7] = fmaf(g, bf16hi(u.w), acc[i][7]);
-        }
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (p[j] >= 0) {
+        acc[0] = fmaf(g[j], bf16lo(u[j].x), acc[0]); acc[1] = fmaf(g[j], bf16hi(u[j].x), acc[1]);
+        acc[2] = fmaf(g[j], bf16lo(u[j].y), acc[2]); acc[3] = fmaf(g[j], bf16hi(u[j].y), acc[3]);
+        acc[4] = fmaf(g[j], bf16lo(u[j].z), acc[4]); acc[5] = fmaf(g[j], bf16hi(u[j].z), acc[5]);
+        acc[6] = fmaf(g[j], bf16lo(u[j].w), acc[6]); acc[7] = fmaf(g[j], bf16hi(u[j].w), acc[7]);
       }
     }
     if (y_shared != nullptr) {
-      const uint4* src = reinterpret_cast<const uint4*>(y_shared + (size_t)t * d);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int v = v0 + lane + 32 * i;
-        if (v < nvec) {
-          const uint4 u = src[v];
-          acc[i][0] += bf16lo(u.x); acc[i][1] += bf16hi(u.x); acc[i][2] += bf16lo(u.y); acc[i][3] += bf16hi(u.y);
-          acc[i][4] += bf16lo(u.z); acc[i][5] += bf16hi(u.z); acc[i][6] += bf16lo(u.w); acc[i][7] += bf16hi(u.w);
-        }
-      }
+      acc[0] += bf16lo(us.x); acc[1] += bf16hi(us.x); acc[2] += bf16lo(us.y); acc[3] += bf16hi(us.y);
+      acc[4] += bf16lo(us.z); acc[5] += bf16hi(us.z); acc[6] += bf16lo(us.w); acc[7] += bf16hi(us.w);
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + (size_t)t * d);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int v = v0 + lane + 32 * i;
-      if (v < nvec) {
-        uint4 o;
-        o.x = pack_bf16x2(acc[i][0], acc[i][1]); o.y = pack_bf16x2(acc[i][2], acc[i][3]);
-        o.z = pack_bf16x2(acc[i][4], acc[i][5]); o.w = pack_bf16x2(acc[i][6], acc[i][7]);
-        dst[v] = o;
-      }
-    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]); o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]); o.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(out + (size_t)t * d)[v] = o;
   }
 }
 

@@ -158,14 +158,27 @@ __device__ __forceinline__ void warp_argmax(float& bv, int& bi) {
   }
 }
 
-// Exact fp32 logit of one expert for one token, computed by the whole warp:
-// lane l accumulates inputs l, l+32, ... with fmaf, then a fixed xor tree.
-__device__ __forceinline__ float warp_dot(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ wr, int d) {
-  float acc = 0.f;
-  for (int i = lane_id(); i < d; i += 32) acc = fmaf(__bfloat162float(xr[i]), wr[i], acc);
+// Exact fp32 logits of up to 8 experts for one token, computed by the whole
+// warp: lane l accumulates inputs l, l+32, ... with fmaf (one chain per
+// expert), then a fixed xor tree.  The order does not depend on how many
+// experts are batched together.
+__device__ __forceinline__ void warp_dot_multi(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ W,
+                                               int d, const int (&ex)[8], int n, float (&out)[8]) {
+  float acc[8];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  return acc;
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  for (int i = lane_id(); i < d; i += 32) {
+    const float xv = __bfloat162float(xr[i]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (c < n) acc[c] = fmaf(xv, W[(size_t)ex[c] * d + i], acc[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+    out[c] = acc[c];
+  }
 }
 
 struct RefineArgs {
@@ -177,14 +190,91 @@ struct RefineArgs {
   float gamma;             // bound factor of the screening logits: |err| <= gamma * ||x_t|| * ||w_e||
 };
 
+// Per-token tail of the router, shared by every logit source: softmax, top-k
+// (k rounds of warp argmax on (logit desc, index asc)), gates, and the
+// per-warp running statistics (sum of p per expert, picks per expert).
+template <int EPL>
+__device__ __forceinline__ void route_token(const float (&z)[EPL], int t, int E, int k, int renorm,
+                                            float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_w, float (&pacc)[EPL], int (&cacc)[EPL]) {
+  const int lane = lane_id();
+  if (logits_out != nullptr) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (lane + 32 * i < E) logits_out[(size_t)t * E + lane + 32 * i] = z[i];
+  }
+  float m = z[0];
+#pragma unroll
+  for (int i = 1; i < EPL; ++i) m = fmaxf(m, z[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float ez[EPL], ssum = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    ez[i] = (lane + 32 * i < E) ? expf(z[i] - m) : 0.f;
+    ssum += ez[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+  const float inv = 1.f / ssum;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) pacc[i] += ez[i] * inv;
+
+  unsigned taken = 0u;
+  float wv = 0.f, wsum = 0.f;
+  int iv = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
+    }
+    warp_argmax(bv, bi);
+    if ((bi & 31) == lane) {
+      const int i = bi >> 5;
+      taken |= 1u << i;
+#pragma unroll
+      for (int q = 0; q < EPL; ++q)
+        if (q == i) cacc[q] += 1;
+    }
+    const float pj = expf(bv - m) * inv;
+    if (lane == j) { wv = pj; iv = bi; }
+    wsum += pj;
+  }
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = iv;
+    topk_w[(size_t)t * k + lane] = renorm ? wv / wsum : wv;
+  }
+}
+
+// Chunk statistics of a CTA of 8 warps, combined in fixed warp order.
+template <int EPL>
+__device__ __forceinline__ void chunk_stats(float (&s_p)[8][EPL * 32], int (&s_c)[8][EPL * 32],
+                                            const float (&pacc)[EPL], const int (&cacc)[EPL], int chunk, int E,
+                                            int32_t* __restrict__ cnt, float* __restrict__ psum) {
+  const int lane = lane_id(), warp = warp_id();
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) { s_p[warp][lane + 32 * i] = pacc[i]; s_c[warp][lane + 32 * i] = cacc[i]; }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ps = 0.f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
+    cnt[(size_t)chunk * E + e] = cs;
+    psum[(size_t)chunk * E + e] = ps;
+  }
+}
+
 // One warp per token.  Lane l holds the logits of experts l, l+32, ...
 //   logits = sum_split part[split] (+ bias); softmax; top-k; gates.
 // With refine.x set, `part` holds screening logits from the tensor cores whose
 // error is at most gamma * ||x_t|| * ||w_e||.  Every expert that could still be
 // in the top k under that bound (screening logit >= k-th largest - 2 bound) is
 // recomputed as a plain fp32 dot product, so the top-k decision is made on
-// fp32 FMA logits exactly as in the CUDA-core router; the others are
-// certified out of the top k.
+// fp32 FMA logits; the others are certified out of the top k.
 // Per chunk of kChunk tokens (one CTA, 8 warps x 16 tokens):
 //   cnt[chunk][e]  tokens of the chunk that chose e
 //   psum[chunk][e] sum over the chunk's tokens of p[t,e] (fixed order)
@@ -260,83 +350,156 @@ __global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ p
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float bound = refine.gamma * sqrtf(ss) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
       const float thr = kth - 2.f * bound;
+      // recompute the candidates exactly, up to 8 experts per pass
+      int ex[8];
+      int n = 0;
+      auto flush = [&]() {
+        float v[8];
+        warp_dot_multi(xr, refine.W, refine.d, ex, n, v);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c < n) {
+            const int e = ex[c];
+            float zz = v[c];
+            if (refine.bias != nullptr) zz += refine.bias[e];
+            if ((e & 31) == lane) {
+#pragma unroll
+              for (int i = 0; i < EPL; ++i)
+                if (i == (e >> 5)) z[i] = zz;
+            }
+          }
+        }
+        n = 0;
+      };
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const int e0 = 32 * i;
-        unsigned cand = __ballot_sync(0xffffffffu, lane + e0 < E && z[i] >= thr);
+        unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && z[i] >= thr);
         while (cand) {
           const int l = __ffs(cand) - 1;
           cand &= cand - 1;
-          const int e = e0 + l;
-          float v = warp_dot(xr, refine.W + (size_t)e * refine.d, refine.d);
-          if (refine.bias != nullptr) v += refine.bias[e];
-          if (lane == l) z[i] = v;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c == n) ex[c] = 32 * i + l;
+          if (++n == 8) flush();
+        }
+      }
+      if (n > 0) flush();
+    }
+    route_token<EPL>(z, t, E, k, renorm, logits_out, topk_idx, topk_w, pacc, cacc);
+  }
+  chunk_stats<EPL>(s_p, s_c, pacc, cacc, chunk, E, cnt, psum);
+}
+
+// Router fully in one kernel for small E * d: the CTA keeps W_r^T in shared
+// memory ([d][32 EPL + 1] fp32, padded against bank conflicts); each warp
+// computes its tokens' logits as plain fp32 FMA chains over the inputs (lane l
+// owns experts l, l+32, ...), then softmax / top-k / gates as above.
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_fused(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                                                      const float* __restrict__ bias, float* __restrict__ logits_out,
+                                                      int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                                      int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
+                                                      int d, int E, int k, int renorm) {
+  extern __shared__ float s_wt[];
+  __shared__ float s_p[8][EPL * 32];
+  __shared__ int s_c[8][EPL * 32];
+  constexpr int EP = EPL * 32 + 1;
+  for (int i = threadIdx.x; i < E * d; i += blockDim.x) {  // coalesced reads; odd row pitch: no bank conflicts
+    const int e = i / d, c = i - e * d;
+    s_wt[c * EP + e] = W[i];
+  }
+  __syncthreads();
+  const int lane = lane_id(), warp = warp_id();
+  const int chunk = blockIdx.x;
+  float pacc[EPL];
+  int cacc[EPL];
+  float b[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    pacc[i] = 0.f;
+    cacc[i] = 0;
+    const int e = lane + 32 * i;
+    b[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+  }
+  const int t_first = chunk * kChunk + warp * (kChunk / 8);
+  const int t_end = min(T, t_first + kChunk / 8);
+  for (int t = t_first; t < t_end; ++t) {
+    float acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+#pragma unroll 2
+    for (int c0 = 0; c0 < d; c0 += 8) {
+      const uint4 u = xr[c0 >> 3];  // same address in every lane: one broadcast load
+      const float xv[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                           bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float* wr = s_wt + (size_t)(c0 + q) * EP + lane;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] = fmaf(xv[q], wr[32 * i], acc[i]);
+      }
+    }
+    float z[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = (lane + 32 * i < E) ? acc[i] + b[i] : -INFINITY;
+    route_token<EPL>(z, t, E, k, renorm, logits_out, topk_idx, topk_w, pacc, cacc);
+  }
+  chunk_stats<EPL>(s_p, s_c, pacc, cacc, chunk, E, cnt, psum);
+}
+
+// Router logits for small T (decode): W_r is the large operand and is
+// streamed once.  A CTA of 8 warps owns 2 experts; the 4 warps of an expert
+// split the inputs into quarters, lane l of a warp takes inputs 4l..4l+3 of
+// each 128-input step, and keeps one fp32 FMA chain per token (TT tokens per
+// pass).  Lanes, then quarters, are combined in fixed order.
+template <int TT>
+__global__ void __launch_bounds__(256) k_router_skinny(const __nv_bfloat16* __restrict__ x,
+                                                       const float* __restrict__ W, float* __restrict__ logits, int T,
+                                                       int d, int E) {
+  __shared__ float s_part[8][TT];
+  const int lane = lane_id(), warp = warp_id();
+  const int e = blockIdx.x * 2 + (warp >> 2);
+  const int quarter = warp & 3;
+  const int span = ((d + 511) / 512) * 128;  // inputs per quarter, a multiple of 128
+  const int i_beg = quarter * span, i_end = min(d, i_beg + span);
+  for (int t0 = 0; t0 < T; t0 += TT) {
+    float acc[TT];
+#pragma unroll
+    for (int j = 0; j < TT; ++j) acc[j] = 0.f;
+    if (e < E) {
+      for (int i = i_beg + lane * 4; i < i_end; i += 128) {
+        const float4 w4 = *reinterpret_cast<const float4*>(W + (size_t)e * d + i);
+#pragma unroll
+        for (int j = 0; j < TT; ++j) {
+          if (t0 + j < T) {
+            const uint2 u = *reinterpret_cast<const uint2*>(x + (size_t)(t0 + j) * d + i);
+            acc[j] = fmaf(bf16lo(u.x), w4.x, acc[j]);
+            acc[j] = fmaf(bf16hi(u.x), w4.y, acc[j]);
+            acc[j] = fmaf(bf16lo(u.y), w4.z, acc[j]);
+            acc[j] = fmaf(bf16hi(u.y), w4.w, acc[j]);
+          }
         }
       }
     }
-    if (logits_out != nullptr) {
 #pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (lane + 32 * i < E) logits_out[(size_t)t * E + lane + 32 * i] = z[i];
+    for (int j = 0; j < TT; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
     }
-    // softmax
-    float m = z[0];
+    if (lane == 0) {
 #pragma unroll
-    for (int i = 1; i < EPL; ++i) m = fmaxf(m, z[i]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float ez[EPL], ssum = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      ez[i] = (lane + 32 * i < E) ? expf(z[i] - m) : 0.f;
-      ssum += ez[i];
+      for (int j = 0; j < TT; ++j) s_part[warp][j] = acc[j];
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-    const float inv = 1.f / ssum;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) pacc[i] += ez[i] * inv;
-
-    // top-k: k rounds of warp argmax on (logit desc, index asc)
-    unsigned taken = 0u;
-    float wv = 0.f, wsum = 0.f;
-    int iv = 0;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
+    __syncthreads();
+    if (quarter == 0 && e < E) {
+      for (int j = lane; j < TT && t0 + j < T; j += 32) {
+        const int w0 = warp;  // warps w0..w0+3 hold the quarters of expert e
+        logits[(size_t)(t0 + j) * E + e] =
+            ((s_part[w0][j] + s_part[w0 + 1][j]) + s_part[w0 + 2][j]) + s_part[w0 + 3][j];
       }
-      warp_argmax(bv, bi);
-      if ((bi & 31) == lane) {
-        const int i = bi >> 5;
-        taken |= 1u << i;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q)
-          if (q == i) cacc[q] += 1;
-      }
-      const float pj = expf(bv - m) * inv;
-      if (lane == j) { wv = pj; iv = bi; }
-      wsum += pj;
     }
-    if (lane < k) {
-      topk_idx[(size_t)t * k + lane] = iv;
-      topk_w[(size_t)t * k + lane] = renorm ? wv / wsum : wv;
-    }
-  }
-  // chunk statistics: warps combined in fixed order
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) { s_p[warp][lane + 32 * i] = pacc[i]; s_c[warp][lane + 32 * i] = cacc[i]; }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float ps = 0.f;
-    int cs = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
-    cnt[(size_t)chunk * E + e] = cs;
-    psum[(size_t)chunk * E + e] = ps;
+    __syncthreads();
   }
 }
 
