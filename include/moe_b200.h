@@ -213,6 +213,29 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
 int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream);
 
 /*
+ * moe_permute without a workspace argument.  No counterpart on the pages: it
+ * exists for callers that cannot allocate device memory for scratch -- code
+ * that runs where cudaMalloc is not allowed or not safe (inside a framework
+ * that owns every device allocation, on a path that must not synchronise the
+ * device, in a plug-in handed only its input and output buffers).
+ *   Same arguments, outputs and rules as moe_permute, minus workspace/ws_bytes.
+ *   Scratch: a fixed device array inside this library (about 1 MiB, held by
+ *   every GPU that loads the library until the process exits) -- so
+ *   ceil(T / 128) * E must be <= 262144, otherwise MOE_UNSUPPORTED_SHAPE is
+ *   returned and nothing is enqueued.
+ *   Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Every call shares the one array, which keeps the last call's contents:
+ *   calls that overlap on the GPU (concurrent streams, or several host
+ *   threads) race on it and must be serialised by the caller.
+ */
+int moe_permute_noalloc(const moe_shape* s, const void* x, const int32_t* topk_idx, int32_t* slot_pos,
+                        uint8_t* drop_mask, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_src,
+                        void* x_perm, moe_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's status word.
  * *device_status receives MOE_OK or the first device-side error recorded
  * (MOE_DEVICE_TIMEOUT); *site (may be NULL) where it happened.  Returns

@@ -28,7 +28,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_INVALID_ARGUMENT", 2: "MOE_UNSUPPORTED_SHAPE", 3:
 
 EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route", "moe_route_from_logits",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
-            "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string"]
+            "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
+            "moe_permute_noalloc"]
 
 
 class MoeError(RuntimeError):
@@ -83,6 +84,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_selftest_wait_timeout": (ctypes.c_int, [_P]),
         "moe_launch_count": (u64, []),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "moe_permute_noalloc": (ctypes.c_int, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -208,6 +210,31 @@ def moe_permute(shape: MoeShape, x, topk_idx, *, ws=None, stream=None):
                           _ptr(out["drop_mask"]), _ptr(out["counts"]), _ptr(out["kept"]), _ptr(out["offsets"]),
                           _ptr(out["row_src"]), _ptr(out["x_perm"]), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_permute")
+    return out
+
+
+def moe_permute_noalloc(shape: MoeShape, x, topk_idx, *, stream=None):
+    """moe_permute without a workspace: the library's fixed scratch array is used instead.
+
+    For callers that cannot allocate device scratch; the outputs here are still
+    torch tensors.  Calls that overlap on the GPU race on the shared scratch.
+    """
+    T, d, E, k = shape.T, shape.d, shape.E, shape.k
+    _want(x, torch.bfloat16, (T, d), "x")
+    _want(topk_idx, torch.int32, (T, k), "topk_idx")
+    dev = x.device
+    R = shape.R
+    out = dict(slot_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
+               drop_mask=torch.empty(T, k, dtype=torch.uint8, device=dev),
+               counts=torch.empty(E, dtype=torch.int32, device=dev),
+               kept=torch.empty(E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               row_src=torch.full((R,), -1, dtype=torch.int32, device=dev),
+               x_perm=torch.zeros(R, d, dtype=torch.bfloat16, device=dev))
+    rc = _L().moe_permute_noalloc(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(out["slot_pos"]),
+                                  _ptr(out["drop_mask"]), _ptr(out["counts"]), _ptr(out["kept"]),
+                                  _ptr(out["offsets"]), _ptr(out["row_src"]), _ptr(out["x_perm"]), _stream(stream))
+    _check(rc, "moe_permute_noalloc")
     return out
 
 

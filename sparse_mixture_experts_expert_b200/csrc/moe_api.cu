@@ -658,3 +658,61 @@ extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
   count_launch();
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR;
 }
+
+// ====================================================================== allocation-free grouping
+//
+// moe_permute_noalloc: the grouping of moe_permute for callers that cannot
+// hand the library a workspace.  Its scratch (the per-chunk expert histogram
+// and, when the caller passes no counts buffer, the per-expert counts) lives in
+// the fixed array below, which every GPU that loads this library keeps for the
+// life of the process.  Host code must not pass the array's name to a kernel:
+// on the host it is only a stand-in symbol, so the device address is looked up
+// once per device with cudaGetSymbolAddress and cached.
+
+namespace moe {
+
+constexpr long long kNoAllocHistInts = 262144;  // ceil(T / 128) * E must not exceed this
+constexpr int kNoAllocCountInts = kMaxE;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocHistInts + kNoAllocCountInts];
+
+static std::mutex g_noalloc_mu;
+static int32_t* g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device (set up on the first call per device).
+static int noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_CUDA_ERROR;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_CUDA_ERROR;
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int moe_permute_noalloc(const moe_shape* s, const void* x, const int32_t* topk_idx, int32_t* slot_pos,
+                                   uint8_t* drop_mask, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                   int32_t* row_src, void* x_perm, moe_stream_t stream) {
+  using namespace moe;
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!x || !topk_idx || !slot_pos || !kept || !offsets || !x_perm) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_INVALID_ARGUMENT;
+  const long long nchunks = cdiv(s->T, kChunk);
+  if (nchunks * s->E > kNoAllocHistInts) return MOE_UNSUPPORTED_SHAPE;  // beyond the fixed scratch
+  int32_t* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  int32_t* cnt = scratch;                                   // fully rewritten by k_chunk_hist every call
+  int32_t* cts = counts ? counts : scratch + kNoAllocHistInts;  // fully rewritten by k_chunk_scan
+  k_chunk_hist<<<(unsigned)nchunks, 256, s->E * sizeof(int), stream>>>(topk_idx, cnt, (int)s->T, s->E, s->k);
+  MOE_LAUNCH_CHECK();
+  rc = launch_scan(s, cnt, nullptr, cts, nullptr, nullptr, stream);
+  if (rc) return rc;
+  return launch_scatter(s, x, topk_idx, cnt, cts, slot_pos, drop_mask, row_src, x_perm, kept, offsets, stream);
+}
