@@ -145,7 +145,7 @@ int moe_route_from_logits(const moe_shape* s, const float* logits, int32_t* topk
  *   kept      [E] int32          out  rows filled in group e
  *   offsets   [E+1] int32        out  first row of group e (e*C with a capacity, else
  *                                     prefix sum of counts); offsets[E] = R
- *   row_src   [R] int32 / NULL   out  t*k + j for filled rows, -1 for unfilled rows
+ *   row_src   [R] int32 / NULL   out  t*k + j for filled rows; unfilled rows untouched
  *   x_perm    [R, d] bf16        out  x_perm[slot_pos[t,j]] = x[t]; unfilled rows untouched
  * Rows of a group are in token order; an assignment is dropped when its rank
  * (tokens before it that chose the same expert) is >= C.  Bit-exact and
@@ -221,7 +221,7 @@ int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void*
  *   Same arguments, outputs and rules as moe_permute, minus workspace/ws_bytes.
  *   Scratch: a fixed device array inside this library (about 1 MiB, held by
  *   every GPU that loads the library until the process exits) -- so
- *   ceil(T / 128) * E must be <= 262144, otherwise MOE_UNSUPPORTED_SHAPE is
+ *   ceil(T / 32) * E must be <= 262144, otherwise MOE_UNSUPPORTED_SHAPE is
  *   returned and nothing is enqueued.
  *   Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
  *   The first call on each device looks up the array's device address
@@ -245,6 +245,15 @@ int moe_get_status(moe_stream_t stream, int32_t* device_status, uint32_t* site);
 
 /* Upper bound, in nanoseconds, of every device-side wait (default 2e9). */
 int moe_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * Kernel choice for the bf16 expert GEMMs (process-wide, default 1).  1: groups
+ * averaging at least 192 rows run on CTA pairs (256-row tiles, tcgen05
+ * cta_group::2); 0: single-CTA 128-row tiles everywhere.  Both compute the same
+ * products in the same fp32 order per output.  Returns MOE_INVALID_ARGUMENT
+ * for other values.  Implementation choice only; the pages have no counterpart.
+ */
+int moe_set_pair_gemm(int32_t enable);
 
 /* Enqueue a kernel whose bounded wait on an mbarrier nobody arrives on must give
  * up after the wait limit: exercises the MOE_DEVICE_TIMEOUT path safely. */

@@ -29,7 +29,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_INVALID_ARGUMENT", 2: "MOE_UNSUPPORTED_SHAPE", 3:
 EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route", "moe_route_from_logits",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
             "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
-            "moe_permute_noalloc"]
+            "moe_permute_noalloc", "moe_set_pair_gemm"]
 
 
 class MoeError(RuntimeError):
@@ -81,6 +81,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_quantize_int4": (ctypes.c_int, [_P, i64, i32, _P, _P, _P]),
         "moe_get_status": (ctypes.c_int, [_P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_uint32)]),
         "moe_set_wait_limit_ns": (ctypes.c_int, [u64]),
+        "moe_set_pair_gemm": (ctypes.c_int, [i32]),
         "moe_selftest_wait_timeout": (ctypes.c_int, [_P]),
         "moe_launch_count": (u64, []),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -192,19 +193,31 @@ def moe_route_from_logits(shape: MoeShape, logits, *, aux=False, ws=None, stream
     return out
 
 
-def moe_permute(shape: MoeShape, x, topk_idx, *, ws=None, stream=None):
+def permute_outputs(shape: MoeShape, device):
+    """Output buffers of moe_permute: row_src = -1 and x_perm = 0 in the rows the call leaves unfilled."""
+    T, d, E, k, R = shape.T, shape.d, shape.E, shape.k, shape.R
+    return dict(slot_pos=torch.empty(T, k, dtype=torch.int32, device=device),
+                drop_mask=torch.empty(T, k, dtype=torch.uint8, device=device),
+                counts=torch.empty(E, dtype=torch.int32, device=device),
+                kept=torch.empty(E, dtype=torch.int32, device=device),
+                offsets=torch.empty(E + 1, dtype=torch.int32, device=device),
+                row_src=torch.full((R,), -1, dtype=torch.int32, device=device),
+                x_perm=torch.zeros(R, d, dtype=torch.bfloat16, device=device))
+
+
+def moe_permute(shape: MoeShape, x, topk_idx, *, ws=None, stream=None, out=None):
+    """Grouping by expert.  `out` (from permute_outputs) reuses buffers: rows this call leaves unfilled keep
+    what they held, and nothing is allocated or filled here."""
     T, d, E, k = shape.T, shape.d, shape.E, shape.k
     _want(x, torch.bfloat16, (T, d), "x")
     _want(topk_idx, torch.int32, (T, k), "topk_idx")
     dev = x.device
-    R = shape.R
-    out = dict(slot_pos=torch.empty(T, k, dtype=torch.int32, device=dev),
-               drop_mask=torch.empty(T, k, dtype=torch.uint8, device=dev),
-               counts=torch.empty(E, dtype=torch.int32, device=dev),
-               kept=torch.empty(E, dtype=torch.int32, device=dev),
-               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
-               row_src=torch.full((R,), -1, dtype=torch.int32, device=dev),
-               x_perm=torch.zeros(R, d, dtype=torch.bfloat16, device=dev))
+    if out is None:
+        out = permute_outputs(shape, dev)
+    else:
+        _want(out["x_perm"], torch.bfloat16, (shape.R, d), "out['x_perm']")
+        _want(out["row_src"], torch.int32, (shape.R,), "out['row_src']")
+        _want(out["slot_pos"], torch.int32, (T, k), "out['slot_pos']")
     ws = ws if ws is not None else workspace(shape, dev)
     rc = _L().moe_permute(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(out["slot_pos"]),
                           _ptr(out["drop_mask"]), _ptr(out["counts"]), _ptr(out["kept"]), _ptr(out["offsets"]),
@@ -316,3 +329,8 @@ def moe_get_status(stream=None):
 
 def moe_launch_count() -> int:
     return int(_L().moe_launch_count())
+
+
+def moe_set_pair_gemm(enable: bool) -> None:
+    """Select CTA-pair (True, default) or single-CTA (False) tiles for the bf16 expert GEMMs, process-wide."""
+    _check(_L().moe_set_pair_gemm(1 if enable else 0), "moe_set_pair_gemm")

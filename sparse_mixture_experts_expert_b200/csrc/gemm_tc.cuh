@@ -12,7 +12,7 @@
 // optimisation path of its routed-expert kernel; this is that GEMM for sm_100a.
 //
 // Structure: persistent CTAs (one per SM), 8 warps.
-//   warp 0 lane 0  TMA producer: A tile 128 x 64 and B tile N x 64 per stage
+//   warp 0         TMA producer: A tile 128 x 64 and B tile N x 64 per stage
 //                  (128-byte swizzle), ring of kStages stages.
 //   warp 1         allocates 2 x BN TMEM columns; lane 0 issues tcgen05.mma
 //                  (M=128, N=BN, K=16, bf16 -> fp32) and commits stages back.
@@ -23,6 +23,18 @@
 // tiles, enumerated from the device-side group table (no host sync).  Row tiles
 // that run past a group's end read the next group's rows (or TMA zero fill);
 // their outputs are masked.  Every wait is bounded.
+//
+// CTA-pair variant (CG = 2, launched as clusters of 2): the pair owns a tile of
+// 256 rows x BN columns.  Each CTA loads its own 128 rows of A and half of the
+// B tile (BN/2 rows: the gate slice in CTA 0 and the up slice in CTA 1 for the
+// gated GEMM), both copies counting on the leader CTA's stage barrier; the
+// leader issues one M = 256 MMA per k-step (tcgen05 cta_group::2), which reads
+// both CTAs' shared memory and leaves each CTA's 128 x BN accumulator in that
+// CTA's tensor memory.  Per CTA this moves (128 + BN/2) x 64 operand elements
+// per k-step instead of (128 + BN) x 64 for the same MMA work, which is what
+// bounds the single-CTA kernel (L2 -> SM bandwidth) for short reductions.
+// Stage and accumulator releases are multicast commits to both CTAs; the
+// epilogue warps of both CTAs release an accumulator on the leader's barrier.
 #pragma once
 
 #include "common.cuh"
@@ -54,14 +66,14 @@ constexpr int kEpiW = 64;                                   // columns staged pe
 constexpr int kEpiRow = kEpiW + 8;                          // padded staging row (bf16), conflict-free
 constexpr int kEpiBytes = 4 * 32 * kEpiRow * 2;             // four epilogue warps x 32 rows
 
-template <int BN>
+template <int BN, int CG = 1>
 struct GemmCfg {
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = (CG == 2 ? BN / 2 : BN) * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBudget = 219 * 1024 - 1024 - kEpiBytes;
   static constexpr int kStages = kBudget / kStageBytes > 8 ? 8 : kBudget / kStageBytes;
-  static constexpr int kTmemCols = 2 * BN;  // two accumulators
+  static constexpr int kTmemCols = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);  // two accumulators, pow2
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kEpiBytes;
 };
 
@@ -69,16 +81,19 @@ struct GemmCfg {
 __device__ __forceinline__ float act_silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + erff(g * 0.7071067811865476f)); }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int CG = 1>
 __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, CG>;
   constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
+  constexpr bool kPair = CG == 2;
+  static_assert(!kPair || MODE != kModeF32, "the router GEMM runs on single CTAs");
   constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
-  constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box
+  constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box (single CTA)
+  constexpr int TM = kBM * CG;              // rows per tile
   constexpr int S = Cfg::kStages;
-  constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN);
+  constexpr uint32_t IDESC = idesc_bf16_f32(TM, BN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -90,6 +105,9 @@ __global__ void __launch_bounds__(256, 1)
   __shared__ int s_grows[kMaxGroupsSmem];
 
   const int warp = warp_id(), lane = lane_id();
+  const int crank = kPair ? (int)cluster_ctarank() : 0;   // 0 = leader of the pair
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int n_tiles = (p.N + OUTN - 1) / OUTN;
   const int nk = (p.K + kBK - 1) / kBK;
   const bool single = p.group_rows == nullptr;
@@ -102,7 +120,7 @@ __global__ void __launch_bounds__(256, 1)
     int local = 0;
     for (int g = g0; g < g1; ++g) {
       const long long rows = single ? p.R : (long long)p.group_rows[g];
-      local += (int)((rows + kBM - 1) / kBM);
+      local += (int)((rows + TM - 1) / TM);
     }
     int incl = local;
 #pragma unroll
@@ -116,13 +134,14 @@ __global__ void __launch_bounds__(256, 1)
       const long long rows = single ? p.R : (long long)p.group_rows[g];
       s_grows[g] = (int)rows;
       s_gstart[g] = single ? 0 : p.group_start[g];
-      run += (int)((rows + kBM - 1) / kBM);
+      run += (int)((rows + TM - 1) / TM);
     }
     if (lane == 31) s_prefix[G] = incl;
   }
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&bar_full[s], 1); mbar_init(&bar_empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&bar_tfull[a], 1); mbar_init(&bar_tempty[a], 128); }
+    // accumulator release: 128 epilogue threads, or (pair) one arrival per epilogue warp of both CTAs
+    for (int a = 0; a < 2; ++a) { mbar_init(&bar_tfull[a], 1); mbar_init(&bar_tempty[a], kPair ? 8 : 128); }
     mbar_init(&bar_final, 1);
     s_abort = 0;
     fence_mbar_init();
@@ -130,11 +149,17 @@ __global__ void __launch_bounds__(256, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(&s_tmem, Cfg::kTmemCols);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(&s_tmem, Cfg::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&s_tmem, Cfg::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all();  // both CTAs' barriers initialised before any cross-CTA arrival
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
   const int total_m = s_prefix[G];
@@ -149,29 +174,43 @@ __global__ void __launch_bounds__(256, 1)
       if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
     }
     g = lo;
-    const long long m_local = (long long)(mt - s_prefix[g]) * kBM;
+    const long long m_local = (long long)(mt - s_prefix[g]) * TM + (long long)crank * kBM;
     const long long start = s_gstart[g];
     const long long rows = s_grows[g];
-    row0 = start + m_local;
-    rows_valid = (int)min((long long)kBM, rows - m_local);
+    row0 = start + m_local;   // this CTA's first row
+    rows_valid = (int)max(0ll, min((long long)kBM, rows - m_local));
     n0 = nt * OUTN;
   };
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      long long issued = 0;
-      for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
-        int g, rows_valid, n0;
-        long long row0;
-        locate(tile, g, row0, rows_valid, n0);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&bar_empty[stage], phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0101)) break;
-          uint8_t* a_s = smem + (size_t)stage * Cfg::kStageBytes;
-          uint8_t* b_s = a_s + Cfg::kABytes;
-          mbar_arrive_expect_tx(&bar_full[stage], Cfg::kStageBytes);
+    // The whole warp walks the tiles; lane 0 waits, arms the barriers and issues the copies.
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    for (long long tile = unit; tile < total && !__any_sync(0xffffffffu, s_abort); tile += n_units) {
+      int g, rows_valid, n0;
+      long long row0;
+      locate(tile, g, row0, rows_valid, n0);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        uint8_t* a_s = smem + (size_t)stage * Cfg::kStageBytes;
+        uint8_t* b_s = a_s + Cfg::kABytes;
+        if (lane == 0) {
+          ok = mbar_wait(&bar_empty[stage], phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0101);
+          // the leader's barrier counts the bytes of both CTAs of a pair
+          if (ok && crank == 0) mbar_arrive_expect_tx(&bar_full[stage], CG * Cfg::kStageBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (kPair) {
+          if (lane == 0) {
+            const uint32_t fb = mapa_shared(smem_u32(&bar_full[stage]), 0);
+            tma_load_2d_pair(a_s, &tmA, fb, kb * kBK, (int)row0);
+            const int brow = kGLU ? (crank == 0 ? n0 : p.up_row0 + n0) : n0 + crank * (BN / 2);
+            tma_load_3d_pair(b_s, &tmB, fb, kb * kBK, brow, g);
+          }
+        } else if (lane == 0) {
           const int ka = p.a_kwrap > 0 ? (kb * kBK) % p.a_kwrap : kb * kBK;
           tma_load_2d(a_s, &tmA, &bar_full[stage], ka, (int)row0);
           if (kGLU) {
@@ -180,11 +219,16 @@ __global__ void __launch_bounds__(256, 1)
           } else {
             tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
           }
-          ++issued;
-          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
+        ++issued;
+        if (++stage == S) { stage = 0; phase ^= 1u; }
       }
-      // Make sure no copy is still landing in shared memory when the CTA ends.
+      __syncwarp();
+      if (!ok) break;
+    }
+    // Make sure no copy is still landing in shared memory when the CTA ends (in a
+    // pair the leader's barriers count both CTAs' copies; the pair leaves together).
+    if (lane == 0 && crank == 0) {
       const int last = (int)(issued < S ? issued : (long long)S);
       for (int i = 1; i <= last; ++i) {
         const long long n = issued - i;
@@ -197,12 +241,12 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && crank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+      for (long long tile = unit; tile < total && !s_abort; tile += n_units) {
         if (!mbar_wait(&bar_tempty[acc], acc_phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0103)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -214,18 +258,25 @@ __global__ void __launch_bounds__(256, 1)
           const uint32_t b_addr = a_addr + Cfg::kABytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
+            if (kPair)
+              tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+                               (kb > 0 || kk > 0) ? 1u : 0u);
+            else
+              tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
+                          (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(&bar_empty[stage]);
+          if (kPair) tc_commit_pair_mc(&bar_empty[stage], 0x3);
+          else tc_commit(&bar_empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(&bar_tfull[acc]);
+        if (kPair) tc_commit_pair_mc(&bar_tfull[acc], 0x3);
+        else tc_commit(&bar_tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // all issued MMAs complete before TMEM is released
-      tc_commit(&bar_final);
+      if (kPair) tc_commit_pair(&bar_final);
+      else tc_commit(&bar_final);
       volatile int dummy = 0;
       mbar_wait(&bar_final, 0, p.wait_limit_ns, &dummy, 0x0105);
     }
@@ -236,8 +287,7 @@ __global__ void __launch_bounds__(256, 1)
     // memory -> coalesced row-segment stores (128 contiguous bytes per row per
     // 8 lanes).  The accumulator is handed back to the MMA warp as soon as its
     // last TMEM load has completed.
-    const int q = warp & 3;  // TMEM lane quarter
-    const int r = q * 32 + lane;
+    const int q = warp & 3;  // TMEM lane quarter: this warp's 32 accumulator rows
     constexpr int OUTW = OUTN < kEpiW ? OUTN : kEpiW;
     constexpr int ROUNDS = OUTN / OUTW;
     constexpr int LPR = OUTW / 8;   // lanes per staged row in the copy-out
@@ -245,7 +295,17 @@ __global__ void __launch_bounds__(256, 1)
     __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)S * Cfg::kStageBytes) + q * 32 * kEpiRow;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
+    // accumulator release: each thread (single CTA) or each warp on the leader's barrier (pair)
+    auto release_acc = [&](int a) {
+      tc_fence_before();
+      if (kPair) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bar_tempty[a]), 0));
+      } else {
+        mbar_arrive(&bar_tempty[a]);
+      }
+    };
+    for (long long tile = unit; tile < total && !s_abort; tile += n_units) {
       int g, rows_valid, n0;
       long long row0;
       locate(tile, g, row0, rows_valid, n0);
@@ -253,62 +313,77 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       if (MODE == kModeF32) {
-        const bool row_ok = r < rows_valid;
+        // fp32 rows through the staging buffer, 32 columns (128 bytes per row) per round
+        float* fstg = reinterpret_cast<float*>(stg);  // 32 rows x 36 floats per warp
+        constexpr int FR = 36;
 #pragma unroll 1
-        for (int c = 0; c < OUTN; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(t_row + c, v);
+        for (int c0 = 0; c0 < OUTN; c0 += 32) {
+          uint32_t v[2][16];
+          tmem_ld16(t_row + c0, v[0]);
+          tmem_ld16(t_row + c0 + 16, v[1]);
           tmem_ld_wait();
-          if (row_ok) {
-            float* frow = p.out_f32 + (row0 + r) * p.ldo + n0 + c;
+          if (c0 + 32 >= OUTN) release_acc(acc);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if (n0 + c + i < p.N) {
-                float f = __uint_as_float(v[i]);
-                if (p.bias != nullptr) f += p.bias[n0 + c + i];
-                frow[i] = f;
-              }
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              float4 f;
+              const int col = n0 + c0 + h * 16 + i;
+              f.x = __uint_as_float(v[h][i]) + (p.bias != nullptr && col + 0 < p.N ? p.bias[col + 0] : 0.f);
+              f.y = __uint_as_float(v[h][i + 1]) + (p.bias != nullptr && col + 1 < p.N ? p.bias[col + 1] : 0.f);
+              f.z = __uint_as_float(v[h][i + 2]) + (p.bias != nullptr && col + 2 < p.N ? p.bias[col + 2] : 0.f);
+              f.w = __uint_as_float(v[h][i + 3]) + (p.bias != nullptr && col + 3 < p.N ? p.bias[col + 3] : 0.f);
+              *reinterpret_cast<float4*>(fstg + lane * FR + h * 16 + i) = f;
             }
           }
+          __syncwarp();
+          // 8 lanes per 128-byte row segment, 4 rows per step
+          const int cb = (lane & 7) * 4;
+          const int col = n0 + c0 + cb;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            if (q * 32 + rr < rows_valid && col < p.N) {
+              const float4 val = *reinterpret_cast<const float4*>(fstg + rr * FR + cb);
+              *reinterpret_cast<float4*>(p.out_f32 + (row0 + q * 32 + rr) * p.ldo + col) = val;
+            }
+          }
+          __syncwarp();
         }
-        tc_fence_before();
-        mbar_arrive(&bar_tempty[acc]);
       } else {
 #pragma unroll 1
         for (int rd = 0; rd < ROUNDS; ++rd) {
+          // all TMEM loads of the round are issued before one wait
+          constexpr int NCH = OUTW / 16;
+          uint32_t v[NCH][16];
+          uint32_t u[kGLU ? NCH : 1][16];
 #pragma unroll
-          for (int c = 0; c < OUTW; c += 16) {
-            const int cc = rd * OUTW + c;
-            uint32_t v[16];
+          for (int ch = 0; ch < NCH; ++ch) {
+            tmem_ld16(t_row + rd * OUTW + ch * 16, v[ch]);
+            if (kGLU) tmem_ld16(t_row + OUTN + rd * OUTW + ch * 16, u[kGLU ? ch : 0]);
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
             uint32_t o[8];
-            if (kGLU) {
-              uint32_t u[16];
-              tmem_ld16(t_row + cc, v);
-              tmem_ld16(t_row + OUTN + cc, u);
-              tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
-                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            for (int i = 0; i < 8; ++i) {
+              if (kGLU) {
+                const float g0 = __uint_as_float(v[ch][2 * i]), g1 = __uint_as_float(v[ch][2 * i + 1]);
+                const float u0 = __uint_as_float(u[kGLU ? ch : 0][2 * i]);
+                const float u1 = __uint_as_float(u[kGLU ? ch : 0][2 * i + 1]);
                 const float a0 = MODE == kModeSwiGLU ? act_silu(g0) : act_gelu(g0);
                 const float a1 = MODE == kModeSwiGLU ? act_silu(g1) : act_gelu(g1);
                 o[i] = pack_bf16x2(a0 * u0, a1 * u1);
+              } else {
+                o[i] = pack_bf16x2(__uint_as_float(v[ch][2 * i]), __uint_as_float(v[ch][2 * i + 1]));
               }
-            } else {
-              tmem_ld16(t_row + cc, v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
             }
-            uint4* sp = reinterpret_cast<uint4*>(stg + lane * kEpiRow + c);
+            uint4* sp = reinterpret_cast<uint4*>(stg + lane * kEpiRow + ch * 16);
             sp[0] = make_uint4(o[0], o[1], o[2], o[3]);
             sp[1] = make_uint4(o[4], o[5], o[6], o[7]);
           }
-          if (rd == ROUNDS - 1) {
-            tc_fence_before();
-            mbar_arrive(&bar_tempty[acc]);
-          }
+          if (rd == ROUNDS - 1) release_acc(acc);
           __syncwarp();
           const int cb = (lane % LPR) * 8;
           const int col = n0 + rd * OUTW + cb;
@@ -327,10 +402,12 @@ __global__ void __launch_bounds__(256, 1)
     }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kPair) cluster_sync_all();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    if (kPair) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+    else tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
 }
 

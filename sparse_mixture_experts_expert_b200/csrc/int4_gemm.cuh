@@ -6,25 +6,20 @@
 // packed_input].  Scales here are bf16, one per 128 consecutive inputs of an
 // output row; two's-complement nibbles, the even input in the low nibble.
 //
-// Decode batches put ~1-8 rows on each touched expert, so the kernel is bound
-// by streaming the weights from HBM: every weight byte is read once, every
-// row of the group reuses it from registers.
-//   * one warp = one task = 16 output rows of one expert (gated mode: 16 gate
-//     rows W1 and the matching 16 up rows W3) over the full reduction length;
-//   * a thread loads 16 bytes (32 nibbles) per row per 128-input group; the
-//     nibbles are turned into bf16 pairs with one LOP3 each (the nibble, with
-//     its sign bit flipped, becomes the low mantissa bits of 128.0) and one
-//     packed subtraction of 136;
-//   * mma.sync m16n8k16 (bf16 in, fp32 out) multiplies the integer codes q
-//     (exact in bf16) by up to 8 activation rows; the reduction order inside
-//     a 128-group is permuted identically for weights and activations, so a
+// Decode batches put ~1-8 rows on each touched expert, so the GEMM is bound
+// by streaming the weights from HBM: every weight byte is read once and every
+// activation row of the group reuses it from registers.
+//   * the nibbles become bf16 pairs with one LOP3 each (the nibble, with its
+//     sign bit flipped, becomes the low mantissa bits of 128.0), optionally
+//     followed by one packed subtraction of 136 -- or not, in which case the
+//     product uses the codes q + 136 and 136 * sum(x) is removed per group;
+//   * mma.sync m16n8k16 (bf16 in, fp32 out) multiplies the integer codes
+//     (exact in bf16) by up to 8 activation rows; the reduction order inside a
+//     128-group is permuted identically for weights and activations, so a
 //     thread's 32 consecutive nibbles feed its fragments directly;
-//   * the fp32 partial of each 128-group is scaled by its bf16 scale and
-//     added to the fp32 total: w = q * s is applied exactly;
+//   * the fp32 partial of each 128-group is scaled by its bf16 scale and added
+//     to the fp32 total: w = q * s is applied exactly;
 //   * gated mode writes h = act(x W1^T) * (x W3^T) in bf16, plain mode y.
-// Groups with more than 8 rows are split into 8-row chunks, one task each;
-// the chunks of one 16-row block run on neighbouring warps, so the repeat
-// weight reads hit L2.
 #pragma once
 
 #include "common.cuh"
@@ -77,14 +72,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
@@ -96,6 +83,31 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 
 __device__ __forceinline__ uint32_t u4get(const uint4& v, int j) {
   return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+}
+
+// Word of 8 nibbles -> four bf16 pairs holding q + 136 (= 128 + (q + 8)), no
+// subtraction: the caller removes 136 * sum(x) per 128-group afterwards.
+__device__ __forceinline__ void offset_word(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t kMask = 0x000F000Fu, kMagic = 0x43084308u;
+  p[0] = lop3_and_xor(w, kMask, kMagic);
+  p[1] = lop3_and_xor(w >> 4, kMask, kMagic);
+  p[2] = lop3_and_xor(w >> 8, kMask, kMagic);
+  p[3] = lop3_and_xor(w >> 12, kMask, kMagic);
+}
+
+// acc += (q + 136)[16 x 128] . x[8 x 128]^T for one 16-row block (rows g and g+8 of this thread).
+// xf[j]: the activations of inputs 32c + 8j .. + 8 already in fragment order
+// (x0,x4), (x1,x5), (x2,x6), (x3,x7) -- see k_int4_act_prep.
+__device__ __forceinline__ void mma_group_offset(float (&acc)[4], const uint4& wa, const uint4& wb,
+                                                 const uint4 (&xf)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t pa[4], pb[4];
+    offset_word(u4get(wa, j), pa);
+    offset_word(u4get(wb, j), pb);
+    mma_bf16_16816(acc, pa[0], pb[0], pa[1], pb[1], xf[j].x, xf[j].y);
+    mma_bf16_16816(acc, pa[2], pb[2], pa[3], pb[3], xf[j].z, xf[j].w);
+  }
 }
 
 // MMA of one 128-group for one 16-row block: acc += q[16 x 128] . x[8 x 128]^T.
@@ -115,14 +127,66 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4& wa, cons
   }
 }
 
-template <bool GLU, int ACT>
-__global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
+// ---------------------------------------------------------------------------
+// Activation preparation of the offset-code product, one thread per 8 inputs:
+//   Aq: a copy of A with every 8 inputs x0..x7 stored as x0,x4,x1,x5,x2,x6,x3,x7,
+//       the order in which the nibble pairs of a weight word come out, so the
+//       streaming kernel uses 16-byte loads as B fragments without permutes;
+//   sums[r][g]: the sum of the 128 inputs of group g of row r (each thread adds
+//       its 8 in order, then the 16 threads of a group combine by a fixed xor
+//       tree), the correction term 136 * sum(x) of the offset codes.
+__global__ void __launch_bounds__(256) k_int4_act_prep(const __nv_bfloat16* __restrict__ A, long long rows, int K,
+                                                       float* __restrict__ sums, __nv_bfloat16* __restrict__ Aq) {
+  const long long n = rows * (K / 8);
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool on = i < n;
+  uint4 u = make_uint4(0, 0, 0, 0);
+  if (on) u = reinterpret_cast<const uint4*>(A)[i];
+  float acc = 0.f;
+  acc += bf16lo(u.x); acc += bf16hi(u.x); acc += bf16lo(u.y); acc += bf16hi(u.y);
+  acc += bf16lo(u.z); acc += bf16hi(u.z); acc += bf16lo(u.w); acc += bf16hi(u.w);
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (on) {
+    uint4 q;
+    q.x = prmt(u.x, u.z, 0x5410);
+    q.y = prmt(u.x, u.z, 0x7632);
+    q.z = prmt(u.y, u.w, 0x5410);
+    q.w = prmt(u.y, u.w, 0x7632);
+    reinterpret_cast<uint4*>(Aq)[i] = q;
+    if ((i & 15) == 0) sums[i >> 4] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming variant: the packed weights travel HBM -> shared memory by TMA
+// (2-D tensor map over [experts * rows, K/2] bytes), each warp owning a ring
+// of kI4Stages slabs of 32 rows x 128 bytes (256 inputs).  A warp's work is a
+// sequence of (task, slab) items; its lane 0 keeps kI4Stages items in flight
+// across task boundaries, so one SM has up to 16 x 3 x 4 KB of weight reads
+// outstanding.  Each task covers 32 weight rows: the 16 gate rows and the 16
+// matching up rows (gated mode) or 32 consecutive output rows (plain mode).
+constexpr int kI4Warps = 16;
+constexpr int kI4Stages = 3;
+constexpr int kI4SlabBytes = 32 * 128;
+constexpr int kI4Smem = kI4Warps * kI4Stages * kI4SlabBytes;
+
+// OFFS: multiply the offset codes q + 136 and subtract 136 * xsum[row][group]
+// (the activation group sums) once per group, instead of one packed
+// subtraction per pair of weights; p.act is then the fragment-ordered copy
+// written by k_int4_act_prep.
+template <bool GLU, int ACT, bool OFFS>
+__global__ void __launch_bounds__(kI4Warps * 32, 1)
+    k_int4_stream(const __grid_constant__ CUtensorMap tmW, const Int4Params p, unsigned long long wait_limit_ns,
+                  const float* __restrict__ xsum) {
+  extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ int s_prefix[kMaxGroupsSmem + 1];
+  __shared__ __align__(8) uint64_t s_bar[kI4Warps][kI4Stages];
+  __shared__ volatile int s_abort[kI4Warps];
   const int lane = lane_id(), warp = warp_id();
   const bool single = p.group_rows == nullptr;
   const int G = single ? 1 : p.n_groups;
-  const int oblocks = p.N / 16;
-  // tasks of group g: oblocks x ceil(rows / 8) (16 output rows x 8 activation rows each)
+  const int oblocks = GLU ? p.N / 16 : p.N / 32;   // 32 weight rows per task
   auto group_tasks = [&](int g) -> int {
     const long long rows = single ? p.R : (long long)p.group_rows[g];
     return (int)(oblocks * ((rows + 7) / 8));
@@ -145,83 +209,193 @@ __global__ void __launch_bounds__(256, 2) k_int4_gemm(const Int4Params p) {
     }
     if (lane == 31) s_prefix[G] = incl;
   }
+  if (lane == 0) {
+    for (int st = 0; st < kI4Stages; ++st) mbar_init(&s_bar[warp][st], 1);
+    s_abort[warp] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
   __syncthreads();
+
   const int total = s_prefix[G];
+  const int nslab = (p.K + 255) / 256;               // items per task (the last slab may hold one 128-group)
+  const int tfirst = blockIdx.x * kI4Warps + warp;
+  const int tstride = gridDim.x * kI4Warps;
+  uint8_t* ring = i4_smem + (size_t)warp * kI4Stages * kI4SlabBytes;
   const int gq = lane >> 2, c = lane & 3;
   const int ngroups_k = p.K / 128;
-  const long long wrow_bytes = p.K / 2;
 
-  for (int task = blockIdx.x * 8 + warp; task < total; task += gridDim.x * 8) {
-    int lo = 0, hi = G - 1;  // last group with s_prefix[g] <= task
+  struct TaskPos { int g, o0, n0, n_rows; long long row0; };
+  auto locate = [&](int task) -> TaskPos {
+    int lo = 0, hi = G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_prefix[mid] <= task) lo = mid; else hi = mid - 1;
     }
-    const int g = lo;
-    const long long row0 = single ? 0 : p.group_start[g];
-    const int n_rows = (int)(single ? p.R : (long long)p.group_rows[g]);
-    const int nchunks = (n_rows + 7) / 8;
-    const int tg = task - s_prefix[g];
-    const int o0 = (tg / nchunks) * 16;  // chunks of one row block are adjacent tasks: the repeat reads hit L2
-    const int n0 = (tg % nchunks) * 8;
-    const long long wbase = (long long)g * p.b_rows;
-    // this thread's weight rows: gate (or plain) rows o0+gq, o0+gq+8; up rows up_row0 + same
-    const uint8_t* wg0 = p.wq + (wbase + o0 + gq) * wrow_bytes + c * 16;
-    const uint8_t* wg1 = wg0 + 8 * wrow_bytes;
-    const uint8_t* wu0 = p.wq + (wbase + p.up_row0 + o0 + gq) * wrow_bytes + c * 16;
-    const uint8_t* wu1 = wu0 + 8 * wrow_bytes;
-    const __nv_bfloat16* sg0 = p.ws + (wbase + o0 + gq) * ngroups_k;
-    const __nv_bfloat16* sg1 = sg0 + 8 * ngroups_k;
-    const __nv_bfloat16* su0 = p.ws + (wbase + p.up_row0 + o0 + gq) * ngroups_k;
-    const __nv_bfloat16* su1 = su0 + 8 * ngroups_k;
+    TaskPos tp;
+    tp.g = lo;
+    tp.row0 = single ? 0 : p.group_start[lo];
+    tp.n_rows = (int)(single ? p.R : (long long)p.group_rows[lo]);
+    const int nchunks = (tp.n_rows + 7) / 8;
+    const int tg = task - s_prefix[lo];
+    tp.o0 = (tg / nchunks) * (GLU ? 16 : 32);
+    tp.n0 = (tg % nchunks) * 8;
+    return tp;
+  };
+  // weight rows of a task's two 16-row blocks (rows of the flattened [experts * b_rows] map)
+  auto rows_of = [&](const TaskPos& tp, int& ra, int& rb) {
+    ra = tp.g * p.b_rows + tp.o0;
+    rb = GLU ? tp.g * p.b_rows + p.up_row0 + tp.o0 : ra + 16;
+  };
 
-    {
-      const int tok = n0 + gq;            // B column this thread feeds
-      const bool tok_ok = tok < n_rows;
-      const __nv_bfloat16* xrow = p.act + (row0 + (tok_ok ? tok : 0)) * (long long)p.K + c * 32;
-      float tg[4] = {0.f, 0.f, 0.f, 0.f}, tu[4] = {0.f, 0.f, 0.f, 0.f};
-      uint4 a0 = ldg_stream(wg0), a1 = ldg_stream(wg1);
-      uint4 u0 = make_uint4(0, 0, 0, 0), u1 = make_uint4(0, 0, 0, 0);
-      if (GLU) { u0 = ldg_stream(wu0); u1 = ldg_stream(wu1); }
-      for (int kg = 0; kg < ngroups_k; ++kg) {
-        // prefetch the next group's weights
-        uint4 na0 = a0, na1 = a1, nu0 = u0, nu1 = u1;
-        if (kg + 1 < ngroups_k) {
-          na0 = ldg_stream(wg0 + (kg + 1) * 64);
-          na1 = ldg_stream(wg1 + (kg + 1) * 64);
-          if (GLU) { nu0 = ldg_stream(wu0 + (kg + 1) * 64); nu1 = ldg_stream(wu1 + (kg + 1) * 64); }
-        }
-        uint4 xv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          xv[j] = tok_ok ? *reinterpret_cast<const uint4*>(xrow + kg * 128 + 8 * j) : make_uint4(0, 0, 0, 0);
-        float pg[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_group(pg, a0, a1, xv);
-        const float s0 = __bfloat162float(sg0[kg]), s1 = __bfloat162float(sg1[kg]);
-        tg[0] = fmaf(pg[0], s0, tg[0]); tg[1] = fmaf(pg[1], s0, tg[1]);
-        tg[2] = fmaf(pg[2], s1, tg[2]); tg[3] = fmaf(pg[3], s1, tg[3]);
-        if (GLU) {
-          float pu[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_group(pu, u0, u1, xv);
-          const float r0 = __bfloat162float(su0[kg]), r1 = __bfloat162float(su1[kg]);
-          tu[0] = fmaf(pu[0], r0, tu[0]); tu[1] = fmaf(pu[1], r0, tu[1]);
-          tu[2] = fmaf(pu[2], r1, tu[2]); tu[3] = fmaf(pu[3], r1, tu[3]);
-        }
-        a0 = na0; a1 = na1; u0 = nu0; u1 = nu1;
+  // Producer state (lane 0 issues the copies; the values are warp-uniform).
+  // Items are (task, slab) pairs in order; issued - consumed <= kI4Stages.
+  int issued = 0, consumed = 0;
+  int p_task = tfirst, p_slab = 0, p_st = 0, p_ra = 0, p_rb = 0;
+  auto refill = [&]() {
+    while (issued - consumed < kI4Stages) {
+      if (p_slab == 0) {
+        if (p_task >= total) return;
+        const TaskPos tp = locate(p_task);
+        rows_of(tp, p_ra, p_rb);
       }
-      // D fragment: (m = gq, n = 2c, 2c+1) in [0],[1]; (m = gq+8, same n) in [2],[3]
+      if (lane == 0) {
+        uint8_t* dst = ring + p_st * kI4SlabBytes;
+        mbar_arrive_expect_tx(&s_bar[warp][p_st], kI4SlabBytes);
+        tma_load_2d(dst, &tmW, &s_bar[warp][p_st], p_slab * 128, p_ra);
+        tma_load_2d(dst + 16 * 128, &tmW, &s_bar[warp][p_st], p_slab * 128, p_rb);
+      }
+      ++issued;
+      if (++p_st == kI4Stages) p_st = 0;
+      if (++p_slab == nslab) { p_slab = 0; p_task += tstride; }
+    }
+  };
+
+  float tA[4], tB[4];
+  TaskPos cur{0, 0, 0, 0, 0};
+  const __nv_bfloat16* xrow = nullptr;   // this thread's activation row (token n0 + gq), inputs c*32 ..
+  const __nv_bfloat16* sA = nullptr;     // scales of weight row ra + gq (row + 8: + 8 * ngroups_k)
+  const __nv_bfloat16* sB = nullptr;     // scales of weight row rb + gq
+  const float* xs0 = nullptr;            // group sums of tokens n0 + 2c, n0 + 2c + 1
+  bool tok_ok = false, ok0 = false, ok1 = false;
+  const long long s8 = 8ll * ngroups_k;
+  int c_task = tfirst, c_slab = 0, c_st = 0;
+  uint32_t c_phase = 0;
+  while (true) {
+    if (c_slab == 0) {
+      if (c_task >= total || s_abort[warp]) break;
+      cur = locate(c_task);
+      int ra, rb;
+      rows_of(cur, ra, rb);
+      const int tok = cur.n0 + gq;
+      tok_ok = tok < cur.n_rows;
+      xrow = p.act + (cur.row0 + (tok_ok ? tok : 0)) * (long long)p.K + c * 32;
+      sA = p.ws + (long long)(ra + gq) * ngroups_k;
+      sB = p.ws + (long long)(rb + gq) * ngroups_k;
+      ok0 = cur.n0 + 2 * c < cur.n_rows;
+      ok1 = cur.n0 + 2 * c + 1 < cur.n_rows;
+      if (OFFS) xs0 = xsum + (cur.row0 + (ok0 ? cur.n0 + 2 * c : 0)) * (long long)ngroups_k;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = gq + (i >= 2 ? 8 : 0);
-        const int n = n0 + 2 * c + (i & 1);
-        if (n < n_rows) {
-          float v = tg[i];
-          if (GLU) v = (ACT == kModeSwiGLU ? act_silu(v) : act_gelu(v)) * tu[i];
-          p.out[(row0 + n) * p.ldo + o0 + m] = __float2bfloat16_rn(v);
+      for (int i = 0; i < 4; ++i) { tA[i] = 0.f; tB[i] = 0.f; }
+    }
+    refill();
+    // Operands that do not come through the ring are loaded before the wait so
+    // that their latency overlaps it: activations and scales of the slab's two
+    // 128-groups (the second absent when K % 256 == 128 on the last slab).
+    const int kg0 = c_slab * 2;
+    const bool two = kg0 + 1 < ngroups_k;
+    uint4 xv[2][4];
+    float sc[4][2];
+    float xsv[2][2];
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const bool on = tok_ok && (gi == 0 || two);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        xv[gi][q] = on ? *reinterpret_cast<const uint4*>(xrow + (kg0 + gi) * 128 + 8 * q) : make_uint4(0, 0, 0, 0);
+    }
+    {
+      const __nv_bfloat16* sp[4] = {sA + kg0, sA + s8 + kg0, sB + kg0, sB + s8 + kg0};
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        if ((ngroups_k & 1) == 0) {
+          const uint32_t w2 = *reinterpret_cast<const uint32_t*>(sp[rr]);
+          sc[rr][0] = bf16lo(w2);
+          sc[rr][1] = bf16hi(w2);
+        } else {
+          sc[rr][0] = __bfloat162float(sp[rr][0]);
+          sc[rr][1] = two ? __bfloat162float(sp[rr][1]) : 0.f;
         }
       }
     }
+    if (OFFS) {
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const bool on = gi == 0 || two;
+        xsv[gi][0] = (ok0 && on) ? xs0[kg0 + gi] : 0.f;
+        xsv[gi][1] = (ok1 && on) ? xs0[ngroups_k + kg0 + gi] : 0.f;
+      }
+    }
+    if (!mbar_wait(&s_bar[warp][c_st], c_phase, wait_limit_ns, &s_abort[warp], 0x0201)) break;
+    const uint8_t* slabp = ring + c_st * kI4SlabBytes;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      if (gi == 1 && !two) break;  // the slab's second half is TMA zero fill
+      const uint4 a0 = *reinterpret_cast<const uint4*>(slabp + gq * 128 + gi * 64 + c * 16);
+      const uint4 a1 = *reinterpret_cast<const uint4*>(slabp + (gq + 8) * 128 + gi * 64 + c * 16);
+      const uint4 b0 = *reinterpret_cast<const uint4*>(slabp + (gq + 16) * 128 + gi * 64 + c * 16);
+      const uint4 b1 = *reinterpret_cast<const uint4*>(slabp + (gq + 24) * 128 + gi * 64 + c * 16);
+      float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (OFFS) {
+        mma_group_offset(pa, a0, a1, xv[gi]);
+        mma_group_offset(pb, b0, b1, xv[gi]);
+        // D columns are tokens n0 + 2c and n0 + 2c + 1: remove 136 * (their group sums)
+        const float x0 = xsv[gi][0], x1 = xsv[gi][1];
+        pa[0] = fmaf(-136.f, x0, pa[0]); pa[1] = fmaf(-136.f, x1, pa[1]);
+        pa[2] = fmaf(-136.f, x0, pa[2]); pa[3] = fmaf(-136.f, x1, pa[3]);
+        pb[0] = fmaf(-136.f, x0, pb[0]); pb[1] = fmaf(-136.f, x1, pb[1]);
+        pb[2] = fmaf(-136.f, x0, pb[2]); pb[3] = fmaf(-136.f, x1, pb[3]);
+      } else {
+        mma_group(pa, a0, a1, xv[gi]);
+        mma_group(pb, b0, b1, xv[gi]);
+      }
+      tA[0] = fmaf(pa[0], sc[0][gi], tA[0]); tA[1] = fmaf(pa[1], sc[0][gi], tA[1]);
+      tA[2] = fmaf(pa[2], sc[1][gi], tA[2]); tA[3] = fmaf(pa[3], sc[1][gi], tA[3]);
+      tB[0] = fmaf(pb[0], sc[2][gi], tB[0]); tB[1] = fmaf(pb[1], sc[2][gi], tB[1]);
+      tB[2] = fmaf(pb[2], sc[3][gi], tB[2]); tB[3] = fmaf(pb[3], sc[3][gi], tB[3]);
+    }
+    __syncwarp();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slab reads done before TMA reuses it
+    ++consumed;
+    if (++c_st == kI4Stages) { c_st = 0; c_phase ^= 1u; }
+    refill();
+    if (c_slab == nslab - 1) {
+      // D fragments: (m = gq, n = 2c, 2c+1) in [0],[1]; (m = gq + 8, same n) in [2],[3]
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = gq + (i >= 2 ? 8 : 0);
+        const int n = cur.n0 + 2 * c + (i & 1);
+        if (n < cur.n_rows) {
+          __nv_bfloat16* orow = p.out + (cur.row0 + n) * p.ldo + cur.o0;
+          if (GLU) {
+            const float a = ACT == kModeSwiGLU ? act_silu(tA[i]) : act_gelu(tA[i]);
+            orow[m] = __float2bfloat16_rn(a * tB[i]);
+          } else {
+            orow[m] = __float2bfloat16_rn(tA[i]);
+            orow[m + 16] = __float2bfloat16_rn(tB[i]);
+          }
+        }
+      }
+    }
+    if (++c_slab == nslab) { c_slab = 0; c_task += tstride; }
   }
+  // never leave the CTA with copies still landing in its shared memory
+  {
+    volatile int dummy = 0;
+    for (int i = consumed; i < issued; ++i)
+      mbar_wait(&s_bar[warp][i % kI4Stages], (uint32_t)((i / kI4Stages) & 1), wait_limit_ns, &dummy, 0x0202);
+  }
+  __syncwarp();
 }
 
 }  // namespace moe

@@ -18,6 +18,8 @@ namespace moe {
 
 static std::atomic<unsigned long long> g_launches{0};
 static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+// CTA-pair expert GEMMs (on by default; moe_set_pair_gemm(0) selects the single-CTA kernel everywhere).
+static std::atomic<int> g_pair_gemm{1};
 
 static inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -97,7 +99,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, wsplit, wmax, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+  size_t part, wsplit, wnorm, xsum, xq, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
 };
 
 static Workspace ws_layout(const moe_shape* s) {
@@ -110,7 +112,11 @@ static Workspace ws_layout(const moe_shape* s) {
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   L.part = take((size_t)ns * s->T * s->E * 4);
   L.wsplit = take((size_t)3 * s->E * s->d * 2);
-  L.wmax = take(16);
+  L.wnorm = take((size_t)s->E * 4);
+  const long long xs_rows = std::max<long long>(grouped_rows(s), s->T);
+  const int xs_cols = std::max(s->d, std::max(s->H, s->H_s));
+  L.xsum = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * (xs_cols / 128) * 4 : 16);
+  L.xq = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * xs_cols * 2 : 16);
   L.cnt = take((size_t)nchunks * s->E * 4);
   L.psum = take((size_t)nchunks * s->E * 4);
   L.idx = take((size_t)s->T * s->k * 4);
@@ -165,25 +171,49 @@ static int make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t
   return r == CUDA_SUCCESS ? MOE_OK : MOE_CUDA_ERROR;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int CG>
 static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, long long ub_mtiles,
                          cudaStream_t st) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, CG>;
   constexpr int OUTN = (MODE == kModeSwiGLU || MODE == kModeGeGLU) ? BN / 2 : BN;
   // the shared-memory opt-in is set once per device for each instantiation
   static std::atomic<unsigned long long> done_mask{0};
   const int dev = current_device();
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(done_mask.load(std::memory_order_relaxed) & bit)) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    MOE_CUDA_TRY(cudaFuncSetAttribute(k_grouped_gemm<MODE, BN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)Cfg::kSmemBytes));
     done_mask.fetch_or(bit);
   }
   const long long tiles = ub_mtiles * cdiv(p.N, OUTN);
-  const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
-  k_grouped_gemm<MODE, BN><<<grid, 256, Cfg::kSmemBytes, st>>>(ta, tb, p);
+  if (CG == 1) {
+    const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
+    k_grouped_gemm<MODE, BN, 1><<<grid, 256, Cfg::kSmemBytes, st>>>(ta, tb, p);
+  } else {
+    // clusters of 2 CTAs, one pair per two SMs
+    const int pairs = (int)std::max<long long>(1, std::min<long long>(num_sms() / 2, tiles));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_grouped_gemm<MODE, BN, CG>, ta, tb, p));
+  }
   MOE_LAUNCH_CHECK();
   return MOE_OK;
+}
+
+// CTA pairs (M = 256 tiles) for the bf16 expert GEMMs when the groups are large enough
+// to fill them: on average at least 192 rows per group.
+static bool use_pair_gemm(int mode, int BN, long long R, int n_groups) {
+  return mode != kModeF32 && BN == 256 && R >= 192ll * n_groups && g_pair_gemm.load();
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
@@ -209,8 +239,10 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   if (R == 0) return MOE_OK;
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
-  const int BN = pick_bn(glu, N, ub_m);
-  const int box_rows = glu ? BN / 2 : BN;
+  // router logits: one column tile as wide as the expert count (fewer A re-reads)
+  const int BN = mode == kModeF32 ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
+  const bool pair = use_pair_gemm(mode, BN, R, n_groups);
+  const int box_rows = (glu || pair) ? BN / 2 : BN;
   CUtensorMap ta, tb;
   cuuint64_t da[2] = {(cuuint64_t)(a_kwrap > 0 ? a_kwrap : K), (cuuint64_t)R};
   cuuint64_t db[3] = {(cuuint64_t)K, (cuuint64_t)b_rows, (cuuint64_t)n_groups};
@@ -233,31 +265,67 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.out_f32 = reinterpret_cast<float*>(out);
   p.bias = bias;
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
+  if (pair) {
+    const long long ub2 = grows ? (R / (2 * kBM) + n_groups) : cdiv(R, 2 * kBM);
+    if (mode == kModePlain) return launch_gemm_t<kModePlain, 256, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeSwiGLU) return launch_gemm_t<kModeSwiGLU, 256, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeGeGLU) return launch_gemm_t<kModeGeGLU, 256, 2>(ta, tb, p, ub2, st);
+    return MOE_UNSUPPORTED_SHAPE;
+  }
 #define MOE_GEMM_CASE(M_, BN_) \
-  if (mode == M_ && BN == BN_) return launch_gemm_t<M_, BN_>(ta, tb, p, ub, st);
+  if (mode == M_ && BN == BN_) return launch_gemm_t<M_, BN_, 1>(ta, tb, p, ub, st);
   MOE_GEMM_CASE(kModePlain, 256) MOE_GEMM_CASE(kModePlain, 128) MOE_GEMM_CASE(kModePlain, 64)
   MOE_GEMM_CASE(kModeSwiGLU, 256) MOE_GEMM_CASE(kModeSwiGLU, 128) MOE_GEMM_CASE(kModeSwiGLU, 64)
   MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
-  MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 128) MOE_GEMM_CASE(kModeF32, 64)
+  MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 192) MOE_GEMM_CASE(kModeF32, 128)
+  MOE_GEMM_CASE(kModeF32, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
 
 // ------------------------------------------------------------------ launch helpers
 
+// Selection kernel.  Large batches: one CTA of 8 warps per 32-token chunk, chunk tables formed in the kernel.
+// Small batches (T <= 2048): 4 tokens per CTA so the tokens spread over the SMs; the probabilities are written
+// to p_scratch (which may be `part` itself: each warp writes its row after reading it) and k_chunk_stats forms
+// the chunk tables.
 static int launch_topk(const moe_shape* s, const float* part, int nsplit, const float* bias, float* logits,
-                       int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st,
+                       int32_t* idx, float* w, int32_t* cnt, float* psum, float* p_scratch, cudaStream_t st,
                        RefineArgs refine = RefineArgs{nullptr, nullptr, nullptr, nullptr, 0, 0.f}) {
   const int nchunks = (int)cdiv(s->T, kChunk);
   const int epl = (int)cdiv(s->E, 32);
-#define MOE_TOPK_CASE(N_)                                                                                         \
-  if (epl <= N_) {                                                                                                \
-    k_router_topk<N_><<<nchunks, 256, 0, st>>>(part, nsplit, bias, logits, idx, w, cnt, psum, (int)s->T, s->E,   \
-                                               s->k, s->renorm, refine);                                          \
+  const bool small = s->T <= 2048;
+  // the certifying recompute holds the token's inputs in registers when d <= 1024
+  const bool xreg = refine.x != nullptr && refine.d <= 1024;
+#define MOE_TOPK_CASE(N_, NW_, XR_, ST_)                                                                          \
+  if (epl <= N_ && (small ? 4 : 8) == NW_ && xreg == XR_) {                                                       \
+    const size_t smem = ST_ ? (size_t)2 * NW_ * s->E * sizeof(float) : 0;                                         \
+    if (smem > 48 * 1024) {                                                                                       \
+      static int attr_done[64] = {0};                                                                             \
+      const int dev = current_device();                                                                           \
+      if (dev < 64 && !attr_done[dev]) {                                                                          \
+        MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_topk<N_, NW_, XR_, ST_>,                                       \
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,                           \
+                                          2 * NW_ * kMaxRouterE * (int)sizeof(float)));                           \
+        attr_done[dev] = 1;                                                                                       \
+      }                                                                                                           \
+    }                                                                                                             \
+    const unsigned grid = ST_ ? (unsigned)nchunks : (unsigned)cdiv(s->T, NW_);                                    \
+    k_router_topk<N_, NW_, XR_, ST_><<<grid, NW_ * 32, smem, st>>>(part, nsplit, bias, logits, idx, w, cnt, psum,  \
+                                                                   p_scratch, (int)s->T, s->E, s->k, s->renorm,  \
+                                                                   refine);                                       \
     MOE_LAUNCH_CHECK();                                                                                           \
+    if (!ST_) {                                                                                                   \
+      k_chunk_stats<<<nchunks, 256, 0, st>>>(idx, p_scratch, cnt, psum, (int)s->T, s->E, s->k);                   \
+      MOE_LAUNCH_CHECK();                                                                                         \
+    }                                                                                                             \
     return MOE_OK;                                                                                                \
   }
-  MOE_TOPK_CASE(1) MOE_TOPK_CASE(2) MOE_TOPK_CASE(4) MOE_TOPK_CASE(8) MOE_TOPK_CASE(16)
+#define MOE_TOPK_EPL(NW_, XR_, ST_)                                                                               \
+  MOE_TOPK_CASE(1, NW_, XR_, ST_) MOE_TOPK_CASE(2, NW_, XR_, ST_) MOE_TOPK_CASE(4, NW_, XR_, ST_)                 \
+  MOE_TOPK_CASE(8, NW_, XR_, ST_) MOE_TOPK_CASE(16, NW_, XR_, ST_)
+  MOE_TOPK_EPL(8, false, true) MOE_TOPK_EPL(8, true, true) MOE_TOPK_EPL(4, false, false) MOE_TOPK_EPL(4, true, false)
+#undef MOE_TOPK_EPL
 #undef MOE_TOPK_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -272,18 +340,21 @@ static int launch_scan(const moe_shape* s, int32_t* cnt, const float* psum, int3
 
 static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx, const int32_t* cbase,
                           const int32_t* counts, int32_t* slot, uint8_t* drop, int32_t* row_src, void* x_perm,
-                          int32_t* kept, int32_t* offs, cudaStream_t st) {
+                          int32_t* kept, int32_t* offs, cudaStream_t st, bool move_rows = true) {
   const int nchunks = (int)cdiv(s->T, kChunk);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(x_perm);
   const unsigned mv_blocks = (unsigned)cdiv(s->T * (long long)(s->d / 8), 256);
 #define MOE_SCATTER_CASE(N_)                                                                                  \
   if (s->k <= N_) {                                                                                           \
-    k_scatter<N_><<<nchunks, 128, 0, st>>>(xb, idx, cbase, counts, (int)s->T, s->d, s->E, s->k, s->capacity, \
+    k_scatter<N_><<<(unsigned)cdiv(nchunks, 4), 128, 0, st>>>(xb, idx, cbase, counts, (int)s->T, s->d, s->E,   \
+                                                              s->k, s->capacity,                              \
                                            slot, drop, row_src, xp, kept, offs);                              \
     MOE_LAUNCH_CHECK();                                                                                       \
-    k_move_rows<N_><<<mv_blocks, 256, 0, st>>>(xb, slot, (int)s->T, s->d, s->k, xp);                         \
-    MOE_LAUNCH_CHECK();                                                                                       \
+    if (move_rows) {                                                                                          \
+      k_move_rows<N_><<<mv_blocks, 256, 0, st>>>(xb, slot, (int)s->T, s->d, s->k, xp);                       \
+      MOE_LAUNCH_CHECK();                                                                                     \
+    }                                                                                                         \
     return MOE_OK;                                                                                            \
   }
   MOE_SCATTER_CASE(2) MOE_SCATTER_CASE(4) MOE_SCATTER_CASE(8) MOE_SCATTER_CASE(16)
@@ -291,9 +362,17 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   return MOE_UNSUPPORTED_SHAPE;
 }
 
+// Optional scratch for the offset-code kernel: xsum [R, K/128] fp32 (activation group sums) and
+// xq [R, K] bf16 (the fragment-ordered copy of A).  Without it the plain-code kernel runs.
+struct Int4Scratch {
+  float* xsum;
+  void* xq;
+};
+
 static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const void* wq, const void* wsc,
                      int n_groups, int b_rows, int up_row0, int N, const int32_t* gstart, const int32_t* grows,
-                     void* out, cudaStream_t st) {
+                     void* out, cudaStream_t st, Int4Scratch scr = Int4Scratch{nullptr, nullptr}) {
+  float* xsum = scr.xq != nullptr ? scr.xsum : nullptr;
   if (R == 0) return MOE_OK;
   Int4Params p;
   p.wq = reinterpret_cast<const uint8_t*>(wq);
@@ -309,24 +388,72 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
   p.up_row0 = up_row0;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ldo = N;
-  const long long ub_tasks = (long long)(N / 16) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8));
-  const int grid = (int)std::max<long long>(1, std::min<long long>(2ll * num_sms(), cdiv(ub_tasks, 8)));
-  if (!glu) k_int4_gemm<false, kModePlain><<<grid, 256, 0, st>>>(p);
-  else if (act == MOE_ACT_SWIGLU) k_int4_gemm<true, kModeSwiGLU><<<grid, 256, 0, st>>>(p);
-  else k_int4_gemm<true, kModeGeGLU><<<grid, 256, 0, st>>>(p);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  {
+    // 2-D byte map over all experts' packed rows; box = 16 rows x 128 bytes (256 inputs)
+    EncodeTiledFn enc = get_encoder();
+    if (!enc) return MOE_CUDA_ERROR;
+    CUtensorMap tm;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)n_groups * (cuuint64_t)b_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128, 16};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(wq), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MOE_CUDA_ERROR;
+    const int dev = current_device();
+    const unsigned long long bit = 1ull << (dev & 63);
+    static std::atomic<unsigned long long> done{0};
+    if (!(done.load() & bit)) {
+#define MOE_I4_ATTR(G_, A_, O_)                                                                          \
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_stream<G_, A_, O_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                        kI4Smem));
+      MOE_I4_ATTR(false, kModePlain, false) MOE_I4_ATTR(true, kModeSwiGLU, false) MOE_I4_ATTR(true, kModeGeGLU, false)
+      MOE_I4_ATTR(false, kModePlain, true) MOE_I4_ATTR(true, kModeSwiGLU, true) MOE_I4_ATTR(true, kModeGeGLU, true)
+#undef MOE_I4_ATTR
+      done.fetch_or(bit);
+    }
+    if (xsum != nullptr) {
+      k_int4_act_prep<<<(unsigned)cdiv(R * (K / 8), 256), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(A), R,
+                                                                         K, xsum,
+                                                                         reinterpret_cast<__nv_bfloat16*>(scr.xq));
+      MOE_LAUNCH_CHECK();
+      p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);
+    }
+    const long long rows_per_task = glu ? 16 : 32;
+    const long long ub = (long long)(N / rows_per_task) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8));
+    const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), cdiv(ub, kI4Warps)));
+    const unsigned long long lim = g_wait_limit_ns.load();
+    const int nt = kI4Warps * 32;
+#define MOE_I4_LAUNCH(G_, A_, O_) k_int4_stream<G_, A_, O_><<<grid, nt, kI4Smem, st>>>(tm, p, lim, xsum)
+    if (xsum != nullptr) {
+      if (!glu) MOE_I4_LAUNCH(false, kModePlain, true);
+      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true);
+      else MOE_I4_LAUNCH(true, kModeGeGLU, true);
+    } else {
+      if (!glu) MOE_I4_LAUNCH(false, kModePlain, false);
+      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, false);
+      else MOE_I4_LAUNCH(true, kModeGeGLU, false);
+    }
+#undef MOE_I4_LAUNCH
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+  }
 }
 
 // Gated expert FFN over groups of rows: h = act(A W1^T) * (A W3^T), y = h W2^T.
+// scr (optional, INT4 only): scratch of at least R * max(d, hidden) / 128 floats (group sums) and
+// R * max(d, hidden) bf16 (fragment-ordered activations).
 static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const void* A, const int32_t* gstart,
                            const int32_t* grows, int n_groups, const void* w13, const void* s13, const void* w2,
-                           const void* s2, void* h, void* y, cudaStream_t st) {
+                           const void* s2, void* h, void* y, cudaStream_t st,
+                           Int4Scratch scr = Int4Scratch{nullptr, nullptr}) {
   int rc;
   if (s->wfmt == MOE_WFMT_INT4_G128) {
-    rc = int4_gemm(true, s->act, A, R, s->d, w13, s13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st);
+    rc = int4_gemm(true, s->act, A, R, s->d, w13, s13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st,
+                   scr);
     if (rc) return rc;
-    return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
+    return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st, scr);
   }
   const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
   rc = grouped_gemm(mode, A, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st);
@@ -336,7 +463,8 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
 
 // Fused CUDA-core router when W_r^T fits in shared memory: returns its experts-per-lane template, else 0.
 static int fused_router_epl(const moe_shape* s) {
-  const int epl = s->E <= 32 ? 1 : s->E <= 64 ? 2 : s->E <= 128 ? 4 : s->E <= 256 ? 8 : 16;
+  if (s->E > 256) return 0;
+  const int epl = s->E <= 32 ? 1 : s->E <= 64 ? 2 : s->E <= 128 ? 4 : 8;
   const size_t bytes = (size_t)s->d * (epl * 32 + 1) * 4;
   return bytes <= 160 * 1024 ? epl : 0;
 }
@@ -352,22 +480,27 @@ static int launch_fused_router(const moe_shape* s, int epl, const void* x, const
   if (epl == N_) {                                                                                                \
     static std::atomic<unsigned long long> done{0};                                                               \
     if (!(done.load() & bit)) {                                                                                   \
-      MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_fused<N_>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_fused<N_, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
                                         160 * 1024));                                                             \
       done.fetch_or(bit);                                                                                         \
     }                                                                                                             \
-    k_router_fused<N_><<<nchunks, 256, smem, st>>>(xb, w_router, bias, logits, idx, w, cnt, psum, (int)s->T, s->d, \
-                                                   s->E, s->k, s->renorm);                                        \
+    k_router_fused<N_, 8><<<nchunks, 256, smem, st>>>(xb, w_router, bias, logits, idx, w, cnt, psum, (int)s->T,    \
+                                                      s->d, s->E, s->k, s->renorm);                               \
     MOE_LAUNCH_CHECK();                                                                                           \
     return MOE_OK;                                                                                                \
   }
-  MOE_FUSED_CASE(1) MOE_FUSED_CASE(2) MOE_FUSED_CASE(4) MOE_FUSED_CASE(8) MOE_FUSED_CASE(16)
+  MOE_FUSED_CASE(1) MOE_FUSED_CASE(2) MOE_FUSED_CASE(4) MOE_FUSED_CASE(8)
 #undef MOE_FUSED_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
 
 // Large routers go to the tensor cores as an exact three-way bf16 split of W_r
 // (fp32 accumulation); small ones stay on the fp32 CUDA-core GEMM.
+// Decode router: dynamic shared memory of the staged x slice (16 tokens x one input slice, fp32).
+static constexpr size_t kSkinnyMaxSmem = 100 * 1024;
+static int g_skinny_attr[64] = {0};
+static size_t skinny_smem(int d) { return (size_t)kSkTok * skinny_slice(d) * sizeof(float); }
+
 static bool use_tc_router(const moe_shape* s) {
   return s->E % 16 == 0 && s->d % 64 == 0 && (double)s->T * s->E * s->d >= (double)(1ll << 28);
 }
@@ -388,24 +521,27 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     rc = launch_fused_router(s, epl_fused, x, w_router, bias, logits, idx, w, cnt, psum, st);
   } else if (logits_in == nullptr && use_tc_router(s)) {
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
-    const long long n = (long long)s->E * s->d;
-    k_router_split<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(w_router, wsplit, s->E, s->d);
-    MOE_LAUNCH_CHECK();
-    float* wmax = reinterpret_cast<float*>(ws + L.wmax);
-    k_router_wmax<<<1, 256, 0, st>>>(w_router, wmax, s->E, s->d);
+    float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
+    k_router_prep<<<(unsigned)cdiv(s->E, 8), 256, 0, st>>>(w_router, wsplit, wnorm, s->E, s->d);
     MOE_LAUNCH_CHECK();
     rc = grouped_gemm(kModeF32, x, s->T, 3 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
                       bias);
     if (rc) return rc;
     // screening bound: fp32 accumulation of 3d products (any rounding direction) plus the bias add
-    RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wmax, s->d,
+    RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d,
                    (float)((3.0 * s->d + 2.0) * std::ldexp(1.0, -23) * (1.0 + std::ldexp(1.0, -7)))};
-    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, st, ref);
-  } else if (logits_in == nullptr && s->T <= 256) {
-    k_router_skinny<32><<<(unsigned)cdiv(s->E, 2), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router,
-                                                                 part, (int)s->T, s->d, s->E);
+    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
+  } else if (logits_in == nullptr && s->T <= 256 && skinny_smem(s->d) <= kSkinnyMaxSmem) {
+    const int dev = current_device();
+    if (dev >= 0 && dev < 64 && !g_skinny_attr[dev]) {
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_skinny, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkinnyMaxSmem));
+      g_skinny_attr[dev] = 1;
+    }
+    dim3 grid((unsigned)cdiv(s->E, 8 * kSkExp), (unsigned)cdiv(s->T, kSkTok), kSkSplit);
+    k_router_skinny<<<grid, 256, skinny_smem(s->d), st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, part,
+                                                           (int)s->T, s->d, s->E);
     MOE_LAUNCH_CHECK();
-    rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum, st);
+    rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum, part, st);
   } else if (logits_in == nullptr) {
     int kps = 0;
     nsplit = router_splits(s, &kps);
@@ -413,9 +549,9 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     k_router_logits<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, part, (int)s->T,
                                           s->d, s->E, kps);
     MOE_LAUNCH_CHECK();
-    rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum, st);
+    rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum, part, st);
   } else {
-    rc = launch_topk(s, logits_in, 1, nullptr, nullptr, idx, w, cnt, psum, st);
+    rc = launch_topk(s, logits_in, 1, nullptr, nullptr, idx, w, cnt, psum, part, st);
   }
   if (rc) return rc;
   const bool want_fp = aux_f || aux_p || aux;
@@ -453,6 +589,12 @@ uint64_t moe_launch_count(void) { return g_launches.load(); }
 int moe_set_wait_limit_ns(uint64_t ns) {
   if (ns == 0) return MOE_INVALID_ARGUMENT;
   g_wait_limit_ns.store(ns);
+  return MOE_OK;
+}
+
+int moe_set_pair_gemm(int32_t enable) {
+  if (enable != 0 && enable != 1) return MOE_INVALID_ARGUMENT;
+  g_pair_gemm.store(enable);
   return MOE_OK;
 }
 
@@ -599,13 +741,16 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   if (rc) return rc;
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream);
   if (rc) return rc;
-  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream);
+  const Int4Scratch scr = s->wfmt == MOE_WFMT_INT4_G128
+                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq}
+                              : Int4Scratch{nullptr, nullptr};
+  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
   if (rc) return rc;
   void* ys = nullptr;
   if (s->H_s > 0) {
     ys = ws + L.ys;
     rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
-                         stream);
+                         stream, scr);
     if (rc) return rc;
   }
   return moe_combine(s, yperm, slot, w, ys, out, stream);
@@ -671,7 +816,7 @@ extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
 
 namespace moe {
 
-constexpr long long kNoAllocHistInts = 262144;  // ceil(T / 128) * E must not exceed this
+constexpr long long kNoAllocHistInts = 262144;  // ceil(T / 32) * E must not exceed this
 constexpr int kNoAllocCountInts = kMaxE;
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocHistInts + kNoAllocCountInts];

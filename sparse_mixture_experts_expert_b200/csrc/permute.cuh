@@ -54,7 +54,13 @@ __device__ __forceinline__ void group_offsets(const int32_t* __restrict__ counts
   __syncthreads();
 }
 
-// One CTA (128 threads, one token per thread) per chunk of 128 tokens.
+// One CTA = 128 threads = four chunks of 32 tokens, one warp per chunk.
+// rank = (tokens of earlier chunks that chose e, from the per-chunk prefix
+// table) + (earlier tokens of the chunk that chose e).  The in-chunk part
+// walks the chunk's (token, slot) pairs in order, 32 / kp tokens per step
+// (kp = k rounded up to a power of two, lane = token * kp + slot): lanes with
+// the same expert find each other with match.any, take consecutive ranks from
+// a per-warp shared counter, and the last of them advances the counter.
 template <int KMAX>
 __global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict__ x,
                                                  const int32_t* __restrict__ topk_idx,
@@ -65,91 +71,65 @@ __global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict
                                                  int32_t* __restrict__ offsets_out) {
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_kept[kMaxE];
-  __shared__ int s_base[kMaxE];
-  __shared__ int s_wcnt[4][kMaxE];
   __shared__ int s_tmp[4];
+  __shared__ int s_cnt[4][kMaxE];
+  __shared__ int s_ix[4][kChunk * KMAX];
+  __shared__ int s_rk[4][kChunk * KMAX];
   const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-  const int chunk = blockIdx.x;
+  const int chunk = blockIdx.x * 4 + warp;
+  const int nchunks = (T + kChunk - 1) / kChunk;
 
   group_offsets(counts, E, cap, s_off, s_kept, s_tmp);
-  if (chunk == 0) {
+  if (blockIdx.x == 0) {
     for (int e = tid; e < E; e += 128) {
       if (kept_out) kept_out[e] = s_kept[e];
       if (offsets_out) offsets_out[e] = s_off[e];
     }
     if (tid == 0 && offsets_out) offsets_out[E] = s_off[E];
   }
-  for (int e = tid; e < E; e += 128) {
-    s_base[e] = cbase[(size_t)chunk * E + e];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) s_wcnt[w][e] = 0;
-  }
-  __syncthreads();
+  if (chunk >= nchunks) return;
 
-  const int t = chunk * kChunk + tid;
-  const bool valid = t < T;
-  int ex[KMAX], rk[KMAX];
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    ex[j] = (valid && j < k) ? topk_idx[(size_t)t * k + j] : -1;
-    rk[j] = 0;
-  }
-  unsigned pending = valid ? ((1u << k) - 1u) : 0u;
+  const int t0 = chunk * kChunk;
+  const int ntok = min(kChunk, T - t0);
+  int* ix = s_ix[warp];
+  int* rk = s_rk[warp];
+  int* cnt = s_cnt[warp];
+  for (int q = lane; q < ntok * k; q += 32) ix[q] = topk_idx[(size_t)t0 * k + q];
+  __syncwarp();
+  for (int q = lane; q < ntok * k; q += 32) cnt[ix[q]] = 0;
+  __syncwarp();
+  const int kp = k == 1 ? 1 : 1 << (32 - __clz(k - 1));
+  const int lg = 31 - __clz(kp);
   const unsigned lt = (1u << lane) - 1u;
-  // In-warp ranks: one ballot per distinct expert present in the warp.
-  while (true) {
-    const unsigned active = __ballot_sync(0xffffffffu, pending != 0u);
-    if (active == 0u) break;
-    const int leader = __ffs(active) - 1;
-    int mykey = -1;
-    if (pending) {
-      const int jj = __ffs(pending) - 1;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j == jj) mykey = ex[j];
+  for (int tb = 0; tb < ntok; tb += 32 / kp) {
+    const int tt = tb + (lane >> lg), j = lane & (kp - 1);
+    const bool on = j < k && tt < ntok;
+    const int e = on ? ix[tt * k + j] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int base = on ? cnt[e] : 0;
+    __syncwarp();
+    if (on) {
+      rk[tt * k + j] = base + __popc(peers & lt);
+      if (lane == 31 - __clz(peers)) cnt[e] = base + __popc(peers);
     }
-    const int key = __shfl_sync(0xffffffffu, mykey, leader);
-    int myslot = -1;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-      if (((pending >> j) & 1u) && ex[j] == key) myslot = j;
-    const unsigned mask = __ballot_sync(0xffffffffu, myslot >= 0);
-    if (myslot >= 0) {
-      const int r = __popc(mask & lt);
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j == myslot) rk[j] = r;
-      pending &= ~(1u << myslot);
-    }
-    if (lane == leader) s_wcnt[warp][key] = __popc(mask);
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += 128) {
-    int run = 0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int v = s_wcnt[w][e];
-      s_wcnt[w][e] = run;
-      run += v;
-    }
-  }
-  __syncthreads();
-
-  int pos[KMAX];
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    pos[j] = -1;
-    if (valid && j < k) {
-      const int e = ex[j];
-      const int rank = s_base[e] + s_wcnt[warp][e] + rk[j];
-      const bool dropped = cap > 0 && rank >= cap;
-      pos[j] = dropped ? -1 : s_off[e] + rank;
-      slot_pos[(size_t)t * k + j] = pos[j];
-      if (drop) drop[(size_t)t * k + j] = dropped ? 1 : 0;
-      if (!dropped && row_src) row_src[pos[j]] = t * k + j;
-    }
+    __syncwarp();
   }
 
+  if (lane < ntok) {
+    const int t = t0 + lane;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j < k) {
+        const int e = ix[lane * k + j];
+        const int rank = cbase[(size_t)e * nchunks + chunk] + rk[lane * k + j];
+        const bool dropped = cap > 0 && rank >= cap;
+        const int pos = dropped ? -1 : s_off[e] + rank;
+        slot_pos[(size_t)t * k + j] = pos;
+        if (drop) drop[(size_t)t * k + j] = dropped ? 1 : 0;
+        if (!dropped && row_src) row_src[pos] = t * k + j;
+      }
+    }
+  }
 }
 
 // Row moves: one thread per (token, 16-byte column slice); it copies the slice

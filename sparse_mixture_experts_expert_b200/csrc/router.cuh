@@ -11,9 +11,14 @@
 
 #include "common.cuh"
 
+#include <cooperative_groups.h>
+
 namespace moe {
 
-constexpr int kChunk = 128;  // tokens per router / permute chunk (one CTA)
+namespace cg = cooperative_groups;
+
+constexpr int kChunk = 32;         // tokens per router / grouping chunk (one warp)
+constexpr int kMaxRouterE = 512;   // experts the routers handle
 
 // ---------------------------------------------------------------------------
 // logits_part[split][T][E] = sum over this split's K range of x[t,i] * W_r[e,i]
@@ -104,46 +109,33 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 }
 
 // ---------------------------------------------------------------------------
-// Exact three-way bf16 split of the fp32 router weight: W = hi + mid + lo with
-// each part a bf16 value (24 significand bits = 3 x 8), written as one
-// [E, 3d] bf16 operand [hi | mid | lo].  x is bf16, so every product x * part
-// is exact in fp32 and x W^T = [x | x | x] [hi | mid | lo]^T.
-__global__ void __launch_bounds__(256) k_router_split(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
-                                                      int E, int d) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)E * d) return;
-  const long long e = i / d, k = i - e * d;
-  const float w = W[i];
-  const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-  const float r1 = w - __bfloat162float(hi);
-  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(mid);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-  __nv_bfloat16* row = Ws + e * 3 * d;
-  row[k] = hi;
-  row[d + k] = mid;
-  row[2 * d + k] = lo;
-}
-
-// wmax[0] = max_e ||W_r[e]||_2 (one CTA, fixed order).
-__global__ void __launch_bounds__(256) k_router_wmax(const float* __restrict__ W, float* __restrict__ wmax, int E,
-                                                     int d) {
-  __shared__ float s_m[8];
-  float m = 0.f;
-  for (int e = warp_id(); e < E; e += 8) {
-    float ss = 0.f;
-    for (int i = lane_id(); i < d; i += 32) ss = fmaf(W[(size_t)e * d + i], W[(size_t)e * d + i], ss);
+// Router weight preparation for the tensor-core screening pass, one warp per
+// expert row:
+//  * exact three-way bf16 split W = hi + mid + lo (24 significand bits = 3 x 8),
+//    written as one [E, 3d] bf16 operand [hi | mid | lo]; x is bf16, so every
+//    product x * part is exact in fp32 and x W^T = [x | x | x] [hi | mid | lo]^T;
+//  * the row norm ||W_r[e]||_2 for the screening error bound.
+__global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
+                                                     float* __restrict__ wnorm, int E, int d) {
+  const int e = blockIdx.x * 8 + warp_id();
+  if (e >= E) return;
+  const float* wr = W + (size_t)e * d;
+  __nv_bfloat16* row = Ws + (size_t)e * 3 * d;
+  float ss = 0.f;
+  for (int k = lane_id(); k < d; k += 32) {
+    const float w = wr[k];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    row[k] = hi;
+    row[d + k] = mid;
+    row[2 * d + k] = __float2bfloat16_rn(r2);
+    ss = fmaf(w, w, ss);
+  }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    m = fmaxf(m, sqrtf(ss));
-  }
-  if (lane_id() == 0) s_m[warp_id()] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float r = s_m[0];
-    for (int w = 1; w < 8; ++w) r = fmaxf(r, s_m[w]);
-    *wmax = r;
-  }
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane_id() == 0) wnorm[e] = sqrtf(ss);
 }
 
 // ---------------------------------------------------------------------------
@@ -158,34 +150,11 @@ __device__ __forceinline__ void warp_argmax(float& bv, int& bi) {
   }
 }
 
-// Exact fp32 logits of up to 8 experts for one token, computed by the whole
-// warp: lane l accumulates inputs l, l+32, ... with fmaf (one chain per
-// expert), then a fixed xor tree.  The order does not depend on how many
-// experts are batched together.
-__device__ __forceinline__ void warp_dot_multi(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ W,
-                                               int d, const int (&ex)[8], int n, float (&out)[8]) {
-  float acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  for (int i = lane_id(); i < d; i += 32) {
-    const float xv = __bfloat162float(xr[i]);
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (c < n) acc[c] = fmaf(xv, W[(size_t)ex[c] * d + i], acc[c]);
-  }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
-    out[c] = acc[c];
-  }
-}
-
 struct RefineArgs {
   const __nv_bfloat16* x;  // [T, d]; nullptr = logits are final
   const float* W;          // [E, d] fp32 router weight
   const float* bias;       // [E] or nullptr
-  const float* wmax;       // max_e ||W_r[e]||_2 (one float)
+  const float* wnorm;      // [E] ||W_r[e]||_2
   int d;
   float gamma;             // bound factor of the screening logits: |err| <= gamma * ||x_t|| * ||w_e||
 };
@@ -249,160 +218,255 @@ __device__ __forceinline__ void route_token(const float (&z)[EPL], int t, int E,
   }
 }
 
-// Chunk statistics of a CTA of 8 warps, combined in fixed warp order.
-template <int EPL>
-__device__ __forceinline__ void chunk_stats(float (&s_p)[8][EPL * 32], int (&s_c)[8][EPL * 32],
-                                            const float (&pacc)[EPL], const int (&cacc)[EPL], int chunk, int E,
-                                            int32_t* __restrict__ cnt, float* __restrict__ psum) {
-  const int lane = lane_id(), warp = warp_id();
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) { s_p[warp][lane + 32 * i] = pacc[i]; s_c[warp][lane + 32 * i] = cacc[i]; }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float ps = 0.f;
-    int cs = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
-    cnt[(size_t)chunk * E + e] = cs;
-    psum[(size_t)chunk * E + e] = ps;
+// Exact fp32 logit of one (token, expert) pair by the whole warp: lane l takes
+// the 8-input slices l, l+32, ... (16-byte loads of x, 32-byte loads of W),
+// one fmaf chain, then a fixed xor tree.  d % 8 == 0.
+__device__ __forceinline__ float warp_dot(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ wr, int d) {
+  float acc = 0.f;
+  const int nv = d >> 3;
+  for (int v = lane_id(); v < nv; v += 32) {
+    const uint4 u = reinterpret_cast<const uint4*>(xr)[v];
+    const float4 w0 = reinterpret_cast<const float4*>(wr)[2 * v], w1 = reinterpret_cast<const float4*>(wr)[2 * v + 1];
+    acc = fmaf(bf16lo(u.x), w0.x, acc); acc = fmaf(bf16hi(u.x), w0.y, acc);
+    acc = fmaf(bf16lo(u.y), w0.z, acc); acc = fmaf(bf16hi(u.y), w0.w, acc);
+    acc = fmaf(bf16lo(u.z), w1.x, acc); acc = fmaf(bf16hi(u.z), w1.y, acc);
+    acc = fmaf(bf16lo(u.w), w1.z, acc); acc = fmaf(bf16hi(u.w), w1.w, acc);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
 }
 
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...
-//   logits = sum_split part[split] (+ bias); softmax; top-k; gates.
-// With refine.x set, `part` holds screening logits from the tensor cores whose
-// error is at most gamma * ||x_t|| * ||w_e||.  Every expert that could still be
-// in the top k under that bound (screening logit >= k-th largest - 2 bound) is
-// recomputed as a plain fp32 dot product, so the top-k decision is made on
-// fp32 FMA logits; the others are certified out of the top k.
-// Per chunk of kChunk tokens (one CTA, 8 warps x 16 tokens):
-//   cnt[chunk][e]  tokens of the chunk that chose e
-//   psum[chunk][e] sum over the chunk's tokens of p[t,e] (fixed order)
+// Warp argmax on (value desc, index asc) by two warp reductions: the largest
+// value (redux.sync max.f32; NaNs are never chosen, -0.0 == +0.0), then the
+// lowest index among the lanes holding it.
+__device__ __forceinline__ void warp_argmax_redux(float& bv, int& bi) {
+  float m;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(bv));
+  bi = (int)__reduce_min_sync(0xffffffffu, bv == m ? (unsigned)bi : 0xffffffffu);
+  bv = m;
+}
+
+// k rounds of warp argmax over the lanes' logits (lane l holds experts l, l+32, ...):
+// fills sel_v / sel_i (lane j keeps pick j) and returns the k-th largest value.
 template <int EPL>
-__global__ void __launch_bounds__(256) k_router_topk(const float* __restrict__ part, int nsplit,
-                                                     const float* __restrict__ bias, float* __restrict__ logits_out,
-                                                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                                                     int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
-                                                     int E, int k, int renorm, const RefineArgs refine) {
-  __shared__ float s_p[8][EPL * 32];
-  __shared__ int s_c[8][EPL * 32];
+__device__ __forceinline__ float warp_topk(const float (&z)[EPL], int E, int k, float& sel_v, int& sel_i,
+                                           unsigned& taken) {
+  const int lane = lane_id();
+  taken = 0u;
+  float kth = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && z[i] > bv) { bv = z[i]; bi = e; }  // ascending e: first max wins
+    }
+    warp_argmax_redux(bv, bi);
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) { sel_v = bv; sel_i = bi; }
+    kth = bv;
+  }
+  return kth;
+}
+
+// Exact fp32 logit of one (token, expert) pair with the token's inputs held in
+// registers as fp32 (xf[8q + i] = x[8 (lane + 32 q) + i], d <= 1024): the same
+// per-lane order and xor tree as warp_dot, without the bf16 unpacking.
+__device__ __forceinline__ float warp_dot_reg(const float (&xf)[32], const float* __restrict__ wr, int d) {
+  float acc = 0.f;
+  const int nv = d >> 3, lane = lane_id();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int v = lane + 32 * q;
+    if (v < nv) {
+      const float4 w0 = reinterpret_cast<const float4*>(wr)[2 * v], w1 = reinterpret_cast<const float4*>(wr)[2 * v + 1];
+      acc = fmaf(xf[8 * q + 0], w0.x, acc); acc = fmaf(xf[8 * q + 1], w0.y, acc);
+      acc = fmaf(xf[8 * q + 2], w0.z, acc); acc = fmaf(xf[8 * q + 3], w0.w, acc);
+      acc = fmaf(xf[8 * q + 4], w1.x, acc); acc = fmaf(xf[8 * q + 5], w1.y, acc);
+      acc = fmaf(xf[8 * q + 6], w1.z, acc); acc = fmaf(xf[8 * q + 7], w1.w, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+// Router selection, one warp per token: lane l holds the logits of experts l,
+// l+32, ...; a CTA of NW warps is one chunk of kChunk = 32 tokens (32 / NW
+// tokens per warp).
+//   logits = sum_split part[split] (+ bias); top-k (k rounds of warp argmax on
+//   (value desc, index asc)); softmax; gates; chunk statistics.
+// With refine.x set, `part` holds screening logits from the tensor cores whose
+// error is at most gamma * ||x_t|| * max_e ||w_e||.  Every expert whose
+// screening logit is >= (k-th largest - 2 bound) may still be in the top k and
+// is recomputed exactly (warp_dot: a plain fp32 FMA dot product), then the top
+// k is taken again; the others are certified out of the top k.  The softmax
+// uses the exact values where they exist and the screening values elsewhere.
+// Chunk statistics, expert-major: cnt[e][chunk] = picks, psum[e][chunk] = sum
+// over the chunk's tokens of p[t,e].
+//   STATS (large batches; a CTA of NW warps is one chunk of kChunk = 32
+//   tokens, 32 / NW per warp): each warp accumulates its own row of the dynamic
+//   shared memory (2 * NW * E words), then the rows are added in warp order.
+//   !STATS (small batches; NW warps = NW tokens per CTA, so the tokens spread
+//   over the SMs): the probabilities p[t,e] go to p_out and k_chunk_stats
+//   forms the tables.  p_out may alias part: a warp writes row t only after
+//   reading every split of row t.
+template <int EPL, int NW, bool XREG, bool STATS>
+__global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int nsplit,
+                                                         const float* __restrict__ bias, float* __restrict__ logits_out,
+                                                         int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                                         int32_t* __restrict__ cnt, float* __restrict__ psum,
+                                                         float* p_out, int T, int E, int k, int renorm,
+                                                         const RefineArgs refine) {
+  extern __shared__ float s_stat[];
+  constexpr int TPW = STATS ? kChunk / NW : 1;
   const int lane = lane_id(), warp = warp_id();
   const int chunk = blockIdx.x;
-  float pacc[EPL];
-  int cacc[EPL];
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  float* s_p = s_stat + (size_t)warp * E;
+  int* s_c = reinterpret_cast<int*>(s_stat + (size_t)NW * E) + (size_t)warp * E;
+  if (STATS)
+    for (int e = lane; e < E; e += 32) { s_p[e] = 0.f; s_c[e] = 0; }
+  float wmax = 0.f;
+  if (refine.x != nullptr) {
+    for (int e = lane; e < E; e += 32) wmax = fmaxf(wmax, refine.wnorm[e]);
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) { pacc[i] = 0.f; cacc[i] = 0; }
-  float b[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    b[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
   }
-  const float wmax = refine.x != nullptr ? *refine.wmax : 0.f;
-  const int t_first = chunk * kChunk + warp * (kChunk / 8);
-  const int t_end = min(T, t_first + kChunk / 8);
-
-  auto load_z = [&](int t, float (&z)[EPL]) {
+  for (int tt = 0; tt < TPW; ++tt) {
+    const int t = STATS ? chunk * kChunk + warp * TPW + tt : blockIdx.x * NW + warp;
+    if (t >= T) break;
+    float z[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
       float v = -INFINITY;
-      if (e < E && t < t_end) {
+      if (e < E) {
         v = part[(size_t)t * E + e];
-        for (int s = 1; s < nsplit; ++s) v += part[(size_t)s * T * E + (size_t)t * E + e];
-        if (bias != nullptr) v += b[i];
+        for (int sp = 1; sp < nsplit; ++sp) v += part[(size_t)sp * T * E + (size_t)t * E + e];
+        if (bias != nullptr) v += bias[e];
       }
       z[i] = v;
     }
-  };
-
-  float znext[EPL];
-  load_z(t_first, znext);
-  for (int t = t_first; t < t_end; ++t) {
-    float z[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) z[i] = znext[i];
-    load_z(t + 1, znext);  // prefetch the next token's logits
-
+    float sel_v = 0.f;
+    int sel_i = 0;
+    unsigned taken;
+    float kth = warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
     if (refine.x != nullptr) {
-      // k-th largest screening logit
-      unsigned tk = 0u;
-      float kth = -INFINITY;
-      for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          if (e < E && !((tk >> i) & 1u) && (z[i] > bv || (z[i] == bv && e < bi))) { bv = z[i]; bi = e; }
-        }
-        warp_argmax(bv, bi);
-        if ((bi & 31) == lane) tk |= 1u << (bi >> 5);
-        kth = bv;
-      }
       const __nv_bfloat16* xr = refine.x + (size_t)t * refine.d;
       float ss = 0.f;
-      for (int i = lane; i < refine.d; i += 32) {
-        const float v = __bfloat162float(xr[i]);
-        ss = fmaf(v, v, ss);
+      float xf[XREG ? 32 : 1];
+      if constexpr (XREG) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int v = lane + 32 * q;
+          uint4 u = make_uint4(0, 0, 0, 0);
+          if (v < (refine.d >> 3)) u = reinterpret_cast<const uint4*>(xr)[v];
+          xf[8 * q + 0] = bf16lo(u.x); xf[8 * q + 1] = bf16hi(u.x); xf[8 * q + 2] = bf16lo(u.y);
+          xf[8 * q + 3] = bf16hi(u.y); xf[8 * q + 4] = bf16lo(u.z); xf[8 * q + 5] = bf16hi(u.z);
+          xf[8 * q + 6] = bf16lo(u.w); xf[8 * q + 7] = bf16hi(u.w);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(xf[8 * q + j], xf[8 * q + j], ss);
+        }
+      } else {
+        for (int v = lane; v < (refine.d >> 3); v += 32) {
+          const uint4 u = reinterpret_cast<const uint4*>(xr)[v];
+          const float q[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                              bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(q[j], q[j], ss);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float bound = refine.gamma * sqrtf(ss) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
       const float thr = kth - 2.f * bound;
-      // recompute the candidates exactly, up to 8 experts per pass
-      int ex[8];
-      int n = 0;
-      auto flush = [&]() {
-        float v[8];
-        warp_dot_multi(xr, refine.W, refine.d, ex, n, v);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if (c < n) {
-            const int e = ex[c];
-            float zz = v[c];
-            if (refine.bias != nullptr) zz += refine.bias[e];
-            if ((e & 31) == lane) {
-#pragma unroll
-              for (int i = 0; i < EPL; ++i)
-                if (i == (e >> 5)) z[i] = zz;
-            }
-          }
-        }
-        n = 0;
-      };
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && z[i] >= thr);
         while (cand) {
           const int l = __ffs(cand) - 1;
           cand &= cand - 1;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            if (c == n) ex[c] = 32 * i + l;
-          if (++n == 8) flush();
+          const int e = 32 * i + l;
+          float v;
+          if constexpr (XREG) v = warp_dot_reg(xf, refine.W + (size_t)e * refine.d, refine.d);
+          else v = warp_dot(xr, refine.W + (size_t)e * refine.d, refine.d);
+          if (refine.bias != nullptr) v += refine.bias[e];
+          if (lane == l) z[i] = v;
         }
       }
-      if (n > 0) flush();
+      kth = warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
     }
-    route_token<EPL>(z, t, E, k, renorm, logits_out, topk_idx, topk_w, pacc, cacc);
+    if (logits_out != nullptr) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i < E) logits_out[(size_t)t * E + lane + 32 * i] = z[i];
+    }
+    // softmax (the largest logit is the first pick)
+    const float m = __shfl_sync(0xffffffffu, sel_v, 0);
+    float ssum = 0.f;
+    float ez[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      ez[i] = (lane + 32 * i < E) ? expf(z[i] - m) : 0.f;
+      ssum += ez[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    const float inv = 1.f / ssum;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        if (STATS) {
+          s_p[e] += ez[i] * inv;
+          if ((taken >> i) & 1u) s_c[e] += 1;
+        } else {
+          p_out[(size_t)t * E + e] = ez[i] * inv;
+        }
+      }
+    }
+    const float pj = lane < k ? expf(sel_v - m) * inv : 0.f;
+    float wsum = pj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = sel_i;
+      topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
+    }
   }
-  chunk_stats<EPL>(s_p, s_c, pacc, cacc, chunk, E, cnt, psum);
+  if (!STATS) return;
+  // chunk statistics: warps combined in fixed order
+  __syncthreads();
+  const int* s_c0 = reinterpret_cast<const int*>(s_stat + (size_t)NW * E);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ps = 0.f;
+    int cs = 0;
+#pragma unroll 8
+    for (int w = 0; w < NW; ++w) { ps += s_stat[(size_t)w * E + e]; cs += s_c0[(size_t)w * E + e]; }
+    cnt[(size_t)e * nchunks + chunk] = cs;
+    psum[(size_t)e * nchunks + chunk] = ps;
+  }
 }
 
 // Router fully in one kernel for small E * d: the CTA keeps W_r^T in shared
 // memory ([d][32 EPL + 1] fp32, padded against bank conflicts); each warp
 // computes its tokens' logits as plain fp32 FMA chains over the inputs (lane l
-// owns experts l, l+32, ...), then softmax / top-k / gates as above.
-template <int EPL>
-__global__ void __launch_bounds__(256) k_router_fused(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
-                                                      const float* __restrict__ bias, float* __restrict__ logits_out,
-                                                      int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
-                                                      int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
-                                                      int d, int E, int k, int renorm) {
+// owns experts l, l+32, ...), then softmax / top-k / gates as above.  A token's
+// row is read once, 16 bytes per lane, and its values are broadcast by
+// shuffles; the next token's row is prefetched.
+template <int EPL, int NW>
+__global__ void __launch_bounds__(NW * 32) k_router_fused(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ W, const float* __restrict__ bias,
+                                                          float* __restrict__ logits_out,
+                                                          int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                                                          int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
+                                                          int d, int E, int k, int renorm) {
   extern __shared__ float s_wt[];
-  __shared__ float s_p[8][EPL * 32];
-  __shared__ int s_c[8][EPL * 32];
+  __shared__ float s_p[NW][EPL * 32];
+  __shared__ int s_c[NW][EPL * 32];
   constexpr int EP = EPL * 32 + 1;
   for (int i = threadIdx.x; i < E * d; i += blockDim.x) {  // coalesced reads; odd row pitch: no bank conflicts
     const int e = i / d, c = i - e * d;
@@ -421,23 +485,37 @@ __global__ void __launch_bounds__(256) k_router_fused(const __nv_bfloat16* __res
     const int e = lane + 32 * i;
     b[i] = (bias != nullptr && e < E) ? bias[e] : 0.f;
   }
-  const int t_first = chunk * kChunk + warp * (kChunk / 8);
-  const int t_end = min(T, t_first + kChunk / 8);
+  constexpr int TPW = (kChunk + NW - 1) / NW;  // tokens per warp
+  const int t_first = chunk * kChunk + warp * TPW;
+  const int t_end = min(T, t_first + TPW);
+  const int nv = d >> 3;
+  uint4 nxt = make_uint4(0, 0, 0, 0);
+  if (t_first < t_end && lane < nv) nxt = reinterpret_cast<const uint4*>(x + (size_t)t_first * d)[lane];
   for (int t = t_first; t < t_end; ++t) {
     float acc[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-#pragma unroll 2
-    for (int c0 = 0; c0 < d; c0 += 8) {
-      const uint4 u = xr[c0 >> 3];  // same address in every lane: one broadcast load
-      const float xv[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
-                           bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+    for (int v0 = 0; v0 < nv; v0 += 32) {
+      const uint4 u = nxt;
+      // prefetch: the next 256-input slice of this token, or the first slice of the next token
+      if (v0 + 32 < nv) {
+        nxt = (v0 + 32 + lane < nv) ? reinterpret_cast<const uint4*>(x + (size_t)t * d)[v0 + 32 + lane]
+                                    : make_uint4(0, 0, 0, 0);
+      } else if (t + 1 < t_end) {
+        nxt = lane < nv ? reinterpret_cast<const uint4*>(x + (size_t)(t + 1) * d)[lane] : make_uint4(0, 0, 0, 0);
+      }
+      const int nl = min(32, nv - v0);
+      for (int sl = 0; sl < nl; ++sl) {
+        const uint32_t w0 = __shfl_sync(0xffffffffu, u.x, sl), w1 = __shfl_sync(0xffffffffu, u.y, sl);
+        const uint32_t w2 = __shfl_sync(0xffffffffu, u.z, sl), w3 = __shfl_sync(0xffffffffu, u.w, sl);
+        const float xv[8] = {bf16lo(w0), bf16hi(w0), bf16lo(w1), bf16hi(w1),
+                             bf16lo(w2), bf16hi(w2), bf16lo(w3), bf16hi(w3)};
+        const float* wr = s_wt + (size_t)((v0 + sl) * 8) * EP + lane;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float* wr = s_wt + (size_t)(c0 + q) * EP + lane;
+        for (int q = 0; q < 8; ++q) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) acc[i] = fmaf(xv[q], wr[32 * i], acc[i]);
+          for (int i = 0; i < EPL; ++i) acc[i] = fmaf(xv[q], wr[q * EP + 32 * i], acc[i]);
+        }
       }
     }
     float z[EPL];
@@ -445,62 +523,133 @@ __global__ void __launch_bounds__(256) k_router_fused(const __nv_bfloat16* __res
     for (int i = 0; i < EPL; ++i) z[i] = (lane + 32 * i < E) ? acc[i] + b[i] : -INFINITY;
     route_token<EPL>(z, t, E, k, renorm, logits_out, topk_idx, topk_w, pacc, cacc);
   }
-  chunk_stats<EPL>(s_p, s_c, pacc, cacc, chunk, E, cnt, psum);
+  // chunk statistics: warps combined in fixed order
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) { s_p[warp][lane + 32 * i] = pacc[i]; s_c[warp][lane + 32 * i] = cacc[i]; }
+  __syncthreads();
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ps = 0.f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
+    cnt[(size_t)e * nchunks + chunk] = cs;
+    psum[(size_t)e * nchunks + chunk] = ps;
+  }
 }
 
-// Router logits for small T (decode): W_r is the large operand and is
-// streamed once.  A CTA of 8 warps owns 2 experts; the 4 warps of an expert
-// split the inputs into quarters, lane l of a warp takes inputs 4l..4l+3 of
-// each 128-input step, and keeps one fp32 FMA chain per token (TT tokens per
-// pass).  Lanes, then quarters, are combined in fixed order.
-template <int TT>
-__global__ void __launch_bounds__(256) k_router_skinny(const __nv_bfloat16* __restrict__ x,
-                                                       const float* __restrict__ W, float* __restrict__ logits, int T,
-                                                       int d, int E) {
-  __shared__ float s_part[8][TT];
+// Router logits for small T (decode), exact fp32: W_r is the large operand and
+// is streamed from HBM once (later token blocks re-read it from L2).
+//   Grid: (ceil(E / 32), ceil(T / 16), kSkSplit) with clusters of kSkSplit CTAs
+//   along the inputs.  A CTA stages its 16 tokens x ks-input slice of x in
+//   shared memory as fp32; each of its 8 warps owns 4 experts, and lane l takes
+//   inputs 4l .. 4l+3 of every 128-input step: per step 4 coalesced float4
+//   loads of W_r rows and 16 broadcast-free float4 reads of x feed 256 FMAs
+//   (one fp32 chain per (expert, token) per lane, inputs in order).
+//   The 64 chains of a warp are combined across lanes by a transposing xor
+//   tree (62 shuffles; lane l ends with entries 2l and 2l + 1), the kSkSplit
+//   partial tiles in cluster rank order through distributed shared memory.
+//   Logits are written without bias.
+constexpr int kSkSplit = 8;
+constexpr int kSkTok = 16;
+constexpr int kSkExp = 4;   // experts per warp
+
+__host__ __device__ constexpr int skinny_slice(int d) {
+  return ((d + 128 * kSkSplit - 1) / (128 * kSkSplit)) * 128;   // inputs per split, a multiple of 128
+}
+
+__global__ void __cluster_dims__(1, 1, kSkSplit) __launch_bounds__(256, 2) k_router_skinny(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ W, float* __restrict__ logits,
+                                                          int T, int d, int E) {
+  extern __shared__ __align__(16) float s_x[];      // [kSkTok][ks]
+  __shared__ float s_tile[kSkTok][8 * kSkExp];      // this CTA's partial [token][expert]
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
   const int lane = lane_id(), warp = warp_id();
-  const int e = blockIdx.x * 2 + (warp >> 2);
-  const int quarter = warp & 3;
-  const int span = ((d + 511) / 512) * 128;  // inputs per quarter, a multiple of 128
-  const int i_beg = quarter * span, i_end = min(d, i_beg + span);
-  for (int t0 = 0; t0 < T; t0 += TT) {
-    float acc[TT];
-#pragma unroll
-    for (int j = 0; j < TT; ++j) acc[j] = 0.f;
-    if (e < E) {
-      for (int i = i_beg + lane * 4; i < i_end; i += 128) {
-        const float4 w4 = *reinterpret_cast<const float4*>(W + (size_t)e * d + i);
-#pragma unroll
-        for (int j = 0; j < TT; ++j) {
-          if (t0 + j < T) {
-            const uint2 u = *reinterpret_cast<const uint2*>(x + (size_t)(t0 + j) * d + i);
-            acc[j] = fmaf(bf16lo(u.x), w4.x, acc[j]);
-            acc[j] = fmaf(bf16hi(u.x), w4.y, acc[j]);
-            acc[j] = fmaf(bf16lo(u.y), w4.z, acc[j]);
-            acc[j] = fmaf(bf16hi(u.y), w4.w, acc[j]);
-          }
-        }
-      }
+  const int ks = skinny_slice(d);
+  const int k0 = rank * ks;
+  const int kn = max(0, min(ks, d - k0));
+  const int t0 = blockIdx.y * kSkTok;
+  const int nt = min(kSkTok, T - t0);
+  const int eb = blockIdx.x * 8 * kSkExp;
+  // stage x (zeros for absent tokens and past the slice end)
+  const int nv = ks >> 3;
+  for (int i = threadIdx.x; i < kSkTok * nv; i += blockDim.x) {
+    const int t = i / nv, v = i - t * nv;
+    float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+    if (t < nt && 8 * v < kn) {
+      const uint4 u = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d + k0 + 8 * v);
+      lo = make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
+      hi = make_float4(bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w));
     }
-#pragma unroll
-    for (int j = 0; j < TT; ++j) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int j = 0; j < TT; ++j) s_part[warp][j] = acc[j];
-    }
-    __syncthreads();
-    if (quarter == 0 && e < E) {
-      for (int j = lane; j < TT && t0 + j < T; j += 32) {
-        const int w0 = warp;  // warps w0..w0+3 hold the quarters of expert e
-        logits[(size_t)(t0 + j) * E + e] =
-            ((s_part[w0][j] + s_part[w0 + 1][j]) + s_part[w0 + 2][j]) + s_part[w0 + 3][j];
-      }
-    }
-    __syncthreads();
+    float4* dst = reinterpret_cast<float4*>(s_x + (size_t)t * ks + 8 * v);
+    dst[0] = lo;
+    dst[1] = hi;
   }
+  __syncthreads();
+  float acc[kSkExp * kSkTok];
+#pragma unroll
+  for (int j = 0; j < kSkExp * kSkTok; ++j) acc[j] = 0.f;
+  const int e_first = eb + warp * kSkExp;
+  const int n_e = max(0, min(kSkExp, E - e_first));   // experts of this warp that exist
+  const float* wbase = W + (size_t)(n_e > 0 ? e_first : 0) * d + k0 + 4 * lane;
+  const int nsteps = (kn + 127) >> 7;
+  auto load_w = [&](int st, int q) -> float4 {
+    return (q < n_e && st < nsteps && st * 128 + 4 * lane < kn)
+               ? __ldg(reinterpret_cast<const float4*>(wbase + (size_t)q * d + st * 128))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  float4 wn[kSkExp];
+#pragma unroll
+  for (int q = 0; q < kSkExp; ++q) wn[q] = load_w(0, q);
+  for (int st = 0; st < nsteps; ++st) {
+    float4 w[kSkExp];
+#pragma unroll
+    for (int q = 0; q < kSkExp; ++q) {
+      w[q] = wn[q];
+      wn[q] = load_w(st + 1, q);   // next step's rows, in flight during this step's FMAs
+    }
+#pragma unroll
+    for (int t = 0; t < kSkTok; ++t) {
+      const float4 xv = reinterpret_cast<const float4*>(s_x + (size_t)t * ks + st * 128)[lane];
+#pragma unroll
+      for (int q = 0; q < kSkExp; ++q) {
+        float& a = acc[q * kSkTok + t];
+        a = fmaf(xv.x, w[q].x, a);
+        a = fmaf(xv.y, w[q].y, a);
+        a = fmaf(xv.z, w[q].z, a);
+        a = fmaf(xv.w, w[q].w, a);
+      }
+    }
+  }
+  // transposing xor tree: at offset o the lane keeps the half of its entries
+  // selected by lane bit o and adds the partner's copy of that half
+#pragma unroll
+  for (int o = 16, n = kSkExp * kSkTok; o >= 1; o >>= 1, n >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = up ? acc[j] : acc[j + n / 2];
+      const float keep = up ? acc[j + n / 2] : acc[j];
+      acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  // lane l holds entries 2l, 2l + 1 of (expert q, token t) = (idx / 16, idx % 16)
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int idx = 2 * lane + j;
+    s_tile[idx % kSkTok][warp * kSkExp + idx / kSkTok] = acc[j];
+  }
+  cluster.sync();
+  // rank r finishes tokens 2r, 2r + 1 of the block (kSkTok / kSkSplit = 2) for the CTA's 32 experts
+  if (threadIdx.x < 64) {
+    const int tl = rank * 2 + (threadIdx.x >> 5), el = threadIdx.x & 31;
+    float v = 0.f;
+#pragma unroll
+    for (int r = 0; r < kSkSplit; ++r) v += cluster.map_shared_rank(&s_tile[0][0], r)[tl * 32 + el];
+    if (tl < nt && eb + el < E) logits[(size_t)(t0 + tl) * E + eb + el] = v;
+  }
+  cluster.sync();  // tiles stay alive until every CTA of the cluster has read them
 }
 
 // ---------------------------------------------------------------------------
@@ -517,47 +666,66 @@ __global__ void __launch_bounds__(256) k_chunk_hist(const int32_t* __restrict__ 
     atomicAdd(&s_h[e], 1);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)blockIdx.x * E + e] = s_h[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)e * gridDim.x + blockIdx.x] = s_h[e];
+}
+
+// Chunk tables from per-token routing (small batches): one CTA per chunk of
+// kChunk tokens.  cnt[e][c] by shared-memory integer counts (order-free),
+// psum[e][c] = sum over the chunk's tokens, in token order, of p[t,e].
+__global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__ topk_idx,
+                                                     const float* __restrict__ p, int32_t* __restrict__ cnt,
+                                                     float* __restrict__ psum, int T, int E, int k) {
+  __shared__ int s_h[kMaxRouterE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_h[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kChunk;
+  const int nt = min(kChunk, T - t0);
+  for (int i = threadIdx.x; i < nt * k; i += blockDim.x) atomicAdd(&s_h[topk_idx[(size_t)t0 * k + i]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ps = 0.f;
+    for (int t = 0; t < nt; ++t) ps += p[(size_t)(t0 + t) * E + e];
+    cnt[(size_t)e * gridDim.x + blockIdx.x] = s_h[e];
+    psum[(size_t)e * gridDim.x + blockIdx.x] = ps;
+  }
 }
 
 // ---------------------------------------------------------------------------
-// One warp per expert: cnt[c][e] -> exclusive prefix over chunks (in place),
-// counts[e]; optional f[e] = counts/T, P[e] = sum_c psum[c][e] / T.
+// Chunk tables are expert-major: cnt[e][c], psum[e][c].  One warp per expert:
+// cnt[e][c] -> exclusive prefix over chunks (in place), counts[e]; optional
+// f[e] = counts/T and P[e] = sum_c psum[e][c] / T (lanes in order, then a fixed
+// xor tree).  Lanes read 32 consecutive chunks at a time (coalesced).
 __global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, const float* __restrict__ psum,
                                                     int32_t* __restrict__ counts, float* __restrict__ f_out,
                                                     float* __restrict__ p_out, int nchunks, int E, int T) {
   const int e = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   if (e >= E) return;
-  const int per = (nchunks + 31) / 32;
-  const int c0 = min(nchunks, lane * per), c1 = min(nchunks, c0 + per);
-  int seg = 0;
+  int32_t* row = cnt + (size_t)e * nchunks;
+  const float* prow = psum != nullptr ? psum + (size_t)e * nchunks : nullptr;
+  int run = 0;
   float ps = 0.f;
-  for (int c = c0; c < c1; ++c) {
-    seg += cnt[(size_t)c * E + e];
-    if (psum != nullptr) ps += psum[(size_t)c * E + e];
-  }
-  int incl = seg;
+  for (int c0 = 0; c0 < nchunks; c0 += 32) {
+    const int c = c0 + lane;
+    const int v = c < nchunks ? row[c] : 0;
+    if (prow != nullptr && c < nchunks) ps += prow[c];
+    int incl = v;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (c < nchunks) row[c] = run + incl - v;
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
-  int run = incl - seg;
-  for (int c = c0; c < c1; ++c) {
-    const int v = cnt[(size_t)c * E + e];
-    cnt[(size_t)c * E + e] = run;
-    run += v;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  if (psum != nullptr) {
+  if (prow != nullptr) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
   }
   if (lane == 0) {
-    if (counts != nullptr) counts[e] = total;
-    if (f_out != nullptr) f_out[e] = (float)total / (float)T;
-    if (p_out != nullptr && psum != nullptr) p_out[e] = ps / (float)T;
+    if (counts != nullptr) counts[e] = run;
+    if (f_out != nullptr) f_out[e] = (float)run / (float)T;
+    if (p_out != nullptr && prow != nullptr) p_out[e] = ps / (float)T;
   }
 }
 

@@ -60,6 +60,26 @@ def assert_bf16_rounded(got, want, scale, what="value"):
         f"{float((np.abs(got - want) / bound).max()):.2f}x"
 
 
+def glu_accum_scale(x, w13, act):
+    """Propagated fp32 accumulation error of h = act(x W1^T) * (x W3^T), as a ``scale`` for assert_bf16_rounded.
+
+    Each of g = x W1^T and u = x W3^T is a d-term fp32 dot product, off by at most d * 2^-24 * |x| @ |W|^T
+    (recursive summation); |act'| <= 1.13 for SiLU and exact-erf GELU, so
+    |dh| <= gamma_d * (1.13 * (|x| @ |W1|^T) * |u| + |act(g)| * (|x| @ |W3|^T)).  At points where g or u
+    cancels to nearly zero this term, not the bf16 rounding of h, dominates.
+    """
+    import oracle
+    x = np.asarray(x, np.float64)
+    w13 = np.asarray(w13, np.float64)
+    H = w13.shape[0] // 2
+    d = x.shape[1]
+    g, u = x @ w13[:H].T, x @ w13[H:].T
+    a = oracle.silu(g) if act == 0 else oracle.gelu_erf(g)
+    gam = 1.01 * d * 2.0 ** -24
+    err = gam * (1.13 * (np.abs(x) @ np.abs(w13[:H]).T) * np.abs(u) + np.abs(a) * (np.abs(x) @ np.abs(w13[H:]).T))
+    return err * 2.0 ** 8
+
+
 def int4_expert_weights(moe, wl, seed=0, device="cuda", experts=None):
     """Draw every expert's fp32 weights with synth (on ``device``) and pack them with the library's INT4 quantiser.
 

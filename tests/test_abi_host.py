@@ -97,3 +97,4 @@ def test_null_and_workspace_errors_return_before_device_work(L):
     rc = L.moe_quantize_int4(fake, 4, 100, fake, fake, None)
     assert rc == 1            # K % 128 != 0
     assert L.moe_set_wait_limit_ns(0) == 1
+    assert L.moe_set_pair_gemm(2) == 1 and L.moe_set_pair_gemm(-1) == 1

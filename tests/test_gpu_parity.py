@@ -15,7 +15,7 @@ import torch
 
 import oracle as O
 import synth
-from helpers import MARGIN, assert_bf16_rounded, assert_out_close, np64, npi, rel_frob, shape_of
+from helpers import MARGIN, assert_bf16_rounded, assert_out_close, glu_accum_scale, np64, npi, rel_frob, shape_of
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -63,10 +63,16 @@ def _route_case(moe, wl, T, seed):
     return wl, inp, r, ref, x64, W64, b64
 
 
-@pytest.mark.parametrize("name,T", [("tiny", 256), ("small", 4096), ("skewed", 3000), ("geglu", 2000),
-                                    ("decode_int4", 64)])
-def test_route_matches_oracle(lib, name, T):
-    wl, inp, r, ref, x64, W64, b64 = _route_case(lib, synth.get_workload(name), T, seed=1)
+# Router paths: fused shared-memory router (tiny, small, geglu), certified tensor-core router (skewed,
+# granular shapes), weight-streaming decode router (decode_int4; T <= 256: one token, a ragged token
+# block with E = 200 and a ragged last input slice with d = 784), split-K CUDA-core router (E = 200,
+# which is neither a multiple of 16 nor small enough for the fused router).
+@pytest.mark.parametrize("name,T,over", [("tiny", 256, {}), ("small", 4096, {}), ("skewed", 3000, {}),
+                                         ("geglu", 2000, {}), ("decode_int4", 64, {}), ("decode_int4", 1, {}),
+                                         ("granular", 37, {"E": 200, "d": 784}),
+                                         ("granular", 1000, {"E": 200}), ("decode_int4", 300, {"E": 96})])
+def test_route_matches_oracle(lib, name, T, over):
+    wl, inp, r, ref, x64, W64, b64 = _route_case(lib, synth.get_workload(name).replace(**over), T, seed=1)
     # Logits.  Every logit is within the bound of an fp32 accumulation of 3d products in any rounding
     # direction (the tensor-core screening pass); the logits of the chosen experts are plain fp32 FMA dot
     # products, within the round-to-nearest bound gamma_{d+2} * sum|x_i w_i| (+ |bias|).
@@ -147,9 +153,52 @@ def test_expert_ffn_matches_oracle(lib, E, d, H, act, max_rows, cap):
             continue
         h_ref = O.glu_hidden(x64[a:a + n], w13_64[e], act)
         y_ref = h_ref @ w2_64[e].T
-        assert_bf16_rounded(hg[a:a + n], h_ref, 0.0, f"h[e={e}]")
+        assert_bf16_rounded(hg[a:a + n], h_ref, glu_accum_scale(x64[a:a + n], w13_64[e], act), f"h[e={e}]")
         assert_bf16_rounded(yg[a:a + n], y_ref, np.abs(h_ref) @ np.abs(w2_64[e]).T, f"y[e={e}]")
         assert rel_frob(yg[a:a + n], y_ref) <= 5e-3
+
+
+# CTA-pair tiles (256 rows, tcgen05 cta_group::2) against the oracle and against the single-CTA kernel on the
+# same inputs: ragged groups (an empty one, tails shorter than the second CTA's 128 rows), gated SwiGLU and GeGLU
+# GEMMs and a plain down GEMM wide enough for 256-column tiles.
+@pytest.mark.parametrize("d,H,act,rows", [(256, 2048, 0, [1000, 0, 1001]), (512, 1024, 1, [1500, 129]),
+                                          (1024, 512, 0, [1500, 1500])])
+def test_expert_ffn_pair_tiles(lib, d, H, act, rows):
+    moe = lib
+    E = len(rows)
+    rows_t = torch.tensor(rows, dtype=torch.int32)
+    start = torch.cumsum(torch.tensor([0] + rows[:-1]), 0).to(torch.int32)
+    R = int(sum(rows))
+    wl = synth.Workload("t", T=1, d=d, E=E, k=1, H=H, act=act)
+    w13 = torch.stack([synth.expert_weights_f32(wl, 4, e)[0] for e in range(E)]).to(torch.bfloat16)
+    w2 = torch.stack([synth.expert_weights_f32(wl, 4, e)[1] for e in range(E)]).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(d + H)
+    xg = torch.randn(R, d, generator=g).to(torch.bfloat16)
+    s = _shape(moe, 1, E, 1, d=d, H=H, act=act)
+    outs = {}
+    try:
+        for pair in (True, False):
+            moe.moe_set_pair_gemm(pair)
+            h, y = moe.moe_expert_ffn(s, xg.to(DEV), w13.to(DEV), w2.to(DEV), hidden=H, group_start=start.to(DEV),
+                                      group_rows=rows_t.to(DEV))
+            torch.cuda.synchronize()
+            outs[pair] = (np64(h), np64(y))
+    finally:
+        moe.moe_set_pair_gemm(True)
+    x64, w13_64, w2_64 = np64(xg), np64(w13), np64(w2)
+    for pair, (hg, yg) in outs.items():
+        for e in range(E):
+            a, n = int(start[e]), int(rows[e])
+            if n == 0:
+                continue
+            h_ref = O.glu_hidden(x64[a:a + n], w13_64[e], act)
+            y_ref = h_ref @ w2_64[e].T
+            assert_bf16_rounded(hg[a:a + n], h_ref, glu_accum_scale(x64[a:a + n], w13_64[e], act), f"h[e={e}, pair={pair}]")
+            assert_bf16_rounded(yg[a:a + n], y_ref, np.abs(h_ref) @ np.abs(w2_64[e]).T, f"y[e={e}, pair={pair}]")
+            assert rel_frob(yg[a:a + n], y_ref) <= 5e-3
+    same_h = np.array_equal(outs[True][0], outs[False][0])
+    same_y = np.array_equal(outs[True][1], outs[False][1])
+    print(f"pair vs single: h identical={same_h} y identical={same_y}")
 
 
 def test_expert_ffn_single_dense_group(lib):
@@ -346,7 +395,7 @@ def test_expert_ffn_int4_matches_oracle(lib, E, d, H, act, max_rows):
             continue
         w13e, w2e = oracle_int4_expert(wl, 4, e, DEV)
         h_ref = O.glu_hidden(x64[a:a + n], w13e, act)
-        assert_bf16_rounded(hg[a:a + n], h_ref, 0.0, f"h[e={e}]")
+        assert_bf16_rounded(hg[a:a + n], h_ref, glu_accum_scale(x64[a:a + n], w13e, act), f"h[e={e}]")
         assert_bf16_rounded(yg[a:a + n], h_ref @ w2e.T, np.abs(h_ref) @ np.abs(w2e).T, f"y[e={e}]")
 
 

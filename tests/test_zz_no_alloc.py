@@ -54,7 +54,7 @@ def test_noalloc_permute_matches_workspace_permute_twice(lib):
 def test_noalloc_permute_rejects_shapes_beyond_its_scratch(lib):
     moe = lib
     L = moe.load()
-    s = _shape(moe, 128 * 513, 512, 2, 16, 0)              # ceil(T/128) * E = 262656 > 262144
+    s = _shape(moe, 32 * 513, 512, 2, 16, 0)               # ceil(T/32) * E = 262656 > 262144
     fake = ctypes.c_void_p(4096)                            # never dereferenced: the size check fails first
     rc = L.moe_permute_noalloc(ctypes.byref(s), fake, fake, fake, None, None, fake, fake, None, fake, None)
     assert rc == 2                                          # MOE_UNSUPPORTED_SHAPE
