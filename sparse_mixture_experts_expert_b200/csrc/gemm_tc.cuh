@@ -59,6 +59,10 @@ struct GemmParams {
   const float* bias;   // kModeF32: optional per-column bias [N]
 };
 
+#ifndef MOE_GEMM_MAX_STAGES
+#define MOE_GEMM_MAX_STAGES 8   // TMA -> MMA ring depth cap (the shared-memory budget usually binds first)
+#endif
+
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // one 128-byte swizzle atom of bf16
 constexpr int kMaxGroupsSmem = 512;
@@ -72,7 +76,8 @@ struct GemmCfg {
   static constexpr int kBBytes = (CG == 2 ? BN / 2 : BN) * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBudget = 219 * 1024 - 1024 - kEpiBytes;
-  static constexpr int kStages = kBudget / kStageBytes > 8 ? 8 : kBudget / kStageBytes;
+  static constexpr int kStages = kBudget / kStageBytes > MOE_GEMM_MAX_STAGES ? MOE_GEMM_MAX_STAGES
+                                                                            : kBudget / kStageBytes;
   static constexpr int kTmemCols = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);  // two accumulators, pow2
   static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kEpiBytes;
 };
@@ -85,6 +90,7 @@ template <int MODE, int BN, int CG = 1>
 __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   using Cfg = GemmCfg<BN, CG>;
   constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
   constexpr bool kPair = CG == 2;

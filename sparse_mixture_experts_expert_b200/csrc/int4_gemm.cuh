@@ -41,6 +41,8 @@ struct Int4Params {
   int up_row0;                   // gated: first up row (H)
   __nv_bfloat16* out;            // [R, N]
   long long ldo;
+  int ksplit;                    // >= 1: each task's slabs are split into this many contiguous ranges
+  float* part;                   // ksplit > 1: fp32 partials [ksplit, R, 2N] (gated: gate | up) or [ksplit, R, N]
 };
 
 __device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t mask, uint32_t c) {
@@ -137,6 +139,7 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4& wa, cons
 //       tree), the correction term 136 * sum(x) of the offset codes.
 __global__ void __launch_bounds__(256) k_int4_act_prep(const __nv_bfloat16* __restrict__ A, long long rows, int K,
                                                        float* __restrict__ sums, __nv_bfloat16* __restrict__ Aq) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const long long n = rows * (K / 8);
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const bool on = i < n;
@@ -175,10 +178,11 @@ constexpr int kI4Smem = kI4Warps * kI4Stages * kI4SlabBytes;
 // (the activation group sums) once per group, instead of one packed
 // subtraction per pair of weights; p.act is then the fragment-ordered copy
 // written by k_int4_act_prep.
-template <bool GLU, int ACT, bool OFFS>
+template <bool GLU, int ACT, bool OFFS, bool SPLIT>
 __global__ void __launch_bounds__(kI4Warps * 32, 1)
     k_int4_stream(const __grid_constant__ CUtensorMap tmW, const Int4Params p, unsigned long long wait_limit_ns,
                   const float* __restrict__ xsum) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ int s_prefix[kMaxGroupsSmem + 1];
   __shared__ __align__(8) uint64_t s_bar[kI4Warps][kI4Stages];
@@ -217,16 +221,20 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
   __syncthreads();
 
-  const int total = s_prefix[G];
-  const int nslab = (p.K + 255) / 256;               // items per task (the last slab may hold one 128-group)
+  const int KS = SPLIT ? p.ksplit : 1;   // compile-time 1 unless the reduction is split
+  const int total = s_prefix[G] * KS;
+  const int nslab = (p.K + 255) / 256;               // slabs of a whole reduction (the last may hold one 128-group)
   const int tfirst = blockIdx.x * kI4Warps + warp;
   const int tstride = gridDim.x * kI4Warps;
   uint8_t* ring = i4_smem + (size_t)warp * kI4Stages * kI4SlabBytes;
   const int gq = lane >> 2, c = lane & 3;
   const int ngroups_k = p.K / 128;
 
-  struct TaskPos { int g, o0, n0, n_rows; long long row0; };
-  auto locate = [&](int task) -> TaskPos {
+  // task = base * KS + split: a base task is (group, 16 or 32 output rows, 8 tokens); split s covers
+  // slabs [s * nslab / KS, (s + 1) * nslab / KS) of its reduction
+  struct TaskPos { int g, o0, n0, n_rows, s, sb, se; long long row0; };
+  auto locate = [&](int t) -> TaskPos {
+    const int task = SPLIT ? t / KS : t;
     int lo = 0, hi = G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -240,6 +248,9 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
     const int tg = task - s_prefix[lo];
     tp.o0 = (tg / nchunks) * (GLU ? 16 : 32);
     tp.n0 = (tg % nchunks) * 8;
+    tp.s = SPLIT ? t - task * KS : 0;
+    tp.sb = SPLIT ? tp.s * nslab / KS : 0;
+    tp.se = SPLIT ? (tp.s + 1) * nslab / KS : nslab;
     return tp;
   };
   // weight rows of a task's two 16-row blocks (rows of the flattened [experts * b_rows] map)
@@ -251,13 +262,17 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   // Producer state (lane 0 issues the copies; the values are warp-uniform).
   // Items are (task, slab) pairs in order; issued - consumed <= kI4Stages.
   int issued = 0, consumed = 0;
-  int p_task = tfirst, p_slab = 0, p_st = 0, p_ra = 0, p_rb = 0;
+  int p_task = tfirst, p_slab = 0, p_se = 0, p_st = 0, p_ra = 0, p_rb = 0;
+  bool p_new = true;
   auto refill = [&]() {
     while (issued - consumed < kI4Stages) {
-      if (p_slab == 0) {
+      if (p_new) {
         if (p_task >= total) return;
         const TaskPos tp = locate(p_task);
         rows_of(tp, p_ra, p_rb);
+        p_slab = tp.sb;
+        p_se = tp.se;
+        p_new = false;
       }
       if (lane == 0) {
         uint8_t* dst = ring + p_st * kI4SlabBytes;
@@ -267,7 +282,7 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
       }
       ++issued;
       if (++p_st == kI4Stages) p_st = 0;
-      if (++p_slab == nslab) { p_slab = 0; p_task += tstride; }
+      if (++p_slab == p_se) { p_new = true; p_task += tstride; }
     }
   };
 
@@ -281,10 +296,13 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   const long long s8 = 8ll * ngroups_k;
   int c_task = tfirst, c_slab = 0, c_st = 0;
   uint32_t c_phase = 0;
+  bool c_new = true;
   while (true) {
-    if (c_slab == 0) {
+    if (c_new) {
       if (c_task >= total || s_abort[warp]) break;
       cur = locate(c_task);
+      c_slab = cur.sb;
+      c_new = false;
       int ra, rb;
       rows_of(cur, ra, rb);
       const int tok = cur.n0 + gq;
@@ -369,25 +387,37 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
     ++consumed;
     if (++c_st == kI4Stages) { c_st = 0; c_phase ^= 1u; }
     refill();
-    if (c_slab == nslab - 1) {
+    if (c_slab == cur.se - 1) {
       // D fragments: (m = gq, n = 2c, 2c+1) in [0],[1]; (m = gq + 8, same n) in [2],[3]
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = gq + (i >= 2 ? 8 : 0);
         const int n = cur.n0 + 2 * c + (i & 1);
         if (n < cur.n_rows) {
-          __nv_bfloat16* orow = p.out + (cur.row0 + n) * p.ldo + cur.o0;
-          if (GLU) {
-            const float a = ACT == kModeSwiGLU ? act_silu(tA[i]) : act_gelu(tA[i]);
-            orow[m] = __float2bfloat16_rn(a * tB[i]);
+          if (SPLIT) {
+            // fp32 partials of this slab range; k_int4_splitk_reduce adds the ranges in order
+            float* prow = p.part + ((long long)cur.s * p.R + cur.row0 + n) * (GLU ? 2 * p.N : p.N) + cur.o0;
+            if (GLU) {
+              prow[m] = tA[i];
+              prow[p.N + m] = tB[i];
+            } else {
+              prow[m] = tA[i];
+              prow[m + 16] = tB[i];
+            }
           } else {
-            orow[m] = __float2bfloat16_rn(tA[i]);
-            orow[m + 16] = __float2bfloat16_rn(tB[i]);
+            __nv_bfloat16* orow = p.out + (cur.row0 + n) * p.ldo + cur.o0;
+            if (GLU) {
+              const float a = ACT == kModeSwiGLU ? act_silu(tA[i]) : act_gelu(tA[i]);
+              orow[m] = __float2bfloat16_rn(a * tB[i]);
+            } else {
+              orow[m] = __float2bfloat16_rn(tA[i]);
+              orow[m + 16] = __float2bfloat16_rn(tB[i]);
+            }
           }
         }
       }
     }
-    if (++c_slab == nslab) { c_slab = 0; c_task += tstride; }
+    if (++c_slab == cur.se) { c_new = true; c_task += tstride; }
   }
   // never leave the CTA with copies still landing in its shared memory
   {
@@ -396,6 +426,31 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
       mbar_wait(&s_bar[warp][i % kI4Stages], (uint32_t)((i / kI4Stages) & 1), wait_limit_ns, &dummy, 0x0202);
   }
   __syncwarp();
+}
+
+// Split reduction of k_int4_stream: out[r, o] from the ksplit fp32 partials added
+// in split order (gated: h = act(sum g) * (sum u); plain: y = sum).
+template <bool GLU, int ACT>
+__global__ void __launch_bounds__(256) k_int4_splitk_reduce(const float* __restrict__ part, int ksplit, long long R,
+                                                            int N, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= R * N) return;
+  const long long r = i / N;
+  const int o = (int)(i - r * N);
+  const int W = GLU ? 2 * N : N;
+  float g = 0.f, u = 0.f;
+  for (int sp = 0; sp < ksplit; ++sp) {
+    const float* row = part + ((long long)sp * R + r) * W;
+    g += row[o];
+    if (GLU) u += row[N + o];
+  }
+  if (GLU) {
+    const float a = ACT == kModeSwiGLU ? act_silu(g) : act_gelu(g);
+    out[i] = __float2bfloat16_rn(a * u);
+  } else {
+    out[i] = __float2bfloat16_rn(g);
+  }
 }
 
 }  // namespace moe

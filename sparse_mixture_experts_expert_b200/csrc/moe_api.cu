@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -33,6 +34,43 @@ static inline void count_launch() { g_launches.fetch_add(1, std::memory_order_re
   do {                                           \
     count_launch();                              \
     if (cudaGetLastError() != cudaSuccess) return MOE_CUDA_ERROR; \
+  } while (0)
+
+// Every kernel is launched with programmatic stream serialisation (programmatic dependent launch): its
+// grid may be scheduled while the previous kernel on the stream drains, and it waits (griddepcontrol.wait,
+// first statement of every kernel here) before touching memory.  This hides most of the launch gap between
+// the short kernels of one forward, also inside CUDA graphs.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+#ifndef MOE_NO_PDL
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+#endif
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+#define MOE_LAUNCH(kern, grid, block, smem, st, ...)                                                      \
+  do {                                                                                                   \
+    if (launch_pdl(kern, dim3(grid), dim3(block), (size_t)(smem), st, 1u, __VA_ARGS__) != cudaSuccess)   \
+      return MOE_CUDA_ERROR;                                                                             \
   } while (0)
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -99,8 +137,15 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, wsplit, wnorm, xsum, xq, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+  size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
 };
+
+// Split-reduction partials of the INT4 shared expert (decode batches: T <= 256): up to 8 ranges of
+// T x max(2 H_s, d) fp32.
+static size_t i4part_floats(const moe_shape* s) {
+  if (s->wfmt != MOE_WFMT_INT4_G128 || s->H_s == 0 || s->T > 256) return 0;
+  return (size_t)8 * s->T * std::max(2 * s->H_s, s->d);
+}
 
 static Workspace ws_layout(const moe_shape* s) {
   Workspace L{};
@@ -117,6 +162,7 @@ static Workspace ws_layout(const moe_shape* s) {
   const int xs_cols = std::max(s->d, std::max(s->H, s->H_s));
   L.xsum = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * (xs_cols / 128) * 4 : 16);
   L.xq = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * xs_cols * 2 : 16);
+  L.i4part = take(i4part_floats(s) * 4 + 16);
   L.cnt = take((size_t)nchunks * s->E * 4);
   L.psum = take((size_t)nchunks * s->E * 4);
   L.idx = take((size_t)s->T * s->k * 4);
@@ -188,7 +234,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   const long long tiles = ub_mtiles * cdiv(p.N, OUTN);
   if (CG == 1) {
     const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
-    k_grouped_gemm<MODE, BN, 1><<<grid, 256, Cfg::kSmemBytes, st>>>(ta, tb, p);
+    MOE_LAUNCH((k_grouped_gemm<MODE, BN, 1>), grid, 256, Cfg::kSmemBytes, st, ta, tb, p);
   } else {
     // clusters of 2 CTAs, one pair per two SMs
     const int pairs = (int)std::max<long long>(1, std::min<long long>(num_sms() / 2, tiles));
@@ -197,14 +243,8 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = Cfg::kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, k_grouped_gemm<MODE, BN, CG>, ta, tb, p));
+    MOE_CUDA_TRY(launch_pdl(k_grouped_gemm<MODE, BN, CG>, cfg.gridDim, cfg.blockDim, cfg.dynamicSmemBytes, st, 2u,
+                            ta, tb, p));
   }
   MOE_LAUNCH_CHECK();
   return MOE_OK;
@@ -217,18 +257,21 @@ static bool use_pair_gemm(int mode, int BN, long long R, int n_groups) {
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
-// Column tile: the largest of 256/128/64 unless a narrower one fills the SMs in fewer
-// tile-widths of work (cost = waves x tile width, ties to the wider tile).
+// Column tile: 256, 128 or 64, the one with the least modelled time = waves x time per tile.  Per k-step a
+// tile costs max(MMA, operand traffic): the MMA scales with BN, the L2 -> SM traffic with 128 + BN rows,
+// which measured about 1.1 MMA-column units per row on B200 (a 128 x 256 tile runs at ~60% of the tensor
+// peak).  Narrow tiles are therefore only chosen where they cut the number of waves substantially.
 static int pick_bn(bool glu, int N, long long mtiles) {
   const int sms = num_sms();
   int best = 0;
-  long long best_cost = 0;
+  double best_cost = 0.0;
   for (int bn : {256, 128, 64}) {
     const int outn = glu ? bn / 2 : bn;
     if (bn > 64 && outn / 2 >= N) continue;  // mostly padding
     const long long tiles = mtiles * cdiv(N, outn);
-    const long long cost = cdiv(tiles, sms) * bn;
-    if (best == 0 || cost * 100 < best_cost * 95) { best = bn; best_cost = cost; }
+    const double per_tile = std::max((double)bn, 1.1 * (128.0 + bn));
+    const double cost = (double)cdiv(tiles, sms) * per_tile;
+    if (best == 0 || cost < best_cost * 0.97) { best = bn; best_cost = cost; }
   }
   return best == 0 ? 64 : best;
 }
@@ -311,12 +354,12 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
       }                                                                                                           \
     }                                                                                                             \
     const unsigned grid = ST_ ? (unsigned)nchunks : (unsigned)cdiv(s->T, NW_);                                    \
-    k_router_topk<N_, NW_, XR_, ST_><<<grid, NW_ * 32, smem, st>>>(part, nsplit, bias, logits, idx, w, cnt, psum,  \
+    MOE_LAUNCH((k_router_topk<N_, NW_, XR_, ST_>), grid, NW_ * 32, smem, st, part, nsplit, bias, logits, idx, w, cnt, psum,  \
                                                                    p_scratch, (int)s->T, s->E, s->k, s->renorm,  \
                                                                    refine);                                       \
     MOE_LAUNCH_CHECK();                                                                                           \
     if (!ST_) {                                                                                                   \
-      k_chunk_stats<<<nchunks, 256, 0, st>>>(idx, p_scratch, cnt, psum, (int)s->T, s->E, s->k);                   \
+      MOE_LAUNCH((k_chunk_stats), nchunks, 256, 0, st, idx, p_scratch, cnt, psum, (int)s->T, s->E, s->k);                   \
       MOE_LAUNCH_CHECK();                                                                                         \
     }                                                                                                             \
     return MOE_OK;                                                                                                \
@@ -333,7 +376,7 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
 static int launch_scan(const moe_shape* s, int32_t* cnt, const float* psum, int32_t* counts, float* f, float* P,
                        cudaStream_t st) {
   const int nchunks = (int)cdiv(s->T, kChunk);
-  k_chunk_scan<<<(int)cdiv(s->E, 8), 256, 0, st>>>(cnt, psum, counts, f, P, nchunks, s->E, (int)s->T);
+  MOE_LAUNCH((k_chunk_scan), (int)cdiv(s->E, 8), 256, 0, st, cnt, psum, counts, f, P, nchunks, s->E, (int)s->T);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -347,12 +390,12 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   const unsigned mv_blocks = (unsigned)cdiv(s->T * (long long)(s->d / 8), 256);
 #define MOE_SCATTER_CASE(N_)                                                                                  \
   if (s->k <= N_) {                                                                                           \
-    k_scatter<N_><<<(unsigned)cdiv(nchunks, 4), 128, 0, st>>>(xb, idx, cbase, counts, (int)s->T, s->d, s->E,   \
+    MOE_LAUNCH((k_scatter<N_>), (unsigned)cdiv(nchunks, 4), 128, 0, st, xb, idx, cbase, counts, (int)s->T, s->d, s->E,   \
                                                               s->k, s->capacity,                              \
                                            slot, drop, row_src, xp, kept, offs);                              \
     MOE_LAUNCH_CHECK();                                                                                       \
     if (move_rows) {                                                                                          \
-      k_move_rows<N_><<<mv_blocks, 256, 0, st>>>(xb, slot, (int)s->T, s->d, s->k, xp);                       \
+      MOE_LAUNCH((k_move_rows<N_>), mv_blocks, 256, 0, st, xb, slot, (int)s->T, s->d, s->k, xp);                       \
       MOE_LAUNCH_CHECK();                                                                                     \
     }                                                                                                         \
     return MOE_OK;                                                                                            \
@@ -367,6 +410,8 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
 struct Int4Scratch {
   float* xsum;
   void* xq;
+  float* part = nullptr;        // split-reduction partials (dense groups with few tasks), or none
+  size_t part_floats = 0;
 };
 
 static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const void* wq, const void* wsc,
@@ -388,6 +433,23 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
   p.up_row0 = up_row0;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ldo = N;
+  p.ksplit = 1;
+  p.part = nullptr;
+  // A single dense group with too few (16 or 32 rows x 8 tokens) tasks to occupy every warp of every SM
+  // (the shared expert of a decode batch) splits each task's reduction into contiguous slab ranges; fp32
+  // partials go to scratch and k_int4_splitk_reduce adds them in order.
+  {
+    const long long base = (long long)(N / (glu ? 16 : 32)) * cdiv(R, 8);
+    const long long warps = (long long)num_sms() * kI4Warps;
+    const int nslab = (int)cdiv(K, 256);
+    if (grows == nullptr && scr.part != nullptr && scr.xq != nullptr && base < warps) {
+      const int ks = (int)std::min<long long>(std::min(nslab / 2, 8), cdiv(2 * warps, base));
+      if (ks > 1 && (size_t)ks * R * (glu ? 2 * N : N) <= scr.part_floats) {
+        p.ksplit = ks;
+        p.part = scr.part;
+      }
+    }
+  }
   {
     // 2-D byte map over all experts' packed rows; box = 16 rows x 128 bytes (256 inputs)
     EncodeTiledFn enc = get_encoder();
@@ -405,38 +467,55 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
     const unsigned long long bit = 1ull << (dev & 63);
     static std::atomic<unsigned long long> done{0};
     if (!(done.load() & bit)) {
-#define MOE_I4_ATTR(G_, A_, O_)                                                                          \
-      MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_stream<G_, A_, O_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define MOE_I4_ATTR(G_, A_, O_, S_)                                                                          \
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_stream<G_, A_, O_, S_>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                         kI4Smem));
-      MOE_I4_ATTR(false, kModePlain, false) MOE_I4_ATTR(true, kModeSwiGLU, false) MOE_I4_ATTR(true, kModeGeGLU, false)
-      MOE_I4_ATTR(false, kModePlain, true) MOE_I4_ATTR(true, kModeSwiGLU, true) MOE_I4_ATTR(true, kModeGeGLU, true)
+      MOE_I4_ATTR(false, kModePlain, false, false) MOE_I4_ATTR(true, kModeSwiGLU, false, false)
+      MOE_I4_ATTR(true, kModeGeGLU, false, false) MOE_I4_ATTR(false, kModePlain, true, false)
+      MOE_I4_ATTR(true, kModeSwiGLU, true, false) MOE_I4_ATTR(true, kModeGeGLU, true, false)
+      MOE_I4_ATTR(false, kModePlain, true, true) MOE_I4_ATTR(true, kModeSwiGLU, true, true)
+      MOE_I4_ATTR(true, kModeGeGLU, true, true)
 #undef MOE_I4_ATTR
       done.fetch_or(bit);
     }
     if (xsum != nullptr) {
-      k_int4_act_prep<<<(unsigned)cdiv(R * (K / 8), 256), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(A), R,
+      MOE_LAUNCH((k_int4_act_prep), (unsigned)cdiv(R * (K / 8), 256), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(A), R,
                                                                          K, xsum,
                                                                          reinterpret_cast<__nv_bfloat16*>(scr.xq));
       MOE_LAUNCH_CHECK();
       p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);
     }
     const long long rows_per_task = glu ? 16 : 32;
-    const long long ub = (long long)(N / rows_per_task) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8));
+    const long long ub = (long long)(N / rows_per_task) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8)) * p.ksplit;
     const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), cdiv(ub, kI4Warps)));
     const unsigned long long lim = g_wait_limit_ns.load();
     const int nt = kI4Warps * 32;
-#define MOE_I4_LAUNCH(G_, A_, O_) k_int4_stream<G_, A_, O_><<<grid, nt, kI4Smem, st>>>(tm, p, lim, xsum)
-    if (xsum != nullptr) {
-      if (!glu) MOE_I4_LAUNCH(false, kModePlain, true);
-      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true);
-      else MOE_I4_LAUNCH(true, kModeGeGLU, true);
+#define MOE_I4_LAUNCH(G_, A_, O_, S_) \
+  MOE_LAUNCH((k_int4_stream<G_, A_, O_, S_>), grid, nt, kI4Smem, st, tm, p, lim, xsum)
+    if (xsum != nullptr && p.ksplit > 1) {
+      if (!glu) MOE_I4_LAUNCH(false, kModePlain, true, true);
+      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true, true);
+      else MOE_I4_LAUNCH(true, kModeGeGLU, true, true);
+    } else if (xsum != nullptr) {
+      if (!glu) MOE_I4_LAUNCH(false, kModePlain, true, false);
+      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true, false);
+      else MOE_I4_LAUNCH(true, kModeGeGLU, true, false);
     } else {
-      if (!glu) MOE_I4_LAUNCH(false, kModePlain, false);
-      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, false);
-      else MOE_I4_LAUNCH(true, kModeGeGLU, false);
+      if (!glu) MOE_I4_LAUNCH(false, kModePlain, false, false);
+      else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, false, false);
+      else MOE_I4_LAUNCH(true, kModeGeGLU, false, false);
     }
 #undef MOE_I4_LAUNCH
     MOE_LAUNCH_CHECK();
+    if (p.ksplit > 1) {
+      const unsigned blocks = (unsigned)cdiv(R * N, 256);
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+      if (!glu) MOE_LAUNCH((k_int4_splitk_reduce<false, kModePlain>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+      else if (act == MOE_ACT_SWIGLU)
+        MOE_LAUNCH((k_int4_splitk_reduce<true, kModeSwiGLU>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+      else MOE_LAUNCH((k_int4_splitk_reduce<true, kModeGeGLU>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+      MOE_LAUNCH_CHECK();
+    }
     return MOE_OK;
   }
 }
@@ -462,6 +541,40 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
 }
 
 // Fused CUDA-core router when W_r^T fits in shared memory: returns its experts-per-lane template, else 0.
+// Lane-per-token router for E <= 16 (W_r^T as [d][EC] fp32 in shared memory, at most 160 KiB).  Wider
+// expert counts use the expert-per-lane router: every lane busy, no shared-memory bank conflicts.
+static int lanes_router_ec(const moe_shape* s) {
+  const int ec = s->E <= 8 ? 8 : s->E <= 16 ? 16 : 0;
+  if (ec == 0 || (size_t)s->d * ec * 4 > 160 * 1024) return 0;
+  return ec;
+}
+
+static int launch_lanes_router(const moe_shape* s, int ec, const void* x, const float* w_router, const float* bias,
+                               float* logits, int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st) {
+  // 4 lanes per token when one lane per token would leave SMs idle or the chains long (E * d FMAs each)
+  const int kp = (cdiv(s->T, 256) < 2 * num_sms() || (long long)ec * s->d > 4096) ? 4 : 1;
+  const size_t smem = (size_t)s->d * ec * 4;
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+#define MOE_LANES_CASE(N_, KP_)                                                                                    \
+  if (ec == N_ && kp == KP_) {                                                                                    \
+    static std::atomic<unsigned long long> done{0};                                                               \
+    if (!(done.load() & bit)) {                                                                                   \
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_lanes<N_, KP_>, cudaFuncAttributeMaxDynamicSharedMemorySize,      \
+                                        160 * 1024));                                                             \
+      done.fetch_or(bit);                                                                                         \
+    }                                                                                                             \
+    MOE_LAUNCH((k_router_lanes<N_, KP_>), (unsigned)cdiv(s->T, 256 / KP_), 256, smem, st, xb, w_router, bias,      \
+               logits, idx, w, cnt, psum, (int)s->T, s->d, s->E, s->k, s->renorm);                                \
+    MOE_LAUNCH_CHECK();                                                                                           \
+    return MOE_OK;                                                                                                \
+  }
+  MOE_LANES_CASE(8, 1) MOE_LANES_CASE(16, 1) MOE_LANES_CASE(8, 4) MOE_LANES_CASE(16, 4)
+#undef MOE_LANES_CASE
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
 static int fused_router_epl(const moe_shape* s) {
   if (s->E > 256) return 0;
   const int epl = s->E <= 32 ? 1 : s->E <= 64 ? 2 : s->E <= 128 ? 4 : 8;
@@ -484,7 +597,7 @@ static int launch_fused_router(const moe_shape* s, int epl, const void* x, const
                                         160 * 1024));                                                             \
       done.fetch_or(bit);                                                                                         \
     }                                                                                                             \
-    k_router_fused<N_, 8><<<nchunks, 256, smem, st>>>(xb, w_router, bias, logits, idx, w, cnt, psum, (int)s->T,    \
+    MOE_LAUNCH((k_router_fused<N_, 8>), nchunks, 256, smem, st, xb, w_router, bias, logits, idx, w, cnt, psum, (int)s->T,    \
                                                       s->d, s->E, s->k, s->renorm);                               \
     MOE_LAUNCH_CHECK();                                                                                           \
     return MOE_OK;                                                                                                \
@@ -516,13 +629,16 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   float* P = aux_p ? aux_p : reinterpret_cast<float*>(ws + L.fP) + s->E;
   int rc;
   int nsplit = 1;
+  const int ec_lanes = lanes_router_ec(s);
   const int epl_fused = fused_router_epl(s);
-  if (logits_in == nullptr && epl_fused > 0) {
+  if (logits_in == nullptr && ec_lanes > 0) {
+    rc = launch_lanes_router(s, ec_lanes, x, w_router, bias, logits, idx, w, cnt, psum, st);
+  } else if (logits_in == nullptr && epl_fused > 0) {
     rc = launch_fused_router(s, epl_fused, x, w_router, bias, logits, idx, w, cnt, psum, st);
   } else if (logits_in == nullptr && use_tc_router(s)) {
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
-    k_router_prep<<<(unsigned)cdiv(s->E, 8), 256, 0, st>>>(w_router, wsplit, wnorm, s->E, s->d);
+    MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d);
     MOE_LAUNCH_CHECK();
     rc = grouped_gemm(kModeF32, x, s->T, 3 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
                       bias);
@@ -538,7 +654,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       g_skinny_attr[dev] = 1;
     }
     dim3 grid((unsigned)cdiv(s->E, 8 * kSkExp), (unsigned)cdiv(s->T, kSkTok), kSkSplit);
-    k_router_skinny<<<grid, 256, skinny_smem(s->d), st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, part,
+    MOE_LAUNCH((k_router_skinny), grid, 256, skinny_smem(s->d), st, reinterpret_cast<const __nv_bfloat16*>(x), w_router, part,
                                                            (int)s->T, s->d, s->E);
     MOE_LAUNCH_CHECK();
     rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum, part, st);
@@ -546,7 +662,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     int kps = 0;
     nsplit = router_splits(s, &kps);
     dim3 grid((unsigned)cdiv(s->T, kLgBM), (unsigned)cdiv(s->E, kLgBN), (unsigned)nsplit);
-    k_router_logits<<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, part, (int)s->T,
+    MOE_LAUNCH((k_router_logits), grid, 128, 0, st, reinterpret_cast<const __nv_bfloat16*>(x), w_router, part, (int)s->T,
                                           s->d, s->E, kps);
     MOE_LAUNCH_CHECK();
     rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum, part, st);
@@ -558,7 +674,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   rc = launch_scan(s, cnt, want_fp ? psum : nullptr, counts, want_fp ? f : nullptr, want_fp ? P : nullptr, st);
   if (rc) return rc;
   if (aux) {
-    k_aux_finalize<<<1, 32, 0, st>>>(f, P, aux, s->E);
+    MOE_LAUNCH((k_aux_finalize), 1, 32, 0, st, f, P, aux, s->E);
     MOE_LAUNCH_CHECK();
   }
   return MOE_OK;
@@ -658,7 +774,7 @@ int moe_permute(const moe_shape* s, const void* x, const int32_t* topk_idx, int3
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   int32_t* cts = counts ? counts : reinterpret_cast<int32_t*>(ws + L.counts);
   const int nchunks = (int)cdiv(s->T, kChunk);
-  k_chunk_hist<<<nchunks, 256, s->E * sizeof(int), stream>>>(topk_idx, cnt, (int)s->T, s->E, s->k);
+  MOE_LAUNCH((k_chunk_hist), nchunks, 256, s->E * sizeof(int), stream, topk_idx, cnt, (int)s->T, s->E, s->k);
   MOE_LAUNCH_CHECK();
   rc = launch_scan(s, cnt, nullptr, cts, nullptr, nullptr, stream);
   if (rc) return rc;
@@ -698,7 +814,7 @@ int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos,
   const unsigned blocks = (unsigned)cdiv(s->T, 8);
 #define MOE_COMBINE_CASE(N_)                                                                                   \
   if (s->k <= N_) {                                                                                            \
-    k_combine<N_><<<blocks, 256, 0, stream>>>(yp, slot_pos, topk_w, ysh, o, (int)s->T, s->d, s->k);           \
+    MOE_LAUNCH((k_combine<N_>), blocks, 256, 0, stream, yp, slot_pos, topk_w, ysh, o, (int)s->T, s->d, s->k);           \
     MOE_LAUNCH_CHECK();                                                                                        \
     return MOE_OK;                                                                                             \
   }
@@ -742,7 +858,8 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream);
   if (rc) return rc;
   const Int4Scratch scr = s->wfmt == MOE_WFMT_INT4_G128
-                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq}
+                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq,
+                                            reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
                               : Int4Scratch{nullptr, nullptr};
   rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
   if (rc) return rc;
@@ -762,7 +879,7 @@ int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void*
     return MOE_INVALID_ARGUMENT;
   if (rows == 0) return MOE_OK;
   const long long items = rows * (K / 128);
-  k_quantize_int4<<<(unsigned)cdiv(items, 8), 256, 0, stream>>>(w, rows, K, q,
+  MOE_LAUNCH((k_quantize_int4), (unsigned)cdiv(items, 8), 256, 0, stream, w, rows, K, q,
                                                                  reinterpret_cast<__nv_bfloat16*>(scales));
   MOE_LAUNCH_CHECK();
   return MOE_OK;
@@ -786,6 +903,7 @@ int moe_get_status(moe_stream_t stream, int32_t* device_status, uint32_t* site) 
 namespace moe {
 // One mbarrier that nothing arrives on; the bounded wait must give up.
 __global__ void k_selftest_wait(unsigned long long limit_ns) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ __align__(8) uint64_t bar;
   __shared__ volatile int abort_flag;
   if (threadIdx.x == 0) {
@@ -799,7 +917,7 @@ __global__ void k_selftest_wait(unsigned long long limit_ns) {
 }  // namespace moe
 
 extern "C" int moe_selftest_wait_timeout(moe_stream_t stream) {
-  moe::k_selftest_wait<<<1, 32, 0, stream>>>(moe::g_wait_limit_ns.load());
+  MOE_LAUNCH((moe::k_selftest_wait), 1, 32, 0, stream, moe::g_wait_limit_ns.load());
   count_launch();
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR;
 }
@@ -855,7 +973,7 @@ extern "C" int moe_permute_noalloc(const moe_shape* s, const void* x, const int3
   if (rc) return rc;
   int32_t* cnt = scratch;                                   // fully rewritten by k_chunk_hist every call
   int32_t* cts = counts ? counts : scratch + kNoAllocHistInts;  // fully rewritten by k_chunk_scan
-  k_chunk_hist<<<(unsigned)nchunks, 256, s->E * sizeof(int), stream>>>(topk_idx, cnt, (int)s->T, s->E, s->k);
+  MOE_LAUNCH((k_chunk_hist), (unsigned)nchunks, 256, s->E * sizeof(int), stream, topk_idx, cnt, (int)s->T, s->E, s->k);
   MOE_LAUNCH_CHECK();
   rc = launch_scan(s, cnt, nullptr, cts, nullptr, nullptr, stream);
   if (rc) return rc;

@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict
                                                  uint8_t* __restrict__ drop, int32_t* __restrict__ row_src,
                                                  __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ kept_out,
                                                  int32_t* __restrict__ offsets_out) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_kept[kMaxE];
   __shared__ int s_tmp[4];
@@ -138,6 +139,7 @@ template <int KMAX>
 __global__ void __launch_bounds__(256) k_move_rows(const __nv_bfloat16* __restrict__ x,
                                                    const int32_t* __restrict__ slot_pos, int T, int d, int k,
                                                    __nv_bfloat16* __restrict__ x_perm) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int nvec = d >> 3;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)T * nvec) return;
@@ -156,6 +158,7 @@ __global__ void __launch_bounds__(256) k_move_rows(const __nv_bfloat16* __restri
 // used by moe_forward when only the tables are needed.  (kept, offsets)
 __global__ void __launch_bounds__(128) k_group_table(const int32_t* __restrict__ counts, int E, int cap,
                                                      int32_t* __restrict__ kept_out, int32_t* __restrict__ offsets_out) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_kept[kMaxE];
   __shared__ int s_tmp[4];
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
                                                  const int32_t* __restrict__ slot_pos, const float* __restrict__ w,
                                                  const __nv_bfloat16* __restrict__ y_shared,
                                                  __nv_bfloat16* __restrict__ out, int T, int d, int k) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int t = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   if (t >= T) return;

@@ -12,6 +12,7 @@ namespace moe {
 // One warp per (row, 128-input group); lane l owns inputs 4l .. 4l+3.
 __global__ void __launch_bounds__(256) k_quantize_int4(const float* __restrict__ w, long long rows, int K,
                                                        uint8_t* __restrict__ q, __nv_bfloat16* __restrict__ scales) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int groups = K / 128;
   const long long item = (long long)blockIdx.x * 8 + warp_id();
   if (item >= rows * groups) return;

@@ -29,6 +29,7 @@ constexpr int kLgBM = 128, kLgBN = 64, kLgBK = 32;
 __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __restrict__ x,
                                                        const float* __restrict__ W, float* __restrict__ part,
                                                        int T, int d, int E, int k_per_split) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ __align__(16) float As[kLgBK][kLgBM + 4];
   __shared__ __align__(16) float Bs[kLgBK][kLgBN + 4];
   const int m0 = blockIdx.x * kLgBM, n0 = blockIdx.y * kLgBN;
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
 __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
                                                      float* __restrict__ wnorm, int E, int d) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
   const float* wr = W + (size_t)e * d;
@@ -320,6 +322,7 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
                                                          int32_t* __restrict__ cnt, float* __restrict__ psum,
                                                          float* p_out, int T, int E, int k, int renorm,
                                                          const RefineArgs refine) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ float s_stat[];
   constexpr int TPW = STATS ? kChunk / NW : 1;
   const int lane = lane_id(), warp = warp_id();
@@ -451,6 +454,182 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
   }
 }
 
+// W_r [E][d] fp32 (global) -> shared memory as [d][pitch] (column e of row c =
+// W_r[e][c]; columns E..pitch-1 untouched).  Coalesced float4 reads, eight in
+// flight per thread before the transposed stores.  d % 4 == 0.
+__device__ __forceinline__ void load_wt_transposed(const float* __restrict__ W, int E, int d, float* s_wt, int pitch) {
+  const int n4 = E * d / 4;
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  for (int base = threadIdx.x; base < n4; base += 8 * blockDim.x) {
+    float4 r[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i4 = base + j * blockDim.x;
+      r[j] = i4 < n4 ? __ldg(W4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i4 = base + j * blockDim.x;
+      if (i4 < n4) {
+        const int e = (4 * i4) / d, c = 4 * i4 - e * d;
+        s_wt[(c + 0) * pitch + e] = r[j].x;
+        s_wt[(c + 1) * pitch + e] = r[j].y;
+        s_wt[(c + 2) * pitch + e] = r[j].z;
+        s_wt[(c + 3) * pitch + e] = r[j].w;
+      }
+    }
+  }
+}
+
+// Router fully in one kernel for few experts (E <= EC <= 32).  KP lanes share
+// one token (32 / KP tokens per warp, 256 / KP per CTA): lane part q takes the
+// 8-input slices q, q + KP, q + 2 KP, ... and keeps E fp32 FMA chains over them
+// in order; an xor tree over the KP lanes then gives every lane of the token
+// its full logits.  W_r^T sits in shared memory as [d][EC] fp32 and all lanes
+// read the same row at the same time (broadcast).  Top-k runs per token (k
+// ascending scans with a strict >: the lowest index wins ties), then softmax
+// and gates.  Chunk statistics: fixed xor trees over the warp's tokens, then
+// the KP warps of a 32-token chunk in warp order through shared memory.
+template <int EC, int KP>
+__global__ void __launch_bounds__(256) k_router_lanes(const __nv_bfloat16* __restrict__ x,
+                                                      const float* __restrict__ W, const float* __restrict__ bias,
+                                                      float* __restrict__ logits_out, int32_t* __restrict__ topk_idx,
+                                                      float* __restrict__ topk_w, int32_t* __restrict__ cnt,
+                                                      float* __restrict__ psum, int T, int d, int E, int k,
+                                                      int renorm) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  extern __shared__ __align__(16) float s_wt[];  // [d][EC]
+  __shared__ float s_ps[8][EC];
+  __shared__ int s_cn[8][EC];
+  load_wt_transposed(W, E, d, s_wt, EC);
+  for (int i = threadIdx.x; i < (EC - E) * d; i += blockDim.x) {   // zero columns E..EC-1
+    const int c = i / (EC - E), e = E + (i - c * (EC - E));
+    s_wt[c * EC + e] = 0.f;
+  }
+  __syncthreads();
+  constexpr int TPW = 32 / KP;                 // tokens per warp
+  const int lane = lane_id(), warp = warp_id();
+  const int q = lane % KP, tw = lane / KP;
+  const int t = blockIdx.x * (8 * TPW) + warp * TPW + tw;
+  const bool on = t < T;
+  float z[EC];
+#pragma unroll
+  for (int e = 0; e < EC; ++e) z[e] = 0.f;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(on ? t : 0) * d);
+  const int nv = d >> 3;
+  // the lane's 8-input slices q, q + KP, ...: four loads in flight, then their FMAs
+  for (int v0 = q; v0 < nv; v0 += 4 * KP) {
+    uint4 ub[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = v0 + j * KP;
+      ub[j] = (on && v < nv) ? __ldg(xr + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = v0 + j * KP;
+      if (v >= nv) break;
+      const uint4 u = ub[j];
+      const float xv[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                           bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4* wr = reinterpret_cast<const float4*>(s_wt + (size_t)(8 * v + i) * EC);
+#pragma unroll
+        for (int e4 = 0; e4 < EC / 4; ++e4) {
+          const float4 w4 = wr[e4];
+          z[4 * e4 + 0] = fmaf(xv[i], w4.x, z[4 * e4 + 0]);
+          z[4 * e4 + 1] = fmaf(xv[i], w4.y, z[4 * e4 + 1]);
+          z[4 * e4 + 2] = fmaf(xv[i], w4.z, z[4 * e4 + 2]);
+          z[4 * e4 + 3] = fmaf(xv[i], w4.w, z[4 * e4 + 3]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < KP; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < EC; ++e) z[e] += __shfl_xor_sync(0xffffffffu, z[e], o);
+  const bool lead = on && q == 0;   // the lane that writes the token's outputs
+  float m = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < EC; ++e) {
+    if (e < E) {
+      if (bias != nullptr) z[e] += bias[e];
+      m = fmaxf(m, z[e]);
+    } else {
+      z[e] = -INFINITY;
+    }
+  }
+  if (lead && logits_out != nullptr)
+    for (int e = 0; e < E; ++e) logits_out[(size_t)t * E + e] = z[e];
+  // softmax
+  float ez[EC], ssum = 0.f;
+#pragma unroll
+  for (int e = 0; e < EC; ++e) {
+    ez[e] = e < E ? expf(z[e] - m) : 0.f;
+    ssum += ez[e];
+  }
+  const float inv = 1.f / ssum;
+  // top-k: k scans in ascending index with a strict >, the picked entries masked
+  uint32_t taken = 0u;
+  float wsum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = 0.f;
+    int bi = -1;
+#pragma unroll
+    for (int e = 0; e < EC; ++e)
+      if (e < E && !((taken >> e) & 1u) && (bi < 0 || z[e] > bv)) {
+        bv = z[e];
+        bi = e;
+      }
+    taken |= 1u << bi;
+    float pj = 0.f;
+#pragma unroll
+    for (int e = 0; e < EC; ++e)
+      if (e == bi) pj = ez[e] * inv;
+    wsum += pj;
+    if (lead) {
+      topk_idx[(size_t)t * k + j] = bi;
+      topk_w[(size_t)t * k + j] = pj;
+    }
+  }
+  if (lead && renorm) {
+    const float r = 1.f / wsum;
+    for (int j = 0; j < k; ++j) topk_w[(size_t)t * k + j] *= r;
+  }
+  // chunk statistics: this warp's tokens (one lane each), then the chunk's KP warps in order
+#pragma unroll
+  for (int e = 0; e < EC; ++e) {
+    if (e >= E) break;
+    float pe = lead ? ez[e] * inv : 0.f;
+#pragma unroll
+    for (int o = KP; o < 32; o <<= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
+    const int ce = __popc(__ballot_sync(0xffffffffu, lead && ((taken >> e) & 1u)));
+    if (lane == 0) {
+      s_ps[warp][e] = pe;
+      s_cn[warp][e] = ce;
+    }
+  }
+  __syncthreads();
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  constexpr int CPB = 8 / KP;                 // chunks per CTA
+  for (int i = threadIdx.x; i < CPB * E; i += blockDim.x) {
+    const int cl = i / E, e = i - cl * E;
+    const int chunk = blockIdx.x * CPB + cl;
+    if (chunk >= nchunks) continue;
+    float ps = 0.f;
+    int cs = 0;
+#pragma unroll
+    for (int w = 0; w < KP; ++w) {
+      ps += s_ps[cl * KP + w][e];
+      cs += s_cn[cl * KP + w][e];
+    }
+    psum[(size_t)e * nchunks + chunk] = ps;
+    cnt[(size_t)e * nchunks + chunk] = cs;
+  }
+}
+
 // Router fully in one kernel for small E * d: the CTA keeps W_r^T in shared
 // memory ([d][32 EPL + 1] fp32, padded against bank conflicts); each warp
 // computes its tokens' logits as plain fp32 FMA chains over the inputs (lane l
@@ -464,14 +643,12 @@ __global__ void __launch_bounds__(NW * 32) k_router_fused(const __nv_bfloat16* _
                                                           int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                                           int32_t* __restrict__ cnt, float* __restrict__ psum, int T,
                                                           int d, int E, int k, int renorm) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ float s_wt[];
   __shared__ float s_p[NW][EPL * 32];
   __shared__ int s_c[NW][EPL * 32];
   constexpr int EP = EPL * 32 + 1;
-  for (int i = threadIdx.x; i < E * d; i += blockDim.x) {  // coalesced reads; odd row pitch: no bank conflicts
-    const int e = i / d, c = i - e * d;
-    s_wt[c * EP + e] = W[i];
-  }
+  load_wt_transposed(W, E, d, s_wt, EP);   // odd row pitch: no bank conflicts in the compute loop
   __syncthreads();
   const int lane = lane_id(), warp = warp_id();
   const int chunk = blockIdx.x;
@@ -561,6 +738,7 @@ __host__ __device__ constexpr int skinny_slice(int d) {
 __global__ void __cluster_dims__(1, 1, kSkSplit) __launch_bounds__(256, 2) k_router_skinny(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ W, float* __restrict__ logits,
                                                           int T, int d, int E) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ __align__(16) float s_x[];      // [kSkTok][ks]
   __shared__ float s_tile[kSkTok][8 * kSkExp];      // this CTA's partial [token][expert]
   cg::cluster_group cluster = cg::this_cluster();
@@ -656,6 +834,7 @@ __global__ void __cluster_dims__(1, 1, kSkSplit) __launch_bounds__(256, 2) k_rou
 // Per-chunk expert histogram from caller routing (moe_permute without moe_route).
 __global__ void __launch_bounds__(256) k_chunk_hist(const int32_t* __restrict__ topk_idx, int32_t* __restrict__ cnt,
                                                     int T, int E, int k) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ int s_h[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_h[e] = 0;
   __syncthreads();
@@ -675,6 +854,7 @@ __global__ void __launch_bounds__(256) k_chunk_hist(const int32_t* __restrict__ 
 __global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__ topk_idx,
                                                      const float* __restrict__ p, int32_t* __restrict__ cnt,
                                                      float* __restrict__ psum, int T, int E, int k) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ int s_h[kMaxRouterE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_h[e] = 0;
   __syncthreads();
@@ -698,6 +878,7 @@ __global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__
 __global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, const float* __restrict__ psum,
                                                     int32_t* __restrict__ counts, float* __restrict__ f_out,
                                                     float* __restrict__ p_out, int nchunks, int E, int T) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int e = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   if (e >= E) return;
@@ -705,18 +886,29 @@ __global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, c
   const float* prow = psum != nullptr ? psum + (size_t)e * nchunks : nullptr;
   int run = 0;
   float ps = 0.f;
-  for (int c0 = 0; c0 < nchunks; c0 += 32) {
-    const int c = c0 + lane;
-    const int v = c < nchunks ? row[c] : 0;
-    if (prow != nullptr && c < nchunks) ps += prow[c];
-    int incl = v;
+  // eight 32-chunk rows per round: their loads are all in flight before the scans
+  for (int c0 = 0; c0 < nchunks; c0 += 8 * 32) {
+    int v[8];
+    float pv[8];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + 32 * j + lane;
+      v[j] = c < nchunks ? row[c] : 0;
+      pv[j] = (prow != nullptr && c < nchunks) ? prow[c] : 0.f;
     }
-    if (c < nchunks) row[c] = run + incl - v;
-    run += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + 32 * j + lane;
+      ps += pv[j];
+      int incl = v[j];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (c < nchunks) row[c] = run + incl - v[j];
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
   if (prow != nullptr) {
 #pragma unroll
@@ -732,6 +924,7 @@ __global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, c
 // aux = E * sum_e f_e P_e, one warp, fixed order.
 __global__ void k_aux_finalize(const float* __restrict__ f, const float* __restrict__ P, float* __restrict__ aux,
                                int E) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   float s = 0.f;
   for (int e = lane_id(); e < E; e += 32) s += f[e] * P[e];
 #pragma unroll

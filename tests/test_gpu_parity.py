@@ -63,11 +63,13 @@ def _route_case(moe, wl, T, seed):
     return wl, inp, r, ref, x64, W64, b64
 
 
-# Router paths: fused shared-memory router (tiny, small, geglu), certified tensor-core router (skewed,
-# granular shapes), weight-streaming decode router (decode_int4; T <= 256: one token, a ragged token
-# block with E = 200 and a ragged last input slice with d = 784), split-K CUDA-core router (E = 200,
-# which is neither a multiple of 16 nor small enough for the fused router).
-@pytest.mark.parametrize("name,T,over", [("tiny", 256, {}), ("small", 4096, {}), ("skewed", 3000, {}),
+# Router paths: lane-per-token router for E <= 32 (tiny, small, geglu, E = 13), shared-memory router for
+# 32 < E <= 256 with a small W_r (E = 64), certified tensor-core router (skewed, granular shapes),
+# weight-streaming decode router (decode_int4; T <= 256: one token, a ragged token block with E = 200
+# and a ragged last input slice with d = 784), split-K CUDA-core router (E = 200, which is neither a
+# multiple of 16 nor small enough for the shared-memory router).
+@pytest.mark.parametrize("name,T,over", [("tiny", 256, {}), ("small", 4096, {}), ("tiny", 300, {"E": 13}),
+                                         ("small", 1000, {"E": 64, "k": 4}), ("skewed", 3000, {}),
                                          ("geglu", 2000, {}), ("decode_int4", 64, {}), ("decode_int4", 1, {}),
                                          ("granular", 37, {"E": 200, "d": 784}),
                                          ("granular", 1000, {"E": 200}), ("decode_int4", 300, {"E": 96})])
