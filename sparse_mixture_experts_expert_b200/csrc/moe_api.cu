@@ -156,7 +156,7 @@ static Workspace ws_layout(const moe_shape* s) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   L.part = take((size_t)ns * s->T * s->E * 4);
-  L.wsplit = take((size_t)3 * s->E * s->d * 2);
+  L.wsplit = take((size_t)2 * s->E * s->d * 2);
   L.wnorm = take((size_t)s->E * 4);
   const long long xs_rows = std::max<long long>(grouped_rows(s), s->T);
   const int xs_cols = std::max(s->d, std::max(s->H, s->H_s));
@@ -376,7 +376,7 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
 static int launch_scan(const moe_shape* s, int32_t* cnt, const float* psum, int32_t* counts, float* f, float* P,
                        cudaStream_t st) {
   const int nchunks = (int)cdiv(s->T, kChunk);
-  MOE_LAUNCH((k_chunk_scan), (int)cdiv(s->E, 8), 256, 0, st, cnt, psum, counts, f, P, nchunks, s->E, (int)s->T);
+  MOE_LAUNCH((k_chunk_scan), s->E, 256, 0, st, cnt, psum, counts, f, P, nchunks, s->E, (int)s->T);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -541,11 +541,11 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
 }
 
 // Fused CUDA-core router when W_r^T fits in shared memory: returns its experts-per-lane template, else 0.
-// Lane-per-token router for E <= 16 (W_r^T as [d][EC] fp32 in shared memory, at most 160 KiB).  Wider
+// Lane-per-token router for E <= 16 (W_r^T as [d][EC + 4] fp32 in shared memory, at most 160 KiB).  Wider
 // expert counts use the expert-per-lane router: every lane busy, no shared-memory bank conflicts.
 static int lanes_router_ec(const moe_shape* s) {
   const int ec = s->E <= 8 ? 8 : s->E <= 16 ? 16 : 0;
-  if (ec == 0 || (size_t)s->d * ec * 4 > 160 * 1024) return 0;
+  if (ec == 0 || (size_t)s->d * (ec + 4) * 4 > 160 * 1024) return 0;
   return ec;
 }
 
@@ -553,7 +553,7 @@ static int launch_lanes_router(const moe_shape* s, int ec, const void* x, const 
                                float* logits, int32_t* idx, float* w, int32_t* cnt, float* psum, cudaStream_t st) {
   // 4 lanes per token when one lane per token would leave SMs idle or the chains long (E * d FMAs each)
   const int kp = (cdiv(s->T, 256) < 2 * num_sms() || (long long)ec * s->d > 4096) ? 4 : 1;
-  const size_t smem = (size_t)s->d * ec * 4;
+  const size_t smem = (size_t)s->d * (ec + 4) * 4;
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   const int dev = current_device();
   const unsigned long long bit = 1ull << (dev & 63);
@@ -640,12 +640,16 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
     MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d);
     MOE_LAUNCH_CHECK();
-    rc = grouped_gemm(kModeF32, x, s->T, 3 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
+    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
                       bias);
     if (rc) return rc;
-    // screening bound: fp32 accumulation of 3d products (any rounding direction) plus the bias add
+    // screening bound, relative to ||x_t|| max_e ||w_e|| (>= sum |x_i w_i|): the split's representation error
+    // 2^-16, fp32 accumulation of 2d products in any rounding direction plus the bias add, and the error of the
+    // exact recompute's own d-term fp32 chain; all with a 2^-7 margin
     RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d,
-                   (float)((3.0 * s->d + 2.0) * std::ldexp(1.0, -23) * (1.0 + std::ldexp(1.0, -7)))};
+                   (float)((std::ldexp(1.0, -16) + (2.0 * s->d + 2.0) * std::ldexp(1.0, -23) +
+                            (s->d + 2.0) * std::ldexp(1.0, -24)) *
+                           (1.0 + std::ldexp(1.0, -7)))};
     rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
   } else if (logits_in == nullptr && s->T <= 256 && skinny_smem(s->d) <= kSkinnyMaxSmem) {
     const int dev = current_device();

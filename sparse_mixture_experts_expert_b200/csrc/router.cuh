@@ -112,9 +112,10 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 // ---------------------------------------------------------------------------
 // Router weight preparation for the tensor-core screening pass, one warp per
 // expert row:
-//  * exact three-way bf16 split W = hi + mid + lo (24 significand bits = 3 x 8),
-//    written as one [E, 3d] bf16 operand [hi | mid | lo]; x is bf16, so every
-//    product x * part is exact in fp32 and x W^T = [x | x | x] [hi | mid | lo]^T;
+//  * two-term bf16 split W ~ hi + lo (hi = bf16(w), lo = bf16(w - hi): 16
+//    significand bits, |w - hi - lo| <= 2^-16 |w|), written as one [E, 2d] bf16
+//    operand [hi | lo]; x is bf16, so every product x * part is exact in fp32
+//    and the screening logits are [x | x] [hi | lo]^T;
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
 __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
                                                      float* __restrict__ wnorm, int E, int d) {
@@ -122,17 +123,13 @@ __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
   const float* wr = W + (size_t)e * d;
-  __nv_bfloat16* row = Ws + (size_t)e * 3 * d;
+  __nv_bfloat16* row = Ws + (size_t)e * 2 * d;
   float ss = 0.f;
   for (int k = lane_id(); k < d; k += 32) {
     const float w = wr[k];
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
     row[k] = hi;
-    row[d + k] = mid;
-    row[2 * d + k] = __float2bfloat16_rn(r2);
+    row[d + k] = __float2bfloat16_rn(w - __bfloat162float(hi));
     ss = fmaf(w, w, ss);
   }
 #pragma unroll
@@ -386,6 +383,10 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float bound = refine.gamma * sqrtf(ss) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
       const float thr = kth - 2.f * bound;
+      // candidate c (in expert order) is parked in lane c: exact value cv, index ci
+      int nc = 0;
+      float cv = -INFINITY;
+      int ci = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         unsigned cand = __ballot_sync(0xffffffffu, lane + 32 * i < E && z[i] >= thr);
@@ -398,9 +399,33 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
           else v = warp_dot(xr, refine.W + (size_t)e * refine.d, refine.d);
           if (refine.bias != nullptr) v += refine.bias[e];
           if (lane == l) z[i] = v;
+          if (lane == nc) { cv = v; ci = e; }
+          ++nc;
         }
       }
-      kth = warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
+      if (nc <= 32) {
+        // The exact top k lies among the candidates: rank them by (value desc, index asc) with shuffles
+        // instead of another k rounds over all experts.
+        int rank = 0;
+        for (int j = 0; j < nc; ++j) {
+          const float vj = __shfl_sync(0xffffffffu, cv, j);
+          const int ij = __shfl_sync(0xffffffffu, ci, j);
+          rank += (vj > cv || (vj == cv && ij < ci)) ? 1 : 0;
+        }
+        for (int j = 0; j < nc; ++j) {
+          const int rj = __shfl_sync(0xffffffffu, rank, j);
+          const float vj = __shfl_sync(0xffffffffu, cv, j);
+          const int ij = __shfl_sync(0xffffffffu, ci, j);
+          if (lane == rj) { sel_v = vj; sel_i = ij; }
+        }
+        taken = 0u;
+        for (int j = 0; j < k; ++j) {
+          const int e = __shfl_sync(0xffffffffu, sel_i, j);
+          if ((e & 31) == lane) taken |= 1u << (e >> 5);
+        }
+      } else {
+        kth = warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
+      }
     }
     if (logits_out != nullptr) {
 #pragma unroll
@@ -481,12 +506,14 @@ __device__ __forceinline__ void load_wt_transposed(const float* __restrict__ W, 
   }
 }
 
-// Router fully in one kernel for few experts (E <= EC <= 32).  KP lanes share
+// Router fully in one kernel for few experts (E <= EC <= 16).  KP lanes share
 // one token (32 / KP tokens per warp, 256 / KP per CTA): lane part q takes the
-// 8-input slices q, q + KP, q + 2 KP, ... and keeps E fp32 FMA chains over them
-// in order; an xor tree over the KP lanes then gives every lane of the token
-// its full logits.  W_r^T sits in shared memory as [d][EC] fp32 and all lanes
-// read the same row at the same time (broadcast).  Top-k runs per token (k
+// input pairs (2w, 2w + 1) for w = q, q + KP, q + 2 KP, ... and keeps E fp32
+// FMA chains over them in order; an xor tree over the KP lanes then gives
+// every lane of the token its full logits.  W_r^T sits in shared memory as
+// [d][EC + 4] fp32: the lanes of a token read rows 2 apart, which the padded
+// pitch puts in different banks, and the tokens of a warp read the same rows
+// (broadcast).  Top-k runs per token (k
 // ascending scans with a strict >: the lowest index wins ties), then softmax
 // and gates.  Chunk statistics: fixed xor trees over the warp's tokens, then
 // the KP warps of a 32-token chunk in warp order through shared memory.
@@ -501,10 +528,11 @@ __global__ void __launch_bounds__(256) k_router_lanes(const __nv_bfloat16* __res
   extern __shared__ __align__(16) float s_wt[];  // [d][EC]
   __shared__ float s_ps[8][EC];
   __shared__ int s_cn[8][EC];
-  load_wt_transposed(W, E, d, s_wt, EC);
+  constexpr int PW = EC + 4;   // row pitch (floats)
+  load_wt_transposed(W, E, d, s_wt, PW);
   for (int i = threadIdx.x; i < (EC - E) * d; i += blockDim.x) {   // zero columns E..EC-1
     const int c = i / (EC - E), e = E + (i - c * (EC - E));
-    s_wt[c * EC + e] = 0.f;
+    s_wt[c * PW + e] = 0.f;
   }
   __syncthreads();
   constexpr int TPW = 32 / KP;                 // tokens per warp
@@ -515,34 +543,38 @@ __global__ void __launch_bounds__(256) k_router_lanes(const __nv_bfloat16* __res
   float z[EC];
 #pragma unroll
   for (int e = 0; e < EC; ++e) z[e] = 0.f;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(on ? t : 0) * d);
-  const int nv = d >> 3;
-  // the lane's 8-input slices q, q + KP, ...: four loads in flight, then their FMAs
-  for (int v0 = q; v0 < nv; v0 += 4 * KP) {
-    uint4 ub[4];
+  const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + (size_t)(on ? t : 0) * d);
+  const int nw = d >> 1;
+  // the lane's input pairs w = q, q + KP, ...: four loads in flight, then their FMAs
+  for (int w0 = q; w0 < nw; w0 += 4 * KP) {
+    uint32_t ub[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int v = v0 + j * KP;
-      ub[j] = (on && v < nv) ? __ldg(xr + v) : make_uint4(0, 0, 0, 0);
+      const int w = w0 + j * KP;
+      ub[j] = (on && w < nw) ? __ldg(xw + w) : 0u;
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int v = v0 + j * KP;
-      if (v >= nv) break;
-      const uint4 u = ub[j];
-      const float xv[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
-                           bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+      const int w = w0 + j * KP;
+      if (w >= nw) break;
+      const float x0 = bf16lo(ub[j]), x1 = bf16hi(ub[j]);
+      const float4* r0 = reinterpret_cast<const float4*>(s_wt + (size_t)(2 * w) * PW);
+      const float4* r1 = reinterpret_cast<const float4*>(s_wt + (size_t)(2 * w + 1) * PW);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4* wr = reinterpret_cast<const float4*>(s_wt + (size_t)(8 * v + i) * EC);
+      for (int e4 = 0; e4 < EC / 4; ++e4) {
+        const float4 a4 = r0[e4];
+        z[4 * e4 + 0] = fmaf(x0, a4.x, z[4 * e4 + 0]);
+        z[4 * e4 + 1] = fmaf(x0, a4.y, z[4 * e4 + 1]);
+        z[4 * e4 + 2] = fmaf(x0, a4.z, z[4 * e4 + 2]);
+        z[4 * e4 + 3] = fmaf(x0, a4.w, z[4 * e4 + 3]);
+      }
 #pragma unroll
-        for (int e4 = 0; e4 < EC / 4; ++e4) {
-          const float4 w4 = wr[e4];
-          z[4 * e4 + 0] = fmaf(xv[i], w4.x, z[4 * e4 + 0]);
-          z[4 * e4 + 1] = fmaf(xv[i], w4.y, z[4 * e4 + 1]);
-          z[4 * e4 + 2] = fmaf(xv[i], w4.z, z[4 * e4 + 2]);
-          z[4 * e4 + 3] = fmaf(xv[i], w4.w, z[4 * e4 + 3]);
-        }
+      for (int e4 = 0; e4 < EC / 4; ++e4) {
+        const float4 b4 = r1[e4];
+        z[4 * e4 + 0] = fmaf(x1, b4.x, z[4 * e4 + 0]);
+        z[4 * e4 + 1] = fmaf(x1, b4.y, z[4 * e4 + 1]);
+        z[4 * e4 + 2] = fmaf(x1, b4.z, z[4 * e4 + 2]);
+        z[4 * e4 + 3] = fmaf(x1, b4.w, z[4 * e4 + 3]);
       }
     }
   }
@@ -871,57 +903,70 @@ __global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// Chunk tables are expert-major: cnt[e][c], psum[e][c].  One warp per expert:
+// Chunk tables are expert-major: cnt[e][c], psum[e][c].  One CTA of 8 warps per
+// expert, each warp owning a contiguous run of 32-chunk rows:
 // cnt[e][c] -> exclusive prefix over chunks (in place), counts[e]; optional
-// f[e] = counts/T and P[e] = sum_c psum[e][c] / T (lanes in order, then a fixed
-// xor tree).  Lanes read 32 consecutive chunks at a time (coalesced).
+// f[e] = counts/T and P[e] = sum_c psum[e][c] / T (per lane in chunk order, a
+// fixed xor tree per warp, then the warps in order).
 __global__ void __launch_bounds__(256) k_chunk_scan(int32_t* __restrict__ cnt, const float* __restrict__ psum,
                                                     int32_t* __restrict__ counts, float* __restrict__ f_out,
                                                     float* __restrict__ p_out, int nchunks, int E, int T) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  const int e = blockIdx.x * 8 + warp_id();
-  const int lane = lane_id();
-  if (e >= E) return;
+  __shared__ int s_tot[8];
+  __shared__ float s_ps[8];
+  const int e = blockIdx.x;
+  const int lane = lane_id(), warp = warp_id();
   int32_t* row = cnt + (size_t)e * nchunks;
   const float* prow = psum != nullptr ? psum + (size_t)e * nchunks : nullptr;
-  int run = 0;
+  const int nrows = (nchunks + 31) / 32;
+  const int rpw = (nrows + 7) / 8;
+  const int r0 = min(nrows, warp * rpw), r1 = min(nrows, r0 + rpw);
+  // pass 1: this warp's total and probability sum (loads of all its rows in flight together)
+  int wt = 0;
   float ps = 0.f;
-  // eight 32-chunk rows per round: their loads are all in flight before the scans
-  for (int c0 = 0; c0 < nchunks; c0 += 8 * 32) {
-    int v[8];
-    float pv[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = c0 + 32 * j + lane;
-      v[j] = c < nchunks ? row[c] : 0;
-      pv[j] = (prow != nullptr && c < nchunks) ? prow[c] : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = c0 + 32 * j + lane;
-      ps += pv[j];
-      int incl = v[j];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
-      }
-      if (c < nchunks) row[c] = run + incl - v[j];
-      run += __shfl_sync(0xffffffffu, incl, 31);
+  for (int r = r0; r < r1; ++r) {
+    const int c = r * 32 + lane;
+    if (c < nchunks) {
+      wt += row[c];
+      if (prow != nullptr) ps += prow[c];
     }
   }
-  if (prow != nullptr) {
+  wt = (int)__reduce_add_sync(0xffffffffu, (unsigned)wt);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-  }
+  for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
   if (lane == 0) {
-    if (counts != nullptr) counts[e] = run;
-    if (f_out != nullptr) f_out[e] = (float)run / (float)T;
-    if (p_out != nullptr && prow != nullptr) p_out[e] = ps / (float)T;
+    s_tot[warp] = wt;
+    s_ps[warp] = ps;
+  }
+  __syncthreads();
+  int run = 0;
+  for (int w = 0; w < warp; ++w) run += s_tot[w];
+  // pass 2: exclusive scan of the warp's rows (re-read from cache), offset by the earlier warps
+  for (int r = r0; r < r1; ++r) {
+    const int c = r * 32 + lane;
+    const int v = c < nchunks ? row[c] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (c < nchunks) row[c] = run + incl - v;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (threadIdx.x == 0) {
+    int total = 0;
+    float pt = 0.f;
+    for (int w = 0; w < 8; ++w) {
+      total += s_tot[w];
+      pt += s_ps[w];
+    }
+    if (counts != nullptr) counts[e] = total;
+    if (f_out != nullptr) f_out[e] = (float)total / (float)T;
+    if (p_out != nullptr && prow != nullptr) p_out[e] = pt / (float)T;
   }
 }
 
-// aux = E * sum_e f_e P_e, one warp, fixed order.
 __global__ void k_aux_finalize(const float* __restrict__ f, const float* __restrict__ P, float* __restrict__ aux,
                                int E) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
