@@ -30,6 +30,10 @@ if ROOT not in sys.path:
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor-core or HBM roofline"
 DEFAULT_WORKLOAD = "small"
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the expert GEMM launches of one forward, from an
+# `ncu --set full --clock-control none -k regex:k_grouped_gemm` capture of `bench.py --workload <name> --steps 1
+# --warmup 3 --no-cpu-baseline` on the current kernels; workloads without a complete capture report null.
+GEMM_TRAFFIC_BYTES = {"small": 12628736 + 21004032}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -442,7 +446,8 @@ def main():
         peak_tf = peaks["bf16_tflops"]
         roofline = {"bound": "tensor", "kernel": "k_grouped_gemm (gate/up + GLU, down; routed + shared)",
                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
-                    "peak_source": peaks["source"] + " burst bf16", "traffic": None,
+                    "peak_source": peaks["source"] + " burst bf16",
+                    "traffic": None if args.experts else GEMM_TRAFFIC_BYTES.get(wl.name),
                     "alg_flops_per_step": flops, "gemm_us": gemm_us}
 
     if rank == 0:

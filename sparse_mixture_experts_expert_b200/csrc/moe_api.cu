@@ -366,7 +366,8 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   }
 #define MOE_TOPK_EPL(NW_, XR_, ST_)                                                                               \
   MOE_TOPK_CASE(1, NW_, XR_, ST_) MOE_TOPK_CASE(2, NW_, XR_, ST_) MOE_TOPK_CASE(4, NW_, XR_, ST_)                 \
-  MOE_TOPK_CASE(8, NW_, XR_, ST_) MOE_TOPK_CASE(16, NW_, XR_, ST_)
+  MOE_TOPK_CASE(6, NW_, XR_, ST_) MOE_TOPK_CASE(8, NW_, XR_, ST_) MOE_TOPK_CASE(12, NW_, XR_, ST_)                \
+  MOE_TOPK_CASE(16, NW_, XR_, ST_)
   MOE_TOPK_EPL(8, false, true) MOE_TOPK_EPL(8, true, true) MOE_TOPK_EPL(4, false, false) MOE_TOPK_EPL(4, true, false)
 #undef MOE_TOPK_EPL
 #undef MOE_TOPK_CASE

@@ -122,15 +122,33 @@ __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
-  const float* wr = W + (size_t)e * d;
+  const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
   __nv_bfloat16* row = Ws + (size_t)e * 2 * d;
   float ss = 0.f;
-  for (int k = lane_id(); k < d; k += 32) {
-    const float w = wr[k];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    row[k] = hi;
-    row[d + k] = __float2bfloat16_rn(w - __bfloat162float(hi));
-    ss = fmaf(w, w, ss);
+  // float4 per lane, four loads in flight per round (d % 16 == 0)
+  for (int v0 = lane_id(); v0 < d / 4; v0 += 128) {
+    float4 wv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wv[j] = v0 + 32 * j < d / 4 ? __ldg(wr + v0 + 32 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int v = v0 + 32 * j;
+      if (v >= d / 4) break;
+      const float w4[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+      uint32_t hi2[2], lo2[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(w4[2 * h], w4[2 * h + 1]);
+        const __nv_bfloat162 lo =
+            __floats2bfloat162_rn(w4[2 * h] - __low2float(hi), w4[2 * h + 1] - __high2float(hi));
+        hi2[h] = *reinterpret_cast<const uint32_t*>(&hi);
+        lo2[h] = *reinterpret_cast<const uint32_t*>(&lo);
+      }
+      reinterpret_cast<uint2*>(row)[v] = make_uint2(hi2[0], hi2[1]);
+      reinterpret_cast<uint2*>(row + d)[v] = make_uint2(lo2[0], lo2[1]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ss = fmaf(w4[q], w4[q], ss);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -270,6 +288,35 @@ __device__ __forceinline__ float warp_topk(const float (&z)[EPL], int E, int k, 
   return kth;
 }
 
+// The k-th largest of the lanes' logits (with multiplicity), without the
+// indices: k rounds of a warp max, each removing one holder of the maximum.
+template <int EPL>
+__device__ __forceinline__ float warp_kth(const float (&z)[EPL], int E, int k) {
+  const int lane = lane_id();
+  unsigned used = 0u;
+  float kth = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    float lm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (lane + 32 * i < E && !((used >> i) & 1u)) lm = fmaxf(lm, z[i]);
+    float m;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(lm));
+    const unsigned holders = __ballot_sync(0xffffffffu, lm == m);
+    if (lane == __ffs(holders) - 1) {
+      bool done = false;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (!done && lane + 32 * i < E && !((used >> i) & 1u) && z[i] == m) {
+          used |= 1u << i;
+          done = true;
+        }
+    }
+    kth = m;
+  }
+  return kth;
+}
+
 // Exact fp32 logit of one (token, expert) pair with the token's inputs held in
 // registers as fp32 (xf[8q + i] = x[8 (lane + 32 q) + i], d <= 1024): the same
 // per-lane order and xor tree as warp_dot, without the bf16 unpacking.
@@ -353,7 +400,8 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
     float sel_v = 0.f;
     int sel_i = 0;
     unsigned taken;
-    float kth = warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
+    // with the certified recompute only the k-th screening value is needed here: the picks come later
+    float kth = refine.x != nullptr ? warp_kth<EPL>(z, E, k) : warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
     if (refine.x != nullptr) {
       const __nv_bfloat16* xr = refine.x + (size_t)t * refine.d;
       float ss = 0.f;
@@ -438,7 +486,7 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
     float ez[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      ez[i] = (lane + 32 * i < E) ? expf(z[i] - m) : 0.f;
+      ez[i] = (lane + 32 * i < E) ? __expf(z[i] - m) : 0.f;
       ssum += ez[i];
     }
 #pragma unroll
@@ -456,7 +504,7 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
         }
       }
     }
-    const float pj = lane < k ? expf(sel_v - m) * inv : 0.f;
+    const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
     float wsum = pj;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
