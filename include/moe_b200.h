@@ -119,6 +119,13 @@ int moe_workspace_size(const moe_shape* s, size_t* bytes);
  *   counts   [E] int32                   out  tokens choosing each expert
  *   aux_f, aux_p [E] fp32 or NULL        out  counts/T and mean softmax probability
  *   aux      [1] fp32 or NULL            out  E * sum_e f_e P_e
+ * Logit precision: fp32 FMA dot products over the inputs in order.  For large
+ * T * E * d the logits are first screened on the tensor cores (two-term bf16
+ * split of W_r, fp32 accumulation) and every expert that can reach the top k
+ * under the screen's error bound, (2^-16 + (2d+2) 2^-23 + (d+2) 2^-24)(1 + 2^-7)
+ * ||x_t|| max_e ||w_e||, is recomputed as an fp32 FMA dot product; the picks
+ * and their gates then come from those values, and the other entries of
+ * `logits` are the screened values (within that bound).
  * Deterministic: identical inputs give bit-identical outputs.
  */
 int moe_route(const moe_shape* s, const void* x, const float* w_router, const float* bias, float* logits,

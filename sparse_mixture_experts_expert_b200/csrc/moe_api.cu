@@ -384,7 +384,8 @@ static int launch_scan(const moe_shape* s, int32_t* cnt, const float* psum, int3
 
 static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx, const int32_t* cbase,
                           const int32_t* counts, int32_t* slot, uint8_t* drop, int32_t* row_src, void* x_perm,
-                          int32_t* kept, int32_t* offs, cudaStream_t st, bool move_rows = true) {
+                          int32_t* kept, int32_t* offs, cudaStream_t st, bool move_rows = true,
+                          const float* aux_f = nullptr, const float* aux_p = nullptr, float* aux = nullptr) {
   const int nchunks = (int)cdiv(s->T, kChunk);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   __nv_bfloat16* xp = reinterpret_cast<__nv_bfloat16*>(x_perm);
@@ -393,7 +394,7 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   if (s->k <= N_) {                                                                                           \
     MOE_LAUNCH((k_scatter<N_>), (unsigned)cdiv(nchunks, 4), 128, 0, st, xb, idx, cbase, counts, (int)s->T, s->d, s->E,   \
                                                               s->k, s->capacity,                              \
-                                           slot, drop, row_src, xp, kept, offs);                              \
+                                           slot, drop, row_src, xp, kept, offs, aux_f, aux_p, aux);           \
     MOE_LAUNCH_CHECK();                                                                                       \
     if (move_rows) {                                                                                          \
       MOE_LAUNCH((k_move_rows<N_>), mv_blocks, 256, 0, st, xb, slot, (int)s->T, s->d, s->k, xp);                       \
@@ -621,7 +622,7 @@ static bool use_tc_router(const moe_shape* s) {
 
 static int route_impl(const moe_shape* s, const void* x, const float* w_router, const float* bias,
                       const float* logits_in, float* logits, int32_t* idx, float* w, int32_t* counts, float* aux_f,
-                      float* aux_p, float* aux, uint8_t* ws, cudaStream_t st) {
+                      float* aux_p, float* aux, uint8_t* ws, cudaStream_t st, bool defer_aux = false) {
   const Workspace L = ws_layout(s);
   float* part = reinterpret_cast<float*>(ws + L.part);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
@@ -678,7 +679,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   const bool want_fp = aux_f || aux_p || aux;
   rc = launch_scan(s, cnt, want_fp ? psum : nullptr, counts, want_fp ? f : nullptr, want_fp ? P : nullptr, st);
   if (rc) return rc;
-  if (aux) {
+  if (aux && !defer_aux) {   // deferred: the caller's grouping kernel forms aux from f and P
     MOE_LAUNCH((k_aux_finalize), 1, 32, 0, st, f, P, aux, s->E);
     MOE_LAUNCH_CHECK();
   }
@@ -858,9 +859,12 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   void* yperm = ws + L.yperm;
   const long long R = grouped_rows(s);
 
-  rc = route_impl(s, x, w_router, bias, nullptr, nullptr, idx, w, cts, aux_f, aux_p, aux, ws, stream);
+  rc = route_impl(s, x, w_router, bias, nullptr, nullptr, idx, w, cts, aux_f, aux_p, aux, ws, stream, true);
   if (rc) return rc;
-  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream);
+  const float* f_used = aux_f ? aux_f : reinterpret_cast<const float*>(ws + L.fP);
+  const float* p_used = aux_p ? aux_p : reinterpret_cast<const float*>(ws + L.fP) + s->E;
+  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream, true, f_used, p_used,
+                      aux);
   if (rc) return rc;
   const Int4Scratch scr = s->wfmt == MOE_WFMT_INT4_G128
                               ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq,

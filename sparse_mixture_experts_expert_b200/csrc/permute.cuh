@@ -68,12 +68,22 @@ __global__ void __launch_bounds__(128) k_scatter(const __nv_bfloat16* __restrict
                                                  int T, int d, int E, int k, int cap, int32_t* __restrict__ slot_pos,
                                                  uint8_t* __restrict__ drop, int32_t* __restrict__ row_src,
                                                  __nv_bfloat16* __restrict__ x_perm, int32_t* __restrict__ kept_out,
-                                                 int32_t* __restrict__ offsets_out) {
+                                                 int32_t* __restrict__ offsets_out, const float* __restrict__ aux_f,
+                                                 const float* __restrict__ aux_p, float* __restrict__ aux_out) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_kept[kMaxE];
   __shared__ int s_tmp[4];
   __shared__ int s_cnt[4][kMaxE];
+  // load-balance statistic of the routing this call groups: aux = E * sum_e f_e P_e (lanes in expert
+  // order, then a fixed xor tree), folded in here so the forward needs no launch of its own for it
+  if (aux_out != nullptr && blockIdx.x == 0 && threadIdx.x < 32) {
+    float a = 0.f;
+    for (int e = threadIdx.x; e < E; e += 32) a += aux_f[e] * aux_p[e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (threadIdx.x == 0) *aux_out = (float)E * a;
+  }
   __shared__ int s_ix[4][kChunk * KMAX];
   __shared__ int s_rk[4][kChunk * KMAX];
   const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
