@@ -593,18 +593,18 @@ __global__ void __launch_bounds__(256) k_router_lanes(const __nv_bfloat16* __res
   for (int e = 0; e < EC; ++e) z[e] = 0.f;
   const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + (size_t)(on ? t : 0) * d);
   const int nw = d >> 1;
-  // the lane's input pairs w = q, q + KP, ...: four loads in flight, then their FMAs
-  for (int w0 = q; w0 < nw; w0 += 4 * KP) {
-    uint32_t ub[4];
+  // the lane's input pairs w = q, q + KP, ...: sixteen loads in flight, then their FMAs
+  for (int w0 = q; w0 < nw; w0 += 16 * KP) {
+    uint32_t ub[16];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 16; ++j) {
       const int w = w0 + j * KP;
       ub[j] = (on && w < nw) ? __ldg(xw + w) : 0u;
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int w = w0 + j * KP;
-      if (w >= nw) break;
+    for (int j = 0; j < 16; ++j) {
+      // past the input end the loaded word is 0 and row 0 is read instead: the FMAs add zeros
+      const int w = w0 + j * KP < nw ? w0 + j * KP : 0;
       const float x0 = bf16lo(ub[j]), x1 = bf16hi(ub[j]);
       const float4* r0 = reinterpret_cast<const float4*>(s_wt + (size_t)(2 * w) * PW);
       const float4* r1 = reinterpret_cast<const float4*>(s_wt + (size_t)(2 * w + 1) * PW);
