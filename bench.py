@@ -11,7 +11,11 @@ tokens (the layer does not shard here; no collective on the data path); the
 reported time is the max over ranks.
 
 Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
-oracle on a bounded sample of the same workload (the reference arm).
+oracle on the same workload (the reference arm): one full-size forward per
+step for the bf16 workloads; for the INT4 decode workload, whose float64
+experts do not fit in host memory at once, one token of the batch per step.
+The default workload is ``granular`` (T=32768, d=768, 192 experts top-4, SwiGLU
+hidden 256, shared expert 512, capacity factor 1.25).
 """
 
 from __future__ import annotations
@@ -29,7 +33,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor-core or HBM roofline"
-DEFAULT_WORKLOAD = "small"
+DEFAULT_WORKLOAD = "granular"
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the expert GEMM launches of one forward, from an
 # `ncu --set full --clock-control none -k regex:k_grouped_gemm` capture of `bench.py --workload <name> --steps 1
 # --warmup 3 --no-cpu-baseline` on the current kernels; workloads without a complete capture report null.
@@ -52,6 +56,15 @@ def load_peaks():
 def hbm_roofline_tokens_per_s(bandwidth_bytes_per_s: float, active_bytes_per_token: float) -> float:
     """Ideal bandwidth-bound decode rate: bandwidth / bytes of active weights per token."""
     return bandwidth_bytes_per_s / active_bytes_per_token
+
+
+def bench_config(wl, capacity: int, world: int) -> dict:
+    """The ``config`` object of the JSON line, identical for both arms on the same workload."""
+    return {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "H": wl.H, "H_s": wl.H_s,
+            "capacity": capacity, "act": "geglu" if wl.act else "swiglu",
+            "wfmt": "int4_g128" if wl.wfmt else "bf16", "router": "fp32", "skew": wl.skew,
+            "l2": "GPU arm: a 256 MiB write flushes L2 before every timed step, outside the timed interval",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def int4_step_bytes(wl, touched: int) -> int:
@@ -209,6 +222,10 @@ def stage_times(moe, s, inp, ws, wl, flush, reps=10):
         state["out"] = moe.moe_combine(s, state["y"], state["p"]["slot_pos"], state["r"]["topk_w"], state["ysh"])
 
     fns = [st_route, st_permute, st_ffn, st_shared, st_combine]
+    if not wl.H_s:                      # no shared expert: no stage (an empty graph would still cost a replay)
+        names.remove("shared_ffn")
+        fns.remove(st_shared)
+        state["ysh"] = None
     for f in fns:                       # eager warm-up (allocations, attributes)
         f()
     torch.cuda.synchronize()
@@ -220,7 +237,7 @@ def stage_times(moe, s, inp, ws, wl, flush, reps=10):
         graphs.append(g)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
     acc = {k: [] for k in names}
     for _ in range(reps):
         flush()
@@ -234,78 +251,102 @@ def stage_times(moe, s, inp, ws, wl, flush, reps=10):
     kept = int(state["p"]["kept"].sum())
     touched = int((state["p"]["kept"] > 0).sum())
     del graphs
-    return {k: statistics.median(v) for k, v in acc.items()}, kept, touched
+    out = {k: statistics.median(v) for k, v in acc.items()}
+    if not wl.H_s:
+        out["shared_ffn"] = 0.0
+    return out, kept, touched
 
 
-def cpu_oracle_sample(wl, budget_s=12.0, max_tokens=None):
-    """Time the float64 oracle on a bounded token sample of the workload; returns (tokens/s, sample, cores)."""
-    import numpy as np
-    import torch
-
-    import oracle as O
-    import synth
-    cores = len(os.sched_getaffinity(0))
+def _blas_threads(cores):
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+        n = max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [0])
+        return min(cores, n) if n else cores
     except Exception:  # noqa: BLE001
-        threads = cores
-    if wl.wfmt != 0:
-        return cpu_oracle_sample_int4(wl, budget_s, cores, threads)
-    n = min(wl.T, max_tokens or wl.T)
-    sub = wl.replace(T=n)
-    inp = synth.make_inputs(sub, seed=0, device="cpu")
-    f64 = lambda t: t.to(torch.float64).numpy() if t is not None else None  # noqa: E731
-    args = dict(x=f64(inp["x"]), w_router=f64(inp["w_router"]), bias=f64(inp["bias"]), w13=f64(inp["w13"]),
-                w2=f64(inp["w2"]), w13_sh=f64(inp.get("w13_sh")), w2_sh=f64(inp.get("w2_sh")))
-    cap = O.capacity(n, wl.k, wl.E, wl.capacity_factor)
-    done, t0 = 0, time.perf_counter()
-    while True:
-        O.moe_forward(args["x"], args["w_router"], args["bias"], args["w13"], args["w2"], k=wl.k, act=wl.act,
-                      renorm=bool(wl.renorm), cap=cap, w13_sh=args["w13_sh"], w2_sh=args["w2_sh"])
-        done += n
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
-    return done / el, f"{done} tokens ({done // n} x {n}-token batches of the {wl.name} workload) in {el:.1f} s", \
-        min(cores, threads) if threads else cores
+        return cores
 
 
-def cpu_oracle_sample_int4(wl, budget_s, cores, threads):  # noqa: C901
-    """INT4 workload: the oracle routes the whole batch, then quantises, dequantises and applies each
-    token's experts one token at a time until the time budget is spent."""
-    import numpy as np
-    import torch
+class OracleRunner:
+    """The float64 oracle on one workload, inputs drawn once (seed 0, CPU generators).
 
-    import oracle as O
-    import synth
-    inp = synth.make_inputs(wl, seed=0, device="cpu", with_expert_weights=False)
-    x = inp["x"].to(torch.float64).numpy()
-    t0 = time.perf_counter()
-    r = O.route(x, inp["w_router"].to(torch.float64).numpy(), None, wl.k, bool(wl.renorm))
+    bf16 workloads: one call = one full-size forward of the whole batch (T tokens).  INT4 decode workload:
+    the whole batch is routed once at set-up; one call = the next token of the batch, whose k experts and
+    the shared expert are drawn, quantised, dequantised and applied by the oracle (the float64 experts of
+    the whole layer would not fit in host memory)."""
 
-    def expert(e):
-        a, b = synth.expert_weights_f32(wl, 0, e, "cpu")
+    def __init__(self, wl):
+        import torch
+
+        import oracle as O
+        import synth
+        self.wl, self.O, self.synth = wl, O, synth
+        self.cap = O.capacity(wl.T, wl.k, wl.E, wl.capacity_factor)
+        f64 = lambda t: t.to(torch.float64).numpy() if t is not None else None  # noqa: E731
+        if wl.wfmt == 0:
+            inp = synth.make_inputs(wl, seed=0, device="cpu")
+            self.args = {k: f64(inp.get(k)) for k in ("x", "w_router", "bias", "w13", "w2", "w13_sh", "w2_sh")}
+        else:
+            inp = synth.make_inputs(wl, seed=0, device="cpu", with_expert_weights=False)
+            self.x = f64(inp["x"])
+            self.r = O.route(self.x, f64(inp["w_router"]), f64(inp["bias"]), wl.k, bool(wl.renorm))
+            self.next_t = 0
+
+    def _expert(self, e):
+        O = self.O
+        a, b = self.synth.expert_weights_f32(self.wl, 0, e, "cpu")
         qa, sa = O.quantize_int4_g128(a.numpy())
         qb, sb = O.quantize_int4_g128(b.numpy())
         return O.dequantize_int4_g128(O.pack_int4(qa), sa), O.dequantize_int4_g128(O.pack_int4(qb), sb)
 
-    done = 0
-    while True:
-        t = done % wl.T
+    def __call__(self) -> int:
+        """One unit of oracle work; returns the tokens it covered."""
+        import numpy as np
+        wl, O = self.wl, self.O
+        if wl.wfmt == 0:
+            a = self.args
+            O.moe_forward(a["x"], a["w_router"], a["bias"], a["w13"], a["w2"], k=wl.k, act=wl.act,
+                          renorm=bool(wl.renorm), cap=self.cap, w13_sh=a["w13_sh"], w2_sh=a["w2_sh"])
+            return wl.T
+        t = self.next_t
+        self.next_t = (t + 1) % wl.T
         out = np.zeros(wl.d)
         for j in range(wl.k):
-            w13, w2 = expert(int(r["idx"][t, j]))
-            out += r["w"][t, j] * O.expert_ffn(x[t:t + 1], w13, w2, wl.act)[0]
+            w13, w2 = self._expert(int(self.r["idx"][t, j]))
+            out += self.r["w"][t, j] * O.expert_ffn(self.x[t:t + 1], w13, w2, wl.act)[0]
         if wl.H_s:
-            w13, w2 = expert(wl.E)
-            out += O.expert_ffn(x[t:t + 1], w13, w2, wl.act)[0]
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
-    return done / el, f"{done} tokens of the {wl.name} workload, routed in a full batch, experts dequantised " \
-        f"per token, {el:.1f} s", min(cores, threads) if threads else cores
+            w13, w2 = self._expert(wl.E)
+            out += O.expert_ffn(self.x[t:t + 1], w13, w2, wl.act)[0]
+        return 1
+
+    def describe(self, done, el):
+        if self.wl.wfmt == 0:
+            return f"{done} tokens ({done // self.wl.T} full {self.wl.T}-token forwards of the {self.wl.name} " \
+                   f"workload) in {el:.1f} s"
+        return f"{done} tokens of the {self.wl.name} workload (batch routed once; each token's {self.wl.k} experts " \
+               f"and the shared expert drawn, quantised and dequantised per token) in {el:.1f} s"
+
+
+def cpu_oracle_sample(wl, budget_s=12.0, single_thread=False):
+    """Time the float64 oracle on the workload for about ``budget_s`` seconds (at least one call).
+    Returns (tokens/s, sample description, threads used)."""
+    cores = len(os.sched_getaffinity(0))
+    run = OracleRunner(wl)
+    limit = None
+    if single_thread:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(limits=1)
+    try:
+        threads = 1 if single_thread else _blas_threads(cores)
+        done, t0 = 0, time.perf_counter()
+        while True:
+            done += run()
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+    finally:
+        if limit is not None:
+            limit.restore_original_limits()
+    return done / el, run.describe(done, el), threads
 
 
 # ------------------------------------------------------------------ main
@@ -335,18 +376,25 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps = []
+        cores = len(os.sched_getaffinity(0))
+        run = OracleRunner(wl)
+        threads = _blas_threads(cores)
+        times, done = [], 0
         for i in range(args.warmup + args.steps):
-            v, sample, cores = cpu_oracle_sample(wl, budget_s=2.0, max_tokens=min(wl.T, 2048))
+            t0 = time.perf_counter()
+            n = run()
+            el = time.perf_counter() - t0
             if i >= args.warmup:
-                steps.append(v)
-        val = statistics.median(steps)
+                times.append(el)
+                done += n
+        total = sum(times)
+        val = done / total
         line = {"metric": METRIC, "value": val, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": wl.T / val * 1e3,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "H": wl.H, "H_s": wl.H_s},
-                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                 "sample": sample},
+                "config": bench_config(wl, run.cap, world),
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                 "sample": run.describe(done, total) + " (timed steps only)"},
                 "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -431,7 +479,7 @@ def main():
     stages, kept, touched = stage_times(moe, s, inp, ws, wl, flush)
     peaks = load_peaks()
     flops = wl.flops_tc(kept)
-    gemm_us = stages["expert_ffn"] + stages["shared_ffn"]
+    gemm_us = stages["expert_ffn"] + (stages["shared_ffn"] if wl.H_s else 0.0)
     if wl.wfmt == synth.WFMT_INT4_G128:
         alg_bytes = int4_step_bytes(wl, touched)
         achieved = alg_bytes / (step_ms * 1e-3) / 1e9
@@ -453,16 +501,15 @@ def main():
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            v, sample, cores = cpu_oracle_sample(wl, budget_s=12.0, max_tokens=min(wl.T, 4096))
+            v, sample, cores = cpu_oracle_sample(wl, budget_s=12.0)
             cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+            if wl.name in ("tiny", "small"):
+                v1, sample1, _ = cpu_oracle_sample(wl, budget_s=6.0, single_thread=True)
+                cpu["single_thread"] = {"value": v1, "unit": "tokens/s", "cores": 1, "sample": sample1}
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "H": wl.H,
-                           "H_s": wl.H_s, "capacity": s.capacity, "act": "geglu" if wl.act else "swiglu",
-                           "wfmt": "int4_g128" if wl.wfmt else "bf16", "router": "fp32",
-                           "l2": "flushed before every step (256 MiB write), outside the timed interval",
-                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "config": bench_config(wl, s.capacity, world),
                 "roofline": roofline, "stages_us": stages, "cpu_baseline": cpu,
                 "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": "tokens/s",
                         "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": out_host.numel() * 2},

@@ -40,6 +40,12 @@
  *    moe_get_status(); kernels never trap.
  *  - Inputs must be finite; routing of NaN logits is undefined.
  *  - Layouts are row-major.  bf16 tensors are passed as void*.
+ *  - Reentrant: every choice a call makes comes from its arguments.  The
+ *    library's only mutable state is (a) the per-device status word above,
+ *    (b) the wait limit of moe_set_wait_limit_ns, (c) the launch counter of
+ *    moe_launch_count, (d) idempotent per-device caches filled on first use
+ *    (SM count, kernel attributes, the tensor-map encoder entry point) and
+ *    (e) the fixed scratch array of moe_permute_noalloc.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -77,10 +83,18 @@ enum moe_wfmt { MOE_WFMT_BF16 = 0, MOE_WFMT_INT4_G128 = 1 };
  *   act      enum moe_act
  *   wfmt     enum moe_wfmt
  *   renorm   1: divide the k gates by their sum; 0: gates are the softmax probabilities
+ *   flags    implementation choices, 0 = automatic; MOE_FLAG_SINGLE_CTA_GEMM runs
+ *            the bf16 expert GEMMs on single-CTA 128-row tiles even where the
+ *            automatic choice would pair CTAs (256-row tiles, tcgen05
+ *            cta_group::2).  Both compute the same products in the same fp32
+ *            order per output.  Unknown bits give MOE_INVALID_ARGUMENT.  (No
+ *            counterpart on the pages.)
  */
+enum moe_flags { MOE_FLAG_SINGLE_CTA_GEMM = 1 };
+
 typedef struct moe_shape {
   int64_t T;
-  int32_t d, E, k, H, H_s, capacity, act, wfmt, renorm;
+  int32_t d, E, k, H, H_s, capacity, act, wfmt, renorm, flags;
 } moe_shape;
 
 /*
@@ -232,8 +246,10 @@ int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void*
  *   returned and nothing is enqueued.
  *   Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and keeps it for later
+ *   calls; make that first call before any stream capture.  A device reset
+ *   (cudaDeviceReset) or a destroyed primary context invalidates the kept
+ *   address: do not call this entry point after one.
  *   Every call shares the one array, which keeps the last call's contents:
  *   calls that overlap on the GPU (concurrent streams, or several host
  *   threads) race on it and must be serialised by the caller.
@@ -250,17 +266,12 @@ int moe_permute_noalloc(const moe_shape* s, const void* x, const int32_t* topk_i
  */
 int moe_get_status(moe_stream_t stream, int32_t* device_status, uint32_t* site);
 
-/* Upper bound, in nanoseconds, of every device-side wait (default 2e9). */
-int moe_set_wait_limit_ns(uint64_t ns);
-
 /*
- * Kernel choice for the bf16 expert GEMMs (process-wide, default 1).  1: groups
- * averaging at least 192 rows run on CTA pairs (256-row tiles, tcgen05
- * cta_group::2); 0: single-CTA 128-row tiles everywhere.  Both compute the same
- * products in the same fp32 order per output.  Returns MOE_INVALID_ARGUMENT
- * for other values.  Implementation choice only; the pages have no counterpart.
+ * Upper bound, in nanoseconds, of every device-side wait (default 2e9).  The one
+ * process-wide setting of the library (a debugging knob for failure tests): it
+ * applies to kernels enqueued after the call, from any thread.
  */
-int moe_set_pair_gemm(int32_t enable);
+int moe_set_wait_limit_ns(uint64_t ns);
 
 /* Enqueue a kernel whose bounded wait on an mbarrier nobody arrives on must give
  * up after the wait limit: exercises the MOE_DEVICE_TIMEOUT path safely. */

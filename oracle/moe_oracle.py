@@ -76,11 +76,6 @@ def bf16_round(a) -> np.ndarray:
     return r.view(np.float32).reshape(f.shape)
 
 
-def bf16_bits_to_f32(bits) -> np.ndarray:
-    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
-    return b.view(np.float32)
-
-
 # ---------------------------------------------------------------- step 1-3: router
 
 def router_logits(x, w_router, bias=None) -> np.ndarray:

@@ -23,13 +23,14 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 ACT_SWIGLU, ACT_GEGLU = 0, 1
 WFMT_BF16, WFMT_INT4_G128 = 0, 1
+FLAG_SINGLE_CTA_GEMM = 1
 STATUS = {0: "MOE_OK", 1: "MOE_INVALID_ARGUMENT", 2: "MOE_UNSUPPORTED_SHAPE", 3: "MOE_WORKSPACE_TOO_SMALL",
           4: "MOE_CUDA_ERROR", 5: "MOE_DEVICE_TIMEOUT"}
 
 EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route", "moe_route_from_logits",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
             "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
-            "moe_permute_noalloc", "moe_set_pair_gemm"]
+            "moe_permute_noalloc"]
 
 
 class MoeError(RuntimeError):
@@ -41,10 +42,11 @@ class MoeError(RuntimeError):
 class MoeShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("H_s", ctypes.c_int32), ("capacity", ctypes.c_int32),
-                ("act", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("renorm", ctypes.c_int32)]
+                ("act", ctypes.c_int32), ("wfmt", ctypes.c_int32), ("renorm", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
 
-    def __init__(self, T, d, E, k, H, H_s=0, capacity=0, act=ACT_SWIGLU, wfmt=WFMT_BF16, renorm=1):
-        super().__init__(T, d, E, k, H, H_s, capacity, act, wfmt, renorm)
+    def __init__(self, T, d, E, k, H, H_s=0, capacity=0, act=ACT_SWIGLU, wfmt=WFMT_BF16, renorm=1, flags=0):
+        super().__init__(T, d, E, k, H, H_s, capacity, act, wfmt, renorm, flags)
 
     @property
     def R(self) -> int:
@@ -81,7 +83,6 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_quantize_int4": (ctypes.c_int, [_P, i64, i32, _P, _P, _P]),
         "moe_get_status": (ctypes.c_int, [_P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_uint32)]),
         "moe_set_wait_limit_ns": (ctypes.c_int, [u64]),
-        "moe_set_pair_gemm": (ctypes.c_int, [i32]),
         "moe_selftest_wait_timeout": (ctypes.c_int, [_P]),
         "moe_launch_count": (u64, []),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -329,8 +330,3 @@ def moe_get_status(stream=None):
 
 def moe_launch_count() -> int:
     return int(_L().moe_launch_count())
-
-
-def moe_set_pair_gemm(enable: bool) -> None:
-    """Select CTA-pair (True, default) or single-CTA (False) tiles for the bf16 expert GEMMs, process-wide."""
-    _check(_L().moe_set_pair_gemm(1 if enable else 0), "moe_set_pair_gemm")

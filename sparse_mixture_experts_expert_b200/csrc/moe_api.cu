@@ -19,8 +19,6 @@ namespace moe {
 
 static std::atomic<unsigned long long> g_launches{0};
 static std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
-// CTA-pair expert GEMMs (on by default; moe_set_pair_gemm(0) selects the single-CTA kernel everywhere).
-static std::atomic<int> g_pair_gemm{1};
 
 static inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -92,6 +90,7 @@ static int check_shape(const moe_shape* s) {
   if (s->act != MOE_ACT_SWIGLU && s->act != MOE_ACT_GEGLU) return MOE_INVALID_ARGUMENT;
   if (s->wfmt != MOE_WFMT_BF16 && s->wfmt != MOE_WFMT_INT4_G128) return MOE_INVALID_ARGUMENT;
   if (s->renorm != 0 && s->renorm != 1) return MOE_INVALID_ARGUMENT;
+  if (s->flags & ~MOE_FLAG_SINGLE_CTA_GEMM) return MOE_INVALID_ARGUMENT;
   if (s->wfmt == MOE_WFMT_INT4_G128 && (s->d % 128 != 0 || s->H % 128 != 0 || s->H_s % 128 != 0))
     return MOE_UNSUPPORTED_SHAPE;
   const long long R = s->capacity > 0 ? (long long)s->E * s->capacity : s->T * s->k;
@@ -252,8 +251,8 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 
 // CTA pairs (M = 256 tiles) for the bf16 expert GEMMs when the groups are large enough
 // to fill them: on average at least 192 rows per group.
-static bool use_pair_gemm(int mode, int BN, long long R, int n_groups) {
-  return mode != kModeF32 && BN == 256 && R >= 192ll * n_groups && g_pair_gemm.load();
+static bool use_pair_gemm(int mode, int BN, long long R, int n_groups, bool allow_pair) {
+  return allow_pair && mode != kModeF32 && BN == 256 && R >= 192ll * n_groups;
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
@@ -278,13 +277,13 @@ static int pick_bn(bool glu, int N, long long mtiles) {
 
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
                         int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
-                        cudaStream_t st, int a_kwrap = 0, const float* bias = nullptr) {
+                        cudaStream_t st, bool allow_pair, int a_kwrap = 0, const float* bias = nullptr) {
   if (R == 0) return MOE_OK;
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   // router logits: one column tile as wide as the expert count (fewer A re-reads)
   const int BN = mode == kModeF32 ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
-  const bool pair = use_pair_gemm(mode, BN, R, n_groups);
+  const bool pair = use_pair_gemm(mode, BN, R, n_groups, allow_pair);
   const int box_rows = (glu || pair) ? BN / 2 : BN;
   CUtensorMap ta, tb;
   cuuint64_t da[2] = {(cuuint64_t)(a_kwrap > 0 ? a_kwrap : K), (cuuint64_t)R};
@@ -344,13 +343,13 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   if (epl <= N_ && (small ? 4 : 8) == NW_ && xreg == XR_) {                                                       \
     const size_t smem = ST_ ? (size_t)2 * NW_ * s->E * sizeof(float) : 0;                                         \
     if (smem > 48 * 1024) {                                                                                       \
-      static int attr_done[64] = {0};                                                                             \
-      const int dev = current_device();                                                                           \
-      if (dev < 64 && !attr_done[dev]) {                                                                          \
+      static std::atomic<unsigned long long> attr_done{0};                                                        \
+      const unsigned long long bit = 1ull << (current_device() & 63);                                             \
+      if (!(attr_done.load() & bit)) {                                                                            \
         MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_topk<N_, NW_, XR_, ST_>,                                       \
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,                           \
                                           2 * NW_ * kMaxRouterE * (int)sizeof(float)));                           \
-        attr_done[dev] = 1;                                                                                       \
+        attr_done.fetch_or(bit);                                                                                  \
       }                                                                                                           \
     }                                                                                                             \
     const unsigned grid = ST_ ? (unsigned)nchunks : (unsigned)cdiv(s->T, NW_);                                    \
@@ -537,9 +536,10 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
     return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st, scr);
   }
   const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
-  rc = grouped_gemm(mode, A, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st);
+  const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
+  rc = grouped_gemm(mode, A, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st, pair);
   if (rc) return rc;
-  return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, gstart, grows, y, st);
+  return grouped_gemm(kModePlain, h, R, hidden, w2, n_groups, s->d, 0, s->d, gstart, grows, y, st, pair);
 }
 
 // Fused CUDA-core router when W_r^T fits in shared memory: returns its experts-per-lane template, else 0.
@@ -613,7 +613,7 @@ static int launch_fused_router(const moe_shape* s, int epl, const void* x, const
 // (fp32 accumulation); small ones stay on the fp32 CUDA-core GEMM.
 // Decode router: dynamic shared memory of the staged x slice (16 tokens x one input slice, fp32).
 static constexpr size_t kSkinnyMaxSmem = 100 * 1024;
-static int g_skinny_attr[64] = {0};
+static std::atomic<unsigned long long> g_skinny_attr{0};   // per-device bit: shared-memory opt-in done
 static size_t skinny_smem(int d) { return (size_t)kSkTok * skinny_slice(d) * sizeof(float); }
 
 static bool use_tc_router(const moe_shape* s) {
@@ -642,8 +642,8 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
     MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d);
     MOE_LAUNCH_CHECK();
-    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, s->d,
-                      bias);
+    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false,
+                      s->d, bias);
     if (rc) return rc;
     // screening bound, relative to ||x_t|| max_e ||w_e|| (>= sum |x_i w_i|): the split's representation error
     // 2^-16, fp32 accumulation of 2d products in any rounding direction plus the bias add, and the error of the
@@ -654,10 +654,10 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
                            (1.0 + std::ldexp(1.0, -7)))};
     rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
   } else if (logits_in == nullptr && s->T <= 256 && skinny_smem(s->d) <= kSkinnyMaxSmem) {
-    const int dev = current_device();
-    if (dev >= 0 && dev < 64 && !g_skinny_attr[dev]) {
+    const unsigned long long bit = 1ull << (current_device() & 63);
+    if (!(g_skinny_attr.load() & bit)) {
       MOE_CUDA_TRY(cudaFuncSetAttribute(k_router_skinny, cudaFuncAttributeMaxDynamicSharedMemorySize, kSkinnyMaxSmem));
-      g_skinny_attr[dev] = 1;
+      g_skinny_attr.fetch_or(bit);
     }
     dim3 grid((unsigned)cdiv(s->E, 8 * kSkExp), (unsigned)cdiv(s->T, kSkTok), kSkSplit);
     MOE_LAUNCH((k_router_skinny), grid, 256, skinny_smem(s->d), st, reinterpret_cast<const __nv_bfloat16*>(x), w_router, part,
@@ -711,12 +711,6 @@ uint64_t moe_launch_count(void) { return g_launches.load(); }
 int moe_set_wait_limit_ns(uint64_t ns) {
   if (ns == 0) return MOE_INVALID_ARGUMENT;
   g_wait_limit_ns.store(ns);
-  return MOE_OK;
-}
-
-int moe_set_pair_gemm(int32_t enable) {
-  if (enable != 0 && enable != 1) return MOE_INVALID_ARGUMENT;
-  g_pair_gemm.store(enable);
   return MOE_OK;
 }
 

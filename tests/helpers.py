@@ -104,11 +104,16 @@ def int4_expert_weights(moe, wl, seed=0, device="cuda", experts=None):
     return out
 
 
+def oracle_int4_from_f32(a, b):
+    """float64 (w13, w2) after the oracle's own quantise -> pack -> dequantise of fp32 draws (numpy arrays)."""
+    import oracle as O
+    qa, sa = O.quantize_int4_g128(a)
+    qb, sb = O.quantize_int4_g128(b)
+    return (O.dequantize_int4_g128(O.pack_int4(qa), sa), O.dequantize_int4_g128(O.pack_int4(qb), sb))
+
+
 def oracle_int4_expert(wl, seed, e, device="cuda"):
     """float64 (w13, w2) of expert e after the oracle's own quantise -> dequantise of the same fp32 draws."""
-    import oracle as O
     import synth
     a, b = synth.expert_weights_f32(wl, seed, e, device)
-    qa, sa = O.quantize_int4_g128(a.cpu().numpy())
-    qb, sb = O.quantize_int4_g128(b.cpu().numpy())
-    return (O.dequantize_int4_g128(O.pack_int4(qa), sa), O.dequantize_int4_g128(O.pack_int4(qb), sb))
+    return oracle_int4_from_f32(a.cpu().numpy(), b.cpu().numpy())

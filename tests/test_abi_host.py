@@ -63,7 +63,8 @@ def test_capacity_and_rows(L):
 
 @pytest.mark.parametrize("kw,code", [({"k": 9}, 1), ({"d": 60}, 2), ({"H": 0}, 2), ({"E": 513}, 2),
                                      ({"T": 0}, 2), ({"act": 7}, 1), ({"wfmt": 1, "d": 64}, 2),
-                                     ({"renorm": 2}, 1), ({"capacity": -1}, 1)])
+                                     ({"renorm": 2}, 1), ({"capacity": -1}, 1), ({"flags": 2}, 1),
+                                     ({"flags": -1}, 1), ({"flags": 1}, 0)])
 def test_shape_validation(L, kw, code):
     import sparse_mixture_experts_expert_b200 as moe
     s = _shape(moe, **kw)
@@ -97,4 +98,3 @@ def test_null_and_workspace_errors_return_before_device_work(L):
     rc = L.moe_quantize_int4(fake, 4, 100, fake, fake, None)
     assert rc == 1            # K % 128 != 0
     assert L.moe_set_wait_limit_ns(0) == 1
-    assert L.moe_set_pair_gemm(2) == 1 and L.moe_set_pair_gemm(-1) == 1

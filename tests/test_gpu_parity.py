@@ -63,8 +63,8 @@ def _route_case(moe, wl, T, seed):
     return wl, inp, r, ref, x64, W64, b64
 
 
-# Router paths: lane-per-token router for E <= 32 (tiny, small, geglu, E = 13), shared-memory router for
-# 32 < E <= 256 with a small W_r (E = 64), certified tensor-core router (skewed, granular shapes),
+# Router paths: lane-per-token router for E <= 16 (tiny, small, E = 13), shared-memory router for
+# 16 < E <= 256 with a small W_r (geglu's E = 32, E = 64), certified tensor-core router (skewed, granular shapes),
 # weight-streaming decode router (decode_int4; T <= 256: one token, a ragged token block with E = 200
 # and a ragged last input slice with d = 784), split-K CUDA-core router (E = 200, which is neither a
 # multiple of 16 nor small enough for the shared-memory router).
@@ -129,6 +129,31 @@ def test_permute_bit_exact(lib, T, E, k, cap, skew, d):
     assert (xp[filled] == xs[rs[filled] // k]).all()          # bit-exact row moves
 
 
+@pytest.mark.parametrize("cap", [854, 0])
+def test_permute_bit_exact_full_size(lib, cap):
+    """The granular/skewed grouping at full size (T=32768, E=192, top-4; 1024 chunks of 32 tokens), Zipf-like
+    skew 1.2, with the workload's capacity C = 854 (heavy drops on the popular experts) and without a capacity."""
+    moe = lib
+    T, E, k, d = 32768, 192, 4, 768
+    idx = synth.draw_topk_idx(T, E, k, seed=4242, skew=1.2)
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    s = _shape(moe, T, E, k, d=d, cap=cap)
+    r = moe.moe_permute(s, x.to(DEV), idx.to(DEV))
+    torch.cuda.synchronize()
+    ref = O.permute(npi(idx), E, cap)
+    for key in ("slot_pos", "counts", "kept", "offsets", "row_src"):
+        assert (npi(r[key]) == ref[key]).all(), key
+    assert (npi(r["drop_mask"]) == ref["drop"]).all()
+    if cap:
+        assert ref["drop"].sum() > 0
+    rs = ref["row_src"]
+    filled = rs >= 0
+    xp = npi(r["x_perm"].view(torch.int16))
+    xs = npi(x.view(torch.int16))
+    assert (xp[filled] == xs[rs[filled] // k]).all()
+
+
 # ---------------------------------------------------------------- grouped expert FFN
 
 
@@ -177,17 +202,13 @@ def test_expert_ffn_pair_tiles(lib, d, H, act, rows):
     w2 = torch.stack([synth.expert_weights_f32(wl, 4, e)[1] for e in range(E)]).to(torch.bfloat16)
     g = torch.Generator().manual_seed(d + H)
     xg = torch.randn(R, d, generator=g).to(torch.bfloat16)
-    s = _shape(moe, 1, E, 1, d=d, H=H, act=act)
     outs = {}
-    try:
-        for pair in (True, False):
-            moe.moe_set_pair_gemm(pair)
-            h, y = moe.moe_expert_ffn(s, xg.to(DEV), w13.to(DEV), w2.to(DEV), hidden=H, group_start=start.to(DEV),
-                                      group_rows=rows_t.to(DEV))
-            torch.cuda.synchronize()
-            outs[pair] = (np64(h), np64(y))
-    finally:
-        moe.moe_set_pair_gemm(True)
+    for pair in (True, False):
+        s = moe.MoeShape(T=1, d=d, E=E, k=1, H=H, act=act, flags=0 if pair else moe.FLAG_SINGLE_CTA_GEMM)
+        h, y = moe.moe_expert_ffn(s, xg.to(DEV), w13.to(DEV), w2.to(DEV), hidden=H, group_start=start.to(DEV),
+                                  group_rows=rows_t.to(DEV))
+        torch.cuda.synchronize()
+        outs[pair] = (np64(h), np64(y))
     x64, w13_64, w2_64 = np64(xg), np64(w13), np64(w2)
     for pair, (hg, yg) in outs.items():
         for e in range(E):
@@ -439,25 +460,49 @@ def _int4_forward(moe, wl, seed=0):
 
 
 def _check_int4_forward(wl, inp, r, sample, seed=0):
-    from helpers import oracle_int4_expert
+    """Oracle output of the sampled tokens, one expert at a time: each touched expert's fp32 draw is quantised
+    and dequantised by the oracle, applied to the sampled tokens that chose it, then released (the whole
+    decode layer in float64 would not fit in host memory).  The oracle work of several experts runs on a thread
+    pool (numpy releases the GIL); the fp32 draws come from the device generator in the calling thread."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from helpers import oracle_int4_from_f32
     x64 = np64(inp["x"])
     b64 = np64(inp["bias"]) if inp["bias"] is not None else None
     ref = O.route(x64, np64(inp["w_router"]), b64, wl.k, bool(wl.renorm))
     idx = npi(r["topk_idx"])
     amb = O.topk_margin(ref["z"], wl.k) < MARGIN
     assert (idx[~amb] == ref["idx"][~amb]).all()
-    toks = [t for t in sample if (idx[t] == ref["idx"][t]).all()]
-    need = sorted({int(e) for t in toks for e in ref["idx"][t]})
-    cache = {e: oracle_int4_expert(wl, seed, e, DEV) for e in need}
-    out_ref = np.zeros((len(toks), wl.d))
-    sh = oracle_int4_expert(wl, seed, wl.E, DEV) if wl.H_s else None
-    for n, t in enumerate(toks):
+    toks = np.array([t for t in sample if (idx[t] == ref["idx"][t]).all()], np.int64)
+    sel = ref["idx"][toks]                                  # [n, k]
+    users = {}                                              # expert -> [(row in toks, slot j)]
+    for n in range(toks.size):
         for j in range(wl.k):
-            w13e, w2e = cache[int(ref["idx"][t, j])]
-            out_ref[n] += ref["w"][t, j] * O.expert_ffn(x64[t:t + 1], w13e, w2e, wl.act)[0]
-        if sh is not None:
-            out_ref[n] += O.expert_ffn(x64[t:t + 1], sh[0], sh[1], wl.act)[0]
+            users.setdefault(int(sel[n, j]), []).append((n, j))
+    if wl.H_s:
+        users[wl.E] = [(n, -1) for n in range(toks.size)]   # the shared expert, weight one
+
+    def job(e, a, b):
+        w13e, w2e = oracle_int4_from_f32(a, b)
+        rows = np.array([n for n, _ in users[e]], np.int64)
+        gate = np.array([1.0 if j < 0 else ref["w"][toks[n], j] for n, j in users[e]])
+        return rows, gate[:, None] * O.expert_ffn(x64[toks[rows]], w13e, w2e, wl.act)
+
+    out_ref = np.zeros((toks.size, wl.d))
+    import os
+    with ThreadPoolExecutor(max_workers=max(1, min(8, len(os.sched_getaffinity(0)) // 2))) as pool:
+        futs = []
+        for e in sorted(users):
+            a, b = synth.expert_weights_f32(wl, seed, e, DEV)
+            futs.append(pool.submit(job, e, a.cpu().numpy(), b.cpu().numpy()))
+            if len(futs) >= 16:                             # bound the host memory in flight
+                rows, y = futs.pop(0).result()
+                np.add.at(out_ref, rows, y)
+        for f in futs:
+            rows, y = f.result()
+            np.add.at(out_ref, rows, y)
     assert_out_close(np64(r["out"])[toks], out_ref)
+    return toks.size
 
 
 def test_forward_int4_reduced(lib):
@@ -466,8 +511,10 @@ def test_forward_int4_reduced(lib):
     _check_int4_forward(wl, inp, r, sample=list(range(wl.T)))
 
 
-def test_forward_int4_full_size_sampled(lib):
-    """The decode workload at full size (8.7 GB of INT4 experts), oracle on sampled tokens."""
+def test_forward_int4_full_size(lib):
+    """The decode workload at full size (8.7 GB of INT4 experts), every one of the 64 tokens against the oracle
+    (about 285 touched experts, each dequantised by the oracle once)."""
     wl = synth.get_workload("decode_int4")
     inp, r = _int4_forward(lib, wl)
-    _check_int4_forward(wl, inp, r, sample=[0, 37, 63])
+    n = _check_int4_forward(wl, inp, r, sample=list(range(wl.T)))
+    assert n >= wl.T - 2
