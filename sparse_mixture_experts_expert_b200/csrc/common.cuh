@@ -11,6 +11,9 @@
 
 namespace moe {
 
+// Candidates per token kept by the certified router selection (screening GEMM epilogue -> exact recompute).
+constexpr int kSelMaxCand = 32;
+
 // Device status word: 0 = fine, otherwise a moe_status code (first error wins).
 // One per device (module-scope), read and cleared by moe_get_status().
 __device__ unsigned int g_status;

@@ -41,7 +41,28 @@
 
 namespace moe {
 
-enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3 };
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3, kModeRouterSel = 4 };
+
+// Outputs of the router-selection epilogue (kModeRouterSel): for every token t
+// (one accumulator row) the screening logits of all experts sit in one TMEM
+// lane; the epilogue takes their k-th largest value, marks every expert whose
+// screening logit may still reach the exact top k (z >= k-th - 2 * bound), and
+// appends each such (token, candidate slot) to its expert's list for the exact
+// recompute.  Up to kSelMaxCand candidates per token are kept; a token with
+// more records only its count (the finishing kernel then recomputes all experts
+// for it).
+struct RouterSelArgs {
+  const float* xnorm2;   // [T] sum of x_t^2
+  const float* wnorm;    // [E] ||W_r[e]||_2
+  float gamma;           // screening bound factor: |err| <= gamma ||x_t|| max_e ||w_e||
+  int E, k;
+  uint8_t* cidx;         // [T][kSelMaxCand] candidate experts in expert order
+  int32_t* ncand;        // [T] candidate count
+  float* zmax;           // [T] largest screening logit m_s
+  float* snc;            // [T] sum over non-candidates of exp(z_e - m_s)
+  int32_t* ecount;       // [E] list lengths (zero before the launch)
+  int32_t* elist;        // [E][T] entries t * kSelMaxCand + slot
+};
 
 struct GemmParams {
   const int32_t* group_start;  // [n_groups] or nullptr (one group of R rows)
@@ -56,7 +77,8 @@ struct GemmParams {
   unsigned long long wait_limit_ns;
   int a_kwrap;         // > 0: the A operand repeats every a_kwrap columns of the reduction (split router)
   float* out_f32;      // kModeF32: fp32 output [R, N]
-  const float* bias;   // kModeF32: optional per-column bias [N]
+  const float* bias;   // kModeF32 / kModeRouterSel: optional per-column bias [N]
+  RouterSelArgs sel;   // kModeRouterSel
 };
 
 #ifndef MOE_GEMM_MAX_STAGES
@@ -96,6 +118,80 @@ __device__ __forceinline__ float erf_as7126(float x) {
 }
 __device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + erf_as7126(g * 0.7071067811865476f)); }
 
+// Router selection for one token (one TMEM lane = one accumulator row of BN
+// screening logits; columns >= E are padding).  Pass 1: the largest value and
+// the k-th largest (with multiplicity) by a KM-slot descending insertion
+// network.  Pass 2: the candidates (z >= k-th - 2 bound), written in expert
+// order and appended to their experts' lists (order inside a list is
+// irrelevant: each entry's exact value does not depend on it), and the sum of
+// exp(z - max) over the non-candidates; the accumulator is released after its
+// last read.
+template <int BN, int KM, typename Release>
+__device__ __forceinline__ void router_select(const RouterSelArgs a, const float* __restrict__ bias, long long R,
+                                              uint32_t t_row, bool valid, long long t, float wmax, Release release) {
+  float top[KM];
+#pragma unroll
+  for (int i = 0; i < KM; ++i) top[i] = -INFINITY;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t v[2][16];
+    tmem_ld16(t_row + c0, v[0]);
+    tmem_ld16(t_row + c0 + 16, v[1]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int col = c0 + i;
+      const float z = col < a.E ? __uint_as_float(v[i >> 4][i & 15]) + (bias != nullptr ? bias[col] : 0.f)
+                                : -INFINITY;
+#pragma unroll
+      for (int j = KM - 1; j > 0; --j) top[j] = fmaxf(top[j], fminf(top[j - 1], z));
+      top[0] = fmaxf(top[0], z);
+    }
+  }
+  // top[] is sorted descending, so the k-th largest is the least of its first k entries (a running
+  // minimum rather than top[k - 1], which would index the array at run time)
+  float kth = top[0];
+#pragma unroll
+  for (int j = 1; j < KM; ++j) kth = j < a.k ? fminf(kth, top[j]) : kth;
+  const float m_s = top[0];
+  const float xn = valid ? sqrtf(a.xnorm2[t]) : 0.f;
+  const float bound = a.gamma * xn * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
+  const float thr = kth - 2.f * bound;
+  float snc = 0.f;
+  int nc = 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t v[2][16];
+    tmem_ld16(t_row + c0, v[0]);
+    tmem_ld16(t_row + c0 + 16, v[1]);
+    tmem_ld_wait();
+    if (c0 + 32 >= BN) release();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int col = c0 + i;
+      if (col < a.E) {
+        const float z = __uint_as_float(v[i >> 4][i & 15]) + (bias != nullptr ? bias[col] : 0.f);
+        if (z >= thr) {
+          // candidate: kept in expert order; past kSelMaxCand only counted (the finishing kernel then
+          // ignores this token's list entries and recomputes every expert)
+          if (valid && nc < kSelMaxCand) {
+            a.cidx[t * kSelMaxCand + nc] = (uint8_t)col;
+            const int pos = atomicAdd(&a.ecount[col], 1);
+            a.elist[(long long)col * R + pos] = (int32_t)(t * kSelMaxCand + nc);
+          }
+          ++nc;
+        } else {
+          snc += __expf(z - m_s);
+        }
+      }
+    }
+  }
+  if (!valid) return;
+  a.ncand[t] = nc;
+  a.zmax[t] = m_s;
+  a.snc[t] = snc;
+}
+
 template <int MODE, int BN, int CG = 1>
 __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -104,7 +200,7 @@ __global__ void __launch_bounds__(256, 1)
   using Cfg = GemmCfg<BN, CG>;
   constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
   constexpr bool kPair = CG == 2;
-  static_assert(!kPair || MODE != kModeF32, "the router GEMM runs on single CTAs");
+  static_assert(!kPair || (MODE != kModeF32 && MODE != kModeRouterSel), "the router GEMM runs on single CTAs");
   constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
   constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box (single CTA)
   constexpr int TM = kBM * CG;              // rows per tile
@@ -311,6 +407,12 @@ __global__ void __launch_bounds__(256, 1)
     __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)S * Cfg::kStageBytes) + q * 32 * kEpiRow;
     int acc = 0;
     uint32_t acc_phase = 0;
+    float wmax = 0.f;   // kModeRouterSel: max_e ||W_r[e]||
+    if (MODE == kModeRouterSel) {
+      for (int e = lane; e < p.sel.E; e += 32) wmax = fmaxf(wmax, p.sel.wnorm[e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+    }
     // accumulator release: each thread (single CTA) or each warp on the leader's barrier (pair)
     auto release_acc = [&](int a) {
       tc_fence_before();
@@ -328,7 +430,12 @@ __global__ void __launch_bounds__(256, 1)
       if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0106)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (MODE == kModeF32) {
+      if constexpr (MODE == kModeRouterSel) {
+        const bool valid = q * 32 + lane < rows_valid;
+        const long long t = row0 + q * 32 + lane;
+        if (p.sel.k <= 4) router_select<BN, 4>(p.sel, p.bias, p.R, t_row, valid, t, wmax, [&]() { release_acc(acc); });
+        else router_select<BN, 16>(p.sel, p.bias, p.R, t_row, valid, t, wmax, [&]() { release_acc(acc); });
+      } else if (MODE == kModeF32) {
         // fp32 rows through the staging buffer, 32 columns (128 bytes per row) per round
         float* fstg = reinterpret_cast<float*>(stg);  // 32 rows x 36 floats per warp
         constexpr int FR = 36;

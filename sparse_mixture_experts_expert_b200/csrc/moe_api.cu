@@ -136,7 +136,9 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab, total;
+  size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
+  size_t xnorm2, cidx, ncand, zmax, snc, zex, ecount;   // certified selection inside the screening GEMM
+  size_t total;
 };
 
 // Split-reduction partials of the INT4 shared expert (decode batches: T <= 256): up to 8 ranges of
@@ -178,6 +180,13 @@ static Workspace ws_layout(const moe_shape* s) {
   L.hs = take((size_t)s->T * std::max(s->H_s, 16) * 2);
   L.ys = take((size_t)s->T * s->d * 2);
   L.shtab = take(64);
+  L.xnorm2 = take((size_t)s->T * 4);
+  L.cidx = take((size_t)s->T * kSelMaxCand);
+  L.ncand = take((size_t)s->T * 4);
+  L.zmax = take((size_t)s->T * 4);
+  L.snc = take((size_t)s->T * 4);
+  L.zex = take((size_t)s->T * kSelMaxCand * 4);
+  L.ecount = take((size_t)s->E * 4);
   L.total = o;
   return L;
 }
@@ -252,7 +261,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 // CTA pairs (M = 256 tiles) for the bf16 expert GEMMs when the groups are large enough
 // to fill them: on average at least 192 rows per group.
 static bool use_pair_gemm(int mode, int BN, long long R, int n_groups, bool allow_pair) {
-  return allow_pair && mode != kModeF32 && BN == 256 && R >= 192ll * n_groups;
+  return allow_pair && mode != kModeF32 && mode != kModeRouterSel && BN == 256 && R >= 192ll * n_groups;
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
@@ -277,12 +286,14 @@ static int pick_bn(bool glu, int N, long long mtiles) {
 
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
                         int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
-                        cudaStream_t st, bool allow_pair, int a_kwrap = 0, const float* bias = nullptr) {
+                        cudaStream_t st, bool allow_pair, int a_kwrap = 0, const float* bias = nullptr,
+                        const RouterSelArgs* sel = nullptr) {
   if (R == 0) return MOE_OK;
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   // router logits: one column tile as wide as the expert count (fewer A re-reads)
-  const int BN = mode == kModeF32 ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
+  const bool router = mode == kModeF32 || mode == kModeRouterSel;
+  const int BN = router ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
   const bool pair = use_pair_gemm(mode, BN, R, n_groups, allow_pair);
   const int box_rows = (glu || pair) ? BN / 2 : BN;
   CUtensorMap ta, tb;
@@ -306,6 +317,7 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.a_kwrap = a_kwrap;
   p.out_f32 = reinterpret_cast<float*>(out);
   p.bias = bias;
+  p.sel = sel != nullptr ? *sel : RouterSelArgs{};
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   if (pair) {
     const long long ub2 = grows ? (R / (2 * kBM) + n_groups) : cdiv(R, 2 * kBM);
@@ -321,6 +333,8 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
   MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 192) MOE_GEMM_CASE(kModeF32, 128)
   MOE_GEMM_CASE(kModeF32, 64)
+  MOE_GEMM_CASE(kModeRouterSel, 256) MOE_GEMM_CASE(kModeRouterSel, 192) MOE_GEMM_CASE(kModeRouterSel, 128)
+  MOE_GEMM_CASE(kModeRouterSel, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -642,17 +656,48 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
     MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d);
     MOE_LAUNCH_CHECK();
-    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false,
-                      s->d, bias);
-    if (rc) return rc;
     // screening bound, relative to ||x_t|| max_e ||w_e|| (>= sum |x_i w_i|): the split's representation error
     // 2^-16, fp32 accumulation of 2d products in any rounding direction plus the bias add, and the error of the
     // exact recompute's own d-term fp32 chain; all with a 2^-7 margin
-    RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d,
-                   (float)((std::ldexp(1.0, -16) + (2.0 * s->d + 2.0) * std::ldexp(1.0, -23) +
-                            (s->d + 2.0) * std::ldexp(1.0, -24)) *
-                           (1.0 + std::ldexp(1.0, -7)))};
-    rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
+    const float gamma = (float)((std::ldexp(1.0, -16) + (2.0 * s->d + 2.0) * std::ldexp(1.0, -23) +
+                                 (s->d + 2.0) * std::ldexp(1.0, -24)) *
+                                (1.0 + std::ldexp(1.0, -7)));
+    const bool want_stats = aux_f || aux_p || aux;
+    if (logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD) {
+      // selection inside the screening GEMM's epilogue, exact recompute by expert, finish per token
+      float* xnorm2 = reinterpret_cast<float*>(ws + L.xnorm2);
+      int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
+      RouterSelArgs sel{xnorm2, wnorm, gamma, s->E, s->k, reinterpret_cast<uint8_t*>(ws + L.cidx),
+                        reinterpret_cast<int32_t*>(ws + L.ncand), reinterpret_cast<float*>(ws + L.zmax),
+                        reinterpret_cast<float*>(ws + L.snc), ecount, reinterpret_cast<int32_t*>(part)};
+      MOE_LAUNCH((k_router_xnorm), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
+                 xnorm2, ecount, (long long)s->T, s->d, s->E);
+      MOE_LAUNCH_CHECK();
+      rc = grouped_gemm(kModeRouterSel, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, nullptr, st,
+                        false, s->d, bias, &sel);
+      if (rc) return rc;
+      float* zex = reinterpret_cast<float*>(ws + L.zex);
+      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, kRecompSplit), 128, 0, st,
+                 reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, ecount, sel.elist, zex, (long long)s->T,
+                 s->d);
+      MOE_LAUNCH_CHECK();
+      const unsigned nch = (unsigned)cdiv(s->T, kChunk);
+      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+      if (s->E <= 128)
+        MOE_LAUNCH((k_router_finish<4>), nch, 256, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
+                   bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
+      else
+        MOE_LAUNCH((k_router_finish<8>), nch, 256, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
+                   bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
+      MOE_LAUNCH_CHECK();
+      rc = MOE_OK;
+    } else {
+      rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false,
+                        s->d, bias);
+      if (rc) return rc;
+      RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d, gamma};
+      rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
+    }
   } else if (logits_in == nullptr && s->T <= 256 && skinny_smem(s->d) <= kSkinnyMaxSmem) {
     const unsigned long long bit = 1ull << (current_device() & 63);
     if (!(g_skinny_attr.load() & bit)) {
@@ -811,10 +856,16 @@ int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos,
   const __nv_bfloat16* yp = reinterpret_cast<const __nv_bfloat16*>(y_perm);
   const __nv_bfloat16* ysh = reinterpret_cast<const __nv_bfloat16*>(y_shared);
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-  const unsigned blocks = (unsigned)cdiv(s->T, 8);
+  // 8 tokens per CTA; the columns split into ranges of whole 32-lane sweeps until there are about two CTAs
+  // per SM (a decode batch of 64 tokens would otherwise occupy 8 SMs)
+  const unsigned tok_blocks = (unsigned)cdiv(s->T, 8);
+  const int sweeps = (int)cdiv(s->d / 8, 32);
+  const int ranges = (int)std::max<long long>(1, std::min<long long>(sweeps, cdiv(2ll * num_sms(), tok_blocks)));
+  const int vpr = (int)cdiv(sweeps, ranges) * 32;
+  const dim3 grid(tok_blocks, (unsigned)cdiv(s->d / 8, vpr));
 #define MOE_COMBINE_CASE(N_)                                                                                   \
   if (s->k <= N_) {                                                                                            \
-    MOE_LAUNCH((k_combine<N_>), blocks, 256, 0, stream, yp, slot_pos, topk_w, ysh, o, (int)s->T, s->d, s->k);           \
+    MOE_LAUNCH((k_combine<N_>), grid, 256, 0, stream, yp, slot_pos, topk_w, ysh, o, (int)s->T, s->d, s->k, vpr);   \
     MOE_LAUNCH_CHECK();                                                                                        \
     return MOE_OK;                                                                                             \
   }

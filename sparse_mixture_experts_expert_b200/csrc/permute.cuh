@@ -181,19 +181,23 @@ __global__ void __launch_bounds__(128) k_group_table(const int32_t* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// Combine: one warp per token, fp32 sum over slots j = 0..k-1 in order, then
-// the shared expert, one bf16 rounding.  Each lane owns 16-byte column slices;
-// the k row loads of a slice are issued together.
+// Combine: one warp per (token, column range), fp32 sum over slots j = 0..k-1
+// in order, then the shared expert, one bf16 rounding.  Each lane owns 16-byte
+// column slices; the k row loads of a slice are issued together.  blockIdx.y
+// splits the columns into gridDim.y ranges of `vec_per_range` 16-byte slices so
+// that small batches (decode) still spread over every SM.
 template <int KMAX>
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict__ y_perm,
                                                  const int32_t* __restrict__ slot_pos, const float* __restrict__ w,
                                                  const __nv_bfloat16* __restrict__ y_shared,
-                                                 __nv_bfloat16* __restrict__ out, int T, int d, int k) {
+                                                 __nv_bfloat16* __restrict__ out, int T, int d, int k,
+                                                 int vec_per_range) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const int t = blockIdx.x * 8 + warp_id();
   const int lane = lane_id();
   if (t >= T) return;
-  const int nvec = d >> 3;
+  const int v_begin = blockIdx.y * vec_per_range;
+  const int nvec = min(d >> 3, v_begin + vec_per_range);
   int p[KMAX];
   float g[KMAX];
 #pragma unroll
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16* __restrict
     p[j] = j < k ? slot_pos[(size_t)t * k + j] : -1;
     g[j] = j < k ? w[(size_t)t * k + j] : 0.f;
   }
-  for (int v = lane; v < nvec; v += 32) {
+  for (int v = v_begin + lane; v < nvec; v += 32) {
     uint4 u[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)

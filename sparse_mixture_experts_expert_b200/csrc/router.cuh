@@ -155,6 +155,92 @@ __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W
   if (lane_id() == 0) wnorm[e] = sqrtf(ss);
 }
 
+// Token statistics for the certified selection inside the screening GEMM, one
+// warp per token: xnorm2[t] = sum_i x[t,i]^2 (bounds the screening error of
+// token t); block 0 also clears the per-expert candidate counters.
+__global__ void __launch_bounds__(256) k_router_xnorm(const __nv_bfloat16* __restrict__ x, float* __restrict__ xnorm2,
+                                                      int32_t* __restrict__ ecount, long long T, int d, int E) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) ecount[e] = 0;
+  const long long t = (long long)blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+  const int nv = d >> 3;
+  float ss = 0.f;
+  for (int v0 = lane_id(); v0 < nv; v0 += 128) {
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = v0 + 32 * j < nv ? xr[v0 + 32 * j] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float q[8] = {bf16lo(u[j].x), bf16hi(u[j].x), bf16lo(u[j].y), bf16hi(u[j].y),
+                          bf16lo(u[j].z), bf16hi(u[j].z), bf16lo(u[j].w), bf16hi(u[j].w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(q[i], q[i], ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane_id() == 0) xnorm2[t] = ss;
+}
+
+// Exact recompute of the selection candidates, expert-major: CTA (e, s) takes
+// slice s of expert e's candidate list, keeps W_r[e] (fp32) in shared memory
+// and computes each entry's logit with the whole warp -- lane l takes the
+// 8-input slices l, l+32, ..., one fmaf chain, a fixed xor tree, then the bias:
+// the same value for a (token, expert) pair whichever CTA or warp computes it.
+// Two entries per warp are in flight together.  zex[t][slot] = exact logit.
+constexpr int kRecompSplit = 4;     // CTAs per expert
+constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
+__global__ void __launch_bounds__(128) k_router_recompute(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ W, const float* __restrict__ bias,
+                                                          const int32_t* __restrict__ ecount,
+                                                          const int32_t* __restrict__ elist, float* __restrict__ zex,
+                                                          long long T, int d) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  __shared__ __align__(16) float s_w[kSelMaxD];
+  const int e = blockIdx.x;
+  const int L = ecount[e];
+  const int b = (int)((long long)L * blockIdx.y / gridDim.y), en = (int)((long long)L * (blockIdx.y + 1) / gridDim.y);
+  if (b >= en) return;
+  const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+  for (int i = threadIdx.x; i < d / 4; i += blockDim.x) reinterpret_cast<float4*>(s_w)[i] = wr[i];
+  __syncthreads();
+  const float be = bias != nullptr ? bias[e] : 0.f;
+  const int32_t* lst = elist + (size_t)e * T;
+  const int lane = lane_id(), nv = d >> 3;
+  for (int i = b + 2 * warp_id(); i < en; i += 2 * (blockDim.x / 32)) {
+    const bool two = i + 1 < en;
+    const int ent0 = lst[i], ent1 = two ? lst[i + 1] : ent0;
+    const uint4* x0 = reinterpret_cast<const uint4*>(x + (size_t)(ent0 / kSelMaxCand) * d);
+    const uint4* x1 = reinterpret_cast<const uint4*>(x + (size_t)(ent1 / kSelMaxCand) * d);
+    float a0 = 0.f, a1 = 0.f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 u0 = x0[v], u1 = x1[v];
+      const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
+      const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
+      a0 = fmaf(bf16lo(u0.x), w0.x, a0); a0 = fmaf(bf16hi(u0.x), w0.y, a0);
+      a0 = fmaf(bf16lo(u0.y), w0.z, a0); a0 = fmaf(bf16hi(u0.y), w0.w, a0);
+      a0 = fmaf(bf16lo(u0.z), w1.x, a0); a0 = fmaf(bf16hi(u0.z), w1.y, a0);
+      a0 = fmaf(bf16lo(u0.w), w1.z, a0); a0 = fmaf(bf16hi(u0.w), w1.w, a0);
+      a1 = fmaf(bf16lo(u1.x), w0.x, a1); a1 = fmaf(bf16hi(u1.x), w0.y, a1);
+      a1 = fmaf(bf16lo(u1.y), w0.z, a1); a1 = fmaf(bf16hi(u1.y), w0.w, a1);
+      a1 = fmaf(bf16lo(u1.z), w1.x, a1); a1 = fmaf(bf16hi(u1.z), w1.y, a1);
+      a1 = fmaf(bf16lo(u1.w), w1.z, a1); a1 = fmaf(bf16hi(u1.w), w1.w, a1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+    }
+    if (lane == 0) {
+      zex[ent0] = a0 + be;
+      if (two) zex[ent1] = a1 + be;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Warp argmax over the lanes' (value, index) pairs: larger value first, lower
 // index first among equal values (-0.0 == +0.0, so the index decides).
@@ -525,6 +611,99 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
     cnt[(size_t)e * nchunks + chunk] = cs;
     psum[(size_t)e * nchunks + chunk] = ps;
   }
+}
+
+// Selection finish, one warp per token, a CTA of 8 warps per 32-token chunk.
+// Lane c holds candidate c (exact logit, expert); the top k among them by
+// (value desc, index asc) -- certified to be the top k of all experts --
+// come from k rounds of warp argmax.  Softmax: m = the first pick's value,
+// sum = snc * exp(m_s - m) + sum over candidates of exp(z - m), where snc is
+// the epilogue's sum of exp(z_e - m_s) over the non-candidates (screening
+// values).  A token with more than kSelMaxCand candidates (degenerate logits)
+// is finished here from exact logits of every expert.  cnt[e][chunk] = picks.
+// Top k of one token from exact fp32 logits of every expert (lane l: experts
+// l, l+32, ...), for tokens with too many selection candidates.  Returns the
+// softmax denominator; m receives the largest logit.  Kept out of line: the
+// path is rare and must not weigh on the common one's registers.
+template <int EPL>
+__device__ __noinline__ float select_all_exact(const __nv_bfloat16* __restrict__ xr, const float* __restrict__ W,
+                                               const float* __restrict__ bias, int d, int E, int k, float& sel_v,
+                                               int& sel_i, float& m) {
+  const int lane = lane_id();
+  float z[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) z[i] = -INFINITY;
+  for (int e = 0; e < E; ++e) {
+    float v = warp_dot(xr, W + (size_t)e * d, d);
+    if (bias != nullptr) v += bias[e];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (e == lane + 32 * i) z[i] = v;
+  }
+  unsigned taken;
+  warp_topk<EPL>(z, E, k, sel_v, sel_i, taken);
+  m = __shfl_sync(0xffffffffu, sel_v, 0);
+  float ez = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) ez += (lane + 32 * i < E) ? __expf(z[i] - m) : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
+  return ez;
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict__ ncand,
+                                                       const uint8_t* __restrict__ cidx, const float* __restrict__ zex,
+                                                       const float* __restrict__ zmax, const float* __restrict__ snc,
+                                                       const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                                                       const float* __restrict__ bias, int32_t* __restrict__ topk_idx,
+                                                       float* __restrict__ topk_w, int32_t* __restrict__ cnt, int T,
+                                                       int d, int E, int k, int renorm) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  __shared__ int s_c[kMaxRouterE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_c[e] = 0;
+  __syncthreads();
+  const int lane = lane_id(), warp = warp_id();
+  const int chunk = blockIdx.x;
+  const int nchunks = (T + kChunk - 1) / kChunk;
+  for (int tt = 0; tt < kChunk / 8; ++tt) {
+    const int t = chunk * kChunk + warp * (kChunk / 8) + tt;
+    if (t >= T) break;
+    const int nc = ncand[t];
+    float sel_v = 0.f, m, ssum;
+    int sel_i = 0;
+    if (nc <= kSelMaxCand) {
+      float cv = lane < nc ? zex[(size_t)t * kSelMaxCand + lane] : -INFINITY;
+      int ci = lane < nc ? (int)cidx[(size_t)t * kSelMaxCand + lane] : 0x7fffffff;
+      const float cv0 = cv;
+      for (int j = 0; j < k; ++j) {
+        float bv = cv;
+        int bi = ci;
+        warp_argmax_redux(bv, bi);
+        if (lane == j) { sel_v = bv; sel_i = bi; }
+        if (ci == bi) cv = -INFINITY;    // taken (candidate ids are distinct)
+      }
+      m = __shfl_sync(0xffffffffu, sel_v, 0);
+      float ez = lane < nc ? __expf(cv0 - m) : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
+      ssum = ez + snc[t] * __expf(zmax[t] - m);
+    } else {
+      ssum = select_all_exact<EPL>(x + (size_t)t * d, W, bias, d, E, k, sel_v, sel_i, m);
+    }
+    const float inv = 1.f / ssum;
+    const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
+    float wsum = pj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = sel_i;
+      topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
+      atomicAdd(&s_c[sel_i], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)e * nchunks + chunk] = s_c[e];
 }
 
 // W_r [E][d] fp32 (global) -> shared memory as [d][pitch] (column e of row c =

@@ -102,6 +102,55 @@ def test_route_matches_oracle(lib, name, T, over):
         np.testing.assert_allclose(np64(r["aux"])[0], ref["aux"], rtol=5e-5)
 
 
+# Tensor-core router with the selection in the screening GEMM's epilogue (taken when neither logits nor the
+# load-balance statistic is requested): every k up to 16 (4- and 16-slot selection networks), column tiles of
+# 64 (E = 48: 16 padding columns), 192 and 256, the largest input width it takes (d = 2048), a skew bias, the
+# full granular batch, and tokens whose input row is zero (every logit equal, more candidates than the
+# selection keeps: those tokens are finished from exact logits of every expert, lowest indices first).
+@pytest.mark.parametrize("name,T,over,zero_rows", [("skewed", 3000, {}, 0), ("granular", 32768, {}, 0),
+                                                   ("granular", 1100, {"E": 256, "k": 8, "d": 1024}, 0),
+                                                   ("granular", 2100, {"E": 64, "k": 2, "d": 2048}, 0),
+                                                   ("skewed", 8000, {"E": 48, "k": 3}, 0),
+                                                   ("granular", 2000, {"k": 16}, 0),
+                                                   ("granular", 2000, {}, 37)])
+def test_route_select_path_matches_oracle(lib, name, T, over, zero_rows):
+    moe = lib
+    wl = synth.get_workload(name).replace(T=T, **over)
+    inp = synth.make_inputs(wl, seed=2, device="cpu", with_expert_weights=False)
+    x = inp["x"].clone()
+    if zero_rows:
+        x[5:5 + zero_rows] = 0
+    s = shape_of(moe, wl)
+    assert T * wl.E * wl.d >= 1 << 28 and wl.E % 16 == 0        # the tensor-core router's range
+    bias = inp["bias"].to(DEV) if inp["bias"] is not None else None
+    r = moe.moe_route(s, x.to(DEV), inp["w_router"].to(DEV), bias)                 # selection path
+    full = moe.moe_route(s, x.to(DEV), inp["w_router"].to(DEV), bias, logits=True)  # logits path
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    # both certify the same exact fp32 decisions
+    assert (npi(r["topk_idx"]) == npi(full["topk_idx"])).all()
+    assert (npi(r["counts"]) == npi(full["counts"])).all()
+    np.testing.assert_allclose(np64(r["topk_w"]), np64(full["topk_w"]), rtol=2e-6, atol=1e-9)
+    x64 = np64(x)
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref = O.route(x64, np64(inp["w_router"]), b64, wl.k, bool(wl.renorm))
+    amb = O.topk_margin(ref["z"], wl.k) < MARGIN
+    idx = npi(r["topk_idx"])
+    assert (idx[~amb] == ref["idx"][~amb]).all()
+    for t in np.nonzero(amb)[0]:
+        kth = np.sort(ref["z"][t])[::-1][wl.k - 1]
+        assert len(set(idx[t].tolist())) == wl.k
+        assert (ref["z"][t, idx[t]] >= kth - MARGIN).all()
+    if zero_rows:
+        # all logits equal the bias (none here): the k lowest expert indices, equal gates
+        assert (idx[5:5 + zero_rows] == np.arange(wl.k)[None, :]).all()
+        np.testing.assert_allclose(np64(r["topk_w"])[5:5 + zero_rows], 1.0 / wl.k, rtol=1e-6)
+    ok = ~amb
+    np.testing.assert_allclose(np64(r["topk_w"])[ok], ref["w"][ok], rtol=5e-5)
+    if not amb.any():
+        assert (npi(r["counts"]) == ref["counts"]).all()
+
+
 # ---------------------------------------------------------------- grouping
 
 
