@@ -41,7 +41,7 @@
 
 namespace moe {
 
-enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3, kModeRouterSel = 4 };
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3, kModeRouterSel = 4, kModeCombine = 5 };
 
 // Outputs of the router-selection epilogue (kModeRouterSel): for every token t
 // (one accumulator row) the screening logits of all experts sit in one TMEM
@@ -79,6 +79,12 @@ struct GemmParams {
   float* out_f32;      // kModeF32: fp32 output [R, N]
   const float* bias;   // kModeF32 / kModeRouterSel: optional per-column bias [N]
   RouterSelArgs sel;   // kModeRouterSel
+  // kModeCombine (the shared expert's down GEMM; row r = token r): out[r] = bf16(sum_j w[r,j] y_perm[slot[r,j]]
+  // + acc[r]), the routed sum in fp32 in slot order, then the shared expert's fp32 accumulator, one rounding
+  const int32_t* cmb_slot;        // [R, k] grouped row of (token, slot), -1 = dropped
+  const float* cmb_w;             // [R, k] gates
+  const __nv_bfloat16* cmb_y;     // [rows, N] routed expert outputs, row pitch ldo
+  int cmb_k;
 };
 
 #ifndef MOE_GEMM_MAX_STAGES
@@ -435,7 +441,7 @@ __global__ void __launch_bounds__(256, 1)
         const long long t = row0 + q * 32 + lane;
         if (p.sel.k <= 4) router_select<BN, 4>(p.sel, p.bias, p.R, t_row, valid, t, wmax, [&]() { release_acc(acc); });
         else router_select<BN, 16>(p.sel, p.bias, p.R, t_row, valid, t, wmax, [&]() { release_acc(acc); });
-      } else if (MODE == kModeF32) {
+      } else if (MODE == kModeF32 || MODE == kModeCombine) {
         // fp32 rows through the staging buffer, 32 columns (128 bytes per row) per round
         float* fstg = reinterpret_cast<float*>(stg);  // 32 rows x 36 floats per warp
         constexpr int FR = 36;
@@ -468,7 +474,26 @@ __global__ void __launch_bounds__(256, 1)
             const int rr = it * 4 + (lane >> 3);
             if (q * 32 + rr < rows_valid && col < p.N) {
               const float4 val = *reinterpret_cast<const float4*>(fstg + rr * FR + cb);
-              *reinterpret_cast<float4*>(p.out_f32 + (row0 + q * 32 + rr) * p.ldo + col) = val;
+              const long long r = row0 + q * 32 + rr;
+              if constexpr (MODE == kModeCombine) {
+                // weighted top-k sum of the token's routed rows (4 columns), slot order, then the shared expert
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int j = 0; j < p.cmb_k; ++j) {
+                  const int pos = p.cmb_slot[r * p.cmb_k + j];
+                  if (pos < 0) continue;
+                  const float g = p.cmb_w[r * p.cmb_k + j];
+                  const uint2 yv = *reinterpret_cast<const uint2*>(p.cmb_y + (long long)pos * p.ldo + col);
+                  c[0] = fmaf(g, bf16lo(yv.x), c[0]);
+                  c[1] = fmaf(g, bf16hi(yv.x), c[1]);
+                  c[2] = fmaf(g, bf16lo(yv.y), c[2]);
+                  c[3] = fmaf(g, bf16hi(yv.y), c[3]);
+                }
+                const uint2 o = make_uint2(pack_bf16x2(c[0] + val.x, c[1] + val.y),
+                                           pack_bf16x2(c[2] + val.z, c[3] + val.w));
+                *reinterpret_cast<uint2*>(p.out + r * p.ldo + col) = o;
+              } else {
+                *reinterpret_cast<float4*>(p.out_f32 + r * p.ldo + col) = val;
+              }
             }
           }
           __syncwarp();

@@ -284,10 +284,21 @@ static int pick_bn(bool glu, int N, long long mtiles) {
   return best == 0 ? 64 : best;
 }
 
+// Mode-specific inputs of grouped_gemm beyond the operands.
+struct GemmExtras {
+  int a_kwrap = 0;                   // router: A repeats every a_kwrap reduction columns
+  const float* bias = nullptr;       // router: per-expert logit bias
+  const RouterSelArgs* sel = nullptr;  // kModeRouterSel
+  const int32_t* cmb_slot = nullptr;   // kModeCombine: slot_pos [R, k]
+  const float* cmb_w = nullptr;        // kModeCombine: gates [R, k]
+  const void* cmb_y = nullptr;         // kModeCombine: routed outputs y_perm
+  int cmb_k = 0;
+};
+
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
                         int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
-                        cudaStream_t st, bool allow_pair, int a_kwrap = 0, const float* bias = nullptr,
-                        const RouterSelArgs* sel = nullptr) {
+                        cudaStream_t st, bool allow_pair, const GemmExtras& ex = GemmExtras{}) {
+  const int a_kwrap = ex.a_kwrap;
   if (R == 0) return MOE_OK;
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
@@ -316,14 +327,19 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.wait_limit_ns = g_wait_limit_ns.load();
   p.a_kwrap = a_kwrap;
   p.out_f32 = reinterpret_cast<float*>(out);
-  p.bias = bias;
-  p.sel = sel != nullptr ? *sel : RouterSelArgs{};
+  p.bias = ex.bias;
+  p.sel = ex.sel != nullptr ? *ex.sel : RouterSelArgs{};
+  p.cmb_slot = ex.cmb_slot;
+  p.cmb_w = ex.cmb_w;
+  p.cmb_y = reinterpret_cast<const __nv_bfloat16*>(ex.cmb_y);
+  p.cmb_k = ex.cmb_k;
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   if (pair) {
     const long long ub2 = grows ? (R / (2 * kBM) + n_groups) : cdiv(R, 2 * kBM);
     if (mode == kModePlain) return launch_gemm_t<kModePlain, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeSwiGLU) return launch_gemm_t<kModeSwiGLU, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeGeGLU) return launch_gemm_t<kModeGeGLU, 256, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeCombine) return launch_gemm_t<kModeCombine, 256, 2>(ta, tb, p, ub2, st);
     return MOE_UNSUPPORTED_SHAPE;
   }
 #define MOE_GEMM_CASE(M_, BN_) \
@@ -335,6 +351,7 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   MOE_GEMM_CASE(kModeF32, 64)
   MOE_GEMM_CASE(kModeRouterSel, 256) MOE_GEMM_CASE(kModeRouterSel, 192) MOE_GEMM_CASE(kModeRouterSel, 128)
   MOE_GEMM_CASE(kModeRouterSel, 64)
+  MOE_GEMM_CASE(kModeCombine, 256) MOE_GEMM_CASE(kModeCombine, 128) MOE_GEMM_CASE(kModeCombine, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -673,8 +690,12 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       MOE_LAUNCH((k_router_xnorm), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
                  xnorm2, ecount, (long long)s->T, s->d, s->E);
       MOE_LAUNCH_CHECK();
+      GemmExtras ex;
+      ex.a_kwrap = s->d;
+      ex.bias = bias;
+      ex.sel = &sel;
       rc = grouped_gemm(kModeRouterSel, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, nullptr, st,
-                        false, s->d, bias, &sel);
+                        false, ex);
       if (rc) return rc;
       float* zex = reinterpret_cast<float*>(ws + L.zex);
       MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, kRecompSplit), 128, 0, st,
@@ -692,8 +713,11 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       MOE_LAUNCH_CHECK();
       rc = MOE_OK;
     } else {
+      GemmExtras ex;
+      ex.a_kwrap = s->d;
+      ex.bias = bias;
       rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false,
-                        s->d, bias);
+                        ex);
       if (rc) return rc;
       RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d, gamma};
       rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
@@ -918,6 +942,22 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
   if (rc) return rc;
   void* ys = nullptr;
+  if (s->H_s > 0 && s->wfmt == MOE_WFMT_BF16) {
+    // shared expert: gate/up, then the down GEMM whose epilogue adds each token's weighted routed rows (the
+    // combine) to the shared expert's fp32 accumulator and rounds once
+    const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
+    const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
+    rc = grouped_gemm(mode, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, s->H_s, s->H_s, nullptr, nullptr, ws + L.hs,
+                      stream, pair);
+    if (rc) return rc;
+    GemmExtras ex;
+    ex.cmb_slot = slot;
+    ex.cmb_w = w;
+    ex.cmb_y = yperm;
+    ex.cmb_k = s->k;
+    return grouped_gemm(kModeCombine, ws + L.hs, s->T, s->H_s, w2_sh, 1, s->d, 0, s->d, nullptr, nullptr, out,
+                        stream, pair, ex);
+  }
   if (s->H_s > 0) {
     ys = ws + L.ys;
     rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
