@@ -186,9 +186,12 @@ int moe_permute(const moe_shape* s, const void* x, const int32_t* topk_idx, int3
  *   x_grouped     [R, d] bf16             in
  *   w13, w2       expert weights, layout per s->wfmt (n_groups experts)
  *   s13, s2       INT4 scales (NULL for bf16)
- *   h             [R, hidden] bf16        out (scratch the caller may read)
+ *   h             [R, hidden] bf16        out (scratch the caller may read), or NULL for bf16 experts of
+ *                                         hidden 128 or 256: then one fused kernel keeps each row tile's h
+ *                                         in shared memory and h is not written (other shapes: NULL gives
+ *                                         MOE_INVALID_ARGUMENT)
  *   y             [R, d] bf16             out  rows outside every group are untouched
- * Accumulation is fp32; h is rounded to bf16 once, y once.
+ * Accumulation is fp32; h is rounded to bf16 once, y once (the same values with h NULL or not).
  */
 int moe_expert_ffn(const moe_shape* s, int32_t n_groups, int32_t hidden, int64_t R, const void* x_grouped,
                    const int32_t* group_start, const int32_t* group_rows, const void* w13, const void* s13,

@@ -253,12 +253,14 @@ def moe_permute_noalloc(shape: MoeShape, x, topk_idx, *, stream=None):
 
 
 def moe_expert_ffn(shape: MoeShape, x_grouped, w13, w2, *, hidden=None, group_start=None, group_rows=None,
-                   s13=None, s2=None, h=None, y=None, stream=None):
+                   s13=None, s2=None, h=None, y=None, want_h=True, stream=None):
+    """Grouped gated expert FFN.  Returns (h, y); with ``want_h=False`` (bf16 experts of hidden 128 or 256) h
+    stays on chip in the fused kernel and None is returned in its place."""
     hidden = shape.H if hidden is None else hidden
     R = x_grouped.shape[0]
     n_groups = w13.shape[0]
     dev = x_grouped.device
-    if h is None:
+    if h is None and want_h:
         h = torch.empty(R, hidden, dtype=torch.bfloat16, device=dev)
     if y is None:
         y = torch.empty(R, shape.d, dtype=torch.bfloat16, device=dev)

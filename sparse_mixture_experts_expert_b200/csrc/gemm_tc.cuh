@@ -130,7 +130,7 @@ __device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + e
 // network.  Pass 2: the candidates (z >= k-th - 2 bound), written in expert
 // order and appended to their experts' lists (order inside a list is
 // irrelevant: each entry's exact value does not depend on it), and the sum of
-// exp(z - max) over the non-candidates; the accumulator is released after its
+// exp(z - max) over the non-candidates.  The accumulator is released after its
 // last read.
 template <int BN, int KM, typename Release>
 __device__ __forceinline__ void router_select(const RouterSelArgs a, const float* __restrict__ bias, long long R,
@@ -163,35 +163,50 @@ __device__ __forceinline__ void router_select(const RouterSelArgs a, const float
   const float xn = valid ? sqrtf(a.xnorm2[t]) : 0.f;
   const float bound = a.gamma * xn * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
   const float thr = kth - 2.f * bound;
+  // pass 2, 32 columns at a time: the warp's candidates of each column (ballot), one list reservation per
+  // column for the whole warp (all 32 atomics of a chunk are issued before any result is used), then each
+  // candidate's slot (its rank among the token's candidates, expert order) and list entry
+  const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
   float snc = 0.f;
-  int nc = 0;
+  int nc = 0;        // the token's candidates so far (all of them)
+  int slot = 0;      // candidates written (at most kSelMaxCand)
 #pragma unroll 1
   for (int c0 = 0; c0 < BN; c0 += 32) {
     uint32_t v[2][16];
     tmem_ld16(t_row + c0, v[0]);
     tmem_ld16(t_row + c0 + 16, v[1]);
     tmem_ld_wait();
-    if (c0 + 32 >= BN) release();
+    uint32_t m[32];
+    int base[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int col = c0 + i;
+      bool keep = false;
       if (col < a.E) {
         const float z = __uint_as_float(v[i >> 4][i & 15]) + (bias != nullptr ? bias[col] : 0.f);
-        if (z >= thr) {
-          // candidate: kept in expert order; past kSelMaxCand only counted (the finishing kernel then
-          // ignores this token's list entries and recomputes every expert)
-          if (valid && nc < kSelMaxCand) {
-            a.cidx[t * kSelMaxCand + nc] = (uint8_t)col;
-            const int pos = atomicAdd(&a.ecount[col], 1);
-            a.elist[(long long)col * R + pos] = (int32_t)(t * kSelMaxCand + nc);
-          }
-          ++nc;
-        } else {
-          snc += __expf(z - m_s);
+        const bool isc = valid && z >= thr;
+        keep = isc && nc < kSelMaxCand;
+        nc += isc ? 1 : 0;
+        if (!isc) snc += __expf(z - m_s);
+      }
+      m[i] = __ballot_sync(0xffffffffu, keep);
+      base[i] = 0;
+      if (m[i] != 0u && (threadIdx.x & 31) == __ffs(m[i]) - 1) base[i] = atomicAdd(&a.ecount[col], __popc(m[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (m[i] != 0u) {
+        const int col = c0 + i;
+        const int b = __shfl_sync(0xffffffffu, base[i], __ffs(m[i]) - 1);
+        if ((m[i] >> (threadIdx.x & 31)) & 1u) {
+          a.cidx[t * kSelMaxCand + slot] = (uint8_t)col;
+          a.elist[(long long)col * R + b + __popc(m[i] & lt)] = (int32_t)(t * kSelMaxCand + slot);
+          ++slot;
         }
       }
     }
   }
+  release();
   if (!valid) return;
   a.ncand[t] = nc;
   a.zmax[t] = m_s;

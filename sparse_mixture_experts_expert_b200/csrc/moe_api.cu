@@ -9,6 +9,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "expert_fused.cuh"
 #include "gemm_tc.cuh"
 #include "int4_gemm.cuh"
 #include "permute.cuh"
@@ -437,6 +438,68 @@ static int launch_scatter(const moe_shape* s, const void* x, const int32_t* idx,
   return MOE_UNSUPPORTED_SHAPE;
 }
 
+// Fused routed expert FFN (bf16, hidden 128 or 256): h stays in shared memory.  y [R, d] bf16.
+template <int MODE, int H, int CG>
+static int launch_fused_t(const void* A, long long R, int d, const void* w13, const void* w2, int n_groups,
+                          const int32_t* gstart, const int32_t* grows, void* y, cudaStream_t st) {
+  using Cfg = FusedCfg<H, CG>;
+  static std::atomic<unsigned long long> done_mask{0};
+  const unsigned long long bit = 1ull << (current_device() & 63);
+  if (!(done_mask.load(std::memory_order_relaxed) & bit)) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(k_expert_fused<MODE, H, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)Cfg::kSmemBytes));
+    done_mask.fetch_or(bit);
+  }
+  CUtensorMap tx, t13, t2;
+  const cuuint64_t dx[2] = {(cuuint64_t)d, (cuuint64_t)R};
+  const cuuint64_t d13[3] = {(cuuint64_t)d, (cuuint64_t)(2 * H), (cuuint64_t)n_groups};
+  const cuuint64_t d2[3] = {(cuuint64_t)H, (cuuint64_t)d, (cuuint64_t)n_groups};
+  int rc = make_map(&tx, A, 2, dx, kBM);
+  if (rc) return rc;
+  rc = make_map(&t13, w13, 3, d13, 128);
+  if (rc) return rc;
+  rc = make_map(&t2, w2, 3, d2, CG == 2 ? 128 : 256);
+  if (rc) return rc;
+  GemmParams p{};
+  p.group_start = gstart;
+  p.group_rows = grows;
+  p.n_groups = n_groups;
+  p.R = R;
+  p.K = d;
+  p.N = d;
+  p.up_row0 = H;
+  p.out = reinterpret_cast<__nv_bfloat16*>(y);
+  p.ldo = d;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const long long TM = (long long)kBM * CG;
+  const long long tiles = grows ? (R / TM + n_groups) : cdiv(R, TM);
+  const int units = (int)std::max<long long>(1, std::min<long long>(num_sms() / CG, tiles));
+  MOE_CUDA_TRY(launch_pdl(k_expert_fused<MODE, H, CG>, dim3((unsigned)(CG * units)), dim3(256), Cfg::kSmemBytes, st,
+                          (unsigned)CG, tx, t13, t2, p));
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+static bool fused_ffn_ok(const moe_shape* s, int hidden) {
+  return s->wfmt == MOE_WFMT_BF16 && (hidden == 128 || hidden == 256);
+}
+
+static int launch_fused(const moe_shape* s, int hidden, long long R, const void* A, const int32_t* gstart,
+                        const int32_t* grows, int n_groups, const void* w13, const void* w2, void* y,
+                        cudaStream_t st) {
+  if (R == 0) return MOE_OK;
+  const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM) && R >= 192ll * n_groups;
+  const bool geglu = s->act == MOE_ACT_GEGLU;
+#define MOE_FUSED_FFN(M_, H_, CG_) \
+  if ((M_ == kModeGeGLU) == geglu && hidden == H_ && (CG_ == 2) == pair) \
+    return launch_fused_t<M_, H_, CG_>(A, R, s->d, w13, w2, n_groups, gstart, grows, y, st);
+  MOE_FUSED_FFN(kModeSwiGLU, 256, 2) MOE_FUSED_FFN(kModeSwiGLU, 256, 1) MOE_FUSED_FFN(kModeSwiGLU, 128, 2)
+  MOE_FUSED_FFN(kModeSwiGLU, 128, 1) MOE_FUSED_FFN(kModeGeGLU, 256, 2) MOE_FUSED_FFN(kModeGeGLU, 256, 1)
+  MOE_FUSED_FFN(kModeGeGLU, 128, 2) MOE_FUSED_FFN(kModeGeGLU, 128, 1)
+#undef MOE_FUSED_FFN
+  return MOE_UNSUPPORTED_SHAPE;
+}
+
 // Optional scratch for the offset-code kernel: xsum [R, K/128] fp32 (activation group sums) and
 // xq [R, K] bf16 (the fragment-ordered copy of A).  Without it the plain-code kernel runs.
 struct Int4Scratch {
@@ -566,6 +629,7 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
     if (rc) return rc;
     return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st, scr);
   }
+  if (h == nullptr) return launch_fused(s, hidden, R, A, gstart, grows, n_groups, w13, w2, y, st);
   const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
   const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
   rc = grouped_gemm(mode, A, R, s->d, w13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st, pair);
@@ -698,17 +762,17 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
                         false, ex);
       if (rc) return rc;
       float* zex = reinterpret_cast<float*>(ws + L.zex);
-      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, kRecompSplit), 128, 0, st,
+      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, kRecompSplit), 256, 0, st,
                  reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, ecount, sel.elist, zex, (long long)s->T,
                  s->d);
       MOE_LAUNCH_CHECK();
       const unsigned nch = (unsigned)cdiv(s->T, kChunk);
       const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
       if (s->E <= 128)
-        MOE_LAUNCH((k_router_finish<4>), nch, 256, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
+        MOE_LAUNCH((k_router_finish<4>), nch, 1024, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
                    bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
       else
-        MOE_LAUNCH((k_router_finish<8>), nch, 256, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
+        MOE_LAUNCH((k_router_finish<8>), nch, 1024, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
                    bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
       MOE_LAUNCH_CHECK();
       rc = MOE_OK;
@@ -860,8 +924,9 @@ int moe_expert_ffn(const moe_shape* s, int32_t n_groups, int32_t hidden, int64_t
   if ((group_start == nullptr) != (group_rows == nullptr)) return MOE_INVALID_ARGUMENT;
   if (group_start == nullptr && n_groups != 1) return MOE_INVALID_ARGUMENT;
   if (R == 0) return MOE_OK;
-  if (!x_grouped || !w13 || !w2 || !h || !y) return MOE_INVALID_ARGUMENT;
-  if (!aligned16(x_grouped) || !aligned16(w13) || !aligned16(w2) || !aligned16(h) || !aligned16(y))
+  if (!x_grouped || !w13 || !w2 || !y) return MOE_INVALID_ARGUMENT;
+  if (h == nullptr && !fused_ffn_ok(s, hidden)) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x_grouped) || !aligned16(w13) || !aligned16(w2) || (h && !aligned16(h)) || !aligned16(y))
     return MOE_INVALID_ARGUMENT;
   if (s->wfmt == MOE_WFMT_INT4_G128) {
     if (hidden % 128 != 0) return MOE_UNSUPPORTED_SHAPE;
@@ -939,7 +1004,8 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
                               ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq,
                                             reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
                               : Int4Scratch{nullptr, nullptr};
-  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
+  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, fused_ffn_ok(s, s->H) ? nullptr : hbuf,
+                       yperm, stream, scr);
   if (rc) return rc;
   void* ys = nullptr;
   if (s->H_s > 0 && s->wfmt == MOE_WFMT_BF16) {

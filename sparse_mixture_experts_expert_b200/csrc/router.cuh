@@ -189,11 +189,13 @@ __global__ void __launch_bounds__(256) k_router_xnorm(const __nv_bfloat16* __res
 // slice s of expert e's candidate list, keeps W_r[e] (fp32) in shared memory
 // and computes each entry's logit with the whole warp -- lane l takes the
 // 8-input slices l, l+32, ..., one fmaf chain, a fixed xor tree, then the bias:
-// the same value for a (token, expert) pair whichever CTA or warp computes it.
-// Two entries per warp are in flight together.  zex[t][slot] = exact logit.
+// the same value for a (token, expert) pair whichever CTA or warp computes it,
+// and the same as warp_dot.  A warp keeps kRecompBatch entries in flight (their
+// input loads issued together).  zex[t][slot] = exact logit.
 constexpr int kRecompSplit = 4;     // CTAs per expert
+constexpr int kRecompBatch = 8;     // entries per warp in flight
 constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
-__global__ void __launch_bounds__(128) k_router_recompute(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ W, const float* __restrict__ bias,
                                                           const int32_t* __restrict__ ecount,
                                                           const int32_t* __restrict__ elist, float* __restrict__ zex,
@@ -210,33 +212,46 @@ __global__ void __launch_bounds__(128) k_router_recompute(const __nv_bfloat16* _
   const float be = bias != nullptr ? bias[e] : 0.f;
   const int32_t* lst = elist + (size_t)e * T;
   const int lane = lane_id(), nv = d >> 3;
-  for (int i = b + 2 * warp_id(); i < en; i += 2 * (blockDim.x / 32)) {
-    const bool two = i + 1 < en;
-    const int ent0 = lst[i], ent1 = two ? lst[i + 1] : ent0;
-    const uint4* x0 = reinterpret_cast<const uint4*>(x + (size_t)(ent0 / kSelMaxCand) * d);
-    const uint4* x1 = reinterpret_cast<const uint4*>(x + (size_t)(ent1 / kSelMaxCand) * d);
-    float a0 = 0.f, a1 = 0.f;
+  const int nwarps = blockDim.x / 32;
+  for (int i0 = b + kRecompBatch * warp_id(); i0 < en; i0 += kRecompBatch * nwarps) {
+    int ent[kRecompBatch];
+    const uint4* xr[kRecompBatch];
+#pragma unroll
+    for (int j = 0; j < kRecompBatch; ++j) {
+      ent[j] = lst[min(i0 + j, en - 1)];
+      xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
+    }
+    float acc[kRecompBatch];
+#pragma unroll
+    for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
     for (int v = lane; v < nv; v += 32) {
-      const uint4 u0 = x0[v], u1 = x1[v];
+      uint4 u[kRecompBatch];
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
       const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
       const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
-      a0 = fmaf(bf16lo(u0.x), w0.x, a0); a0 = fmaf(bf16hi(u0.x), w0.y, a0);
-      a0 = fmaf(bf16lo(u0.y), w0.z, a0); a0 = fmaf(bf16hi(u0.y), w0.w, a0);
-      a0 = fmaf(bf16lo(u0.z), w1.x, a0); a0 = fmaf(bf16hi(u0.z), w1.y, a0);
-      a0 = fmaf(bf16lo(u0.w), w1.z, a0); a0 = fmaf(bf16hi(u0.w), w1.w, a0);
-      a1 = fmaf(bf16lo(u1.x), w0.x, a1); a1 = fmaf(bf16hi(u1.x), w0.y, a1);
-      a1 = fmaf(bf16lo(u1.y), w0.z, a1); a1 = fmaf(bf16hi(u1.y), w0.w, a1);
-      a1 = fmaf(bf16lo(u1.z), w1.x, a1); a1 = fmaf(bf16hi(u1.z), w1.y, a1);
-      a1 = fmaf(bf16lo(u1.w), w1.z, a1); a1 = fmaf(bf16hi(u1.w), w1.w, a1);
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) {
+        float a = acc[j];
+        a = fmaf(bf16lo(u[j].x), w0.x, a); a = fmaf(bf16hi(u[j].x), w0.y, a);
+        a = fmaf(bf16lo(u[j].y), w0.z, a); a = fmaf(bf16hi(u[j].y), w0.w, a);
+        a = fmaf(bf16lo(u[j].z), w1.x, a); a = fmaf(bf16hi(u[j].z), w1.y, a);
+        a = fmaf(bf16lo(u[j].w), w1.z, a); a = fmaf(bf16hi(u[j].w), w1.w, a);
+        acc[j] = a;
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+    for (int j = 0; j < kRecompBatch; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
     }
-    if (lane == 0) {
-      zex[ent0] = a0 + be;
-      if (two) zex[ent1] = a1 + be;
+    if (lane < kRecompBatch) {
+      float mine = acc[0];
+      int my_ent = ent[0];
+#pragma unroll
+      for (int j = 1; j < kRecompBatch; ++j)
+        if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
+      if (i0 + lane < en) zex[my_ent] = mine + be;
     }
   }
 }
@@ -613,7 +628,7 @@ __global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int 
   }
 }
 
-// Selection finish, one warp per token, a CTA of 8 warps per 32-token chunk.
+// Selection finish, one warp per token, a CTA of 32 warps per 32-token chunk.
 // Lane c holds candidate c (exact logit, expert); the top k among them by
 // (value desc, index asc) -- certified to be the top k of all experts --
 // come from k rounds of warp argmax.  Softmax: m = the first pick's value,
@@ -652,7 +667,7 @@ __device__ __noinline__ float select_all_exact(const __nv_bfloat16* __restrict__
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict__ ncand,
+__global__ void __launch_bounds__(1024) k_router_finish(const int32_t* __restrict__ ncand,
                                                        const uint8_t* __restrict__ cidx, const float* __restrict__ zex,
                                                        const float* __restrict__ zmax, const float* __restrict__ snc,
                                                        const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
@@ -666,9 +681,9 @@ __global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict
   const int lane = lane_id(), warp = warp_id();
   const int chunk = blockIdx.x;
   const int nchunks = (T + kChunk - 1) / kChunk;
-  for (int tt = 0; tt < kChunk / 8; ++tt) {
-    const int t = chunk * kChunk + warp * (kChunk / 8) + tt;
-    if (t >= T) break;
+  {
+    const int t = chunk * kChunk + warp;   // one token per warp, kChunk warps per CTA
+    if (t >= T) goto stats;
     const int nc = ncand[t];
     float sel_v = 0.f, m, ssum;
     int sel_i = 0;
@@ -702,6 +717,7 @@ __global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict
       atomicAdd(&s_c[sel_i], 1);
     }
   }
+stats:
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)e * nchunks + chunk] = s_c[e];
 }
