@@ -138,7 +138,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 
 struct Workspace {
   size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
-  size_t xnorm2, cidx, ncand, zmax, snc, zex, ecount;   // certified selection inside the screening GEMM
+  size_t xnorm2, cidx, ncand, zmax, snc, zex, ecnt, elist;   // certified selection inside the screening GEMM
   size_t total;
 };
 
@@ -148,6 +148,8 @@ static size_t i4part_floats(const moe_shape* s) {
   if (s->wfmt != MOE_WFMT_INT4_G128 || s->H_s == 0 || s->T > 256) return 0;
   return (size_t)8 * s->T * std::max(2 * s->H_s, s->d);
 }
+
+static bool use_tc_router(const moe_shape* s);
 
 static Workspace ws_layout(const moe_shape* s) {
   Workspace L{};
@@ -187,7 +189,8 @@ static Workspace ws_layout(const moe_shape* s) {
   L.zmax = take((size_t)s->T * 4);
   L.snc = take((size_t)s->T * 4);
   L.zex = take((size_t)s->T * kSelMaxCand * 4);
-  L.ecount = take((size_t)s->E * 4);
+  L.ecnt = take((size_t)s->E * cdiv(s->T, 128) * 4);
+  L.elist = use_tc_router(s) ? take((size_t)s->E * cdiv(s->T, 128) * 128 * 4) : take(16);
   L.total = o;
   return L;
 }
@@ -371,8 +374,12 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   const bool small = s->T <= 2048;
   // the certifying recompute holds the token's inputs in registers when d <= 1024
   const bool xreg = refine.x != nullptr && refine.d <= 1024;
+  // warps per CTA: decode batches (T <= 256, final logits) two tokens per warp, a 32-token chunk per CTA with
+  // the chunk tables formed in the kernel; other small batches 4 tokens per CTA (tables by k_chunk_stats);
+  // large batches 8 warps per chunk
+  const int nw = (s->T <= 256 && refine.x == nullptr) ? 16 : (small ? 4 : 8);
 #define MOE_TOPK_CASE(N_, NW_, XR_, ST_)                                                                          \
-  if (epl <= N_ && (small ? 4 : 8) == NW_ && xreg == XR_) {                                                       \
+  if (epl <= N_ && nw == NW_ && xreg == XR_) {                                                                    \
     const size_t smem = ST_ ? (size_t)2 * NW_ * s->E * sizeof(float) : 0;                                         \
     if (smem > 48 * 1024) {                                                                                       \
       static std::atomic<unsigned long long> attr_done{0};                                                        \
@@ -400,6 +407,7 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   MOE_TOPK_CASE(6, NW_, XR_, ST_) MOE_TOPK_CASE(8, NW_, XR_, ST_) MOE_TOPK_CASE(12, NW_, XR_, ST_)                \
   MOE_TOPK_CASE(16, NW_, XR_, ST_)
   MOE_TOPK_EPL(8, false, true) MOE_TOPK_EPL(8, true, true) MOE_TOPK_EPL(4, false, false) MOE_TOPK_EPL(4, true, false)
+  MOE_TOPK_EPL(16, false, true)
 #undef MOE_TOPK_EPL
 #undef MOE_TOPK_CASE
   return MOE_UNSUPPORTED_SHAPE;
@@ -747,12 +755,13 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     if (logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD) {
       // selection inside the screening GEMM's epilogue, exact recompute by expert, finish per token
       float* xnorm2 = reinterpret_cast<float*>(ws + L.xnorm2);
-      int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
+      const int ntiles = (int)cdiv(s->T, 128);
       RouterSelArgs sel{xnorm2, wnorm, gamma, s->E, s->k, reinterpret_cast<uint8_t*>(ws + L.cidx),
                         reinterpret_cast<int32_t*>(ws + L.ncand), reinterpret_cast<float*>(ws + L.zmax),
-                        reinterpret_cast<float*>(ws + L.snc), ecount, reinterpret_cast<int32_t*>(part)};
+                        reinterpret_cast<float*>(ws + L.snc), reinterpret_cast<int32_t*>(ws + L.ecnt),
+                        reinterpret_cast<int32_t*>(ws + L.elist), ntiles};
       MOE_LAUNCH((k_router_xnorm), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
-                 xnorm2, ecount, (long long)s->T, s->d, s->E);
+                 xnorm2, (long long)s->T, s->d);
       MOE_LAUNCH_CHECK();
       GemmExtras ex;
       ex.a_kwrap = s->d;
@@ -762,9 +771,8 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
                         false, ex);
       if (rc) return rc;
       float* zex = reinterpret_cast<float*>(ws + L.zex);
-      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, kRecompSplit), 256, 0, st,
-                 reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, ecount, sel.elist, zex, (long long)s->T,
-                 s->d);
+      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, (unsigned)cdiv(ntiles, kRecompTiles)), 256, 0, st,
+                 reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, sel.ecnt, sel.elist, zex, ntiles, s->d);
       MOE_LAUNCH_CHECK();
       const unsigned nch = (unsigned)cdiv(s->T, kChunk);
       const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);

@@ -157,12 +157,10 @@ __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W
 
 // Token statistics for the certified selection inside the screening GEMM, one
 // warp per token: xnorm2[t] = sum_i x[t,i]^2 (bounds the screening error of
-// token t); block 0 also clears the per-expert candidate counters.
+// token t).
 __global__ void __launch_bounds__(256) k_router_xnorm(const __nv_bfloat16* __restrict__ x, float* __restrict__ xnorm2,
-                                                      int32_t* __restrict__ ecount, long long T, int d, int E) {
+                                                      long long T, int d) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  if (blockIdx.x == 0)
-    for (int e = threadIdx.x; e < E; e += blockDim.x) ecount[e] = 0;
   const long long t = (long long)blockIdx.x * 8 + warp_id();
   if (t >= T) return;
   const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
@@ -186,39 +184,67 @@ __global__ void __launch_bounds__(256) k_router_xnorm(const __nv_bfloat16* __res
 }
 
 // Exact recompute of the selection candidates, expert-major: CTA (e, s) takes
-// slice s of expert e's candidate list, keeps W_r[e] (fp32) in shared memory
-// and computes each entry's logit with the whole warp -- lane l takes the
-// 8-input slices l, l+32, ..., one fmaf chain, a fixed xor tree, then the bias:
-// the same value for a (token, expert) pair whichever CTA or warp computes it,
-// and the same as warp_dot.  A warp keeps kRecompBatch entries in flight (their
-// input loads issued together).  zex[t][slot] = exact logit.
-constexpr int kRecompSplit = 4;     // CTAs per expert
+// the (expert e, tile) segments of tiles [s * kRecompTiles, (s+1) *
+// kRecompTiles), keeps W_r[e] (fp32) in shared memory and computes each
+// entry's logit with the whole warp -- lane l takes the 8-input slices l,
+// l+32, ..., one fmaf chain, a fixed xor tree, then the bias: the same value
+// for a (token, expert) pair whichever CTA or warp computes it, and the same as
+// warp_dot.  A warp keeps kRecompBatch entries in flight (their input loads
+// issued together).  zex[t][slot] = exact logit.
+constexpr int kRecompTiles = 64;    // 128-token tiles per CTA
 constexpr int kRecompBatch = 8;     // entries per warp in flight
 constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
 __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ W, const float* __restrict__ bias,
-                                                          const int32_t* __restrict__ ecount,
+                                                          const int32_t* __restrict__ ecnt,
                                                           const int32_t* __restrict__ elist, float* __restrict__ zex,
-                                                          long long T, int d) {
+                                                          int ntiles, int d) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ __align__(16) float s_w[kSelMaxD];
+  __shared__ int s_pre[kRecompTiles + 1];
   const int e = blockIdx.x;
-  const int L = ecount[e];
-  const int b = (int)((long long)L * blockIdx.y / gridDim.y), en = (int)((long long)L * (blockIdx.y + 1) / gridDim.y);
-  if (b >= en) return;
+  const int tb = blockIdx.y * kRecompTiles;
+  const int nt = min(kRecompTiles, ntiles - tb);
+  if (nt <= 0) return;
+  const int lane = lane_id();
+  if (warp_id() == 0) {
+    // exclusive prefix of the segment sizes (two tiles per lane)
+    const int i0 = 2 * lane, i1 = 2 * lane + 1;
+    const int c0 = i0 < nt ? ecnt[(size_t)e * ntiles + tb + i0] : 0;
+    const int c1 = i1 < nt ? ecnt[(size_t)e * ntiles + tb + i1] : 0;
+    int incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - c0 - c1;
+    if (i0 <= nt) s_pre[i0] = excl;
+    if (i1 <= nt) s_pre[i1] = excl + c0;
+    if (lane == 31 && 64 <= nt) s_pre[64] = incl;
+  }
+  __syncthreads();
+  const int total = s_pre[nt];
+  if (total == 0) return;
   const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
   for (int i = threadIdx.x; i < d / 4; i += blockDim.x) reinterpret_cast<float4*>(s_w)[i] = wr[i];
   __syncthreads();
   const float be = bias != nullptr ? bias[e] : 0.f;
-  const int32_t* lst = elist + (size_t)e * T;
-  const int lane = lane_id(), nv = d >> 3;
+  const int32_t* seg = elist + ((size_t)e * ntiles + tb) * 128;
+  const int nv = d >> 3;
   const int nwarps = blockDim.x / 32;
-  for (int i0 = b + kRecompBatch * warp_id(); i0 < en; i0 += kRecompBatch * nwarps) {
+  for (int f0 = kRecompBatch * warp_id(); f0 < total; f0 += kRecompBatch * nwarps) {
     int ent[kRecompBatch];
     const uint4* xr[kRecompBatch];
 #pragma unroll
     for (int j = 0; j < kRecompBatch; ++j) {
-      ent[j] = lst[min(i0 + j, en - 1)];
+      const int f = min(f0 + j, total - 1);
+      int lo = 0, hi = nt - 1;   // last tile with s_pre[tile] <= f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= f) lo = mid; else hi = mid - 1;
+      }
+      ent[j] = seg[lo * 128 + (f - s_pre[lo])];
       xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
     }
     float acc[kRecompBatch];
@@ -251,7 +277,7 @@ __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* _
 #pragma unroll
       for (int j = 1; j < kRecompBatch; ++j)
         if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
-      if (i0 + lane < en) zex[my_ent] = mine + be;
+      if (f0 + lane < total) zex[my_ent] = mine + be;
     }
   }
 }
@@ -461,7 +487,7 @@ __device__ __forceinline__ float warp_dot_reg(const float (&xf)[32], const float
 //   forms the tables.  p_out may alias part: a warp writes row t only after
 //   reading every split of row t.
 template <int EPL, int NW, bool XREG, bool STATS>
-__global__ void __launch_bounds__(NW * 32) k_router_topk(const float* part, int nsplit,
+__global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, int nsplit,
                                                          const float* __restrict__ bias, float* __restrict__ logits_out,
                                                          int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                                                          int32_t* __restrict__ cnt, float* __restrict__ psum,
