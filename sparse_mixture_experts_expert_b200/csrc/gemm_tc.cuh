@@ -41,31 +41,7 @@
 
 namespace moe {
 
-enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3, kModeRouterSel = 4, kModeCombine = 5 };
-
-// Outputs of the router-selection epilogue (kModeRouterSel): for every token t
-// (one accumulator row) the screening logits of all experts sit in one TMEM
-// lane; the epilogue takes their k-th largest value, marks every expert whose
-// screening logit may still reach the exact top k (z >= k-th - 2 * bound), and
-// lists each such (token, candidate slot) under its expert for the exact
-// recompute, in a segment of 128 entries per (expert, 128-token tile) whose
-// positions the tile's four epilogue warps agree on through shared memory (no
-// global atomics).  Up to kSelMaxCand candidates per token are kept; a token
-// with more records only its count (the finishing kernel then recomputes all
-// experts for it).
-struct RouterSelArgs {
-  const float* xnorm2;   // [T] sum of x_t^2
-  const float* wnorm;    // [E] ||W_r[e]||_2
-  float gamma;           // screening bound factor: |err| <= gamma ||x_t|| max_e ||w_e||
-  int E, k;
-  uint8_t* cidx;         // [T][kSelMaxCand] candidate experts in expert order
-  int32_t* ncand;        // [T] candidate count
-  float* zmax;           // [T] largest screening logit m_s
-  float* snc;            // [T] sum over non-candidates of exp(z_e - m_s)
-  int32_t* ecnt;         // [E][ntiles] entries of each (expert, tile) segment
-  int32_t* elist;        // [E][ntiles][128] entries t * kSelMaxCand + slot
-  int ntiles;            // ceil(T / 128)
-};
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3 };
 
 struct GemmParams {
   const int32_t* group_start;  // [n_groups] or nullptr (one group of R rows)
@@ -80,14 +56,7 @@ struct GemmParams {
   unsigned long long wait_limit_ns;
   int a_kwrap;         // > 0: the A operand repeats every a_kwrap columns of the reduction (split router)
   float* out_f32;      // kModeF32: fp32 output [R, N]
-  const float* bias;   // kModeF32 / kModeRouterSel: optional per-column bias [N]
-  RouterSelArgs sel;   // kModeRouterSel
-  // kModeCombine (the shared expert's down GEMM; row r = token r): out[r] = bf16(sum_j w[r,j] y_perm[slot[r,j]]
-  // + acc[r]), the routed sum in fp32 in slot order, then the shared expert's fp32 accumulator, one rounding
-  const int32_t* cmb_slot;        // [R, k] grouped row of (token, slot), -1 = dropped
-  const float* cmb_w;             // [R, k] gates
-  const __nv_bfloat16* cmb_y;     // [rows, N] routed expert outputs, row pitch ldo
-  int cmb_k;
+  const float* bias;   // kModeF32: optional per-column bias [N]
 };
 
 #ifndef MOE_GEMM_MAX_STAGES
@@ -127,104 +96,6 @@ __device__ __forceinline__ float erf_as7126(float x) {
 }
 __device__ __forceinline__ float act_gelu(float g) { return 0.5f * g * (1.0f + erf_as7126(g * 0.7071067811865476f)); }
 
-// Router selection for one token (one TMEM lane = one accumulator row of BN
-// screening logits; columns >= E are padding).  Pass 1: the largest value and
-// the k-th largest (with multiplicity) by a KM-slot descending insertion
-// network.  Pass 2: the candidates (z >= k-th - 2 bound) and the sum of
-// exp(z - max) over the non-candidates; the accumulator is released after its
-// last read.  Pass 3: the candidates are written in expert order and entered in
-// their (expert, tile) segments.  All four epilogue warps call this for every
-// tile (two named barriers among them).
-template <int BN, int KM, typename Release>
-__device__ __forceinline__ void router_select(const RouterSelArgs a, const float* __restrict__ bias, int tile, int q,
-                                              uint32_t* s_mask, uint32_t t_row, bool valid, long long t, float wmax,
-                                              Release release) {
-  float top[KM];
-#pragma unroll
-  for (int i = 0; i < KM; ++i) top[i] = -INFINITY;
-#pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    uint32_t v[2][16];
-    tmem_ld16(t_row + c0, v[0]);
-    tmem_ld16(t_row + c0 + 16, v[1]);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int col = c0 + i;
-      const float z = col < a.E ? __uint_as_float(v[i >> 4][i & 15]) + (bias != nullptr ? bias[col] : 0.f)
-                                : -INFINITY;
-#pragma unroll
-      for (int j = KM - 1; j > 0; --j) top[j] = fmaxf(top[j], fminf(top[j - 1], z));
-      top[0] = fmaxf(top[0], z);
-    }
-  }
-  // top[] is sorted descending, so the k-th largest is the least of its first k entries (a running
-  // minimum rather than top[k - 1], which would index the array at run time)
-  float kth = top[0];
-#pragma unroll
-  for (int j = 1; j < KM; ++j) kth = j < a.k ? fminf(kth, top[j]) : kth;
-  const float m_s = top[0];
-  const float xn = valid ? sqrtf(a.xnorm2[t]) : 0.f;
-  const float bound = a.gamma * xn * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
-  const float thr = kth - 2.f * bound;
-  // pass 2: per column, the warp's candidates (ballot; a token keeps its first kSelMaxCand), published in
-  // shared memory for the tile's four epilogue warps; the exp sum over the non-candidates
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  float snc = 0.f;
-  int nc = 0;        // the token's candidates (all of them)
-#pragma unroll 1
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    uint32_t v[2][16];
-    tmem_ld16(t_row + c0, v[0]);
-    tmem_ld16(t_row + c0 + 16, v[1]);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int col = c0 + i;
-      bool keep = false;
-      if (col < a.E) {
-        const float z = __uint_as_float(v[i >> 4][i & 15]) + (bias != nullptr ? bias[col] : 0.f);
-        const bool isc = valid && z >= thr;
-        keep = isc && nc < kSelMaxCand;
-        nc += isc ? 1 : 0;
-        if (!isc) snc += __expf(z - m_s);
-      }
-      const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0) s_mask[q * BN + col] = m;
-    }
-  }
-  release();
-  named_bar_sync(1, 128);   // the four epilogue warps' masks of this tile are in place
-  // pass 3: each candidate's position in its (expert, tile) segment = candidates of the same expert in earlier
-  // warps of the tile + earlier lanes of this warp; its slot = its rank among the token's candidates
-  int slot = 0;
-#pragma unroll 1
-  for (int col = 0; col < a.E; ++col) {
-    const uint32_t m = s_mask[q * BN + col];
-    if ((m >> lane) & 1u) {
-      int before = __popc(m & lt);
-      for (int w = 0; w < q; ++w) before += __popc(s_mask[w * BN + col]);
-      a.cidx[t * kSelMaxCand + slot] = (uint8_t)col;
-      a.elist[((long long)col * a.ntiles + tile) * 128 + before] = (int32_t)(t * kSelMaxCand + slot);
-      ++slot;
-    }
-  }
-  if (q == 0) {
-    for (int col = lane; col < a.E; col += 32) {
-      int n = 0;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) n += __popc(s_mask[w * BN + col]);
-      a.ecnt[(long long)col * a.ntiles + tile] = n;
-    }
-  }
-  named_bar_sync(1, 128);   // the masks are read before the next tile overwrites them
-  if (!valid) return;
-  a.ncand[t] = nc;
-  a.zmax[t] = m_s;
-  a.snc[t] = snc;
-}
-
 template <int MODE, int BN, int CG = 1>
 __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -233,7 +104,7 @@ __global__ void __launch_bounds__(256, 1)
   using Cfg = GemmCfg<BN, CG>;
   constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
   constexpr bool kPair = CG == 2;
-  static_assert(!kPair || (MODE != kModeF32 && MODE != kModeRouterSel), "the router GEMM runs on single CTAs");
+  static_assert(!kPair || MODE != kModeF32, "the router GEMM runs on single CTAs");
   constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
   constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box (single CTA)
   constexpr int TM = kBM * CG;              // rows per tile
@@ -440,12 +311,6 @@ __global__ void __launch_bounds__(256, 1)
     __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)S * Cfg::kStageBytes) + q * 32 * kEpiRow;
     int acc = 0;
     uint32_t acc_phase = 0;
-    float wmax = 0.f;   // kModeRouterSel: max_e ||W_r[e]||
-    if (MODE == kModeRouterSel) {
-      for (int e = lane; e < p.sel.E; e += 32) wmax = fmaxf(wmax, p.sel.wnorm[e]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-    }
     // accumulator release: each thread (single CTA) or each warp on the leader's barrier (pair)
     auto release_acc = [&](int a) {
       tc_fence_before();
@@ -463,80 +328,7 @@ __global__ void __launch_bounds__(256, 1)
       if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0106)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if constexpr (MODE == kModeRouterSel) {
-        const bool valid = q * 32 + lane < rows_valid;
-        const long long t = row0 + q * 32 + lane;
-        // one column tile: the row tile index is the token tile; the masks use the epilogue staging area
-        const int ttile = (int)(row0 / kBM);
-        uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + (size_t)S * Cfg::kStageBytes);
-        if (p.sel.k <= 4)
-          router_select<BN, 4>(p.sel, p.bias, ttile, q, s_mask, t_row, valid, t, wmax, [&]() { release_acc(acc); });
-        else
-          router_select<BN, 16>(p.sel, p.bias, ttile, q, s_mask, t_row, valid, t, wmax, [&]() { release_acc(acc); });
-      } else if constexpr (MODE == kModeCombine) {
-        // thread = row = token: its routed rows, weighted in slot order in fp32, then the shared expert's fp32
-        // accumulator, one bf16 rounding; 32 columns per round with every routed-row load of the round in
-        // flight (4 slots x 64 bytes per thread), rows read and written as whole 32-byte sectors
-        const bool valid = q * 32 + lane < rows_valid;
-        const long long r = row0 + q * 32 + lane;
-#pragma unroll 1
-        for (int c0 = 0; c0 < OUTN; c0 += 32) {
-          uint32_t v[2][16];
-          tmem_ld16(t_row + c0, v[0]);
-          tmem_ld16(t_row + c0 + 16, v[1]);
-          tmem_ld_wait();
-          if (c0 + 32 >= OUTN) release_acc(acc);
-          float c[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) c[i] = 0.f;
-          const int col = n0 + c0;
-          for (int j0 = 0; j0 < p.cmb_k; j0 += 4) {
-            int pj[4];
-            float gj[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int j = j0 + u;
-              pj[u] = (valid && j < p.cmb_k) ? p.cmb_slot[r * p.cmb_k + j] : -1;
-              gj[u] = (valid && j < p.cmb_k) ? p.cmb_w[r * p.cmb_k + j] : 0.f;
-            }
-            uint4 y[4][4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int h = 0; h < 4; ++h)
-                y[u][h] = (pj[u] >= 0 && col + 8 * h < p.N)
-                              ? *reinterpret_cast<const uint4*>(p.cmb_y + (long long)pj[u] * p.ldo + col + 8 * h)
-                              : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              if (pj[u] < 0) continue;
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const uint32_t w4[4] = {y[u][h].x, y[u][h].y, y[u][h].z, y[u][h].w};
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                  c[8 * h + 2 * e2] = fmaf(gj[u], bf16lo(w4[e2]), c[8 * h + 2 * e2]);
-                  c[8 * h + 2 * e2 + 1] = fmaf(gj[u], bf16hi(w4[e2]), c[8 * h + 2 * e2 + 1]);
-                }
-              }
-            }
-          }
-          if (valid) {
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              if (col + 8 * h >= p.N) continue;
-              uint32_t o[4];
-#pragma unroll
-              for (int e2 = 0; e2 < 4; ++e2) {
-                const int i = 8 * h + 2 * e2;
-                o[e2] = pack_bf16x2(c[i] + __uint_as_float(v[i >> 4][i & 15]),
-                                    c[i + 1] + __uint_as_float(v[(i + 1) >> 4][(i + 1) & 15]));
-              }
-              *reinterpret_cast<uint4*>(p.out + r * p.ldo + col + 8 * h) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          }
-        }
-      } else if (MODE == kModeF32) {
+      if (MODE == kModeF32) {
         // fp32 rows through the staging buffer, 32 columns (128 bytes per row) per round
         float* fstg = reinterpret_cast<float*>(stg);  // 32 rows x 36 floats per warp
         constexpr int FR = 36;

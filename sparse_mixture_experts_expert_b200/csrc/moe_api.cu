@@ -138,7 +138,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 
 struct Workspace {
   size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
-  size_t xnorm2, cidx, ncand, zmax, snc, zex, ecnt, elist;   // certified selection inside the screening GEMM
+  size_t cidx, ncand, zmax, snc, zex, ecount, elist;   // certified selection over the screening logits
   size_t total;
 };
 
@@ -183,14 +183,13 @@ static Workspace ws_layout(const moe_shape* s) {
   L.hs = take((size_t)s->T * std::max(s->H_s, 16) * 2);
   L.ys = take((size_t)s->T * s->d * 2);
   L.shtab = take(64);
-  L.xnorm2 = take((size_t)s->T * 4);
   L.cidx = take((size_t)s->T * kSelMaxCand);
   L.ncand = take((size_t)s->T * 4);
   L.zmax = take((size_t)s->T * 4);
   L.snc = take((size_t)s->T * 4);
   L.zex = take((size_t)s->T * kSelMaxCand * 4);
-  L.ecnt = take((size_t)s->E * cdiv(s->T, 128) * 4);
-  L.elist = use_tc_router(s) ? take((size_t)s->E * cdiv(s->T, 128) * 128 * 4) : take(16);
+  L.ecount = take((size_t)s->E * 4);
+  L.elist = use_tc_router(s) ? take((size_t)s->E * s->T * 4) : take(16);
   L.total = o;
   return L;
 }
@@ -265,7 +264,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 // CTA pairs (M = 256 tiles) for the bf16 expert GEMMs when the groups are large enough
 // to fill them: on average at least 192 rows per group.
 static bool use_pair_gemm(int mode, int BN, long long R, int n_groups, bool allow_pair) {
-  return allow_pair && mode != kModeF32 && mode != kModeRouterSel && BN == 256 && R >= 192ll * n_groups;
+  return allow_pair && mode != kModeF32 && BN == 256 && R >= 192ll * n_groups;
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
@@ -292,11 +291,6 @@ static int pick_bn(bool glu, int N, long long mtiles) {
 struct GemmExtras {
   int a_kwrap = 0;                   // router: A repeats every a_kwrap reduction columns
   const float* bias = nullptr;       // router: per-expert logit bias
-  const RouterSelArgs* sel = nullptr;  // kModeRouterSel
-  const int32_t* cmb_slot = nullptr;   // kModeCombine: slot_pos [R, k]
-  const float* cmb_w = nullptr;        // kModeCombine: gates [R, k]
-  const void* cmb_y = nullptr;         // kModeCombine: routed outputs y_perm
-  int cmb_k = 0;
 };
 
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
@@ -307,7 +301,7 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   // router logits: one column tile as wide as the expert count (fewer A re-reads)
-  const bool router = mode == kModeF32 || mode == kModeRouterSel;
+  const bool router = mode == kModeF32;
   const int BN = router ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
   const bool pair = use_pair_gemm(mode, BN, R, n_groups, allow_pair);
   const int box_rows = (glu || pair) ? BN / 2 : BN;
@@ -332,18 +326,12 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.a_kwrap = a_kwrap;
   p.out_f32 = reinterpret_cast<float*>(out);
   p.bias = ex.bias;
-  p.sel = ex.sel != nullptr ? *ex.sel : RouterSelArgs{};
-  p.cmb_slot = ex.cmb_slot;
-  p.cmb_w = ex.cmb_w;
-  p.cmb_y = reinterpret_cast<const __nv_bfloat16*>(ex.cmb_y);
-  p.cmb_k = ex.cmb_k;
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
   if (pair) {
     const long long ub2 = grows ? (R / (2 * kBM) + n_groups) : cdiv(R, 2 * kBM);
     if (mode == kModePlain) return launch_gemm_t<kModePlain, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeSwiGLU) return launch_gemm_t<kModeSwiGLU, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeGeGLU) return launch_gemm_t<kModeGeGLU, 256, 2>(ta, tb, p, ub2, st);
-    if (mode == kModeCombine) return launch_gemm_t<kModeCombine, 256, 2>(ta, tb, p, ub2, st);
     return MOE_UNSUPPORTED_SHAPE;
   }
 #define MOE_GEMM_CASE(M_, BN_) \
@@ -353,9 +341,6 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
   MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 192) MOE_GEMM_CASE(kModeF32, 128)
   MOE_GEMM_CASE(kModeF32, 64)
-  MOE_GEMM_CASE(kModeRouterSel, 256) MOE_GEMM_CASE(kModeRouterSel, 192) MOE_GEMM_CASE(kModeRouterSel, 128)
-  MOE_GEMM_CASE(kModeRouterSel, 64)
-  MOE_GEMM_CASE(kModeCombine, 256) MOE_GEMM_CASE(kModeCombine, 128) MOE_GEMM_CASE(kModeCombine, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -743,8 +728,6 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   } else if (logits_in == nullptr && use_tc_router(s)) {
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
-    MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d);
-    MOE_LAUNCH_CHECK();
     // screening bound, relative to ||x_t|| max_e ||w_e|| (>= sum |x_i w_i|): the split's representation error
     // 2^-16, fp32 accumulation of 2d products in any rounding direction plus the bias add, and the error of the
     // exact recompute's own d-term fp32 chain; all with a 2^-7 margin
@@ -752,45 +735,45 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
                                  (s->d + 2.0) * std::ldexp(1.0, -24)) *
                                 (1.0 + std::ldexp(1.0, -7)));
     const bool want_stats = aux_f || aux_p || aux;
-    if (logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD) {
-      // selection inside the screening GEMM's epilogue, exact recompute by expert, finish per token
-      float* xnorm2 = reinterpret_cast<float*>(ws + L.xnorm2);
-      const int ntiles = (int)cdiv(s->T, 128);
-      RouterSelArgs sel{xnorm2, wnorm, gamma, s->E, s->k, reinterpret_cast<uint8_t*>(ws + L.cidx),
-                        reinterpret_cast<int32_t*>(ws + L.ncand), reinterpret_cast<float*>(ws + L.zmax),
-                        reinterpret_cast<float*>(ws + L.snc), reinterpret_cast<int32_t*>(ws + L.ecnt),
-                        reinterpret_cast<int32_t*>(ws + L.elist), ntiles};
-      MOE_LAUNCH((k_router_xnorm), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
-                 xnorm2, (long long)s->T, s->d);
-      MOE_LAUNCH_CHECK();
-      GemmExtras ex;
-      ex.a_kwrap = s->d;
-      ex.bias = bias;
-      ex.sel = &sel;
-      rc = grouped_gemm(kModeRouterSel, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, nullptr, st,
-                        false, ex);
-      if (rc) return rc;
-      float* zex = reinterpret_cast<float*>(ws + L.zex);
-      MOE_LAUNCH((k_router_recompute), dim3((unsigned)s->E, (unsigned)cdiv(ntiles, kRecompTiles)), 256, 0, st,
-                 reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, sel.ecnt, sel.elist, zex, ntiles, s->d);
-      MOE_LAUNCH_CHECK();
+    // without logits or statistics to return, the selection lists candidates and recomputes them by expert
+    const bool select = logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD;
+    int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
+    MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d,
+               select ? ecount : nullptr);
+    MOE_LAUNCH_CHECK();
+    GemmExtras ex;
+    ex.a_kwrap = s->d;
+    ex.bias = bias;
+    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false, ex);
+    if (rc) return rc;
+    if (select) {
+      SelectArgs sa{part, reinterpret_cast<const __nv_bfloat16*>(x), wnorm, gamma, (int)s->T, s->d, s->E, s->k,
+                    reinterpret_cast<uint8_t*>(ws + L.cidx), reinterpret_cast<int32_t*>(ws + L.ncand),
+                    reinterpret_cast<float*>(ws + L.zmax), reinterpret_cast<float*>(ws + L.snc), ecount,
+                    reinterpret_cast<int32_t*>(ws + L.elist), cnt};
       const unsigned nch = (unsigned)cdiv(s->T, kChunk);
-      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-      if (s->E <= 128)
-        MOE_LAUNCH((k_router_finish<4>), nch, 1024, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
-                   bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
-      else
-        MOE_LAUNCH((k_router_finish<8>), nch, 1024, 0, st, sel.ncand, sel.cidx, zex, sel.zmax, sel.snc, xb, w_router,
-                   bias, idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm);
+      const int epl = s->E <= 64 ? 2 : s->E <= 128 ? 4 : s->E <= 192 ? 6 : 8;
+      if (epl == 2) MOE_LAUNCH((k_router_select<2>), nch, 256, 0, st, sa);
+      else if (epl == 4) MOE_LAUNCH((k_router_select<4>), nch, 256, 0, st, sa);
+      else if (epl == 6) MOE_LAUNCH((k_router_select<6>), nch, 256, 0, st, sa);
+      else MOE_LAUNCH((k_router_select<8>), nch, 256, 0, st, sa);
+      MOE_LAUNCH_CHECK();
+      float* zex = reinterpret_cast<float*>(ws + L.zex);
+      MOE_LAUNCH((k_router_recompute), (unsigned)(4 * num_sms()), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
+                 w_router, bias, ecount, sa.elist, zex, (int)s->T, s->d, s->E);
+      MOE_LAUNCH_CHECK();
+      const unsigned nfin = (unsigned)cdiv(s->T, 8);
+#define MOE_FINISH(N_)                                                                                        \
+  MOE_LAUNCH((k_router_finish<N_>), nfin, 256, 0, st, sa.ncand, sa.cidx, zex, sa.zmax, sa.snc, sa.x, w_router, bias, \
+             idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm)
+      if (epl == 2) MOE_FINISH(2);
+      else if (epl == 4) MOE_FINISH(4);
+      else if (epl == 6) MOE_FINISH(6);
+      else MOE_FINISH(8);
+#undef MOE_FINISH
       MOE_LAUNCH_CHECK();
       rc = MOE_OK;
     } else {
-      GemmExtras ex;
-      ex.a_kwrap = s->d;
-      ex.bias = bias;
-      rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false,
-                        ex);
-      if (rc) return rc;
       RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d, gamma};
       rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
     }
@@ -1012,26 +995,9 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
                               ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq,
                                             reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
                               : Int4Scratch{nullptr, nullptr};
-  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, fused_ffn_ok(s, s->H) ? nullptr : hbuf,
-                       yperm, stream, scr);
+  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
   if (rc) return rc;
   void* ys = nullptr;
-  if (s->H_s > 0 && s->wfmt == MOE_WFMT_BF16) {
-    // shared expert: gate/up, then the down GEMM whose epilogue adds each token's weighted routed rows (the
-    // combine) to the shared expert's fp32 accumulator and rounds once
-    const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
-    const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
-    rc = grouped_gemm(mode, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, s->H_s, s->H_s, nullptr, nullptr, ws + L.hs,
-                      stream, pair);
-    if (rc) return rc;
-    GemmExtras ex;
-    ex.cmb_slot = slot;
-    ex.cmb_w = w;
-    ex.cmb_y = yperm;
-    ex.cmb_k = s->k;
-    return grouped_gemm(kModeCombine, ws + L.hs, s->T, s->H_s, w2_sh, 1, s->d, 0, s->d, nullptr, nullptr, out,
-                        stream, pair, ex);
-  }
   if (s->H_s > 0) {
     ys = ws + L.ys;
     rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,

@@ -118,8 +118,11 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 //    and the screening logits are [x | x] [hi | lo]^T;
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
 __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
-                                                     float* __restrict__ wnorm, int E, int d) {
+                                                     float* __restrict__ wnorm, int E, int d,
+                                                     int32_t* __restrict__ zero_counts) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  if (zero_counts != nullptr && blockIdx.x == 0)   // per-expert list lengths of the certified selection
+    for (int i = threadIdx.x; i < E; i += blockDim.x) zero_counts[i] = 0;
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
   const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
@@ -153,133 +156,6 @@ __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if (lane_id() == 0) wnorm[e] = sqrtf(ss);
-}
-
-// Token statistics for the certified selection inside the screening GEMM, one
-// warp per token: xnorm2[t] = sum_i x[t,i]^2 (bounds the screening error of
-// token t).
-__global__ void __launch_bounds__(256) k_router_xnorm(const __nv_bfloat16* __restrict__ x, float* __restrict__ xnorm2,
-                                                      long long T, int d) {
-  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  const long long t = (long long)blockIdx.x * 8 + warp_id();
-  if (t >= T) return;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
-  const int nv = d >> 3;
-  float ss = 0.f;
-  for (int v0 = lane_id(); v0 < nv; v0 += 128) {
-    uint4 u[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = v0 + 32 * j < nv ? xr[v0 + 32 * j] : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float q[8] = {bf16lo(u[j].x), bf16hi(u[j].x), bf16lo(u[j].y), bf16hi(u[j].y),
-                          bf16lo(u[j].z), bf16hi(u[j].z), bf16lo(u[j].w), bf16hi(u[j].w)};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(q[i], q[i], ss);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane_id() == 0) xnorm2[t] = ss;
-}
-
-// Exact recompute of the selection candidates, expert-major: CTA (e, s) takes
-// the (expert e, tile) segments of tiles [s * kRecompTiles, (s+1) *
-// kRecompTiles), keeps W_r[e] (fp32) in shared memory and computes each
-// entry's logit with the whole warp -- lane l takes the 8-input slices l,
-// l+32, ..., one fmaf chain, a fixed xor tree, then the bias: the same value
-// for a (token, expert) pair whichever CTA or warp computes it, and the same as
-// warp_dot.  A warp keeps kRecompBatch entries in flight (their input loads
-// issued together).  zex[t][slot] = exact logit.
-constexpr int kRecompTiles = 64;    // 128-token tiles per CTA
-constexpr int kRecompBatch = 8;     // entries per warp in flight
-constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
-__global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
-                                                          const float* __restrict__ W, const float* __restrict__ bias,
-                                                          const int32_t* __restrict__ ecnt,
-                                                          const int32_t* __restrict__ elist, float* __restrict__ zex,
-                                                          int ntiles, int d) {
-  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  __shared__ __align__(16) float s_w[kSelMaxD];
-  __shared__ int s_pre[kRecompTiles + 1];
-  const int e = blockIdx.x;
-  const int tb = blockIdx.y * kRecompTiles;
-  const int nt = min(kRecompTiles, ntiles - tb);
-  if (nt <= 0) return;
-  const int lane = lane_id();
-  if (warp_id() == 0) {
-    // exclusive prefix of the segment sizes (two tiles per lane)
-    const int i0 = 2 * lane, i1 = 2 * lane + 1;
-    const int c0 = i0 < nt ? ecnt[(size_t)e * ntiles + tb + i0] : 0;
-    const int c1 = i1 < nt ? ecnt[(size_t)e * ntiles + tb + i1] : 0;
-    int incl = c0 + c1;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int excl = incl - c0 - c1;
-    if (i0 <= nt) s_pre[i0] = excl;
-    if (i1 <= nt) s_pre[i1] = excl + c0;
-    if (lane == 31 && 64 <= nt) s_pre[64] = incl;
-  }
-  __syncthreads();
-  const int total = s_pre[nt];
-  if (total == 0) return;
-  const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
-  for (int i = threadIdx.x; i < d / 4; i += blockDim.x) reinterpret_cast<float4*>(s_w)[i] = wr[i];
-  __syncthreads();
-  const float be = bias != nullptr ? bias[e] : 0.f;
-  const int32_t* seg = elist + ((size_t)e * ntiles + tb) * 128;
-  const int nv = d >> 3;
-  const int nwarps = blockDim.x / 32;
-  for (int f0 = kRecompBatch * warp_id(); f0 < total; f0 += kRecompBatch * nwarps) {
-    int ent[kRecompBatch];
-    const uint4* xr[kRecompBatch];
-#pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) {
-      const int f = min(f0 + j, total - 1);
-      int lo = 0, hi = nt - 1;   // last tile with s_pre[tile] <= f
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] <= f) lo = mid; else hi = mid - 1;
-      }
-      ent[j] = seg[lo * 128 + (f - s_pre[lo])];
-      xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
-    }
-    float acc[kRecompBatch];
-#pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-      uint4 u[kRecompBatch];
-#pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
-      const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
-      const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
-#pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) {
-        float a = acc[j];
-        a = fmaf(bf16lo(u[j].x), w0.x, a); a = fmaf(bf16hi(u[j].x), w0.y, a);
-        a = fmaf(bf16lo(u[j].y), w0.z, a); a = fmaf(bf16hi(u[j].y), w0.w, a);
-        a = fmaf(bf16lo(u[j].z), w1.x, a); a = fmaf(bf16hi(u[j].z), w1.y, a);
-        a = fmaf(bf16lo(u[j].w), w1.z, a); a = fmaf(bf16hi(u[j].w), w1.w, a);
-        acc[j] = a;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-    }
-    if (lane < kRecompBatch) {
-      float mine = acc[0];
-      int my_ent = ent[0];
-#pragma unroll
-      for (int j = 1; j < kRecompBatch; ++j)
-        if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
-      if (f0 + lane < total) zex[my_ent] = mine + be;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -654,14 +530,261 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
   }
 }
 
-// Selection finish, one warp per token, a CTA of 32 warps per 32-token chunk.
-// Lane c holds candidate c (exact logit, expert); the top k among them by
-// (value desc, index asc) -- certified to be the top k of all experts --
-// come from k rounds of warp argmax.  Softmax: m = the first pick's value,
-// sum = snc * exp(m_s - m) + sum over candidates of exp(z - m), where snc is
-// the epilogue's sum of exp(z_e - m_s) over the non-candidates (screening
-// values).  A token with more than kSelMaxCand candidates (degenerate logits)
-// is finished here from exact logits of every expert.  cnt[e][chunk] = picks.
+// ---------------------------------------------------------------------------
+// Certified selection over tensor-core screening logits, in three kernels that
+// keep the exact fp32 work proportional to the candidates (about k + 0.1 per
+// token) rather than to E:
+//   k_router_select    one warp per token (lane l: experts l, l+32, ...): the
+//                      k-th largest screening logit, ||x_t|| for the error
+//                      bound, the candidates (z >= k-th - 2 bound) in expert
+//                      order, and the sum of exp(z - max) over the others;
+//                      each candidate is listed under its expert;
+//   k_router_recompute exact fp32 logits of the listed (token, expert) pairs,
+//                      the flat list split evenly over the CTAs, W_r[e] in
+//                      shared memory;
+//   k_router_finish    top k among each token's exact candidates, softmax
+//                      (exact candidates + screening rest), gates, picks per
+//                      (expert, chunk).
+// The decision equals the top k of exact fp32 logits: every expert outside
+// the candidates is below the k-th exact logit by the screening bound.
+constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
+constexpr int kRecompBatch = 8;     // list entries per warp in flight
+
+struct SelectArgs {
+  const float* zs;       // [T, E] screening logits (bias included)
+  const __nv_bfloat16* x;
+  const float* wnorm;    // [E] ||W_r[e]||_2
+  float gamma;           // |screen - exact| <= gamma ||x_t|| max_e ||w_e||
+  int T, d, E, k;
+  uint8_t* cidx;         // [T][kSelMaxCand] candidate experts, expert order
+  int32_t* ncand;        // [T] candidates (all of them)
+  float* zmax;           // [T] largest screening logit
+  float* snc;            // [T] sum over non-candidates of exp(z - zmax)
+  int32_t* ecount;       // [E] list lengths (zero before k_router_select)
+  int32_t* elist;        // [E][T] list entries t * kSelMaxCand + slot
+  int32_t* cnt;          // [E][nchunks] pick counts, cleared here for k_router_finish
+};
+
+// One CTA = one 32-token chunk = 8 warps x 4 tokens.  A candidate takes its
+// position in its expert's list in two steps: a shared-memory counter per
+// expert inside the chunk, then one global reservation per (chunk, expert) for
+// the chunk's whole run.  The tokens of a warp are loaded together (screening
+// row and inputs), then processed in order.  A token keeps its first
+// kSelMaxCand candidates; with more, the finishing kernel recomputes every
+// expert for it.
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  constexpr int TPW = kChunk / 8;
+  __shared__ int s_cnt[kMaxRouterE];
+  __shared__ int s_base[kMaxRouterE];
+  __shared__ uint32_t s_rec[kChunk][kSelMaxCand];   // expert << 16 | index inside the chunk's run
+  __shared__ int s_nk[kChunk];
+  const int lane = lane_id(), warp = warp_id();
+  const int chunk = blockIdx.x, nchunks = (a.T + kChunk - 1) / kChunk;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    s_cnt[e] = 0;
+    a.cnt[(size_t)e * nchunks + chunk] = 0;
+  }
+  float wmax = 0.f;
+  for (int e = lane; e < a.E; e += 32) wmax = fmaxf(wmax, a.wnorm[e]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  const int nv = a.d >> 3;
+  // screening rows and input sums of squares of the warp's tokens, loads issued together
+  float z[TPW][EPL];
+  float ss[TPW];
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt) {
+    const int t = chunk * kChunk + warp * TPW + tt;
+    const bool on = t < a.T;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      z[tt][i] = (on && e < a.E) ? a.zs[(size_t)t * a.E + e] : -INFINITY;
+    }
+    float acc = 0.f;
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(on ? t : 0) * a.d);
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 u = on ? xr[v] : make_uint4(0, 0, 0, 0);
+      const float q[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                          bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = fmaf(q[j], q[j], acc);
+    }
+    ss[tt] = acc;
+  }
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt) {
+    const int tl = warp * TPW + tt;
+    const int t = chunk * kChunk + tl;
+    if (t >= a.T) {
+      if (lane == 0) s_nk[tl] = 0;
+      continue;
+    }
+    float x2 = ss[tt];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, o);
+    const float kth = warp_kth<EPL>(z[tt], a.E, a.k);
+    float m_s;
+    {
+      float lm = z[tt][0];
+#pragma unroll
+      for (int i = 1; i < EPL; ++i) lm = fmaxf(lm, z[tt][i]);
+      asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m_s) : "f"(lm));
+    }
+    const float bound = a.gamma * sqrtf(x2) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
+    const float thr = kth - 2.f * bound;
+    int nbefore = 0;      // candidates in earlier expert groups (warp-uniform)
+    float snc = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      const bool cand = e < a.E && z[tt][i] >= thr;
+      const unsigned m = __ballot_sync(0xffffffffu, cand);
+      if (cand) {
+        const int slot = nbefore + __popc(m & lt);
+        if (slot < kSelMaxCand) {
+          a.cidx[(size_t)t * kSelMaxCand + slot] = (uint8_t)e;
+          const int li = atomicAdd(&s_cnt[e], 1);
+          s_rec[tl][slot] = ((uint32_t)e << 16) | (uint32_t)li;
+        }
+      } else if (e < a.E) {
+        snc += __expf(z[tt][i] - m_s);
+      }
+      nbefore += __popc(m);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) snc += __shfl_xor_sync(0xffffffffu, snc, o);
+    if (lane == 0) {
+      a.ncand[t] = nbefore;
+      a.zmax[t] = m_s;
+      a.snc[t] = snc;
+      s_nk[tl] = min(nbefore, kSelMaxCand);
+    }
+  }
+  __syncthreads();
+  // one reservation per expert for the chunk's run (all issued together), then the list entries
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+    if (s_cnt[e] > 0) s_base[e] = atomicAdd(&a.ecount[e], s_cnt[e]);
+  __syncthreads();
+  for (int i = threadIdx.x; i < kChunk * kSelMaxCand; i += blockDim.x) {
+    const int tl = i / kSelMaxCand, slot = i % kSelMaxCand;
+    if (slot < s_nk[tl]) {
+      const uint32_t r = s_rec[tl][slot];
+      const int e = (int)(r >> 16);
+      a.elist[(size_t)e * a.T + s_base[e] + (int)(r & 0xFFFFu)] =
+          (int32_t)((chunk * kChunk + tl) * kSelMaxCand + slot);
+    }
+  }
+}
+
+// Exact fp32 logits of the listed (token, expert) pairs.  The lists of all
+// experts form one flat sequence (expert order); CTA b takes the b-th equal
+// slice of it -- balanced whatever the popularity of the experts -- and walks
+// the experts its slice covers, W_r[e] in shared memory.  Each entry's logit
+// is computed by a whole warp: lane l takes the 8-input slices l, l+32, ...,
+// one fmaf chain, a fixed xor tree, then the bias -- the same value whichever
+// CTA or warp computes it, and the same as warp_dot.  A warp keeps
+// kRecompBatch entries in flight.  zex[t][slot] = exact logit.
+__global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
+                                                          const float* __restrict__ W, const float* __restrict__ bias,
+                                                          const int32_t* __restrict__ ecount,
+                                                          const int32_t* __restrict__ elist, float* __restrict__ zex,
+                                                          int T, int d, int E) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  __shared__ __align__(16) float s_w[kSelMaxD];
+  __shared__ int s_pre[kMaxRouterE + 1];
+  const int lane = lane_id();
+  if (warp_id() == 0) {
+    // exclusive prefix of the list lengths (E <= 512: up to 16 per lane, in expert order)
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) local += ecount[e];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      s_pre[e] = run;
+      run += ecount[e];
+    }
+    if (lane == 31) s_pre[E] = incl;
+  }
+  __syncthreads();
+  const long long N = s_pre[E];
+  const int f_lo = (int)(N * blockIdx.x / gridDim.x), f_hi = (int)(N * (blockIdx.x + 1) / gridDim.x);
+  if (f_lo >= f_hi) return;
+  int e = 0;   // the expert holding flat entry f_lo: last e with s_pre[e] <= f_lo
+  {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= f_lo) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+  }
+  const int nv = d >> 3;
+  const int nwarps = blockDim.x / 32;
+  for (; e < E && s_pre[e] < f_hi; ++e) {
+    const int a0 = max(f_lo, s_pre[e]), a1 = min(f_hi, s_pre[e + 1]);
+    if (a0 >= a1) continue;   // uniform across the CTA
+    __syncthreads();          // the previous expert's row is no longer read
+    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+    for (int i = threadIdx.x; i < d / 4; i += blockDim.x) reinterpret_cast<float4*>(s_w)[i] = wr[i];
+    __syncthreads();
+    const float be = bias != nullptr ? bias[e] : 0.f;
+    const int32_t* lst = elist + (size_t)e * T - s_pre[e];   // indexed by flat entry
+    for (int f0 = a0 + kRecompBatch * warp_id(); f0 < a1; f0 += kRecompBatch * nwarps) {
+      int ent[kRecompBatch];
+      const uint4* xr[kRecompBatch];
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) {
+        ent[j] = lst[min(f0 + j, a1 - 1)];
+        xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
+      }
+      float acc[kRecompBatch];
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
+      for (int v = lane; v < nv; v += 32) {
+        uint4 u[kRecompBatch];
+#pragma unroll
+        for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
+        const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
+        const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
+#pragma unroll
+        for (int j = 0; j < kRecompBatch; ++j) {
+          float s2 = acc[j];
+          s2 = fmaf(bf16lo(u[j].x), w0.x, s2); s2 = fmaf(bf16hi(u[j].x), w0.y, s2);
+          s2 = fmaf(bf16lo(u[j].y), w0.z, s2); s2 = fmaf(bf16hi(u[j].y), w0.w, s2);
+          s2 = fmaf(bf16lo(u[j].z), w1.x, s2); s2 = fmaf(bf16hi(u[j].z), w1.y, s2);
+          s2 = fmaf(bf16lo(u[j].w), w1.z, s2); s2 = fmaf(bf16hi(u[j].w), w1.w, s2);
+          acc[j] = s2;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+      }
+      if (lane < kRecompBatch) {
+        float mine = acc[0];
+        int my_ent = ent[0];
+#pragma unroll
+        for (int j = 1; j < kRecompBatch; ++j)
+          if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
+        if (f0 + lane < a1) zex[my_ent] = mine + be;
+      }
+    }
+  }
+}
+
 // Top k of one token from exact fp32 logits of every expert (lane l: experts
 // l, l+32, ...), for tokens with too many selection candidates.  Returns the
 // softmax denominator; m receives the largest logit.  Kept out of line: the
@@ -692,8 +815,16 @@ __device__ __noinline__ float select_all_exact(const __nv_bfloat16* __restrict__
   return ez;
 }
 
+// Selection finish, one warp per token (8 per CTA).  Lane c holds candidate c
+// (exact logit, expert); the top k among them by (value desc, index asc) --
+// certified to be the top k of all experts -- come from k rounds of warp
+// argmax.  Softmax: m = the first pick's value, sum = snc * exp(m_s - m) + the
+// candidates' exp(z - m), where snc is the selection's sum of exp(z_e - m_s)
+// over the non-candidates (screening values).  A token with more than
+// kSelMaxCand candidates (degenerate logits) is finished from exact logits of
+// every expert.  cnt[e][chunk] += picks (integer atomics: order-free).
 template <int EPL>
-__global__ void __launch_bounds__(1024) k_router_finish(const int32_t* __restrict__ ncand,
+__global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict__ ncand,
                                                        const uint8_t* __restrict__ cidx, const float* __restrict__ zex,
                                                        const float* __restrict__ zmax, const float* __restrict__ snc,
                                                        const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
@@ -701,51 +832,46 @@ __global__ void __launch_bounds__(1024) k_router_finish(const int32_t* __restric
                                                        float* __restrict__ topk_w, int32_t* __restrict__ cnt, int T,
                                                        int d, int E, int k, int renorm) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  __shared__ int s_c[kMaxRouterE];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_c[e] = 0;
-  __syncthreads();
-  const int lane = lane_id(), warp = warp_id();
-  const int chunk = blockIdx.x;
+  const int lane = lane_id();
+  const int t = blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
   const int nchunks = (T + kChunk - 1) / kChunk;
-  {
-    const int t = chunk * kChunk + warp;   // one token per warp, kChunk warps per CTA
-    if (t >= T) goto stats;
-    const int nc = ncand[t];
-    float sel_v = 0.f, m, ssum;
-    int sel_i = 0;
-    if (nc <= kSelMaxCand) {
-      float cv = lane < nc ? zex[(size_t)t * kSelMaxCand + lane] : -INFINITY;
-      int ci = lane < nc ? (int)cidx[(size_t)t * kSelMaxCand + lane] : 0x7fffffff;
-      const float cv0 = cv;
-      for (int j = 0; j < k; ++j) {
-        float bv = cv;
-        int bi = ci;
-        warp_argmax_redux(bv, bi);
-        if (lane == j) { sel_v = bv; sel_i = bi; }
-        if (ci == bi) cv = -INFINITY;    // taken (candidate ids are distinct)
-      }
-      m = __shfl_sync(0xffffffffu, sel_v, 0);
-      float ez = lane < nc ? __expf(cv0 - m) : 0.f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
-      ssum = ez + snc[t] * __expf(zmax[t] - m);
-    } else {
-      ssum = select_all_exact<EPL>(x + (size_t)t * d, W, bias, d, E, k, sel_v, sel_i, m);
+  // every load of the token issued together (the candidate slots past its count are masked afterwards)
+  const int nc = ncand[t];
+  const float zx = zex[(size_t)t * kSelMaxCand + lane];
+  const int cx = (int)cidx[(size_t)t * kSelMaxCand + lane];
+  const float ms = zmax[t], sn = snc[t];
+  float sel_v = 0.f, m, ssum;
+  int sel_i = 0;
+  if (nc <= kSelMaxCand) {
+    float cv = lane < nc ? zx : -INFINITY;
+    const int ci = lane < nc ? cx : 0x7fffffff;
+    const float cv0 = cv;
+    for (int j = 0; j < k; ++j) {
+      float bv = cv;
+      int bi = ci;
+      warp_argmax_redux(bv, bi);
+      if (lane == j) { sel_v = bv; sel_i = bi; }
+      if (ci == bi) cv = -INFINITY;    // taken (candidate ids are distinct)
     }
-    const float inv = 1.f / ssum;
-    const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
-    float wsum = pj;
+    m = __shfl_sync(0xffffffffu, sel_v, 0);
+    float ez = lane < nc ? __expf(cv0 - m) : 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    if (lane < k) {
-      topk_idx[(size_t)t * k + lane] = sel_i;
-      topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
-      atomicAdd(&s_c[sel_i], 1);
-    }
+    for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
+    ssum = ez + sn * __expf(ms - m);
+  } else {
+    ssum = select_all_exact<EPL>(x + (size_t)t * d, W, bias, d, E, k, sel_v, sel_i, m);
   }
-stats:
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(size_t)e * nchunks + chunk] = s_c[e];
+  const float inv = 1.f / ssum;
+  const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
+  float wsum = pj;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = sel_i;
+    topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
+    atomicAdd(&cnt[(size_t)sel_i * nchunks + t / kChunk], 1);
+  }
 }
 
 // W_r [E][d] fp32 (global) -> shared memory as [d][pitch] (column e of row c =
