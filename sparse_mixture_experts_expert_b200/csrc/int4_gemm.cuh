@@ -428,6 +428,191 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   __syncwarp();
 }
 
+// ---------------------------------------------------------------------------
+// Dense small batches (one group of R <= 256 rows: the shared expert of a
+// decode batch).  k_int4_stream gives each task 8 rows, so a 64-row batch
+// would read and dequantise every weight eight times; here a task is one block
+// of 32 weight rows over 32 rows (four 8-row chunks), its reduction split into
+// p.ksplit slab ranges: a 64-row batch reads and dequantises every weight
+// twice, and each dequantised fragment feeds the MMAs of four chunks.  Offset codes
+// (q + 136, the correction 136 * sum(x) per 128-group) as in k_int4_stream's
+// OFFS mode; fp32 partials [ksplit][R][W] in its split layout, which
+// k_int4_splitk_reduce adds in order.  Eight warps per CTA, each with a ring of
+// kI4DStages slabs.
+constexpr int kI4DWarps = 8;
+constexpr int kI4DStages = 4;
+constexpr int kI4DSmem = kI4DWarps * kI4DStages * kI4SlabBytes;
+constexpr int kI4DChunks = 4;            // 8-row chunks per task
+
+template <bool GLU>
+__global__ void __launch_bounds__(kI4DWarps * 32, 1)
+    k_int4_dense(const __grid_constant__ CUtensorMap tmW, const Int4Params p, unsigned long long wait_limit_ns,
+                 const float* __restrict__ xsum) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  extern __shared__ __align__(128) uint8_t i4_smem[];
+  __shared__ __align__(8) uint64_t s_bar[kI4DWarps][kI4DStages];
+  __shared__ volatile int s_abort[kI4DWarps];
+  const int lane = lane_id(), warp = warp_id();
+  if (lane == 0) {
+    for (int st = 0; st < kI4DStages; ++st) mbar_init(&s_bar[warp][st], 1);
+    s_abort[warp] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
+  __syncthreads();
+  const int KS = p.ksplit;
+  const int oblocks = GLU ? p.N / 16 : p.N / 32;
+  const int R = (int)p.R;
+  const int nrh = (R + 8 * kI4DChunks - 1) / (8 * kI4DChunks);   // row blocks of 8 * kI4DChunks rows
+  const int total = oblocks * nrh * KS;                          // task = (weight block, row block, split)
+  const int nslab = (p.K + 255) / 256;
+  const int ngk = p.K / 128;
+  const int gq = lane >> 2, c = lane & 3;
+  const int tstride = gridDim.x * kI4DWarps;
+  uint8_t* ring = i4_smem + (size_t)warp * kI4DStages * kI4SlabBytes;
+  auto rows_of = [&](int ob, int& ra, int& rb) {
+    ra = GLU ? ob * 16 : ob * 32;
+    rb = GLU ? p.up_row0 + ob * 16 : ra + 16;
+  };
+  // producer (lane 0 issues; values warp-uniform): items are (task, slab) in order, at most kI4DStages ahead
+  int issued = 0, consumed = 0;
+  int p_task = blockIdx.x * kI4DWarps + warp, p_slab = 0, p_se = 0, p_st = 0, p_ra = 0, p_rb = 0;
+  bool p_new = true;
+  auto refill = [&]() {
+    while (issued - consumed < kI4DStages) {
+      if (p_new) {
+        if (p_task >= total) return;
+        const int ob = p_task / (KS * nrh), sp = p_task % KS;
+        rows_of(ob, p_ra, p_rb);
+        p_slab = sp * nslab / KS;
+        p_se = (sp + 1) * nslab / KS;
+        p_new = false;
+        if (p_slab == p_se) { p_new = true; p_task += tstride; continue; }
+      }
+      if (lane == 0) {
+        uint8_t* dst = ring + p_st * kI4SlabBytes;
+        mbar_arrive_expect_tx(&s_bar[warp][p_st], kI4SlabBytes);
+        tma_load_2d(dst, &tmW, &s_bar[warp][p_st], p_slab * 128, p_ra);
+        tma_load_2d(dst + 16 * 128, &tmW, &s_bar[warp][p_st], p_slab * 128, p_rb);
+      }
+      ++issued;
+      if (++p_st == kI4DStages) p_st = 0;
+      if (++p_slab == p_se) { p_new = true; p_task += tstride; }
+    }
+  };
+
+  float tA[kI4DChunks][4], tB[kI4DChunks][4];
+  int c_st = 0;
+  uint32_t c_phase = 0;
+  for (int task = blockIdx.x * kI4DWarps + warp; task < total && !s_abort[warp]; task += tstride) {
+    const int ob = task / (KS * nrh), rh = (task / KS) % nrh, sp = task % KS;
+    const int r0 = rh * 8 * kI4DChunks;
+    int ra, rb;
+    rows_of(ob, ra, rb);
+    const int sb = sp * nslab / KS, se = (sp + 1) * nslab / KS;
+    if (sb == se) continue;
+#pragma unroll
+    for (int ch = 0; ch < kI4DChunks; ++ch)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { tA[ch][i] = 0.f; tB[ch][i] = 0.f; }
+    const __nv_bfloat16* sA = p.ws + (long long)(ra + gq) * ngk;
+    const __nv_bfloat16* sB = p.ws + (long long)(rb + gq) * ngk;
+    const long long s8 = 8ll * ngk;
+    bool ok = true;
+    for (int slab = sb; slab < se; ++slab) {
+      refill();
+      if (!mbar_wait(&s_bar[warp][c_st], c_phase, wait_limit_ns, &s_abort[warp], 0x0203)) { ok = false; break; }
+      const uint8_t* slabp = ring + c_st * kI4SlabBytes;
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+        const int kg = slab * 2 + gi;
+        if (kg >= ngk) break;   // the slab's second half is TMA zero fill
+        const uint4 a0 = *reinterpret_cast<const uint4*>(slabp + gq * 128 + gi * 64 + c * 16);
+        const uint4 a1 = *reinterpret_cast<const uint4*>(slabp + (gq + 8) * 128 + gi * 64 + c * 16);
+        const uint4 b0 = *reinterpret_cast<const uint4*>(slabp + (gq + 16) * 128 + gi * 64 + c * 16);
+        const uint4 b1 = *reinterpret_cast<const uint4*>(slabp + (gq + 24) * 128 + gi * 64 + c * 16);
+        float pA[kI4DChunks][4], pB[kI4DChunks][4];
+#pragma unroll
+        for (int ch = 0; ch < kI4DChunks; ++ch)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { pA[ch][i] = 0.f; pB[ch][i] = 0.f; }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t qa0[4], qa1[4], qb0[4], qb1[4];
+          offset_word(u4get(a0, j), qa0);
+          offset_word(u4get(a1, j), qa1);
+          offset_word(u4get(b0, j), qb0);
+          offset_word(u4get(b1, j), qb1);
+          uint4 xf[kI4DChunks];
+#pragma unroll
+          for (int ch = 0; ch < kI4DChunks; ++ch) {
+            const int tok = r0 + 8 * ch + gq;
+            xf[ch] = tok < R ? *reinterpret_cast<const uint4*>(p.act + (long long)tok * p.K + kg * 128 + c * 32 + 8 * j)
+                             : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int ch = 0; ch < kI4DChunks; ++ch) {
+            mma_bf16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch].x, xf[ch].y);
+            mma_bf16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch].z, xf[ch].w);
+            mma_bf16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch].x, xf[ch].y);
+            mma_bf16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch].z, xf[ch].w);
+          }
+        }
+        // offset correction (columns = rows 8 ch + 2c, 8 ch + 2c + 1) and group scales (weight rows gq, gq + 8)
+        const float scA0 = __bfloat162float(sA[kg]), scA1 = __bfloat162float(sA[s8 + kg]);
+        const float scB0 = __bfloat162float(sB[kg]), scB1 = __bfloat162float(sB[s8 + kg]);
+#pragma unroll
+        for (int ch = 0; ch < kI4DChunks; ++ch) {
+          const int n0 = r0 + 8 * ch + 2 * c;
+          const float x0 = n0 < R ? xsum[(long long)n0 * ngk + kg] : 0.f;
+          const float x1 = n0 + 1 < R ? xsum[(long long)(n0 + 1) * ngk + kg] : 0.f;
+          tA[ch][0] = fmaf(fmaf(-136.f, x0, pA[ch][0]), scA0, tA[ch][0]);
+          tA[ch][1] = fmaf(fmaf(-136.f, x1, pA[ch][1]), scA0, tA[ch][1]);
+          tA[ch][2] = fmaf(fmaf(-136.f, x0, pA[ch][2]), scA1, tA[ch][2]);
+          tA[ch][3] = fmaf(fmaf(-136.f, x1, pA[ch][3]), scA1, tA[ch][3]);
+          tB[ch][0] = fmaf(fmaf(-136.f, x0, pB[ch][0]), scB0, tB[ch][0]);
+          tB[ch][1] = fmaf(fmaf(-136.f, x1, pB[ch][1]), scB0, tB[ch][1]);
+          tB[ch][2] = fmaf(fmaf(-136.f, x0, pB[ch][2]), scB1, tB[ch][2]);
+          tB[ch][3] = fmaf(fmaf(-136.f, x1, pB[ch][3]), scB1, tB[ch][3]);
+        }
+      }
+      __syncwarp();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slab reads done before TMA reuses it
+      ++consumed;
+      if (++c_st == kI4DStages) { c_st = 0; c_phase ^= 1u; }
+    }
+    if (!ok) break;
+    // partials of this slab range, in k_int4_stream's split layout
+    const int o0 = GLU ? ob * 16 : ob * 32;
+    const int W = GLU ? 2 * p.N : p.N;
+#pragma unroll
+    for (int ch = 0; ch < kI4DChunks; ++ch) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = gq + (i >= 2 ? 8 : 0);
+        const int n = r0 + 8 * ch + 2 * c + (i & 1);
+        if (n < R) {
+          float* prow = p.part + ((long long)sp * R + n) * W + o0;
+          if (GLU) {
+            prow[m] = tA[ch][i];
+            prow[p.N + m] = tB[ch][i];
+          } else {
+            prow[m] = tA[ch][i];
+            prow[m + 16] = tB[ch][i];
+          }
+        }
+      }
+    }
+  }
+  // never leave the CTA with copies still landing in its shared memory
+  {
+    volatile int dummy = 0;
+    for (int i = consumed; i < issued; ++i)
+      mbar_wait(&s_bar[warp][i % kI4DStages], (uint32_t)((i / kI4DStages) & 1), wait_limit_ns, &dummy, 0x0204);
+  }
+  __syncwarp();
+}
+
 // Split reduction of k_int4_stream: out[r, o] from the ksplit fp32 partials added
 // in split order (gated: h = act(sum g) * (sum u); plain: y = sum).
 template <bool GLU, int ACT>

@@ -564,6 +564,8 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
       MOE_I4_ATTR(false, kModePlain, true, true) MOE_I4_ATTR(true, kModeSwiGLU, true, true)
       MOE_I4_ATTR(true, kModeGeGLU, true, true)
 #undef MOE_I4_ATTR
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_dense<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4DSmem));
+      MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_dense<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4DSmem));
       done.fetch_or(bit);
     }
     if (xsum != nullptr) {
@@ -572,6 +574,31 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
                                                                          reinterpret_cast<__nv_bfloat16*>(scr.xq));
       MOE_LAUNCH_CHECK();
       p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);
+    }
+    if (grows == nullptr && xsum != nullptr && scr.part != nullptr && R <= 256) {
+      // one dense group of a small batch (the shared expert of a decode batch): tasks of 32 weight rows over
+      // 32 rows, each weight dequantised once per 32 rows; the reduction split so that every warp has work
+      const long long base = (long long)(N / (glu ? 16 : 32)) * cdiv(R, 32);
+      const long long warps = (long long)num_sms() * kI4DWarps;
+      int ks = (int)std::min<long long>(std::min<long long>(8, cdiv(K, 256)), std::max<long long>(1, cdiv(2 * warps, base)));
+      while (ks > 1 && (size_t)ks * R * (glu ? 2 * N : N) > scr.part_floats) --ks;
+      if ((size_t)ks * R * (glu ? 2 * N : N) <= scr.part_floats) {
+        p.ksplit = ks;
+        p.part = scr.part;
+        const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), cdiv(base * ks, kI4DWarps)));
+        const unsigned long long lim = g_wait_limit_ns.load();
+        if (glu) MOE_LAUNCH((k_int4_dense<true>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xsum);
+        else MOE_LAUNCH((k_int4_dense<false>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xsum);
+        MOE_LAUNCH_CHECK();
+        const unsigned blocks = (unsigned)cdiv(R * N, 256);
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+        if (!glu) MOE_LAUNCH((k_int4_splitk_reduce<false, kModePlain>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+        else if (act == MOE_ACT_SWIGLU)
+          MOE_LAUNCH((k_int4_splitk_reduce<true, kModeSwiGLU>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+        else MOE_LAUNCH((k_int4_splitk_reduce<true, kModeGeGLU>), blocks, 256, 0, st, p.part, p.ksplit, R, N, o);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+      }
     }
     const long long rows_per_task = glu ? 16 : 32;
     const long long ub = (long long)(N / rows_per_task) * (grows ? cdiv(R, 8) + n_groups : cdiv(R, 8)) * p.ksplit;

@@ -594,8 +594,11 @@ def _check_int4_forward(wl, inp, r, sample, seed=0):
     return toks.size
 
 
-def test_forward_int4_reduced(lib):
-    wl = synth.get_workload("decode_int4").replace(d=1024, E=48, H=256, H_s=256)
+# Reduced decode layers: batches of 64 (two 32-row blocks of the dense shared-expert kernel), 100 (a ragged
+# last row block) and 7 rows; every token against the oracle.
+@pytest.mark.parametrize("T", [64, 100, 7])
+def test_forward_int4_reduced(lib, T):
+    wl = synth.get_workload("decode_int4").replace(T=T, d=1024, E=48, H=256, H_s=256)
     inp, r = _int4_forward(lib, wl)
     _check_int4_forward(wl, inp, r, sample=list(range(wl.T)))
 
