@@ -188,8 +188,8 @@ static Workspace ws_layout(const moe_shape* s) {
   L.zmax = take((size_t)s->T * 4);
   L.snc = take((size_t)s->T * 4);
   L.zex = take((size_t)s->T * kSelMaxCand * 4);
-  L.ecount = take((size_t)s->E * 4);
-  L.elist = use_tc_router(s) ? take((size_t)s->E * s->T * 4) : take(16);
+  L.ecount = take((size_t)s->E * kSelShards * 4);
+  L.elist = use_tc_router(s) ? take((size_t)s->E * kSelShards * sel_shard_cap(s->T) * 4) : take(16);
   L.total = o;
   return L;
 }
@@ -766,7 +766,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     const bool select = logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD;
     int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
     MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d,
-               select ? ecount : nullptr);
+               select ? ecount : nullptr, s->E * kSelShards);
     MOE_LAUNCH_CHECK();
     GemmExtras ex;
     ex.a_kwrap = s->d;
@@ -789,7 +789,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       MOE_LAUNCH((k_router_recompute), (unsigned)(4 * num_sms()), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
                  w_router, bias, ecount, sa.elist, zex, (int)s->T, s->d, s->E);
       MOE_LAUNCH_CHECK();
-      const unsigned nfin = (unsigned)cdiv(s->T, 8);
+      const unsigned nfin = (unsigned)cdiv(s->T, 32);
 #define MOE_FINISH(N_)                                                                                        \
   MOE_LAUNCH((k_router_finish<N_>), nfin, 256, 0, st, sa.ncand, sa.cidx, zex, sa.zmax, sa.snc, sa.x, w_router, bias, \
              idx, w, cnt, (int)s->T, s->d, s->E, s->k, s->renorm)

@@ -119,10 +119,10 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
 __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
                                                      float* __restrict__ wnorm, int E, int d,
-                                                     int32_t* __restrict__ zero_counts) {
+                                                     int32_t* __restrict__ zero_counts, int n_zero) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  if (zero_counts != nullptr && blockIdx.x == 0)   // per-expert list lengths of the certified selection
-    for (int i = threadIdx.x; i < E; i += blockDim.x) zero_counts[i] = 0;
+  if (zero_counts != nullptr && blockIdx.x == 0)   // sub-list lengths of the certified selection
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_counts[i] = 0;
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
   const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
@@ -547,8 +547,14 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
 //                      (expert, chunk).
 // The decision equals the top k of exact fp32 logits: every expert outside
 // the candidates is below the k-th exact logit by the screening bound.
-constexpr int kSelMaxD = 2048;      // W_r row held in shared memory (fp32)
+constexpr int kSelMaxD = 2048;      // largest input width of the selection path
 constexpr int kRecompBatch = 8;     // list entries per warp in flight
+constexpr int kSelShards = 16;      // sub-lists per expert (chunk % kSelShards): spreads the reservations
+
+// Entries one sub-list can hold: the tokens of its chunks (a token appears at most once per expert).
+__host__ __device__ constexpr long long sel_shard_cap(long long T) {
+  return ((T + kChunk - 1) / kChunk + kSelShards - 1) / kSelShards * kChunk;
+}
 
 struct SelectArgs {
   const float* zs;       // [T, E] screening logits (bias included)
@@ -560,15 +566,16 @@ struct SelectArgs {
   int32_t* ncand;        // [T] candidates (all of them)
   float* zmax;           // [T] largest screening logit
   float* snc;            // [T] sum over non-candidates of exp(z - zmax)
-  int32_t* ecount;       // [E] list lengths (zero before k_router_select)
-  int32_t* elist;        // [E][T] list entries t * kSelMaxCand + slot
+  int32_t* ecount;       // [E][kSelShards] sub-list lengths (zero before k_router_select)
+  int32_t* elist;        // [E][kSelShards][sel_shard_cap(T)] list entries t * kSelMaxCand + slot
   int32_t* cnt;          // [E][nchunks] pick counts, cleared here for k_router_finish
 };
 
 // One CTA = one 32-token chunk = 8 warps x 4 tokens.  A candidate takes its
 // position in its expert's list in two steps: a shared-memory counter per
 // expert inside the chunk, then one global reservation per (chunk, expert) for
-// the chunk's whole run.  The tokens of a warp are loaded together (screening
+// the chunk's whole run, in the sub-list chunk % kSelShards of the expert (so
+// no more than a few chunks reserve on the same counter).  The tokens of a warp are loaded together (screening
 // row and inputs), then processed in order.  A token keeps its first
 // kSelMaxCand candidates; with more, the finishing kernel recomputes every
 // expert for it.
@@ -667,120 +674,123 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
   }
   __syncthreads();
   // one reservation per expert for the chunk's run (all issued together), then the list entries
+  const int shard = chunk % kSelShards;
+  const long long cap = sel_shard_cap(a.T);
   for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-    if (s_cnt[e] > 0) s_base[e] = atomicAdd(&a.ecount[e], s_cnt[e]);
+    if (s_cnt[e] > 0) s_base[e] = atomicAdd(&a.ecount[e * kSelShards + shard], s_cnt[e]);
   __syncthreads();
   for (int i = threadIdx.x; i < kChunk * kSelMaxCand; i += blockDim.x) {
     const int tl = i / kSelMaxCand, slot = i % kSelMaxCand;
     if (slot < s_nk[tl]) {
       const uint32_t r = s_rec[tl][slot];
       const int e = (int)(r >> 16);
-      a.elist[(size_t)e * a.T + s_base[e] + (int)(r & 0xFFFFu)] =
+      a.elist[((size_t)e * kSelShards + shard) * cap + s_base[e] + (int)(r & 0xFFFFu)] =
           (int32_t)((chunk * kChunk + tl) * kSelMaxCand + slot);
     }
   }
 }
 
-// Exact fp32 logits of the listed (token, expert) pairs.  The lists of all
-// experts form one flat sequence (expert order); CTA b takes the b-th equal
-// slice of it -- balanced whatever the popularity of the experts -- and walks
-// the experts its slice covers, W_r[e] in shared memory.  Each entry's logit
-// is computed by a whole warp: lane l takes the 8-input slices l, l+32, ...,
-// one fmaf chain, a fixed xor tree, then the bias -- the same value whichever
-// CTA or warp computes it, and the same as warp_dot.  A warp keeps
-// kRecompBatch entries in flight.  zex[t][slot] = exact logit.
+// Exact fp32 logits of the listed (token, expert) pairs.  The sub-lists of all
+// experts form one flat sequence (expert-major); the warps of the grid take
+// equal runs of it, kRecompBatch entries at a time -- balanced whatever the
+// popularity of the experts -- and each entry finds its sub-list by a binary
+// search over the sub-list prefix (shared memory).  Each entry's logit is
+// computed by a whole warp: lane l takes the 8-input slices l, l+32, ..., one
+// fmaf chain, a fixed xor tree, then the bias -- the same value whichever warp
+// computes it, and the same as warp_dot.  W_r rows come through L1 (the
+// entries of a run mostly share an expert).  zex[t][slot] = exact logit.
 __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
                                                           const float* __restrict__ W, const float* __restrict__ bias,
                                                           const int32_t* __restrict__ ecount,
                                                           const int32_t* __restrict__ elist, float* __restrict__ zex,
                                                           int T, int d, int E) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  __shared__ __align__(16) float s_w[kSelMaxD];
-  __shared__ int s_pre[kMaxRouterE + 1];
-  const int lane = lane_id();
-  if (warp_id() == 0) {
-    // exclusive prefix of the list lengths (E <= 512: up to 16 per lane, in expert order)
-    const int per = (E + 31) / 32;
-    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  __shared__ int s_pre[kMaxRouterE * kSelShards + 1];
+  const int nl = E * kSelShards;
+  {
+    // exclusive prefix of the sub-list lengths, block-wide (each thread a contiguous run, then the warps)
+    __shared__ int s_wt[8];
+    const int per = (nl + blockDim.x - 1) / blockDim.x;
+    const int i0 = min(nl, (int)threadIdx.x * per), i1 = min(nl, i0 + per);
     int local = 0;
-    for (int e = e0; e < e1; ++e) local += ecount[e];
+    for (int i = i0; i < i1; ++i) local += ecount[i];
     int incl = local;
+    const int lane = lane_id(), wp = warp_id();
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    int run = incl - local;
-    for (int e = e0; e < e1; ++e) {
-      s_pre[e] = run;
-      run += ecount[e];
-    }
-    if (lane == 31) s_pre[E] = incl;
-  }
-  __syncthreads();
-  const long long N = s_pre[E];
-  const int f_lo = (int)(N * blockIdx.x / gridDim.x), f_hi = (int)(N * (blockIdx.x + 1) / gridDim.x);
-  if (f_lo >= f_hi) return;
-  int e = 0;   // the expert holding flat entry f_lo: last e with s_pre[e] <= f_lo
-  {
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pre[mid] <= f_lo) lo = mid; else hi = mid - 1;
-    }
-    e = lo;
-  }
-  const int nv = d >> 3;
-  const int nwarps = blockDim.x / 32;
-  for (; e < E && s_pre[e] < f_hi; ++e) {
-    const int a0 = max(f_lo, s_pre[e]), a1 = min(f_hi, s_pre[e + 1]);
-    if (a0 >= a1) continue;   // uniform across the CTA
-    __syncthreads();          // the previous expert's row is no longer read
-    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
-    for (int i = threadIdx.x; i < d / 4; i += blockDim.x) reinterpret_cast<float4*>(s_w)[i] = wr[i];
+    if (lane == 31) s_wt[wp] = incl;
     __syncthreads();
-    const float be = bias != nullptr ? bias[e] : 0.f;
-    const int32_t* lst = elist + (size_t)e * T - s_pre[e];   // indexed by flat entry
-    for (int f0 = a0 + kRecompBatch * warp_id(); f0 < a1; f0 += kRecompBatch * nwarps) {
-      int ent[kRecompBatch];
-      const uint4* xr[kRecompBatch];
+    int base = 0;
+    for (int w2 = 0; w2 < wp; ++w2) base += s_wt[w2];
+    int run = base + incl - local;
+    for (int i = i0; i < i1; ++i) {
+      s_pre[i] = run;
+      run += ecount[i];
+    }
+    if (threadIdx.x == blockDim.x - 1) s_pre[nl] = base + incl;
+    __syncthreads();
+  }
+  const long long N = s_pre[nl];
+  const long long cap = sel_shard_cap(T);
+  const int lane = lane_id(), nv = d >> 3;
+  const long long gw = (long long)blockIdx.x * (blockDim.x / 32) + warp_id();
+  const long long nw = (long long)gridDim.x * (blockDim.x / 32);
+  // warp gw takes flat entries [gw * N / nw, (gw + 1) * N / nw)
+  const long long f_lo = N * gw / nw, f_hi = N * (gw + 1) / nw;
+  for (long long f0 = f_lo; f0 < f_hi; f0 += kRecompBatch) {
+    int ent[kRecompBatch], ee[kRecompBatch];
+    const uint4* xr[kRecompBatch];
+    const float4* wr[kRecompBatch];
+#pragma unroll
+    for (int j = 0; j < kRecompBatch; ++j) {
+      const int f = (int)min(f0 + j, f_hi - 1);
+      int lo = 0, hi = nl - 1;   // the sub-list holding f: last l with s_pre[l] <= f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= f) lo = mid; else hi = mid - 1;
+      }
+      ent[j] = elist[(size_t)lo * cap + (f - s_pre[lo])];
+      ee[j] = lo / kSelShards;
+      xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
+      wr[j] = reinterpret_cast<const float4*>(W + (size_t)ee[j] * d);
+    }
+    float acc[kRecompBatch];
+#pragma unroll
+    for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
+    for (int v = lane; v < nv; v += 32) {
+      uint4 u[kRecompBatch];
+      float4 w0[kRecompBatch], w1[kRecompBatch];
 #pragma unroll
       for (int j = 0; j < kRecompBatch; ++j) {
-        ent[j] = lst[min(f0 + j, a1 - 1)];
-        xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
-      }
-      float acc[kRecompBatch];
-#pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
-      for (int v = lane; v < nv; v += 32) {
-        uint4 u[kRecompBatch];
-#pragma unroll
-        for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
-        const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
-        const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
-#pragma unroll
-        for (int j = 0; j < kRecompBatch; ++j) {
-          float s2 = acc[j];
-          s2 = fmaf(bf16lo(u[j].x), w0.x, s2); s2 = fmaf(bf16hi(u[j].x), w0.y, s2);
-          s2 = fmaf(bf16lo(u[j].y), w0.z, s2); s2 = fmaf(bf16hi(u[j].y), w0.w, s2);
-          s2 = fmaf(bf16lo(u[j].z), w1.x, s2); s2 = fmaf(bf16hi(u[j].z), w1.y, s2);
-          s2 = fmaf(bf16lo(u[j].w), w1.z, s2); s2 = fmaf(bf16hi(u[j].w), w1.w, s2);
-          acc[j] = s2;
-        }
+        u[j] = xr[j][v];
+        w0[j] = __ldg(wr[j] + 2 * v);
+        w1[j] = __ldg(wr[j] + 2 * v + 1);
       }
 #pragma unroll
       for (int j = 0; j < kRecompBatch; ++j) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        float s2 = acc[j];
+        s2 = fmaf(bf16lo(u[j].x), w0[j].x, s2); s2 = fmaf(bf16hi(u[j].x), w0[j].y, s2);
+        s2 = fmaf(bf16lo(u[j].y), w0[j].z, s2); s2 = fmaf(bf16hi(u[j].y), w0[j].w, s2);
+        s2 = fmaf(bf16lo(u[j].z), w1[j].x, s2); s2 = fmaf(bf16hi(u[j].z), w1[j].y, s2);
+        s2 = fmaf(bf16lo(u[j].w), w1[j].z, s2); s2 = fmaf(bf16hi(u[j].w), w1[j].w, s2);
+        acc[j] = s2;
       }
-      if (lane < kRecompBatch) {
-        float mine = acc[0];
-        int my_ent = ent[0];
+    }
 #pragma unroll
-        for (int j = 1; j < kRecompBatch; ++j)
-          if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
-        if (f0 + lane < a1) zex[my_ent] = mine + be;
-      }
+    for (int j = 0; j < kRecompBatch; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+    }
+    if (lane < kRecompBatch) {
+      float mine = acc[0];
+      int my_ent = ent[0], my_e = ee[0];
+#pragma unroll
+      for (int j = 1; j < kRecompBatch; ++j)
+        if (lane == j) { mine = acc[j]; my_ent = ent[j]; my_e = ee[j]; }
+      if (f0 + lane < f_hi) zex[my_ent] = mine + (bias != nullptr ? bias[my_e] : 0.f);
     }
   }
 }
@@ -815,7 +825,7 @@ __device__ __noinline__ float select_all_exact(const __nv_bfloat16* __restrict__
   return ez;
 }
 
-// Selection finish, one warp per token (8 per CTA).  Lane c holds candidate c
+// Selection finish, one warp per four tokens (8 warps per CTA).  Lane c holds candidate c
 // (exact logit, expert); the top k among them by (value desc, index asc) --
 // certified to be the top k of all experts -- come from k rounds of warp
 // argmax.  Softmax: m = the first pick's value, sum = snc * exp(m_s - m) + the
@@ -832,45 +842,56 @@ __global__ void __launch_bounds__(256) k_router_finish(const int32_t* __restrict
                                                        float* __restrict__ topk_w, int32_t* __restrict__ cnt, int T,
                                                        int d, int E, int k, int renorm) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  constexpr int TPW = 4;   // tokens per warp, their loads issued together
   const int lane = lane_id();
-  const int t = blockIdx.x * 8 + warp_id();
-  if (t >= T) return;
+  const int t0 = (blockIdx.x * 8 + warp_id()) * TPW;
   const int nchunks = (T + kChunk - 1) / kChunk;
-  // every load of the token issued together (the candidate slots past its count are masked afterwards)
-  const int nc = ncand[t];
-  const float zx = zex[(size_t)t * kSelMaxCand + lane];
-  const int cx = (int)cidx[(size_t)t * kSelMaxCand + lane];
-  const float ms = zmax[t], sn = snc[t];
-  float sel_v = 0.f, m, ssum;
-  int sel_i = 0;
-  if (nc <= kSelMaxCand) {
-    float cv = lane < nc ? zx : -INFINITY;
-    const int ci = lane < nc ? cx : 0x7fffffff;
-    const float cv0 = cv;
-    for (int j = 0; j < k; ++j) {
-      float bv = cv;
-      int bi = ci;
-      warp_argmax_redux(bv, bi);
-      if (lane == j) { sel_v = bv; sel_i = bi; }
-      if (ci == bi) cv = -INFINITY;    // taken (candidate ids are distinct)
-    }
-    m = __shfl_sync(0xffffffffu, sel_v, 0);
-    float ez = lane < nc ? __expf(cv0 - m) : 0.f;
+  int nc[TPW], cx[TPW];
+  float zx[TPW], ms[TPW], sn[TPW];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
-    ssum = ez + sn * __expf(ms - m);
-  } else {
-    ssum = select_all_exact<EPL>(x + (size_t)t * d, W, bias, d, E, k, sel_v, sel_i, m);
+  for (int tt = 0; tt < TPW; ++tt) {
+    const int t = min(t0 + tt, T - 1);
+    nc[tt] = ncand[t];
+    zx[tt] = zex[(size_t)t * kSelMaxCand + lane];      // slots past the count are masked below
+    cx[tt] = (int)cidx[(size_t)t * kSelMaxCand + lane];
+    ms[tt] = zmax[t];
+    sn[tt] = snc[t];
   }
-  const float inv = 1.f / ssum;
-  const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
-  float wsum = pj;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = sel_i;
-    topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
-    atomicAdd(&cnt[(size_t)sel_i * nchunks + t / kChunk], 1);
+  for (int tt = 0; tt < TPW; ++tt) {
+    const int t = t0 + tt;
+    if (t >= T) break;
+    float sel_v = 0.f, m, ssum;
+    int sel_i = 0;
+    if (nc[tt] <= kSelMaxCand) {
+      float cv = lane < nc[tt] ? zx[tt] : -INFINITY;
+      const int ci = lane < nc[tt] ? cx[tt] : 0x7fffffff;
+      const float cv0 = cv;
+      for (int j = 0; j < k; ++j) {
+        float bv = cv;
+        int bi = ci;
+        warp_argmax_redux(bv, bi);
+        if (lane == j) { sel_v = bv; sel_i = bi; }
+        if (ci == bi) cv = -INFINITY;    // taken (candidate ids are distinct)
+      }
+      m = __shfl_sync(0xffffffffu, sel_v, 0);
+      float ez = lane < nc[tt] ? __expf(cv0 - m) : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ez += __shfl_xor_sync(0xffffffffu, ez, o);
+      ssum = ez + sn[tt] * __expf(ms[tt] - m);
+    } else {
+      ssum = select_all_exact<EPL>(x + (size_t)t * d, W, bias, d, E, k, sel_v, sel_i, m);
+    }
+    const float inv = 1.f / ssum;
+    const float pj = lane < k ? __expf(sel_v - m) * inv : 0.f;
+    float wsum = pj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (lane < k) {
+      topk_idx[(size_t)t * k + lane] = sel_i;
+      topk_w[(size_t)t * k + lane] = renorm ? pj / wsum : pj;
+      atomicAdd(&cnt[(size_t)sel_i * nchunks + t / kChunk], 1);
+    }
   }
 }
 
