@@ -1165,19 +1165,20 @@ __global__ void __launch_bounds__(NW * 32) k_router_fused(const __nv_bfloat16* _
 
 // Router logits for small T (decode), exact fp32: W_r is the large operand and
 // is streamed from HBM once (later token blocks re-read it from L2).
-//   Grid: (ceil(E / 32), ceil(T / 16), kSkSplit) with clusters of kSkSplit CTAs
-//   along the inputs.  A CTA stages its 16 tokens x ks-input slice of x in
-//   shared memory as fp32; each of its 8 warps owns 4 experts, and lane l takes
-//   inputs 4l .. 4l+3 of every 128-input step: per step 4 coalesced float4
-//   loads of W_r rows and 16 broadcast-free float4 reads of x feed 256 FMAs
-//   (one fp32 chain per (expert, token) per lane, inputs in order).
-//   The 64 chains of a warp are combined across lanes by a transposing xor
-//   tree (62 shuffles; lane l ends with entries 2l and 2l + 1), the kSkSplit
-//   partial tiles in cluster rank order through distributed shared memory.
-//   Logits are written without bias.
-constexpr int kSkSplit = 8;
-constexpr int kSkTok = 16;
+//   Grid: (ceil(E / 32), ceil(T / kSkTok), kSkSplit) with clusters of
+//   kSkSplit CTAs along the inputs.  A CTA stages its kSkTok tokens x ks-input
+//   slice of x in shared memory as fp32; each of its 8 warps owns 4 experts, and
+//   lane l takes inputs 4l .. 4l+3 of every 128-input step: per step 4
+//   coalesced float4 loads of W_r rows and kSkTok broadcast-free float4 reads
+//   of x feed 16 kSkTok FMAs (one fp32 chain per (expert, token) per lane,
+//   inputs in order), the W_r rows of the next three steps in flight.
+//   The 4 kSkTok chains of a warp are combined across lanes by a transposing
+//   xor tree, the kSkSplit partial tiles in cluster rank order through
+//   distributed shared memory.  Logits are written without bias.
+constexpr int kSkSplit = 4;
+constexpr int kSkTok = 8;
 constexpr int kSkExp = 4;   // experts per warp
+static_assert(kSkTok == 2 * kSkSplit, "each rank of the cluster finishes two tokens");
 
 __host__ __device__ constexpr int skinny_slice(int d) {
   return ((d + 128 * kSkSplit - 1) / (128 * kSkSplit)) * 128;   // inputs per split, a multiple of 128
@@ -1225,15 +1226,22 @@ __global__ void __cluster_dims__(1, 1, kSkSplit) __launch_bounds__(256, 2) k_rou
                ? __ldg(reinterpret_cast<const float4*>(wbase + (size_t)q * d + st * 128))
                : make_float4(0.f, 0.f, 0.f, 0.f);
   };
-  float4 wn[kSkExp];
+  // the rows of the next three steps are in flight during a step's FMAs
+  float4 w1[kSkExp], w2[kSkExp], w3[kSkExp];
 #pragma unroll
-  for (int q = 0; q < kSkExp; ++q) wn[q] = load_w(0, q);
+  for (int q = 0; q < kSkExp; ++q) {
+    w1[q] = load_w(0, q);
+    w2[q] = load_w(1, q);
+    w3[q] = load_w(2, q);
+  }
   for (int st = 0; st < nsteps; ++st) {
     float4 w[kSkExp];
 #pragma unroll
     for (int q = 0; q < kSkExp; ++q) {
-      w[q] = wn[q];
-      wn[q] = load_w(st + 1, q);   // next step's rows, in flight during this step's FMAs
+      w[q] = w1[q];
+      w1[q] = w2[q];
+      w2[q] = w3[q];
+      w3[q] = load_w(st + 3, q);
     }
 #pragma unroll
     for (int t = 0; t < kSkTok; ++t) {
@@ -1260,10 +1268,11 @@ __global__ void __cluster_dims__(1, 1, kSkSplit) __launch_bounds__(256, 2) k_rou
       acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
     }
   }
-  // lane l holds entries 2l, 2l + 1 of (expert q, token t) = (idx / 16, idx % 16)
+  // lane l holds entries EL l .. EL l + EL - 1 of (expert q, token t) = (idx / kSkTok, idx % kSkTok)
+  constexpr int EL = kSkExp * kSkTok / 32;
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int idx = 2 * lane + j;
+  for (int j = 0; j < EL; ++j) {
+    const int idx = EL * lane + j;
     s_tile[idx % kSkTok][warp * kSkExp + idx / kSkTok] = acc[j];
   }
   cluster.sync();
