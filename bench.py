@@ -75,6 +75,17 @@ def int4_step_bytes(wl, touched: int) -> int:
     return touched * per_expert + shared + wl.E * wl.d * 4 + 2 * wl.T * wl.d * 2
 
 
+def gemm_step_bytes(wl, kept: int, touched: int) -> int:
+    """Algorithmic HBM bytes of the bf16 expert GEMMs of one forward: routed gate/up reads the grouped rows and
+    the touched experts' w13 and writes h; down reads h and w2 and writes y; the shared expert likewise on all T
+    tokens."""
+    routed = kept * wl.d * 2 + touched * 2 * wl.H * wl.d * 2 + 2 * kept * wl.H * 2 \
+        + touched * wl.d * wl.H * 2 + kept * wl.d * 2
+    shared = (wl.T * wl.d * 2 + 2 * wl.H_s * wl.d * 2 + 2 * wl.T * wl.H_s * 2 + wl.d * wl.H_s * 2 + wl.T * wl.d * 2) \
+        if wl.H_s else 0
+    return routed + shared
+
+
 def max_over_ranks(value: float, world: int) -> float:
     if world <= 1:
         return value
@@ -492,11 +503,17 @@ def main():
     else:
         achieved_tf = flops / (gemm_us * 1e-6) / 1e12
         peak_tf = peaks["bf16_tflops"]
+        gbytes = gemm_step_bytes(wl, kept, touched)
         roofline = {"bound": "tensor", "kernel": "k_grouped_gemm (gate/up + GLU, down; routed + shared)",
                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved_tf / peak_tf,
                     "peak_source": peaks["source"] + " burst bf16",
                     "traffic": None if args.experts else GEMM_TRAFFIC_BYTES.get(wl.name),
-                    "alg_flops_per_step": flops, "gemm_us": gemm_us}
+                    "alg_flops_per_step": flops, "gemm_us": gemm_us,
+                    # the same kernels against HBM: operands and results they must move (grouped rows, weights of
+                    # the touched experts, h written and read back, y written)
+                    "hbm_view": {"alg_bytes_per_step": gbytes, "achieved_GBps": gbytes / (gemm_us * 1e-6) / 1e9,
+                                 "peak_GBps": peaks["hbm_gbs"],
+                                 "frac": gbytes / (gemm_us * 1e-6) / 1e9 / peaks["hbm_gbs"]}}
 
     if rank == 0:
         cpu = None

@@ -138,7 +138,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 
 struct Workspace {
   size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
-  size_t cidx, ncand, zmax, snc, zex, ecount, elist;   // certified selection over the screening logits
+  size_t cidx, ncand, zmax, snc, zex, ecount, elist, xnorm2;   // certified selection over the screening logits
   size_t total;
 };
 
@@ -189,6 +189,7 @@ static Workspace ws_layout(const moe_shape* s) {
   L.snc = take((size_t)s->T * 4);
   L.zex = take((size_t)s->T * kSelMaxCand * 4);
   L.ecount = take((size_t)s->E * kSelShards * 4);
+  L.xnorm2 = take((size_t)s->T * 4);
   L.elist = use_tc_router(s) ? take((size_t)s->E * kSelShards * sel_shard_cap(s->T) * 4) : take(16);
   L.total = o;
   return L;
@@ -765,8 +766,10 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     // without logits or statistics to return, the selection lists candidates and recomputes them by expert
     const bool select = logits == nullptr && !want_stats && s->E <= 256 && s->d <= kSelMaxD;
     int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
-    MOE_LAUNCH((k_router_prep), (unsigned)cdiv(s->E, 8), 256, 0, st, w_router, wsplit, wnorm, s->E, s->d,
-               select ? ecount : nullptr, s->E * kSelShards);
+    float* xnorm2 = reinterpret_cast<float*>(ws + L.xnorm2);
+    MOE_LAUNCH((k_router_prep), (unsigned)(cdiv(s->E, 8) + (select ? cdiv(s->T, 8) : 0)), 256, 0, st, w_router, wsplit,
+               wnorm, s->E, s->d, select ? ecount : nullptr, s->E * kSelShards,
+               select ? reinterpret_cast<const __nv_bfloat16*>(x) : nullptr, xnorm2, (int)s->T);
     MOE_LAUNCH_CHECK();
     GemmExtras ex;
     ex.a_kwrap = s->d;
@@ -774,7 +777,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false, ex);
     if (rc) return rc;
     if (select) {
-      SelectArgs sa{part, reinterpret_cast<const __nv_bfloat16*>(x), wnorm, gamma, (int)s->T, s->d, s->E, s->k,
+      SelectArgs sa{part, xnorm2, reinterpret_cast<const __nv_bfloat16*>(x), wnorm, gamma, (int)s->T, s->d, s->E, s->k,
                     reinterpret_cast<uint8_t*>(ws + L.cidx), reinterpret_cast<int32_t*>(ws + L.ncand),
                     reinterpret_cast<float*>(ws + L.zmax), reinterpret_cast<float*>(ws + L.snc), ecount,
                     reinterpret_cast<int32_t*>(ws + L.elist), cnt};

@@ -117,12 +117,40 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 //    operand [hi | lo]; x is bf16, so every product x * part is exact in fp32
 //    and the screening logits are [x | x] [hi | lo]^T;
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
+//  * with x set (the certified selection path), blocks past the weight rows
+//    also compute xnorm2[t] = sum_i x[t,i]^2, one warp per token, every load of
+//    the row in flight together (d <= 2048), and block 0 clears the list
+//    lengths.
 __global__ void __launch_bounds__(256) k_router_prep(const float* __restrict__ W, __nv_bfloat16* __restrict__ Ws,
                                                      float* __restrict__ wnorm, int E, int d,
-                                                     int32_t* __restrict__ zero_counts, int n_zero) {
+                                                     int32_t* __restrict__ zero_counts, int n_zero,
+                                                     const __nv_bfloat16* __restrict__ x, float* __restrict__ xnorm2,
+                                                     int T) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  if (zero_counts != nullptr && blockIdx.x == 0)   // sub-list lengths of the certified selection
+  if (zero_counts != nullptr && blockIdx.x == 0)   // list lengths of the certified selection
     for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero_counts[i] = 0;
+  const int wblocks = (E + 7) / 8;
+  if ((int)blockIdx.x >= wblocks) {
+    const long long t = (long long)(blockIdx.x - wblocks) * 8 + warp_id();
+    if (x == nullptr || t >= T) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + t * d);
+    const int nv = d >> 3;
+    uint4 u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j] = lane_id() + 32 * j < nv ? xr[lane_id() + 32 * j] : make_uint4(0, 0, 0, 0);
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float q[8] = {bf16lo(u[j].x), bf16hi(u[j].x), bf16lo(u[j].y), bf16hi(u[j].y),
+                          bf16lo(u[j].z), bf16hi(u[j].z), bf16lo(u[j].w), bf16hi(u[j].w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(q[i], q[i], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane_id() == 0) xnorm2[t] = ss;
+    return;
+  }
   const int e = blockIdx.x * 8 + warp_id();
   if (e >= E) return;
   const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
@@ -549,7 +577,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
 // the candidates is below the k-th exact logit by the screening bound.
 constexpr int kSelMaxD = 2048;      // largest input width of the selection path
 constexpr int kRecompBatch = 8;     // list entries per warp in flight
-constexpr int kSelShards = 16;      // sub-lists per expert (chunk % kSelShards): spreads the reservations
+constexpr int kSelShards = 1;       // sub-lists per expert (chunk % kSelShards)
 
 // Entries one sub-list can hold: the tokens of its chunks (a token appears at most once per expert).
 __host__ __device__ constexpr long long sel_shard_cap(long long T) {
@@ -558,6 +586,7 @@ __host__ __device__ constexpr long long sel_shard_cap(long long T) {
 
 struct SelectArgs {
   const float* zs;       // [T, E] screening logits (bias included)
+  const float* xnorm2;   // [T] sum of x_t^2
   const __nv_bfloat16* x;
   const float* wnorm;    // [E] ||W_r[e]||_2
   float gamma;           // |screen - exact| <= gamma ||x_t|| max_e ||w_e||
@@ -599,10 +628,9 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
   for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
-  const int nv = a.d >> 3;
-  // screening rows and input sums of squares of the warp's tokens, loads issued together
+  // screening rows and input norms of the warp's tokens, loads issued together
   float z[TPW][EPL];
-  float ss[TPW];
+  float x2s[TPW];
 #pragma unroll
   for (int tt = 0; tt < TPW; ++tt) {
     const int t = chunk * kChunk + warp * TPW + tt;
@@ -612,16 +640,7 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
       const int e = lane + 32 * i;
       z[tt][i] = (on && e < a.E) ? a.zs[(size_t)t * a.E + e] : -INFINITY;
     }
-    float acc = 0.f;
-    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(on ? t : 0) * a.d);
-    for (int v = lane; v < nv; v += 32) {
-      const uint4 u = on ? xr[v] : make_uint4(0, 0, 0, 0);
-      const float q[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
-                          bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc = fmaf(q[j], q[j], acc);
-    }
-    ss[tt] = acc;
+    x2s[tt] = on ? a.xnorm2[t] : 0.f;
   }
 #pragma unroll
   for (int tt = 0; tt < TPW; ++tt) {
@@ -631,9 +650,7 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
       if (lane == 0) s_nk[tl] = 0;
       continue;
     }
-    float x2 = ss[tt];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x2 += __shfl_xor_sync(0xffffffffu, x2, o);
+    const float x2 = x2s[tt];
     const float kth = warp_kth<EPL>(z[tt], a.E, a.k);
     float m_s;
     {
@@ -710,7 +727,7 @@ __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* _
   {
     // exclusive prefix of the sub-list lengths, block-wide (each thread a contiguous run, then the warps)
     __shared__ int s_wt[8];
-    const int per = (nl + blockDim.x - 1) / blockDim.x;
+    const int per = (nl + blockDim.x - 1) / blockDim.x;   // <= 2 (nl <= 512)
     const int i0 = min(nl, (int)threadIdx.x * per), i1 = min(nl, i0 + per);
     int local = 0;
     for (int i = i0; i < i1; ++i) local += ecount[i];
@@ -740,6 +757,14 @@ __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* _
   const long long nw = (long long)gridDim.x * (blockDim.x / 32);
   // warp gw takes flat entries [gw * N / nw, (gw + 1) * N / nw)
   const long long f_lo = N * gw / nw, f_hi = N * (gw + 1) / nw;
+  int l = 0;   // the sub-list holding f_lo: last l with s_pre[l] <= f_lo
+  {
+    int hi = nl - 1;
+    while (l < hi) {
+      const int mid = (l + hi + 1) >> 1;
+      if (s_pre[mid] <= f_lo) l = mid; else hi = mid - 1;
+    }
+  }
   for (long long f0 = f_lo; f0 < f_hi; f0 += kRecompBatch) {
     int ent[kRecompBatch], ee[kRecompBatch];
     const uint4* xr[kRecompBatch];
@@ -747,11 +772,8 @@ __global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* _
 #pragma unroll
     for (int j = 0; j < kRecompBatch; ++j) {
       const int f = (int)min(f0 + j, f_hi - 1);
-      int lo = 0, hi = nl - 1;   // the sub-list holding f: last l with s_pre[l] <= f
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_pre[mid] <= f) lo = mid; else hi = mid - 1;
-      }
+      while (s_pre[l + 1] <= f) ++l;   // entries are visited in order: the sub-list only moves forward
+      const int lo = l;
       ent[j] = elist[(size_t)lo * cap + (f - s_pre[lo])];
       ee[j] = lo / kSelShards;
       xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
