@@ -188,9 +188,9 @@ static Workspace ws_layout(const moe_shape* s) {
   L.zmax = take((size_t)s->T * 4);
   L.snc = take((size_t)s->T * 4);
   L.zex = take((size_t)s->T * kSelMaxCand * 4);
-  L.ecount = take((size_t)s->E * kSelShards * 4);
+  L.ecount = take((size_t)s->E * 4);
   L.xnorm2 = take((size_t)s->T * 4);
-  L.elist = use_tc_router(s) ? take((size_t)s->E * kSelShards * sel_shard_cap(s->T) * 4) : take(16);
+  L.elist = use_tc_router(s) ? take((size_t)s->E * s->T * 4) : take(16);
   L.total = o;
   return L;
 }
@@ -768,7 +768,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     int32_t* ecount = reinterpret_cast<int32_t*>(ws + L.ecount);
     float* xnorm2 = reinterpret_cast<float*>(ws + L.xnorm2);
     MOE_LAUNCH((k_router_prep), (unsigned)(cdiv(s->E, 8) + (select ? cdiv(s->T, 8) : 0)), 256, 0, st, w_router, wsplit,
-               wnorm, s->E, s->d, select ? ecount : nullptr, s->E * kSelShards,
+               wnorm, s->E, s->d, select ? ecount : nullptr, s->E,
                select ? reinterpret_cast<const __nv_bfloat16*>(x) : nullptr, xnorm2, (int)s->T);
     MOE_LAUNCH_CHECK();
     GemmExtras ex;
@@ -789,7 +789,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       else MOE_LAUNCH((k_router_select<8>), nch, 256, 0, st, sa);
       MOE_LAUNCH_CHECK();
       float* zex = reinterpret_cast<float*>(ws + L.zex);
-      MOE_LAUNCH((k_router_recompute), (unsigned)(4 * num_sms()), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
+      MOE_LAUNCH((k_router_recompute), (unsigned)(2 * num_sms()), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
                  w_router, bias, ecount, sa.elist, zex, (int)s->T, s->d, s->E);
       MOE_LAUNCH_CHECK();
       const unsigned nfin = (unsigned)cdiv(s->T, 32);

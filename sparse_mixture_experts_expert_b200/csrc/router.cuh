@@ -577,12 +577,6 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
 // the candidates is below the k-th exact logit by the screening bound.
 constexpr int kSelMaxD = 2048;      // largest input width of the selection path
 constexpr int kRecompBatch = 8;     // list entries per warp in flight
-constexpr int kSelShards = 1;       // sub-lists per expert (chunk % kSelShards)
-
-// Entries one sub-list can hold: the tokens of its chunks (a token appears at most once per expert).
-__host__ __device__ constexpr long long sel_shard_cap(long long T) {
-  return ((T + kChunk - 1) / kChunk + kSelShards - 1) / kSelShards * kChunk;
-}
 
 struct SelectArgs {
   const float* zs;       // [T, E] screening logits (bias included)
@@ -595,16 +589,15 @@ struct SelectArgs {
   int32_t* ncand;        // [T] candidates (all of them)
   float* zmax;           // [T] largest screening logit
   float* snc;            // [T] sum over non-candidates of exp(z - zmax)
-  int32_t* ecount;       // [E][kSelShards] sub-list lengths (zero before k_router_select)
-  int32_t* elist;        // [E][kSelShards][sel_shard_cap(T)] list entries t * kSelMaxCand + slot
+  int32_t* ecount;       // [E] list lengths (zero before k_router_select)
+  int32_t* elist;        // [E][T] list entries t * kSelMaxCand + slot (a token at most once per expert)
   int32_t* cnt;          // [E][nchunks] pick counts, cleared here for k_router_finish
 };
 
 // One CTA = one 32-token chunk = 8 warps x 4 tokens.  A candidate takes its
 // position in its expert's list in two steps: a shared-memory counter per
 // expert inside the chunk, then one global reservation per (chunk, expert) for
-// the chunk's whole run, in the sub-list chunk % kSelShards of the expert (so
-// no more than a few chunks reserve on the same counter).  The tokens of a warp are loaded together (screening
+// the chunk's whole run.  The tokens of a warp are loaded together (screening
 // row and inputs), then processed in order.  A token keeps its first
 // kSelMaxCand candidates; with more, the finishing kernel recomputes every
 // expert for it.
@@ -691,128 +684,122 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
   }
   __syncthreads();
   // one reservation per expert for the chunk's run (all issued together), then the list entries
-  const int shard = chunk % kSelShards;
-  const long long cap = sel_shard_cap(a.T);
   for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-    if (s_cnt[e] > 0) s_base[e] = atomicAdd(&a.ecount[e * kSelShards + shard], s_cnt[e]);
+    if (s_cnt[e] > 0) s_base[e] = atomicAdd(&a.ecount[e], s_cnt[e]);
   __syncthreads();
   for (int i = threadIdx.x; i < kChunk * kSelMaxCand; i += blockDim.x) {
     const int tl = i / kSelMaxCand, slot = i % kSelMaxCand;
     if (slot < s_nk[tl]) {
       const uint32_t r = s_rec[tl][slot];
       const int e = (int)(r >> 16);
-      a.elist[((size_t)e * kSelShards + shard) * cap + s_base[e] + (int)(r & 0xFFFFu)] =
+      a.elist[(size_t)e * a.T + s_base[e] + (int)(r & 0xFFFFu)] =
           (int32_t)((chunk * kChunk + tl) * kSelMaxCand + slot);
     }
   }
 }
 
-// Exact fp32 logits of the listed (token, expert) pairs.  The sub-lists of all
-// experts form one flat sequence (expert-major); the warps of the grid take
-// equal runs of it, kRecompBatch entries at a time -- balanced whatever the
-// popularity of the experts -- and each entry finds its sub-list by a binary
-// search over the sub-list prefix (shared memory).  Each entry's logit is
-// computed by a whole warp: lane l takes the 8-input slices l, l+32, ..., one
-// fmaf chain, a fixed xor tree, then the bias -- the same value whichever warp
-// computes it, and the same as warp_dot.  W_r rows come through L1 (the
-// entries of a run mostly share an expert).  zex[t][slot] = exact logit.
-__global__ void __launch_bounds__(256) k_router_recompute(const __nv_bfloat16* __restrict__ x,
-                                                          const float* __restrict__ W, const float* __restrict__ bias,
-                                                          const int32_t* __restrict__ ecount,
-                                                          const int32_t* __restrict__ elist, float* __restrict__ zex,
-                                                          int T, int d, int E) {
+// Exact fp32 logits of the listed (token, expert) pairs, expert-major.  The
+// work items are slices of kRecompSlice consecutive entries of one expert's
+// list (lists of popular experts give many items, so the load stays balanced
+// whatever the routing skew); CTA b takes items b, b + gridDim.x, ...  Per
+// item the CTA stages the expert's W_r row (fp32, reloaded only when the
+// expert changes) and the slice's entries in shared memory, then each warp
+// computes kRecompBatch entries with their input-row loads in flight together:
+// lane l takes the 8-input slices l, l+32, ..., one fmaf chain, a fixed xor
+// tree, then the bias -- the same value for a (token, expert) pair whichever
+// CTA or warp computes it, and the same as warp_dot.  zex[t][slot] = exact logit.
+constexpr int kRecompSlice = 128;
+__global__ void __launch_bounds__(256, 2) k_router_recompute(const __nv_bfloat16* __restrict__ x,
+                                                             const float* __restrict__ W,
+                                                             const float* __restrict__ bias,
+                                                             const int32_t* __restrict__ ecount,
+                                                             const int32_t* __restrict__ elist,
+                                                             float* __restrict__ zex, int T, int d, int E) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  __shared__ int s_pre[kMaxRouterE * kSelShards + 1];
-  const int nl = E * kSelShards;
-  {
-    // exclusive prefix of the sub-list lengths, block-wide (each thread a contiguous run, then the warps)
-    __shared__ int s_wt[8];
-    const int per = (nl + blockDim.x - 1) / blockDim.x;   // <= 2 (nl <= 512)
-    const int i0 = min(nl, (int)threadIdx.x * per), i1 = min(nl, i0 + per);
+  static_assert(kRecompSlice == 8 * 2 * kRecompBatch, "a slice is two batches per warp of a 256-thread CTA");
+  __shared__ __align__(16) float s_w[kSelMaxD];
+  __shared__ int s_ipre[kMaxRouterE + 1];   // items of experts < e
+  __shared__ int s_ent[kRecompSlice];
+  const int lane = lane_id();
+  if (warp_id() == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
     int local = 0;
-    for (int i = i0; i < i1; ++i) local += ecount[i];
+    for (int e = e0; e < e1; ++e) local += (ecount[e] + kRecompSlice - 1) / kRecompSlice;
     int incl = local;
-    const int lane = lane_id(), wp = warp_id();
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    if (lane == 31) s_wt[wp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w2 = 0; w2 < wp; ++w2) base += s_wt[w2];
-    int run = base + incl - local;
-    for (int i = i0; i < i1; ++i) {
-      s_pre[i] = run;
-      run += ecount[i];
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      s_ipre[e] = run;
+      run += (ecount[e] + kRecompSlice - 1) / kRecompSlice;
     }
-    if (threadIdx.x == blockDim.x - 1) s_pre[nl] = base + incl;
-    __syncthreads();
+    if (lane == 31) s_ipre[E] = incl;
   }
-  const long long N = s_pre[nl];
-  const long long cap = sel_shard_cap(T);
-  const int lane = lane_id(), nv = d >> 3;
-  const long long gw = (long long)blockIdx.x * (blockDim.x / 32) + warp_id();
-  const long long nw = (long long)gridDim.x * (blockDim.x / 32);
-  // warp gw takes flat entries [gw * N / nw, (gw + 1) * N / nw)
-  const long long f_lo = N * gw / nw, f_hi = N * (gw + 1) / nw;
-  int l = 0;   // the sub-list holding f_lo: last l with s_pre[l] <= f_lo
-  {
-    int hi = nl - 1;
-    while (l < hi) {
-      const int mid = (l + hi + 1) >> 1;
-      if (s_pre[mid] <= f_lo) l = mid; else hi = mid - 1;
+  __syncthreads();
+  const int nitems = s_ipre[E];
+  const int nv = d >> 3;
+  int cur_e = -1;
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+    int lo = 0, hi = E - 1;   // the item's expert: last e with s_ipre[e] <= item
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_ipre[mid] <= item) lo = mid; else hi = mid - 1;
     }
-  }
-  for (long long f0 = f_lo; f0 < f_hi; f0 += kRecompBatch) {
-    int ent[kRecompBatch], ee[kRecompBatch];
-    const uint4* xr[kRecompBatch];
-    const float4* wr[kRecompBatch];
-#pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) {
-      const int f = (int)min(f0 + j, f_hi - 1);
-      while (s_pre[l + 1] <= f) ++l;   // entries are visited in order: the sub-list only moves forward
-      const int lo = l;
-      ent[j] = elist[(size_t)lo * cap + (f - s_pre[lo])];
-      ee[j] = lo / kSelShards;
-      xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
-      wr[j] = reinterpret_cast<const float4*>(W + (size_t)ee[j] * d);
-    }
-    float acc[kRecompBatch];
-#pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-      uint4 u[kRecompBatch];
-      float4 w0[kRecompBatch], w1[kRecompBatch];
+    const int e = lo;
+    const int a0 = (item - s_ipre[e]) * kRecompSlice;
+    const int n = min(kRecompSlice, ecount[e] - a0);
+    __syncthreads();   // the previous item's row and entries are no longer read
+    if (e != cur_e)
+      for (int i = threadIdx.x; i < d / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(s_w)[i] = reinterpret_cast<const float4*>(W + (size_t)e * d)[i];
+    if (threadIdx.x < n) s_ent[threadIdx.x] = elist[(size_t)e * T + a0 + threadIdx.x];
+    cur_e = e;
+    __syncthreads();
+    const float be = bias != nullptr ? bias[e] : 0.f;
+    for (int b0 = kRecompBatch * warp_id(); b0 < n; b0 += kRecompBatch * (blockDim.x / 32)) {
+      int ent[kRecompBatch];
+      const uint4* xr[kRecompBatch];
 #pragma unroll
       for (int j = 0; j < kRecompBatch; ++j) {
-        u[j] = xr[j][v];
-        w0[j] = __ldg(wr[j] + 2 * v);
-        w1[j] = __ldg(wr[j] + 2 * v + 1);
+        ent[j] = s_ent[min(b0 + j, n - 1)];
+        xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
+      }
+      float acc[kRecompBatch];
+#pragma unroll
+      for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
+      for (int v = lane; v < nv; v += 32) {
+        uint4 u[kRecompBatch];
+#pragma unroll
+        for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
+        const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
+        const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
+#pragma unroll
+        for (int j = 0; j < kRecompBatch; ++j) {
+          float s2 = acc[j];
+          s2 = fmaf(bf16lo(u[j].x), w0.x, s2); s2 = fmaf(bf16hi(u[j].x), w0.y, s2);
+          s2 = fmaf(bf16lo(u[j].y), w0.z, s2); s2 = fmaf(bf16hi(u[j].y), w0.w, s2);
+          s2 = fmaf(bf16lo(u[j].z), w1.x, s2); s2 = fmaf(bf16hi(u[j].z), w1.y, s2);
+          s2 = fmaf(bf16lo(u[j].w), w1.z, s2); s2 = fmaf(bf16hi(u[j].w), w1.w, s2);
+          acc[j] = s2;
+        }
       }
 #pragma unroll
       for (int j = 0; j < kRecompBatch; ++j) {
-        float s2 = acc[j];
-        s2 = fmaf(bf16lo(u[j].x), w0[j].x, s2); s2 = fmaf(bf16hi(u[j].x), w0[j].y, s2);
-        s2 = fmaf(bf16lo(u[j].y), w0[j].z, s2); s2 = fmaf(bf16hi(u[j].y), w0[j].w, s2);
-        s2 = fmaf(bf16lo(u[j].z), w1[j].x, s2); s2 = fmaf(bf16hi(u[j].z), w1[j].y, s2);
-        s2 = fmaf(bf16lo(u[j].w), w1[j].z, s2); s2 = fmaf(bf16hi(u[j].w), w1[j].w, s2);
-        acc[j] = s2;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
       }
-    }
+      if (lane < kRecompBatch) {
+        float mine = acc[0];
+        int my_ent = ent[0];
 #pragma unroll
-    for (int j = 0; j < kRecompBatch; ++j) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-    }
-    if (lane < kRecompBatch) {
-      float mine = acc[0];
-      int my_ent = ent[0], my_e = ee[0];
-#pragma unroll
-      for (int j = 1; j < kRecompBatch; ++j)
-        if (lane == j) { mine = acc[j]; my_ent = ent[j]; my_e = ee[j]; }
-      if (f0 + lane < f_hi) zex[my_ent] = mine + (bias != nullptr ? bias[my_e] : 0.f);
+        for (int j = 1; j < kRecompBatch; ++j)
+          if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
+        if (b0 + lane < n) zex[my_ent] = mine + be;
+      }
     }
   }
 }
