@@ -536,6 +536,15 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
         for (int ch = 0; ch < kI4DChunks; ++ch)
 #pragma unroll
           for (int i = 0; i < 4; ++i) { pA[ch][i] = 0.f; pB[ch][i] = 0.f; }
+        // the group's activation fragments of every chunk, loads in flight together
+        uint4 xf[kI4DChunks][4];
+#pragma unroll
+        for (int ch = 0; ch < kI4DChunks; ++ch) {
+          const int tok = r0 + 8 * ch + gq;
+          const uint4* xrow = reinterpret_cast<const uint4*>(p.act + (long long)(tok < R ? tok : 0) * p.K + kg * 128 + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) xf[ch][j] = tok < R ? xrow[j] : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t qa0[4], qa1[4], qb0[4], qb1[4];
@@ -543,19 +552,12 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
           offset_word(u4get(a1, j), qa1);
           offset_word(u4get(b0, j), qb0);
           offset_word(u4get(b1, j), qb1);
-          uint4 xf[kI4DChunks];
 #pragma unroll
           for (int ch = 0; ch < kI4DChunks; ++ch) {
-            const int tok = r0 + 8 * ch + gq;
-            xf[ch] = tok < R ? *reinterpret_cast<const uint4*>(p.act + (long long)tok * p.K + kg * 128 + c * 32 + 8 * j)
-                             : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int ch = 0; ch < kI4DChunks; ++ch) {
-            mma_bf16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch].x, xf[ch].y);
-            mma_bf16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch].z, xf[ch].w);
-            mma_bf16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch].x, xf[ch].y);
-            mma_bf16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch].z, xf[ch].w);
+            mma_bf16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch][j].x, xf[ch][j].y);
+            mma_bf16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch][j].z, xf[ch][j].w);
+            mma_bf16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch][j].x, xf[ch][j].y);
+            mma_bf16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch][j].z, xf[ch][j].w);
           }
         }
         // offset correction (columns = rows 8 ch + 2c, 8 ch + 2c + 1) and group scales (weight rows gq, gq + 8)

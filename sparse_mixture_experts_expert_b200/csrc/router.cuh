@@ -320,32 +320,32 @@ __device__ __forceinline__ float warp_topk(const float (&z)[EPL], int E, int k, 
 }
 
 // The k-th largest of the lanes' logits (with multiplicity), without the
-// indices: k rounds of a warp max, each removing one holder of the maximum.
+// indices: rounds of (warp maximum, how many entries equal it); the k-th
+// largest is the maximum of the round at which the running count reaches k,
+// and each earlier round removes its maximum's entries.  Entries past the
+// expert count must be -inf.  At most k rounds (each removes at least one).
 template <int EPL>
 __device__ __forceinline__ float warp_kth(const float (&z)[EPL], int E, int k) {
-  const int lane = lane_id();
-  unsigned used = 0u;
-  float kth = -INFINITY;
-  for (int j = 0; j < k; ++j) {
-    float lm = -INFINITY;
+  (void)E;
+  float zz[EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i)
-      if (lane + 32 * i < E && !((used >> i) & 1u)) lm = fmaxf(lm, z[i]);
+  for (int i = 0; i < EPL; ++i) zz[i] = z[i];
+  int need = k;
+  for (;;) {
+    float lm = zz[0];
+#pragma unroll
+    for (int i = 1; i < EPL; ++i) lm = fmaxf(lm, zz[i]);
     float m;
     asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(lm));
-    const unsigned holders = __ballot_sync(0xffffffffu, lm == m);
-    if (lane == __ffs(holders) - 1) {
-      bool done = false;
+    int c = 0;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (!done && lane + 32 * i < E && !((used >> i) & 1u) && z[i] == m) {
-          used |= 1u << i;
-          done = true;
-        }
-    }
-    kth = m;
+    for (int i = 0; i < EPL; ++i) c += zz[i] == m ? 1 : 0;
+    const int total = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+    if (total >= need) return m;
+    need -= total;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) zz[i] = zz[i] == m ? -INFINITY : zz[i];
   }
-  return kth;
 }
 
 // Exact fp32 logit of one (token, expert) pair with the token's inputs held in
