@@ -34,10 +34,12 @@ if ROOT not in sys.path:
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200; % of bf16 tensor-core or HBM roofline"
 DEFAULT_WORKLOAD = "granular"
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the expert GEMM launches of one forward, from an
-# `ncu --set full --clock-control none -k regex:k_grouped_gemm` capture of `bench.py --workload <name> --steps 1
-# --warmup 3 --no-cpu-baseline` on the current kernels; workloads without a complete capture report null.
-GEMM_TRAFFIC_BYTES = {"small": 12628736 + 21004032}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the expert GEMM launches of one forward (routed
+# gate/up, routed down, shared gate/up, shared down), from an `ncu --set full --clock-control none
+# -k regex:k_grouped_gemm -s 5 -c 5` capture of `bench.py --workload <name> --steps 1 --warmup 1
+# --no-cpu-baseline` on the current kernels; workloads without a complete capture report null.
+GEMM_TRAFFIC_BYTES = {"small": 12628736 + 21004032,
+                      "granular": (380195584 + 152007424 + 51951872 + 34377216) + (56189184 + 151253248 + 5779456 + 4224256)}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
