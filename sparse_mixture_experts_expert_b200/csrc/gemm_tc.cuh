@@ -8,6 +8,11 @@
 //     GeGLU: exact-erf GELU).  MoEEvolve README "SwiGLU hidden 256",
 //     kieve-moe "top-k GeGLU", the Kvasir worker's "3 mat-muls".
 //   GEMM 2 (down): A = h [R, H], B_g = w2[g] [d, H], epilogue writes y in bf16.
+//   Router screen: A = x [T, d], B = [W_hi | W_lo] [E, 2d] (the two bf16 terms
+//     of W_r side by side); each k-step loads the A tile once and both terms'
+//     B tiles, whose MMAs accumulate into one fp32 accumulator, so the 2d
+//     products x_i W_hi[e,i] and x_i W_lo[e,i] are summed as one reduction;
+//     the epilogue adds the bias and writes fp32 logits.
 // The ExpertMesh README names a grouped GEMM with fused gate/up/down as the
 // optimisation path of its routed-expert kernel; this is that GEMM for sm_100a.
 //
@@ -41,22 +46,21 @@
 
 namespace moe {
 
-enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeF32 = 3 };
+enum GemmMode { kModePlain = 0, kModeSwiGLU = 1, kModeGeGLU = 2, kModeScreen = 3 };
 
 struct GemmParams {
   const int32_t* group_start;  // [n_groups] or nullptr (one group of R rows)
   const int32_t* group_rows;   // [n_groups] or nullptr
   int n_groups;
   long long R;
-  int K;          // reduction length
+  int K;          // reduction length (screen: of A; B holds 2K columns)
   int N;          // output columns
   int up_row0;    // GLU: first row of the up half in B (= H)
   __nv_bfloat16* out;
   long long ldo;
   unsigned long long wait_limit_ns;
-  int a_kwrap;         // > 0: the A operand repeats every a_kwrap columns of the reduction (split router)
-  float* out_f32;      // kModeF32: fp32 output [R, N]
-  const float* bias;   // kModeF32: optional per-column bias [N]
+  float* out_f32;      // kModeScreen: fp32 output [R, N]
+  const float* bias;   // kModeScreen: optional per-column bias [N]
 };
 
 #ifndef MOE_GEMM_MAX_STAGES
@@ -70,10 +74,11 @@ constexpr int kEpiW = 64;                                   // columns staged pe
 constexpr int kEpiRow = kEpiW + 8;                          // padded staging row (bf16), conflict-free
 constexpr int kEpiBytes = 4 * 32 * kEpiRow * 2;             // four epilogue warps x 32 rows
 
-template <int BN, int CG = 1>
+template <int BN, int CG = 1, int NB = 1>   // NB: B tiles per k-step (2 for the router screen)
 struct GemmCfg {
   static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = (CG == 2 ? BN / 2 : BN) * kBK * 2;
+  static constexpr int kBBox = (CG == 2 ? BN / 2 : BN) * kBK * 2;   // one B box, a whole number of 1 KB atoms
+  static constexpr int kBBytes = kBBox * NB;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBudget = 219 * 1024 - 1024 - kEpiBytes;
   static constexpr int kStages = kBudget / kStageBytes > MOE_GEMM_MAX_STAGES ? MOE_GEMM_MAX_STAGES
@@ -101,10 +106,10 @@ __global__ void __launch_bounds__(256, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  using Cfg = GemmCfg<BN, CG>;
+  constexpr bool kScreen = MODE == kModeScreen;
+  using Cfg = GemmCfg<BN, CG, kScreen ? 2 : 1>;
   constexpr bool kGLU = MODE == kModeSwiGLU || MODE == kModeGeGLU;
   constexpr bool kPair = CG == 2;
-  static_assert(!kPair || MODE != kModeF32, "the router GEMM runs on single CTAs");
   constexpr int OUTN = kGLU ? BN / 2 : BN;  // output columns per tile
   constexpr int BOXB = kGLU ? BN / 2 : BN;  // rows per B box (single CTA)
   constexpr int TM = kBM * CG;              // rows per tile
@@ -225,15 +230,16 @@ __global__ void __launch_bounds__(256, 1)
             tma_load_2d_pair(a_s, &tmA, fb, kb * kBK, (int)row0);
             const int brow = kGLU ? (crank == 0 ? n0 : p.up_row0 + n0) : n0 + crank * (BN / 2);
             tma_load_3d_pair(b_s, &tmB, fb, kb * kBK, brow, g);
+            if (kScreen) tma_load_3d_pair(b_s + Cfg::kBBox, &tmB, fb, p.K + kb * kBK, brow, g);
           }
         } else if (lane == 0) {
-          const int ka = p.a_kwrap > 0 ? (kb * kBK) % p.a_kwrap : kb * kBK;
-          tma_load_2d(a_s, &tmA, &bar_full[stage], ka, (int)row0);
+          tma_load_2d(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0);
           if (kGLU) {
             tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
             tma_load_3d(b_s + BOXB * 128, &tmB, &bar_full[stage], kb * kBK, p.up_row0 + n0, g);
           } else {
             tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
+            if (kScreen) tma_load_3d(b_s + Cfg::kBBox, &tmB, &bar_full[stage], p.K + kb * kBK, n0, g);
           }
         }
         ++issued;
@@ -280,6 +286,11 @@ __global__ void __launch_bounds__(256, 1)
             else
               tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b_addr + kk * 32), IDESC,
                           (kb > 0 || kk > 0) ? 1u : 0u);
+            if (kScreen) {   // the second term of W_r, same A tile, same accumulator
+              const uint32_t b2 = b_addr + Cfg::kBBox + kk * 32;
+              if (kPair) tc_mma_bf16_pair(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b2), IDESC, 1u);
+              else tc_mma_bf16(d_tmem, smem_desc_k128(a_addr + kk * 32), smem_desc_k128(b2), IDESC, 1u);
+            }
           }
           if (kPair) tc_commit_pair_mc(&bar_empty[stage], 0x3);
           else tc_commit(&bar_empty[stage]);
@@ -328,7 +339,7 @@ __global__ void __launch_bounds__(256, 1)
       if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0106)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (MODE == kModeF32) {
+      if (kScreen) {
         // fp32 rows through the staging buffer, 32 columns (128 bytes per row) per round
         float* fstg = reinterpret_cast<float*>(stg);  // 32 rows x 36 floats per warp
         constexpr int FR = 36;

@@ -9,14 +9,19 @@
 // Decode batches put ~1-8 rows on each touched expert, so the GEMM is bound
 // by streaming the weights from HBM: every weight byte is read once and every
 // activation row of the group reuses it from registers.
-//   * the nibbles become bf16 pairs with one LOP3 each (the nibble, with its
-//     sign bit flipped, becomes the low mantissa bits of 128.0), optionally
-//     followed by one packed subtraction of 136 -- or not, in which case the
-//     product uses the codes q + 136 and 136 * sum(x) is removed per group;
-//   * mma.sync m16n8k16 (bf16 in, fp32 out) multiplies the integer codes
-//     (exact in bf16) by up to 8 activation rows; the reduction order inside a
-//     128-group is permuted identically for weights and activations, so a
-//     thread's 32 consecutive nibbles feed its fragments directly;
+//   * the nibbles become 16-bit float pairs with one LOP3 each (the nibble,
+//     with its sign bit flipped, becomes mantissa bits of a power of two):
+//     - offset codes (the forward's path): f16 codes 1032 + q (even inputs,
+//       mantissa bits 0..3 of 1024.0) and 72 + q (odd inputs, mantissa bits
+//       4..7 of 64.0), one shift per word of 8 nibbles; the activations are
+//       f16 copies scaled by a power of two per 128-group, and the offsets'
+//       share, sum(off_i x_i), is removed per group afterwards;
+//     - exact codes (the per-step entry point): bf16 128 + (q + 8) followed by
+//       one packed subtraction of 136, three shifts per word;
+//   * mma.sync m16n8k16 (fp32 accumulation) multiplies the integer codes
+//     (exact in f16 / bf16) by up to 8 activation rows; the reduction order
+//     inside a 128-group is permuted identically for weights and activations,
+//     so a thread's 32 consecutive nibbles feed its fragments directly;
 //   * the fp32 partial of each 128-group is scaled by its bf16 scale and added
 //     to the fp32 total: w = q * s is applied exactly;
 //   * gated mode writes h = act(x W1^T) * (x W3^T) in bf16, plain mode y.
@@ -30,7 +35,7 @@ namespace moe {
 struct Int4Params {
   const uint8_t* wq;             // [G, b_rows, K/2]
   const __nv_bfloat16* ws;       // [G, b_rows, K/128]
-  const __nv_bfloat16* act;      // [R, K]
+  const __nv_bfloat16* act;      // [R, K] (offset-code kernels: the f16 copy of k_int4_act_prep)
   const int32_t* group_start;    // [G] or nullptr (one group of R rows)
   const int32_t* group_rows;     // [G] or nullptr
   int n_groups;
@@ -87,28 +92,34 @@ __device__ __forceinline__ uint32_t u4get(const uint4& v, int j) {
   return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-// Word of 8 nibbles -> four bf16 pairs holding q + 136 (= 128 + (q + 8)), no
-// subtraction: the caller removes 136 * sum(x) per 128-group afterwards.
-__device__ __forceinline__ void offset_word(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t kMask = 0x000F000Fu, kMagic = 0x43084308u;
-  p[0] = lop3_and_xor(w, kMask, kMagic);
-  p[1] = lop3_and_xor(w >> 4, kMask, kMagic);
-  p[2] = lop3_and_xor(w >> 8, kMask, kMagic);
-  p[3] = lop3_and_xor(w >> 12, kMask, kMagic);
+// Word of 8 nibbles -> four f16 pairs of offset codes, one shift per word.  An
+// f16 of exponent 2^10 has unit mantissa steps, so a nibble in mantissa bits
+// 0..3 of 1024.0 reads 1024 + (nibble); one in bits 4..7 of 64.0 reads
+// 64 + (nibble).  With the nibble's sign bit flipped (q + 8 in 0..15):
+//   p[0] = (n0, n4), p[2] = (n2, n6): 1032 + q   (even inputs)
+//   p[1] = (n1, n5), p[3] = (n3, n7):   72 + q   (odd inputs)
+// All are integers below 2^11, exact in f16.
+constexpr float kOffEven = 1032.f, kOffOdd = 72.f;
+__device__ __forceinline__ void offset_word_f16(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = lop3_and_xor(w, 0x000F000Fu, 0x64086408u);    // 1024.0 = 0x6400, sign bit of the nibble at bit 3
+  p[1] = lop3_and_xor(w, 0x00F000F0u, 0x54805480u);    //   64.0 = 0x5400, sign bit of the nibble at bit 7
+  p[2] = lop3_and_xor(w8, 0x000F000Fu, 0x64086408u);
+  p[3] = lop3_and_xor(w8, 0x00F000F0u, 0x54805480u);
 }
 
-// acc += (q + 136)[16 x 128] . x[8 x 128]^T for one 16-row block (rows g and g+8 of this thread).
-// xf[j]: the activations of inputs 32c + 8j .. + 8 already in fragment order
+// acc += codes[16 x 128] . x'[8 x 128]^T for one 16-row block (rows g and g+8 of this thread), f16 operands.
+// xf[j]: the scaled f16 activations of inputs 32c + 8j .. + 8 already in fragment order
 // (x0,x4), (x1,x5), (x2,x6), (x3,x7) -- see k_int4_act_prep.
 __device__ __forceinline__ void mma_group_offset(float (&acc)[4], const uint4& wa, const uint4& wb,
                                                  const uint4 (&xf)[4]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t pa[4], pb[4];
-    offset_word(u4get(wa, j), pa);
-    offset_word(u4get(wb, j), pb);
-    mma_bf16_16816(acc, pa[0], pb[0], pa[1], pb[1], xf[j].x, xf[j].y);
-    mma_bf16_16816(acc, pa[2], pb[2], pa[3], pb[3], xf[j].z, xf[j].w);
+    offset_word_f16(u4get(wa, j), pa);
+    offset_word_f16(u4get(wb, j), pb);
+    mma_f16_16816(acc, pa[0], pb[0], pa[1], pb[1], xf[j].x, xf[j].y);
+    mma_f16_16816(acc, pa[2], pb[2], pa[3], pb[3], xf[j].z, xf[j].w);
   }
 }
 
@@ -130,34 +141,70 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4& wa, cons
 }
 
 // ---------------------------------------------------------------------------
-// Activation preparation of the offset-code product, one thread per 8 inputs:
-//   Aq: a copy of A with every 8 inputs x0..x7 stored as x0,x4,x1,x5,x2,x6,x3,x7,
+// Activation preparation of the offset-code product, one CTA per row (blockDim
+// a multiple of 32, at most 1024: a row of up to 8192 inputs in one pass):
+//   e:  the power of two that brings the row's largest |x| into [2^14, 2^15)
+//       (0 for an all-zero row; clamped to [-100, 113]).  x' = x 2^-e is exact
+//       in fp32, and its f16 rounding is exact from 2^-14 up (bf16 carries 8
+//       significant bits, f16 11), so the f16 copy differs from x' only for
+//       inputs below 2^-28 of the row's largest, by at most 2^-25;
+//   Aq: x' in f16 with every 8 inputs x0..x7 stored as x0,x4,x1,x5,x2,x6,x3,x7,
 //       the order in which the nibble pairs of a weight word come out, so the
 //       streaming kernel uses 16-byte loads as B fragments without permutes;
-//   sums[r][g]: the sum of the 128 inputs of group g of row r (each thread adds
-//       its 8 in order, then the 16 threads of a group combine by a fixed xor
-//       tree), the correction term 136 * sum(x) of the offset codes.
-__global__ void __launch_bounds__(256) k_int4_act_prep(const __nv_bfloat16* __restrict__ A, long long rows, int K,
-                                                       float* __restrict__ sums, __nv_bfloat16* __restrict__ Aq) {
+//   csum[r][g]: c = sum of off_i x'_i over 128-group g (off = 1032 for even
+//       inputs, 72 for odd ones: the offsets of offset_word_f16's codes), each
+//       thread adding its 8 in order, then a fixed xor tree over the group's 16;
+//   rscale[r] = 2^e.
+// The product of the codes with x' minus c is sum(q x') = 2^-e sum(q x).
+__global__ void __launch_bounds__(1024) k_int4_act_prep(const __nv_bfloat16* __restrict__ A, int K,
+                                                       float* __restrict__ csum, float* __restrict__ rscale,
+                                                       __half* __restrict__ Aq) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  const long long n = rows * (K / 8);
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool on = i < n;
-  uint4 u = make_uint4(0, 0, 0, 0);
-  if (on) u = reinterpret_cast<const uint4*>(A)[i];
-  float acc = 0.f;
-  acc += bf16lo(u.x); acc += bf16hi(u.x); acc += bf16lo(u.y); acc += bf16hi(u.y);
-  acc += bf16lo(u.z); acc += bf16hi(u.z); acc += bf16lo(u.w); acc += bf16hi(u.w);
+  __shared__ float s_m[32];
+  const long long row = blockIdx.x;
+  const int nv = K / 8;   // 16 per 128-group; a pass covers whole groups
+  const uint4* src = reinterpret_cast<const uint4*>(A + row * K);
+  // the first pass's inputs stay in registers for the conversion (the whole row when nv <= blockDim)
+  const uint4 u0 = (int)threadIdx.x < nv ? src[threadIdx.x] : make_uint4(0, 0, 0, 0);
+  float m = 0.f;
+  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    const uint4 u = v == (int)threadIdx.x ? u0 : src[v];
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.x)), fabsf(bf16hi(u.x))), fmaxf(fabsf(bf16lo(u.y)), fabsf(bf16hi(u.y)))));
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16lo(u.z)), fabsf(bf16hi(u.z))), fmaxf(fabsf(bf16lo(u.w)), fabsf(bf16hi(u.w)))));
+  }
 #pragma unroll
-  for (int o = 1; o < 16; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (on) {
-    uint4 q;
-    q.x = prmt(u.x, u.z, 0x5410);
-    q.y = prmt(u.x, u.z, 0x7632);
-    q.z = prmt(u.y, u.w, 0x5410);
-    q.w = prmt(u.y, u.w, 0x7632);
-    reinterpret_cast<uint4*>(Aq)[i] = q;
-    if ((i & 15) == 0) sums[i >> 4] = acc;
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane_id() == 0) s_m[warp_id()] = m;
+  __syncthreads();
+  m = s_m[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, s_m[w]);
+  const int eb = (int)((__float_as_uint(m) >> 23) & 0xFFu);   // biased exponent of the row's largest |x|
+  const int e = m == 0.f ? 0 : (eb == 0 ? -100 : max(-100, min(113, eb - 127 - 14)));
+  const float down = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, a normal float for e in [-100, 113]
+  if (threadIdx.x == 0) rscale[row] = __uint_as_float((uint32_t)(127 + e) << 23);
+  uint4* dst = reinterpret_cast<uint4*>(Aq + row * K);
+  for (int base = 0; base < nv; base += blockDim.x) {   // every thread takes part in each pass's xor tree
+    const int v = base + threadIdx.x;
+    const bool on = v < nv;
+    const uint4 u = base == 0 ? u0 : (on ? src[v] : make_uint4(0, 0, 0, 0));
+    const float x[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                        bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+    __half h[8];
+    float c = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      h[j] = __float2half_rn(x[j] * down);
+      c = fmaf((j & 1) ? kOffOdd : kOffEven, __half2float(h[j]), c);
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (on) {
+      auto pack = [](__half lo, __half hi) {
+        return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+      };
+      dst[v] = make_uint4(pack(h[0], h[4]), pack(h[1], h[5]), pack(h[2], h[6]), pack(h[3], h[7]));
+      if ((v & 15) == 0) csum[row * (K / 128) + (v >> 4)] = c;
+    }
   }
 }
 
@@ -174,14 +221,15 @@ constexpr int kI4Stages = 3;
 constexpr int kI4SlabBytes = 32 * 128;
 constexpr int kI4Smem = kI4Warps * kI4Stages * kI4SlabBytes;
 
-// OFFS: multiply the offset codes q + 136 and subtract 136 * xsum[row][group]
-// (the activation group sums) once per group, instead of one packed
-// subtraction per pair of weights; p.act is then the fragment-ordered copy
-// written by k_int4_act_prep.
+// OFFS: multiply the f16 offset codes by the scaled f16 activations and remove
+// the offsets' share c once per group, instead of one packed subtraction per
+// pair of weights; p.act is then the fragment-ordered copy written by
+// k_int4_act_prep, xcs[row][group] the offsets' share c of each group and
+// xrs[row] = 2^e the row's scale, applied once to the finished sums.
 template <bool GLU, int ACT, bool OFFS, bool SPLIT>
 __global__ void __launch_bounds__(kI4Warps * 32, 1)
     k_int4_stream(const __grid_constant__ CUtensorMap tmW, const Int4Params p, unsigned long long wait_limit_ns,
-                  const float* __restrict__ xsum) {
+                  const float* __restrict__ xcs, const float* __restrict__ xrs) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ int s_prefix[kMaxGroupsSmem + 1];
@@ -291,7 +339,8 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   const __nv_bfloat16* xrow = nullptr;   // this thread's activation row (token n0 + gq), inputs c*32 ..
   const __nv_bfloat16* sA = nullptr;     // scales of weight row ra + gq (row + 8: + 8 * ngroups_k)
   const __nv_bfloat16* sB = nullptr;     // scales of weight row rb + gq
-  const float* xs0 = nullptr;            // group sums of tokens n0 + 2c, n0 + 2c + 1
+  const float* xs0 = nullptr;            // offsets' shares c of tokens n0 + 2c, n0 + 2c + 1
+  float rs0 = 1.f, rs1 = 1.f;            // their row scales 2^e
   bool tok_ok = false, ok0 = false, ok1 = false;
   const long long s8 = 8ll * ngroups_k;
   int c_task = tfirst, c_slab = 0, c_st = 0;
@@ -312,7 +361,11 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
       sB = p.ws + (long long)(rb + gq) * ngroups_k;
       ok0 = cur.n0 + 2 * c < cur.n_rows;
       ok1 = cur.n0 + 2 * c + 1 < cur.n_rows;
-      if (OFFS) xs0 = xsum + (cur.row0 + (ok0 ? cur.n0 + 2 * c : 0)) * (long long)ngroups_k;
+      if (OFFS) {
+        xs0 = xcs + (cur.row0 + (ok0 ? cur.n0 + 2 * c : 0)) * (long long)ngroups_k;
+        rs0 = ok0 ? xrs[cur.row0 + cur.n0 + 2 * c] : 0.f;
+        rs1 = ok1 ? xrs[cur.row0 + cur.n0 + 2 * c + 1] : 0.f;
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) { tA[i] = 0.f; tB[i] = 0.f; }
     }
@@ -367,20 +420,21 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
       if (OFFS) {
         mma_group_offset(pa, a0, a1, xv[gi]);
         mma_group_offset(pb, b0, b1, xv[gi]);
-        // D columns are tokens n0 + 2c and n0 + 2c + 1: remove 136 * (their group sums)
+        // D columns are tokens n0 + 2c and n0 + 2c + 1: remove the offsets' share c of each, then the weight
+        // row's group scale
         const float x0 = xsv[gi][0], x1 = xsv[gi][1];
-        pa[0] = fmaf(-136.f, x0, pa[0]); pa[1] = fmaf(-136.f, x1, pa[1]);
-        pa[2] = fmaf(-136.f, x0, pa[2]); pa[3] = fmaf(-136.f, x1, pa[3]);
-        pb[0] = fmaf(-136.f, x0, pb[0]); pb[1] = fmaf(-136.f, x1, pb[1]);
-        pb[2] = fmaf(-136.f, x0, pb[2]); pb[3] = fmaf(-136.f, x1, pb[3]);
+        tA[0] = fmaf(pa[0] - x0, sc[0][gi], tA[0]); tA[1] = fmaf(pa[1] - x1, sc[0][gi], tA[1]);
+        tA[2] = fmaf(pa[2] - x0, sc[1][gi], tA[2]); tA[3] = fmaf(pa[3] - x1, sc[1][gi], tA[3]);
+        tB[0] = fmaf(pb[0] - x0, sc[2][gi], tB[0]); tB[1] = fmaf(pb[1] - x1, sc[2][gi], tB[1]);
+        tB[2] = fmaf(pb[2] - x0, sc[3][gi], tB[2]); tB[3] = fmaf(pb[3] - x1, sc[3][gi], tB[3]);
       } else {
         mma_group(pa, a0, a1, xv[gi]);
         mma_group(pb, b0, b1, xv[gi]);
+        tA[0] = fmaf(pa[0], sc[0][gi], tA[0]); tA[1] = fmaf(pa[1], sc[0][gi], tA[1]);
+        tA[2] = fmaf(pa[2], sc[1][gi], tA[2]); tA[3] = fmaf(pa[3], sc[1][gi], tA[3]);
+        tB[0] = fmaf(pb[0], sc[2][gi], tB[0]); tB[1] = fmaf(pb[1], sc[2][gi], tB[1]);
+        tB[2] = fmaf(pb[2], sc[3][gi], tB[2]); tB[3] = fmaf(pb[3], sc[3][gi], tB[3]);
       }
-      tA[0] = fmaf(pa[0], sc[0][gi], tA[0]); tA[1] = fmaf(pa[1], sc[0][gi], tA[1]);
-      tA[2] = fmaf(pa[2], sc[1][gi], tA[2]); tA[3] = fmaf(pa[3], sc[1][gi], tA[3]);
-      tB[0] = fmaf(pb[0], sc[2][gi], tB[0]); tB[1] = fmaf(pb[1], sc[2][gi], tB[1]);
-      tB[2] = fmaf(pb[2], sc[3][gi], tB[2]); tB[3] = fmaf(pb[3], sc[3][gi], tB[3]);
     }
     __syncwarp();
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slab reads done before TMA reuses it
@@ -389,6 +443,13 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
     refill();
     if (c_slab == cur.se - 1) {
       // D fragments: (m = gq, n = 2c, 2c+1) in [0],[1]; (m = gq + 8, same n) in [2],[3]
+      if (OFFS) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // back from the scaled activations: the token's 2^e (exact)
+          tA[i] *= (i & 1) ? rs1 : rs0;
+          tB[i] *= (i & 1) ? rs1 : rs0;
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int m = gq + (i >= 2 ? 8 : 0);
@@ -434,9 +495,9 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
 // would read and dequantise every weight eight times; here a task is one block
 // of 32 weight rows over 32 rows (four 8-row chunks), its reduction split into
 // p.ksplit slab ranges: a 64-row batch reads and dequantises every weight
-// twice, and each dequantised fragment feeds the MMAs of four chunks.  Offset codes
-// (q + 136, the correction 136 * sum(x) per 128-group) as in k_int4_stream's
-// OFFS mode; fp32 partials [ksplit][R][W] in its split layout, which
+// twice, and each dequantised fragment feeds the MMAs of four chunks.  f16 offset
+// codes and scaled activations, with the group terms (c, 2^e), as in
+// k_int4_stream's OFFS mode; fp32 partials [ksplit][R][W] in its split layout, which
 // k_int4_splitk_reduce adds in order.  Eight warps per CTA, each with a ring of
 // kI4DStages slabs.
 constexpr int kI4DWarps = 8;
@@ -447,7 +508,7 @@ constexpr int kI4DChunks = 4;            // 8-row chunks per task
 template <bool GLU>
 __global__ void __launch_bounds__(kI4DWarps * 32, 1)
     k_int4_dense(const __grid_constant__ CUtensorMap tmW, const Int4Params p, unsigned long long wait_limit_ns,
-                 const float* __restrict__ xsum) {
+                 const float* __restrict__ xcs, const float* __restrict__ xrs) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ __align__(8) uint64_t s_bar[kI4DWarps][kI4DStages];
@@ -548,34 +609,35 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t qa0[4], qa1[4], qb0[4], qb1[4];
-          offset_word(u4get(a0, j), qa0);
-          offset_word(u4get(a1, j), qa1);
-          offset_word(u4get(b0, j), qb0);
-          offset_word(u4get(b1, j), qb1);
+          offset_word_f16(u4get(a0, j), qa0);
+          offset_word_f16(u4get(a1, j), qa1);
+          offset_word_f16(u4get(b0, j), qb0);
+          offset_word_f16(u4get(b1, j), qb1);
 #pragma unroll
           for (int ch = 0; ch < kI4DChunks; ++ch) {
-            mma_bf16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch][j].x, xf[ch][j].y);
-            mma_bf16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch][j].z, xf[ch][j].w);
-            mma_bf16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch][j].x, xf[ch][j].y);
-            mma_bf16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch][j].z, xf[ch][j].w);
+            mma_f16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch][j].x, xf[ch][j].y);
+            mma_f16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch][j].z, xf[ch][j].w);
+            mma_f16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch][j].x, xf[ch][j].y);
+            mma_f16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch][j].z, xf[ch][j].w);
           }
         }
-        // offset correction (columns = rows 8 ch + 2c, 8 ch + 2c + 1) and group scales (weight rows gq, gq + 8)
+        // offsets' share (columns = rows 8 ch + 2c, 8 ch + 2c + 1), then the weight rows' group scales (rows gq,
+        // gq + 8)
         const float scA0 = __bfloat162float(sA[kg]), scA1 = __bfloat162float(sA[s8 + kg]);
         const float scB0 = __bfloat162float(sB[kg]), scB1 = __bfloat162float(sB[s8 + kg]);
 #pragma unroll
         for (int ch = 0; ch < kI4DChunks; ++ch) {
           const int n0 = r0 + 8 * ch + 2 * c;
-          const float x0 = n0 < R ? xsum[(long long)n0 * ngk + kg] : 0.f;
-          const float x1 = n0 + 1 < R ? xsum[(long long)(n0 + 1) * ngk + kg] : 0.f;
-          tA[ch][0] = fmaf(fmaf(-136.f, x0, pA[ch][0]), scA0, tA[ch][0]);
-          tA[ch][1] = fmaf(fmaf(-136.f, x1, pA[ch][1]), scA0, tA[ch][1]);
-          tA[ch][2] = fmaf(fmaf(-136.f, x0, pA[ch][2]), scA1, tA[ch][2]);
-          tA[ch][3] = fmaf(fmaf(-136.f, x1, pA[ch][3]), scA1, tA[ch][3]);
-          tB[ch][0] = fmaf(fmaf(-136.f, x0, pB[ch][0]), scB0, tB[ch][0]);
-          tB[ch][1] = fmaf(fmaf(-136.f, x1, pB[ch][1]), scB0, tB[ch][1]);
-          tB[ch][2] = fmaf(fmaf(-136.f, x0, pB[ch][2]), scB1, tB[ch][2]);
-          tB[ch][3] = fmaf(fmaf(-136.f, x1, pB[ch][3]), scB1, tB[ch][3]);
+          const float x0 = n0 < R ? xcs[(long long)n0 * ngk + kg] : 0.f;
+          const float x1 = n0 + 1 < R ? xcs[(long long)(n0 + 1) * ngk + kg] : 0.f;
+          tA[ch][0] = fmaf(pA[ch][0] - x0, scA0, tA[ch][0]);
+          tA[ch][1] = fmaf(pA[ch][1] - x1, scA0, tA[ch][1]);
+          tA[ch][2] = fmaf(pA[ch][2] - x0, scA1, tA[ch][2]);
+          tA[ch][3] = fmaf(pA[ch][3] - x1, scA1, tA[ch][3]);
+          tB[ch][0] = fmaf(pB[ch][0] - x0, scB0, tB[ch][0]);
+          tB[ch][1] = fmaf(pB[ch][1] - x1, scB0, tB[ch][1]);
+          tB[ch][2] = fmaf(pB[ch][2] - x0, scB1, tB[ch][2]);
+          tB[ch][3] = fmaf(pB[ch][3] - x1, scB1, tB[ch][3]);
         }
       }
       __syncwarp();
@@ -595,12 +657,13 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
         const int n = r0 + 8 * ch + 2 * c + (i & 1);
         if (n < R) {
           float* prow = p.part + ((long long)sp * R + n) * W + o0;
+          const float rs = xrs[n];   // back from the scaled activations: the row's 2^e (exact)
           if (GLU) {
-            prow[m] = tA[ch][i];
-            prow[p.N + m] = tB[ch][i];
+            prow[m] = tA[ch][i] * rs;
+            prow[p.N + m] = tB[ch][i] * rs;
           } else {
-            prow[m] = tA[ch][i];
-            prow[m + 16] = tB[ch][i];
+            prow[m] = tA[ch][i] * rs;
+            prow[m + 16] = tB[ch][i] * rs;
           }
         }
       }

@@ -137,7 +137,7 @@ static int router_splits(const moe_shape* s, int* k_per_split) {
 // ------------------------------------------------------------------ workspace layout
 
 struct Workspace {
-  size_t part, wsplit, wnorm, xsum, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
+  size_t part, wsplit, wnorm, xcs, xrs, xq, i4part, cnt, psum, idx, w, counts, fP, slot, drop, kept, offs, xperm, h, yperm, hs, ys, shtab;
   size_t cidx, ncand, zmax, snc, zex, ecount, elist, xnorm2;   // certified selection over the screening logits
   size_t total;
 };
@@ -164,7 +164,8 @@ static Workspace ws_layout(const moe_shape* s) {
   L.wnorm = take((size_t)s->E * 4);
   const long long xs_rows = std::max<long long>(grouped_rows(s), s->T);
   const int xs_cols = std::max(s->d, std::max(s->H, s->H_s));
-  L.xsum = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * (xs_cols / 128) * 4 : 16);
+  L.xcs = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * (xs_cols / 128) * 4 : 16);
+  L.xrs = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * 4 : 16);
   L.xq = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * xs_cols * 2 : 16);
   L.i4part = take(i4part_floats(s) * 4 + 16);
   L.cnt = take((size_t)nchunks * s->E * 4);
@@ -232,7 +233,7 @@ static int make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t
 template <int MODE, int BN, int CG>
 static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, long long ub_mtiles,
                          cudaStream_t st) {
-  using Cfg = GemmCfg<BN, CG>;
+  using Cfg = GemmCfg<BN, CG, MODE == kModeScreen ? 2 : 1>;
   constexpr int OUTN = (MODE == kModeSwiGLU || MODE == kModeGeGLU) ? BN / 2 : BN;
   // the shared-memory opt-in is set once per device for each instantiation
   static std::atomic<unsigned long long> done_mask{0};
@@ -265,7 +266,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 // CTA pairs (M = 256 tiles) for the bf16 expert GEMMs when the groups are large enough
 // to fill them: on average at least 192 rows per group.
 static bool use_pair_gemm(int mode, int BN, long long R, int n_groups, bool allow_pair) {
-  return allow_pair && mode != kModeF32 && BN == 256 && R >= 192ll * n_groups;
+  return allow_pair && mode != kModeScreen && BN == 256 && R >= 192ll * n_groups;
 }
 
 // out[R, N] = epilogue(A[R, K] . B_g^T) over groups.  B is [n_groups, b_rows, K].
@@ -290,25 +291,25 @@ static int pick_bn(bool glu, int N, long long mtiles) {
 
 // Mode-specific inputs of grouped_gemm beyond the operands.
 struct GemmExtras {
-  int a_kwrap = 0;                   // router: A repeats every a_kwrap reduction columns
-  const float* bias = nullptr;       // router: per-expert logit bias
+  const float* bias = nullptr;       // router screen: per-expert logit bias
 };
 
 static int grouped_gemm(int mode, const void* A, long long R, int K, const void* B, int n_groups, int b_rows,
                         int up_row0, int N, const int32_t* gstart, const int32_t* grows, void* out,
                         cudaStream_t st, bool allow_pair, const GemmExtras& ex = GemmExtras{}) {
-  const int a_kwrap = ex.a_kwrap;
   if (R == 0) return MOE_OK;
   const bool glu = mode == kModeSwiGLU || mode == kModeGeGLU;
   const long long ub_m = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
-  // router logits: one column tile as wide as the expert count (fewer A re-reads)
-  const bool router = mode == kModeF32;
+  // router screen: one column tile as wide as the expert count (fewer A re-reads); CTA pairs (256-row tiles,
+  // half the B tiles per CTA) once the batch fills a wave of single-CTA tiles
+  const bool router = mode == kModeScreen;
   const int BN = router ? (N <= 64 ? 64 : N <= 128 ? 128 : N <= 192 ? 192 : 256) : pick_bn(glu, N, ub_m);
-  const bool pair = use_pair_gemm(mode, BN, R, n_groups, allow_pair);
+  const bool pair = router ? (allow_pair && R >= (long long)kBM * num_sms())
+                           : use_pair_gemm(mode, BN, R, n_groups, allow_pair);
   const int box_rows = (glu || pair) ? BN / 2 : BN;
   CUtensorMap ta, tb;
-  cuuint64_t da[2] = {(cuuint64_t)(a_kwrap > 0 ? a_kwrap : K), (cuuint64_t)R};
-  cuuint64_t db[3] = {(cuuint64_t)K, (cuuint64_t)b_rows, (cuuint64_t)n_groups};
+  cuuint64_t da[2] = {(cuuint64_t)K, (cuuint64_t)R};
+  cuuint64_t db[3] = {(cuuint64_t)(router ? 2 * K : K), (cuuint64_t)b_rows, (cuuint64_t)n_groups};
   int rc = make_map(&ta, A, 2, da, kBM);
   if (rc) return rc;
   rc = make_map(&tb, B, 3, db, box_rows);
@@ -324,7 +325,6 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ldo = N;
   p.wait_limit_ns = g_wait_limit_ns.load();
-  p.a_kwrap = a_kwrap;
   p.out_f32 = reinterpret_cast<float*>(out);
   p.bias = ex.bias;
   const long long ub = grows ? (R / kBM + n_groups) : cdiv(R, kBM);
@@ -333,6 +333,10 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
     if (mode == kModePlain) return launch_gemm_t<kModePlain, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeSwiGLU) return launch_gemm_t<kModeSwiGLU, 256, 2>(ta, tb, p, ub2, st);
     if (mode == kModeGeGLU) return launch_gemm_t<kModeGeGLU, 256, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeScreen && BN == 256) return launch_gemm_t<kModeScreen, 256, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeScreen && BN == 192) return launch_gemm_t<kModeScreen, 192, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeScreen && BN == 128) return launch_gemm_t<kModeScreen, 128, 2>(ta, tb, p, ub2, st);
+    if (mode == kModeScreen && BN == 64) return launch_gemm_t<kModeScreen, 64, 2>(ta, tb, p, ub2, st);
     return MOE_UNSUPPORTED_SHAPE;
   }
 #define MOE_GEMM_CASE(M_, BN_) \
@@ -340,8 +344,8 @@ static int grouped_gemm(int mode, const void* A, long long R, int K, const void*
   MOE_GEMM_CASE(kModePlain, 256) MOE_GEMM_CASE(kModePlain, 128) MOE_GEMM_CASE(kModePlain, 64)
   MOE_GEMM_CASE(kModeSwiGLU, 256) MOE_GEMM_CASE(kModeSwiGLU, 128) MOE_GEMM_CASE(kModeSwiGLU, 64)
   MOE_GEMM_CASE(kModeGeGLU, 256) MOE_GEMM_CASE(kModeGeGLU, 128) MOE_GEMM_CASE(kModeGeGLU, 64)
-  MOE_GEMM_CASE(kModeF32, 256) MOE_GEMM_CASE(kModeF32, 192) MOE_GEMM_CASE(kModeF32, 128)
-  MOE_GEMM_CASE(kModeF32, 64)
+  MOE_GEMM_CASE(kModeScreen, 256) MOE_GEMM_CASE(kModeScreen, 192) MOE_GEMM_CASE(kModeScreen, 128)
+  MOE_GEMM_CASE(kModeScreen, 64)
 #undef MOE_GEMM_CASE
   return MOE_UNSUPPORTED_SHAPE;
 }
@@ -360,10 +364,9 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   const bool small = s->T <= 2048;
   // the certifying recompute holds the token's inputs in registers when d <= 1024
   const bool xreg = refine.x != nullptr && refine.d <= 1024;
-  // warps per CTA: decode batches (T <= 256, final logits) two tokens per warp, a 32-token chunk per CTA with
-  // the chunk tables formed in the kernel; other small batches 4 tokens per CTA (tables by k_chunk_stats);
-  // large batches 8 warps per chunk
-  const int nw = (s->T <= 256 && refine.x == nullptr) ? 16 : (small ? 4 : 8);
+  // warps per CTA: small batches 4 tokens per CTA, so that the tokens spread over the SMs (tables by
+  // k_chunk_stats); large batches 8 warps per 32-token chunk with the chunk tables formed in the kernel
+  const int nw = small ? 4 : 8;
 #define MOE_TOPK_CASE(N_, NW_, XR_, ST_)                                                                          \
   if (epl <= N_ && nw == NW_ && xreg == XR_) {                                                                    \
     const size_t smem = ST_ ? (size_t)2 * NW_ * s->E * sizeof(float) : 0;                                         \
@@ -393,7 +396,6 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
   MOE_TOPK_CASE(6, NW_, XR_, ST_) MOE_TOPK_CASE(8, NW_, XR_, ST_) MOE_TOPK_CASE(12, NW_, XR_, ST_)                \
   MOE_TOPK_CASE(16, NW_, XR_, ST_)
   MOE_TOPK_EPL(8, false, true) MOE_TOPK_EPL(8, true, true) MOE_TOPK_EPL(4, false, false) MOE_TOPK_EPL(4, true, false)
-  MOE_TOPK_EPL(16, false, true)
 #undef MOE_TOPK_EPL
 #undef MOE_TOPK_CASE
   return MOE_UNSUPPORTED_SHAPE;
@@ -494,10 +496,12 @@ static int launch_fused(const moe_shape* s, int hidden, long long R, const void*
   return MOE_UNSUPPORTED_SHAPE;
 }
 
-// Optional scratch for the offset-code kernel: xsum [R, K/128] fp32 (activation group sums) and
-// xq [R, K] bf16 (the fragment-ordered copy of A).  Without it the plain-code kernel runs.
+// Optional scratch for the offset-code kernel, written by k_int4_act_prep: xcs [R, K/128] (the offsets' share
+// of each group), xrs [R] (row scales 2^e) and xq [R, K] f16 (the scaled, fragment-ordered copy of A).
+// Without it the exact-code kernel runs.
 struct Int4Scratch {
-  float* xsum;
+  float* xcs;
+  float* xrs;
   void* xq;
   float* part = nullptr;        // split-reduction partials (dense groups with few tasks), or none
   size_t part_floats = 0;
@@ -505,8 +509,9 @@ struct Int4Scratch {
 
 static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const void* wq, const void* wsc,
                      int n_groups, int b_rows, int up_row0, int N, const int32_t* gstart, const int32_t* grows,
-                     void* out, cudaStream_t st, Int4Scratch scr = Int4Scratch{nullptr, nullptr}) {
-  float* xsum = scr.xq != nullptr ? scr.xsum : nullptr;
+                     void* out, cudaStream_t st, Int4Scratch scr = Int4Scratch{nullptr, nullptr, nullptr}) {
+  float* xcs = scr.xq != nullptr ? scr.xcs : nullptr;
+  float* xrs = scr.xrs;
   if (R == 0) return MOE_OK;
   Int4Params p;
   p.wq = reinterpret_cast<const uint8_t*>(wq);
@@ -569,14 +574,14 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
       MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_dense<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4DSmem));
       done.fetch_or(bit);
     }
-    if (xsum != nullptr) {
-      MOE_LAUNCH((k_int4_act_prep), (unsigned)cdiv(R * (K / 8), 256), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(A), R,
-                                                                         K, xsum,
-                                                                         reinterpret_cast<__nv_bfloat16*>(scr.xq));
+    if (xcs != nullptr) {
+      const int pt = (int)std::min<long long>(1024, std::max<long long>(64, cdiv(K / 8, 32) * 32));
+      MOE_LAUNCH((k_int4_act_prep), (unsigned)R, pt, 0, st, reinterpret_cast<const __nv_bfloat16*>(A), K, xcs, xrs,
+                 reinterpret_cast<__half*>(scr.xq));
       MOE_LAUNCH_CHECK();
-      p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);
+      p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);   // f16 bytes: loaded as raw fragments
     }
-    if (grows == nullptr && xsum != nullptr && scr.part != nullptr && R <= 256) {
+    if (grows == nullptr && xcs != nullptr && scr.part != nullptr && R <= 256) {
       // one dense group of a small batch (the shared expert of a decode batch): tasks of 32 weight rows over
       // 32 rows, each weight dequantised once per 32 rows; the reduction split so that every warp has work
       const long long base = (long long)(N / (glu ? 16 : 32)) * cdiv(R, 32);
@@ -588,8 +593,8 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
         p.part = scr.part;
         const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), cdiv(base * ks, kI4DWarps)));
         const unsigned long long lim = g_wait_limit_ns.load();
-        if (glu) MOE_LAUNCH((k_int4_dense<true>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xsum);
-        else MOE_LAUNCH((k_int4_dense<false>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xsum);
+        if (glu) MOE_LAUNCH((k_int4_dense<true>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xcs, xrs);
+        else MOE_LAUNCH((k_int4_dense<false>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xcs, xrs);
         MOE_LAUNCH_CHECK();
         const unsigned blocks = (unsigned)cdiv(R * N, 256);
         __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
@@ -607,12 +612,12 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
     const unsigned long long lim = g_wait_limit_ns.load();
     const int nt = kI4Warps * 32;
 #define MOE_I4_LAUNCH(G_, A_, O_, S_) \
-  MOE_LAUNCH((k_int4_stream<G_, A_, O_, S_>), grid, nt, kI4Smem, st, tm, p, lim, xsum)
-    if (xsum != nullptr && p.ksplit > 1) {
+  MOE_LAUNCH((k_int4_stream<G_, A_, O_, S_>), grid, nt, kI4Smem, st, tm, p, lim, xcs, xrs)
+    if (xcs != nullptr && p.ksplit > 1) {
       if (!glu) MOE_I4_LAUNCH(false, kModePlain, true, true);
       else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true, true);
       else MOE_I4_LAUNCH(true, kModeGeGLU, true, true);
-    } else if (xsum != nullptr) {
+    } else if (xcs != nullptr) {
       if (!glu) MOE_I4_LAUNCH(false, kModePlain, true, false);
       else if (act == MOE_ACT_SWIGLU) MOE_I4_LAUNCH(true, kModeSwiGLU, true, false);
       else MOE_I4_LAUNCH(true, kModeGeGLU, true, false);
@@ -642,7 +647,7 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
 static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const void* A, const int32_t* gstart,
                            const int32_t* grows, int n_groups, const void* w13, const void* s13, const void* w2,
                            const void* s2, void* h, void* y, cudaStream_t st,
-                           Int4Scratch scr = Int4Scratch{nullptr, nullptr}) {
+                           Int4Scratch scr = Int4Scratch{nullptr, nullptr, nullptr}) {
   int rc;
   if (s->wfmt == MOE_WFMT_INT4_G128) {
     rc = int4_gemm(true, s->act, A, R, s->d, w13, s13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st,
@@ -772,9 +777,9 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
                select ? reinterpret_cast<const __nv_bfloat16*>(x) : nullptr, xnorm2, (int)s->T);
     MOE_LAUNCH_CHECK();
     GemmExtras ex;
-    ex.a_kwrap = s->d;
     ex.bias = bias;
-    rc = grouped_gemm(kModeF32, x, s->T, 2 * s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st, false, ex);
+    rc = grouped_gemm(kModeScreen, x, s->T, s->d, wsplit, 1, s->E, 0, s->E, nullptr, nullptr, part, st,
+                      !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM), ex);
     if (rc) return rc;
     if (select) {
       SelectArgs sa{part, xnorm2, reinterpret_cast<const __nv_bfloat16*>(x), wnorm, gamma, (int)s->T, s->d, s->E, s->k,
@@ -789,8 +794,23 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       else MOE_LAUNCH((k_router_select<8>), nch, 256, 0, st, sa);
       MOE_LAUNCH_CHECK();
       float* zex = reinterpret_cast<float*>(ws + L.zex);
-      MOE_LAUNCH((k_router_recompute), (unsigned)(2 * num_sms()), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(x),
-                 w_router, bias, ecount, sa.elist, zex, (int)s->T, s->d, s->E);
+      // 16-byte input slices per lane (d <= kSelMaxD: at most 8); entries per batch and resident CTAs chosen so
+      // that the input loads of a batch and the W_r slices fit the registers
+      const int vpl = (int)cdiv(s->d / 8, 32);
+#define MOE_RECOMP(V_, N_, M_)                                                                                \
+  MOE_LAUNCH((k_router_recompute<V_, N_, M_>), (unsigned)(M_ * num_sms()), 256, 0, st,                        \
+             reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, ecount, sa.elist, zex, (int)s->T, s->d, s->E)
+      switch (vpl) {
+        case 1: MOE_RECOMP(1, 8, 3); break;
+        case 2: MOE_RECOMP(2, 4, 3); break;
+        case 3: MOE_RECOMP(3, 4, 2); break;
+        case 4: MOE_RECOMP(4, 4, 2); break;
+        case 5: MOE_RECOMP(5, 3, 2); break;
+        case 6: MOE_RECOMP(6, 2, 2); break;
+        case 7: MOE_RECOMP(7, 1, 2); break;
+        default: MOE_RECOMP(8, 1, 2); break;
+      }
+#undef MOE_RECOMP
       MOE_LAUNCH_CHECK();
       const unsigned nfin = (unsigned)cdiv(s->T, 32);
 #define MOE_FINISH(N_)                                                                                        \
@@ -1022,9 +1042,9 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
                       aux);
   if (rc) return rc;
   const Int4Scratch scr = s->wfmt == MOE_WFMT_INT4_G128
-                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xsum), ws + L.xq,
-                                            reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
-                              : Int4Scratch{nullptr, nullptr};
+                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xcs), reinterpret_cast<float*>(ws + L.xrs),
+                                            ws + L.xq, reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
+                              : Int4Scratch{nullptr, nullptr, nullptr};
   rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
   if (rc) return rc;
   void* ys = nullptr;

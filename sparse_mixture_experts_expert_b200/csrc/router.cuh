@@ -115,7 +115,8 @@ __global__ void __launch_bounds__(128) k_router_logits(const __nv_bfloat16* __re
 //  * two-term bf16 split W ~ hi + lo (hi = bf16(w), lo = bf16(w - hi): 16
 //    significand bits, |w - hi - lo| <= 2^-16 |w|), written as one [E, 2d] bf16
 //    operand [hi | lo]; x is bf16, so every product x * part is exact in fp32
-//    and the screening logits are [x | x] [hi | lo]^T;
+//    and the screening logits x hi^T + x lo^T are one fp32 reduction of 2d
+//    products (the screening GEMM accumulates both terms in one accumulator);
 //  * the row norm ||W_r[e]||_2 for the screening error bound.
 //  * with x set (the certified selection path), blocks past the weight rows
 //    also compute xnorm2[t] = sum_i x[t,i]^2, one warp per token, every load of
@@ -562,21 +563,23 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
 // Certified selection over tensor-core screening logits, in three kernels that
 // keep the exact fp32 work proportional to the candidates (about k + 0.1 per
 // token) rather than to E:
-//   k_router_select    one warp per token (lane l: experts l, l+32, ...): the
-//                      k-th largest screening logit, ||x_t|| for the error
-//                      bound, the candidates (z >= k-th - 2 bound) in expert
-//                      order, and the sum of exp(z - max) over the others;
-//                      each candidate is listed under its expert;
+//   k_router_select    one warp per token (lane l: experts l, l+32, ...): a
+//                      lower bound L of the k-th largest screening logit,
+//                      ||x_t|| for the error bound, the candidates
+//                      (z >= L - 2 bound) in expert order, and the sum of
+//                      exp(z - max) over the others; each candidate is listed
+//                      under its expert;
 //   k_router_recompute exact fp32 logits of the listed (token, expert) pairs,
 //                      the flat list split evenly over the CTAs, W_r[e] in
 //                      shared memory;
 //   k_router_finish    top k among each token's exact candidates, softmax
 //                      (exact candidates + screening rest), gates, picks per
 //                      (expert, chunk).
-// The decision equals the top k of exact fp32 logits: every expert outside
-// the candidates is below the k-th exact logit by the screening bound.
+// The decision equals the top k of exact fp32 logits: an expert outside the
+// candidates has z < L - 2 bound <= (k-th screening value) - 2 bound, so its
+// exact logit is below those of the k experts whose screening value reaches
+// the k-th.
 constexpr int kSelMaxD = 2048;      // largest input width of the selection path
-constexpr int kRecompBatch = 8;     // list entries per warp in flight
 
 struct SelectArgs {
   const float* zs;       // [T, E] screening logits (bias included)
@@ -598,11 +601,11 @@ struct SelectArgs {
 // position in its expert's list in two steps: a shared-memory counter per
 // expert inside the chunk, then one global reservation per (chunk, expert) for
 // the chunk's whole run.  The tokens of a warp are loaded together (screening
-// row and inputs), then processed in order.  A token keeps its first
+// row and inputs), then processed side by side.  A token keeps its first
 // kSelMaxCand candidates; with more, the finishing kernel recomputes every
 // expert for it.
 template <int EPL>
-__global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
+__global__ void __launch_bounds__(256, EPL <= 6 ? 3 : 2) k_router_select(const SelectArgs a) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   constexpr int TPW = kChunk / 8;
   __shared__ int s_cnt[kMaxRouterE];
@@ -635,6 +638,45 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
     }
     x2s[tt] = on ? a.xnorm2[t] : 0.f;
   }
+  // A lower bound of each token's k-th largest screening value, the warp's tokens side by side: the k-th
+  // largest of the 32 lane maxima (k lanes hold a maximum >= it, so at least k entries are >= it).  Rounds of
+  // (warp maximum of the lane maxima, how many lanes hold it); the bound is the maximum of the round at which
+  // the running count reaches k, and each earlier round retires its lanes.  Round 0's maximum is the token's
+  // largest screening value.  Thresholding at this bound lists every expert the exact k-th value would, and
+  // more only when two of a token's k largest share a lane.
+  float lm[TPW], kth[TPW], m_s[TPW];
+  int need[TPW];
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt) {
+    float v = z[tt][0];
+#pragma unroll
+    for (int i = 1; i < EPL; ++i) v = fmaxf(v, z[tt][i]);
+    lm[tt] = v;
+    need[tt] = a.k;
+    kth[tt] = -INFINITY;
+  }
+  for (int r = 0; r < a.k; ++r) {
+    bool open = false;
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      float m;
+      asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(lm[tt]));
+      if (r == 0) m_s[tt] = m;
+      const bool at = lm[tt] == m;
+      const int c = __popc(__ballot_sync(0xffffffffu, at));
+      if (need[tt] > 0) {
+        if (c >= need[tt]) {
+          kth[tt] = m;
+          need[tt] = 0;
+        } else {
+          need[tt] -= c;
+          if (at) lm[tt] = -INFINITY;
+        }
+      }
+      open |= need[tt] > 0;
+    }
+    if (!open) break;   // warp-uniform
+  }
 #pragma unroll
   for (int tt = 0; tt < TPW; ++tt) {
     const int tl = warp * TPW + tt;
@@ -643,17 +685,8 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
       if (lane == 0) s_nk[tl] = 0;
       continue;
     }
-    const float x2 = x2s[tt];
-    const float kth = warp_kth<EPL>(z[tt], a.E, a.k);
-    float m_s;
-    {
-      float lm = z[tt][0];
-#pragma unroll
-      for (int i = 1; i < EPL; ++i) lm = fmaxf(lm, z[tt][i]);
-      asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m_s) : "f"(lm));
-    }
-    const float bound = a.gamma * sqrtf(x2) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth) + 1.f);
-    const float thr = kth - 2.f * bound;
+    const float bound = a.gamma * sqrtf(x2s[tt]) * 1.001f * wmax * 1.001f + 1e-6f * (fabsf(kth[tt]) + 1.f);
+    const float thr = kth[tt] - 2.f * bound;
     int nbefore = 0;      // candidates in earlier expert groups (warp-uniform)
     float snc = 0.f;
 #pragma unroll
@@ -661,6 +694,8 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
       const int e = lane + 32 * i;
       const bool cand = e < a.E && z[tt][i] >= thr;
       const unsigned m = __ballot_sync(0xffffffffu, cand);
+      // non-candidates (experts past E hold -inf: their term is +0)
+      snc += cand ? 0.f : __expf(z[tt][i] - m_s[tt]);
       if (cand) {
         const int slot = nbefore + __popc(m & lt);
         if (slot < kSelMaxCand) {
@@ -668,8 +703,6 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
           const int li = atomicAdd(&s_cnt[e], 1);
           s_rec[tl][slot] = ((uint32_t)e << 16) | (uint32_t)li;
         }
-      } else if (e < a.E) {
-        snc += __expf(z[tt][i] - m_s);
       }
       nbefore += __popc(m);
     }
@@ -677,7 +710,7 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
     for (int o = 16; o > 0; o >>= 1) snc += __shfl_xor_sync(0xffffffffu, snc, o);
     if (lane == 0) {
       a.ncand[t] = nbefore;
-      a.zmax[t] = m_s;
+      a.zmax[t] = m_s[tt];
       a.snc[t] = snc;
       s_nk[tl] = min(nbefore, kSelMaxCand);
     }
@@ -698,28 +731,29 @@ __global__ void __launch_bounds__(256) k_router_select(const SelectArgs a) {
   }
 }
 
-// Exact fp32 logits of the listed (token, expert) pairs, expert-major.  The
-// work items are slices of kRecompSlice consecutive entries of one expert's
-// list (lists of popular experts give many items, so the load stays balanced
-// whatever the routing skew); CTA b takes items b, b + gridDim.x, ...  Per
-// item the CTA stages the expert's W_r row (fp32, reloaded only when the
-// expert changes) and the slice's entries in shared memory, then each warp
-// computes kRecompBatch entries with their input-row loads in flight together:
-// lane l takes the 8-input slices l, l+32, ..., one fmaf chain, a fixed xor
-// tree, then the bias -- the same value for a (token, expert) pair whichever
-// CTA or warp computes it, and the same as warp_dot.  zex[t][slot] = exact logit.
-constexpr int kRecompSlice = 128;
-__global__ void __launch_bounds__(256, 2) k_router_recompute(const __nv_bfloat16* __restrict__ x,
-                                                             const float* __restrict__ W,
-                                                             const float* __restrict__ bias,
-                                                             const int32_t* __restrict__ ecount,
-                                                             const int32_t* __restrict__ elist,
-                                                             float* __restrict__ zex, int T, int d, int E) {
+// Exact fp32 logits of the listed (token, expert) pairs, expert-major.  A work
+// item is a slice of kRecompSlice consecutive entries of one expert's list
+// (popular experts give many items, so the load stays balanced whatever the
+// routing skew) and belongs to one warp: warp g of the grid takes items g,
+// g + (warps in the grid), ...  The warps run independently (no CTA barrier).
+// Per item the warp holds the lane's slices of the expert's W_r row in
+// registers, then computes NB entries at a time with all their input-row loads
+// in flight together: lane l takes the 8-input slices l, l+32, ..., one fmaf
+// chain, a fixed xor tree, then the bias -- the same value for a (token,
+// expert) pair whichever warp computes it, and the same as warp_dot.
+// zex[t][slot] = exact logit.
+constexpr int kRecompSlice = 16;
+// VPL: 16-byte input slices per lane (d <= 256 VPL); NB: entries per batch; MINB: resident CTAs per SM.
+template <int VPL, int NB, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_router_recompute(const __nv_bfloat16* __restrict__ x,
+                                                                const float* __restrict__ W,
+                                                                const float* __restrict__ bias,
+                                                                const int32_t* __restrict__ ecount,
+                                                                const int32_t* __restrict__ elist,
+                                                                float* __restrict__ zex, int T, int d, int E) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  static_assert(kRecompSlice == 8 * 2 * kRecompBatch, "a slice is two batches per warp of a 256-thread CTA");
-  __shared__ __align__(16) float s_w[kSelMaxD];
+  static_assert(NB <= kRecompSlice && kRecompSlice <= 32, "one lane per entry of an item");
   __shared__ int s_ipre[kMaxRouterE + 1];   // items of experts < e
-  __shared__ int s_ent[kRecompSlice];
   const int lane = lane_id();
   if (warp_id() == 0) {
     const int per = (E + 31) / 32;
@@ -742,8 +776,8 @@ __global__ void __launch_bounds__(256, 2) k_router_recompute(const __nv_bfloat16
   __syncthreads();
   const int nitems = s_ipre[E];
   const int nv = d >> 3;
-  int cur_e = -1;
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int item = blockIdx.x * (blockDim.x >> 5) + warp_id(); item < nitems; item += nwarps) {
     int lo = 0, hi = E - 1;   // the item's expert: last e with s_ipre[e] <= item
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -752,53 +786,60 @@ __global__ void __launch_bounds__(256, 2) k_router_recompute(const __nv_bfloat16
     const int e = lo;
     const int a0 = (item - s_ipre[e]) * kRecompSlice;
     const int n = min(kRecompSlice, ecount[e] - a0);
-    __syncthreads();   // the previous item's row and entries are no longer read
-    if (e != cur_e)
-      for (int i = threadIdx.x; i < d / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(s_w)[i] = reinterpret_cast<const float4*>(W + (size_t)e * d)[i];
-    if (threadIdx.x < n) s_ent[threadIdx.x] = elist[(size_t)e * T + a0 + threadIdx.x];
-    cur_e = e;
-    __syncthreads();
+    const int my_ent = lane < n ? elist[(size_t)e * T + a0 + lane] : 0;
+    // this lane's slices of W_r[e]: inputs 8v .. 8v + 7 for v = lane + 32 q
+    float4 w[VPL][2];
+    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int v = lane + 32 * q;
+      w[q][0] = v < nv ? __ldg(wr + 2 * v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      w[q][1] = v < nv ? __ldg(wr + 2 * v + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     const float be = bias != nullptr ? bias[e] : 0.f;
-    for (int b0 = kRecompBatch * warp_id(); b0 < n; b0 += kRecompBatch * (blockDim.x / 32)) {
-      int ent[kRecompBatch];
-      const uint4* xr[kRecompBatch];
+    for (int b0 = 0; b0 < n; b0 += NB) {
+      int ent[NB];
+      uint4 u[VPL][NB];
 #pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) {
-        ent[j] = s_ent[min(b0 + j, n - 1)];
-        xr[j] = reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d);
+      for (int j = 0; j < NB; ++j) ent[j] = __shfl_sync(0xffffffffu, my_ent, min(b0 + j, n - 1));
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) {
+        const int v = lane + 32 * q;
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+          u[q][j] = v < nv ? reinterpret_cast<const uint4*>(x + (size_t)(ent[j] / kSelMaxCand) * d)[v]
+                           : make_uint4(0, 0, 0, 0);
       }
-      float acc[kRecompBatch];
+      float acc[NB];
 #pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) acc[j] = 0.f;
-      for (int v = lane; v < nv; v += 32) {
-        uint4 u[kRecompBatch];
+      for (int j = 0; j < NB; ++j) acc[j] = 0.f;
 #pragma unroll
-        for (int j = 0; j < kRecompBatch; ++j) u[j] = xr[j][v];
-        const float4 w0 = reinterpret_cast<const float4*>(s_w)[2 * v];
-        const float4 w1 = reinterpret_cast<const float4*>(s_w)[2 * v + 1];
+      for (int q = 0; q < VPL; ++q) {
+        if (lane + 32 * q < nv) {   // the slices warp_dot visits, in its order
+          const float4 w0 = w[q][0], w1 = w[q][1];
 #pragma unroll
-        for (int j = 0; j < kRecompBatch; ++j) {
-          float s2 = acc[j];
-          s2 = fmaf(bf16lo(u[j].x), w0.x, s2); s2 = fmaf(bf16hi(u[j].x), w0.y, s2);
-          s2 = fmaf(bf16lo(u[j].y), w0.z, s2); s2 = fmaf(bf16hi(u[j].y), w0.w, s2);
-          s2 = fmaf(bf16lo(u[j].z), w1.x, s2); s2 = fmaf(bf16hi(u[j].z), w1.y, s2);
-          s2 = fmaf(bf16lo(u[j].w), w1.z, s2); s2 = fmaf(bf16hi(u[j].w), w1.w, s2);
-          acc[j] = s2;
+          for (int j = 0; j < NB; ++j) {
+            float s2 = acc[j];
+            s2 = fmaf(bf16lo(u[q][j].x), w0.x, s2); s2 = fmaf(bf16hi(u[q][j].x), w0.y, s2);
+            s2 = fmaf(bf16lo(u[q][j].y), w0.z, s2); s2 = fmaf(bf16hi(u[q][j].y), w0.w, s2);
+            s2 = fmaf(bf16lo(u[q][j].z), w1.x, s2); s2 = fmaf(bf16hi(u[q][j].z), w1.y, s2);
+            s2 = fmaf(bf16lo(u[q][j].w), w1.z, s2); s2 = fmaf(bf16hi(u[q][j].w), w1.w, s2);
+            acc[j] = s2;
+          }
         }
       }
 #pragma unroll
-      for (int j = 0; j < kRecompBatch; ++j) {
+      for (int j = 0; j < NB; ++j) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
       }
-      if (lane < kRecompBatch) {
+      if (lane < NB) {
         float mine = acc[0];
-        int my_ent = ent[0];
+        int me = ent[0];
 #pragma unroll
-        for (int j = 1; j < kRecompBatch; ++j)
-          if (lane == j) { mine = acc[j]; my_ent = ent[j]; }
-        if (b0 + lane < n) zex[my_ent] = mine + be;
+        for (int j = 1; j < NB; ++j)
+          if (lane == j) { mine = acc[j]; me = ent[j]; }
+        if (b0 + lane < n) zex[me] = mine + be;
       }
     }
   }

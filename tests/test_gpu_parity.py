@@ -102,15 +102,17 @@ def test_route_matches_oracle(lib, name, T, over):
         np.testing.assert_allclose(np64(r["aux"])[0], ref["aux"], rtol=5e-5)
 
 
-# Tensor-core router with the selection in the screening GEMM's epilogue (taken when neither logits nor the
-# load-balance statistic is requested): every k up to 16 (4- and 16-slot selection networks), column tiles of
-# 64 (E = 48: 16 padding columns), 192 and 256, the largest input width it takes (d = 2048), a skew bias, the
-# full granular batch, and tokens whose input row is zero (every logit equal, more candidates than the
-# selection keeps: those tokens are finished from exact logits of every expert, lowest indices first).
+# Tensor-core router with the certified selection kernels (taken when neither logits nor the load-balance
+# statistic is requested): every k up to 16, column tiles of 64 (E = 48: 16 padding columns), 128, 192 and
+# 256, single-CTA screening tiles (batches below a wave of 128-row tiles) and CTA-pair tiles (the full granular
+# batch; 20000 tokens: a ragged last 256-row tile), the largest input width it takes (d = 2048), a skew bias,
+# and tokens whose input row is zero (every logit equal, more candidates than the selection keeps: those tokens
+# are finished from exact logits of every expert, lowest indices first).
 @pytest.mark.parametrize("name,T,over,zero_rows", [("skewed", 3000, {}, 0), ("granular", 32768, {}, 0),
                                                    ("granular", 1100, {"E": 256, "k": 8, "d": 1024}, 0),
                                                    ("granular", 2100, {"E": 64, "k": 2, "d": 2048}, 0),
-                                                   ("skewed", 8000, {"E": 48, "k": 3}, 0),
+                                                   ("skewed", 20000, {"E": 48, "k": 3}, 0),
+                                                   ("granular", 19500, {"E": 128, "k": 4, "d": 512}, 0),
                                                    ("granular", 2000, {"k": 16}, 0),
                                                    ("granular", 2000, {}, 37)])
 def test_route_select_path_matches_oracle(lib, name, T, over, zero_rows):
