@@ -156,12 +156,37 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint4& wa, cons
 //       thread adding its 8 in order, then a fixed xor tree over the group's 16;
 //   rscale[r] = 2^e.
 // The product of the codes with x' minus c is sum(q x') = 2^-e sum(q x).
+// With slot_pos (the grouping of a routed batch), block t converts token row t
+// of A once and writes it to every grouped row slot_pos[t * kk + j] >= 0: the
+// grouped copy of the activations is formed here, with no bf16 copy between;
+// with Aq2 set, row t also goes to row t of (csum2, rscale2, Aq2): the ungrouped
+// copy the shared expert reads.
 __global__ void __launch_bounds__(1024) k_int4_act_prep(const __nv_bfloat16* __restrict__ A, int K,
                                                        float* __restrict__ csum, float* __restrict__ rscale,
-                                                       __half* __restrict__ Aq) {
+                                                       __half* __restrict__ Aq,
+                                                       const int32_t* __restrict__ slot_pos, int kk,
+                                                       float* __restrict__ csum2, float* __restrict__ rscale2,
+                                                       __half* __restrict__ Aq2) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   __shared__ float s_m[32];
-  const long long row = blockIdx.x;
+  __shared__ int s_dst[16];
+  __shared__ int s_nd;
+  const long long row = blockIdx.x;   // source row
+  int ndst = 1;
+  if (slot_pos != nullptr) {          // destination rows of this token (kk <= 16), dropped slots skipped
+    if (threadIdx.x == 0) {
+      int nd = 0;
+      for (int j = 0; j < kk; ++j) {
+        const int pos = slot_pos[row * kk + j];
+        if (pos >= 0) s_dst[nd++] = pos;
+      }
+      s_nd = nd;
+    }
+    __syncthreads();
+    ndst = s_nd;
+  } else if (threadIdx.x == 0) {
+    s_dst[0] = (int)row;
+  }
   const int nv = K / 8;   // 16 per 128-group; a pass covers whole groups
   const uint4* src = reinterpret_cast<const uint4*>(A + row * K);
   // the first pass's inputs stay in registers for the conversion (the whole row when nv <= blockDim)
@@ -181,8 +206,9 @@ __global__ void __launch_bounds__(1024) k_int4_act_prep(const __nv_bfloat16* __r
   const int eb = (int)((__float_as_uint(m) >> 23) & 0xFFu);   // biased exponent of the row's largest |x|
   const int e = m == 0.f ? 0 : (eb == 0 ? -100 : max(-100, min(113, eb - 127 - 14)));
   const float down = __uint_as_float((uint32_t)(127 - e) << 23);   // 2^-e, a normal float for e in [-100, 113]
-  if (threadIdx.x == 0) rscale[row] = __uint_as_float((uint32_t)(127 + e) << 23);
-  uint4* dst = reinterpret_cast<uint4*>(Aq + row * K);
+  const float up = __uint_as_float((uint32_t)(127 + e) << 23);   // 2^e
+  if ((int)threadIdx.x < ndst) rscale[s_dst[threadIdx.x]] = up;
+  if (Aq2 != nullptr && threadIdx.x == 0) rscale2[row] = up;
   for (int base = 0; base < nv; base += blockDim.x) {   // every thread takes part in each pass's xor tree
     const int v = base + threadIdx.x;
     const bool on = v < nv;
@@ -202,8 +228,16 @@ __global__ void __launch_bounds__(1024) k_int4_act_prep(const __nv_bfloat16* __r
       auto pack = [](__half lo, __half hi) {
         return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
       };
-      dst[v] = make_uint4(pack(h[0], h[4]), pack(h[1], h[5]), pack(h[2], h[6]), pack(h[3], h[7]));
-      if ((v & 15) == 0) csum[row * (K / 128) + (v >> 4)] = c;
+      const uint4 q = make_uint4(pack(h[0], h[4]), pack(h[1], h[5]), pack(h[2], h[6]), pack(h[3], h[7]));
+      for (int j = 0; j < ndst; ++j) {
+        const long long dr = s_dst[j];
+        reinterpret_cast<uint4*>(Aq + dr * K)[v] = q;
+        if ((v & 15) == 0) csum[dr * (K / 128) + (v >> 4)] = c;
+      }
+      if (Aq2 != nullptr) {
+        reinterpret_cast<uint4*>(Aq2 + row * K)[v] = q;
+        if ((v & 15) == 0) csum2[row * (K / 128) + (v >> 4)] = c;
+      }
     }
   }
 }
@@ -491,19 +525,28 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
 
 // ---------------------------------------------------------------------------
 // Dense small batches (one group of R <= 256 rows: the shared expert of a
-// decode batch).  k_int4_stream gives each task 8 rows, so a 64-row batch
-// would read and dequantise every weight eight times; here a task is one block
-// of 32 weight rows over 32 rows (four 8-row chunks), its reduction split into
-// p.ksplit slab ranges: a 64-row batch reads and dequantises every weight
-// twice, and each dequantised fragment feeds the MMAs of four chunks.  f16 offset
-// codes and scaled activations, with the group terms (c, 2^e), as in
-// k_int4_stream's OFFS mode; fp32 partials [ksplit][R][W] in its split layout, which
-// k_int4_splitk_reduce adds in order.  Eight warps per CTA, each with a ring of
-// kI4DStages slabs.
+// decode batch).  A CTA task is (kI4DWarps weight blocks, a block of 64 rows, a
+// slab range of the reduction).  Warp w owns weight block kI4DWarps obg + w
+// (16 gate + 16 up rows, or 32 output rows) and streams its packed weights by
+// TMA through its own ring; the 64 rows' activations (the f16 copy written by
+// k_int4_act_prep) and the slab's offset shares go to shared memory once per
+// slab for all warps, by cp.async into two buffers, so slab s + 1 loads while
+// slab s computes.  Each weight is read once per 64 rows and dequantised once
+// per 32 (the MMAs of four 8-row chunks).  f16 offset codes as in k_int4_stream's OFFS
+// mode; fp32 partials [ksplit][R][W] in its split layout, which
+// k_int4_splitk_reduce adds in order.
 constexpr int kI4DWarps = 8;
 constexpr int kI4DStages = 4;
-constexpr int kI4DSmem = kI4DWarps * kI4DStages * kI4SlabBytes;
-constexpr int kI4DChunks = 4;            // 8-row chunks per task
+constexpr int kI4DChunks = 8;                      // 8-row chunks per task
+constexpr int kI4DRows = 8 * kI4DChunks;           // rows per task
+constexpr int kI4DActBytes = kI4DRows * 512;       // one slab of activations: 64 rows x 256 f16
+constexpr int kI4DSmem = kI4DWarps * kI4DStages * kI4SlabBytes + 2 * kI4DActBytes;
+
+// 16-byte chunk q (of the 32 in a 256-input activation row) of row r is stored at
+// chunk q ^ (bit 3 of q, as bit 1 | bit 0 of r): the fragment reads of a
+// quarter-warp (rows 2i, 2i+1; lanes c = 0..3 reading chunks 4c + j) then hit
+// eight different bank groups.
+__device__ __forceinline__ int dense_act_chunk(int q, int r) { return q ^ ((((q >> 3) & 1) << 1) | (r & 1)); }
 
 template <bool GLU>
 __global__ void __launch_bounds__(kI4DWarps * 32, 1)
@@ -513,6 +556,7 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
   extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ __align__(8) uint64_t s_bar[kI4DWarps][kI4DStages];
   __shared__ volatile int s_abort[kI4DWarps];
+  __shared__ float s_c[2][kI4DRows][2];    // offsets' shares of a slab's two groups, per row
   const int lane = lane_id(), warp = warp_id();
   if (lane == 0) {
     for (int st = 0; st < kI4DStages; ++st) mbar_init(&s_bar[warp][st], 1);
@@ -521,34 +565,44 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
   __syncthreads();
+  uint8_t* ring = i4_smem + (size_t)warp * kI4DStages * kI4SlabBytes;
+  uint8_t* act = i4_smem + (size_t)kI4DWarps * kI4DStages * kI4SlabBytes;
   const int KS = p.ksplit;
   const int oblocks = GLU ? p.N / 16 : p.N / 32;
+  const int nobg = (oblocks + kI4DWarps - 1) / kI4DWarps;
   const int R = (int)p.R;
-  const int nrh = (R + 8 * kI4DChunks - 1) / (8 * kI4DChunks);   // row blocks of 8 * kI4DChunks rows
-  const int total = oblocks * nrh * KS;                          // task = (weight block, row block, split)
+  const int nrh = (R + kI4DRows - 1) / kI4DRows;
+  const int total = nobg * nrh * KS;       // task = (weight block group, row block, split), split fastest
   const int nslab = (p.K + 255) / 256;
   const int ngk = p.K / 128;
   const int gq = lane >> 2, c = lane & 3;
-  const int tstride = gridDim.x * kI4DWarps;
-  uint8_t* ring = i4_smem + (size_t)warp * kI4DStages * kI4SlabBytes;
+  auto task_pos = [&](int task, int& ob, int& rh, int& sb, int& se) {
+    const int sp = task % KS;
+    rh = (task / KS) % nrh;
+    ob = (task / (KS * nrh)) * kI4DWarps + warp;
+    sb = sp * nslab / KS;
+    se = (sp + 1) * nslab / KS;
+  };
   auto rows_of = [&](int ob, int& ra, int& rb) {
     ra = GLU ? ob * 16 : ob * 32;
     rb = GLU ? p.up_row0 + ob * 16 : ra + 16;
   };
-  // producer (lane 0 issues; values warp-uniform): items are (task, slab) in order, at most kI4DStages ahead
+  // weight producer (lane 0 issues; values warp-uniform): the warp's slabs of the CTA's tasks in order, at
+  // most kI4DStages ahead; tasks whose weight block is past the last one have none
   int issued = 0, consumed = 0;
-  int p_task = blockIdx.x * kI4DWarps + warp, p_slab = 0, p_se = 0, p_st = 0, p_ra = 0, p_rb = 0;
+  int p_task = blockIdx.x, p_slab = 0, p_se = 0, p_st = 0, p_ra = 0, p_rb = 0;
   bool p_new = true;
   auto refill = [&]() {
-    while (issued - consumed < kI4DStages) {
+    while (issued - consumed < kI4DStages && !s_abort[warp]) {
       if (p_new) {
         if (p_task >= total) return;
-        const int ob = p_task / (KS * nrh), sp = p_task % KS;
+        int ob, rh, sb, se;
+        task_pos(p_task, ob, rh, sb, se);
+        if (ob >= oblocks || sb == se) { p_task += gridDim.x; continue; }
         rows_of(ob, p_ra, p_rb);
-        p_slab = sp * nslab / KS;
-        p_se = (sp + 1) * nslab / KS;
+        p_slab = sb;
+        p_se = se;
         p_new = false;
-        if (p_slab == p_se) { p_new = true; p_task += tstride; continue; }
       }
       if (lane == 0) {
         uint8_t* dst = ring + p_st * kI4SlabBytes;
@@ -558,20 +612,37 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
       }
       ++issued;
       if (++p_st == kI4DStages) p_st = 0;
-      if (++p_slab == p_se) { p_new = true; p_task += tstride; }
+      if (++p_slab == p_se) { p_new = true; p_task += gridDim.x; }
     }
+  };
+  // activations of slab s for rows r0 .. r0 + 63 into buffer b (zeros past R and past K)
+  auto load_act = [&](int s, int b, int r0) {
+    uint8_t* dst = act + (size_t)b * kI4DActBytes;
+    for (int q = threadIdx.x; q < kI4DRows * 32; q += blockDim.x) {
+      const int r = q >> 5, ch = q & 31;
+      const int tok = r0 + r, kin = s * 256 + ch * 8;
+      const bool on = tok < R && kin < p.K;
+      const __nv_bfloat16* src = on ? p.act + (size_t)tok * p.K + kin : p.act;
+      cp_async16(dst + r * 512 + dense_act_chunk(ch, r) * 16, src, on ? 16 : 0);
+    }
+  };
+  // the offsets' share of group g of slab s for row r (thread i < 128: r = i / 2, g = i % 2)
+  auto share = [&](int s, int r0) -> float {
+    const int r = threadIdx.x >> 1, kg = 2 * s + (threadIdx.x & 1), tok = r0 + r;
+    return (tok < R && kg < ngk) ? xcs[(size_t)tok * ngk + kg] : 0.f;
   };
 
   float tA[kI4DChunks][4], tB[kI4DChunks][4];
   int c_st = 0;
   uint32_t c_phase = 0;
-  for (int task = blockIdx.x * kI4DWarps + warp; task < total && !s_abort[warp]; task += tstride) {
-    const int ob = task / (KS * nrh), rh = (task / KS) % nrh, sp = task % KS;
-    const int r0 = rh * 8 * kI4DChunks;
-    int ra, rb;
-    rows_of(ob, ra, rb);
-    const int sb = sp * nslab / KS, se = (sp + 1) * nslab / KS;
-    if (sb == se) continue;
+  for (int task = blockIdx.x; task < total; task += gridDim.x) {
+    int ob, rh, sb, se;
+    task_pos(task, ob, rh, sb, se);
+    if (sb == se) continue;                  // the same for every warp of the CTA
+    const bool mine = ob < oblocks;
+    const int r0 = rh * kI4DRows;
+    int ra = 0, rb = 0;
+    if (mine) rows_of(ob, ra, rb);
 #pragma unroll
     for (int ch = 0; ch < kI4DChunks; ++ch)
 #pragma unroll
@@ -579,76 +650,103 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
     const __nv_bfloat16* sA = p.ws + (long long)(ra + gq) * ngk;
     const __nv_bfloat16* sB = p.ws + (long long)(rb + gq) * ngk;
     const long long s8 = 8ll * ngk;
-    bool ok = true;
-    for (int slab = sb; slab < se; ++slab) {
-      refill();
-      if (!mbar_wait(&s_bar[warp][c_st], c_phase, wait_limit_ns, &s_abort[warp], 0x0203)) { ok = false; break; }
-      const uint8_t* slabp = ring + c_st * kI4SlabBytes;
+    load_act(sb, 0, r0);
+    if (threadIdx.x < kI4DRows * 2) s_c[0][threadIdx.x >> 1][threadIdx.x & 1] = share(sb, r0);
+    for (int s = sb; s < se; ++s) {
+      const int b = (s - sb) & 1;
+      // slab s + 1's activations and shares start loading (buffer b ^ 1 was last read at slab s - 1, before the
+      // barrier that closed it)
+      float cnext = 0.f;
+      if (s + 1 < se) {
+        load_act(s + 1, b ^ 1, r0);
+        if (threadIdx.x < kI4DRows * 2) cnext = share(s + 1, r0);
+      }
+      cp_async_commit();                     // an empty group on the last slab keeps the count uniform
+      // the group scales of weight rows gq, gq + 8 (gate / first half) and the other half, before the waits
+      float sc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+      if (mine) {
+        const __nv_bfloat16* sp4[4] = {sA, sA + s8, sB, sB + s8};
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const int kg = slab * 2 + gi;
-        if (kg >= ngk) break;   // the slab's second half is TMA zero fill
-        const uint4 a0 = *reinterpret_cast<const uint4*>(slabp + gq * 128 + gi * 64 + c * 16);
-        const uint4 a1 = *reinterpret_cast<const uint4*>(slabp + (gq + 8) * 128 + gi * 64 + c * 16);
-        const uint4 b0 = *reinterpret_cast<const uint4*>(slabp + (gq + 16) * 128 + gi * 64 + c * 16);
-        const uint4 b1 = *reinterpret_cast<const uint4*>(slabp + (gq + 24) * 128 + gi * 64 + c * 16);
-        float pA[kI4DChunks][4], pB[kI4DChunks][4];
+        for (int rr = 0; rr < 4; ++rr)
 #pragma unroll
-        for (int ch = 0; ch < kI4DChunks; ++ch)
+          for (int gi = 0; gi < 2; ++gi)
+            sc[rr][gi] = 2 * s + gi < ngk ? __bfloat162float(sp4[rr][2 * s + gi]) : 0.f;
+        refill();
+      }
+      cp_async_wait<1>();                    // this thread's copies of slab s have landed
+      __syncthreads();                       // and everyone's: slab s's activations and shares are visible
+      if (mine && !s_abort[warp] &&
+          mbar_wait(&s_bar[warp][c_st], c_phase, wait_limit_ns, &s_abort[warp], 0x0203)) {
+        const uint8_t* slabp = ring + c_st * kI4SlabBytes;
+        const uint8_t* abuf = act + (size_t)b * kI4DActBytes;
+#pragma unroll 1
+        for (int gi = 0; gi < 2; ++gi) {
+          if (2 * s + gi >= ngk) break;      // the slab's second half is TMA zero fill
+          const uint4 a0 = *reinterpret_cast<const uint4*>(slabp + gq * 128 + gi * 64 + c * 16);
+          const uint4 a1 = *reinterpret_cast<const uint4*>(slabp + (gq + 8) * 128 + gi * 64 + c * 16);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(slabp + (gq + 16) * 128 + gi * 64 + c * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(slabp + (gq + 24) * 128 + gi * 64 + c * 16);
+          // two halves of four 8-row chunks each (the weights are dequantised once per half: the group
+          // partials of all eight chunks would not fit the registers beside the running sums)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) { pA[ch][i] = 0.f; pB[ch][i] = 0.f; }
-        // the group's activation fragments of every chunk, loads in flight together
-        uint4 xf[kI4DChunks][4];
+          for (int hf = 0; hf < 2; ++hf) {
+            constexpr int HC = kI4DChunks / 2;
+            float pA[HC][4], pB[HC][4];
 #pragma unroll
-        for (int ch = 0; ch < kI4DChunks; ++ch) {
-          const int tok = r0 + 8 * ch + gq;
-          const uint4* xrow = reinterpret_cast<const uint4*>(p.act + (long long)(tok < R ? tok : 0) * p.K + kg * 128 + c * 32);
+            for (int ch = 0; ch < HC; ++ch)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) xf[ch][j] = tok < R ? xrow[j] : make_uint4(0, 0, 0, 0);
-        }
+              for (int i = 0; i < 4; ++i) { pA[ch][i] = 0.f; pB[ch][i] = 0.f; }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t qa0[4], qa1[4], qb0[4], qb1[4];
-          offset_word_f16(u4get(a0, j), qa0);
-          offset_word_f16(u4get(a1, j), qa1);
-          offset_word_f16(u4get(b0, j), qb0);
-          offset_word_f16(u4get(b1, j), qb1);
+            for (int j = 0; j < 4; ++j) {
+              uint32_t qa0[4], qa1[4], qb0[4], qb1[4];
+              offset_word_f16(u4get(a0, j), qa0);
+              offset_word_f16(u4get(a1, j), qa1);
+              offset_word_f16(u4get(b0, j), qb0);
+              offset_word_f16(u4get(b1, j), qb1);
+              const int q = gi * 16 + c * 4 + j;   // 16-byte chunk of the activation row
 #pragma unroll
-          for (int ch = 0; ch < kI4DChunks; ++ch) {
-            mma_f16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf[ch][j].x, xf[ch][j].y);
-            mma_f16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf[ch][j].z, xf[ch][j].w);
-            mma_f16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf[ch][j].x, xf[ch][j].y);
-            mma_f16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf[ch][j].z, xf[ch][j].w);
+              for (int ch = 0; ch < HC; ++ch) {
+                const int r = 8 * (hf * HC + ch) + gq;
+                const uint4 xf = *reinterpret_cast<const uint4*>(abuf + r * 512 + dense_act_chunk(q, r) * 16);
+                mma_f16_16816(pA[ch], qa0[0], qa1[0], qa0[1], qa1[1], xf.x, xf.y);
+                mma_f16_16816(pA[ch], qa0[2], qa1[2], qa0[3], qa1[3], xf.z, xf.w);
+                mma_f16_16816(pB[ch], qb0[0], qb1[0], qb0[1], qb1[1], xf.x, xf.y);
+                mma_f16_16816(pB[ch], qb0[2], qb1[2], qb0[3], qb1[3], xf.z, xf.w);
+              }
+            }
+            // offsets' share (columns = rows 8 ch + 2c, 8 ch + 2c + 1), then the weight rows' group scales
+            const float s0 = gi ? sc[0][1] : sc[0][0], s1 = gi ? sc[1][1] : sc[1][0];
+            const float s2 = gi ? sc[2][1] : sc[2][0], s3 = gi ? sc[3][1] : sc[3][0];
+#pragma unroll
+            for (int ch = 0; ch < HC; ++ch) {
+              const int cc = hf * HC + ch;
+              const float x0 = s_c[b][8 * cc + 2 * c][gi], x1 = s_c[b][8 * cc + 2 * c + 1][gi];
+              tA[cc][0] = fmaf(pA[ch][0] - x0, s0, tA[cc][0]);
+              tA[cc][1] = fmaf(pA[ch][1] - x1, s0, tA[cc][1]);
+              tA[cc][2] = fmaf(pA[ch][2] - x0, s1, tA[cc][2]);
+              tA[cc][3] = fmaf(pA[ch][3] - x1, s1, tA[cc][3]);
+              tB[cc][0] = fmaf(pB[ch][0] - x0, s2, tB[cc][0]);
+              tB[cc][1] = fmaf(pB[ch][1] - x1, s2, tB[cc][1]);
+              tB[cc][2] = fmaf(pB[ch][2] - x0, s3, tB[cc][2]);
+              tB[cc][3] = fmaf(pB[ch][3] - x1, s3, tB[cc][3]);
+            }
           }
         }
-        // offsets' share (columns = rows 8 ch + 2c, 8 ch + 2c + 1), then the weight rows' group scales (rows gq,
-        // gq + 8)
-        const float scA0 = __bfloat162float(sA[kg]), scA1 = __bfloat162float(sA[s8 + kg]);
-        const float scB0 = __bfloat162float(sB[kg]), scB1 = __bfloat162float(sB[s8 + kg]);
-#pragma unroll
-        for (int ch = 0; ch < kI4DChunks; ++ch) {
-          const int n0 = r0 + 8 * ch + 2 * c;
-          const float x0 = n0 < R ? xcs[(long long)n0 * ngk + kg] : 0.f;
-          const float x1 = n0 + 1 < R ? xcs[(long long)(n0 + 1) * ngk + kg] : 0.f;
-          tA[ch][0] = fmaf(pA[ch][0] - x0, scA0, tA[ch][0]);
-          tA[ch][1] = fmaf(pA[ch][1] - x1, scA0, tA[ch][1]);
-          tA[ch][2] = fmaf(pA[ch][2] - x0, scA1, tA[ch][2]);
-          tA[ch][3] = fmaf(pA[ch][3] - x1, scA1, tA[ch][3]);
-          tB[ch][0] = fmaf(pB[ch][0] - x0, scB0, tB[ch][0]);
-          tB[ch][1] = fmaf(pB[ch][1] - x1, scB0, tB[ch][1]);
-          tB[ch][2] = fmaf(pB[ch][2] - x0, scB1, tB[ch][2]);
-          tB[ch][3] = fmaf(pB[ch][3] - x1, scB1, tB[ch][3]);
-        }
+        __syncwarp();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slab reads done before TMA reuses it
+        ++consumed;
+        if (++c_st == kI4DStages) { c_st = 0; c_phase ^= 1u; }
       }
-      __syncwarp();
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // slab reads done before TMA reuses it
-      ++consumed;
-      if (++c_st == kI4DStages) { c_st = 0; c_phase ^= 1u; }
+      // slab s + 1's shares into their buffer (its readers finished at slab s - 1)
+      if (s + 1 < se && threadIdx.x < kI4DRows * 2) s_c[b ^ 1][threadIdx.x >> 1][threadIdx.x & 1] = cnext;
+      __syncthreads();                       // buffer b is read by every warp before slab s + 2 refills it
     }
-    if (!ok) break;
-    // partials of this slab range, in k_int4_stream's split layout
+    cp_async_wait<0>();
+    if (!mine || s_abort[warp]) continue;
+    // partials of this slab range, in k_int4_stream's split layout, back from the scaled activations
     const int o0 = GLU ? ob * 16 : ob * 32;
     const int W = GLU ? 2 * p.N : p.N;
+    const int sp = task % KS;
 #pragma unroll
     for (int ch = 0; ch < kI4DChunks; ++ch) {
 #pragma unroll
@@ -657,7 +755,7 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
         const int n = r0 + 8 * ch + 2 * c + (i & 1);
         if (n < R) {
           float* prow = p.part + ((long long)sp * R + n) * W + o0;
-          const float rs = xrs[n];   // back from the scaled activations: the row's 2^e (exact)
+          const float rs = xrs[n];
           if (GLU) {
             prow[m] = tA[ch][i] * rs;
             prow[p.N + m] = tB[ch][i] * rs;
@@ -670,6 +768,7 @@ __global__ void __launch_bounds__(kI4DWarps * 32, 1)
     }
   }
   // never leave the CTA with copies still landing in its shared memory
+  cp_async_wait<0>();
   {
     volatile int dummy = 0;
     for (int i = consumed; i < issued; ++i)

@@ -162,7 +162,8 @@ static Workspace ws_layout(const moe_shape* s) {
   L.part = take((size_t)ns * s->T * s->E * 4);
   L.wsplit = take((size_t)2 * s->E * s->d * 2);
   L.wnorm = take((size_t)s->E * 4);
-  const long long xs_rows = std::max<long long>(grouped_rows(s), s->T);
+  // routed rows, then the shared expert's token rows (its copy is written with the routed one)
+  const long long xs_rows = grouped_rows(s) + s->T;   // rows of xs_cols elements
   const int xs_cols = std::max(s->d, std::max(s->H, s->H_s));
   L.xcs = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * (xs_cols / 128) * 4 : 16);
   L.xrs = take(s->wfmt == MOE_WFMT_INT4_G128 ? (size_t)xs_rows * 4 : 16);
@@ -382,8 +383,8 @@ static int launch_topk(const moe_shape* s, const float* part, int nsplit, const 
     }                                                                                                             \
     const unsigned grid = ST_ ? (unsigned)nchunks : (unsigned)cdiv(s->T, NW_);                                    \
     MOE_LAUNCH((k_router_topk<N_, NW_, XR_, ST_>), grid, NW_ * 32, smem, st, part, nsplit, bias, logits, idx, w, cnt, psum,  \
-                                                                   p_scratch, (int)s->T, s->E, s->k, s->renorm,  \
-                                                                   refine);                                       \
+                                                                   psum ? p_scratch : nullptr, (int)s->T, s->E,  \
+                                                                   s->k, s->renorm, refine);                      \
     MOE_LAUNCH_CHECK();                                                                                           \
     if (!ST_) {                                                                                                   \
       MOE_LAUNCH((k_chunk_stats), nchunks, 256, 0, st, idx, p_scratch, cnt, psum, (int)s->T, s->E, s->k);                   \
@@ -505,6 +506,14 @@ struct Int4Scratch {
   void* xq;
   float* part = nullptr;        // split-reduction partials (dense groups with few tasks), or none
   size_t part_floats = 0;
+  // grouping of a routed batch: the activation copy is formed from the token rows (src_x, src_T tokens) and
+  // slot_pos directly, with no bf16 grouped copy in between (the first GEMM of the routed FFN only)
+  const void* src_x = nullptr;
+  long long src_T = 0;
+  const int32_t* slot_pos = nullptr;
+  int slot_k = 0;
+  const Int4Scratch* also = nullptr;   // with slot_pos: also write token t's copy to row t of these buffers
+  bool prepped = false;         // xcs, xrs, xq already hold this GEMM's activations: no preparation launch
 };
 
 static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const void* wq, const void* wsc,
@@ -574,24 +583,31 @@ static int int4_gemm(bool glu, int act, const void* A, long long R, int K, const
       MOE_CUDA_TRY(cudaFuncSetAttribute(k_int4_dense<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI4DSmem));
       done.fetch_or(bit);
     }
-    if (xcs != nullptr) {
+    if (xcs != nullptr && !scr.prepped) {
       const int pt = (int)std::min<long long>(1024, std::max<long long>(64, cdiv(K / 8, 32) * 32));
-      MOE_LAUNCH((k_int4_act_prep), (unsigned)R, pt, 0, st, reinterpret_cast<const __nv_bfloat16*>(A), K, xcs, xrs,
-                 reinterpret_cast<__half*>(scr.xq));
+      if (scr.slot_pos != nullptr)
+        MOE_LAUNCH((k_int4_act_prep), (unsigned)scr.src_T, pt, 0, st, reinterpret_cast<const __nv_bfloat16*>(scr.src_x),
+                   K, xcs, xrs, reinterpret_cast<__half*>(scr.xq), scr.slot_pos, scr.slot_k,
+                   scr.also ? scr.also->xcs : nullptr, scr.also ? scr.also->xrs : nullptr,
+                   scr.also ? reinterpret_cast<__half*>(scr.also->xq) : nullptr);
+      else
+        MOE_LAUNCH((k_int4_act_prep), (unsigned)R, pt, 0, st, reinterpret_cast<const __nv_bfloat16*>(A), K, xcs, xrs,
+                   reinterpret_cast<__half*>(scr.xq), (const int32_t*)nullptr, 0, (float*)nullptr, (float*)nullptr,
+                   (__half*)nullptr);
       MOE_LAUNCH_CHECK();
-      p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);   // f16 bytes: loaded as raw fragments
     }
+    if (xcs != nullptr) p.act = reinterpret_cast<const __nv_bfloat16*>(scr.xq);   // f16 bytes: raw fragments
     if (grows == nullptr && xcs != nullptr && scr.part != nullptr && R <= 256) {
-      // one dense group of a small batch (the shared expert of a decode batch): tasks of 32 weight rows over
-      // 32 rows, each weight dequantised once per 32 rows; the reduction split so that every warp has work
-      const long long base = (long long)(N / (glu ? 16 : 32)) * cdiv(R, 32);
-      const long long warps = (long long)num_sms() * kI4DWarps;
-      int ks = (int)std::min<long long>(std::min<long long>(8, cdiv(K, 256)), std::max<long long>(1, cdiv(2 * warps, base)));
+      // one dense group of a small batch (the shared expert of a decode batch): CTA tasks of kI4DWarps weight
+      // blocks over 64 rows, each weight dequantised once per 64 rows; the reduction split so that the tasks
+      // fill the SMs once (a second partial round would double the time)
+      const long long base = cdiv(N / (glu ? 16 : 32), kI4DWarps) * cdiv(R, kI4DRows);
+      int ks = (int)std::min<long long>(std::min<long long>(8, cdiv(K, 256)), std::max<long long>(1, num_sms() / base));
       while (ks > 1 && (size_t)ks * R * (glu ? 2 * N : N) > scr.part_floats) --ks;
       if ((size_t)ks * R * (glu ? 2 * N : N) <= scr.part_floats) {
         p.ksplit = ks;
         p.part = scr.part;
-        const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), cdiv(base * ks, kI4DWarps)));
+        const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), base * ks));
         const unsigned long long lim = g_wait_limit_ns.load();
         if (glu) MOE_LAUNCH((k_int4_dense<true>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xcs, xrs);
         else MOE_LAUNCH((k_int4_dense<false>), grid, kI4DWarps * 32, kI4DSmem, st, tm, p, lim, xcs, xrs);
@@ -653,7 +669,10 @@ static int expert_ffn_impl(const moe_shape* s, int hidden, long long R, const vo
     rc = int4_gemm(true, s->act, A, R, s->d, w13, s13, n_groups, 2 * hidden, hidden, hidden, gstart, grows, h, st,
                    scr);
     if (rc) return rc;
-    return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st, scr);
+    Int4Scratch scr2 = scr;
+    scr2.slot_pos = nullptr;   // h is already grouped
+    scr2.prepped = false;
+    return int4_gemm(false, s->act, h, R, hidden, w2, s2, n_groups, s->d, 0, s->d, gstart, grows, y, st, scr2);
   }
   if (h == nullptr) return launch_fused(s, hidden, R, A, gstart, grows, n_groups, w13, w2, y, st);
   const int mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
@@ -752,12 +771,15 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   float* P = aux_p ? aux_p : reinterpret_cast<float*>(ws + L.fP) + s->E;
   int rc;
   int nsplit = 1;
+  // chunk probability sums only when the load-balance statistic (f, P or aux) is requested
+  const bool want_fp = aux_f || aux_p || aux;
+  float* psum_w = want_fp ? psum : nullptr;
   const int ec_lanes = lanes_router_ec(s);
   const int epl_fused = fused_router_epl(s);
   if (logits_in == nullptr && ec_lanes > 0) {
-    rc = launch_lanes_router(s, ec_lanes, x, w_router, bias, logits, idx, w, cnt, psum, st);
+    rc = launch_lanes_router(s, ec_lanes, x, w_router, bias, logits, idx, w, cnt, psum_w, st);
   } else if (logits_in == nullptr && epl_fused > 0) {
-    rc = launch_fused_router(s, epl_fused, x, w_router, bias, logits, idx, w, cnt, psum, st);
+    rc = launch_fused_router(s, epl_fused, x, w_router, bias, logits, idx, w, cnt, psum_w, st);
   } else if (logits_in == nullptr && use_tc_router(s)) {
     __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + L.wsplit);
     float* wnorm = reinterpret_cast<float*>(ws + L.wnorm);
@@ -825,7 +847,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
       rc = MOE_OK;
     } else {
       RefineArgs ref{reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias, wnorm, s->d, gamma};
-      rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum, part, st, ref);
+      rc = launch_topk(s, part, 1, nullptr, logits, idx, w, cnt, psum_w, part, st, ref);
     }
   } else if (logits_in == nullptr && s->T <= 256 && skinny_smem(s->d) <= kSkinnyMaxSmem) {
     const unsigned long long bit = 1ull << (current_device() & 63);
@@ -837,7 +859,7 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     MOE_LAUNCH((k_router_skinny), grid, 256, skinny_smem(s->d), st, reinterpret_cast<const __nv_bfloat16*>(x), w_router, part,
                                                            (int)s->T, s->d, s->E);
     MOE_LAUNCH_CHECK();
-    rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum, part, st);
+    rc = launch_topk(s, part, 1, bias, logits, idx, w, cnt, psum_w, part, st);
   } else if (logits_in == nullptr) {
     int kps = 0;
     nsplit = router_splits(s, &kps);
@@ -845,12 +867,11 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
     MOE_LAUNCH((k_router_logits), grid, 128, 0, st, reinterpret_cast<const __nv_bfloat16*>(x), w_router, part, (int)s->T,
                                           s->d, s->E, kps);
     MOE_LAUNCH_CHECK();
-    rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum, part, st);
+    rc = launch_topk(s, part, nsplit, bias, logits, idx, w, cnt, psum_w, part, st);
   } else {
-    rc = launch_topk(s, logits_in, 1, nullptr, nullptr, idx, w, cnt, psum, part, st);
+    rc = launch_topk(s, logits_in, 1, nullptr, nullptr, idx, w, cnt, psum_w, part, st);
   }
   if (rc) return rc;
-  const bool want_fp = aux_f || aux_p || aux;
   rc = launch_scan(s, cnt, want_fp ? psum : nullptr, counts, want_fp ? f : nullptr, want_fp ? P : nullptr, st);
   if (rc) return rc;
   if (aux && !defer_aux) {   // deferred: the caller's grouping kernel forms aux from f and P
@@ -1038,20 +1059,38 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   if (rc) return rc;
   const float* f_used = aux_f ? aux_f : reinterpret_cast<const float*>(ws + L.fP);
   const float* p_used = aux_p ? aux_p : reinterpret_cast<const float*>(ws + L.fP) + s->E;
-  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream, true, f_used, p_used,
+  const bool int4 = s->wfmt == MOE_WFMT_INT4_G128;
+  // INT4: the grouped activation copy is formed by k_int4_act_prep from x and the slots, so no bf16 rows move
+  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream, !int4, f_used, p_used,
                       aux);
   if (rc) return rc;
-  const Int4Scratch scr = s->wfmt == MOE_WFMT_INT4_G128
-                              ? Int4Scratch{reinterpret_cast<float*>(ws + L.xcs), reinterpret_cast<float*>(ws + L.xrs),
-                                            ws + L.xq, reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
-                              : Int4Scratch{nullptr, nullptr, nullptr};
-  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr);
+  const Int4Scratch scr = int4 ? Int4Scratch{reinterpret_cast<float*>(ws + L.xcs), reinterpret_cast<float*>(ws + L.xrs),
+                                             ws + L.xq, reinterpret_cast<float*>(ws + L.i4part), i4part_floats(s)}
+                               : Int4Scratch{nullptr, nullptr, nullptr};
+  Int4Scratch scr_routed = scr, scr_shared = scr;
+  if (int4) {
+    scr_routed.src_x = x;
+    scr_routed.src_T = s->T;
+    scr_routed.slot_pos = slot;
+    scr_routed.slot_k = s->k;
+    if (s->H_s > 0) {
+      // the shared expert's input copy, written with the routed one: past the R routed rows of the widest
+      // reduction, so that the routed down GEMM's own copy (R rows of H) leaves it intact
+      const long long cols = std::max(s->d, std::max(s->H, s->H_s));
+      scr_shared.xcs = scr.xcs + (size_t)R * (cols / 128);
+      scr_shared.xrs = scr.xrs + R;
+      scr_shared.xq = reinterpret_cast<__half*>(scr.xq) + (size_t)R * cols;
+      scr_shared.prepped = true;
+      scr_routed.also = &scr_shared;
+    }
+  }
+  rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr_routed);
   if (rc) return rc;
   void* ys = nullptr;
   if (s->H_s > 0) {
     ys = ws + L.ys;
     rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
-                         stream, scr);
+                         stream, scr_shared);
     if (rc) return rc;
   }
   return moe_combine(s, yperm, slot, w, ys, out, stream);

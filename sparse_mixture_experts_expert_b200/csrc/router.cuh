@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
         if (STATS) {
           s_p[e] += ez[i] * inv;
           if ((taken >> i) & 1u) s_c[e] += 1;
-        } else {
+        } else if (p_out != nullptr) {   // for the chunk probability sums, when they are wanted
           p_out[(size_t)t * E + e] = ez[i] * inv;
         }
       }
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_router_topk(const float* part, i
 #pragma unroll 8
     for (int w = 0; w < NW; ++w) { ps += s_stat[(size_t)w * E + e]; cs += s_c0[(size_t)w * E + e]; }
     cnt[(size_t)e * nchunks + chunk] = cs;
-    psum[(size_t)e * nchunks + chunk] = ps;
+    if (psum != nullptr) psum[(size_t)e * nchunks + chunk] = ps;
   }
 }
 
@@ -1123,7 +1123,7 @@ __global__ void __launch_bounds__(256) k_router_lanes(const __nv_bfloat16* __res
       ps += s_ps[cl * KP + w][e];
       cs += s_cn[cl * KP + w][e];
     }
-    psum[(size_t)e * nchunks + chunk] = ps;
+    if (psum != nullptr) psum[(size_t)e * nchunks + chunk] = ps;
     cnt[(size_t)e * nchunks + chunk] = cs;
   }
 }
@@ -1209,7 +1209,7 @@ __global__ void __launch_bounds__(NW * 32) k_router_fused(const __nv_bfloat16* _
 #pragma unroll
     for (int w = 0; w < NW; ++w) { ps += s_p[w][e]; cs += s_c[w][e]; }
     cnt[(size_t)e * nchunks + chunk] = cs;
-    psum[(size_t)e * nchunks + chunk] = ps;
+    if (psum != nullptr) psum[(size_t)e * nchunks + chunk] = ps;
   }
 }
 
@@ -1357,7 +1357,8 @@ __global__ void __launch_bounds__(256) k_chunk_hist(const int32_t* __restrict__ 
 
 // Chunk tables from per-token routing (small batches): one CTA per chunk of
 // kChunk tokens.  cnt[e][c] by shared-memory integer counts (order-free),
-// psum[e][c] = sum over the chunk's tokens, in token order, of p[t,e].
+// psum[e][c] = sum over the chunk's tokens, in token order, of p[t,e] (skipped
+// when psum is null: no load-balance statistic requested).
 __global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__ topk_idx,
                                                      const float* __restrict__ p, int32_t* __restrict__ cnt,
                                                      float* __restrict__ psum, int T, int E, int k) {
@@ -1370,10 +1371,12 @@ __global__ void __launch_bounds__(256) k_chunk_stats(const int32_t* __restrict__
   for (int i = threadIdx.x; i < nt * k; i += blockDim.x) atomicAdd(&s_h[topk_idx[(size_t)t0 * k + i]], 1);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float ps = 0.f;
-    for (int t = 0; t < nt; ++t) ps += p[(size_t)(t0 + t) * E + e];
     cnt[(size_t)e * gridDim.x + blockIdx.x] = s_h[e];
-    psum[(size_t)e * gridDim.x + blockIdx.x] = ps;
+    if (psum != nullptr) {
+      float ps = 0.f;
+      for (int t = 0; t < nt; ++t) ps += p[(size_t)(t0 + t) * E + e];
+      psum[(size_t)e * gridDim.x + blockIdx.x] = ps;
+    }
   }
 }
 
