@@ -251,6 +251,7 @@ __global__ void __launch_bounds__(1024) k_int4_act_prep(const __nv_bfloat16* __r
 // outstanding.  Each task covers 32 weight rows: the 16 gate rows and the 16
 // matching up rows (gated mode) or 32 consecutive output rows (plain mode).
 constexpr int kI4Warps = 16;
+constexpr int kI4Coarse = 2048;   // entries of the stream kernel's task -> group table
 constexpr int kI4Stages = 3;
 constexpr int kI4SlabBytes = 32 * 128;
 constexpr int kI4Smem = kI4Warps * kI4Stages * kI4SlabBytes;
@@ -267,6 +268,9 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   extern __shared__ __align__(128) uint8_t i4_smem[];
   __shared__ int s_prefix[kMaxGroupsSmem + 1];
+  __shared__ int s_gstart[kMaxGroupsSmem];
+  __shared__ int s_grows[kMaxGroupsSmem];
+  __shared__ unsigned short s_cg[kI4Coarse];   // group of base task i * cstride
   __shared__ __align__(8) uint64_t s_bar[kI4Warps][kI4Stages];
   __shared__ volatile int s_abort[kI4Warps];
   const int lane = lane_id(), warp = warp_id();
@@ -291,6 +295,8 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
     int run = incl - local;
     for (int g = g0; g < g1; ++g) {
       s_prefix[g] = run;
+      s_gstart[g] = single ? 0 : p.group_start[g];
+      s_grows[g] = (int)(single ? p.R : (long long)p.group_rows[g]);
       run += group_tasks(g);
     }
     if (lane == 31) s_prefix[G] = incl;
@@ -301,6 +307,14 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
+  __syncthreads();
+  // coarse task -> group table: entry i holds the group of base task i * cstride, so a lookup is one load
+  // and a short forward scan instead of a binary search over the groups
+  const int cstride = max(1, (s_prefix[G] + kI4Coarse - 1) / kI4Coarse);
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int a = (s_prefix[g] + cstride - 1) / cstride, b = (s_prefix[g + 1] + cstride - 1) / cstride;
+    for (int i = a; i < b; ++i) s_cg[i] = (unsigned short)g;
+  }
   __syncthreads();
 
   const int KS = SPLIT ? p.ksplit : 1;   // compile-time 1 unless the reduction is split
@@ -317,15 +331,12 @@ __global__ void __launch_bounds__(kI4Warps * 32, 1)
   struct TaskPos { int g, o0, n0, n_rows, s, sb, se; long long row0; };
   auto locate = [&](int t) -> TaskPos {
     const int task = SPLIT ? t / KS : t;
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_prefix[mid] <= task) lo = mid; else hi = mid - 1;
-    }
+    int lo = s_cg[task / cstride];   // the last group starting at or before task
+    while (s_prefix[lo + 1] <= task) ++lo;
     TaskPos tp;
     tp.g = lo;
-    tp.row0 = single ? 0 : p.group_start[lo];
-    tp.n_rows = (int)(single ? p.R : (long long)p.group_rows[lo]);
+    tp.row0 = s_gstart[lo];
+    tp.n_rows = s_grows[lo];
     const int nchunks = (tp.n_rows + 7) / 8;
     const int tg = task - s_prefix[lo];
     tp.o0 = (tg / nchunks) * (GLU ? 16 : 32);
