@@ -209,9 +209,6 @@ __global__ void __launch_bounds__(256, 1)
     int stage = 0;
     uint32_t phase = 0;
     long long issued = 0;
-    // gated GEMM: the grouped rows are read by this launch's column tiles and never again, so they leave L2
-    // first and leave room for h, which the down GEMM reads next
-    const uint64_t a_policy = l2_policy_evict_first();
     for (long long tile = unit; tile < total && !__any_sync(0xffffffffu, s_abort); tile += n_units) {
       int g, rows_valid, n0;
       long long row0;
@@ -230,15 +227,13 @@ __global__ void __launch_bounds__(256, 1)
         if (kPair) {
           if (lane == 0) {
             const uint32_t fb = mapa_shared(smem_u32(&bar_full[stage]), 0);
-            if (kGLU) tma_load_2d_pair_hint(a_s, &tmA, fb, kb * kBK, (int)row0, a_policy);
-            else tma_load_2d_pair(a_s, &tmA, fb, kb * kBK, (int)row0);
+            tma_load_2d_pair(a_s, &tmA, fb, kb * kBK, (int)row0);
             const int brow = kGLU ? (crank == 0 ? n0 : p.up_row0 + n0) : n0 + crank * (BN / 2);
             tma_load_3d_pair(b_s, &tmB, fb, kb * kBK, brow, g);
             if (kScreen) tma_load_3d_pair(b_s + Cfg::kBBox, &tmB, fb, p.K + kb * kBK, brow, g);
           }
         } else if (lane == 0) {
-          if (kGLU) tma_load_2d_hint(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0, a_policy);
-          else tma_load_2d(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0);
+          tma_load_2d(a_s, &tmA, &bar_full[stage], kb * kBK, (int)row0);
           if (kGLU) {
             tma_load_3d(b_s, &tmB, &bar_full[stage], kb * kBK, n0, g);
             tma_load_3d(b_s + BOXB * 128, &tmB, &bar_full[stage], kb * kBK, p.up_row0 + n0, g);
@@ -327,7 +322,6 @@ __global__ void __launch_bounds__(256, 1)
     __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem + (size_t)S * Cfg::kStageBytes) + q * 32 * kEpiRow;
     int acc = 0;
     uint32_t acc_phase = 0;
-    const uint64_t h_policy = l2_policy_evict_last();   // gated GEMM: h stays in L2 for the down GEMM
     // accumulator release: each thread (single CTA) or each warp on the leader's barrier (pair)
     auto release_acc = [&](int a) {
       tc_fence_before();
@@ -425,8 +419,7 @@ __global__ void __launch_bounds__(256, 1)
             const int rr = it * RPI + lane / LPR;
             if (q * 32 + rr < rows_valid && col < p.N) {
               const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * kEpiRow + cb);
-              if (kGLU) st_global_v4_hint(p.out + (row0 + q * 32 + rr) * p.ldo + col, val, h_policy);
-              else *reinterpret_cast<uint4*>(p.out + (row0 + q * 32 + rr) * p.ldo + col) = val;
+              *reinterpret_cast<uint4*>(p.out + (row0 + q * 32 + rr) * p.ldo + col) = val;
             }
           }
           __syncwarp();
