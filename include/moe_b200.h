@@ -219,6 +219,9 @@ int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos,
  *   out        [T, d] bf16     out
  *   topk_idx, topk_w, counts, drop_mask, aux_f, aux_p, aux: optional outputs (NULL = not returned)
  *   workspace  >= moe_workspace_size() bytes of device memory, 256-byte aligned
+ * INT4 experts: the activations are scaled per row by a power of two and rounded to f16 (exact for bf16
+ * inputs from 2^-28 of the row's largest |x| up); the weights enter the MMAs as exact f16 integer codes
+ * with a per-group offset that is removed in fp32, and the bf16 group scales multiply the fp32 group sums.
  */
 int moe_forward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
                 const void* s13, const void* w2, const void* s2, const void* w13_sh, const void* s13_sh,
