@@ -39,7 +39,7 @@ DEFAULT_WORKLOAD = "granular"
 # -k regex:k_grouped_gemm -s 5 -c 5` capture of `bench.py --workload <name> --steps 1 --warmup 1
 # --no-cpu-baseline` on the current kernels; workloads without a complete capture report null.
 GEMM_TRAFFIC_BYTES = {"small": 12628736 + 21004032,
-                      "granular": (380195584 + 152007424 + 51951872 + 34377216) + (56189184 + 151253248 + 5779456 + 4224256)}
+                      "granular": (380192256 + 151918592 + 51950848 + 34377472) + (55830784 + 150960896 + 5970432 + 4317440)}
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
