@@ -550,7 +550,7 @@ def _int4_forward(moe, wl, seed=0):
     return inp, r
 
 
-def _check_int4_forward(wl, inp, r, sample, seed=0):
+def _check_int4_forward(wl, inp, r, sample, seed=0, cap=0):
     """Oracle output of the sampled tokens, one expert at a time: each touched expert's fp32 draw is quantised
     and dequantised by the oracle, applied to the sampled tokens that chose it, then released (the whole
     decode layer in float64 would not fit in host memory).  The oracle work of several experts runs on a thread
@@ -564,12 +564,21 @@ def _check_int4_forward(wl, inp, r, sample, seed=0):
     idx = npi(r["topk_idx"])
     amb = O.topk_margin(ref["z"], wl.k) < MARGIN
     assert (idx[~amb] == ref["idx"][~amb]).all()
+    drop = np.zeros((wl.T, wl.k), bool)
+    if cap:
+        # with a capacity every later drop decision depends on every routing decision: the seeded cases
+        # have no near-ties, so the whole routing must agree, and then the drops bit for bit
+        assert (idx == ref["idx"]).all()
+        drop = O.permute(ref["idx"], wl.E, cap)["drop"].astype(bool)
+        assert (npi(r["drop_mask"]).astype(bool) == drop).all()
+        assert drop.any()
     toks = np.array([t for t in sample if (idx[t] == ref["idx"][t]).all()], np.int64)
     sel = ref["idx"][toks]                                  # [n, k]
     users = {}                                              # expert -> [(row in toks, slot j)]
     for n in range(toks.size):
         for j in range(wl.k):
-            users.setdefault(int(sel[n, j]), []).append((n, j))
+            if not drop[toks[n], j]:
+                users.setdefault(int(sel[n, j]), []).append((n, j))
     if wl.H_s:
         users[wl.E] = [(n, -1) for n in range(toks.size)]   # the shared expert, weight one
 
@@ -603,6 +612,17 @@ def test_forward_int4_reduced(lib, T):
     wl = synth.get_workload("decode_int4").replace(T=T, d=1024, E=48, H=256, H_s=256)
     inp, r = _int4_forward(lib, wl)
     _check_int4_forward(wl, inp, r, sample=list(range(wl.T)))
+
+
+# Capacity drops (the grouped activation copy skips dropped slots) and hidden widths above d (the shared
+# expert's activation copy sits past the routed rows of the widest reduction), every token against the oracle.
+@pytest.mark.parametrize("over", [{"T": 100, "d": 1024, "E": 48, "H": 256, "H_s": 256, "capacity_factor": 0.5},
+                                  {"T": 64, "d": 512, "E": 32, "H": 1024, "H_s": 1024}])
+def test_forward_int4_capacity_and_wide_hidden(lib, over):
+    wl = synth.get_workload("decode_int4").replace(**over)
+    cap = O.capacity(wl.T, wl.k, wl.E, wl.capacity_factor) if wl.capacity_factor else 0
+    inp, r = _int4_forward(lib, wl)
+    _check_int4_forward(wl, inp, r, sample=list(range(wl.T)), cap=cap)
 
 
 def test_forward_int4_full_size(lib):
