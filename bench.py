@@ -365,6 +365,69 @@ def cpu_oracle_sample(wl, budget_s=12.0, single_thread=False):
 # ------------------------------------------------------------------ main
 
 
+def run_ep(args, wl, world, rank, device):
+    """Expert-parallel timing: rank r holds experts [r E/N, (r + 1) E/N) and its own T tokens (weak scaling);
+    moe_forward_ep runs eagerly (its splits reach the host), L2 flushed before every step, the step time is
+    the max over ranks of the mean device time between events around each forward."""
+    import socket
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_expert_b200 as moe
+    import synth
+    from sparse_mixture_experts_expert_b200.ep import moe_forward_ep
+    if wl.capacity_factor or wl.wfmt != synth.WFMT_BF16 or wl.E % world:
+        raise SystemExit("--ep takes bf16 workloads without a capacity whose experts split evenly over the ranks")
+    own = not dist.is_initialized()
+    if own:   # one rank: a process group of one, the exchanges are local copies
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=timedelta(seconds=120), device_id=device)
+    s, inp, _, _ = setup(wl, rank, device)
+    E_loc = wl.E // world
+    mine = slice(rank * E_loc, (rank + 1) * E_loc)
+    w13, w2 = inp["w13"][mine].contiguous(), inp["w2"][mine].contiguous()
+    flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def step():
+        return moe_forward_ep(s, inp["x"], inp["w_router"], w13, w2, bias=inp["bias"], w13_sh=inp.get("w13_sh"),
+                              w2_sh=inp.get("w2_sh"))
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for a, b in evs:
+            flushbuf.fill_(1)
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+    dist.barrier()
+    status, site = moe.moe_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    if rank == 0:
+        cfg = bench_config(wl, 0, world)
+        cfg["parallelism"] = f"expert-parallel x{world} (E/N experts per rank, NCCL all-to-all-v)"
+        print(json.dumps({"metric": METRIC, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                          "data": "synthetic", "config": cfg, "mode": "expert-parallel",
+                          "clocks": clk.summary()}), flush=True)
+    if own:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -373,6 +436,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert-parallel forward instead of replicas: each of the N ranks holds E / N experts and "
+                         "T tokens; the rows travel by NCCL all-to-all-v (bf16 workloads without a capacity)")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: run the workload with this many experts (a small case for ncu); the "
                          "line's config names it")
@@ -424,6 +490,9 @@ def main():
     else:
         torch.cuda.set_device(0)
     device = torch.device("cuda", torch.cuda.current_device())
+    if args.ep:
+        run_ep(args, wl, world, rank, device)
+        return
     s, inp, ws, out = setup(wl, rank, device)
     flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
 

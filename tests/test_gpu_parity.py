@@ -632,3 +632,49 @@ def test_forward_int4_full_size(lib):
     inp, r = _int4_forward(lib, wl)
     n = _check_int4_forward(wl, inp, r, sample=list(range(wl.T)))
     assert n >= wl.T - 2
+
+
+# ---------------------------------------------------------------- expert parallelism
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("granular", {"T": 2048, "skew": 1.2, "capacity_factor": 0.0}),
+                                       ("small", {})])
+def test_expert_parallel_single_rank_equals_forward(lib, name, over):
+    """moe_forward_ep on one NCCL rank (the exchanges are identities) runs the same kernels on the same grouped
+    rows as moe_forward, so the outputs agree bit for bit; the two-rank exchange is covered on gloo (CPU)."""
+    import socket
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    from sparse_mixture_experts_expert_b200.ep import moe_forward_ep
+    moe = lib
+    own = not dist.is_initialized()
+    if own:
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=timedelta(seconds=60),
+                                device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        _ep_single_rank_case(moe, moe_forward_ep, name, over)
+    finally:
+        if own:
+            dist.destroy_process_group()
+
+
+def _ep_single_rank_case(moe, moe_forward_ep, name, over):
+    wl = synth.get_workload(name).replace(**over)
+    inp = synth.make_inputs(wl, seed=5, device=DEV)
+    s = shape_of(moe, wl)
+    assert s.capacity == 0
+    ref = moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
+                          w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), routing=True)
+    out, idx, w = moe_forward_ep(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
+                                 w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"))
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    assert torch.equal(idx, ref["topk_idx"])
+    assert torch.equal(out, ref["out"])
