@@ -287,6 +287,83 @@ def moe_forward(x, w_router, bias, w13, w2, *, k: int, act: int = ACT_SWIGLU, re
     return res
 
 
+# ---------------------------------------------------------------- backward: the input gradient
+# Training is the setting of p1 (kieve-moe Features: the load-balancing auxiliary loss), p2 (MoEEvolve
+# Architecture) and p5 (MoEFFN.forward, "Load balancing loss").  The input gradient of
+# L = sum(dout * out) + aux_coef * aux follows the forward above by the chain rule.  The routing decision (the
+# top-k and the capacity drops) is piecewise constant in x and passes no gradient; the gate values and the
+# softmax do.  The count fractions f_e of the statistic are counts, also constant.
+
+def silu_grad(z):
+    """d/dz of z sigmoid(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))."""
+    z = np.asarray(z, np.float64)
+    s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def gelu_erf_grad(z):
+    """d/dz of z Phi(z) = Phi(z) + z phi(z), with the standard normal cdf Phi and density phi."""
+    z = np.asarray(z, np.float64)
+    return 0.5 * (1.0 + _erf(z / math.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+
+
+def expert_ffn_backward_x(x, w13, w2, act: int, dy) -> np.ndarray:
+    """dL/dx of y = (act(x W1^T) * (x W3^T)) W2^T given dy = dL/dy; x, dy [n, d], w13 [2H, d], w2 [d, H]."""
+    x = np.asarray(x, np.float64)
+    w13 = np.asarray(w13, np.float64)
+    H = w13.shape[0] // 2
+    w1, w3 = w13[:H], w13[H:]
+    g, u = x @ w1.T, x @ w3.T
+    dh = np.asarray(dy, np.float64) @ np.asarray(w2, np.float64)
+    a = silu(g) if act == ACT_SWIGLU else gelu_erf(g)
+    da = silu_grad(g) if act == ACT_SWIGLU else gelu_erf_grad(g)
+    return (dh * u * da) @ w1 + (dh * a) @ w3
+
+
+def moe_backward_x(x, w_router, bias, w13, w2, dout, *, k: int, act: int = ACT_SWIGLU, renorm: bool = True,
+                   cap: int = 0, w13_sh=None, w2_sh=None, aux_coef: float = 0.0):
+    """dL/dx [T, d] of L = sum(dout * out) + aux_coef * aux for the layer of moe_forward.
+
+    Parts: the routed experts (each kept slot: w_tj times the expert's input gradient of dout_t), the shared
+    expert, and the router: dw_tj = <dout_t, y_{e_tj}(x_t)> on kept slots -> the gate derivative (renorm:
+    w_j = p_j / S) -> dp on the selected experts, plus aux_coef E f_e / T on every expert (P_e = mean_t p) ->
+    through the softmax, dz = p (dp - <p, dp>) -> dz W_r.  Returns a dict with dx and the intermediates.
+    """
+    x = np.asarray(x, np.float64)
+    dout = np.asarray(dout, np.float64)
+    fw = moe_forward(x, w_router, bias, w13, w2, k=k, act=act, renorm=renorm, cap=cap, w13_sh=w13_sh,
+                     w2_sh=w2_sh)
+    T = x.shape[0]
+    E = np.asarray(w_router).shape[0]
+    idx, w, p, slot = fw["idx"], fw["w"], fw["p"], fw["slot_pos"]
+    dx = np.zeros_like(x)
+    dw = np.zeros((T, k))
+    for e in range(E):
+        tj = np.argwhere((idx == e) & (slot >= 0))
+        if tj.size == 0:
+            continue
+        t, j = tj[:, 0], tj[:, 1]
+        dx_e = expert_ffn_backward_x(x[t], np.asarray(w13[e]), np.asarray(w2[e]), act, w[t, j, None] * dout[t])
+        np.add.at(dx, t, dx_e)
+        dw[t, j] = np.sum(dout[t] * fw["y_perm"][slot[t, j]], axis=1)
+    if w13_sh is not None:
+        dx += expert_ffn_backward_x(x, np.asarray(w13_sh)[0], np.asarray(w2_sh)[0], act, dout)
+    psel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    if renorm:
+        S = psel.sum(axis=1, keepdims=True)
+        dpsel = (dw - np.sum(dw * w, axis=1, keepdims=True)) / S
+    else:
+        dpsel = dw
+    dp = np.zeros((T, E))
+    np.add.at(dp, (np.repeat(np.arange(T), k), idx.astype(np.int64).ravel()), dpsel.ravel())
+    if aux_coef:
+        f = fw["counts"] / T
+        dp += aux_coef * E * f[None, :] / T
+    dz = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+    dx += dz @ np.asarray(w_router, np.float64)
+    return dict(dx=dx, dw=dw, dz=dz, forward=fw)
+
+
 def dense_moe_forward(x, w13, w2, idx, w, drop=None, *, act: int = ACT_SWIGLU, w13_sh=None, w2_sh=None):
     """Dense evaluation: every expert on every token, mixed by the masked gate matrix.
 
