@@ -21,6 +21,7 @@ hidden 256, shared expert 512, capacity factor 1.25).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -428,6 +429,72 @@ def run_ep(args, wl, world, rank, device):
         dist.destroy_process_group()
 
 
+def run_backward(args, wl, world, rank, device):
+    """Backward timing: one moe_backward_x (forward recompute + input gradient) captured as a CUDA graph and
+    replayed per step, L2 flushed before every step; tokens/s and the bf16 GEMM work over the step time."""
+    import torch
+
+    import sparse_mixture_experts_expert_b200 as moe
+    import synth
+    if wl.wfmt != synth.WFMT_BF16:
+        raise SystemExit("--backward takes bf16 workloads")
+    s, inp, _, _ = setup(wl, rank, device)
+    g = torch.Generator(device=device).manual_seed(1234 + rank)
+    dout = torch.randn(wl.T, wl.d, generator=g, device=device).to(torch.bfloat16)
+    t13, t2 = moe.moe_transpose_experts(inp["w13"]), moe.moe_transpose_experts(inp["w2"])
+    t13s = moe.moe_transpose_experts(inp["w13_sh"]) if wl.H_s else None
+    t2s = moe.moe_transpose_experts(inp["w2_sh"]) if wl.H_s else None
+    n = ctypes.c_size_t(0)
+    moe.load().moe_backward_workspace_size(ctypes.byref(s), ctypes.byref(n))
+    ws = torch.empty(int(n.value), dtype=torch.uint8, device=device)
+
+    def step():
+        return moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
+                                  w13t=t13, w2t=t2, w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"),
+                                  w13t_sh=t13s, w2t_sh=t2s, aux_coef=0.01, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    launches0 = moe.moe_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    per_step = moe.moe_launch_count() - launches0
+    flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for a, b in evs:
+            flushbuf.fill_(1)
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize()
+    status, site = moe.moe_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    R = s.R
+    ldE = (wl.E + 63) // 64 * 64
+    # bf16 GEMM work: recompute [g | u], h, y; dh, dx of the grouped rows; shared [g | u], dh, dx; router dz W_r
+    flops = 2.0 * R * (wl.d * 2 * wl.H * 2 + wl.H * wl.d * 2 + 2 * wl.H * wl.d) \
+        + 2.0 * wl.T * (wl.d * 2 * wl.H_s + wl.d * wl.H_s + 2 * wl.H_s * wl.d) + 2.0 * wl.T * ldE * wl.d
+    peaks = load_peaks()
+    if rank == 0:
+        print(json.dumps({"metric": "MoE-layer input-gradient backward tokens/s on 1 B200; % of bf16 tensor-core roofline",
+                          "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                          "config": bench_config(wl, s.capacity, world), "mode": "backward (input gradient)",
+                          "roofline": {"bound": "tensor", "kernel": "whole moe_backward_x",
+                                       "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                                       "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                       "peak_source": peaks["source"] + " burst bf16", "alg_flops_per_step": flops},
+                          "gpu_launches": per_step * args.steps, "clocks": clk.summary()}), flush=True)
+    del graph
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,6 +506,8 @@ def main():
     ap.add_argument("--ep", action="store_true",
                     help="expert-parallel forward instead of replicas: each of the N ranks holds E / N experts and "
                          "T tokens; the rows travel by NCCL all-to-all-v (bf16 workloads without a capacity)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the input-gradient backward (moe_backward_x, bf16 experts) instead of the forward")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: run the workload with this many experts (a small case for ncu); the "
                          "line's config names it")
@@ -492,6 +561,9 @@ def main():
     device = torch.device("cuda", torch.cuda.current_device())
     if args.ep:
         run_ep(args, wl, world, rank, device)
+        return
+    if args.backward:
+        run_backward(args, wl, world, rank, device)
         return
     s, inp, ws, out = setup(wl, rank, device)
     flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)

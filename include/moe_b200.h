@@ -230,6 +230,38 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
                 size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Transposed copies of expert weights for the backward pass: wt[i][c][r] = w[i][r][c] for i < n, bf16.
+ *   w   [n, rows, cols] in, wt [n, cols, rows] out (caller-owned device memory); n <= 65535.
+ * For moe_backward_x: w13t = transpose of w13 ([E, d, 2H]), w2t = transpose of w2 ([E, H, d]), and the same
+ * for the shared expert (n = 1).
+ */
+int moe_transpose_experts(const void* w, int64_t n, int32_t rows, int32_t cols, void* wt, moe_stream_t stream);
+
+/* Scratch bytes moe_backward_x needs for this shape. */
+int moe_backward_workspace_size(const moe_shape* s, size_t* bytes);
+
+/*
+ * Input gradient of the layer (training is the setting of kieve-moe Features, the MoEEvolve README and
+ * MoEFFN.forward): dx = dL/dx for L = sum(dout * out) + aux_coef * aux, out as moe_forward computes it.
+ * The routing decision (top-k, capacity drops) passes no gradient; the gate values, their renormalisation,
+ * the softmax and the load-balance statistic aux = E sum_e f_e P_e (f_e counts, constant) do.  The forward's
+ * routing, grouping and expert activations are recomputed here.  bf16 experts only (MOE_UNSUPPORTED_SHAPE
+ * for INT4).
+ *   x, w_router, bias, w13, w2, w13_sh, w2_sh   as moe_forward
+ *   w13t, w2t, w13t_sh, w2t_sh                  their transposes (moe_transpose_experts)
+ *   dout      [T, d] bf16   in   dL/dout
+ *   aux_coef                     weight of the statistic in L (0: none)
+ *   dx        [T, d] fp32   out
+ *   workspace >= moe_backward_workspace_size() bytes, 256-byte aligned
+ * Precision: the expert steps run as bf16 GEMMs with fp32 accumulation (dy, dh, [dg | du] and the recomputed
+ * [g | u] rounded to bf16); the router's dz W_r takes bf16 operands.  dx sums its parts in fp32.
+ */
+int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                   const void* w2, const void* w13t, const void* w2t, const void* w13_sh, const void* w2_sh,
+                   const void* w13t_sh, const void* w2t_sh, const void* dout, float aux_coef, float* dx,
+                   void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Group-scaled signed INT4 quantiser (ExpertMesh README: signed INT4 weights
  * with group scales).  For each row of w [rows, K] fp32 (K % 128 == 0) and
  * each group of 128 inputs: s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7)

@@ -30,7 +30,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_INVALID_ARGUMENT", 2: "MOE_UNSUPPORTED_SHAPE", 3:
 EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route", "moe_route_from_logits",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
             "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
-            "moe_permute_noalloc"]
+            "moe_permute_noalloc", "moe_transpose_experts", "moe_backward_workspace_size", "moe_backward_x"]
 
 
 class MoeError(RuntimeError):
@@ -87,6 +87,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_launch_count": (u64, []),
         "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "moe_permute_noalloc": (ctypes.c_int, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "moe_transpose_experts": (ctypes.c_int, [_P, i64, i32, i32, _P, _P]),
+        "moe_backward_workspace_size": (ctypes.c_int, [S, ctypes.POINTER(sz)]),
+        "moe_backward_x": (ctypes.c_int, [S] + [_P] * 12 + [ctypes.c_float, _P, _P, sz, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -309,6 +312,40 @@ def moe_forward(shape: MoeShape, x, w_router, w13, w2, *, bias=None, s13=None, s
         r["out"] = out
         return r
     return out
+
+
+def moe_transpose_experts(w, *, out=None, stream=None):
+    """[n, rows, cols] bf16 -> [n, cols, rows] bf16 (the transposed expert weights moe_backward_x takes)."""
+    n, rows, cols = w.shape
+    _want(w, torch.bfloat16, (n, rows, cols), "w")
+    if out is None:
+        out = torch.empty(n, cols, rows, dtype=torch.bfloat16, device=w.device)
+    _check(_L().moe_transpose_experts(_ptr(w), n, rows, cols, _ptr(out), _stream(stream)), "moe_transpose_experts")
+    return out
+
+
+def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
+                   w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
+    """Input gradient dL/dx [T, d] fp32 of L = sum(dout * out) + aux_coef * aux (bf16 experts).  The transposed
+    weights are made here when not given (moe_transpose_experts)."""
+    T, d = shape.T, shape.d
+    _want(x, torch.bfloat16, (T, d), "x")
+    _want(dout, torch.bfloat16, (T, d), "dout")
+    w13t = w13t if w13t is not None else moe_transpose_experts(w13, stream=stream)
+    w2t = w2t if w2t is not None else moe_transpose_experts(w2, stream=stream)
+    if shape.H_s:
+        w13t_sh = w13t_sh if w13t_sh is not None else moe_transpose_experts(w13_sh, stream=stream)
+        w2t_sh = w2t_sh if w2t_sh is not None else moe_transpose_experts(w2_sh, stream=stream)
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        _check(_L().moe_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "moe_backward_workspace_size")
+        ws = torch.empty(int(n.value), dtype=torch.uint8, device=x.device)
+    dx = torch.empty(T, d, dtype=torch.float32, device=x.device)
+    rc = _L().moe_backward_x(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w2),
+                             _ptr(w13t), _ptr(w2t), _ptr(w13_sh), _ptr(w2_sh), _ptr(w13t_sh), _ptr(w2t_sh),
+                             _ptr(dout), float(aux_coef), _ptr(dx), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_backward_x")
+    return dx
 
 
 def moe_quantize_int4(w, *, q=None, scales=None, stream=None):

@@ -1,0 +1,247 @@
+// Input gradient of the layer (bf16 experts).  Training is the setting of the
+// kieve-moe Features (load-balancing auxiliary loss), the MoEEvolve README
+// (Architecture) and MoEFFN.forward in moe_stream.py ("Load balancing loss").
+// For L = sum(dout * out) + aux_coef * aux the chain rule gives, per token t:
+//   dx_t = sum over kept slots j of  w_tj * J_e(x_t)^T dout_t      (routed experts)
+//        + J_shared(x_t)^T dout_t                                  (shared expert)
+//        + W_r^T dz_t                                              (router)
+// with the expert input gradient J^T dy = (dh u act'(g)) W1 + (dh act(g)) W3,
+// dh = dy W2, and the router part: dw_tj = <dout_t, y_e(x_t)> on kept slots,
+// the gate derivative (renormalised gates: (dw_j - sum_i dw_i w_i) / S), the
+// statistic aux = E sum_e f_e P_e (d/dp = E f_e / T per expert, counts fixed),
+// then the softmax: dz = p (dp - <p, dp>).  The routing decision passes no
+// gradient.  The three expert GEMMs (dh, the recomputed activations, dx of the
+// grouped rows) run on k_grouped_gemm with transposed weights; the kernels
+// here are the elementwise and gather steps around them.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace moe {
+
+// wt[n][c][r] = w[n][r][c] (bf16), 32 x 32 tiles through shared memory.  Grid (ceil(cols/32),
+// ceil(rows/32), n), block (32, 8).
+__global__ void __launch_bounds__(256) k_transpose_bf16(const __nv_bfloat16* __restrict__ w,
+                                                        __nv_bfloat16* __restrict__ wt, int rows, int cols) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  __shared__ __nv_bfloat16 tile[32][34];
+  const size_t base = (size_t)blockIdx.z * rows * cols;
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = blockIdx.y * 32 + i;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = w[base + (size_t)r * cols + c];
+  }
+  __syncthreads();
+  const int r = blockIdx.y * 32 + threadIdx.x;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int cc = blockIdx.x * 32 + i;
+    if (cc < cols && r < rows) wt[base + (size_t)cc * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+// W_r [E][d] fp32 -> W_r^T [d][ldE] bf16 (the B operand of dx_router = dz W_r), zeros in columns E .. ldE.
+// Same tiling, grid (ceil(d/32), ceil(ldE/32)).
+__global__ void __launch_bounds__(256) k_transpose_router(const float* __restrict__ w, __nv_bfloat16* __restrict__ wt,
+                                                          int E, int d, int ldE) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  __shared__ float tile[32][33];
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int e = blockIdx.y * 32 + i;
+    tile[i][threadIdx.x] = (e < E && c < d) ? w[(size_t)e * d + c] : 0.f;
+  }
+  __syncthreads();
+  const int e = blockIdx.y * 32 + threadIdx.x;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int cc = blockIdx.x * 32 + i;
+    if (cc < d && e < ldE) wt[(size_t)cc * ldE + e] = __float2bfloat16_rn(e < E ? tile[threadIdx.x][i] : 0.f);
+  }
+}
+
+// Per (token, slot), one warp per token: dy_perm[slot] = bf16(w_tj * dout_t) and dw_tj = <dout_t, y_perm[slot]>
+// (fp32, lanes over 8-input slices in order, then a fixed xor tree); dropped slots: dw_tj = 0, no row.
+__global__ void __launch_bounds__(256) k_bwd_dispatch(const __nv_bfloat16* __restrict__ dout,
+                                                      const __nv_bfloat16* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ slot_pos,
+                                                      const float* __restrict__ topk_w, int T, int d, int k,
+                                                      __nv_bfloat16* __restrict__ dy_perm, float* __restrict__ dw) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long t = (long long)blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id(), nv = d >> 3;
+  const uint4* drow = reinterpret_cast<const uint4*>(dout + t * d);
+  for (int j = 0; j < k; ++j) {
+    const int slot = slot_pos[t * k + j];
+    if (slot < 0) {
+      if (lane == 0) dw[t * k + j] = 0.f;
+      continue;
+    }
+    const float wj = topk_w[t * k + j];
+    const uint4* yrow = reinterpret_cast<const uint4*>(y_perm + (size_t)slot * d);
+    uint4* orow = reinterpret_cast<uint4*>(dy_perm + (size_t)slot * d);
+    float acc = 0.f;
+    for (int v = lane; v < nv; v += 32) {
+      const uint4 a = drow[v], y = yrow[v];
+      const float av[8] = {bf16lo(a.x), bf16hi(a.x), bf16lo(a.y), bf16hi(a.y),
+                           bf16lo(a.z), bf16hi(a.z), bf16lo(a.w), bf16hi(a.w)};
+      const float yv[8] = {bf16lo(y.x), bf16hi(y.x), bf16lo(y.y), bf16hi(y.y),
+                           bf16lo(y.z), bf16hi(y.z), bf16lo(y.w), bf16hi(y.w)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc = fmaf(av[i], yv[i], acc);
+      orow[v] = make_uint4(pack_bf16x2(wj * av[0], wj * av[1]), pack_bf16x2(wj * av[2], wj * av[3]),
+                           pack_bf16x2(wj * av[4], wj * av[5]), pack_bf16x2(wj * av[6], wj * av[7]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) dw[t * k + j] = acc;
+  }
+}
+
+// d/dz of the activations: SiLU' = s (1 + z (1 - s)); GELU' = Phi(z) + z phi(z) (erf by Abramowitz & Stegun
+// 7.1.26, as in the forward epilogue).
+__device__ __forceinline__ float act_silu_grad(float z) {
+  const float s = __fdividef(1.0f, 1.0f + __expf(-z));
+  return s * (1.0f + z * (1.0f - s));
+}
+__device__ __forceinline__ float act_gelu_grad(float z) {
+  return 0.5f * (1.0f + erf_as7126(z * 0.7071067811865476f)) + z * 0.3989422804014327f * __expf(-0.5f * z * z);
+}
+
+// GLU backward over rows of [g | u] (bf16 pre-activations, g in columns [0, H), u in [H, 2H)) and dh [., H]:
+// in place, gu becomes [dg | du] with dg = dh u act'(g), du = dh act(g).  One thread per 8 columns of a row.
+template <int ACT>
+__global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu, const __nv_bfloat16* __restrict__ dh,
+                                                 long long rows, int H) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nv = H >> 3;
+  if (i >= rows * nv) return;
+  const long long r = i / nv;
+  const int v = (int)(i - r * nv);
+  uint4* g4 = reinterpret_cast<uint4*>(gu + r * 2 * H) + v;
+  uint4* u4 = reinterpret_cast<uint4*>(gu + r * 2 * H + H) + v;
+  const uint4 G = *g4, U = *u4, D = reinterpret_cast<const uint4*>(dh + r * H)[v];
+  const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dw[4] = {D.x, D.y, D.z, D.w};
+  uint32_t og[4], ou[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float dg[2], du[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float g = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
+      const float u = h ? bf16hi(uw[q]) : bf16lo(uw[q]);
+      const float d = h ? bf16hi(dw[q]) : bf16lo(dw[q]);
+      const float a = ACT == kModeSwiGLU ? act_silu(g) : act_gelu(g);
+      const float da = ACT == kModeSwiGLU ? act_silu_grad(g) : act_gelu_grad(g);
+      dg[h] = d * u * da;
+      du[h] = d * a;
+    }
+    og[q] = pack_bf16x2(dg[0], dg[1]);
+    ou[q] = pack_bf16x2(du[0], du[1]);
+  }
+  *g4 = make_uint4(og[0], og[1], og[2], og[3]);
+  *u4 = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+}
+
+// Router backward, one warp per token (lane l: experts l, l + 32, ...): p = softmax(z_t); dp on the selected
+// experts from dw (renormalised gates: (dw_j - sum_i dw_i w_i) / S, S = sum of the selected p); plus
+// aux_coef E counts_e / T^2 on every expert; dz = p (dp - <p, dp>), written as bf16 (the A operand of dz W_r)
+// into rows of ldz >= E columns, zeros past E (the reduction of dz W_r runs over whole 64-column steps).
+template <int EPL>
+__global__ void __launch_bounds__(256) k_router_bwd(const float* __restrict__ z, const int32_t* __restrict__ topk_idx,
+                                                    const float* __restrict__ topk_w, const float* __restrict__ dw,
+                                                    const int32_t* __restrict__ counts, float aux_coef, int T, int E,
+                                                    int k, int renorm, int ldz, __nv_bfloat16* __restrict__ dz) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long t = (long long)blockIdx.x * 8 + warp_id();
+  if (t >= T) return;
+  const int lane = lane_id();
+  float p[EPL], dp[EPL];
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    p[i] = e < E ? z[t * E + e] : -INFINITY;
+    m = fmaxf(m, p[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    p[i] = (lane + 32 * i < E) ? __expf(p[i] - m) : 0.f;
+    sum += p[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = 1.f / sum;
+  const float auxs = aux_coef * (float)E / ((float)T * (float)T);
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    p[i] *= inv;
+    dp[i] = (e < E && aux_coef != 0.f) ? auxs * (float)counts[e] : 0.f;
+  }
+  // gates: S and sum_i dw_i w_i over the token's k slots (the same on every lane)
+  float S = 0.f, dwsum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[t * k + j];
+    float pj = 0.f;   // p of expert e, held by lane e % 32
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) pj = (lane + 32 * i == e) ? p[i] : pj;
+    pj = __shfl_sync(0xffffffffu, pj, e & 31);
+    S += pj;
+    dwsum += dw[t * k + j] * topk_w[t * k + j];
+  }
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[t * k + j];
+    const float dpsel = renorm ? (dw[t * k + j] - dwsum) / S : dw[t * k + j];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (lane + 32 * i == e) dp[i] += dpsel;
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) s = fmaf(p[i], dp[i], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) dz[t * ldz + e] = __float2bfloat16_rn(p[i] * (dp[i] - s));
+  }
+  for (int e = E + lane; e < ldz; e += 32) dz[t * ldz + e] = __float2bfloat16_rn(0.f);
+}
+
+// dx_t = sum over kept slots of dx_perm[slot] + dx_shared_t (if any) + dx_router_t, fp32, one thread per 8
+// columns (slot order, then the shared and router terms).
+__global__ void __launch_bounds__(256) k_bwd_final(const __nv_bfloat16* __restrict__ dx_perm,
+                                                   const int32_t* __restrict__ slot_pos,
+                                                   const __nv_bfloat16* __restrict__ dx_shared,
+                                                   const __nv_bfloat16* __restrict__ dx_router, int T, int d, int k,
+                                                   float* __restrict__ dx) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nv = d >> 3;
+  if (i >= (long long)T * nv) return;
+  const long long t = i / nv;
+  const int v = (int)(i - t * nv);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  auto add = [&](const __nv_bfloat16* row) {
+    const uint4 a = reinterpret_cast<const uint4*>(row)[v];
+    acc[0] += bf16lo(a.x); acc[1] += bf16hi(a.x); acc[2] += bf16lo(a.y); acc[3] += bf16hi(a.y);
+    acc[4] += bf16lo(a.z); acc[5] += bf16hi(a.z); acc[6] += bf16lo(a.w); acc[7] += bf16hi(a.w);
+  };
+  for (int j = 0; j < k; ++j) {
+    const int slot = slot_pos[t * k + j];
+    if (slot >= 0) add(dx_perm + (size_t)slot * d);
+  }
+  if (dx_shared != nullptr) add(dx_shared + t * d);
+  add(dx_router + t * d);
+  float4* o = reinterpret_cast<float4*>(dx + t * d) + 2 * v;
+  o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+}  // namespace moe

@@ -8,6 +8,7 @@
 #include <mutex>
 #include <utility>
 
+#include "backward.cuh"
 #include "common.cuh"
 #include "expert_fused.cuh"
 #include "gemm_tc.cuh"
@@ -881,6 +882,49 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
   return MOE_OK;
 }
 
+
+// ------------------------------------------------------------------ backward (input gradient)
+
+// Scratch of moe_backward_x past the forward's regions (which it reuses: routing, grouping, x_perm for dx of the
+// grouped rows, h for dh, y_perm).
+struct BwdWorkspace {
+  size_t gu, dyp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, total;
+  int ldE;   // columns of dz and W_r^T: E rounded up to whole 64-column reduction steps
+};
+
+static BwdWorkspace bwd_layout(const moe_shape* s) {
+  const Workspace F = ws_layout(s);
+  BwdWorkspace B{};
+  const long long R = grouped_rows(s);
+  size_t o = F.total;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  B.ldE = (int)((s->E + 63) / 64 * 64);
+  B.gu = take((size_t)R * 2 * s->H * 2);
+  B.dyp = take((size_t)R * s->d * 2);
+  B.gus = take((size_t)s->T * 2 * std::max(s->H_s, 16) * 2);
+  B.dhs = take((size_t)s->T * std::max(s->H_s, 16) * 2);
+  B.dxs = take((size_t)s->T * s->d * 2);
+  B.logits = take((size_t)s->T * s->E * 4);
+  B.dw = take((size_t)s->T * s->k * 4);
+  B.dz = take((size_t)s->T * B.ldE * 2);
+  B.wrt = take((size_t)s->d * B.ldE * 2);
+  B.dxr = take((size_t)s->T * s->d * 2);
+  B.total = o;
+  return B;
+}
+
+static int launch_glu_bwd(int act, void* gu, const void* dh, long long rows, int H, cudaStream_t st) {
+  const unsigned blocks = (unsigned)cdiv(rows * (H / 8), 256);
+  if (act == MOE_ACT_SWIGLU)
+    MOE_LAUNCH((k_glu_bwd<kModeSwiGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
+               reinterpret_cast<const __nv_bfloat16*>(dh), rows, H);
+  else
+    MOE_LAUNCH((k_glu_bwd<kModeGeGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
+               reinterpret_cast<const __nv_bfloat16*>(dh), rows, H);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -1094,6 +1138,133 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
     if (rc) return rc;
   }
   return moe_combine(s, yperm, slot, w, ys, out, stream);
+}
+
+int moe_transpose_experts(const void* w, int64_t n, int32_t rows, int32_t cols, void* wt, moe_stream_t stream) {
+  if (!w || !wt || n < 1 || n > 65535 || rows < 1 || cols < 1) return MOE_INVALID_ARGUMENT;
+  const dim3 grid((unsigned)cdiv(cols, 32), (unsigned)cdiv(rows, 32), (unsigned)n);
+  MOE_LAUNCH((k_transpose_bf16), grid, dim3(32, 8), 0, stream, reinterpret_cast<const __nv_bfloat16*>(w),
+             reinterpret_cast<__nv_bfloat16*>(wt), (int)rows, (int)cols);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+int moe_backward_workspace_size(const moe_shape* s, size_t* bytes) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (!bytes) return MOE_INVALID_ARGUMENT;
+  *bytes = bwd_layout(s).total;
+  return MOE_OK;
+}
+
+int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                   const void* w2, const void* w13t, const void* w2t, const void* w13_sh, const void* w2_sh,
+                   const void* w13t_sh, const void* w2t_sh, const void* dout, float aux_coef, float* dx,
+                   void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shape(s);
+  if (rc) return rc;
+  if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
+  if (!x || !w_router || !w13 || !w2 || !w13t || !w2t || !dout || !dx || !workspace) return MOE_INVALID_ARGUMENT;
+  if (s->H_s > 0 && (!w13_sh || !w2_sh || !w13t_sh || !w2t_sh)) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(w13t) ||
+      !aligned16(w2t) || !aligned16(dout) || !aligned16(dx) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return MOE_INVALID_ARGUMENT;
+  const Workspace L = ws_layout(s);
+  const BwdWorkspace B = bwd_layout(s);
+  if (ws_bytes < B.total) return MOE_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = stream;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* cts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* slot = reinterpret_cast<int32_t*>(ws + L.slot);
+  uint8_t* drop = reinterpret_cast<uint8_t*>(ws + L.drop);
+  int32_t* kept = reinterpret_cast<int32_t*>(ws + L.kept);
+  int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offs);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  void* xperm = ws + L.xperm;   // the grouped rows, then dx of the grouped rows
+  void* hbuf = ws + L.h;        // h, then dh
+  void* yperm = ws + L.yperm;
+  void* gu = ws + B.gu;         // [g | u] of the grouped rows, then [dg | du]
+  void* dyp = ws + B.dyp;
+  float* logits = reinterpret_cast<float*>(ws + B.logits);
+  float* dwb = reinterpret_cast<float*>(ws + B.dw);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + B.dz);
+  __nv_bfloat16* wrt = reinterpret_cast<__nv_bfloat16*>(ws + B.wrt);
+  void* dxr = ws + B.dxr;
+  const long long R = grouped_rows(s);
+  const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
+  const int glu_mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
+
+  // forward recompute: routing (with the logits for the softmax), grouping, [g | u], h, y
+  rc = route_impl(s, x, w_router, bias, nullptr, logits, idx, w, cts, nullptr, nullptr, nullptr, ws, st);
+  if (rc) return rc;
+  rc = launch_scatter(s, x, idx, cnt, cts, slot, drop, nullptr, xperm, kept, offs, st, true);
+  if (rc) return rc;
+  rc = grouped_gemm(kModePlain, xperm, R, s->d, w13, s->E, 2 * s->H, 0, 2 * s->H, offs, kept, gu, st, pair);
+  if (rc) return rc;
+  rc = grouped_gemm(glu_mode, xperm, R, s->d, w13, s->E, 2 * s->H, s->H, s->H, offs, kept, hbuf, st, pair);
+  if (rc) return rc;
+  rc = grouped_gemm(kModePlain, hbuf, R, s->H, w2, s->E, s->d, 0, s->d, offs, kept, yperm, st, pair);
+  if (rc) return rc;
+
+  // routed experts: dy of the grouped rows and the gate gradients, dh = dy W2, [dg | du], dx = [dg | du] W13
+  MOE_LAUNCH((k_bwd_dispatch), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(dout),
+             reinterpret_cast<const __nv_bfloat16*>(yperm), slot, w, (int)s->T, s->d, s->k,
+             reinterpret_cast<__nv_bfloat16*>(dyp), dwb);
+  MOE_LAUNCH_CHECK();
+  rc = grouped_gemm(kModePlain, dyp, R, s->d, w2t, s->E, s->H, 0, s->H, offs, kept, hbuf, st, pair);
+  if (rc) return rc;
+  rc = launch_glu_bwd(s->act, gu, hbuf, R, s->H, st);
+  if (rc) return rc;
+  rc = grouped_gemm(kModePlain, gu, R, 2 * s->H, w13t, s->E, s->d, 0, s->d, offs, kept, xperm, st, pair);
+  if (rc) return rc;
+
+  // shared expert on the tokens: [g | u] recomputed, dh = dout W2, [dg | du], dx = [dg | du] W13
+  void* dxs = nullptr;
+  if (s->H_s > 0) {
+    void* gus = ws + B.gus;
+    void* dhs = ws + B.dhs;
+    dxs = ws + B.dxs;
+    rc = grouped_gemm(kModePlain, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, 0, 2 * s->H_s, nullptr, nullptr, gus, st,
+                      pair);
+    if (rc) return rc;
+    rc = grouped_gemm(kModePlain, dout, s->T, s->d, w2t_sh, 1, s->H_s, 0, s->H_s, nullptr, nullptr, dhs, st, pair);
+    if (rc) return rc;
+    rc = launch_glu_bwd(s->act, gus, dhs, s->T, s->H_s, st);
+    if (rc) return rc;
+    rc = grouped_gemm(kModePlain, gus, s->T, 2 * s->H_s, w13t_sh, 1, s->d, 0, s->d, nullptr, nullptr, dxs, st,
+                      pair);
+    if (rc) return rc;
+  }
+
+  // router: dz through the gates, the statistic and the softmax, then dz W_r (bf16 operands, fp32 accumulation)
+  const int epl = (int)cdiv(s->E, 32);
+  const unsigned tb = (unsigned)cdiv(s->T, 8);
+#define MOE_RBWD(N_)                                                                                          \
+  MOE_LAUNCH((k_router_bwd<N_>), tb, 256, 0, st, logits, idx, w, dwb, cts, aux_coef, (int)s->T, s->E, s->k,    \
+             s->renorm, B.ldE, dz)
+  if (epl <= 1) MOE_RBWD(1);
+  else if (epl <= 2) MOE_RBWD(2);
+  else if (epl <= 4) MOE_RBWD(4);
+  else if (epl <= 8) MOE_RBWD(8);
+  else MOE_RBWD(16);
+#undef MOE_RBWD
+  MOE_LAUNCH_CHECK();
+  {
+    const dim3 grid((unsigned)cdiv(s->d, 32), (unsigned)cdiv(B.ldE, 32));
+    MOE_LAUNCH((k_transpose_router), grid, dim3(32, 8), 0, st, w_router, wrt, s->E, s->d, B.ldE);
+    MOE_LAUNCH_CHECK();
+  }
+  rc = grouped_gemm(kModePlain, dz, s->T, B.ldE, wrt, 1, s->d, 0, s->d, nullptr, nullptr, dxr, st, pair);
+  if (rc) return rc;
+
+  // dx = the token's grouped rows (slot order) + the shared expert's part + the router's part, fp32
+  MOE_LAUNCH((k_bwd_final), (unsigned)cdiv(s->T * (long long)(s->d / 8), 256), 256, 0, st,
+             reinterpret_cast<const __nv_bfloat16*>(xperm), slot, reinterpret_cast<const __nv_bfloat16*>(dxs),
+             reinterpret_cast<const __nv_bfloat16*>(dxr), (int)s->T, s->d, s->k, dx);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
 }
 
 int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream) {

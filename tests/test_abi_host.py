@@ -38,6 +38,28 @@ def test_library_exports_every_declared_symbol(L):
     assert sorted(moe.EXPORTED) == names
 
 
+def _declared_arity():
+    """Number of parameters of every declared entry point (from the header's prototypes)."""
+    out = {}
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            for m in re.finditer(r"(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+                params = m.group(2).strip()
+                out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(L):
+    # every ctypes prototype the binding sets takes as many arguments as the header declares
+    arity = _declared_arity()
+    for name in arity:
+        f = getattr(L, name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == arity[name], (name, len(f.argtypes), arity[name])
+
+
 def _shape(moe, **kw):
     base = dict(T=256, d=64, E=8, k=2, H=128)
     base.update(kw)

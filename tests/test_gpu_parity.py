@@ -678,3 +678,75 @@ def _ep_single_rank_case(moe, moe_forward_ep, name, over):
     assert moe.moe_get_status()[0] == 0
     assert torch.equal(idx, ref["topk_idx"])
     assert torch.equal(out, ref["out"])
+
+
+# ---------------------------------------------------------------- backward (input gradient)
+
+# rel-Frobenius bound of dx: the expert steps round dy, dh, the recomputed [g | u], [dg | du] and the grouped dx
+# to bf16 (each about 2^-9 / sqrt(3) = 1.1e-3 relative, independent), and the router's dz W_r rounds both
+# operands: about 2.5e-3 in quadrature, bounded here at 1e-2.
+BWD_REL_FROB = 1e-2
+
+
+@pytest.mark.parametrize("name,over,aux_coef", [("tiny", {}, 0.0),
+                                                ("tiny", {"H_s": 64, "act": 1, "capacity_factor": 0.5}, 0.1),
+                                                ("small", {}, 0.05),
+                                                ("granular", {"T": 1024, "skew": 1.2}, 0.0),
+                                                ("geglu", {"T": 512}, 0.0)])
+def test_backward_x_matches_oracle(lib, name, over, aux_coef):
+    moe = lib
+    wl = synth.get_workload(name).replace(**over)
+    inp = synth.make_inputs(wl, seed=6, device=DEV)
+    s = shape_of(moe, wl)
+    g = torch.Generator(device=DEV).manual_seed(17)
+    dout = torch.randn(wl.T, wl.d, generator=g, device=DEV).to(torch.bfloat16)
+    dx = moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
+                            w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), aux_coef=aux_coef)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref = O.moe_backward_x(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
+                           np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
+                           w13_sh=np64(inp["w13_sh"]) if wl.H_s else None,
+                           w2_sh=np64(inp["w2_sh"]) if wl.H_s else None, aux_coef=aux_coef)
+    # the routing must agree (the seeded cases have no near-ties): the gradient is taken at the same decision
+    r = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"])
+    assert (npi(r["topk_idx"]) == ref["forward"]["idx"]).all()
+    got, want = np64(dx), ref["dx"]
+    rel = rel_frob(got, want)
+    print(f"{name}: rel-Frobenius {rel:.2e}, max|d| {np.abs(got - want).max():.2e}, max|dx| {np.abs(want).max():.2e}")
+    assert rel <= BWD_REL_FROB
+    assert np.isfinite(got).all()
+    # each part of dx is far above the bound, so dropping one would fail: the router (dz W_r) and the shared expert
+    router = ref["dz"] @ np64(inp["w_router"])
+    assert rel_frob(want - router, want) > 5 * BWD_REL_FROB
+    if wl.H_s:
+        sh = O.expert_ffn_backward_x(np64(inp["x"]), np64(inp["w13_sh"])[0], np64(inp["w2_sh"])[0], wl.act, np64(dout))
+        assert rel_frob(want - sh, want) > 5 * BWD_REL_FROB
+
+
+# The load-balance term alone (dout = 0, so L = aux_coef * aux): dx = W_r^T dz with dp = aux_coef E f_e / T; a
+# uniform f has no effect through the softmax, so the routing is skewed.
+@pytest.mark.parametrize("name,over", [("tiny", {"skew": 1.2}), ("granular", {"T": 1024, "skew": 1.2})])
+def test_backward_x_load_balance_term_alone(lib, name, over):
+    moe = lib
+    wl = synth.get_workload(name).replace(**over)
+    inp = synth.make_inputs(wl, seed=6, device=DEV)
+    s = shape_of(moe, wl)
+    dout = torch.zeros(wl.T, wl.d, dtype=torch.bfloat16, device=DEV)
+    dx = moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
+                            w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), aux_coef=1.0)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref = O.moe_backward_x(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
+                           np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
+                           w13_sh=np64(inp["w13_sh"]) if wl.H_s else None,
+                           w2_sh=np64(inp["w2_sh"]) if wl.H_s else None, aux_coef=1.0)
+    r = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"])
+    assert (npi(r["topk_idx"]) == ref["forward"]["idx"]).all()
+    want = ref["dx"]
+    assert np.abs(want).max() > 0
+    rel = rel_frob(np64(dx), want)
+    print(f"{name}: load-balance term alone, rel-Frobenius {rel:.2e}")
+    assert rel <= BWD_REL_FROB
