@@ -287,10 +287,10 @@ def moe_forward(x, w_router, bias, w13, w2, *, k: int, act: int = ACT_SWIGLU, re
     return res
 
 
-# ---------------------------------------------------------------- backward: the input gradient
+# ---------------------------------------------------------------- backward: input and weight gradients
 # Training is the setting of p1 (kieve-moe Features: the load-balancing auxiliary loss), p2 (MoEEvolve
-# Architecture) and p5 (MoEFFN.forward, "Load balancing loss").  The input gradient of
-# L = sum(dout * out) + aux_coef * aux follows the forward above by the chain rule.  The routing decision (the
+# Architecture) and p5 (MoEFFN.forward, "Load balancing loss").  The gradients of
+# L = sum(dout * out) + aux_coef * aux follow the forward above by the chain rule.  The routing decision (the
 # top-k and the capacity drops) is piecewise constant in x and passes no gradient; the gate values and the
 # softmax do.  The count fractions f_e of the statistic are counts, also constant.
 
@@ -320,14 +320,34 @@ def expert_ffn_backward_x(x, w13, w2, act: int, dy) -> np.ndarray:
     return (dh * u * da) @ w1 + (dh * a) @ w3
 
 
-def moe_backward_x(x, w_router, bias, w13, w2, dout, *, k: int, act: int = ACT_SWIGLU, renorm: bool = True,
-                   cap: int = 0, w13_sh=None, w2_sh=None, aux_coef: float = 0.0):
-    """dL/dx [T, d] of L = sum(dout * out) + aux_coef * aux for the layer of moe_forward.
+def expert_ffn_backward_weights(x, w13, w2, act: int, dy):
+    """Weight gradients of y = (act(x W1^T) * (x W3^T)) W2^T given dy = dL/dy, summed over the rows:
+    dW2 = dy^T h [d, H] with h = act(g) u; dW1 = (dh u act'(g))^T x and dW3 = (dh act(g))^T x, stacked as
+    dW13 [2H, d] like w13.  x, dy [n, d], w13 [2H, d], w2 [d, H]."""
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    w13 = np.asarray(w13, np.float64)
+    H = w13.shape[0] // 2
+    g, u = x @ w13[:H].T, x @ w13[H:].T
+    a = silu(g) if act == ACT_SWIGLU else gelu_erf(g)
+    da = silu_grad(g) if act == ACT_SWIGLU else gelu_erf_grad(g)
+    dh = dy @ np.asarray(w2, np.float64)
+    dw2 = dy.T @ (a * u)
+    dw13 = np.concatenate([(dh * u * da).T @ x, (dh * a).T @ x], axis=0)
+    return dw13, dw2
 
-    Parts: the routed experts (each kept slot: w_tj times the expert's input gradient of dout_t), the shared
-    expert, and the router: dw_tj = <dout_t, y_{e_tj}(x_t)> on kept slots -> the gate derivative (renorm:
-    w_j = p_j / S) -> dp on the selected experts, plus aux_coef E f_e / T on every expert (P_e = mean_t p) ->
-    through the softmax, dz = p (dp - <p, dp>) -> dz W_r.  Returns a dict with dx and the intermediates.
+
+def moe_backward(x, w_router, bias, w13, w2, dout, *, k: int, act: int = ACT_SWIGLU, renorm: bool = True,
+                 cap: int = 0, w13_sh=None, w2_sh=None, aux_coef: float = 0.0):
+    """Gradients of L = sum(dout * out) + aux_coef * aux for the layer of moe_forward: dx [T, d] and the
+    weight gradients dw13 [E, 2H, d], dw2 [E, d, H], dw13_sh [1, 2H_s, d], dw2_sh [1, d, H_s] (None without a
+    shared expert) and dw_router [E, d].  The exploration bias added to the logits is taken as a constant.
+
+    Parts of dx: the routed experts (each kept slot: w_tj times the expert's input gradient of dout_t), the
+    shared expert, and the router: dw_tj = <dout_t, y_{e_tj}(x_t)> on kept slots -> the gate derivative
+    (renorm: w_j = p_j / S) -> dp on the selected experts, plus aux_coef E f_e / T on every expert
+    (P_e = mean_t p) -> through the softmax, dz = p (dp - <p, dp>) -> dz W_r.  Each expert's weight gradient
+    sums its kept rows with dy = w_tj dout_t; dW_r = dz^T x.  Returns a dict with these and the intermediates.
     """
     x = np.asarray(x, np.float64)
     dout = np.asarray(dout, np.float64)
@@ -338,16 +358,23 @@ def moe_backward_x(x, w_router, bias, w13, w2, dout, *, k: int, act: int = ACT_S
     idx, w, p, slot = fw["idx"], fw["w"], fw["p"], fw["slot_pos"]
     dx = np.zeros_like(x)
     dw = np.zeros((T, k))
+    dw13 = np.zeros(np.shape(w13), np.float64)
+    dw2 = np.zeros(np.shape(w2), np.float64)
     for e in range(E):
         tj = np.argwhere((idx == e) & (slot >= 0))
         if tj.size == 0:
             continue
         t, j = tj[:, 0], tj[:, 1]
-        dx_e = expert_ffn_backward_x(x[t], np.asarray(w13[e]), np.asarray(w2[e]), act, w[t, j, None] * dout[t])
+        dy_e = w[t, j, None] * dout[t]
+        dx_e = expert_ffn_backward_x(x[t], np.asarray(w13[e]), np.asarray(w2[e]), act, dy_e)
         np.add.at(dx, t, dx_e)
+        dw13[e], dw2[e] = expert_ffn_backward_weights(x[t], w13[e], w2[e], act, dy_e)
         dw[t, j] = np.sum(dout[t] * fw["y_perm"][slot[t, j]], axis=1)
+    dw13_sh = dw2_sh = None
     if w13_sh is not None:
         dx += expert_ffn_backward_x(x, np.asarray(w13_sh)[0], np.asarray(w2_sh)[0], act, dout)
+        g13, g2 = expert_ffn_backward_weights(x, np.asarray(w13_sh)[0], np.asarray(w2_sh)[0], act, dout)
+        dw13_sh, dw2_sh = g13[None], g2[None]
     psel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     if renorm:
         S = psel.sum(axis=1, keepdims=True)
@@ -361,7 +388,8 @@ def moe_backward_x(x, w_router, bias, w13, w2, dout, *, k: int, act: int = ACT_S
         dp += aux_coef * E * f[None, :] / T
     dz = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
     dx += dz @ np.asarray(w_router, np.float64)
-    return dict(dx=dx, dw=dw, dz=dz, forward=fw)
+    return dict(dx=dx, dw13=dw13, dw2=dw2, dw13_sh=dw13_sh, dw2_sh=dw2_sh, dw_router=dz.T @ x, dw=dw, dz=dz,
+                forward=fw)
 
 
 def dense_moe_forward(x, w13, w2, idx, w, drop=None, *, act: int = ACT_SWIGLU, w13_sh=None, w2_sh=None):

@@ -705,7 +705,7 @@ def test_backward_x_matches_oracle(lib, name, over, aux_coef):
     torch.cuda.synchronize()
     assert moe.moe_get_status()[0] == 0
     b64 = np64(inp["bias"]) if inp["bias"] is not None else None
-    ref = O.moe_backward_x(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
+    ref = O.moe_backward(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
                            np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
                            w13_sh=np64(inp["w13_sh"]) if wl.H_s else None,
                            w2_sh=np64(inp["w2_sh"]) if wl.H_s else None, aux_coef=aux_coef)
@@ -739,7 +739,7 @@ def test_backward_x_load_balance_term_alone(lib, name, over):
     torch.cuda.synchronize()
     assert moe.moe_get_status()[0] == 0
     b64 = np64(inp["bias"]) if inp["bias"] is not None else None
-    ref = O.moe_backward_x(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
+    ref = O.moe_backward(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
                            np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
                            w13_sh=np64(inp["w13_sh"]) if wl.H_s else None,
                            w2_sh=np64(inp["w2_sh"]) if wl.H_s else None, aux_coef=1.0)
