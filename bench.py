@@ -475,11 +475,11 @@ def run_backward(args, wl, world, rank, device):
     if status != 0:
         raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
-    R = s.R
-    ldE = (wl.E + 63) // 64 * 64
-    # bf16 GEMM work: recompute [g | u], h, y; dh, dx of the grouped rows; shared [g | u], dh, dx; router dz W_r
-    flops = 2.0 * R * (wl.d * 2 * wl.H * 2 + wl.H * wl.d * 2 + 2 * wl.H * wl.d) \
-        + 2.0 * wl.T * (wl.d * 2 * wl.H_s + wl.d * wl.H_s + 2 * wl.H_s * wl.d) + 2.0 * wl.T * ldE * wl.d
+    # bf16 GEMM work per row: the recomputed [g | u] (2 H d), dout W2 (H d), dx = [dg | du] W13 (2 H d), for the
+    # kept grouped rows and the shared expert's tokens; the router's dz W_r (E d per token)
+    kept = int(moe.moe_permute(s, inp["x"], moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"])["topk_idx"])
+               ["kept"].sum())
+    flops = 2.0 * 5 * (kept * wl.H + wl.T * wl.H_s) * wl.d + 2.0 * wl.T * wl.E * wl.d
     peaks = load_peaks()
     if rank == 0:
         print(json.dumps({"metric": "MoE-layer input-gradient backward tokens/s on 1 B200; % of bf16 tensor-core roofline",

@@ -245,21 +245,24 @@ int moe_backward_workspace_size(const moe_shape* s, size_t* bytes);
  * MoEFFN.forward): dx = dL/dx for L = sum(dout * out) + aux_coef * aux, out as moe_forward computes it.
  * The routing decision (top-k, capacity drops) passes no gradient; the gate values, their renormalisation,
  * the softmax and the load-balance statistic aux = E sum_e f_e P_e (f_e counts, constant) do.  The forward's
- * routing, grouping and expert activations are recomputed here.  bf16 experts only (MOE_UNSUPPORTED_SHAPE
- * for INT4).
- *   x, w_router, bias, w13, w2, w13_sh, w2_sh   as moe_forward
- *   w13t, w2t, w13t_sh, w2t_sh                  their transposes (moe_transpose_experts)
+ * routing, grouping and [g | u] are recomputed here; h and y are not (the gate gradient <dout, y> is taken as
+ * <act(g) u, dout W2>).  bf16 experts only (MOE_UNSUPPORTED_SHAPE for INT4).
+ *   x, w_router, bias, w13, w13_sh   as moe_forward (w13_sh NULL when H_s == 0)
+ *   w13t, w2t, w13t_sh, w2t_sh       transposes of w13, w2, w13_sh, w2_sh (moe_transpose_experts); the down
+ *                                    projections enter only through these
  *   dout      [T, d] bf16   in   dL/dout
  *   aux_coef                     weight of the statistic in L (0: none)
  *   dx        [T, d] fp32   out
  *   workspace >= moe_backward_workspace_size() bytes, 256-byte aligned
- * Precision: the expert steps run as bf16 GEMMs with fp32 accumulation (dy, dh, [dg | du] and the recomputed
+ * Precision: the expert steps run as bf16 GEMMs with fp32 accumulation (dout W2, [dg | du] and the recomputed
  * [g | u] rounded to bf16); the router's dz W_r takes bf16 operands.  dx sums its parts in fp32.
+ * Errors: MOE_INVALID_ARGUMENT for a NULL or misaligned pointer, MOE_WORKSPACE_TOO_SMALL, a shape error as
+ * moe_forward; nothing is enqueued then.
  */
 int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
-                   const void* w2, const void* w13t, const void* w2t, const void* w13_sh, const void* w2_sh,
-                   const void* w13t_sh, const void* w2t_sh, const void* dout, float aux_coef, float* dx,
-                   void* workspace, size_t ws_bytes, moe_stream_t stream);
+                   const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
+                   const void* dout, float aux_coef, float* dx, void* workspace, size_t ws_bytes,
+                   moe_stream_t stream);
 
 /*
  * Group-scaled signed INT4 quantiser (ExpertMesh README: signed INT4 weights

@@ -89,7 +89,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute_noalloc": (ctypes.c_int, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moe_transpose_experts": (ctypes.c_int, [_P, i64, i32, i32, _P, _P]),
         "moe_backward_workspace_size": (ctypes.c_int, [S, ctypes.POINTER(sz)]),
-        "moe_backward_x": (ctypes.c_int, [S] + [_P] * 12 + [ctypes.c_float, _P, _P, sz, _P]),
+        "moe_backward_x": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float, _P, _P, sz, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -327,7 +327,7 @@ def moe_transpose_experts(w, *, out=None, stream=None):
 def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
                    w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
     """Input gradient dL/dx [T, d] fp32 of L = sum(dout * out) + aux_coef * aux (bf16 experts).  The transposed
-    weights are made here when not given (moe_transpose_experts)."""
+    weights are made here when not given (moe_transpose_experts); the down projections enter only transposed."""
     T, d = shape.T, shape.d
     _want(x, torch.bfloat16, (T, d), "x")
     _want(dout, torch.bfloat16, (T, d), "dout")
@@ -341,9 +341,9 @@ def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w1
         _check(_L().moe_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "moe_backward_workspace_size")
         ws = torch.empty(int(n.value), dtype=torch.uint8, device=x.device)
     dx = torch.empty(T, d, dtype=torch.float32, device=x.device)
-    rc = _L().moe_backward_x(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w2),
-                             _ptr(w13t), _ptr(w2t), _ptr(w13_sh), _ptr(w2_sh), _ptr(w13t_sh), _ptr(w2t_sh),
-                             _ptr(dout), float(aux_coef), _ptr(dx), _ptr(ws), ws.numel(), _stream(stream))
+    rc = _L().moe_backward_x(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w13t),
+                             _ptr(w2t), _ptr(w13_sh), _ptr(w13t_sh), _ptr(w2t_sh), _ptr(dout), float(aux_coef),
+                             _ptr(dx), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "moe_backward_x")
     return dx
 

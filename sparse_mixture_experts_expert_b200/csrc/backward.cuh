@@ -10,9 +10,10 @@
 // the gate derivative (renormalised gates: (dw_j - sum_i dw_i w_i) / S), the
 // statistic aux = E sum_e f_e P_e (d/dp = E f_e / T per expert, counts fixed),
 // then the softmax: dz = p (dp - <p, dp>).  The routing decision passes no
-// gradient.  The three expert GEMMs (dh, the recomputed activations, dx of the
-// grouped rows) run on k_grouped_gemm with transposed weights; the kernels
-// here are the elementwise and gather steps around them.
+// gradient.  Per routed row three GEMMs run on k_grouped_gemm: the recomputed
+// [g | u] = x W13^T, dh' = dout W2 (unscaled; dh = w dh') and dx = [dg | du] W13
+// (transposed weights).  The gate gradient needs no h or y: <dout, y> equals
+// <act(g) u, dh'>.  The kernels here are the elementwise and gather steps.
 #pragma once
 
 #include "common.cuh"
@@ -56,45 +57,6 @@ __global__ void __launch_bounds__(256) k_transpose_router(const float* __restric
   for (int i = threadIdx.y; i < 32; i += 8) {
     const int cc = blockIdx.x * 32 + i;
     if (cc < d && e < ldE) wt[(size_t)cc * ldE + e] = __float2bfloat16_rn(e < E ? tile[threadIdx.x][i] : 0.f);
-  }
-}
-
-// Per (token, slot), one warp per token: dy_perm[slot] = bf16(w_tj * dout_t) and dw_tj = <dout_t, y_perm[slot]>
-// (fp32, lanes over 8-input slices in order, then a fixed xor tree); dropped slots: dw_tj = 0, no row.
-__global__ void __launch_bounds__(256) k_bwd_dispatch(const __nv_bfloat16* __restrict__ dout,
-                                                      const __nv_bfloat16* __restrict__ y_perm,
-                                                      const int32_t* __restrict__ slot_pos,
-                                                      const float* __restrict__ topk_w, int T, int d, int k,
-                                                      __nv_bfloat16* __restrict__ dy_perm, float* __restrict__ dw) {
-  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  const long long t = (long long)blockIdx.x * 8 + warp_id();
-  if (t >= T) return;
-  const int lane = lane_id(), nv = d >> 3;
-  const uint4* drow = reinterpret_cast<const uint4*>(dout + t * d);
-  for (int j = 0; j < k; ++j) {
-    const int slot = slot_pos[t * k + j];
-    if (slot < 0) {
-      if (lane == 0) dw[t * k + j] = 0.f;
-      continue;
-    }
-    const float wj = topk_w[t * k + j];
-    const uint4* yrow = reinterpret_cast<const uint4*>(y_perm + (size_t)slot * d);
-    uint4* orow = reinterpret_cast<uint4*>(dy_perm + (size_t)slot * d);
-    float acc = 0.f;
-    for (int v = lane; v < nv; v += 32) {
-      const uint4 a = drow[v], y = yrow[v];
-      const float av[8] = {bf16lo(a.x), bf16hi(a.x), bf16lo(a.y), bf16hi(a.y),
-                           bf16lo(a.z), bf16hi(a.z), bf16lo(a.w), bf16hi(a.w)};
-      const float yv[8] = {bf16lo(y.x), bf16hi(y.x), bf16lo(y.y), bf16hi(y.y),
-                           bf16lo(y.z), bf16hi(y.z), bf16lo(y.w), bf16hi(y.w)};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(av[i], yv[i], acc);
-      orow[v] = make_uint4(pack_bf16x2(wj * av[0], wj * av[1]), pack_bf16x2(wj * av[2], wj * av[3]),
-                           pack_bf16x2(wj * av[4], wj * av[5]), pack_bf16x2(wj * av[6], wj * av[7]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) dw[t * k + j] = acc;
   }
 }
 
@@ -142,6 +104,62 @@ __global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu,
   }
   *g4 = make_uint4(og[0], og[1], og[2], og[3]);
   *u4 = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+}
+
+// GLU backward of the routed rows with the gate gradients, one warp per (token, slot) i = t k + j with grouped row
+// r = slot_pos[i]: from dh'_r = dout_t W2 (unscaled, bf16) and [g | u]_r, dw_tj = <act(g) u, dh'_r>, which is
+// <dout_t, y_e(x_t)> since y = (act(g) u) W2^T, so neither h nor y is recomputed; then dh = w_tj dh' and
+// gu_r becomes [dh u act'(g) | dh act(g)] in place.  Dropped slots: dw_tj = 0.  Lanes take 8-column slices in
+// order, then a fixed xor tree.
+template <int ACT>
+__global__ void __launch_bounds__(256) k_glu_bwd_slots(__nv_bfloat16* __restrict__ gu,
+                                                       const __nv_bfloat16* __restrict__ dhp,
+                                                       const int32_t* __restrict__ slot_pos,
+                                                       const float* __restrict__ topk_w, long long n_slots, int H,
+                                                       float* __restrict__ dw) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long i = (long long)blockIdx.x * 8 + warp_id();
+  if (i >= n_slots) return;
+  const int lane = lane_id();
+  const int row = slot_pos[i];
+  if (row < 0) {
+    if (lane == 0) dw[i] = 0.f;
+    return;
+  }
+  const float wj = topk_w[i];
+  const int nv = H >> 3;
+  uint4* g4 = reinterpret_cast<uint4*>(gu + (size_t)row * 2 * H);
+  uint4* u4 = g4 + nv;
+  const uint4* d4 = reinterpret_cast<const uint4*>(dhp + (size_t)row * H);
+  float acc = 0.f;
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 G = g4[v], U = u4[v], D = d4[v];
+    const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dv[4] = {D.x, D.y, D.z, D.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float dg[2], du[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float g = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
+        const float u = h ? bf16hi(uw[q]) : bf16lo(uw[q]);
+        const float d = h ? bf16hi(dv[q]) : bf16lo(dv[q]);
+        const float a = ACT == kModeSwiGLU ? act_silu(g) : act_gelu(g);
+        const float da = ACT == kModeSwiGLU ? act_silu_grad(g) : act_gelu_grad(g);
+        acc = fmaf(a * u, d, acc);
+        const float dh = wj * d;
+        dg[h] = dh * u * da;
+        du[h] = dh * a;
+      }
+      og[q] = pack_bf16x2(dg[0], dg[1]);
+      ou[q] = pack_bf16x2(du[0], du[1]);
+    }
+    g4[v] = make_uint4(og[0], og[1], og[2], og[3]);
+    u4[v] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) dw[i] = acc;
 }
 
 // Router backward, one warp per token (lane l: experts l, l + 32, ...): p = softmax(z_t); dp on the selected

@@ -886,9 +886,9 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
 // ------------------------------------------------------------------ backward (input gradient)
 
 // Scratch of moe_backward_x past the forward's regions (which it reuses: routing, grouping, x_perm for dx of the
-// grouped rows, h for dh, y_perm).
+// grouped rows, h for dh').
 struct BwdWorkspace {
-  size_t gu, dyp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, total;
+  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, total;
   int ldE;   // columns of dz and W_r^T: E rounded up to whole 64-column reduction steps
 };
 
@@ -900,7 +900,7 @@ static BwdWorkspace bwd_layout(const moe_shape* s) {
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
   B.ldE = (int)((s->E + 63) / 64 * 64);
   B.gu = take((size_t)R * 2 * s->H * 2);
-  B.dyp = take((size_t)R * s->d * 2);
+  B.doutp = take((size_t)R * s->d * 2);
   B.gus = take((size_t)s->T * 2 * std::max(s->H_s, 16) * 2);
   B.dhs = take((size_t)s->T * std::max(s->H_s, 16) * 2);
   B.dxs = take((size_t)s->T * s->d * 2);
@@ -921,6 +921,33 @@ static int launch_glu_bwd(int act, void* gu, const void* dh, long long rows, int
   else
     MOE_LAUNCH((k_glu_bwd<kModeGeGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
                reinterpret_cast<const __nv_bfloat16*>(dh), rows, H);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+static int launch_glu_bwd_slots(int act, void* gu, const void* dhp, const int32_t* slot, const float* w,
+                                long long n_slots, int H, float* dw, cudaStream_t st) {
+  const unsigned blocks = (unsigned)cdiv(n_slots, 8);
+  if (act == MOE_ACT_SWIGLU)
+    MOE_LAUNCH((k_glu_bwd_slots<kModeSwiGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
+               reinterpret_cast<const __nv_bfloat16*>(dhp), slot, w, n_slots, H, dw);
+  else
+    MOE_LAUNCH((k_glu_bwd_slots<kModeGeGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
+               reinterpret_cast<const __nv_bfloat16*>(dhp), slot, w, n_slots, H, dw);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+// Copy row t of src to the grouped row of each of its kept slots (the row move of the dispatch, for any [T, d]
+// bf16 tensor).
+static int launch_move_rows(const moe_shape* s, const void* src, const int32_t* slot, void* dst, cudaStream_t st) {
+  const unsigned blocks = (unsigned)cdiv(s->T * (long long)(s->d / 8), 256);
+  const __nv_bfloat16* a = reinterpret_cast<const __nv_bfloat16*>(src);
+  __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(dst);
+  if (s->k <= 2) MOE_LAUNCH((k_move_rows<2>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
+  else if (s->k <= 4) MOE_LAUNCH((k_move_rows<4>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
+  else if (s->k <= 8) MOE_LAUNCH((k_move_rows<8>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
+  else MOE_LAUNCH((k_move_rows<16>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -1158,15 +1185,15 @@ int moe_backward_workspace_size(const moe_shape* s, size_t* bytes) {
 }
 
 int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
-                   const void* w2, const void* w13t, const void* w2t, const void* w13_sh, const void* w2_sh,
-                   const void* w13t_sh, const void* w2t_sh, const void* dout, float aux_coef, float* dx,
-                   void* workspace, size_t ws_bytes, moe_stream_t stream) {
+                   const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
+                   const void* dout, float aux_coef, float* dx, void* workspace, size_t ws_bytes,
+                   moe_stream_t stream) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
-  if (!x || !w_router || !w13 || !w2 || !w13t || !w2t || !dout || !dx || !workspace) return MOE_INVALID_ARGUMENT;
-  if (s->H_s > 0 && (!w13_sh || !w2_sh || !w13t_sh || !w2t_sh)) return MOE_INVALID_ARGUMENT;
-  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w2) || !aligned16(w13t) ||
+  if (!x || !w_router || !w13 || !w13t || !w2t || !dout || !dx || !workspace) return MOE_INVALID_ARGUMENT;
+  if (s->H_s > 0 && (!w13_sh || !w13t_sh || !w2t_sh)) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w13t) ||
       !aligned16(w2t) || !aligned16(dout) || !aligned16(dx) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return MOE_INVALID_ARGUMENT;
   const Workspace L = ws_layout(s);
@@ -1183,10 +1210,9 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
   int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offs);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   void* xperm = ws + L.xperm;   // the grouped rows, then dx of the grouped rows
-  void* hbuf = ws + L.h;        // h, then dh
-  void* yperm = ws + L.yperm;
+  void* hbuf = ws + L.h;        // dh' = dout W2 of the grouped rows
   void* gu = ws + B.gu;         // [g | u] of the grouped rows, then [dg | du]
-  void* dyp = ws + B.dyp;
+  void* doutp = ws + B.doutp;   // dout of the grouped rows
   float* logits = reinterpret_cast<float*>(ws + B.logits);
   float* dwb = reinterpret_cast<float*>(ws + B.dw);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + B.dz);
@@ -1194,28 +1220,22 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
   void* dxr = ws + B.dxr;
   const long long R = grouped_rows(s);
   const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
-  const int glu_mode = s->act == MOE_ACT_SWIGLU ? kModeSwiGLU : kModeGeGLU;
 
-  // forward recompute: routing (with the logits for the softmax), grouping, [g | u], h, y
+  // forward recompute: routing (with the logits for the softmax), grouping, [g | u]
   rc = route_impl(s, x, w_router, bias, nullptr, logits, idx, w, cts, nullptr, nullptr, nullptr, ws, st);
   if (rc) return rc;
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop, nullptr, xperm, kept, offs, st, true);
   if (rc) return rc;
   rc = grouped_gemm(kModePlain, xperm, R, s->d, w13, s->E, 2 * s->H, 0, 2 * s->H, offs, kept, gu, st, pair);
   if (rc) return rc;
-  rc = grouped_gemm(glu_mode, xperm, R, s->d, w13, s->E, 2 * s->H, s->H, s->H, offs, kept, hbuf, st, pair);
-  if (rc) return rc;
-  rc = grouped_gemm(kModePlain, hbuf, R, s->H, w2, s->E, s->d, 0, s->d, offs, kept, yperm, st, pair);
-  if (rc) return rc;
 
-  // routed experts: dy of the grouped rows and the gate gradients, dh = dy W2, [dg | du], dx = [dg | du] W13
-  MOE_LAUNCH((k_bwd_dispatch), (unsigned)cdiv(s->T, 8), 256, 0, st, reinterpret_cast<const __nv_bfloat16*>(dout),
-             reinterpret_cast<const __nv_bfloat16*>(yperm), slot, w, (int)s->T, s->d, s->k,
-             reinterpret_cast<__nv_bfloat16*>(dyp), dwb);
-  MOE_LAUNCH_CHECK();
-  rc = grouped_gemm(kModePlain, dyp, R, s->d, w2t, s->E, s->H, 0, s->H, offs, kept, hbuf, st, pair);
+  // routed experts: dout of the grouped rows, dh' = dout W2, the gate gradients and [dg | du] (dh = w dh'),
+  // dx = [dg | du] W13
+  rc = launch_move_rows(s, dout, slot, doutp, st);
   if (rc) return rc;
-  rc = launch_glu_bwd(s->act, gu, hbuf, R, s->H, st);
+  rc = grouped_gemm(kModePlain, doutp, R, s->d, w2t, s->E, s->H, 0, s->H, offs, kept, hbuf, st, pair);
+  if (rc) return rc;
+  rc = launch_glu_bwd_slots(s->act, gu, hbuf, slot, w, s->T * (long long)s->k, s->H, dwb, st);
   if (rc) return rc;
   rc = grouped_gemm(kModePlain, gu, R, 2 * s->H, w13t, s->E, s->d, 0, s->d, offs, kept, xperm, st, pair);
   if (rc) return rc;
