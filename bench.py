@@ -430,8 +430,8 @@ def run_ep(args, wl, world, rank, device):
 
 
 def run_backward(args, wl, world, rank, device):
-    """Backward timing: one moe_backward_x (forward recompute + input gradient) captured as a CUDA graph and
-    replayed per step, L2 flushed before every step; tokens/s and the bf16 GEMM work over the step time."""
+    """Backward timing: one moe_backward (forward recompute, input and weight gradients) captured as a CUDA graph
+    and replayed per step, L2 flushed before every step; tokens/s and the bf16 GEMM work over the step time."""
     import torch
 
     import sparse_mixture_experts_expert_b200 as moe
@@ -449,9 +449,9 @@ def run_backward(args, wl, world, rank, device):
     ws = torch.empty(int(n.value), dtype=torch.uint8, device=device)
 
     def step():
-        return moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
-                                  w13t=t13, w2t=t2, w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"),
-                                  w13t_sh=t13s, w2t_sh=t2s, aux_coef=0.01, ws=ws)
+        return moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
+                                w13t=t13, w2t=t2, w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"),
+                                w13t_sh=t13s, w2t_sh=t2s, aux_coef=0.01, ws=ws)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -475,19 +475,21 @@ def run_backward(args, wl, world, rank, device):
     if status != 0:
         raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
-    # bf16 GEMM work per row: the recomputed [g | u] (2 H d), dout W2 (H d), dx = [dg | du] W13 (2 H d), for the
-    # kept grouped rows and the shared expert's tokens; the router's dz W_r (E d per token)
+    # bf16 GEMM work per row: the recomputed [g | u] (2 H d), dout W2 (H d), dx = [dg | du] W13 (2 H d), the
+    # weight gradients dW13 (2 H d) and dW2 (H d), for the kept grouped rows and the shared expert's tokens;
+    # the router's dz W_r and dW_r (E d each per token)
     kept = int(moe.moe_permute(s, inp["x"], moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"])["topk_idx"])
                ["kept"].sum())
-    flops = 2.0 * 5 * (kept * wl.H + wl.T * wl.H_s) * wl.d + 2.0 * wl.T * wl.E * wl.d
+    flops = 2.0 * 8 * (kept * wl.H + wl.T * wl.H_s) * wl.d + 2.0 * 2 * wl.T * wl.E * wl.d
     peaks = load_peaks()
     if rank == 0:
-        print(json.dumps({"metric": "MoE-layer input-gradient backward tokens/s on 1 B200; % of bf16 tensor-core roofline",
+        metric = "MoE-layer backward (input and weight gradients) tokens/s on 1 B200; % of bf16 tensor-core roofline"
+        print(json.dumps({"metric": metric,
                           "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                          "config": bench_config(wl, s.capacity, world), "mode": "backward (input gradient)",
-                          "roofline": {"bound": "tensor", "kernel": "whole moe_backward_x",
+                          "config": bench_config(wl, s.capacity, world), "mode": "backward (input and weight gradients)",
+                          "roofline": {"bound": "tensor", "kernel": "whole moe_backward",
                                        "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
                                        "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                                        "peak_source": peaks["source"] + " burst bf16", "alg_flops_per_step": flops},
@@ -507,7 +509,8 @@ def main():
                     help="expert-parallel forward instead of replicas: each of the N ranks holds E / N experts and "
                          "T tokens; the rows travel by NCCL all-to-all-v (bf16 workloads without a capacity)")
     ap.add_argument("--backward", action="store_true",
-                    help="time the input-gradient backward (moe_backward_x, bf16 experts) instead of the forward")
+                    help="time the backward (moe_backward: input and weight gradients, bf16 experts) instead of the "
+                         "forward")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: run the workload with this many experts (a small case for ncu); the "
                          "line's config names it")

@@ -265,6 +265,26 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
                    moe_stream_t stream);
 
 /*
+ * The input gradient of moe_backward_x and the weight gradients of the same L (training: kieve-moe Features,
+ * the MoEEvolve README Architecture, MoEFFN.forward), fp32, each summed over its rows:
+ *   dw13      [E, 2H, d]    out  per expert, [dg | du]^T x over the expert's kept (token, slot) rows, with
+ *                                dy = w_tj dout_t (dg = dh u act'(g), du = dh act(g), dh = dy W2)
+ *   dw2       [E, d, H]     out  per expert, dy^T h over the same rows (h = act(g) u)
+ *   dw13_sh   [1, 2H_s, d], dw2_sh [1, d, H_s]   out  the shared expert's, over all tokens with dy = dout
+ *   dw_router [E, d]        out  dz^T x (dz = dL/dz of the logits, as in moe_backward_x)
+ * Any weight-gradient pointer may be NULL: that gradient is not computed.  The exploration bias is a constant
+ * here (its gradient would be the column sums of dz).  Other arguments, workspace and errors as
+ * moe_backward_x (the same moe_backward_workspace_size covers both).
+ * Precision: the weight gradients are bf16 GEMMs with fp32 accumulation over the rows of [dg | du], x,
+ * dout, w h (bf16) and dz (bf16); a dense gradient (shared expert, router) sums row chunks in a fixed order.
+ * Experts without kept rows get zeros.
+ */
+int moe_backward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                 const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
+                 const void* dout, float aux_coef, float* dx, float* dw13, float* dw2, float* dw13_sh,
+                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Group-scaled signed INT4 quantiser (ExpertMesh README: signed INT4 weights
  * with group scales).  For each row of w [rows, K] fp32 (K % 128 == 0) and
  * each group of 128 inputs: s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7)

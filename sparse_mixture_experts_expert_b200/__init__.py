@@ -30,7 +30,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_INVALID_ARGUMENT", 2: "MOE_UNSUPPORTED_SHAPE", 3:
 EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route", "moe_route_from_logits",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
             "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
-            "moe_permute_noalloc", "moe_transpose_experts", "moe_backward_workspace_size", "moe_backward_x"]
+            "moe_permute_noalloc", "moe_transpose_experts", "moe_backward_workspace_size", "moe_backward_x",
+            "moe_backward"]
 
 
 class MoeError(RuntimeError):
@@ -90,6 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_transpose_experts": (ctypes.c_int, [_P, i64, i32, i32, _P, _P]),
         "moe_backward_workspace_size": (ctypes.c_int, [S, ctypes.POINTER(sz)]),
         "moe_backward_x": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float, _P, _P, sz, _P]),
+        "moe_backward": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float] + [_P] * 7 + [sz, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -324,28 +326,50 @@ def moe_transpose_experts(w, *, out=None, stream=None):
     return out
 
 
-def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
-                   w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
-    """Input gradient dL/dx [T, d] fp32 of L = sum(dout * out) + aux_coef * aux (bf16 experts).  The transposed
-    weights are made here when not given (moe_transpose_experts); the down projections enter only transposed."""
-    T, d = shape.T, shape.d
+def _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef, ws,
+              stream, weights):
+    T, d, E, H, Hs = shape.T, shape.d, shape.E, shape.H, shape.H_s
     _want(x, torch.bfloat16, (T, d), "x")
     _want(dout, torch.bfloat16, (T, d), "dout")
     w13t = w13t if w13t is not None else moe_transpose_experts(w13, stream=stream)
     w2t = w2t if w2t is not None else moe_transpose_experts(w2, stream=stream)
-    if shape.H_s:
+    if Hs:
         w13t_sh = w13t_sh if w13t_sh is not None else moe_transpose_experts(w13_sh, stream=stream)
         w2t_sh = w2t_sh if w2t_sh is not None else moe_transpose_experts(w2_sh, stream=stream)
     if ws is None:
         n = ctypes.c_size_t(0)
         _check(_L().moe_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)), "moe_backward_workspace_size")
         ws = torch.empty(int(n.value), dtype=torch.uint8, device=x.device)
-    dx = torch.empty(T, d, dtype=torch.float32, device=x.device)
-    rc = _L().moe_backward_x(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w13t),
-                             _ptr(w2t), _ptr(w13_sh), _ptr(w13t_sh), _ptr(w2t_sh), _ptr(dout), float(aux_coef),
-                             _ptr(dx), _ptr(ws), ws.numel(), _stream(stream))
-    _check(rc, "moe_backward_x")
-    return dx
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = dict(dx=torch.empty(T, d, **f32))
+    head = [ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w13), _ptr(w13t), _ptr(w2t),
+            _ptr(w13_sh), _ptr(w13t_sh), _ptr(w2t_sh), _ptr(dout), float(aux_coef), _ptr(g["dx"])]
+    tail = [_ptr(ws), ws.numel(), _stream(stream)]
+    if not weights:
+        _check(_L().moe_backward_x(*head, *tail), "moe_backward_x")
+        return g
+    g.update(dw13=torch.empty(E, 2 * H, d, **f32), dw2=torch.empty(E, d, H, **f32),
+             dw13_sh=torch.empty(1, 2 * Hs, d, **f32) if Hs else None,
+             dw2_sh=torch.empty(1, d, Hs, **f32) if Hs else None, dw_router=torch.empty(E, d, **f32))
+    _check(_L().moe_backward(*head, _ptr(g["dw13"]), _ptr(g["dw2"]), _ptr(g["dw13_sh"]), _ptr(g["dw2_sh"]),
+                             _ptr(g["dw_router"]), *tail), "moe_backward")
+    return g
+
+
+def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
+                   w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
+    """Input gradient dL/dx [T, d] fp32 of L = sum(dout * out) + aux_coef * aux (bf16 experts).  The transposed
+    weights are made here when not given (moe_transpose_experts); the down projections enter only transposed."""
+    return _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef,
+                     ws, stream, False)["dx"]
+
+
+def moe_backward(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
+                 w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
+    """All gradients of L = sum(dout * out) + aux_coef * aux: a dict of fp32 tensors dx [T, d], dw13 [E, 2H, d],
+    dw2 [E, d, H], dw13_sh [1, 2H_s, d] and dw2_sh [1, d, H_s] (None without a shared expert), dw_router [E, d]."""
+    return _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef,
+                     ws, stream, True)
 
 
 def moe_quantize_int4(w, *, q=None, scales=None, stream=None):

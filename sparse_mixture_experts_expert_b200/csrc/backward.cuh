@@ -71,10 +71,11 @@ __device__ __forceinline__ float act_gelu_grad(float z) {
 }
 
 // GLU backward over rows of [g | u] (bf16 pre-activations, g in columns [0, H), u in [H, 2H)) and dh [., H]:
-// in place, gu becomes [dg | du] with dg = dh u act'(g), du = dh act(g).  One thread per 8 columns of a row.
+// in place, gu becomes [dg | du] with dg = dh u act'(g), du = dh act(g); with write_h, h = act(g) u (bf16)
+// replaces dh.  One thread per 8 columns of a row.
 template <int ACT>
-__global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu, const __nv_bfloat16* __restrict__ dh,
-                                                 long long rows, int H) {
+__global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu, __nv_bfloat16* __restrict__ dh,
+                                                 long long rows, int H, int write_h) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int nv = H >> 3;
@@ -83,12 +84,13 @@ __global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu,
   const int v = (int)(i - r * nv);
   uint4* g4 = reinterpret_cast<uint4*>(gu + r * 2 * H) + v;
   uint4* u4 = reinterpret_cast<uint4*>(gu + r * 2 * H + H) + v;
-  const uint4 G = *g4, U = *u4, D = reinterpret_cast<const uint4*>(dh + r * H)[v];
+  uint4* d4 = reinterpret_cast<uint4*>(dh + r * H) + v;
+  const uint4 G = *g4, U = *u4, D = *d4;
   const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dw[4] = {D.x, D.y, D.z, D.w};
-  uint32_t og[4], ou[4];
+  uint32_t og[4], ou[4], oh[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    float dg[2], du[2];
+    float dg[2], du[2], hh[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const float g = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
@@ -98,25 +100,28 @@ __global__ void __launch_bounds__(256) k_glu_bwd(__nv_bfloat16* __restrict__ gu,
       const float da = ACT == kModeSwiGLU ? act_silu_grad(g) : act_gelu_grad(g);
       dg[h] = d * u * da;
       du[h] = d * a;
+      hh[h] = a * u;
     }
     og[q] = pack_bf16x2(dg[0], dg[1]);
     ou[q] = pack_bf16x2(du[0], du[1]);
+    oh[q] = pack_bf16x2(hh[0], hh[1]);
   }
   *g4 = make_uint4(og[0], og[1], og[2], og[3]);
   *u4 = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+  if (write_h) *d4 = make_uint4(oh[0], oh[1], oh[2], oh[3]);
 }
 
 // GLU backward of the routed rows with the gate gradients, one warp per (token, slot) i = t k + j with grouped row
 // r = slot_pos[i]: from dh'_r = dout_t W2 (unscaled, bf16) and [g | u]_r, dw_tj = <act(g) u, dh'_r>, which is
 // <dout_t, y_e(x_t)> since y = (act(g) u) W2^T, so neither h nor y is recomputed; then dh = w_tj dh' and
-// gu_r becomes [dh u act'(g) | dh act(g)] in place.  Dropped slots: dw_tj = 0.  Lanes take 8-column slices in
-// order, then a fixed xor tree.
+// gu_r becomes [dh u act'(g) | dh act(g)] in place.  With write_wh, w_tj h (bf16, the B operand of the W2
+// gradient dout^T (w h)) replaces dh'_r.  Dropped slots: dw_tj = 0.  Lanes take 8-column slices in order,
+// then a fixed xor tree.
 template <int ACT>
-__global__ void __launch_bounds__(256) k_glu_bwd_slots(__nv_bfloat16* __restrict__ gu,
-                                                       const __nv_bfloat16* __restrict__ dhp,
+__global__ void __launch_bounds__(256) k_glu_bwd_slots(__nv_bfloat16* __restrict__ gu, __nv_bfloat16* __restrict__ dhp,
                                                        const int32_t* __restrict__ slot_pos,
                                                        const float* __restrict__ topk_w, long long n_slots, int H,
-                                                       float* __restrict__ dw) {
+                                                       int write_wh, float* __restrict__ dw) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
   const long long i = (long long)blockIdx.x * 8 + warp_id();
   if (i >= n_slots) return;
@@ -130,15 +135,15 @@ __global__ void __launch_bounds__(256) k_glu_bwd_slots(__nv_bfloat16* __restrict
   const int nv = H >> 3;
   uint4* g4 = reinterpret_cast<uint4*>(gu + (size_t)row * 2 * H);
   uint4* u4 = g4 + nv;
-  const uint4* d4 = reinterpret_cast<const uint4*>(dhp + (size_t)row * H);
+  uint4* d4 = reinterpret_cast<uint4*>(dhp + (size_t)row * H);
   float acc = 0.f;
   for (int v = lane; v < nv; v += 32) {
     const uint4 G = g4[v], U = u4[v], D = d4[v];
     const uint32_t gw[4] = {G.x, G.y, G.z, G.w}, uw[4] = {U.x, U.y, U.z, U.w}, dv[4] = {D.x, D.y, D.z, D.w};
-    uint32_t og[4], ou[4];
+    uint32_t og[4], ou[4], oh[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float dg[2], du[2];
+      float dg[2], du[2], wh[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float g = h ? bf16hi(gw[q]) : bf16lo(gw[q]);
@@ -150,12 +155,15 @@ __global__ void __launch_bounds__(256) k_glu_bwd_slots(__nv_bfloat16* __restrict
         const float dh = wj * d;
         dg[h] = dh * u * da;
         du[h] = dh * a;
+        wh[h] = wj * a * u;
       }
       og[q] = pack_bf16x2(dg[0], dg[1]);
       ou[q] = pack_bf16x2(du[0], du[1]);
+      oh[q] = pack_bf16x2(wh[0], wh[1]);
     }
     g4[v] = make_uint4(og[0], og[1], og[2], og[3]);
     u4[v] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+    if (write_wh) d4[v] = make_uint4(oh[0], oh[1], oh[2], oh[3]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);

@@ -16,6 +16,7 @@
 #include "permute.cuh"
 #include "quant.cuh"
 #include "router.cuh"
+#include "wgrad.cuh"
 
 namespace moe {
 
@@ -761,6 +762,13 @@ static bool use_tc_router(const moe_shape* s) {
   return s->E % 16 == 0 && s->d % 64 == 0 && (double)s->T * s->E * s->d >= (double)(1ll << 28);
 }
 
+// True when route_impl, asked for neither logits nor statistics, takes the tensor-core screen and selection
+// path: the screen's fp32 logits (bias included) are then left in the workspace at L.part, [T, E].
+static bool route_keeps_screen(const moe_shape* s) {
+  return lanes_router_ec(s) == 0 && fused_router_epl(s) == 0 && use_tc_router(s) && s->E <= 256 &&
+         s->d <= kSelMaxD;
+}
+
 static int route_impl(const moe_shape* s, const void* x, const float* w_router, const float* bias,
                       const float* logits_in, float* logits, int32_t* idx, float* w, int32_t* counts, float* aux_f,
                       float* aux_p, float* aux, uint8_t* ws, cudaStream_t st, bool defer_aux = false) {
@@ -885,10 +893,24 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
 
 // ------------------------------------------------------------------ backward (input gradient)
 
+// Row splits of a dense weight gradient (one group of `rows` rows): about two waves of 148 tiles, at least 512
+// rows per split.  Independent of the device, so that the workspace size is.
+struct WgradSplit {
+  int n, chunk;
+};
+static int wgrad_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
+static WgradSplit wgrad_split(long long rows, int M, int N) {
+  const long long tiles = cdiv(M, kBM) * cdiv(N, wgrad_bn(N));
+  long long n = std::min<long long>(cdiv(296, tiles), std::max<long long>(1, rows / 512));
+  n = std::max<long long>(1, std::min<long long>(n, 32));
+  const long long chunk = cdiv(cdiv(rows, n), 64) * 64;
+  return WgradSplit{(int)cdiv(rows, chunk), (int)chunk};
+}
+
 // Scratch of moe_backward_x past the forward's regions (which it reuses: routing, grouping, x_perm for dx of the
 // grouped rows, h for dh').
 struct BwdWorkspace {
-  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, total;
+  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, part, total;
   int ldE;   // columns of dz and W_r^T: E rounded up to whole 64-column reduction steps
 };
 
@@ -909,31 +931,43 @@ static BwdWorkspace bwd_layout(const moe_shape* s) {
   B.dz = take((size_t)s->T * B.ldE * 2);
   B.wrt = take((size_t)s->d * B.ldE * 2);
   B.dxr = take((size_t)s->T * s->d * 2);
+  // split partials of the dense weight gradients: the router's, and the shared expert's two
+  size_t part = 0;
+  auto need = [&](int M, int N) {
+    const WgradSplit sp = wgrad_split(s->T, M, N);
+    if (sp.n > 1) part = std::max(part, (size_t)sp.n * M * N * 4);
+  };
+  need(s->E, s->d);
+  if (s->H_s > 0) {
+    need(2 * s->H_s, s->d);
+    need(s->d, s->H_s);
+  }
+  B.part = take(part);
   B.total = o;
   return B;
 }
 
-static int launch_glu_bwd(int act, void* gu, const void* dh, long long rows, int H, cudaStream_t st) {
+static int launch_glu_bwd(int act, void* gu, void* dh, long long rows, int H, bool write_h, cudaStream_t st) {
   const unsigned blocks = (unsigned)cdiv(rows * (H / 8), 256);
   if (act == MOE_ACT_SWIGLU)
     MOE_LAUNCH((k_glu_bwd<kModeSwiGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
-               reinterpret_cast<const __nv_bfloat16*>(dh), rows, H);
+               reinterpret_cast<__nv_bfloat16*>(dh), rows, H, (int)write_h);
   else
     MOE_LAUNCH((k_glu_bwd<kModeGeGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
-               reinterpret_cast<const __nv_bfloat16*>(dh), rows, H);
+               reinterpret_cast<__nv_bfloat16*>(dh), rows, H, (int)write_h);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
 
-static int launch_glu_bwd_slots(int act, void* gu, const void* dhp, const int32_t* slot, const float* w,
-                                long long n_slots, int H, float* dw, cudaStream_t st) {
+static int launch_glu_bwd_slots(int act, void* gu, void* dhp, const int32_t* slot, const float* w,
+                                long long n_slots, int H, bool write_wh, float* dw, cudaStream_t st) {
   const unsigned blocks = (unsigned)cdiv(n_slots, 8);
   if (act == MOE_ACT_SWIGLU)
     MOE_LAUNCH((k_glu_bwd_slots<kModeSwiGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
-               reinterpret_cast<const __nv_bfloat16*>(dhp), slot, w, n_slots, H, dw);
+               reinterpret_cast<__nv_bfloat16*>(dhp), slot, w, n_slots, H, (int)write_wh, dw);
   else
     MOE_LAUNCH((k_glu_bwd_slots<kModeGeGLU>), blocks, 256, 0, st, reinterpret_cast<__nv_bfloat16*>(gu),
-               reinterpret_cast<const __nv_bfloat16*>(dhp), slot, w, n_slots, H, dw);
+               reinterpret_cast<__nv_bfloat16*>(dhp), slot, w, n_slots, H, (int)write_wh, dw);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -949,6 +983,71 @@ static int launch_move_rows(const moe_shape* s, const void* src, const int32_t* 
   else if (s->k <= 8) MOE_LAUNCH((k_move_rows<8>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
   else MOE_LAUNCH((k_move_rows<16>), blocks, 256, 0, st, a, slot, (int)s->T, s->d, s->k, b);
   MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ weight gradients
+
+template <int BN>
+static int launch_wgrad_t(const CUtensorMap& ta, const CUtensorMap& tb, const WgradParams& p, cudaStream_t st) {
+  using Cfg = WgradCfg<BN>;
+  static std::atomic<unsigned long long> done_mask{0};
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(done_mask.load(std::memory_order_relaxed) & bit)) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(k_wgrad_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)Cfg::kSmemBytes));
+    done_mask.fetch_or(bit);
+  }
+  const long long tiles = cdiv(p.M, kBM) * cdiv(p.N, BN) * p.G;
+  const int grid = (int)std::max<long long>(1, std::min<long long>(num_sms(), tiles));
+  MOE_LAUNCH((k_wgrad_gemm<BN>), grid, 256, Cfg::kSmemBytes, st, ta, tb, p);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+// out[g] [M, N] fp32 = A_g^T B_g over the rows of group g, A [R, lda] and B [R, N] bf16 row-major (columns
+// M .. lda of A are not read into the output).  Groups: (gstart, grows) [G] on the device, or nullptr: one
+// group of all R rows, split by wgrad_split into partials in `part` (>= n * M * N floats) summed into out.
+static int wgrad_gemm(const void* A, int lda, int M, const void* B, int N, long long R, const int32_t* gstart,
+                      const int32_t* grows, int G, float* out, float* part, cudaStream_t st) {
+  if (N % 8 || lda % 8 || lda < M) return MOE_UNSUPPORTED_SHAPE;   // 16-byte row strides for TMA
+  CUtensorMap ta, tb;
+  cuuint64_t da[2] = {(cuuint64_t)lda, (cuuint64_t)std::max<long long>(R, 1)};
+  cuuint64_t db[2] = {(cuuint64_t)N, (cuuint64_t)std::max<long long>(R, 1)};
+  int rc = make_map(&ta, A, 2, da, 64);
+  if (rc) return rc;
+  rc = make_map(&tb, B, 2, db, 64);
+  if (rc) return rc;
+  WgradParams p;
+  p.group_start = gstart;
+  p.group_rows = grows;
+  p.R = R;
+  p.M = M;
+  p.N = N;
+  p.out_stride = (long long)M * N;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  WgradSplit sp{1, (int)std::max<long long>(R, 1)};
+  if (gstart == nullptr) {
+    sp = wgrad_split(R, M, N);
+    p.G = sp.n;
+    p.chunk = sp.chunk;
+    p.out = sp.n > 1 ? part : out;
+  } else {
+    p.G = G;
+    p.chunk = 0;
+    p.out = out;
+  }
+  const int BN = wgrad_bn(N);
+  if (BN == 256) rc = launch_wgrad_t<256>(ta, tb, p, st);
+  else if (BN == 128) rc = launch_wgrad_t<128>(ta, tb, p, st);
+  else rc = launch_wgrad_t<64>(ta, tb, p, st);
+  if (rc) return rc;
+  if (gstart == nullptr && sp.n > 1) {
+    const long long n = (long long)M * N;
+    MOE_LAUNCH((k_sum_splits), (unsigned)cdiv(n / 4, 256), 256, 0, st, part, sp.n, n, out);
+    MOE_LAUNCH_CHECK();
+  }
   return MOE_OK;
 }
 
@@ -1184,17 +1283,18 @@ int moe_backward_workspace_size(const moe_shape* s, size_t* bytes) {
   return MOE_OK;
 }
 
-int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
-                   const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
-                   const void* dout, float aux_coef, float* dx, void* workspace, size_t ws_bytes,
-                   moe_stream_t stream) {
+int moe_backward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                 const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
+                 const void* dout, float aux_coef, float* dx, float* dw13, float* dw2, float* dw13_sh,
+                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
   if (!x || !w_router || !w13 || !w13t || !w2t || !dout || !dx || !workspace) return MOE_INVALID_ARGUMENT;
   if (s->H_s > 0 && (!w13_sh || !w13t_sh || !w2t_sh)) return MOE_INVALID_ARGUMENT;
-  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w13t) ||
-      !aligned16(w2t) || !aligned16(dout) || !aligned16(dx) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w13) || !aligned16(w13t) || !aligned16(w2t) ||
+      !aligned16(dout) || !aligned16(dx) || !aligned16(dw13) || !aligned16(dw2) || !aligned16(dw13_sh) ||
+      !aligned16(dw2_sh) || !aligned16(dw_router) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return MOE_INVALID_ARGUMENT;
   const Workspace L = ws_layout(s);
   const BwdWorkspace B = bwd_layout(s);
@@ -1210,7 +1310,7 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
   int32_t* offs = reinterpret_cast<int32_t*>(ws + L.offs);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   void* xperm = ws + L.xperm;   // the grouped rows, then dx of the grouped rows
-  void* hbuf = ws + L.h;        // dh' = dout W2 of the grouped rows
+  void* hbuf = ws + L.h;        // dh' = dout W2 of the grouped rows, then w h
   void* gu = ws + B.gu;         // [g | u] of the grouped rows, then [dg | du]
   void* doutp = ws + B.doutp;   // dout of the grouped rows
   float* logits = reinterpret_cast<float*>(ws + B.logits);
@@ -1218,29 +1318,44 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(ws + B.dz);
   __nv_bfloat16* wrt = reinterpret_cast<__nv_bfloat16*>(ws + B.wrt);
   void* dxr = ws + B.dxr;
+  float* part = reinterpret_cast<float*>(ws + B.part);
   const long long R = grouped_rows(s);
   const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
 
-  // forward recompute: routing (with the logits for the softmax), grouping, [g | u]
-  rc = route_impl(s, x, w_router, bias, nullptr, logits, idx, w, cts, nullptr, nullptr, nullptr, ws, st);
+  // forward recompute: routing, grouping, [g | u].  The softmax backward takes the logits of every expert: the
+  // tensor-core screen's (two-term bf16 split of W_r, fp32 accumulation, within about 2^-16 |x| |w_e| of the
+  // fp32 logits) where the routing runs through it, else the router's own fp32 logits.
+  const bool screen = route_keeps_screen(s);
+  rc = route_impl(s, x, w_router, bias, nullptr, screen ? nullptr : logits, idx, w, cts, nullptr, nullptr, nullptr,
+                  ws, st);
   if (rc) return rc;
+  const float* z_all = screen ? reinterpret_cast<const float*>(ws + L.part) : logits;
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop, nullptr, xperm, kept, offs, st, true);
   if (rc) return rc;
   rc = grouped_gemm(kModePlain, xperm, R, s->d, w13, s->E, 2 * s->H, 0, 2 * s->H, offs, kept, gu, st, pair);
   if (rc) return rc;
 
   // routed experts: dout of the grouped rows, dh' = dout W2, the gate gradients and [dg | du] (dh = w dh'),
-  // dx = [dg | du] W13
+  // the weight gradients (dW2 = dout^T (w h), dW13 = [dg | du]^T x), dx = [dg | du] W13
   rc = launch_move_rows(s, dout, slot, doutp, st);
   if (rc) return rc;
   rc = grouped_gemm(kModePlain, doutp, R, s->d, w2t, s->E, s->H, 0, s->H, offs, kept, hbuf, st, pair);
   if (rc) return rc;
-  rc = launch_glu_bwd_slots(s->act, gu, hbuf, slot, w, s->T * (long long)s->k, s->H, dwb, st);
+  rc = launch_glu_bwd_slots(s->act, gu, hbuf, slot, w, s->T * (long long)s->k, s->H, dw2 != nullptr, dwb, st);
   if (rc) return rc;
+  if (dw2) {
+    rc = wgrad_gemm(doutp, s->d, s->d, hbuf, s->H, R, offs, kept, s->E, dw2, nullptr, st);
+    if (rc) return rc;
+  }
+  if (dw13) {
+    rc = wgrad_gemm(gu, 2 * s->H, 2 * s->H, xperm, s->d, R, offs, kept, s->E, dw13, nullptr, st);
+    if (rc) return rc;
+  }
   rc = grouped_gemm(kModePlain, gu, R, 2 * s->H, w13t, s->E, s->d, 0, s->d, offs, kept, xperm, st, pair);
   if (rc) return rc;
 
-  // shared expert on the tokens: [g | u] recomputed, dh = dout W2, [dg | du], dx = [dg | du] W13
+  // shared expert on the tokens: [g | u] recomputed, dh = dout W2, [dg | du] (and h), its weight gradients,
+  // dx = [dg | du] W13
   void* dxs = nullptr;
   if (s->H_s > 0) {
     void* gus = ws + B.gus;
@@ -1251,18 +1366,27 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
     if (rc) return rc;
     rc = grouped_gemm(kModePlain, dout, s->T, s->d, w2t_sh, 1, s->H_s, 0, s->H_s, nullptr, nullptr, dhs, st, pair);
     if (rc) return rc;
-    rc = launch_glu_bwd(s->act, gus, dhs, s->T, s->H_s, st);
+    rc = launch_glu_bwd(s->act, gus, dhs, s->T, s->H_s, dw2_sh != nullptr, st);
     if (rc) return rc;
+    if (dw2_sh) {
+      rc = wgrad_gemm(dout, s->d, s->d, dhs, s->H_s, s->T, nullptr, nullptr, 1, dw2_sh, part, st);
+      if (rc) return rc;
+    }
+    if (dw13_sh) {
+      rc = wgrad_gemm(gus, 2 * s->H_s, 2 * s->H_s, x, s->d, s->T, nullptr, nullptr, 1, dw13_sh, part, st);
+      if (rc) return rc;
+    }
     rc = grouped_gemm(kModePlain, gus, s->T, 2 * s->H_s, w13t_sh, 1, s->d, 0, s->d, nullptr, nullptr, dxs, st,
                       pair);
     if (rc) return rc;
   }
 
   // router: dz through the gates, the statistic and the softmax, then dz W_r (bf16 operands, fp32 accumulation)
+  // and dW_r = dz^T x
   const int epl = (int)cdiv(s->E, 32);
   const unsigned tb = (unsigned)cdiv(s->T, 8);
 #define MOE_RBWD(N_)                                                                                          \
-  MOE_LAUNCH((k_router_bwd<N_>), tb, 256, 0, st, logits, idx, w, dwb, cts, aux_coef, (int)s->T, s->E, s->k,    \
+  MOE_LAUNCH((k_router_bwd<N_>), tb, 256, 0, st, z_all, idx, w, dwb, cts, aux_coef, (int)s->T, s->E, s->k,     \
              s->renorm, B.ldE, dz)
   if (epl <= 1) MOE_RBWD(1);
   else if (epl <= 2) MOE_RBWD(2);
@@ -1271,6 +1395,10 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
   else MOE_RBWD(16);
 #undef MOE_RBWD
   MOE_LAUNCH_CHECK();
+  if (dw_router) {
+    rc = wgrad_gemm(dz, B.ldE, s->E, x, s->d, s->T, nullptr, nullptr, 1, dw_router, part, st);
+    if (rc) return rc;
+  }
   {
     const dim3 grid((unsigned)cdiv(s->d, 32), (unsigned)cdiv(B.ldE, 32));
     MOE_LAUNCH((k_transpose_router), grid, dim3(32, 8), 0, st, w_router, wrt, s->E, s->d, B.ldE);
@@ -1285,6 +1413,14 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
              reinterpret_cast<const __nv_bfloat16*>(dxr), (int)s->T, s->d, s->k, dx);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
+}
+
+int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
+                   const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
+                   const void* dout, float aux_coef, float* dx, void* workspace, size_t ws_bytes,
+                   moe_stream_t stream) {
+  return moe_backward(s, x, w_router, bias, w13, w13t, w2t, w13_sh, w13t_sh, w2t_sh, dout, aux_coef, dx, nullptr,
+                      nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
 int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream) {

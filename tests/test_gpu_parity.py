@@ -750,3 +750,48 @@ def test_backward_x_load_balance_term_alone(lib, name, over):
     rel = rel_frob(np64(dx), want)
     print(f"{name}: load-balance term alone, rel-Frobenius {rel:.2e}")
     assert rel <= BWD_REL_FROB
+
+
+# Weight gradients: each a bf16 GEMM with fp32 accumulation down the rows, of operands rounded once to bf16
+# ([dg | du], w h, dz; x and dout are exact), so about 2^-9 / sqrt(3) relative per term: bounded at 1e-2 in
+# rel-Frobenius per tensor, 3e-2 per expert (an expert's few rows average less).
+@pytest.mark.parametrize("name,over,aux_coef", [("tiny", {"H_s": 64, "act": 1, "capacity_factor": 0.5}, 0.1),
+                                                ("small", {}, 0.05),
+                                                ("granular", {"T": 1024, "skew": 1.2}, 0.0),
+                                                ("geglu", {"T": 512, "H": 1024}, 0.0)])
+def test_backward_weights_match_oracle(lib, name, over, aux_coef):
+    moe = lib
+    wl = synth.get_workload(name).replace(**over)
+    inp = synth.make_inputs(wl, seed=6, device=DEV)
+    s = shape_of(moe, wl)
+    g = torch.Generator(device=DEV).manual_seed(17)
+    dout = torch.randn(wl.T, wl.d, generator=g, device=DEV).to(torch.bfloat16)
+    kw = dict(bias=inp["bias"], w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), aux_coef=aux_coef)
+    got = moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, **kw)
+    dx_only = moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, **kw)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    assert torch.equal(got["dx"], dx_only)   # the weight gradients leave the input gradient's path unchanged
+    b64 = np64(inp["bias"]) if inp["bias"] is not None else None
+    ref = O.moe_backward(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
+                         np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
+                         w13_sh=np64(inp["w13_sh"]) if wl.H_s else None,
+                         w2_sh=np64(inp["w2_sh"]) if wl.H_s else None, aux_coef=aux_coef)
+    r = moe.moe_route(s, inp["x"], inp["w_router"], inp["bias"])
+    assert (npi(r["topk_idx"]) == ref["forward"]["idx"]).all()
+    keys = ["dx", "dw13", "dw2", "dw_router"] + (["dw13_sh", "dw2_sh"] if wl.H_s else [])
+    for key in keys:
+        a, b = np64(got[key]), ref[key]
+        rel = rel_frob(a, b)
+        print(f"{name} {key}: rel-Frobenius {rel:.2e}")
+        assert np.isfinite(a).all() and rel <= BWD_REL_FROB, key
+    kept = ref["forward"]["kept"]
+    for key in ("dw13", "dw2"):
+        a, b = np64(got[key]), ref[key]
+        for e in range(wl.E):
+            if kept[e] == 0:
+                assert not a[e].any(), f"{key}[{e}]: an expert without rows has a zero gradient"
+            else:
+                assert rel_frob(a[e], b[e]) <= 3 * BWD_REL_FROB, f"{key}[{e}] ({kept[e]} rows)"
+    if not wl.H_s:
+        assert got["dw13_sh"] is None and got["dw2_sh"] is None
