@@ -149,6 +149,50 @@ def route_from_logits(z, k: int, renorm: bool):
     return dict(z=z, p=p, idx=idx, w=w, counts=counts, f=f, P=P, aux=aux)
 
 
+# ---------------------------------------------------------------- hierarchical ("fractal") router
+# kieve-moe Features, "Fractal tiling routing": self-similar hierarchical routing over a branch^levels expert tree,
+# a cheap router for very large expert pools.  The page names it without the rule; the reading taken here:
+# expert e is the leaf whose base-`branch` digits (most significant first) d_0 .. d_{L-1} give the child taken
+# at each level; every level l has its own router W_l [branch, d] (and bias), shared by all nodes of the level
+# (the same split repeated at every node: the self-similarity); the level probabilities q_l = softmax(x W_l^T)
+# multiply along the path, p(e) = prod_l q_l[d_l], a distribution over the E = branch^levels leaves that costs
+# levels * branch logits per token instead of E.  Top-k, gates, renormalisation and the load-balance statistic
+# then follow the flat router on p (lower expert index first among equal p).
+
+def tree_digits(e, branch: int, levels: int) -> np.ndarray:
+    """Base-branch digits of the expert indices e, most significant first: [..., levels]."""
+    e = np.asarray(e, np.int64)
+    return np.stack([(e // branch ** (levels - 1 - l)) % branch for l in range(levels)], axis=-1)
+
+
+def route_tree(x, w_tree, bias_tree, branch: int, levels: int, k: int, renorm: bool):
+    """Tree routing on float64 level logits.  w_tree [levels * branch, d] stacks W_0 .. W_{L-1}; bias_tree
+    [levels * branch] or None.  Returns dict(z, q, p, idx, w, counts, f, P, aux) with z [T, L*B] the level
+    logits, q [T, L, B] the level probabilities and p [T, B^L] the leaf probabilities."""
+    z = router_logits(x, w_tree, bias_tree)
+    T = z.shape[0]
+    E = branch ** levels
+    q = np.stack([softmax(z[:, l * branch:(l + 1) * branch]) for l in range(levels)], axis=1)
+    dig = tree_digits(np.arange(E), branch, levels)                 # [E, L]
+    p = np.ones((T, E))
+    for l in range(levels):
+        p = p * q[:, l, dig[:, l]]
+    idx = topk_select(p, k)
+    w = gate_weights(p, idx, renorm)
+    counts = expert_counts(idx, E)
+    f, P, aux = load_balance(counts, p, T, E)
+    return dict(z=z, q=q, p=p, idx=idx, w=w, counts=counts, f=f, P=P, aux=aux)
+
+
+def tree_topk_margin(p, k: int) -> np.ndarray:
+    """Relative gap between the k-th and (k+1)-th largest leaf probability of each row (inf when k == E)."""
+    p = np.asarray(p, np.float64)
+    if k >= p.shape[1]:
+        return np.full(p.shape[0], np.inf)
+    s = -np.sort(-p, axis=1)
+    return (s[:, k - 1] - s[:, k]) / s[:, k - 1]
+
+
 # ---------------------------------------------------------------- step 4: grouping
 
 def capacity(T: int, k: int, E: int, factor: float) -> int:
