@@ -497,6 +497,66 @@ def run_backward(args, wl, world, rank, device):
     del graph
 
 
+def run_tree(args, wl, world, rank, device):
+    """Hierarchical router timing: moe_route_tree over branch**levels experts on the workload's tokens, captured
+    as a CUDA graph and replayed per step, L2 flushed before every step.  tokens/s, and the HBM roofline of its
+    algorithmic bytes (x, the level routers, the level logits written and read back, the picks)."""
+    import torch
+
+    import sparse_mixture_experts_expert_b200 as moe
+    import synth
+    B, L = args.tree_branch, args.tree_levels
+    E = B ** L
+    inp = synth.draw_tree_router(wl.T, wl.d, B, L, seed=1234 + rank, device=device)
+    s = moe.MoeShape(T=wl.T, d=wl.d, E=E, k=wl.k, H=16, renorm=1)
+    n = ctypes.c_size_t(0)
+    moe.load().moe_route_tree_workspace_size(ctypes.byref(s), B, L, ctypes.byref(n))
+    ws = torch.empty(int(n.value), dtype=torch.uint8, device=device)
+
+    def step():
+        return moe.moe_route_tree(s, B, L, inp["x"], inp["w_tree"], ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    launches0 = moe.moe_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    per_step = moe.moe_launch_count() - launches0
+    flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for a, b in evs:
+            flushbuf.fill_(1)
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize()
+    status, site = moe.moe_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    nl = B * L
+    alg = wl.T * wl.d * 2 + nl * wl.d * 4 + 2 * wl.T * nl * 4 + wl.T * wl.k * 8
+    peaks = load_peaks()
+    if rank == 0:
+        cfg = bench_config(wl, 0, world)
+        cfg.update(E=E, router=f"tree, branch {B}, levels {L} ({nl} level logits per token)", H=None, H_s=None)
+        print(json.dumps({"metric": f"hierarchical router tokens/s over {E} experts on 1 B200",
+                          "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+                          "config": cfg, "mode": "router only (moe_route_tree)",
+                          "roofline": {"bound": "hbm", "kernel": "whole moe_route_tree",
+                                       "achieved": alg / (ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                                       "unit": "GB/s", "frac": alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                       "peak_source": peaks["source"] + " copy", "alg_bytes_per_step": alg},
+                          "gpu_launches": per_step * args.steps, "clocks": clk.summary()}), flush=True)
+    del graph
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -511,6 +571,11 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (moe_backward: input and weight gradients, bf16 experts) instead of the "
                          "forward")
+    ap.add_argument("--tree", action="store_true",
+                    help="time the hierarchical router (moe_route_tree) on the workload's tokens, d and k over "
+                         "--tree-branch ** --tree-levels experts, instead of the forward")
+    ap.add_argument("--tree-branch", type=int, default=16)
+    ap.add_argument("--tree-levels", type=int, default=3)
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling only: run the workload with this many experts (a small case for ncu); the "
                          "line's config names it")
@@ -567,6 +632,9 @@ def main():
         return
     if args.backward:
         run_backward(args, wl, world, rank, device)
+        return
+    if args.tree:
+        run_tree(args, wl, world, rank, device)
         return
     s, inp, ws, out = setup(wl, rank, device)
     flushbuf = torch.empty(256 << 20, dtype=torch.uint8, device=device)

@@ -285,6 +285,35 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
                  float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Hierarchical ("fractal") router (kieve-moe Features, "Fractal tiling routing": self-similar routing over a
+ * branch^levels expert tree, a cheap router for very large expert pools).  Expert e is the leaf whose base-branch
+ * digits d_0 .. d_{levels-1} (most significant first) choose a child per level; level l has its own router
+ * W_l [branch, d] shared by all nodes of the level, q_l = softmax(x W_l^T + b_l), and the leaf probability is
+ * p(e) = prod_l q_l[d_l].  Top-k of p (larger first, lower expert index first among equal values), gates
+ * w_j = p(e_j), divided by their sum when s->renorm.  Cost per token: levels * branch logits, not E.
+ *   s          T, d, k (<= 16, <= E), renorm; E must equal branch^levels (<= 2^20; the grouping and expert
+ *              entry points take E <= 512); the other fields are not read
+ *   branch     2 .. 32 children per node;  levels >= 1;  branch * levels <= 256 and a multiple of 4
+ *   x          [T, d] bf16
+ *   w_tree     [levels * branch, d] fp32: level l's router in rows [l * branch, (l + 1) * branch)
+ *   bias_tree  [levels * branch] fp32 or NULL, added to the level logits
+ *   topk_idx   [T, k] int32 out,  topk_w [T, k] fp32 out
+ *   counts     [E] int32 out or NULL: selections per expert
+ *   level_logits [T, levels * branch] fp32 out or NULL (then kept in the workspace)
+ *   workspace  >= moe_route_tree_workspace_size() bytes, 256-byte aligned
+ * Precision: the level logits are the tensor-core screen of the flat router (W split into two bf16 terms, x
+ * bf16, fp32 accumulation: within about 2^-16 |x| |w| of the fp32 logits); softmax and products in fp32, each
+ * leaf's product formed in level order; the top-k by a beam of the k best partial paths per level, exact for
+ * those products.
+ * Errors: MOE_INVALID_ARGUMENT (NULL or misaligned pointers, E != branch^levels, k > E),
+ * MOE_UNSUPPORTED_SHAPE (limits above), MOE_WORKSPACE_TOO_SMALL; nothing is enqueued then.
+ */
+int moe_route_tree_workspace_size(const moe_shape* s, int32_t branch, int32_t levels, size_t* bytes);
+int moe_route_tree(const moe_shape* s, int32_t branch, int32_t levels, const void* x, const float* w_tree,
+                   const float* bias_tree, int32_t* topk_idx, float* topk_w, int32_t* counts, float* level_logits,
+                   void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Group-scaled signed INT4 quantiser (ExpertMesh README: signed INT4 weights
  * with group scales).  For each row of w [rows, K] fp32 (K % 128 == 0) and
  * each group of 128 inputs: s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7)

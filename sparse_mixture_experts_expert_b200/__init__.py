@@ -31,7 +31,7 @@ EXPORTED = ["moe_grouped_rows", "moe_capacity", "moe_workspace_size", "moe_route
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_int4", "moe_get_status",
             "moe_set_wait_limit_ns", "moe_selftest_wait_timeout", "moe_launch_count", "moe_status_string",
             "moe_permute_noalloc", "moe_transpose_experts", "moe_backward_workspace_size", "moe_backward_x",
-            "moe_backward"]
+            "moe_backward", "moe_route_tree_workspace_size", "moe_route_tree"]
 
 
 class MoeError(RuntimeError):
@@ -92,6 +92,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_backward_workspace_size": (ctypes.c_int, [S, ctypes.POINTER(sz)]),
         "moe_backward_x": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float, _P, _P, sz, _P]),
         "moe_backward": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float] + [_P] * 7 + [sz, _P]),
+        "moe_route_tree_workspace_size": (ctypes.c_int, [S, i32, i32, ctypes.POINTER(sz)]),
+        "moe_route_tree": (ctypes.c_int, [S, i32, i32] + [_P] * 8 + [sz, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -370,6 +372,34 @@ def moe_backward(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t
     dw2 [E, d, H], dw13_sh [1, 2H_s, d] and dw2_sh [1, d, H_s] (None without a shared expert), dw_router [E, d]."""
     return _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef,
                      ws, stream, True)
+
+
+def moe_route_tree(shape: MoeShape, branch: int, levels: int, x, w_tree, bias_tree=None, *, counts=False,
+                   logits=False, ws=None, stream=None):
+    """Hierarchical router over E = branch**levels experts (shape.E).  w_tree [levels * branch, d] fp32 stacks
+    the levels' routers.  Returns dict(topk_idx [T, k] int32, topk_w [T, k] fp32, counts [E] int32 or None,
+    level_logits [T, levels * branch] fp32 or None)."""
+    T, d, E, k = shape.T, shape.d, shape.E, shape.k
+    n = branch * levels
+    _want(x, torch.bfloat16, (T, d), "x")
+    _want(w_tree, torch.float32, (n, d), "w_tree")
+    if bias_tree is not None:
+        _want(bias_tree, torch.float32, (n,), "bias_tree")
+    dev = x.device
+    if ws is None:
+        nb = ctypes.c_size_t(0)
+        _check(_L().moe_route_tree_workspace_size(ctypes.byref(shape), branch, levels, ctypes.byref(nb)),
+               "moe_route_tree_workspace_size")
+        ws = torch.empty(int(nb.value), dtype=torch.uint8, device=dev)
+    out = dict(topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+               topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+               counts=torch.empty(E, dtype=torch.int32, device=dev) if counts else None,
+               level_logits=torch.empty(T, n, dtype=torch.float32, device=dev) if logits else None)
+    rc = _L().moe_route_tree(ctypes.byref(shape), branch, levels, _ptr(x), _ptr(w_tree), _ptr(bias_tree),
+                             _ptr(out["topk_idx"]), _ptr(out["topk_w"]), _ptr(out["counts"]),
+                             _ptr(out["level_logits"]), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "moe_route_tree")
+    return out
 
 
 def moe_quantize_int4(w, *, q=None, scales=None, stream=None):

@@ -16,6 +16,7 @@
 #include "permute.cuh"
 #include "quant.cuh"
 #include "router.cuh"
+#include "tree_router.cuh"
 #include "wgrad.cuh"
 
 namespace moe {
@@ -1051,6 +1052,43 @@ static int wgrad_gemm(const void* A, int lda, int M, const void* B, int N, long 
   return MOE_OK;
 }
 
+// ------------------------------------------------------------------ hierarchical router
+
+// E = branch^levels checked without overflow; the tree's own limits (the full layer's grouping keeps E <= 512).
+static int check_tree(const moe_shape* s, int branch, int levels) {
+  if (s == nullptr) return MOE_INVALID_ARGUMENT;
+  if (s->T < 1 || s->T > (1ll << 24)) return MOE_UNSUPPORTED_SHAPE;
+  if (s->d < 16 || s->d % 16 != 0 || s->d > 65536) return MOE_UNSUPPORTED_SHAPE;
+  if (s->k < 1 || s->k > 16) return MOE_UNSUPPORTED_SHAPE;
+  if (s->renorm != 0 && s->renorm != 1) return MOE_INVALID_ARGUMENT;
+  if (branch < 2 || branch > kTreeMaxBranch || levels < 1) return MOE_UNSUPPORTED_SHAPE;
+  const int n = branch * levels;
+  if (n > kTreeMaxLogits || n % 4 != 0) return MOE_UNSUPPORTED_SHAPE;
+  long long E = 1;
+  for (int l = 0; l < levels; ++l) {
+    E *= branch;
+    if (E > kTreeMaxE) return MOE_UNSUPPORTED_SHAPE;
+  }
+  if (E != s->E) return MOE_INVALID_ARGUMENT;
+  if (s->k > s->E) return MOE_INVALID_ARGUMENT;
+  return MOE_OK;
+}
+
+struct TreeWorkspace {
+  size_t wsplit, wnorm, z, total;
+};
+
+static TreeWorkspace tree_layout(const moe_shape* s, int n) {
+  TreeWorkspace W{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  W.wsplit = take((size_t)2 * n * s->d * 2);
+  W.wnorm = take((size_t)n * 4);
+  W.z = take((size_t)s->T * n * 4);
+  W.total = o;
+  return W;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -1421,6 +1459,51 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
                    moe_stream_t stream) {
   return moe_backward(s, x, w_router, bias, w13, w13t, w2t, w13_sh, w13t_sh, w2t_sh, dout, aux_coef, dx, nullptr,
                       nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes, stream);
+}
+
+int moe_route_tree_workspace_size(const moe_shape* s, int32_t branch, int32_t levels, size_t* bytes) {
+  const int rc = check_tree(s, branch, levels);
+  if (rc) return rc;
+  if (!bytes) return MOE_INVALID_ARGUMENT;
+  *bytes = tree_layout(s, branch * levels).total;
+  return MOE_OK;
+}
+
+int moe_route_tree(const moe_shape* s, int32_t branch, int32_t levels, const void* x, const float* w_tree,
+                   const float* bias_tree, int32_t* topk_idx, float* topk_w, int32_t* counts, float* level_logits,
+                   void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_tree(s, branch, levels);
+  if (rc) return rc;
+  if (!x || !w_tree || !topk_idx || !topk_w || !workspace) return MOE_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_tree) || !aligned16(level_logits) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return MOE_INVALID_ARGUMENT;
+  const int n = branch * levels;
+  const TreeWorkspace W = tree_layout(s, n);
+  if (ws_bytes < W.total) return MOE_WORKSPACE_TOO_SMALL;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(ws + W.wsplit);
+  float* z = level_logits ? level_logits : reinterpret_cast<float*>(ws + W.z);
+  // the levels' routers as one screening operand [n, 2d] (bf16 high and low terms), counts zeroed alongside
+  MOE_LAUNCH((k_router_prep), (unsigned)cdiv(n, 8), 256, 0, stream, w_tree, wsplit,
+             reinterpret_cast<float*>(ws + W.wnorm), n, s->d, counts, counts ? s->E : 0,
+             static_cast<const __nv_bfloat16*>(nullptr), static_cast<float*>(nullptr), (int)s->T);
+  MOE_LAUNCH_CHECK();
+  GemmExtras ex;
+  ex.bias = bias_tree;
+  rc = grouped_gemm(kModeScreen, x, s->T, s->d, wsplit, 1, n, 0, n, nullptr, nullptr, z, stream,
+                    !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM), ex);
+  if (rc) return rc;
+  const unsigned blocks = (unsigned)cdiv(s->T * kTreeGroup, kTreeThreads);
+#define MOE_TREE(K_)                                                                                          \
+  MOE_LAUNCH((k_router_tree<K_>), blocks, kTreeThreads, 0, stream, z, (int)s->T, (int)branch, (int)levels, s->k, \
+             s->renorm, topk_idx, topk_w, counts)
+  if (s->k <= 2) MOE_TREE(2);
+  else if (s->k <= 4) MOE_TREE(4);
+  else if (s->k <= 8) MOE_TREE(8);
+  else MOE_TREE(16);
+#undef MOE_TREE
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
 }
 
 int moe_quantize_int4(const float* w, int64_t rows, int32_t K, uint8_t* q, void* scales, moe_stream_t stream) {

@@ -49,6 +49,7 @@ _STREAM_X = 1
 _STREAM_ROUTER = 2
 _STREAM_TOPK = 3
 _STREAM_LOGITS = 4
+_STREAM_TREE = 5
 _STREAM_EXPERT0 = 1000        # expert e uses 1000 + e; the shared expert uses 1000 + E
 
 
@@ -158,6 +159,17 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu", with_expert_weights: 
             out["w13_sh"] = a.to(torch.bfloat16).unsqueeze(0).contiguous()
             out["w2_sh"] = b.to(torch.bfloat16).unsqueeze(0).contiguous()
     return out
+
+
+def draw_tree_router(T: int, d: int, branch: int, levels: int, seed: int = 0, device="cpu"):
+    """Inputs of a hierarchical router over branch**levels experts: ``x`` [T, d] bf16 (the same draw as
+    :func:`make_inputs` for these T, d and seed) and ``w_tree`` [levels * branch, d] fp32 with std 1/sqrt(d),
+    so that every level's logits are about unit normal."""
+    g = _gen(seed, _STREAM_X, device)
+    x = torch.randn(T, d, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    g = _gen(seed, _STREAM_TREE, device)
+    w = torch.randn(levels * branch, d, generator=g, device=device, dtype=torch.float32) / math.sqrt(d)
+    return dict(x=x, w_tree=w)
 
 
 def draw_topk_idx(T: int, E: int, k: int, seed: int = 0, skew: float = 0.0, device="cpu") -> torch.Tensor:
