@@ -900,6 +900,8 @@ struct WgradSplit {
   int n, chunk;
 };
 static int wgrad_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
+// rows per chunk of a hot expert's weight gradient (32 reduction steps of 64 rows)
+constexpr int kWgradSplitRows = 2048;
 static WgradSplit wgrad_split(long long rows, int M, int N) {
   const long long tiles = cdiv(M, kBM) * cdiv(N, wgrad_bn(N));
   long long n = std::min<long long>(cdiv(296, tiles), std::max<long long>(1, rows / 512));
@@ -911,7 +913,7 @@ static WgradSplit wgrad_split(long long rows, int M, int N) {
 // Scratch of moe_backward_x past the forward's regions (which it reuses: routing, grouping, x_perm for dx of the
 // grouped rows, h for dh').
 struct BwdWorkspace {
-  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, part, total;
+  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, part, wpart, wlist, total;
   int ldE;   // columns of dz and W_r^T: E rounded up to whole 64-column reduction steps
 };
 
@@ -944,6 +946,10 @@ static BwdWorkspace bwd_layout(const moe_shape* s) {
     need(s->d, s->H_s);
   }
   B.part = take(part);
+  // chunk partials of hot experts' weight gradients: the chunks of groups above kWgradSplitRows rows number at
+  // most 2 R / kWgradSplitRows (each such group adds at most one partial chunk beyond R / kWgradSplitRows)
+  B.wpart = take((size_t)2 * cdiv(R, kWgradSplitRows) * std::max(2 * s->H, s->H) * s->d * 4);
+  B.wlist = take((size_t)(1 + 3 * s->E) * 4);
   B.total = o;
   return B;
 }
@@ -1011,7 +1017,8 @@ static int launch_wgrad_t(const CUtensorMap& ta, const CUtensorMap& tb, const Wg
 // M .. lda of A are not read into the output).  Groups: (gstart, grows) [G] on the device, or nullptr: one
 // group of all R rows, split by wgrad_split into partials in `part` (>= n * M * N floats) summed into out.
 static int wgrad_gemm(const void* A, int lda, int M, const void* B, int N, long long R, const int32_t* gstart,
-                      const int32_t* grows, int G, float* out, float* part, cudaStream_t st) {
+                      const int32_t* grows, int G, float* out, float* part, cudaStream_t st, int split_rows = 0,
+                      int32_t* split_list = nullptr) {
   if (N % 8 || lda % 8 || lda < M) return MOE_UNSUPPORTED_SHAPE;   // 16-byte row strides for TMA
   CUtensorMap ta, tb;
   cuuint64_t da[2] = {(cuuint64_t)lda, (cuuint64_t)std::max<long long>(R, 1)};
@@ -1028,6 +1035,9 @@ static int wgrad_gemm(const void* A, int lda, int M, const void* B, int N, long 
   p.N = N;
   p.out_stride = (long long)M * N;
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.split_rows = gstart != nullptr ? split_rows : 0;
+  p.part = part;
+  p.split_list = gstart != nullptr && split_rows > 0 ? split_list : nullptr;
   WgradSplit sp{1, (int)std::max<long long>(R, 1)};
   if (gstart == nullptr) {
     sp = wgrad_split(R, M, N);
@@ -1047,6 +1057,10 @@ static int wgrad_gemm(const void* A, int lda, int M, const void* B, int N, long 
   if (gstart == nullptr && sp.n > 1) {
     const long long n = (long long)M * N;
     MOE_LAUNCH((k_sum_splits), (unsigned)cdiv(n / 4, 256), 256, 0, st, part, sp.n, n, out);
+    MOE_LAUNCH_CHECK();
+  }
+  if (p.split_list != nullptr) {   // the hot groups' chunks (the list may be empty)
+    MOE_LAUNCH((k_wgrad_reduce), (unsigned)(4 * num_sms()), 256, 0, st, part, split_list, (long long)M * N, out);
     MOE_LAUNCH_CHECK();
   }
   return MOE_OK;
@@ -1381,12 +1395,16 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   if (rc) return rc;
   rc = launch_glu_bwd_slots(s->act, gu, hbuf, slot, w, s->T * (long long)s->k, s->H, dw2 != nullptr, dwb, st);
   if (rc) return rc;
+  float* wpart = reinterpret_cast<float*>(ws + B.wpart);
+  int32_t* wlist = reinterpret_cast<int32_t*>(ws + B.wlist);
+  // an expert holds at most C rows (capacity) or T (one row per token): chunk only when that can exceed a chunk
+  const int split = (s->capacity > 0 ? (long long)s->capacity : s->T) > kWgradSplitRows ? kWgradSplitRows : 0;
   if (dw2) {
-    rc = wgrad_gemm(doutp, s->d, s->d, hbuf, s->H, R, offs, kept, s->E, dw2, nullptr, st);
+    rc = wgrad_gemm(doutp, s->d, s->d, hbuf, s->H, R, offs, kept, s->E, dw2, wpart, st, split, wlist);
     if (rc) return rc;
   }
   if (dw13) {
-    rc = wgrad_gemm(gu, 2 * s->H, 2 * s->H, xperm, s->d, R, offs, kept, s->E, dw13, nullptr, st);
+    rc = wgrad_gemm(gu, 2 * s->H, 2 * s->H, xperm, s->d, R, offs, kept, s->E, dw13, wpart, st, split, wlist);
     if (rc) return rc;
   }
   rc = grouped_gemm(kModePlain, gu, R, 2 * s->H, w13t, s->E, s->d, 0, s->d, offs, kept, xperm, st, pair);

@@ -14,8 +14,11 @@
 // in 64-row steps.  Rows of a step past the group's end belong to the next
 // group: the MMA warp zeroes them in shared memory (async-proxy fence after)
 // and skips the 16-row slices that hold none of the group's rows.  A group
-// without rows gets zeros.  Dense gradients with few tiles split their rows
-// into chunks (one partial output each) that k_sum_splits adds in order.
+// without rows gets zeros.  A group of many rows (a hot expert) is reduced in
+// fixed-size row chunks, each its own set of tiles writing a partial that
+// k_wgrad_reduce adds in order, so that one expert's tiles do not outlast the
+// rest of the grid.  Dense gradients with few tiles split their rows into
+// chunks (one partial output each) that k_sum_splits adds in order.
 // Boxes wholly past the last output row or column are not loaded; what their
 // stage space holds reaches only accumulator rows and columns that are never
 // stored.
@@ -36,6 +39,12 @@ struct WgradParams {
   float* out;                   // group g: out + g * out_stride, [M][N] row-major
   long long out_stride;
   unsigned long long wait_limit_ns;
+  // groups (group_start given) of more than split_rows rows are reduced in split_rows-row chunks, one tile
+  // set each, into partials part + slot * out_stride; split_list gets [count, then (group, first slot,
+  // chunks) per split group] for k_wgrad_reduce.  split_rows 0: no splitting.
+  int split_rows;
+  float* part;
+  int32_t* split_list;
 };
 
 constexpr int kWgBox = 64 * 128;   // one 64-row x 64-column bf16 box (8 KB)
@@ -84,11 +93,53 @@ __global__ void __launch_bounds__(256, 1)
   __shared__ __align__(8) uint64_t bar_full[S], bar_empty[S], bar_tfull[2], bar_tempty[2], bar_final;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
+  __shared__ int s_uprefix[kMaxGroupsSmem + 1];   // row chunks before group g
+  __shared__ int s_pslot[kMaxGroupsSmem];         // first partial slot of a split group, -1 otherwise
 
   const int warp = warp_id(), lane = lane_id();
   const int mt = (p.M + kBM - 1) / kBM, nt = (p.N + BN - 1) / BN;
   const long long per_group = (long long)mt * nt;
-  const long long total = per_group * p.G;
+  const bool grouped = p.group_start != nullptr;
+  const int CH = grouped ? p.split_rows : 0;
+
+  // chunk table (warp 2): chunks per group, their prefix, the partial slots; CTA 0 also lists the split groups
+  if (warp == 2) {
+    const int per = (p.G + 31) / 32;
+    const int g0 = min(p.G, lane * per), g1 = min(p.G, g0 + per);
+    int units = 0, slots = 0, nsplit = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int rows = grouped ? p.group_rows[g] : 0;
+      const int nc = (CH > 0 && rows > CH) ? (rows + CH - 1) / CH : 1;
+      units += nc;
+      if (nc > 1) { slots += nc; ++nsplit; }
+    }
+    int iu = units, is = slots, in = nsplit;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, iu, o), b = __shfl_up_sync(0xffffffffu, is, o);
+      const int c = __shfl_up_sync(0xffffffffu, in, o);
+      if (lane >= o) { iu += a; is += b; in += c; }
+    }
+    int u = iu - units, sl = is - slots, li = in - nsplit;
+    for (int g = g0; g < g1; ++g) {
+      const int rows = grouped ? p.group_rows[g] : 0;
+      const int nc = (CH > 0 && rows > CH) ? (rows + CH - 1) / CH : 1;
+      s_uprefix[g] = u;
+      s_pslot[g] = nc > 1 ? sl : -1;
+      if (nc > 1 && blockIdx.x == 0 && p.split_list != nullptr) {
+        p.split_list[1 + 3 * li] = g;
+        p.split_list[2 + 3 * li] = sl;
+        p.split_list[3 + 3 * li] = nc;
+        ++li;
+      }
+      u += nc;
+      if (nc > 1) sl += nc;
+    }
+    if (lane == 31) {
+      s_uprefix[p.G] = iu;
+      if (blockIdx.x == 0 && p.split_list != nullptr) p.split_list[0] = in;
+    }
+  }
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&bar_full[s], 1); mbar_init(&bar_empty[s], 1); }
@@ -107,19 +158,30 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
+  const long long total = per_group * s_uprefix[p.G];
 
-  // tile -> group, its rows [start, start + rows), output origin (m0, n0)
-  auto locate = [&](long long tile, int& g, long long& start, int& rows, int& m0, int& n0) {
-    g = (int)(tile / per_group);
-    const int rem = (int)(tile - (long long)g * per_group);
+  // tile -> group, its rows [start, start + rows), output tile, origin (m0, n0)
+  auto locate = [&](long long tile, int& g, long long& start, int& rows, int& m0, int& n0, float*& out) {
+    const int unit = (int)(tile / per_group);
+    const int rem = (int)(tile - (long long)unit * per_group);
     m0 = (rem / nt) * kBM;
     n0 = (rem % nt) * BN;
-    if (p.group_start != nullptr) {
-      start = p.group_start[g];
-      rows = p.group_rows[g];
+    int lo = 0, hi = p.G - 1;   // last g with s_uprefix[g] <= unit
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_uprefix[mid] <= unit) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    const int c = unit - s_uprefix[g];
+    if (grouped) {
+      const int all = p.group_rows[g];
+      start = (long long)p.group_start[g] + (long long)c * CH;
+      rows = s_pslot[g] < 0 ? all : min(CH, all - c * CH);
+      out = s_pslot[g] < 0 ? p.out + (long long)g * p.out_stride : p.part + (long long)(s_pslot[g] + c) * p.out_stride;
     } else {
       start = (long long)g * p.chunk;
       rows = (int)max(0ll, min((long long)p.chunk, p.R - start));
+      out = p.out + (long long)g * p.out_stride;
     }
   };
 
@@ -131,7 +193,8 @@ __global__ void __launch_bounds__(256, 1)
     for (long long tile = blockIdx.x; tile < total && !__any_sync(0xffffffffu, s_abort); tile += gridDim.x) {
       int g, rows, m0, n0;
       long long start;
-      locate(tile, g, start, rows, m0, n0);
+      float* out;
+      locate(tile, g, start, rows, m0, n0, out);
       const int nk = (rows + 63) / 64;
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
@@ -177,7 +240,8 @@ __global__ void __launch_bounds__(256, 1)
     for (long long tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       int g, rows, m0, n0;
       long long start;
-      locate(tile, g, start, rows, m0, n0);
+      float* out;
+      locate(tile, g, start, rows, m0, n0, out);
       const int nk = (rows + 63) / 64;
       if (lane == 0) ok = mbar_wait(&bar_tempty[acc], acc_phase ^ 1u, p.wait_limit_ns, &s_abort, 0x0703);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -235,11 +299,11 @@ __global__ void __launch_bounds__(256, 1)
     for (long long tile = blockIdx.x; tile < total && !s_abort; tile += gridDim.x) {
       int g, rows, m0, n0;
       long long start;
-      locate(tile, g, start, rows, m0, n0);
+      float* out;
+      locate(tile, g, start, rows, m0, n0, out);
       if (!mbar_wait(&bar_tfull[acc], acc_phase, p.wait_limit_ns, &s_abort, 0x0706)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      float* out = p.out + (long long)g * p.out_stride;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[2][16];
@@ -283,6 +347,27 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// The split groups of k_wgrad_gemm: out[g] = sum over its chunks c (in order) of part[slot + c], fp32.  The list
+// ([count, then (group, slot, chunks)]) comes from the GEMM; a grid-stride loop covers count x mn / 4 vectors.
+__global__ void __launch_bounds__(256) k_wgrad_reduce(const float* __restrict__ part,
+                                                      const int32_t* __restrict__ split_list, long long mn,
+                                                      float* __restrict__ out) {
+  pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
+  const long long nv = mn / 4;
+  const long long total = (long long)split_list[0] * nv;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long item = i / nv, v = i - item * nv;
+    const int g = split_list[1 + 3 * item], slot = split_list[2 + 3 * item], nc = split_list[3 + 3 * item];
+    float4 a = reinterpret_cast<const float4*>(part + (long long)slot * mn)[v];
+    for (int c = 1; c < nc; ++c) {
+      const float4 b = reinterpret_cast<const float4*>(part + (long long)(slot + c) * mn)[v];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    reinterpret_cast<float4*>(out + (long long)g * mn)[v] = a;
   }
 }
 

@@ -754,10 +754,12 @@ def test_backward_x_load_balance_term_alone(lib, name, over):
 
 # Weight gradients: each a bf16 GEMM with fp32 accumulation down the rows, of operands rounded once to bf16
 # ([dg | du], w h, dz; x and dout are exact), so about 2^-9 / sqrt(3) relative per term: bounded at 1e-2 in
-# rel-Frobenius per tensor, 3e-2 per expert (an expert's few rows average less).
+# rel-Frobenius per tensor, 3e-2 per expert (an expert's few rows average less).  skewed at 4096 tokens has
+# three experts above 2048 rows (3770, 2932, 2180), whose gradients are summed from 2048-row chunks.
 @pytest.mark.parametrize("name,over,aux_coef", [("tiny", {"H_s": 64, "act": 1, "capacity_factor": 0.5}, 0.1),
                                                 ("small", {}, 0.05),
                                                 ("granular", {"T": 1024, "skew": 1.2}, 0.0),
+                                                ("skewed", {"T": 4096}, 0.0),
                                                 ("geglu", {"T": 512, "H": 1024}, 0.0)])
 def test_backward_weights_match_oracle(lib, name, over, aux_coef):
     moe = lib
