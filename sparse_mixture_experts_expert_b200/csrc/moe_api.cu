@@ -1511,14 +1511,21 @@ int moe_route_tree(const moe_shape* s, int32_t branch, int32_t levels, const voi
   rc = grouped_gemm(kModeScreen, x, s->T, s->d, wsplit, 1, n, 0, n, nullptr, nullptr, z, stream,
                     !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM), ex);
   if (rc) return rc;
-  const unsigned blocks = (unsigned)cdiv(s->T * kTreeGroup, kTreeThreads);
-#define MOE_TREE(K_)                                                                                          \
-  MOE_LAUNCH((k_router_tree<K_>), blocks, kTreeThreads, 0, stream, z, (int)s->T, (int)branch, (int)levels, s->k, \
-             s->renorm, topk_idx, topk_w, counts)
-  if (s->k <= 2) MOE_TREE(2);
-  else if (s->k <= 4) MOE_TREE(4);
-  else if (s->k <= 8) MOE_TREE(8);
-  else MOE_TREE(16);
+  // lanes per token: enough for kTreeCPL children each
+  const int G = branch <= 2 * kTreeCPL ? 2 : (branch <= 4 * kTreeCPL ? 4 : 8);
+  const unsigned blocks = (unsigned)cdiv(s->T * G, kTreeThreads);
+#define MOE_TREE(K_, G_)                                                                                      \
+  MOE_LAUNCH((k_router_tree<K_, G_>), blocks, kTreeThreads, 0, stream, z, (int)s->T, (int)branch, (int)levels,  \
+             s->k, s->renorm, topk_idx, topk_w, counts)
+#define MOE_TREE_K(G_)                     \
+  if (s->k <= 2) MOE_TREE(2, G_);          \
+  else if (s->k <= 4) MOE_TREE(4, G_);     \
+  else if (s->k <= 8) MOE_TREE(8, G_);     \
+  else MOE_TREE(16, G_);
+  if (G == 2) { MOE_TREE_K(2) }
+  else if (G == 4) { MOE_TREE_K(4) }
+  else { MOE_TREE_K(8) }
+#undef MOE_TREE_K
 #undef MOE_TREE
   MOE_LAUNCH_CHECK();
   return MOE_OK;

@@ -19,25 +19,27 @@ constexpr int kTreeMaxBranch = 32;   // one level's children on the lanes of a w
 constexpr int kTreeMaxLogits = 256;  // levels * branch: one screening tile
 constexpr long long kTreeMaxE = 1ll << 20;   // leaves
 
-constexpr int kTreeGroup = 8;        // lanes per token
-constexpr int kTreeThreads = 128;    // 16 tokens per block
+constexpr int kTreeCPL = 4;          // children per lane: a token takes branch / 4 lanes (rounded up to 2, 4 or 8)
+constexpr int kTreeThreads = 128;
 
-// kTreeGroup lanes per token.  z [T, L * B] fp32 level logits (bias included).  Outputs topk_idx / topk_w
-// [T, k]; counts [E] (zeroed beforehand) gains one per selection when not null.  Per level:
-//   1. softmax: lane g holds children c = g, g + 8, g + 16, g + 24 (c < B); group max and sum;
+// G lanes per token (G = 2, 4 or 8, at least branch / 4).  z [T, L * B] fp32 level logits (bias included).
+// Outputs topk_idx / topk_w [T, k]; counts [E] (zeroed beforehand) gains one per selection when not null.
+// Per level:
+//   1. softmax: lane g holds children c = g, g + G, g + 2 G, g + 3 G (c < B); group max and sum;
 //   2. the level's kk = min(k, B) best children by (q desc, c asc), into shared memory: each lane offers its
-//      best untaken child, a 3-step butterfly picks the winner (exactly the order of a full sort);
+//      best untaken child, a butterfly over the group picks the winner (exactly the order of a full sort);
 //   3. the new beam: nsel = min(k, nb B) rounds over the candidates (bv[j] q[c], bi[j] B + c); lane g owns beam
-//      entries g and g + 8, offers each entry's best untaken child (the first untaken in q order, or among
+//      entries g, g + G, ..., offers each entry's best untaken child (the first untaken in q order, or among
 //      later ones whose product rounds to the same value, the lowest c), and a butterfly picks the largest
 //      product, the lower path index among equal ones.  Only an entry's kk best children can reach the top k.
-template <int KMAX>
+template <int KMAX, int G>
 __global__ void __launch_bounds__(kTreeThreads) k_router_tree(const float* __restrict__ z, int T, int B, int L,
                                                               int k, int renorm, int32_t* __restrict__ topk_idx,
                                                               float* __restrict__ topk_w,
                                                               int32_t* __restrict__ counts) {
   pdl_wait();  // inputs written by the previous kernel on the stream are visible past this point
-  constexpr int CPL = kTreeMaxBranch / kTreeGroup;          // children per lane
+  constexpr int kTreeGroup = G;
+  constexpr int CPL = kTreeCPL;                              // children per lane
   constexpr int EPL = (KMAX + kTreeGroup - 1) / kTreeGroup;  // beam entries per lane
   __shared__ float s_cq[kTreeThreads / kTreeGroup][KMAX];
   __shared__ int s_cc[kTreeThreads / kTreeGroup][KMAX];
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(kTreeThreads) k_router_tree(const float* __res
   const int g = threadIdx.x % kTreeGroup;
   // whole groups leave together (T is a group boundary), so the group shuffles below see every lane
   if (t >= T) return;
-  const unsigned gmask = 0xffu << (lane_id() & ~(kTreeGroup - 1));
+  const unsigned gmask = ((1u << kTreeGroup) - 1u) << (lane_id() & ~(kTreeGroup - 1));
   float* cq = s_cq[threadIdx.x / kTreeGroup];
   int* cc = s_cc[threadIdx.x / kTreeGroup];
   const float* zr = z + t * (long long)(B * L);

@@ -755,8 +755,12 @@ def test_backward_x_load_balance_term_alone(lib, name, over):
 # Weight gradients: each a bf16 GEMM with fp32 accumulation down the rows, of operands rounded once to bf16
 # ([dg | du], w h, dz; x and dout are exact), so about 2^-9 / sqrt(3) relative per term: bounded at 1e-2 in
 # rel-Frobenius per tensor, 3e-2 per expert (an expert's few rows average less).  skewed at 4096 tokens has
-# three experts above 2048 rows (3770, 2932, 2180), whose gradients are summed from 2048-row chunks.
+# three experts above 2048 rows (3770, 2932, 2180), whose gradients are summed from 2048-row chunks.  The tiny
+# cases add a ragged token count (300: a partial 8-token block, a partial 64-row reduction step of the dense
+# gradients) and gates without renormalisation.
 @pytest.mark.parametrize("name,over,aux_coef", [("tiny", {"H_s": 64, "act": 1, "capacity_factor": 0.5}, 0.1),
+                                                ("tiny", {"T": 300, "H_s": 64}, 0.05),
+                                                ("tiny", {"T": 200, "renorm": 0}, 0.1),
                                                 ("small", {}, 0.05),
                                                 ("granular", {"T": 1024, "skew": 1.2}, 0.0),
                                                 ("skewed", {"T": 4096}, 0.0),
