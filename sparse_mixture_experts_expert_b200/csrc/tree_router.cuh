@@ -5,17 +5,18 @@
 // level softmaxes along the path: p(e) = q_0[d_0] q_1[d_1] ... q_{L-1}[d_{L-1}], q_l = softmax(x W_l^T + b_l).
 // Per token that is levels * branch logits instead of E = branch^levels.  The level logits come from the
 // router's tensor-core screen (two-term bf16 split of the fp32 weights, fp32 accumulation); this kernel takes
-// the level softmaxes and the top-k of the leaf probabilities by a beam search, one thread per token: after
-// each level only the k best partial paths survive, ordered by (product desc, path index asc).  The product is monotone in each
-// factor, so the k best leaves are never pruned; each leaf's product is formed in level order, as a direct
-// evaluation would.  Gates are the leaf probabilities, renormalised over the k picks when asked.
+// the level softmaxes and the top-k of the leaf probabilities by a beam search, a small group of lanes per
+// token: after each level only the k best partial paths survive, ordered by (product desc, path index asc).
+// The product is monotone in each factor, so the k best leaves are never pruned; each leaf's product is formed
+// in level order, as a direct evaluation would.  Gates are the leaf probabilities, renormalised over the k
+// picks when asked.
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kTreeMaxBranch = 32;   // one level's children on the lanes of a warp
+constexpr int kTreeMaxBranch = 32;   // one level's children on at most 8 lanes, 4 each
 constexpr int kTreeMaxLogits = 256;  // levels * branch: one screening tile
 constexpr long long kTreeMaxE = 1ll << 20;   // leaves
 
