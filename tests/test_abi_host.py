@@ -120,3 +120,55 @@ def test_null_and_workspace_errors_return_before_device_work(L):
     rc = L.moe_quantize_int4(fake, 4, 100, fake, fake, None)
     assert rc == 1            # K % 128 != 0
     assert L.moe_set_wait_limit_ns(0) == 1
+
+
+@pytest.mark.parametrize("kw,branch,levels,code", [({"E": 4096}, 16, 3, 0), ({"E": 4095}, 16, 3, 1),
+                                                   ({"E": 2 ** 20}, 32, 4, 0), ({"E": 33 ** 2}, 33, 2, 2),
+                                                   ({"E": 27}, 3, 3, 2), ({"E": 16, "k": 17}, 16, 1, 2),
+                                                   ({"E": 4, "k": 3}, 2, 2, 0), ({"E": 4, "k": 5}, 4, 1, 1), ({"E": 2}, 2, 1, 2),
+                                                   ({"E": 2 ** 21}, 2, 21, 2), ({"E": 16, "renorm": 3}, 4, 2, 1)])
+def test_tree_router_shape_validation(L, kw, branch, levels, code):
+    # E = branch^levels; branch 2..32; branch * levels a multiple of 4 and <= 256; E <= 2^20; k <= min(16, E)
+    import sparse_mixture_experts_expert_b200 as moe
+    s = _shape(moe, **kw)
+    n = ctypes.c_size_t(0)
+    assert L.moe_route_tree_workspace_size(ctypes.byref(s), branch, levels, ctypes.byref(n)) == code
+    if code == 0:
+        assert n.value > 0 and n.value % 256 == 0
+
+
+def test_tree_router_errors_return_before_device_work(L):
+    import sparse_mixture_experts_expert_b200 as moe
+    s = _shape(moe, E=16)
+    P = ctypes.c_void_p
+    fake = P(4096)
+    n = ctypes.c_size_t(0)
+    assert L.moe_route_tree_workspace_size(ctypes.byref(s), 4, 2, ctypes.byref(n)) == 0
+    args = lambda x, ws, nb: (ctypes.byref(s), 4, 2, x, fake, None, fake, fake, None, None, ws, nb, None)
+    assert L.moe_route_tree(*args(None, fake, n.value)) == 1            # x missing
+    assert L.moe_route_tree(*args(P(4098), fake, n.value)) == 1         # misaligned x
+    assert L.moe_route_tree(*args(fake, fake, n.value - 256)) == 3      # workspace too small
+    assert L.moe_route_tree(*args(fake, P(4096 + 16), n.value)) == 1    # workspace not 256-byte aligned
+
+
+def test_backward_workspace_and_errors(L):
+    import sparse_mixture_experts_expert_b200 as moe
+    s = _shape(moe, H_s=64)
+    n, f = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert L.moe_backward_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert L.moe_workspace_size(ctypes.byref(s), ctypes.byref(f)) == 0
+    assert n.value > f.value        # the forward's regions plus the backward's own
+    P = ctypes.c_void_p
+    fake = P(4096)
+    head = lambda sh: [ctypes.byref(sh), fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
+                       ctypes.c_float(0.0), fake]
+    assert L.moe_backward_x(*head(s), fake, n.value - 256, None) == 3  # workspace too small
+    assert L.moe_backward(*head(s), None, None, None, None, None, fake, n.value - 256, None) == 3
+    assert L.moe_backward(*head(s), P(4100), None, None, None, None, fake, n.value, None) == 1  # misaligned dw13
+    sh = _shape(moe, H_s=64)
+    sh.wfmt = 1
+    assert L.moe_backward_x(*head(sh), fake, n.value, None) == 2       # INT4 experts: no backward
+    s0 = _shape(moe, H_s=64)
+    args = head(s0)
+    args[7] = None                                                      # shared expert without its weights
+    assert L.moe_backward_x(*args, fake, n.value, None) == 1
