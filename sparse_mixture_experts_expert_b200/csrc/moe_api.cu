@@ -894,8 +894,10 @@ static int route_impl(const moe_shape* s, const void* x, const float* w_router, 
 
 // ------------------------------------------------------------------ backward (input gradient)
 
-// Row splits of a dense weight gradient (one group of `rows` rows): about two waves of 148 tiles, at least 512
-// rows per split.  Independent of the device, so that the workspace size is.
+// Row splits of a dense weight gradient (one group of `rows` rows).  The time goes as the waves of tiles times
+// the rows per split, so n minimises ceil(n tiles / 148) / n over 1 <= n <= min(32, rows / 512), the fewest
+// splits among equals (fewer partials to add).  148 is B200's SM count; the rule does not ask the device, so
+// that the workspace size does not depend on it either.
 struct WgradSplit {
   int n, chunk;
 };
@@ -904,8 +906,10 @@ static int wgrad_bn(int N) { return N >= 256 ? 256 : (N > 64 ? 128 : 64); }
 constexpr int kWgradSplitRows = 2048;
 static WgradSplit wgrad_split(long long rows, int M, int N) {
   const long long tiles = cdiv(M, kBM) * cdiv(N, wgrad_bn(N));
-  long long n = std::min<long long>(cdiv(296, tiles), std::max<long long>(1, rows / 512));
-  n = std::max<long long>(1, std::min<long long>(n, 32));
+  const long long nmax = std::max<long long>(1, std::min<long long>(32, rows / 512));
+  long long n = 1;
+  for (long long c = 2; c <= nmax; ++c)   // waves(c) / c < waves(n) / n
+    if (cdiv(c * tiles, 148) * n < cdiv(n * tiles, 148) * c) n = c;
   const long long chunk = cdiv(cdiv(rows, n), 64) * 64;
   return WgradSplit{(int)cdiv(rows, chunk), (int)chunk};
 }
