@@ -757,14 +757,17 @@ def test_backward_x_load_balance_term_alone(lib, name, over):
 # rel-Frobenius per tensor, 3e-2 per expert (an expert's few rows average less).  skewed at 4096 tokens has
 # three experts above 2048 rows (3770, 2932, 2180), whose gradients are summed from 2048-row chunks.  The tiny
 # cases add a ragged token count (300: a partial 8-token block, a partial 64-row reduction step of the dense
-# gradients) and gates without renormalisation.
+# gradients) and gates without renormalisation; the last case has widths that are no multiple of 64 (d = 80,
+# H = 48, H_s = 32: partial TMA boxes in every GEMM and weight gradient), E = 6 and k = 3.
 @pytest.mark.parametrize("name,over,aux_coef", [("tiny", {"H_s": 64, "act": 1, "capacity_factor": 0.5}, 0.1),
                                                 ("tiny", {"T": 300, "H_s": 64}, 0.05),
                                                 ("tiny", {"T": 200, "renorm": 0}, 0.1),
                                                 ("small", {}, 0.05),
                                                 ("granular", {"T": 1024, "skew": 1.2}, 0.0),
                                                 ("skewed", {"T": 4096}, 0.0),
-                                                ("geglu", {"T": 512, "H": 1024}, 0.0)])
+                                                ("geglu", {"T": 512, "H": 1024}, 0.0),
+                                                ("tiny", {"T": 77, "d": 80, "E": 6, "k": 3, "H": 48, "H_s": 32,
+                                                          "act": 1, "skew": 0.5}, 0.2)])
 def test_backward_weights_match_oracle(lib, name, over, aux_coef):
     moe = lib
     wl = synth.get_workload(name).replace(**over)
