@@ -448,10 +448,12 @@ def run_backward(args, wl, world, rank, device):
     moe.load().moe_backward_workspace_size(ctypes.byref(s), ctypes.byref(n))
     ws = torch.empty(int(n.value), dtype=torch.uint8, device=device)
 
+    side = torch.cuda.Stream() if not args.one_stream else None   # the shared expert's chain runs beside
+
     def step():
         return moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
                                 w13t=t13, w2t=t2, w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"),
-                                w13t_sh=t13s, w2t_sh=t2s, aux_coef=0.01, ws=ws)
+                                w13t_sh=t13s, w2t_sh=t2s, aux_coef=0.01, ws=ws, side_stream=side)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -488,7 +490,9 @@ def run_backward(args, wl, world, rank, device):
                           "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                          "config": bench_config(wl, s.capacity, world), "mode": "backward (input and weight gradients)",
+                          "config": bench_config(wl, s.capacity, world),
+                          "mode": "backward (input and weight gradients)" + (", one stream" if args.one_stream else
+                                                                            ", shared expert on a side stream"),
                           "roofline": {"bound": "tensor", "kernel": "whole moe_backward",
                                        "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
                                        "unit": "TFLOP/s", "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
@@ -571,6 +575,8 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (moe_backward: input and weight gradients, bf16 experts) instead of the "
                          "forward")
+    ap.add_argument("--one-stream", action="store_true",
+                    help="--backward: keep the shared expert's chain on the main stream (no side stream)")
     ap.add_argument("--tree", action="store_true",
                     help="time the hierarchical router (moe_route_tree) on the workload's tokens, d and k over "
                          "--tree-branch ** --tree-levels experts, instead of the forward")

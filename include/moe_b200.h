@@ -278,11 +278,16 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
  * Precision: the weight gradients are bf16 GEMMs with fp32 accumulation over the rows of [dg | du], x,
  * dout, w h (bf16) and dz (bf16); a dense gradient (shared expert, router) sums row chunks in a fixed order.
  * Experts without kept rows get zeros.
+ *   side_stream  NULL, or a second stream of the caller's: the shared expert's chain (which needs only the
+ *                inputs) then runs there, forked from and joined back into `stream` by events, so that it
+ *                overlaps the routed chain.  The results are the same either way.  All work the call enqueues
+ *                is complete once `stream` passes the call's end.
  */
 int moe_backward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
                  const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
                  const void* dout, float aux_coef, float* dx, float* dw13, float* dw2, float* dw13_sh,
-                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream);
+                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream,
+                 moe_stream_t side_stream);
 
 /*
  * Hierarchical ("fractal") router (kieve-moe Features, "Fractal tiling routing": self-similar routing over a

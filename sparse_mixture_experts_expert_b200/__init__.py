@@ -91,7 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_transpose_experts": (ctypes.c_int, [_P, i64, i32, i32, _P, _P]),
         "moe_backward_workspace_size": (ctypes.c_int, [S, ctypes.POINTER(sz)]),
         "moe_backward_x": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float, _P, _P, sz, _P]),
-        "moe_backward": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float] + [_P] * 7 + [sz, _P]),
+        "moe_backward": (ctypes.c_int, [S] + [_P] * 10 + [ctypes.c_float] + [_P] * 7 + [sz, _P, _P]),
         "moe_route_tree_workspace_size": (ctypes.c_int, [S, i32, i32, ctypes.POINTER(sz)]),
         "moe_route_tree": (ctypes.c_int, [S, i32, i32] + [_P] * 8 + [sz, _P]),
     }
@@ -329,7 +329,7 @@ def moe_transpose_experts(w, *, out=None, stream=None):
 
 
 def _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef, ws,
-              stream, weights):
+              stream, weights, side_stream=None):
     T, d, E, H, Hs = shape.T, shape.d, shape.E, shape.H, shape.H_s
     _want(x, torch.bfloat16, (T, d), "x")
     _want(dout, torch.bfloat16, (T, d), "dout")
@@ -353,8 +353,9 @@ def _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh,
     g.update(dw13=torch.empty(E, 2 * H, d, **f32), dw2=torch.empty(E, d, H, **f32),
              dw13_sh=torch.empty(1, 2 * Hs, d, **f32) if Hs else None,
              dw2_sh=torch.empty(1, d, Hs, **f32) if Hs else None, dw_router=torch.empty(E, d, **f32))
+    side = ctypes.c_void_p(side_stream.cuda_stream) if side_stream is not None else None
     _check(_L().moe_backward(*head, _ptr(g["dw13"]), _ptr(g["dw2"]), _ptr(g["dw13_sh"]), _ptr(g["dw2_sh"]),
-                             _ptr(g["dw_router"]), *tail), "moe_backward")
+                             _ptr(g["dw_router"]), *tail, side), "moe_backward")
     return g
 
 
@@ -367,11 +368,12 @@ def moe_backward_x(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w1
 
 
 def moe_backward(shape: MoeShape, x, w_router, w13, w2, dout, *, bias=None, w13t=None, w2t=None, w13_sh=None,
-                 w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None):
+                 w2_sh=None, w13t_sh=None, w2t_sh=None, aux_coef=0.0, ws=None, stream=None, side_stream=None):
     """All gradients of L = sum(dout * out) + aux_coef * aux: a dict of fp32 tensors dx [T, d], dw13 [E, 2H, d],
-    dw2 [E, d, H], dw13_sh [1, 2H_s, d] and dw2_sh [1, d, H_s] (None without a shared expert), dw_router [E, d]."""
+    dw2 [E, d, H], dw13_sh [1, 2H_s, d] and dw2_sh [1, d, H_s] (None without a shared expert), dw_router [E, d].
+    ``side_stream`` (a torch.cuda.Stream) lets the shared expert's chain overlap the routed one."""
     return _backward(shape, x, w_router, w13, w2, dout, bias, w13t, w2t, w13_sh, w2_sh, w13t_sh, w2t_sh, aux_coef,
-                     ws, stream, True)
+                     ws, stream, True, side_stream)
 
 
 def moe_route_tree(shape: MoeShape, branch: int, levels: int, x, w_tree, bias_tree=None, *, counts=False,

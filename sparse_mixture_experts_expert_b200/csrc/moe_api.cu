@@ -917,7 +917,7 @@ static WgradSplit wgrad_split(long long rows, int M, int N) {
 // Scratch of moe_backward_x past the forward's regions (which it reuses: routing, grouping, x_perm for dx of the
 // grouped rows, h for dh').
 struct BwdWorkspace {
-  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, part, wpart, wlist, total;
+  size_t gu, doutp, gus, dhs, dxs, logits, dw, dz, wrt, dxr, part, partsh, wpart, wlist, total;
   int ldE;   // columns of dz and W_r^T: E rounded up to whole 64-column reduction steps
 };
 
@@ -938,18 +938,14 @@ static BwdWorkspace bwd_layout(const moe_shape* s) {
   B.dz = take((size_t)s->T * B.ldE * 2);
   B.wrt = take((size_t)s->d * B.ldE * 2);
   B.dxr = take((size_t)s->T * s->d * 2);
-  // split partials of the dense weight gradients: the router's, and the shared expert's two
-  size_t part = 0;
+  // split partials of the dense weight gradients: the router's, and (apart, since the shared expert's chain may
+  // run on a second stream) the shared expert's two
   auto need = [&](int M, int N) {
     const WgradSplit sp = wgrad_split(s->T, M, N);
-    if (sp.n > 1) part = std::max(part, (size_t)sp.n * M * N * 4);
+    return sp.n > 1 ? (size_t)sp.n * M * N * 4 : (size_t)0;
   };
-  need(s->E, s->d);
-  if (s->H_s > 0) {
-    need(2 * s->H_s, s->d);
-    need(s->d, s->H_s);
-  }
-  B.part = take(part);
+  B.part = take(need(s->E, s->d));
+  B.partsh = take(s->H_s > 0 ? std::max(need(2 * s->H_s, s->d), need(s->d, s->H_s)) : 0);
   // chunk partials of hot experts' weight gradients: the chunks of groups above kWgradSplitRows rows number at
   // most 2 R / kWgradSplitRows (each such group adds at most one partial chunk beyond R / kWgradSplitRows)
   B.wpart = take((size_t)2 * cdiv(R, kWgradSplitRows) * std::max(2 * s->H, s->H) * s->d * 4);
@@ -1342,7 +1338,8 @@ int moe_backward_workspace_size(const moe_shape* s, size_t* bytes) {
 int moe_backward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
                  const void* w13t, const void* w2t, const void* w13_sh, const void* w13t_sh, const void* w2t_sh,
                  const void* dout, float aux_coef, float* dx, float* dw13, float* dw2, float* dw13_sh,
-                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream) {
+                 float* dw2_sh, float* dw_router, void* workspace, size_t ws_bytes, moe_stream_t stream,
+                 moe_stream_t side_stream) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (s->wfmt != MOE_WFMT_BF16) return MOE_UNSUPPORTED_SHAPE;
@@ -1377,6 +1374,51 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   float* part = reinterpret_cast<float*>(ws + B.part);
   const long long R = grouped_rows(s);
   const bool pair = !(s->flags & MOE_FLAG_SINGLE_CTA_GEMM);
+
+  // shared expert on the tokens: [g | u] recomputed, dh = dout W2, [dg | du] (and h), its weight gradients,
+  // dx = [dg | du] W13.  It depends on the inputs only: with a side stream it runs there, beside the routed
+  // chain, from a fork event on `stream`, and joins before the final sum.
+  void* dxs = nullptr;
+  struct EventGuard {   // the join event is released however the call returns
+    cudaEvent_t e = nullptr;
+    ~EventGuard() { if (e != nullptr) cudaEventDestroy(e); }
+  } join;
+  cudaEvent_t& ev_join = join.e;
+  if (s->H_s > 0) {
+    cudaStream_t sst = st;
+    if (side_stream != nullptr && side_stream != stream) {
+      cudaEvent_t ev_fork = nullptr;
+      MOE_CUDA_TRY(cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming));
+      MOE_CUDA_TRY(cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming));
+      MOE_CUDA_TRY(cudaEventRecord(ev_fork, st));
+      MOE_CUDA_TRY(cudaStreamWaitEvent(side_stream, ev_fork, 0));
+      MOE_CUDA_TRY(cudaEventDestroy(ev_fork));
+      sst = side_stream;
+    }
+    float* partsh = reinterpret_cast<float*>(ws + B.partsh);
+    void* gus = ws + B.gus;
+    void* dhs = ws + B.dhs;
+    dxs = ws + B.dxs;
+    rc = grouped_gemm(kModePlain, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, 0, 2 * s->H_s, nullptr, nullptr, gus, sst,
+                      pair);
+    if (rc) return rc;
+    rc = grouped_gemm(kModePlain, dout, s->T, s->d, w2t_sh, 1, s->H_s, 0, s->H_s, nullptr, nullptr, dhs, sst, pair);
+    if (rc) return rc;
+    rc = launch_glu_bwd(s->act, gus, dhs, s->T, s->H_s, dw2_sh != nullptr, sst);
+    if (rc) return rc;
+    if (dw2_sh) {
+      rc = wgrad_gemm(dout, s->d, s->d, dhs, s->H_s, s->T, nullptr, nullptr, 1, dw2_sh, partsh, sst);
+      if (rc) return rc;
+    }
+    if (dw13_sh) {
+      rc = wgrad_gemm(gus, 2 * s->H_s, 2 * s->H_s, x, s->d, s->T, nullptr, nullptr, 1, dw13_sh, partsh, sst);
+      if (rc) return rc;
+    }
+    rc = grouped_gemm(kModePlain, gus, s->T, 2 * s->H_s, w13t_sh, 1, s->d, 0, s->d, nullptr, nullptr, dxs, sst,
+                      pair);
+    if (rc) return rc;
+    if (ev_join != nullptr) MOE_CUDA_TRY(cudaEventRecord(ev_join, sst));
+  }
 
   // forward recompute: routing, grouping, [g | u].  The softmax backward takes the logits of every expert: the
   // tensor-core screen's (two-term bf16 split of W_r, fp32 accumulation, within about 2^-16 |x| |w_e| of the
@@ -1414,33 +1456,6 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   rc = grouped_gemm(kModePlain, gu, R, 2 * s->H, w13t, s->E, s->d, 0, s->d, offs, kept, xperm, st, pair);
   if (rc) return rc;
 
-  // shared expert on the tokens: [g | u] recomputed, dh = dout W2, [dg | du] (and h), its weight gradients,
-  // dx = [dg | du] W13
-  void* dxs = nullptr;
-  if (s->H_s > 0) {
-    void* gus = ws + B.gus;
-    void* dhs = ws + B.dhs;
-    dxs = ws + B.dxs;
-    rc = grouped_gemm(kModePlain, x, s->T, s->d, w13_sh, 1, 2 * s->H_s, 0, 2 * s->H_s, nullptr, nullptr, gus, st,
-                      pair);
-    if (rc) return rc;
-    rc = grouped_gemm(kModePlain, dout, s->T, s->d, w2t_sh, 1, s->H_s, 0, s->H_s, nullptr, nullptr, dhs, st, pair);
-    if (rc) return rc;
-    rc = launch_glu_bwd(s->act, gus, dhs, s->T, s->H_s, dw2_sh != nullptr, st);
-    if (rc) return rc;
-    if (dw2_sh) {
-      rc = wgrad_gemm(dout, s->d, s->d, dhs, s->H_s, s->T, nullptr, nullptr, 1, dw2_sh, part, st);
-      if (rc) return rc;
-    }
-    if (dw13_sh) {
-      rc = wgrad_gemm(gus, 2 * s->H_s, 2 * s->H_s, x, s->d, s->T, nullptr, nullptr, 1, dw13_sh, part, st);
-      if (rc) return rc;
-    }
-    rc = grouped_gemm(kModePlain, gus, s->T, 2 * s->H_s, w13t_sh, 1, s->d, 0, s->d, nullptr, nullptr, dxs, st,
-                      pair);
-    if (rc) return rc;
-  }
-
   // router: dz through the gates, the statistic and the softmax, then dz W_r (bf16 operands, fp32 accumulation)
   // and dW_r = dz^T x
   const int epl = (int)cdiv(s->E, 32);
@@ -1468,6 +1483,7 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   if (rc) return rc;
 
   // dx = the token's grouped rows (slot order) + the shared expert's part + the router's part, fp32
+  if (ev_join != nullptr) MOE_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));
   MOE_LAUNCH((k_bwd_final), (unsigned)cdiv(s->T * (long long)(s->d / 8), 256), 256, 0, st,
              reinterpret_cast<const __nv_bfloat16*>(xperm), slot, reinterpret_cast<const __nv_bfloat16*>(dxs),
              reinterpret_cast<const __nv_bfloat16*>(dxr), (int)s->T, s->d, s->k, dx);
@@ -1480,7 +1496,7 @@ int moe_backward_x(const moe_shape* s, const void* x, const float* w_router, con
                    const void* dout, float aux_coef, float* dx, void* workspace, size_t ws_bytes,
                    moe_stream_t stream) {
   return moe_backward(s, x, w_router, bias, w13, w13t, w2t, w13_sh, w13t_sh, w2t_sh, dout, aux_coef, dx, nullptr,
-                      nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes, stream);
+                      nullptr, nullptr, nullptr, nullptr, workspace, ws_bytes, stream, nullptr);
 }
 
 int moe_route_tree_workspace_size(const moe_shape* s, int32_t branch, int32_t levels, size_t* bytes) {

@@ -163,8 +163,8 @@ def test_backward_workspace_and_errors(L):
     head = lambda sh: [ctypes.byref(sh), fake, fake, None, fake, fake, fake, fake, fake, fake, fake,
                        ctypes.c_float(0.0), fake]
     assert L.moe_backward_x(*head(s), fake, n.value - 256, None) == 3  # workspace too small
-    assert L.moe_backward(*head(s), None, None, None, None, None, fake, n.value - 256, None) == 3
-    assert L.moe_backward(*head(s), P(4100), None, None, None, None, fake, n.value, None) == 1  # misaligned dw13
+    assert L.moe_backward(*head(s), None, None, None, None, None, fake, n.value - 256, None, None) == 3
+    assert L.moe_backward(*head(s), P(4100), None, None, None, None, fake, n.value, None, None) == 1  # misaligned dw13
     sh = _shape(moe, H_s=64)
     sh.wfmt = 1
     assert L.moe_backward_x(*head(sh), fake, n.value, None) == 2       # INT4 experts: no backward

@@ -778,9 +778,13 @@ def test_backward_weights_match_oracle(lib, name, over, aux_coef):
     kw = dict(bias=inp["bias"], w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), aux_coef=aux_coef)
     got = moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, **kw)
     dx_only = moe.moe_backward_x(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, **kw)
+    side = moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, side_stream=torch.cuda.Stream(),
+                            **kw)
     torch.cuda.synchronize()
     assert moe.moe_get_status()[0] == 0
     assert torch.equal(got["dx"], dx_only)   # the weight gradients leave the input gradient's path unchanged
+    for key, v in got.items():               # the shared expert's chain on a second stream: the same results
+        assert (v is None and side[key] is None) or torch.equal(v, side[key]), key
     b64 = np64(inp["bias"]) if inp["bias"] is not None else None
     ref = O.moe_backward(np64(inp["x"]), np64(inp["w_router"]), b64, np64(inp["w13"]), np64(inp["w2"]),
                          np64(dout), k=wl.k, act=wl.act, renorm=bool(wl.renorm), cap=s.capacity,
