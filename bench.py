@@ -197,11 +197,11 @@ def int4_weights(moe, wl, seed, device):
     return out
 
 
-def run_forward(moe, s, inp, ws, out, aux):
+def run_forward(moe, s, inp, ws, out, aux, side=None):
     return moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
                            s13=inp.get("s13"), s2=inp.get("s2"), w13_sh=inp.get("w13_sh"),
                            s13_sh=inp.get("s13_sh"), w2_sh=inp.get("w2_sh"), s2_sh=inp.get("s2_sh"), out=out,
-                           ws=ws, aux=aux)
+                           ws=ws, aux=aux, side_stream=side)
 
 
 def stage_times(moe, s, inp, ws, wl, flush, reps=10):
@@ -576,7 +576,8 @@ def main():
                     help="time the backward (moe_backward: input and weight gradients, bf16 experts) instead of the "
                          "forward")
     ap.add_argument("--one-stream", action="store_true",
-                    help="--backward: keep the shared expert's chain on the main stream (no side stream)")
+                    help="keep the shared expert on the main stream (by default it runs on a side stream, "
+                         "beside the routed path)")
     ap.add_argument("--tree", action="store_true",
                     help="time the hierarchical router (moe_route_tree) on the workload's tokens, d and k over "
                          "--tree-branch ** --tree-levels experts, instead of the forward")
@@ -649,8 +650,9 @@ def main():
         flushbuf.fill_(1)
 
     st = torch.cuda.current_stream()
+    side = torch.cuda.Stream() if not args.one_stream else None   # the shared expert beside the routed path
     for _ in range(max(3, args.warmup)):
-        run_forward(moe, s, inp, ws, out, wl.aux)
+        run_forward(moe, s, inp, ws, out, wl.aux, side)
     torch.cuda.synchronize()
     status, site = moe.moe_get_status()
     if status != 0:
@@ -661,7 +663,7 @@ def main():
     launches0 = moe.moe_launch_count()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run_forward(moe, s, inp, ws, out, wl.aux)
+        run_forward(moe, s, inp, ws, out, wl.aux, side)
     per_step_launches = moe.moe_launch_count() - launches0
     torch.cuda.synchronize()
     for _ in range(2):
@@ -719,7 +721,7 @@ def main():
                 flush()
                 inp_i = dict(inp)
                 inp_i["x"] = x_dev[b]
-                run_forward(moe, s, inp_i, ws, out_dev[b], wl.aux)
+                run_forward(moe, s, inp_i, ws, out_dev[b], wl.aux, side)
                 fwd_done[i].record(cs)
             with torch.cuda.stream(ds):
                 ds.wait_event(fwd_done[i])
@@ -784,7 +786,8 @@ def main():
                         "overlap": "copy streams: step i+1's H2D and step i-1's D2H overlap step i's forward"},
                 "gpu_launches": launches, "launches_per_step": per_step_launches,
                 "timing": "CUDA graph of one moe_forward replayed per step (value); e2e calls the API eagerly, "
-                          "copies pipelined with the forwards",
+                          "copies pipelined with the forwards; shared expert "
+                          + ("on the main stream" if args.one_stream else "on a side stream beside the routed path"),
                 "clocks": clk.summary()}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -222,12 +222,16 @@ int moe_combine(const moe_shape* s, const void* y_perm, const int32_t* slot_pos,
  * INT4 experts: the activations are scaled per row by a power of two and rounded to f16 (exact for bf16
  * inputs from 2^-28 of the row's largest |x| up); the weights enter the MMAs as exact f16 integer codes
  * with a per-group offset that is removed in fp32, and the bf16 group scales multiply the fp32 group sums.
+ *   side_stream  NULL, or a second stream of the caller's: with bf16 experts and a shared expert, the shared
+ *                expert (which needs only x) runs there, forked from `stream` by an event at the start and
+ *                joined back before the combine, so that it overlaps the routing, grouping and routed experts.
+ *                The output is the same bit for bit.  All work is complete once `stream` passes the call's end.
  */
 int moe_forward(const moe_shape* s, const void* x, const float* w_router, const float* bias, const void* w13,
                 const void* s13, const void* w2, const void* s2, const void* w13_sh, const void* s13_sh,
                 const void* w2_sh, const void* s2_sh, void* out, int32_t* topk_idx, float* topk_w,
                 int32_t* counts, uint8_t* drop_mask, float* aux_f, float* aux_p, float* aux, void* workspace,
-                size_t ws_bytes, moe_stream_t stream);
+                size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream);
 
 /*
  * Transposed copies of expert weights for the backward pass: wt[i][c][r] = w[i][r][c] for i < n, bf16.

@@ -80,7 +80,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute": (ctypes.c_int, [S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P]),
         "moe_expert_ffn": (ctypes.c_int, [S, i32, i32, i64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moe_combine": (ctypes.c_int, [S, _P, _P, _P, _P, _P, _P]),
-        "moe_forward": (ctypes.c_int, [S] + [_P] * 20 + [sz, _P]),
+        "moe_forward": (ctypes.c_int, [S] + [_P] * 20 + [sz, _P, _P]),
         "moe_quantize_int4": (ctypes.c_int, [_P, i64, i32, _P, _P, _P]),
         "moe_get_status": (ctypes.c_int, [_P, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_uint32)]),
         "moe_set_wait_limit_ns": (ctypes.c_int, [u64]),
@@ -288,8 +288,9 @@ def moe_combine(shape: MoeShape, y_perm, slot_pos, topk_w, y_shared=None, *, out
 
 
 def moe_forward(shape: MoeShape, x, w_router, w13, w2, *, bias=None, s13=None, s2=None, w13_sh=None, s13_sh=None,
-                w2_sh=None, s2_sh=None, out=None, routing=False, aux=False, ws=None, stream=None):
-    """The whole layer.  Returns ``out`` [T, d] bf16, or a dict with routing outputs when asked."""
+                w2_sh=None, s2_sh=None, out=None, routing=False, aux=False, ws=None, stream=None, side_stream=None):
+    """The whole layer.  Returns ``out`` [T, d] bf16, or a dict with routing outputs when asked.
+    ``side_stream`` (a torch.cuda.Stream) lets a bf16 shared expert overlap the routing and routed experts."""
     T, d, E, k = shape.T, shape.d, shape.E, shape.k
     _want(x, torch.bfloat16, (T, d), "x")
     dev = x.device
@@ -310,7 +311,8 @@ def moe_forward(shape: MoeShape, x, w_router, w13, w2, *, bias=None, s13=None, s
                           _ptr(s2), _ptr(w13_sh), _ptr(s13_sh), _ptr(w2_sh), _ptr(s2_sh), _ptr(out),
                           _ptr(r.get("topk_idx")), _ptr(r.get("topk_w")), _ptr(r.get("counts")),
                           _ptr(r.get("drop_mask")), _ptr(r.get("aux_f")), _ptr(r.get("aux_p")), _ptr(r.get("aux")),
-                          _ptr(ws), ws.numel(), _stream(stream))
+                          _ptr(ws), ws.numel(), _stream(stream),
+                          ctypes.c_void_p(side_stream.cuda_stream) if side_stream is not None else None)
     _check(rc, "moe_forward")
     if r:
         r["out"] = out

@@ -1103,6 +1103,23 @@ static TreeWorkspace tree_layout(const moe_shape* s, int n) {
   return W;
 }
 
+// Fork of independent work onto a caller's second stream: an event recorded on `main` that `side` waits for,
+// and a join event (owned here, released however the call returns) that `main` waits for later.
+struct SideFork {
+  cudaEvent_t join = nullptr;
+  ~SideFork() { if (join != nullptr) cudaEventDestroy(join); }
+  int start(cudaStream_t main, cudaStream_t side) {
+    cudaEvent_t fork = nullptr;
+    if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess) return MOE_CUDA_ERROR;
+    const bool ok = cudaEventCreateWithFlags(&join, cudaEventDisableTiming) == cudaSuccess &&
+                    cudaEventRecord(fork, main) == cudaSuccess && cudaStreamWaitEvent(side, fork, 0) == cudaSuccess;
+    cudaEventDestroy(fork);
+    return ok ? MOE_OK : MOE_CUDA_ERROR;
+  }
+  int end(cudaStream_t side) { return cudaEventRecord(join, side) == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR; }
+  int wait(cudaStream_t main) { return cudaStreamWaitEvent(main, join, 0) == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR; }
+};
+
 }  // namespace moe
 
 using namespace moe;
@@ -1251,7 +1268,7 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
                 const void* s13, const void* w2, const void* s2, const void* w13_sh, const void* s13_sh,
                 const void* w2_sh, const void* s2_sh, void* out, int32_t* topk_idx, float* topk_w,
                 int32_t* counts, uint8_t* drop_mask, float* aux_f, float* aux_p, float* aux, void* workspace,
-                size_t ws_bytes, moe_stream_t stream) {
+                size_t ws_bytes, moe_stream_t stream, moe_stream_t side_stream) {
   int rc = check_shape(s);
   if (rc) return rc;
   if (!x || !w_router || !w13 || !w2 || !out || !workspace) return MOE_INVALID_ARGUMENT;
@@ -1276,12 +1293,29 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   void* hbuf = ws + L.h;
   void* yperm = ws + L.yperm;
   const long long R = grouped_rows(s);
+  const bool int4 = s->wfmt == MOE_WFMT_INT4_G128;
+
+  // bf16 experts: the shared expert needs only x, so with a side stream it runs there from the start, beside the
+  // routing, grouping and routed experts, and joins before the combine.  (INT4: its activation copy is formed
+  // with the routed one, so it stays in order.)
+  void* ys = nullptr;
+  SideFork fork;
+  const bool forked = s->H_s > 0 && !int4 && side_stream != nullptr && side_stream != stream;
+  if (forked) {
+    rc = fork.start(stream, side_stream);
+    if (rc) return rc;
+    ys = ws + L.ys;
+    rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
+                         side_stream, Int4Scratch{nullptr, nullptr, nullptr});
+    if (rc) return rc;
+    rc = fork.end(side_stream);
+    if (rc) return rc;
+  }
 
   rc = route_impl(s, x, w_router, bias, nullptr, nullptr, idx, w, cts, aux_f, aux_p, aux, ws, stream, true);
   if (rc) return rc;
   const float* f_used = aux_f ? aux_f : reinterpret_cast<const float*>(ws + L.fP);
   const float* p_used = aux_p ? aux_p : reinterpret_cast<const float*>(ws + L.fP) + s->E;
-  const bool int4 = s->wfmt == MOE_WFMT_INT4_G128;
   // INT4: the grouped activation copy is formed by k_int4_act_prep from x and the slots, so no bf16 rows move
   rc = launch_scatter(s, x, idx, cnt, cts, slot, drop_mask, nullptr, xperm, kept, offs, stream, !int4, f_used, p_used,
                       aux);
@@ -1308,13 +1342,13 @@ int moe_forward(const moe_shape* s, const void* x, const float* w_router, const 
   }
   rc = expert_ffn_impl(s, s->H, R, xperm, offs, kept, s->E, w13, s13, w2, s2, hbuf, yperm, stream, scr_routed);
   if (rc) return rc;
-  void* ys = nullptr;
-  if (s->H_s > 0) {
+  if (s->H_s > 0 && !forked) {
     ys = ws + L.ys;
     rc = expert_ffn_impl(s, s->H_s, s->T, x, nullptr, nullptr, 1, w13_sh, s13_sh, w2_sh, s2_sh, ws + L.hs, ys,
                          stream, scr_shared);
     if (rc) return rc;
   }
+  if (forked && (rc = fork.wait(stream))) return rc;
   return moe_combine(s, yperm, slot, w, ys, out, stream);
 }
 
@@ -1379,20 +1413,13 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   // dx = [dg | du] W13.  It depends on the inputs only: with a side stream it runs there, beside the routed
   // chain, from a fork event on `stream`, and joins before the final sum.
   void* dxs = nullptr;
-  struct EventGuard {   // the join event is released however the call returns
-    cudaEvent_t e = nullptr;
-    ~EventGuard() { if (e != nullptr) cudaEventDestroy(e); }
-  } join;
-  cudaEvent_t& ev_join = join.e;
+  SideFork fork;
+  const bool forked = s->H_s > 0 && side_stream != nullptr && side_stream != stream;
   if (s->H_s > 0) {
     cudaStream_t sst = st;
-    if (side_stream != nullptr && side_stream != stream) {
-      cudaEvent_t ev_fork = nullptr;
-      MOE_CUDA_TRY(cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming));
-      MOE_CUDA_TRY(cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming));
-      MOE_CUDA_TRY(cudaEventRecord(ev_fork, st));
-      MOE_CUDA_TRY(cudaStreamWaitEvent(side_stream, ev_fork, 0));
-      MOE_CUDA_TRY(cudaEventDestroy(ev_fork));
+    if (forked) {
+      rc = fork.start(st, side_stream);
+      if (rc) return rc;
       sst = side_stream;
     }
     float* partsh = reinterpret_cast<float*>(ws + B.partsh);
@@ -1417,7 +1444,7 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
     rc = grouped_gemm(kModePlain, gus, s->T, 2 * s->H_s, w13t_sh, 1, s->d, 0, s->d, nullptr, nullptr, dxs, sst,
                       pair);
     if (rc) return rc;
-    if (ev_join != nullptr) MOE_CUDA_TRY(cudaEventRecord(ev_join, sst));
+    if (forked && (rc = fork.end(sst))) return rc;
   }
 
   // forward recompute: routing, grouping, [g | u].  The softmax backward takes the logits of every expert: the
@@ -1483,7 +1510,7 @@ int moe_backward(const moe_shape* s, const void* x, const float* w_router, const
   if (rc) return rc;
 
   // dx = the token's grouped rows (slot order) + the shared expert's part + the router's part, fp32
-  if (ev_join != nullptr) MOE_CUDA_TRY(cudaStreamWaitEvent(st, ev_join, 0));
+  if (forked && (rc = fork.wait(st))) return rc;
   MOE_LAUNCH((k_bwd_final), (unsigned)cdiv(s->T * (long long)(s->d / 8), 256), 256, 0, st,
              reinterpret_cast<const __nv_bfloat16*>(xperm), slot, reinterpret_cast<const __nv_bfloat16*>(dxs),
              reinterpret_cast<const __nv_bfloat16*>(dxr), (int)s->T, s->d, s->k, dx);

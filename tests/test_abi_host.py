@@ -115,7 +115,7 @@ def test_null_and_workspace_errors_return_before_device_work(L):
                      None)
     assert rc == 1            # misaligned x
     rc = L.moe_forward(ctypes.byref(s), fake, fake, None, fake, None, fake, None, None, None, None, None, fake,
-                       None, None, None, None, None, None, None, fake, 16, None)
+                       None, None, None, None, None, None, None, fake, 16, None, None)
     assert rc == 3
     rc = L.moe_quantize_int4(fake, 4, 100, fake, fake, None)
     assert rc == 1            # K % 128 != 0

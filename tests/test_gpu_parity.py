@@ -808,3 +808,31 @@ def test_backward_weights_match_oracle(lib, name, over, aux_coef):
                 assert rel_frob(a[e], b[e]) <= 3 * BWD_REL_FROB, f"{key}[{e}] ({kept[e]} rows)"
     if not wl.H_s:
         assert got["dw13_sh"] is None and got["dw2_sh"] is None
+
+
+# The shared expert on a second stream (moe_forward's side_stream) changes nothing in the output: the same kernels
+# on the same inputs, joined before the combine.
+@pytest.mark.parametrize("name,over", [("granular", {"T": 4096}), ("tiny", {"H_s": 64}), ("small", {})])
+def test_forward_side_stream_is_bit_identical(lib, name, over):
+    moe = lib
+    wl = synth.get_workload(name).replace(**over)
+    inp = synth.make_inputs(wl, seed=5, device=DEV)
+    s = shape_of(moe, wl)
+    kw = dict(bias=inp["bias"], w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), routing=True)
+    a = moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], **kw)
+    side = torch.cuda.Stream()
+    b = moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], side_stream=side, **kw)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    for key in ("out", "topk_idx", "topk_w", "counts", "drop_mask"):
+        assert torch.equal(a[key], b[key]), key
+    # and inside a captured graph, replayed
+    g = torch.cuda.CUDAGraph()
+    out = torch.empty_like(a["out"])
+    with torch.cuda.graph(g):
+        moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
+                        w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), out=out, side_stream=side)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, a["out"])
+    del g
