@@ -836,3 +836,31 @@ def test_forward_side_stream_is_bit_identical(lib, name, over):
     torch.cuda.synchronize()
     assert torch.equal(out, a["out"])
     del g
+
+
+# The autograd wrapper: gradients of loss = sum(dout * out) through torch.autograd equal moe_backward's (cast to
+# the parameters' dtypes), and the output equals moe_forward's.
+def test_autograd_layer_matches_the_entry_points(lib):
+    from sparse_mixture_experts_expert_b200.autograd import moe_layer
+    moe = lib
+    wl = synth.get_workload("tiny").replace(H_s=64, skew=0.5)
+    inp = synth.make_inputs(wl, seed=9, device=DEV)
+    s = shape_of(moe, wl)
+    g = torch.Generator(device=DEV).manual_seed(3)
+    dout = torch.randn(wl.T, wl.d, generator=g, device=DEV).to(torch.bfloat16)
+    leaves = {k: inp[k].clone().requires_grad_(True) for k in ("x", "w_router", "w13", "w2", "w13_sh", "w2_sh")}
+    out, aux = moe_layer(s, leaves["x"], leaves["w_router"], leaves["w13"], leaves["w2"], bias=inp["bias"],
+                         w13_sh=leaves["w13_sh"], w2_sh=leaves["w2_sh"], aux_coef=0.1, return_aux=True)
+    (out.float() * dout.float()).sum().backward()
+    ref_out = moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
+                              w13_sh=inp["w13_sh"], w2_sh=inp["w2_sh"])
+    ref = moe.moe_backward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], dout, bias=inp["bias"],
+                           w13_sh=inp["w13_sh"], w2_sh=inp["w2_sh"], aux_coef=0.1)
+    torch.cuda.synchronize()
+    assert moe.moe_get_status()[0] == 0
+    assert torch.equal(out, ref_out) and not aux.requires_grad
+    pairs = [("x", "dx"), ("w_router", "dw_router"), ("w13", "dw13"), ("w2", "dw2"), ("w13_sh", "dw13_sh"),
+             ("w2_sh", "dw2_sh")]
+    for leaf, key in pairs:
+        assert leaves[leaf].grad is not None and leaves[leaf].grad.dtype == leaves[leaf].dtype, leaf
+        assert torch.equal(leaves[leaf].grad, ref[key].to(leaves[leaf].dtype)), leaf
