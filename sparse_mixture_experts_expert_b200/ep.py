@@ -21,8 +21,16 @@ Each (token, slot) row gets the expert output the single-GPU forward gives it, a
 same slot order, so with bf16 experts the output equals ``moe_forward`` on the rank's tokens bit for bit.
 
 The row counts reach the host as the splits of the exchanges: one device synchronisation per forward.
-Capacity-factor dispatch is not supported: its ranks are global in token order across all ranks.
-The exchanges are NCCL all-to-all-v calls (``torch.distributed``), not fused with the expert GEMMs.
+
+With a capacity (``shape.capacity = C > 0``, the same C on every rank: the MoEEvolve README's capacity-factor
+dispatch with static shapes) the exchange has static shapes instead.  Each rank groups its own tokens with
+capacity C (ranks counted in its token order, as ``moe_forward`` with capacity C on those tokens), so the rows for
+rank q are always E_loc * C rows, kept ones first in each expert's block.  Both exchanges then use equal splits
+and the receiver's local grouping is a fixed pattern, so nothing reaches the host and the whole forward can be
+captured in a CUDA graph.  The price is the padding rows: they cross the exchange and run through the local
+experts (their outputs are never combined).  Output: ``moe_forward`` with capacity C on the rank's tokens.
+
+The exchanges are NCCL all-to-all calls (``torch.distributed``), not fused with the expert GEMMs.
 """
 
 from __future__ import annotations
@@ -64,7 +72,8 @@ def moe_forward_ep(shape: MoeShape, x, w_router, w13_local, w2_local, *, bias=No
                    s2_local=None, w13_sh=None, s13_sh=None, w2_sh=None, s2_sh=None, group=None, ops=None):
     """Expert-parallel layer forward on this rank's tokens.
 
-    shape       the layer (E = all routed experts across the group; T = this rank's tokens; capacity 0)
+    shape       the layer (E = all routed experts across the group; T = this rank's tokens; capacity 0 for
+                the exchange of exact counts, or C > 0, the same on every rank, for static shapes)
     x           [T, d] this rank's tokens
     w_router    [E, d] fp32, the same on every rank
     w13_local, w2_local (s13_local, s2_local)   this rank's E / G experts, layout as for moe_forward
@@ -74,11 +83,12 @@ def moe_forward_ep(shape: MoeShape, x, w_router, w13_local, w2_local, *, bias=No
     ops = ops if ops is not None else KernelOps()
     G = dist.get_world_size(group)
     E, k, T, d = shape.E, shape.k, shape.T, shape.d
-    if shape.capacity != 0:
-        raise ValueError("moe_forward_ep: capacity-factor dispatch is not supported across ranks")
     if E % G != 0 or w13_local.shape[0] != E // G:
         raise ValueError(f"moe_forward_ep: {E} experts do not split into {G} ranks of {w13_local.shape[0]}")
     E_loc = E // G
+    if shape.capacity > 0:
+        return _forward_ep_static(shape, x, w_router, w13_local, w2_local, bias, s13_local, s2_local, w13_sh,
+                                  s13_sh, w2_sh, s2_sh, group, ops, G, E_loc)
     s_route = _shape(shape, T, E, k, 0)
 
     # 1-2. route over all experts, group the (token, slot) pairs by global expert
@@ -120,5 +130,34 @@ def moe_forward_ep(shape: MoeShape, x, w_router, w13_local, w2_local, *, bias=No
     y_sh = None
     if shape.H_s > 0:   # one dense group of the T local tokens
         y_sh = ops.expert_ffn(s_route, x, w13_sh, w2_sh, shape.H_s, s13=s13_sh, s2=s2_sh)
+    out = ops.combine(s_route, y_back, p["slot_pos"], topk_w, y_sh)
+    return out, topk_idx, topk_w
+
+
+def _forward_ep_static(shape, x, w_router, w13_local, w2_local, bias, s13_local, s2_local, w13_sh, s13_sh, w2_sh,
+                       s2_sh, group, ops, G, E_loc):
+    """moe_forward_ep with capacity C: equal all-to-all splits, no host synchronisation."""
+    E, k, T, d, C = shape.E, shape.k, shape.T, shape.d, shape.capacity
+    s_route = MoeShape(T=T, d=d, E=E, k=k, H=shape.H, H_s=0, capacity=C, act=shape.act, wfmt=shape.wfmt,
+                       renorm=shape.renorm, flags=shape.flags)
+    topk_idx, topk_w = ops.route(s_route, x, w_router, bias)
+    p = ops.permute(s_route, x, topk_idx)
+    x_perm = p["x_perm"]                       # [E C, d]: expert e's block at rows [e C, (e + 1) C), kept rows first
+    x_recv = x_perm.new_empty((E * C, d))      # [G][E_loc][C]: from each source rank, its blocks of my experts
+    dist.all_to_all_single(x_recv, x_perm, group=group)
+    # every received row goes to the local expert of its block: a fixed pattern (padding rows included)
+    ids = np.tile(np.repeat(np.arange(E_loc, dtype=np.int32), C), G)
+    local_idx = torch.from_numpy(ids).to(topk_idx.device).view(E * C, 1)
+    s_loc = _shape(shape, E * C, E_loc, 1, 0)
+    q = ops.permute(s_loc, x_recv, local_idx)
+    y_grouped = ops.expert_ffn(s_loc, q["x_perm"], w13_local, w2_local, shape.H, group_start=q["offsets"][:E_loc],
+                               group_rows=q["kept"], s13=s13_local, s2=s2_local)
+    ones = torch.ones(E * C, 1, dtype=topk_w.dtype, device=topk_w.device)
+    y_recv = ops.combine(s_loc, y_grouped, q["slot_pos"], ones)
+    y_back = torch.empty_like(y_recv)
+    dist.all_to_all_single(y_back, y_recv, group=group)
+    y_sh = None
+    if shape.H_s > 0:
+        y_sh = ops.expert_ffn(_shape(shape, T, E, k, 0), x, w13_sh, w2_sh, shape.H_s, s13=s13_sh, s2=s2_sh)
     out = ops.combine(s_route, y_back, p["slot_pos"], topk_w, y_sh)
     return out, topk_idx, topk_w

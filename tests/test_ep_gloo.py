@@ -3,7 +3,9 @@
 The per-rank steps (route, grouping, expert FFN, combine) run on the float64 oracle, the exchanges on
 torch.distributed all-to-all; every rank's output must equal the single-process oracle layer on its tokens.
 Cases: a balanced routing, an odd token split with three experts per rank and a skew, and a routing that sends
-every row to rank 0's experts (rank 1 receives nothing).
+every row to rank 0's experts (rank 1 receives nothing).  With a capacity C (static shapes: equal all-to-all
+splits, padding rows included) every rank's output must equal the oracle layer with capacity C on its own
+tokens, drops included.
 """
 
 import os
@@ -34,9 +36,9 @@ class OracleOps:
         return self.torch.from_numpy(r["idx"].astype(np.int32)), self.torch.from_numpy(r["w"])
 
     def permute(self, shape, x, topk_idx):
-        p = self.O.permute(topk_idx.numpy(), shape.E, 0)
+        p = self.O.permute(topk_idx.numpy(), shape.E, shape.capacity)
         rs = p["row_src"]
-        x_perm = np.zeros((shape.T * shape.k, shape.d))
+        x_perm = np.zeros((shape.R, shape.d))
         x_perm[rs >= 0] = x.numpy()[rs[rs >= 0] // shape.k]
         t = lambda a: self.torch.from_numpy(np.ascontiguousarray(a).astype(np.int32))
         return dict(x_perm=self.torch.from_numpy(x_perm), slot_pos=t(p["slot_pos"]), counts=t(p["counts"]),
@@ -91,7 +93,7 @@ def _reference(case):
     return out, r["idx"]
 
 
-def _worker(rank, world, port, case, q):
+def _worker(rank, world, port, case, q, cap=0):
     import sys
     from datetime import timedelta
 
@@ -111,7 +113,7 @@ def _worker(rank, world, port, case, q):
         E_loc = E // world
         mine = slice(rank * E_loc, (rank + 1) * E_loc)
         f = torch.from_numpy
-        shape = moe.MoeShape(T=len(toks), d=d, E=E, k=k, H=H, H_s=H_s, capacity=0, act=0, wfmt=0, renorm=1)
+        shape = moe.MoeShape(T=len(toks), d=d, E=E, k=k, H=H, H_s=H_s, capacity=cap, act=0, wfmt=0, renorm=1)
         out, idx, _ = moe_forward_ep(shape, f(x[toks].copy()), f(w_r), f(w13[mine].copy()), f(w2[mine].copy()),
                                      bias=f(bias), w13_sh=None if w13_sh is None else f(w13_sh),
                                      w2_sh=None if w2_sh is None else f(w2_sh), ops=OracleOps(O, torch))
@@ -138,3 +140,31 @@ def test_expert_parallel_two_ranks_matches_the_single_process_layer(case):
     for rank, toks, out, idx in got:
         assert (idx == ref_idx[toks]).all()
         np.testing.assert_allclose(out, ref[toks], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("case,cap", [((40, 32, 8, 2, 32, 16, "skew"), 6), ((33, 32, 6, 3, 16, 0, "skew"), 4),
+                                      ((24, 16, 8, 2, 16, 16, "rank0"), 3)])
+def test_expert_parallel_static_capacity_matches_the_per_rank_layer(case, cap):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import oracle as O
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, case, q, cap)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(2)]
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    T, d, E, k, H, H_s, mode = case
+    x, w_r, bias, w13, w2, w13_sh, w2_sh = _problem(case)
+    dropped = 0
+    for rank, toks, out, idx in got:
+        ref = O.moe_forward(x[toks], w_r, bias, w13, w2, k=k, act=0, renorm=True, cap=cap, w13_sh=w13_sh,
+                            w2_sh=w2_sh)
+        dropped += int(ref["drop"].sum())
+        assert (idx == ref["idx"]).all()
+        np.testing.assert_allclose(out, ref["out"], rtol=1e-10, atol=1e-12)
+    assert dropped > 0   # the capacity binds somewhere

@@ -638,10 +638,13 @@ def test_forward_int4_full_size(lib):
 
 
 @pytest.mark.parametrize("name,over", [("tiny", {}), ("granular", {"T": 2048, "skew": 1.2, "capacity_factor": 0.0}),
-                                       ("small", {})])
+                                       ("small", {}), ("tiny", {"capacity_factor": 0.5}),
+                                       ("granular", {"T": 2048, "skew": 1.2, "capacity_factor": 1.0})])
 def test_expert_parallel_single_rank_equals_forward(lib, name, over):
     """moe_forward_ep on one NCCL rank (the exchanges are identities) runs the same kernels on the same grouped
-    rows as moe_forward, so the outputs agree bit for bit; the two-rank exchange is covered on gloo (CPU)."""
+    rows as moe_forward, so the outputs agree bit for bit; the two-rank exchange is covered on gloo (CPU).  With a
+    capacity the static-shape exchange also runs the padding rows through the experts, which changes no kept
+    row's output."""
     import socket
     from datetime import timedelta
 
@@ -669,7 +672,7 @@ def _ep_single_rank_case(moe, moe_forward_ep, name, over):
     wl = synth.get_workload(name).replace(**over)
     inp = synth.make_inputs(wl, seed=5, device=DEV)
     s = shape_of(moe, wl)
-    assert s.capacity == 0
+    assert (s.capacity > 0) == (wl.capacity_factor > 0)
     ref = moe.moe_forward(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
                           w13_sh=inp.get("w13_sh"), w2_sh=inp.get("w2_sh"), routing=True)
     out, idx, w = moe_forward_ep(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], bias=inp["bias"],
