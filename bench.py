@@ -368,8 +368,9 @@ def cpu_oracle_sample(wl, budget_s=12.0, single_thread=False):
 
 def run_ep(args, wl, world, rank, device):
     """Expert-parallel timing: rank r holds experts [r E/N, (r + 1) E/N) and its own T tokens (weak scaling);
-    moe_forward_ep runs eagerly (its splits reach the host), L2 flushed before every step, the step time is
-    the max over ranks of the mean device time between events around each forward."""
+    moe_forward_ep runs eagerly (without a capacity its splits reach the host; with one the exchange has static
+    shapes), L2 flushed before every step, the step time is the max over ranks of the mean device time between
+    events around each forward."""
     import socket
     from datetime import timedelta
 
@@ -379,8 +380,8 @@ def run_ep(args, wl, world, rank, device):
     import sparse_mixture_experts_expert_b200 as moe
     import synth
     from sparse_mixture_experts_expert_b200.ep import moe_forward_ep
-    if wl.capacity_factor or wl.wfmt != synth.WFMT_BF16 or wl.E % world:
-        raise SystemExit("--ep takes bf16 workloads without a capacity whose experts split evenly over the ranks")
+    if wl.wfmt != synth.WFMT_BF16 or wl.E % world:
+        raise SystemExit("--ep takes bf16 workloads whose experts split evenly over the ranks")
     own = not dist.is_initialized()
     if own:   # one rank: a process group of one, the exchanges are local copies
         sk = socket.socket()
@@ -418,8 +419,9 @@ def run_ep(args, wl, world, rank, device):
         raise RuntimeError(f"device status {status} at {site:#x} in the timed region")
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
     if rank == 0:
-        cfg = bench_config(wl, 0, world)
-        cfg["parallelism"] = f"expert-parallel x{world} (E/N experts per rank, NCCL all-to-all-v)"
+        cfg = bench_config(wl, s.capacity, world)
+        cfg["parallelism"] = (f"expert-parallel x{world} (E/N experts per rank, NCCL all-to-all"
+                              + (", static shapes with the capacity)" if s.capacity else "-v)"))
         print(json.dumps({"metric": METRIC, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
                           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -571,7 +573,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ep", action="store_true",
                     help="expert-parallel forward instead of replicas: each of the N ranks holds E / N experts and "
-                         "T tokens; the rows travel by NCCL all-to-all-v (bf16 workloads without a capacity)")
+                         "T tokens; the rows travel by NCCL all-to-all (bf16 workloads; with a capacity the "
+                         "exchange has static shapes)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward (moe_backward: input and weight gradients, bf16 experts) instead of the "
                          "forward")
