@@ -145,9 +145,10 @@ def _forward_ep_static(shape, x, w_router, w13_local, w2_local, bias, s13_local,
     x_perm = p["x_perm"]                       # [E C, d]: expert e's block at rows [e C, (e + 1) C), kept rows first
     x_recv = x_perm.new_empty((E * C, d))      # [G][E_loc][C]: from each source rank, its blocks of my experts
     dist.all_to_all_single(x_recv, x_perm, group=group)
-    # every received row goes to the local expert of its block: a fixed pattern (padding rows included)
-    ids = np.tile(np.repeat(np.arange(E_loc, dtype=np.int32), C), G)
-    local_idx = torch.from_numpy(ids).to(topk_idx.device).view(E * C, 1)
+    # every received row goes to the local expert of its block: a fixed pattern (padding rows included), made on
+    # the device so that no host copy breaks a stream capture
+    local_idx = torch.arange(E_loc, dtype=torch.int32, device=topk_idx.device).repeat_interleave(C).repeat(G)
+    local_idx = local_idx.view(E * C, 1)
     s_loc = _shape(shape, E * C, E_loc, 1, 0)
     q = ops.permute(s_loc, x_recv, local_idx)
     y_grouped = ops.expert_ffn(s_loc, q["x_perm"], w13_local, w2_local, shape.H, group_start=q["offsets"][:E_loc],

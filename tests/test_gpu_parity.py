@@ -668,6 +668,45 @@ def test_expert_parallel_single_rank_equals_forward(lib, name, over):
             dist.destroy_process_group()
 
 
+def test_expert_parallel_static_shapes_capture_in_a_graph(lib):
+    """With a capacity, moe_forward_ep has static shapes and no host synchronisation: one NCCL rank captures it
+    in a CUDA graph, and the replay gives the eager output."""
+    import socket
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    from sparse_mixture_experts_expert_b200.ep import moe_forward_ep
+    moe = lib
+    own = not dist.is_initialized()
+    if own:
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=timedelta(seconds=60),
+                                device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        wl = synth.get_workload("tiny").replace(H_s=64, capacity_factor=0.5)
+        inp = synth.make_inputs(wl, seed=5, device=DEV)
+        s = shape_of(moe, wl)
+        kw = dict(bias=inp["bias"], w13_sh=inp["w13_sh"], w2_sh=inp["w2_sh"])
+        eager = moe_forward_ep(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], **kw)[0]
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            out = moe_forward_ep(s, inp["x"], inp["w_router"], inp["w13"], inp["w2"], **kw)[0]
+        g.replay()
+        torch.cuda.synchronize()
+        assert moe.moe_get_status()[0] == 0
+        assert torch.equal(out, eager)
+        del g
+    finally:
+        if own:
+            dist.destroy_process_group()
+
+
 def _ep_single_rank_case(moe, moe_forward_ep, name, over):
     wl = synth.get_workload(name).replace(**over)
     inp = synth.make_inputs(wl, seed=5, device=DEV)
