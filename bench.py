@@ -368,9 +368,9 @@ def cpu_oracle_sample(wl, budget_s=12.0, single_thread=False):
 
 def run_ep(args, wl, world, rank, device):
     """Expert-parallel timing: rank r holds experts [r E/N, (r + 1) E/N) and its own T tokens (weak scaling);
-    moe_forward_ep runs eagerly (without a capacity its splits reach the host; with one the exchange has static
-    shapes), L2 flushed before every step, the step time is the max over ranks of the mean device time between
-    events around each forward."""
+    without a capacity moe_forward_ep runs eagerly (its splits reach the host); with one the exchange has static
+    shapes and the step is captured as a CUDA graph.  L2 flushed before every step; the step time is the max over
+    ranks of the mean device time between events around each forward."""
     import socket
     from datetime import timedelta
 
@@ -403,6 +403,15 @@ def run_ep(args, wl, world, rank, device):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
+    run = step
+    graph = None
+    if s.capacity > 0:   # static shapes, no host synchronisation: the whole step replays as one CUDA graph
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        run = graph.replay
+        run()
+        torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     dist.barrier()
     torch.cuda.synchronize()
@@ -410,7 +419,7 @@ def run_ep(args, wl, world, rank, device):
         for a, b in evs:
             flushbuf.fill_(1)
             a.record()
-            step()
+            run()
             b.record()
         torch.cuda.synchronize()
     dist.barrier()
@@ -425,8 +434,10 @@ def run_ep(args, wl, world, rank, device):
         print(json.dumps({"metric": METRIC, "value": world * wl.T / (ms * 1e-3), "unit": "tokens/s",
                           "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                          "data": "synthetic", "config": cfg, "mode": "expert-parallel",
+                          "data": "synthetic", "config": cfg,
+                          "mode": "expert-parallel" + (", CUDA graph" if graph is not None else ", eager"),
                           "clocks": clk.summary()}), flush=True)
+    del graph   # before the process group goes: a graph that holds NCCL calls is released first
     if own:
         dist.destroy_process_group()
 
