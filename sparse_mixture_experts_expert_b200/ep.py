@@ -54,9 +54,10 @@ class KernelOps:
         return dict(x_perm=p["x_perm"], slot_pos=p["slot_pos"], counts=p["counts"], kept=p["kept"],
                     offsets=p["offsets"])
 
-    def expert_ffn(self, shape, x_grouped, w13, w2, hidden, group_start=None, group_rows=None, s13=None, s2=None):
+    def expert_ffn(self, shape, x_grouped, w13, w2, hidden, group_start=None, group_rows=None, s13=None, s2=None,
+                   y=None):
         _, y = moe_expert_ffn(shape, x_grouped, w13, w2, hidden=hidden, group_start=group_start,
-                              group_rows=group_rows, s13=s13, s2=s2)
+                              group_rows=group_rows, s13=s13, s2=s2, y=y)
         return y
 
     def combine(self, shape, y_perm, slot_pos, topk_w, y_shared=None):
@@ -136,25 +137,30 @@ def moe_forward_ep(shape: MoeShape, x, w_router, w13_local, w2_local, *, bias=No
 
 def _forward_ep_static(shape, x, w_router, w13_local, w2_local, bias, s13_local, s2_local, w13_sh, s13_sh, w2_sh,
                        s2_sh, group, ops, G, E_loc):
-    """moe_forward_ep with capacity C: equal all-to-all splits, no host synchronisation."""
+    """moe_forward_ep with capacity C: equal all-to-all splits, no host synchronisation.
+
+    Source rank q's rows arrive as its E_loc blocks of C rows, kept rows first, one block per local expert, so the
+    local experts run on each source's blocks where they lie (groups at e C with the exchanged kept counts) and
+    write their outputs in place: no regrouping, no restoring copy, and the padding rows are skipped.
+    """
     E, k, T, d, C = shape.E, shape.k, shape.T, shape.d, shape.capacity
     s_route = MoeShape(T=T, d=d, E=E, k=k, H=shape.H, H_s=0, capacity=C, act=shape.act, wfmt=shape.wfmt,
                        renorm=shape.renorm, flags=shape.flags)
     topk_idx, topk_w = ops.route(s_route, x, w_router, bias)
     p = ops.permute(s_route, x, topk_idx)
     x_perm = p["x_perm"]                       # [E C, d]: expert e's block at rows [e C, (e + 1) C), kept rows first
-    x_recv = x_perm.new_empty((E * C, d))      # [G][E_loc][C]: from each source rank, its blocks of my experts
+    kept = p["kept"][:E].to(torch.int32).contiguous()
+    kept_recv = torch.empty_like(kept)         # [G][E_loc]: kept rows of my experts from each source rank
+    dist.all_to_all_single(kept_recv, kept, group=group)
+    x_recv = x_perm.new_empty((E * C, d))      # [G][E_loc][C]
     dist.all_to_all_single(x_recv, x_perm, group=group)
-    # every received row goes to the local expert of its block: a fixed pattern (padding rows included), made on
-    # the device so that no host copy breaks a stream capture
-    local_idx = torch.arange(E_loc, dtype=torch.int32, device=topk_idx.device).repeat_interleave(C).repeat(G)
-    local_idx = local_idx.view(E * C, 1)
-    s_loc = _shape(shape, E * C, E_loc, 1, 0)
-    q = ops.permute(s_loc, x_recv, local_idx)
-    y_grouped = ops.expert_ffn(s_loc, q["x_perm"], w13_local, w2_local, shape.H, group_start=q["offsets"][:E_loc],
-                               group_rows=q["kept"], s13=s13_local, s2=s2_local)
-    ones = torch.ones(E * C, 1, dtype=topk_w.dtype, device=topk_w.device)
-    y_recv = ops.combine(s_loc, y_grouped, q["slot_pos"], ones)
+    y_recv = x_perm.new_empty((E * C, d))
+    starts = torch.arange(E_loc, dtype=torch.int32, device=kept.device) * C
+    s_blk = _shape(shape, E_loc * C, E_loc, 1, 0)
+    for q in range(G):
+        blk = slice(q * E_loc * C, (q + 1) * E_loc * C)
+        ops.expert_ffn(s_blk, x_recv[blk], w13_local, w2_local, shape.H, group_start=starts,
+                       group_rows=kept_recv[q * E_loc:(q + 1) * E_loc], s13=s13_local, s2=s2_local, y=y_recv[blk])
     y_back = torch.empty_like(y_recv)
     dist.all_to_all_single(y_back, y_recv, group=group)
     y_sh = None

@@ -44,14 +44,17 @@ class OracleOps:
         return dict(x_perm=self.torch.from_numpy(x_perm), slot_pos=t(p["slot_pos"]), counts=t(p["counts"]),
                     kept=t(p["kept"]), offsets=t(p["offsets"]))
 
-    def expert_ffn(self, shape, xg, w13, w2, hidden, group_start=None, group_rows=None, s13=None, s2=None):
+    def expert_ffn(self, shape, xg, w13, w2, hidden, group_start=None, group_rows=None, s13=None, s2=None, y=None):
         xg = xg.numpy()
-        y = np.zeros((xg.shape[0], shape.d))
+        yy = np.zeros((xg.shape[0], shape.d))
         groups = [(0, xg.shape[0])] if group_start is None else zip(group_start.tolist(), group_rows.tolist())
         for g, (a, n) in enumerate(groups):
             if n:
-                y[a:a + n] = self.O.expert_ffn(xg[a:a + n], w13[g].numpy(), w2[g].numpy(), shape.act)
-        return self.torch.from_numpy(y)
+                yy[a:a + n] = self.O.expert_ffn(xg[a:a + n], w13[g].numpy(), w2[g].numpy(), shape.act)
+        if y is not None:   # the caller's rows (a view of a larger buffer)
+            y.copy_(self.torch.from_numpy(yy))
+            return y
+        return self.torch.from_numpy(yy)
 
     def combine(self, shape, y_perm, slot_pos, w, y_shared=None):
         return self.torch.from_numpy(self.O.combine(y_perm.numpy(), slot_pos.numpy(), w.numpy(),
