@@ -11,10 +11,10 @@ Per rank r of G ranks, owning experts [r * E_loc, (r + 1) * E_loc) with E_loc = 
    rank q are the contiguous groups of q's experts;
 3. exchange the per-expert row counts (``all_to_all``), then the rows (``all_to_all`` with the counts as
    splits);
-4. regroup the received rows by local expert (``moe_permute`` with k = 1) and run the local experts
-   (``moe_expert_ffn``);
-5. put the outputs back in received order (``moe_combine`` with k = 1 and weight 1, an exact bf16 copy) and
-   send them back (``all_to_all``);
+4. run the local experts on the received rows where they lie: each source's rows are its groups of this
+   rank's experts in expert order, so ``moe_expert_ffn`` takes each source's block as E_loc groups (sizes from
+   the exchanged counts) and writes the outputs in place;
+5. send the outputs back (``all_to_all``);
 6. the weighted top-k reduction in token order plus the shared expert on the local tokens (``moe_combine``).
 
 Each (token, slot) row gets the expert output the single-GPU forward gives it, and the reduction runs in the
@@ -25,10 +25,11 @@ The row counts reach the host as the splits of the exchanges: one device synchro
 With a capacity (``shape.capacity = C > 0``, the same C on every rank: the MoEEvolve README's capacity-factor
 dispatch with static shapes) the exchange has static shapes instead.  Each rank groups its own tokens with
 capacity C (ranks counted in its token order, as ``moe_forward`` with capacity C on those tokens), so the rows for
-rank q are always E_loc * C rows, kept ones first in each expert's block.  Both exchanges then use equal splits
-and the receiver's local grouping is a fixed pattern, so nothing reaches the host and the whole forward can be
-captured in a CUDA graph.  The price is the padding rows: they cross the exchange and run through the local
-experts (their outputs are never combined).  Output: ``moe_forward`` with capacity C on the rank's tokens.
+rank q are always E_loc * C rows, kept ones first in each expert's C-row block.  Both exchanges then use equal
+splits, the kept counts travel as a small device tensor, and the local experts run on each source's blocks where
+they lie (groups at e * C), so nothing reaches the host and the whole forward can be captured in a CUDA graph.
+The price is the padding rows crossing the exchange; the experts skip them.  Output: ``moe_forward`` with
+capacity C on the rank's tokens.
 
 The exchanges are NCCL all-to-all calls (``torch.distributed``), not fused with the expert GEMMs.
 """
@@ -110,19 +111,21 @@ def moe_forward_ep(shape: MoeShape, x, w_router, w13_local, w2_local, *, bias=No
     dist.all_to_all_single(x_recv, x_perm, output_split_sizes=recv_split, input_split_sizes=send_split,
                            group=group)
 
-    # 4-5. the local experts on the received rows, outputs back in received order
-    if n_recv > 0:
-        ids = np.repeat(np.tile(np.arange(E_loc, dtype=np.int32), G), cr.reshape(-1))
-        local_idx = torch.from_numpy(ids).to(topk_idx.device).view(n_recv, 1)
-        s_loc = _shape(shape, n_recv, E_loc, 1, 0)
-        q = ops.permute(s_loc, x_recv, local_idx)
-        y_grouped = ops.expert_ffn(s_loc, q["x_perm"], w13_local, w2_local, shape.H,
-                                   group_start=q["offsets"][:E_loc], group_rows=q["kept"], s13=s13_local,
-                                   s2=s2_local)
-        ones = torch.ones(n_recv, 1, dtype=topk_w.dtype, device=topk_w.device)
-        y_recv = ops.combine(s_loc, y_grouped, q["slot_pos"], ones)
-    else:
-        y_recv = x_perm.new_empty((0, d))
+    # 4-5. the local experts on the received rows where they lie: source q's rows are its groups of my experts in
+    # expert order (counts cr[q]), so each source's block runs as E_loc groups, outputs written in place
+    y_recv = x_perm.new_empty((n_recv, d))
+    base = 0
+    for q in range(G):
+        nq = int(cr[q].sum())
+        if nq > 0:
+            starts = np.concatenate([[0], np.cumsum(cr[q])[:-1]]).astype(np.int32)
+            dev = topk_idx.device
+            s_blk = _shape(shape, nq, E_loc, 1, 0)
+            ops.expert_ffn(s_blk, x_recv[base:base + nq], w13_local, w2_local, shape.H,
+                           group_start=torch.from_numpy(starts).to(dev),
+                           group_rows=torch.from_numpy(cr[q].astype(np.int32)).to(dev), s13=s13_local, s2=s2_local,
+                           y=y_recv[base:base + nq])
+        base += nq
     y_back = x_perm.new_empty((T * k, d))
     dist.all_to_all_single(y_back, y_recv, output_split_sizes=send_split, input_split_sizes=recv_split,
                            group=group)
