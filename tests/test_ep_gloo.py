@@ -171,3 +171,29 @@ def test_expert_parallel_static_capacity_matches_the_per_rank_layer(case, cap):
         assert (idx == ref["idx"]).all()
         np.testing.assert_allclose(out, ref["out"], rtol=1e-10, atol=1e-12)
     assert dropped > 0   # the capacity binds somewhere
+
+
+@pytest.mark.parametrize("cap", [0, 4])
+def test_expert_parallel_four_ranks(cap):
+    # four ranks of two experts each, an uneven token split (37 tokens), with and without a capacity
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import oracle as O
+    case = (37, 16, 8, 2, 16, 16, "skew")
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 4, port, case, q, cap)) for r in range(4)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in range(4)]
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    T, d, E, k, H, H_s, mode = case
+    x, w_r, bias, w13, w2, w13_sh, w2_sh = _problem(case)
+    for rank, toks, out, idx in got:
+        ref = O.moe_forward(x[toks], w_r, bias, w13, w2, k=k, act=0, renorm=True, cap=cap, w13_sh=w13_sh,
+                            w2_sh=w2_sh)
+        assert (idx == ref["idx"]).all()
+        np.testing.assert_allclose(out, ref["out"], rtol=1e-10, atol=1e-12)
